@@ -1,0 +1,250 @@
+"""CPU oracle for decode attention over the DepthWeave-KV compressed cache.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the bench's CPU
+baseline are the only callers.  The product library never imports this package and this
+package never imports the product library.
+
+This module is argument marshalling only (numpy <-> the C functions of
+``dwkv_oracle.c``); every step of the arithmetic lives in that C file, in fp64 for
+decode / probe and in an explicitly ordered fp32 for encode.  Cited source:
+"DepthWeave-KV: Token-Adaptive Cross-Layer Residual Factorization for Long-Context KV
+Cache Compression", §3 Method, Eq. (1) (reconstruction) and Eq. (3) (probe error).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        p = C.c_void_p
+        i = C.c_int
+        d = C.c_double
+        L.oracle_decode_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, i, p, p]
+        L.oracle_decode_head.restype = i
+        L.oracle_probe_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, d, p, p, p]
+        L.oracle_probe_head.restype = i
+        L.oracle_decode_many.argtypes = [i, i, i, i, i, p] + [p] * 12 + [d, p, i]
+        L.oracle_decode_many.restype = i
+        L.oracle_encode_vector.argtypes = [i, i, p, p, i, i, i, p, p, p, p, p, p]
+        L.oracle_encode_vector.restype = i
+        L.oracle_encode_many.argtypes = [i, i, i, p, p, p, i, i, p, p, p, p, p, i]
+        L.oracle_encode_many.restype = i
+        L.oracle_reconstruct.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, p]
+        L.oracle_reconstruct.restype = None
+        for name in ("oracle_f32_to_bf16_rn_many", "oracle_f32_to_fp16_rn_many",
+                     "oracle_fp16_to_f64_many", "oracle_bf16_to_f64_many"):
+            getattr(L, name).argtypes = [C.c_int64, p, p]
+            getattr(L, name).restype = None
+        _LIB = L
+    return _LIB
+
+
+# ----------------------------------------------------------------------------- marshalling
+def _bits16(a) -> np.ndarray:
+    """Raw 16-bit patterns (bf16 / fp16) of a torch tensor or numpy array, C-contiguous."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach().cpu().contiguous()
+            if a.dtype in (torch.bfloat16, torch.float16):
+                a = a.view(torch.int16)
+            return np.ascontiguousarray(a.numpy().view(np.uint16))
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.asarray(a)
+    if a.dtype == np.float16:
+        a = a.view(np.uint16)
+    return np.ascontiguousarray(a.astype(np.uint16, copy=False))
+
+
+def _arr(a, dtype) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach().cpu().contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(a).astype(dtype, copy=False))
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def default_tau(d: int) -> float:
+    return 1.0 / math.sqrt(d)
+
+
+# ----------------------------------------------------------------------------- conversions
+def f32_to_bf16_rn(x) -> np.ndarray:
+    x = _arr(x, np.float32).reshape(-1)
+    out = np.empty(x.size, np.uint16)
+    lib().oracle_f32_to_bf16_rn_many(x.size, _p(x), _p(out))
+    return out
+
+
+def f32_to_fp16_rn(x) -> np.ndarray:
+    x = _arr(x, np.float32).reshape(-1)
+    out = np.empty(x.size, np.uint16)
+    lib().oracle_f32_to_fp16_rn_many(x.size, _p(x), _p(out))
+    return out
+
+
+def fp16_to_f64(bits) -> np.ndarray:
+    b = _bits16(bits).reshape(-1)
+    out = np.empty(b.size, np.float64)
+    lib().oracle_fp16_to_f64_many(b.size, _p(b), _p(out))
+    return out
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    b = _bits16(bits).reshape(-1)
+    out = np.empty(b.size, np.float64)
+    lib().oracle_bf16_to_f64_many(b.size, _p(b), _p(out))
+    return out
+
+
+# ----------------------------------------------------------------------------- reconstruct
+def reconstruct(basis, r_t, coeff, idx, codes, scale, with_residual=True) -> np.ndarray:
+    """One reconstructed vector (fp64 [d]); basis bf16 [d][r_max], coeff bf16 [r_max]."""
+    b = _bits16(basis)
+    d, r_max = b.shape
+    c = _bits16(coeff)
+    ix = _arr(idx, np.uint8)
+    cd = _arr(codes, np.int8)
+    sc = int(_bits16(scale).reshape(-1)[0])
+    out = np.empty(d, np.float64)
+    lib().oracle_reconstruct(d, r_max, _p(b), int(r_t), _p(c), ix.size, _p(ix), _p(cd), sc,
+                             1 if with_residual else 0, _p(out))
+    return out
+
+
+# ----------------------------------------------------------------------------- decode
+class HeadProblem:
+    """Token-ordered inputs of one (sequence, layer, kv-head) decode problem."""
+
+    def __init__(self, basis_k, basis_v, ranks, coeff_k, idx_k, codes_k, scale_k,
+                 coeff_v, idx_v, codes_v, scale_v, q):
+        self.bk = _bits16(basis_k)
+        self.bv = _bits16(basis_v)
+        self.d, self.r_max = self.bk.shape
+        self.rank = _arr(ranks, np.int32).reshape(-1)
+        self.T = self.rank.size
+        self.ck = _bits16(coeff_k).reshape(self.T, self.r_max)
+        self.cv = _bits16(coeff_v).reshape(self.T, self.r_max)
+        ik = _arr(idx_k, np.uint8)
+        self.s = ik.shape[-1] if ik.ndim >= 1 else 0
+        self.ik = ik.reshape(self.T, self.s)
+        self.iv = _arr(idx_v, np.uint8).reshape(self.T, self.s)
+        self.qk = _arr(codes_k, np.int8).reshape(self.T, self.s)
+        self.qv = _arr(codes_v, np.int8).reshape(self.T, self.s)
+        self.sk = _bits16(scale_k).reshape(self.T)
+        self.sv = _bits16(scale_v).reshape(self.T)
+        self.q = _bits16(q).reshape(-1, self.d)
+        self.gq = self.q.shape[0]
+
+    def _ptrs(self):
+        return [_p(self.bk), _p(self.bv), _p(self.rank), _p(self.ck), _p(self.ik), _p(self.qk),
+                _p(self.sk), _p(self.cv), _p(self.iv), _p(self.qv), _p(self.sv), _p(self.q)]
+
+
+def decode_head(prob: HeadProblem, tau=None, with_residual=True, want_p=False):
+    """fp64 attention output [gq][d] (and softmax weights [gq][T] when ``want_p``)."""
+    tau = default_tau(prob.d) if tau is None else tau
+    out = np.empty((prob.gq, prob.d), np.float64)
+    pw = np.empty((prob.gq, max(prob.T, 1)), np.float64) if want_p else None
+    rc = lib().oracle_decode_head(prob.d, prob.r_max, prob.T, prob.gq, prob.s, *prob._ptrs(),
+                                  float(tau), 1 if with_residual else 0, _p(out),
+                                  _p(pw) if want_p else None)
+    if rc != 0:
+        raise MemoryError("oracle_decode_head failed")
+    if want_p:
+        return out, pw[:, :prob.T]
+    return out
+
+
+def probe_head(prob: HeadProblem, tau=None, eps=1e-6):
+    """Relative L2 error (Eq. 3 reading) and both outputs (fp64)."""
+    tau = default_tau(prob.d) if tau is None else tau
+    err = np.zeros(1, np.float64)
+    of = np.empty((prob.gq, prob.d), np.float64)
+    on = np.empty((prob.gq, prob.d), np.float64)
+    rc = lib().oracle_probe_head(prob.d, prob.r_max, prob.T, prob.gq, prob.s, *prob._ptrs(),
+                                 float(tau), float(eps), _p(err), _p(of), _p(on))
+    if rc != 0:
+        raise MemoryError("oracle_probe_head failed")
+    return float(err[0]), of, on
+
+
+def decode_many(problems, tau=None, nthreads=None):
+    """Run many independent problems on ``nthreads`` host threads; list of [gq][d] outputs."""
+    if not problems:
+        return []
+    n = len(problems)
+    p0 = problems[0]
+    tau = default_tau(p0.d) if tau is None else tau
+    nthreads = nthreads or os.cpu_count() or 1
+    T = np.array([pr.T for pr in problems], np.int32)
+    cols = list(zip(*[pr._ptrs() for pr in problems]))
+    arrs = [(C.c_void_p * n)(*col) for col in cols]
+    outs = [np.empty((pr.gq, pr.d), np.float64) for pr in problems]
+    oarr = (C.c_void_p * n)(*[_p(o) for o in outs])
+    rc = lib().oracle_decode_many(n, p0.d, p0.r_max, p0.gq, p0.s, _p(T), *arrs, float(tau), oarr,
+                                  int(nthreads))
+    if rc != 0:
+        raise MemoryError("oracle_decode_many failed")
+    return outs
+
+
+# ----------------------------------------------------------------------------- encode
+def encode_vector(basis, x, r_t, s, bits):
+    """Encode one bf16 vector; dict of coeff (bf16 bits), c32, idx, codes, scale (fp16 bits), resid."""
+    b = _bits16(basis)
+    d, r_max = b.shape
+    xv = _bits16(x).reshape(d)
+    coeff = np.zeros(r_max, np.uint16)
+    c32 = np.zeros(r_max, np.float32)
+    idx = np.zeros(s, np.uint8)
+    codes = np.zeros(s, np.int8)
+    scale = np.zeros(1, np.uint16)
+    resid = np.zeros(d, np.float32)
+    rc = lib().oracle_encode_vector(d, r_max, _p(b), _p(xv), int(r_t), int(s), int(bits), _p(coeff),
+                                    _p(c32), _p(idx), _p(codes), _p(scale), _p(resid))
+    if rc != 0:
+        raise ValueError("oracle_encode_vector: bad arguments")
+    return {"coeff": coeff, "c32": c32, "idx": idx, "codes": codes, "scale": scale[0], "resid": resid}
+
+
+def encode_many(basis, x, ranks, s, bits, nthreads=None, want_c32=False):
+    """Encode n vectors [n][d] sharing one basis; arrays token-ordered."""
+    b = _bits16(basis)
+    d, r_max = b.shape
+    xv = _bits16(x).reshape(-1, d)
+    n = xv.shape[0]
+    rk = _arr(ranks, np.int32).reshape(n)
+    coeff = np.zeros((n, r_max), np.uint16)
+    c32 = np.zeros((n, r_max), np.float32) if want_c32 else None
+    idx = np.zeros((n, s), np.uint8)
+    codes = np.zeros((n, s), np.int8)
+    scale = np.zeros(n, np.uint16)
+    rc = lib().oracle_encode_many(n, d, r_max, _p(b), _p(xv), _p(rk), int(s), int(bits), _p(coeff),
+                                  _p(c32) if want_c32 else None, _p(idx), _p(codes), _p(scale),
+                                  int(nthreads or os.cpu_count() or 1))
+    if rc != 0:
+        raise ValueError("oracle_encode_many: bad arguments")
+    out = {"coeff": coeff, "idx": idx, "codes": codes, "scale": scale}
+    if want_c32:
+        out["c32"] = c32
+    return out
