@@ -1,0 +1,511 @@
+#!/usr/bin/env python
+"""Decode throughput over a DepthWeave-KV compressed KV cache on B200.
+
+Workload (default ``llama8b_64k``): Llama-3-8B attention shapes -- 32 layers in 16
+two-layer groups, 32 query heads / 8 kv heads, head_dim 128, batch 1, 64K context;
+bases r_max = 64 per (group, kv-head, K/V); tiers {16, 32, 64} with probabilities
+0.6 / 0.3 / 0.1; residual s = 16 int4 channels with an fp16 scale.  The cache holds
+65535 compressed tokens (synthetic, seeded, imported before timing).  One step = for
+each of the 32 layers: encode + append one new token (dwkv_append), then fused decode
+attention over the whole context (dwkv_decode_attention).  Metric: decode tokens/s
+(batch / step time) and the compressed-KV bytes/s of the decode kernel against the
+measured HBM copy bandwidth.  Attention only (no projections / MLP: no weights exist).
+
+Timing: W warm-up steps, then K steps captured in one CUDA graph and replayed once,
+bracketed by a barrier + synchronize, timed with CUDA events; max over ranks.  Each
+step streams ~2.6 GB of pages (> 126 MB L2), so no L2 flush is needed.  A second
+replay of the same K steps with an external event around every decode launch gives the
+decode kernel's average duration for the roofline.  ``e2e`` repeats the step with host
+(pinned) inputs copied in and the outputs copied out inside the timed region.
+
+``--impl reference`` times the CPU oracle (plain fp64 C, all host cores) on a bounded
+sample of the same workload and reports the same metric.
+
+Multi-GPU (torchrun): every rank runs an independent replica (the path shards by
+sequence with no exchange); value = total tokens of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode tok/s at 64K (8B shapes); compressed-KV HBM GB/s, % of peak"
+UNIT = "tok/s"
+
+
+def dense_kv_bytes(layers: int, kv_heads: int, head_dim: int, tokens: int, elem_bytes: int = 2) -> int:
+    """Bytes of an uncompressed KV cache: 2 (K and V) x layers x heads x dim x tokens x bytes."""
+    return 2 * layers * kv_heads * head_dim * tokens * elem_bytes
+
+
+def token_bytes(rank: int, s: int, bits: int) -> int:
+    """Stored bytes of one token of one (layer, kv-head), keys + values."""
+    return 2 * (2 * rank + s + s * bits // 8 + 2)
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("dwkv_decode.cu", "dwkv_common.cuh"):
+        h.update(open(os.path.join(ROOT, "decode_attention_depthweave_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the
+    current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", f"decode_{workload}.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 20 ms; summary() keeps the
+    samples that fall inside the marked region (wall clock)."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+        self.t0 = self.t1 = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.5)
+        return self
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        import datetime
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+            os.unlink(self.path)
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        def ts(x):
+            try:
+                return datetime.datetime.strptime(x, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                return None
+
+        inside = [r for r in rows if self.t0 and ts(r[0]) is not None and self.t0 - 0.01 <= ts(r[0]) <= self.t1 + 0.01]
+        use = inside if inside else rows
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [num(r[2]) for r in use if num(r[2]) is not None]
+        mx = [num(r[3]) for r in use if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i in range(4) if r[6 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(use), "samples_in_region": len(inside)}
+
+
+# ----------------------------------------------------------------------------- dist
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- oracle sample
+def cpu_oracle_sample(wl, comp, tiers, bases, q, layer, t_sample, threads):
+    """Time the CPU oracle on the kv-heads of one layer over the first ``t_sample`` cached
+    tokens, on ``threads`` host threads.  Decode cost is linear in the context, so
+    seconds per full step = measured x (T / t_sample) x layers.  Returns (wall s, items)."""
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from helpers import head_problem
+    part = {k: v[:t_sample] for k, v in comp.items()}
+    items = [head_problem(wl, bases, tiers[:t_sample], part, q, layer, h) for h in range(wl.num_kv_heads)]
+    t0 = time.perf_counter()
+    oracle.decode_many(items, nthreads=threads)
+    return time.perf_counter() - t0, len(items)
+
+
+# ----------------------------------------------------------------------------- main path
+def run_dwkv(args, world, rank, local):
+    import torch
+
+    import decode_attention_depthweave_b200 as dw
+    import synth
+
+    wl = synth.workload(args.workload)
+    if args.layers:
+        wl = wl.scaled(num_layers=args.layers)
+    dev = torch.device("cuda", local)
+    T = args.context or wl.context
+    n_steps = args.warmup + args.steps + args.e2e_steps
+    extra = args.profile_steps + 64
+    B = 1
+    bases = synth.make_bases(wl)
+    cfg = dw.config_from(num_layers=wl.num_layers, layers_per_group=wl.layers_per_group,
+                         num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim,
+                         r_max=wl.r_max, tiers=wl.tiers, resid_channels=wl.resid_channels,
+                         resid_bits=wl.resid_bits, max_batch=B, max_context=T + n_steps + extra)
+    stream = torch.cuda.Stream(device=dev)
+    cache = dw.Cache(cfg, bases[0], bases[1], device=dev, ws_seqs=B, stream=stream)
+    if args.tuning:
+        c, w_, s_ = (int(x) for x in args.tuning.split(","))
+        cache.set_decode_tuning(c, w_, s_)
+    h = cache.h
+
+    # ---- import the T-1 cached tokens (seeded synthetic compressed form)
+    keep_layers = {0} if (rank == 0 and world == 1 and not args.no_cpu_baseline) else set()
+    tiers_dev, comp_cpu, tiers_cpu = {}, {}, {}
+    tier_counts = torch.zeros(wl.num_groups, wl.num_kv_heads, len(wl.tiers), dtype=torch.int64)
+    with torch.cuda.stream(stream):
+        for layer in range(wl.num_layers):
+            g = layer // wl.layers_per_group
+            if g not in tiers_dev:
+                tiers_dev[g] = synth.make_tiers(wl, rank, g, T - 1, device=dev)
+                for k in range(len(wl.tiers)):
+                    tier_counts[g, :, k] = (tiers_dev[g] == k).sum(0).cpu()
+            comp = synth.make_compressed(wl, rank, layer, tiers_dev[g], device=dev)
+            cache.append_compressed(layer, [0], [T - 1], tiers_dev[g], comp["coeff"], comp["idx"],
+                                    comp["codes"], comp["scales"], stream=stream)
+            if layer in keep_layers:
+                comp_cpu[layer] = {k: v.cpu() for k, v in comp.items()}
+                tiers_cpu[g] = tiers_dev[g].cpu()
+            del comp
+    cache.sync(stream)
+
+    # ---- per-step inputs, resident in HBM
+    Kn, Vn, Qs = [], [], []
+    Tn = {}
+    for layer in range(wl.num_layers):
+        k, v = synth.make_dense_vectors(wl, rank, layer, n_steps, bases, device=dev, start=T - 1)
+        Kn.append(k.view(n_steps, 1, wl.num_kv_heads, wl.head_dim))
+        Vn.append(v.view(n_steps, 1, wl.num_kv_heads, wl.head_dim))
+        Qs.append(synth.make_queries(wl, layer, batch=n_steps, device=dev).view(n_steps, 1, wl.num_q_heads, wl.head_dim))
+        g = layer // wl.layers_per_group
+        if g not in Tn:
+            Tn[g] = synth.make_tiers(wl, rank, g, n_steps, device=dev, start=T - 1).view(n_steps, 1, wl.num_kv_heads)
+            for k_ in range(len(wl.tiers)):
+                tier_counts[g, :, k_] += (Tn[g][: args.warmup + args.steps] == k_).sum((0, 1)).cpu()
+    out = torch.empty(wl.num_layers, 1, wl.num_q_heads, wl.head_dim, dtype=torch.float32, device=dev)
+    ws = cache.workspace
+    lpg = wl.layers_per_group
+
+    def step(s, ev=None):
+        for layer in range(wl.num_layers):
+            g = layer // lpg
+            dw.dwkv_append(h, layer, [0], [1], Kn[layer][s], Vn[layer][s], Tn[g][s] if layer % lpg == 0 else None,
+                           stream)
+            if ev is not None:
+                ev[layer][0].record(stream)
+            dw.dwkv_decode_attention(h, layer, [0], Qs[layer][s], out[layer], ws, stream)
+            if ev is not None:
+                ev[layer][1].record(stream)
+
+    launches_per_step = wl.num_layers * 2 + wl.num_groups      # encode + decode per layer, place per group
+
+    # ---- warm-up (graph of W steps, replayed once)
+    torch.cuda.synchronize(dev)
+    g_warm = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm, stream=stream):
+        for s in range(args.warmup):
+            step(s)
+    with torch.cuda.stream(stream):
+        g_warm.replay()
+    torch.cuda.synchronize(dev)
+    cache.sync(stream)
+
+    # ---- timed: K steps in one graph, replayed once
+    g_main = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_main, stream=stream):
+        for s in range(args.warmup, args.warmup + args.steps):
+            step(s)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        clk.mark_start()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g_main.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        clk.mark_end()
+    barrier(world)
+    ms_total = e0.elapsed_time(e1)
+    cache.sync(stream)
+    ms_total = max_over_ranks(world, ms_total)
+    ms_per_step = ms_total / args.steps
+    clocks = clk.summary()
+
+    # ---- the decode kernel's own duration: same K steps (state rewound is not needed:
+    #      a re-run appends K more tokens, which changes the work by < 0.1 %)
+    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+            for _ in range(wl.num_layers)] for _ in range(args.profile_steps)]
+    g_prof = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_prof, stream=stream):
+        for i in range(args.profile_steps):
+            step(args.warmup + i, evs[i])
+    with torch.cuda.stream(stream):
+        g_prof.replay()
+    torch.cuda.synchronize(dev)
+    dec_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(args.profile_steps) for l in range(wl.num_layers)]
+    dec_ms_mean = statistics.mean(dec_ms)
+
+    # ---- algorithmic bytes: every stored byte of the attended tokens (per-token bytes of
+    #      its tier), plus the two bases, the query and the output of each launch
+    held = T - 1 + args.warmup + args.steps                  # tokens per head after the timed steps
+    tok_bytes = torch.tensor([token_bytes(r, wl.resid_channels, wl.resid_bits) for r in wl.tiers], dtype=torch.float64)
+    bytes_per_tok_head = float((tier_counts.double() * tok_bytes).sum()) / (wl.num_groups * wl.num_kv_heads * held)
+    basis_bytes = 2 * wl.num_kv_heads * wl.head_dim * wl.r_max * 2
+    io_bytes = wl.num_q_heads * wl.head_dim * (2 + 4)
+
+    def layer_bytes(ctx):
+        return bytes_per_tok_head * wl.num_kv_heads * ctx + basis_bytes + io_bytes
+
+    ctx_timed = T - 1 + args.warmup + (args.steps + 1) / 2.0   # mean attended context in the timed steps
+    ctx_prof = held + (args.profile_steps + 1) / 2.0
+    comp_bytes_layer = bytes_per_tok_head * wl.num_kv_heads * ctx_timed
+    alg_bytes = layer_bytes(ctx_prof)
+    peaks = measured_peaks()
+    achieved = alg_bytes / (dec_ms_mean * 1e-3) / 1e9
+    traffic = profiled_traffic(args.workload)
+
+    # ---- e2e: host inputs in, host outputs out, one step per graph replay
+    e2e = None
+    if args.e2e_steps > 0:
+        sK = torch.stack([Kn[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1).cpu().pin_memory()
+        sV = torch.stack([Vn[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1).cpu().pin_memory()
+        sQ = torch.stack([Qs[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1).cpu().pin_memory()
+        sT = torch.stack([Tn[g][args.warmup + args.steps:] for g in range(wl.num_groups)], 1).cpu().pin_memory()
+        dK = torch.empty_like(sK[0], device=dev)
+        dV = torch.empty_like(sV[0], device=dev)
+        dQ = torch.empty_like(sQ[0], device=dev)
+        dT = torch.empty_like(sT[0], device=dev)
+        host_out = torch.empty((args.e2e_steps,) + tuple(out.shape), dtype=torch.float32).pin_memory()
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e, stream=stream):
+            for layer in range(wl.num_layers):
+                g = layer // lpg
+                dw.dwkv_append(h, layer, [0], [1], dK[layer], dV[layer], dT[g] if layer % lpg == 0 else None, stream)
+                dw.dwkv_decode_attention(h, layer, [0], dQ[layer], out[layer], ws, stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a0.record(stream)
+            for i in range(args.e2e_steps):
+                dK.copy_(sK[i], non_blocking=True)
+                dV.copy_(sV[i], non_blocking=True)
+                dQ.copy_(sQ[i], non_blocking=True)
+                dT.copy_(sT[i], non_blocking=True)
+                g_e2e.replay()
+                host_out[i].copy_(out, non_blocking=True)
+            a1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / args.e2e_steps
+        h2d = sK[0].numel() * 2 + sV[0].numel() * 2 + sQ[0].numel() * 2 + sT[0].numel()
+        d2h = out.numel() * 4
+        assert torch.isfinite(host_out).all()
+        e2e = {"value": round(world * B / (e2e_ms * 1e-3), 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms, 4)}
+    cache.sync(stream)
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only): the 8 kv-heads of layer 0 at full context
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and comp_cpu:
+        threads = min(os.cpu_count() or 1, wl.num_kv_heads)
+        dt, n_items = cpu_oracle_sample(wl, comp_cpu[0], tiers_cpu[0], bases, Qs[0][args.warmup][0].cpu(), 0,
+                                        T - 1, threads)
+        step_s = dt * wl.num_layers * wl.num_kv_heads / n_items
+        cpu = {"value": round(B / step_s, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"layer 0, {n_items} kv-heads x {T - 1} cached tokens (fp64 C oracle, {dt:.1f} s wall "
+                         f"on {threads} threads), scaled x{wl.num_layers} layers to one step"}
+
+    value = world * B / (ms_per_step * 1e-3)
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 storage, fp32 math",
+        "data": "synthetic (seeded compressed cache; no model weights)",
+        "config": {"workload": args.workload, "layers": wl.num_layers, "groups": wl.num_groups,
+                   "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                   "batch_per_gpu": B, "context": T, "r_max": wl.r_max, "tiers": list(wl.tiers),
+                   "tier_probs": list(wl.tier_probs), "resid_channels": wl.resid_channels,
+                   "resid_bits": wl.resid_bits, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (~2.6 GB of pages per step); no flush",
+                   "graph": "CUDA graph of K steps, replayed once"},
+        "gpu_launches": launches_per_step * args.steps,
+        "compressed_gb_per_step": round(comp_bytes_layer * wl.num_layers / 1e9, 4),
+        "compressed_tb_s": round(comp_bytes_layer * wl.num_layers / (ms_per_step * 1e-3) / 1e12, 4),
+        "dense_bf16_gb_per_step": round(dense_kv_bytes(wl.num_layers, wl.num_kv_heads, wl.head_dim, int(ctx_timed)) / 1e9, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": traffic, "kernel": f"dwkv::decode_kernel<{wl.resid_bits},false>",
+                     "alg_bytes_per_launch": int(alg_bytes), "launch_ms": round(dec_ms_mean, 5),
+                     "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
+                     "frac_of_8tbs_spec": round(achieved / 8000.0, 4)},
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    cache.close()
+    return res
+
+
+def run_reference(args, world, rank, local):
+    """The CPU oracle, as it stands, timed on a bounded sample of the same workload: per
+    step, the 8 kv-heads of one layer over a prefix of the context, scaled linearly to the
+    full context and to all layers."""
+    import synth
+    wl = synth.workload(args.workload)
+    T = args.context or wl.context
+    bases = synth.make_bases(wl.scaled(num_layers=wl.layers_per_group))
+    tiers = synth.make_tiers(wl, 0, 0, T - 1)
+    comp = synth.make_compressed(wl, 0, 0, tiers)
+    q = synth.make_queries(wl, 0, batch=1)[0]
+    threads = os.cpu_count() or 1
+    # calibrate: seconds per cached token for the 8 heads, then size the per-step prefix
+    dt, n = cpu_oracle_sample(wl, comp, tiers, bases, q, 0, 2048, min(threads, wl.num_kv_heads))
+    per_tok = dt / 2048
+    budget = min(20.0, 150.0 / max(args.steps + args.warmup, 1))
+    t_s = int(max(512, min(T - 1, budget / max(per_tok, 1e-9))))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, comp, tiers, bases, q, 0, t_s, min(threads, wl.num_kv_heads))
+    times = []
+    for _ in range(args.steps):
+        dt, n = cpu_oracle_sample(wl, comp, tiers, bases, q, 0, t_s, min(threads, wl.num_kv_heads))
+        times.append(dt * ((T - 1) / t_s) * wl.num_layers * wl.num_kv_heads / n)
+    ms = statistics.mean(times) * 1e3
+    value = 1.0 / (ms * 1e-3)
+    used = min(threads, wl.num_kv_heads)
+    sample = (f"per step: layer 0, {n} kv-heads over the first {t_s} of {T - 1} cached tokens (fp64 C oracle on "
+              f"{used} threads), scaled linearly to the full context and x{wl.num_layers} layers")
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded compressed cache)",
+        "config": {"workload": args.workload, "layers": wl.num_layers, "kv_heads": wl.num_kv_heads,
+                   "context": T, "batch_per_gpu": 1},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="dwkv", choices=["dwkv", "reference"])
+    ap.add_argument("--workload", default="llama8b_64k")
+    ap.add_argument("--context", type=int, default=0, help="override the context length")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
+    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--profile-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tuning", default="", help="ctas_per_sm,waves,stages")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 1)
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            if rank != 0:
+                return
+            res = run_reference(args, world, rank, local)
+        else:
+            res = run_dwkv(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

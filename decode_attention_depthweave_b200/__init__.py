@@ -1,0 +1,321 @@
+"""Python binding of libdwkv: decode attention read directly from a DepthWeave-KV
+compressed KV cache on a B200 ("DepthWeave-KV: Token-Adaptive Cross-Layer Residual
+Factorization for Long-Context KV Cache Compression", §3 Method).
+
+Argument marshalling only.  Every step of the hot path runs in the CUDA kernels of
+``_lib/libdwkv.so``; the functions below have the names of the C ABI in
+``include/dwkv.h`` and take torch tensors (device pointers are passed through) or host
+integer lists.  PyTorch provides device memory and streams, nothing else.  There is no
+CPU fallback: importing this package fails if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+__all__ = [
+    "DwkvError", "dwkv_config", "lib", "config_from", "dwkv_version", "dwkv_last_error",
+    "dwkv_config_check", "dwkv_token_bytes", "dwkv_page_bytes", "dwkv_metadata_bytes",
+    "dwkv_arena_bytes", "dwkv_workspace_bytes", "dwkv_create", "dwkv_destroy",
+    "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
+    "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage",
+    "dwkv_sync_status", "dwkv_set_decode_tuning", "Cache", "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libdwkv.so")
+
+DWKV_OK = 0
+STATUS_NAMES = {0: "DWKV_OK", 1: "DWKV_ERR_INVALID_ARG", 2: "DWKV_ERR_CAPACITY", 3: "DWKV_ERR_CUDA",
+                4: "DWKV_ERR_DEVICE_CHECK", 5: "DWKV_ERR_UNSUPPORTED"}
+
+EXPORTED_SYMBOLS = (
+    "dwkv_version", "dwkv_last_error", "dwkv_config_check", "dwkv_token_bytes", "dwkv_page_bytes",
+    "dwkv_metadata_bytes", "dwkv_arena_bytes", "dwkv_workspace_bytes", "dwkv_create", "dwkv_destroy",
+    "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
+    "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage", "dwkv_sync_status",
+    "dwkv_set_decode_tuning",
+)
+
+
+class DwkvError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+
+
+class dwkv_config(C.Structure):
+    _fields_ = [
+        ("num_layers", C.c_int32), ("layers_per_group", C.c_int32), ("num_q_heads", C.c_int32),
+        ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32), ("r_max", C.c_int32),
+        ("num_tiers", C.c_int32), ("tiers", C.c_int32 * 8), ("resid_channels", C.c_int32),
+        ("resid_bits", C.c_int32), ("max_batch", C.c_int32), ("max_context", C.c_int32),
+        ("softmax_scale", C.c_float),
+    ]
+
+
+class dwkv_pool_stats(C.Structure):
+    _fields_ = [("data_bytes_total", C.c_uint64), ("data_bytes_reserved", C.c_uint64),
+                ("free_pages", C.c_uint32 * 8)]
+
+
+_LIB = None
+
+
+def lib():
+    """The loaded libdwkv (raises if it was not built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libdwkv is not built ({LIB_PATH} missing); run "
+                              "`python -m decode_attention_depthweave_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        vp, i32, sz = C.c_void_p, C.c_int32, C.c_size_t
+        cfgp = C.POINTER(dwkv_config)
+        sig = {
+            "dwkv_version": ([], C.c_char_p),
+            "dwkv_last_error": ([], C.c_char_p),
+            "dwkv_config_check": ([cfgp], C.c_int),
+            "dwkv_token_bytes": ([cfgp, i32], sz),
+            "dwkv_page_bytes": ([cfgp, i32], sz),
+            "dwkv_metadata_bytes": ([cfgp], sz),
+            "dwkv_arena_bytes": ([cfgp], sz),
+            "dwkv_workspace_bytes": ([cfgp, i32], sz),
+            "dwkv_create": ([cfgp, vp, sz, vp, vp, vp, C.POINTER(vp)], C.c_int),
+            "dwkv_destroy": ([vp], C.c_int),
+            "dwkv_reset_sequence": ([vp, i32, vp], C.c_int),
+            "dwkv_seq_length": ([vp, i32, i32, C.POINTER(i32)], C.c_int),
+            "dwkv_append": ([vp, i32, i32, vp, vp, vp, vp, vp, vp], C.c_int),
+            "dwkv_append_compressed": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], C.c_int),
+            "dwkv_decode_attention": ([vp, i32, i32, vp, vp, vp, vp, sz, vp], C.c_int),
+            "dwkv_probe": ([vp, i32, i32, vp, vp, vp, vp, vp, sz, vp], C.c_int),
+            "dwkv_export": ([vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], C.c_int),
+            "dwkv_pool_usage": ([vp, vp, C.POINTER(dwkv_pool_stats)], C.c_int),
+            "dwkv_sync_status": ([vp, vp], C.c_int),
+            "dwkv_set_decode_tuning": ([vp, i32, i32, i32], C.c_int),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _LIB = L
+    return _LIB
+
+
+def _check(status: int):
+    if status != DWKV_OK:
+        raise DwkvError(status, dwkv_last_error())
+
+
+def _ptr(t):
+    """Device / host pointer of a tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("tensors passed to libdwkv must be contiguous")
+        return C.c_void_p(t.data_ptr())
+    return t
+
+
+def _i32(xs):
+    arr = (C.c_int32 * max(len(xs), 1))(*[int(x) for x in xs])
+    return arr
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def config_from(num_layers, layers_per_group, num_q_heads, num_kv_heads, head_dim, r_max, tiers,
+                resid_channels, resid_bits, max_batch, max_context, softmax_scale=0.0) -> dwkv_config:
+    c = dwkv_config()
+    c.num_layers, c.layers_per_group = num_layers, layers_per_group
+    c.num_q_heads, c.num_kv_heads, c.head_dim, c.r_max = num_q_heads, num_kv_heads, head_dim, r_max
+    c.num_tiers = len(tiers)
+    for k, r in enumerate(tiers):
+        c.tiers[k] = int(r)
+    c.resid_channels, c.resid_bits = resid_channels, resid_bits
+    c.max_batch, c.max_context, c.softmax_scale = max_batch, max_context, float(softmax_scale)
+    return c
+
+
+# ------------------------------------------------------------------------------ C ABI
+def dwkv_version() -> str:
+    return lib().dwkv_version().decode()
+
+
+def dwkv_last_error() -> str:
+    return lib().dwkv_last_error().decode()
+
+
+def dwkv_config_check(cfg: dwkv_config) -> int:
+    return lib().dwkv_config_check(C.byref(cfg))
+
+
+def dwkv_token_bytes(cfg, tier) -> int:
+    return lib().dwkv_token_bytes(C.byref(cfg), tier)
+
+
+def dwkv_page_bytes(cfg, tier) -> int:
+    return lib().dwkv_page_bytes(C.byref(cfg), tier)
+
+
+def dwkv_metadata_bytes(cfg) -> int:
+    return lib().dwkv_metadata_bytes(C.byref(cfg))
+
+
+def dwkv_arena_bytes(cfg) -> int:
+    return lib().dwkv_arena_bytes(C.byref(cfg))
+
+
+def dwkv_workspace_bytes(cfg, n_seqs) -> int:
+    return lib().dwkv_workspace_bytes(C.byref(cfg), n_seqs)
+
+
+def dwkv_create(cfg, arena: torch.Tensor, basis_k: torch.Tensor, basis_v: torch.Tensor, stream=None,
+                arena_bytes=None) -> C.c_void_p:
+    h = C.c_void_p()
+    nbytes = arena.numel() * arena.element_size() if arena_bytes is None else arena_bytes
+    _check(lib().dwkv_create(C.byref(cfg), _ptr(arena), nbytes, _ptr(basis_k), _ptr(basis_v),
+                             _stream(stream), C.byref(h)))
+    return h
+
+
+def dwkv_destroy(h):
+    _check(lib().dwkv_destroy(h))
+
+
+def dwkv_reset_sequence(h, seq, stream=None):
+    _check(lib().dwkv_reset_sequence(h, seq, _stream(stream)))
+
+
+def dwkv_seq_length(h, seq, layer) -> int:
+    v = C.c_int32()
+    _check(lib().dwkv_seq_length(h, seq, layer, C.byref(v)))
+    return v.value
+
+
+def dwkv_append(h, layer, seq_ids, n_new, k_new, v_new, tier_idx, stream=None):
+    _check(lib().dwkv_append(h, layer, len(seq_ids), _i32(seq_ids), _i32(n_new), _ptr(k_new), _ptr(v_new),
+                             _ptr(tier_idx), _stream(stream)))
+
+
+def dwkv_append_compressed(h, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream=None):
+    _check(lib().dwkv_append_compressed(h, layer, len(seq_ids), _i32(seq_ids), _i32(n_new), _ptr(tier_idx),
+                                        _ptr(coeff), _ptr(idx), _ptr(codes), _ptr(scales), _stream(stream)))
+
+
+def dwkv_decode_attention(h, layer, seq_ids, q, out, workspace, stream=None):
+    _check(lib().dwkv_decode_attention(h, layer, len(seq_ids), _i32(seq_ids), _ptr(q), _ptr(out),
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(stream)))
+
+
+def dwkv_probe(h, layer, seq_ids, q, err, out_full, workspace, stream=None):
+    _check(lib().dwkv_probe(h, layer, len(seq_ids), _i32(seq_ids), _ptr(q), _ptr(err), _ptr(out_full),
+                            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dwkv_export(h, layer, seq, t0, n, tier_idx=None, coeff=None, idx=None, codes=None, scales=None, stream=None):
+    _check(lib().dwkv_export(h, layer, seq, t0, n, _ptr(tier_idx), _ptr(coeff), _ptr(idx), _ptr(codes),
+                             _ptr(scales), _stream(stream)))
+
+
+def dwkv_pool_usage(h, stream=None) -> dict:
+    s = dwkv_pool_stats()
+    _check(lib().dwkv_pool_usage(h, _stream(stream), C.byref(s)))
+    return {"data_bytes_total": s.data_bytes_total, "data_bytes_reserved": s.data_bytes_reserved,
+            "free_pages": list(s.free_pages)}
+
+
+def dwkv_sync_status(h, stream=None):
+    _check(lib().dwkv_sync_status(h, _stream(stream)))
+
+
+def dwkv_set_decode_tuning(h, ctas_per_sm=1, waves=1, stages=0):
+    _check(lib().dwkv_set_decode_tuning(h, ctas_per_sm, waves, stages))
+
+
+# ------------------------------------------------------------------------------ plumbing
+class Cache:
+    """Owns the torch allocations around one handle (arena and workspace) and exposes the
+    C ABI calls with tensors.  Allocation is torch's; computation is libdwkv's."""
+
+    def __init__(self, cfg: dwkv_config, basis_k: torch.Tensor, basis_v: torch.Tensor, device="cuda",
+                 arena_bytes=None, ws_seqs=None, stream=None):
+        if not torch.cuda.is_available():
+            raise RuntimeError("libdwkv needs a CUDA device")
+        _check(dwkv_config_check(cfg))
+        self.cfg = cfg
+        self.device = torch.device(device)
+        nbytes = dwkv_arena_bytes(cfg) if arena_bytes is None else int(arena_bytes)
+        self.arena = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        ws = dwkv_workspace_bytes(cfg, ws_seqs or cfg.max_batch)
+        self.workspace = torch.empty((ws + 15) // 16 * 4, dtype=torch.float32, device=self.device)
+        self.h = dwkv_create(cfg, self.arena, basis_k.to(self.device).contiguous(),
+                             basis_v.to(self.device).contiguous(), stream)
+
+    def close(self):
+        if getattr(self, "h", None):
+            dwkv_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def append(self, layer, seq_ids, n_new, k_new, v_new, tier_idx, stream=None):
+        dwkv_append(self.h, layer, seq_ids, n_new, k_new, v_new, tier_idx, stream)
+
+    def append_compressed(self, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream=None):
+        dwkv_append_compressed(self.h, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream)
+
+    def decode(self, layer, seq_ids, q, out=None, stream=None):
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        dwkv_decode_attention(self.h, layer, seq_ids, q, out, self.workspace, stream)
+        return out
+
+    def probe(self, layer, seq_ids, q, want_out=False, stream=None):
+        err = torch.empty(len(seq_ids), self.cfg.num_kv_heads, dtype=torch.float32, device=q.device)
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device) if want_out else None
+        dwkv_probe(self.h, layer, seq_ids, q, err, out, self.workspace, stream)
+        return (err, out) if want_out else err
+
+    def export(self, layer, seq, t0, n, stream=None):
+        c = self.cfg
+        H, R, s = c.num_kv_heads, c.r_max, c.resid_channels
+        dev = self.device
+        out = {
+            "tier_idx": torch.empty(n, H, dtype=torch.uint8, device=dev),
+            "coeff": torch.empty(n, H, 2, R, dtype=torch.bfloat16, device=dev),
+            "idx": torch.empty(n, H, 2, s, dtype=torch.uint8, device=dev),
+            "codes": torch.empty(n, H, 2, s, dtype=torch.int8, device=dev),
+            "scales": torch.empty(n, H, 2, dtype=torch.float16, device=dev),
+        }
+        if n:
+            dwkv_export(self.h, layer, seq, t0, n, out["tier_idx"], out["coeff"], out["idx"] if s else None,
+                        out["codes"] if s else None, out["scales"], stream)
+        return out
+
+    def reset(self, seq, stream=None):
+        dwkv_reset_sequence(self.h, seq, stream)
+
+    def seq_length(self, seq, layer) -> int:
+        return dwkv_seq_length(self.h, seq, layer)
+
+    def sync(self, stream=None):
+        dwkv_sync_status(self.h, stream)
+
+    def pool_usage(self, stream=None):
+        return dwkv_pool_usage(self.h, stream)
+
+    def set_decode_tuning(self, ctas_per_sm=1, waves=1, stages=0):
+        dwkv_set_decode_tuning(self.h, ctas_per_sm, waves, stages)

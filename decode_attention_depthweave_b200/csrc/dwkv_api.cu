@@ -1,0 +1,669 @@
+// dwkv_api.cu -- host side of libdwkv: argument checks, arena layout, launch set-up.
+// Every public entry point is declared (and documented) in include/dwkv.h.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "dwkv.h"
+#include "dwkv_common.cuh"
+
+namespace dwkv {
+__global__ void place_kernel(const Geom, const State, const AppendCall, const uint8_t*);
+template <int BITS>
+__global__ void encode_kernel(const Geom, const State, const AppendCall, const __nv_bfloat16*, const __nv_bfloat16*);
+template <int BITS>
+__global__ void import_kernel(const Geom, const State, const AppendCall, const __nv_bfloat16*, const uint8_t*,
+                              const int8_t*, const __half*);
+template <int BITS>
+__global__ void export_kernel(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*, uint8_t*,
+                              int8_t*, __half*);
+__global__ void reset_kernel(const Geom, const State, int);
+template <int BITS, bool PROBE>
+__global__ void decode_kernel(const Geom, const State, const DecodeCall);
+}  // namespace dwkv
+
+using namespace dwkv;
+
+namespace {
+
+thread_local std::string g_err;
+
+dwkv_status fail(dwkv_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+dwkv_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(DWKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define DWKV_CUDA(call, what)                            \
+    do {                                                 \
+        cudaError_t e_ = (call);                         \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+uint32_t next_pow2(uint64_t v) {
+    uint64_t p = 1;
+    while (p < v) p <<= 1;
+    return (uint32_t)std::min<uint64_t>(p, 1ull << 31);
+}
+
+bool is_pow2_rank(int r) { return r == 8 || r == 16 || r == 32 || r == 64 || r == 128; }
+
+dwkv_status check_cfg(const dwkv_config* c) {
+    if (!c) return fail(DWKV_ERR_INVALID_ARG, "config is NULL");
+    if (c->num_layers <= 0 || c->layers_per_group <= 0 || c->num_layers % c->layers_per_group)
+        return fail(DWKV_ERR_INVALID_ARG, "num_layers (%d) must be a positive multiple of layers_per_group (%d)",
+                    c->num_layers, c->layers_per_group);
+    if (c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->num_q_heads % c->num_kv_heads)
+        return fail(DWKV_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
+                    c->num_q_heads, c->num_kv_heads);
+    if (c->head_dim <= 0 || c->head_dim > 256)
+        return fail(DWKV_ERR_INVALID_ARG, "head_dim %d out of range", c->head_dim);
+    if (c->r_max <= 0 || c->r_max > c->head_dim || c->r_max % 8)
+        return fail(DWKV_ERR_INVALID_ARG, "r_max %d must be a multiple of 8 in [8, head_dim]", c->r_max);
+    if (c->num_tiers < 1 || c->num_tiers > DWKV_MAX_TIERS)
+        return fail(DWKV_ERR_INVALID_ARG, "num_tiers %d out of [1, %d]", c->num_tiers, DWKV_MAX_TIERS);
+    for (int k = 0; k < c->num_tiers; ++k) {
+        if (c->tiers[k] <= 0 || c->tiers[k] % 8 || c->tiers[k] > c->r_max)
+            return fail(DWKV_ERR_INVALID_ARG, "tier %d rank %d must be a multiple of 8 in [8, r_max]", k, c->tiers[k]);
+        if (k && c->tiers[k] <= c->tiers[k - 1])
+            return fail(DWKV_ERR_INVALID_ARG, "tiers must be strictly ascending");
+    }
+    if (c->resid_bits != 8 && c->resid_bits != 4)
+        return fail(DWKV_ERR_INVALID_ARG, "resid_bits must be 8 or 4 (got %d)", c->resid_bits);
+    if (c->resid_channels < 0 || c->resid_channels > c->head_dim || c->resid_channels % 8)
+        return fail(DWKV_ERR_INVALID_ARG, "resid_channels %d must be a multiple of 8 in [0, head_dim]",
+                    c->resid_channels);
+    if (c->max_batch <= 0 || c->max_context <= 0)
+        return fail(DWKV_ERR_INVALID_ARG, "max_batch and max_context must be positive");
+    if (c->max_context >= (1 << 24))
+        return fail(DWKV_ERR_INVALID_ARG, "max_context must be below 2^24");
+    if (!(c->softmax_scale <= 0.f) && !std::isfinite(c->softmax_scale))
+        return fail(DWKV_ERR_INVALID_ARG, "softmax_scale must be finite");
+    return DWKV_OK;
+}
+
+dwkv_status check_supported(const dwkv_config* c) {
+    if (c->head_dim != kD) return fail(DWKV_ERR_UNSUPPORTED, "this build has kernels for head_dim 128 only");
+    if (c->num_q_heads != kGQ * c->num_kv_heads)
+        return fail(DWKV_ERR_UNSUPPORTED, "this build has kernels for 4 query heads per kv head only");
+    if (!is_pow2_rank(c->r_max)) return fail(DWKV_ERR_UNSUPPORTED, "r_max must be one of 8, 16, 32, 64, 128");
+    for (int k = 0; k < c->num_tiers; ++k)
+        if (!is_pow2_rank(c->tiers[k]))
+            return fail(DWKV_ERR_UNSUPPORTED, "tier ranks must be among 8, 16, 32, 64, 128");
+    return DWKV_OK;
+}
+
+struct MetaLayout {
+    size_t err, bump, free_head, free_tail, free_list, counts, pages, slot_map, tickets, basis_k, basis_v, data;
+    uint32_t free_cap;
+};
+
+Geom make_geom(const dwkv_config* c) {
+    Geom G{};
+    G.L = c->num_layers;
+    G.LPG = c->layers_per_group;
+    G.G = c->num_layers / c->layers_per_group;
+    G.Hq = c->num_q_heads;
+    G.Hkv = c->num_kv_heads;
+    G.d = c->head_dim;
+    G.r_max = c->r_max;
+    G.ntiers = c->num_tiers;
+    G.s = c->resid_channels;
+    G.bits = c->resid_bits;
+    G.max_batch = c->max_batch;
+    G.max_context = c->max_context;
+    G.max_pages = (c->max_context + kPage - 1) / kPage;
+    G.tau = c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / std::sqrt((float)c->head_dim);
+    uint32_t stage = 0;
+    for (int k = 0; k < kMaxTiers; ++k) {
+        if (k < c->num_tiers) {
+            G.tiers[k] = c->tiers[k];
+            G.blk_bytes[k] = blk_bytes_of(c->tiers[k], G.s, G.bits);
+            G.chunk_bytes[k] = 2 * G.blk_bytes[k];
+            G.page_units[k] = G.LPG * G.chunk_bytes[k] / kUnit;
+            stage = std::max(stage, G.chunk_bytes[k]);
+        } else {
+            G.tiers[k] = 0;
+            G.blk_bytes[k] = G.chunk_bytes[k] = G.page_units[k] = 0;
+        }
+    }
+    G.stage_bytes = (uint32_t)align_up(stage, 128);
+    G.free_cap = next_pow2((uint64_t)c->max_batch * G.G * G.Hkv * G.max_pages);
+    return G;
+}
+
+MetaLayout meta_layout(const Geom& G) {
+    MetaLayout M{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+    M.free_cap = G.free_cap;
+    M.err = take(64);
+    M.bump = take(8);
+    M.free_head = take(4 * kMaxTiers);
+    M.free_tail = take(4 * kMaxTiers);
+    M.free_list = take((size_t)4 * kMaxTiers * G.free_cap);
+    M.counts = take((size_t)4 * G.max_batch * G.G * G.Hkv * kMaxTiers);
+    M.pages = take((size_t)4 * G.max_batch * G.G * G.Hkv * kMaxTiers * G.max_pages);
+    M.slot_map = take((size_t)4 * G.max_batch * G.G * G.Hkv * G.max_context);
+    M.tickets = take((size_t)4 * G.max_batch * G.Hkv);
+    M.basis_k = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
+    M.basis_v = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
+    M.data = o;
+    return M;
+}
+
+size_t worst_data_bytes(const Geom& G) {
+    uint32_t big = 0;
+    for (int k = 0; k < G.ntiers; ++k) big = std::max(big, G.page_units[k]);
+    const uint64_t pages_per_head = (uint64_t)G.max_pages + G.ntiers - 1;
+    return (size_t)G.max_batch * G.G * G.Hkv * pages_per_head * big * kUnit;
+}
+
+}  // namespace
+
+struct dwkv_ctx {
+    dwkv_config cfg;
+    Geom geom;
+    State st;
+    MetaLayout meta;
+    uint8_t* arena;
+    size_t arena_bytes;
+    int device, num_sms;
+    size_t smem_optin, smem_per_sm;
+    std::vector<int32_t> len;       // [max_batch][L]
+    std::vector<int32_t> placed;    // [max_batch][G]
+    int dec_ctas_per_sm = 1, dec_waves = 1, dec_stages_req = 0;
+};
+
+namespace {
+
+dwkv_status check_handle(dwkv_handle h) {
+    if (!h) return fail(DWKV_ERR_INVALID_ARG, "handle is NULL");
+    return DWKV_OK;
+}
+
+dwkv_status check_layer(dwkv_handle h, int32_t layer) {
+    if (layer < 0 || layer >= h->geom.L)
+        return fail(DWKV_ERR_INVALID_ARG, "layer %d out of [0, %d)", layer, h->geom.L);
+    return DWKV_OK;
+}
+
+dwkv_status check_seq_list(dwkv_handle h, int32_t n_seqs, const int32_t* seq_ids) {
+    if (n_seqs < 0 || n_seqs > kMaxSeqs)
+        return fail(DWKV_ERR_INVALID_ARG, "n_seqs %d out of [0, %d]", n_seqs, kMaxSeqs);
+    if (n_seqs && !seq_ids) return fail(DWKV_ERR_INVALID_ARG, "seq_ids is NULL");
+    std::vector<char> seen(h->geom.max_batch, 0);
+    for (int i = 0; i < n_seqs; ++i) {
+        const int s = seq_ids[i];
+        if (s < 0 || s >= h->geom.max_batch)
+            return fail(DWKV_ERR_INVALID_ARG, "sequence id %d out of [0, %d)", s, h->geom.max_batch);
+        if (seen[s]) return fail(DWKV_ERR_INVALID_ARG, "sequence id %d listed twice", s);
+        seen[s] = 1;
+    }
+    return DWKV_OK;
+}
+
+State make_state(uint8_t* arena, const MetaLayout& M, size_t arena_bytes) {
+    State S{};
+    S.err = reinterpret_cast<uint32_t*>(arena + M.err);
+    S.bump = reinterpret_cast<unsigned long long*>(arena + M.bump);
+    S.free_head = reinterpret_cast<uint32_t*>(arena + M.free_head);
+    S.free_tail = reinterpret_cast<uint32_t*>(arena + M.free_tail);
+    S.free_list = reinterpret_cast<uint32_t*>(arena + M.free_list);
+    S.counts = reinterpret_cast<uint32_t*>(arena + M.counts);
+    S.pages = reinterpret_cast<uint32_t*>(arena + M.pages);
+    S.slot_map = reinterpret_cast<uint32_t*>(arena + M.slot_map);
+    S.tickets = reinterpret_cast<uint32_t*>(arena + M.tickets);
+    S.basis_k = reinterpret_cast<const __nv_bfloat16*>(arena + M.basis_k);
+    S.basis_v = reinterpret_cast<const __nv_bfloat16*>(arena + M.basis_v);
+    S.data = arena + M.data;
+    S.data_units = (arena_bytes - M.data) / kUnit;
+    return S;
+}
+
+size_t encode_smem(const Geom& G) {
+    return (size_t)2 * kD * (G.r_max + 2) * 2 + (size_t)8 * (2 * kD + 2 * G.r_max + 64) * 4;
+}
+
+int decode_stages(dwkv_handle h, bool probe, size_t* smem_out) {
+    const Geom& G = h->geom;
+    const size_t budget = h->dec_ctas_per_sm == 1 ? h->smem_optin
+                                                  : std::min(h->smem_optin, h->smem_per_sm / 2 - 1024);
+    int best = 0;
+    const int cap = h->dec_stages_req > 0 ? h->dec_stages_req : 16;
+    for (int ns = kConsumerWarps; ns <= cap; ns += kConsumerWarps) {
+        const DecodeSmem L = decode_smem_layout(G, ns, probe);
+        if (L.total <= budget) { best = ns; *smem_out = L.total; }
+    }
+    return best;
+}
+
+dwkv_status prepare_call(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                         const int32_t* n_new, AppendCall& C, bool need_tiers, const void* tier_idx) {
+    const Geom& G = h->geom;
+    dwkv_status st;
+    if ((st = check_layer(h, layer)) != DWKV_OK) return st;
+    if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
+    if (n_seqs && !n_new) return fail(DWKV_ERR_INVALID_ARG, "n_new is NULL");
+    memset(&C, 0, sizeof(C));
+    C.n = n_seqs;
+    C.layer = layer;
+    C.g = layer / G.LPG;
+    C.lig = layer % G.LPG;
+    long long total = 0;
+    bool any_place = false;
+    for (int i = 0; i < n_seqs; ++i) {
+        const int s = seq_ids[i];
+        if (n_new[i] < 0) return fail(DWKV_ERR_INVALID_ARG, "n_new[%d] = %d is negative", i, n_new[i]);
+        const int pos0 = h->len[(size_t)s * G.L + layer];
+        const long long end = (long long)pos0 + n_new[i];
+        if (end > G.max_context)
+            return fail(DWKV_ERR_CAPACITY, "sequence %d would hold %lld tokens at layer %d (max_context %d)", s, end,
+                        layer, G.max_context);
+        const int placed = h->placed[(size_t)s * G.G + C.g];
+        C.seq[i] = s;
+        C.pos0[i] = pos0;
+        C.tok0[i] = (int)total;
+        C.a0[i] = std::max(pos0, placed);
+        C.na[i] = (int)std::max<long long>(0, end - C.a0[i]);
+        any_place |= C.na[i] > 0;
+        total += n_new[i];
+        if (total > (1ll << 30)) return fail(DWKV_ERR_INVALID_ARG, "too many tokens in one call");
+    }
+    C.tok0[n_seqs] = (int)total;
+    C.total = (int)total;
+    if (any_place && need_tiers && !tier_idx)
+        return fail(DWKV_ERR_INVALID_ARG, "tier_idx is NULL but layer %d is the first of its group to append "
+                                          "some of these positions", layer);
+    return DWKV_OK;
+}
+
+void commit_call(dwkv_handle h, const AppendCall& C, const int32_t* n_new) {
+    const Geom& G = h->geom;
+    for (int i = 0; i < C.n; ++i) {
+        const int s = C.seq[i];
+        const int end = C.pos0[i] + n_new[i];
+        h->len[(size_t)s * G.L + C.layer] = end;
+        int& pl = h->placed[(size_t)s * G.G + C.g];
+        pl = std::max(pl, end);
+    }
+}
+
+int grid_rows(dwkv_handle h, long long rows) {
+    const long long per = 8;  // warps per block
+    long long want = (rows + per - 1) / per;
+    const long long cap = std::max(1, 4 * h->num_sms / std::max(1, h->geom.Hkv));
+    return (int)std::max(1ll, std::min(want, cap));
+}
+
+}  // namespace
+
+// =============================================================================== C ABI
+extern "C" {
+
+const char* dwkv_version(void) { return "dwkv 0.1 (sm_100a)"; }
+
+const char* dwkv_last_error(void) { return g_err.c_str(); }
+
+dwkv_status dwkv_config_check(const dwkv_config* cfg) {
+    dwkv_status st = check_cfg(cfg);
+    if (st != DWKV_OK) return st;
+    return check_supported(cfg);
+}
+
+size_t dwkv_token_bytes(const dwkv_config* cfg, int32_t tier) {
+    if (check_cfg(cfg) != DWKV_OK || tier < 0 || tier >= cfg->num_tiers) return 0;
+    const int r = cfg->tiers[tier], s = cfg->resid_channels, b = cfg->resid_bits;
+    return (size_t)2 * (2 * r + s + s * b / 8 + 2);
+}
+
+size_t dwkv_page_bytes(const dwkv_config* cfg, int32_t tier) {
+    if (check_cfg(cfg) != DWKV_OK || tier < 0 || tier >= cfg->num_tiers) return 0;
+    const Geom G = make_geom(cfg);
+    return (size_t)G.page_units[tier] * kUnit;
+}
+
+size_t dwkv_metadata_bytes(const dwkv_config* cfg) {
+    if (check_cfg(cfg) != DWKV_OK) return 0;
+    return meta_layout(make_geom(cfg)).data;
+}
+
+size_t dwkv_arena_bytes(const dwkv_config* cfg) {
+    if (check_cfg(cfg) != DWKV_OK) return 0;
+    const Geom G = make_geom(cfg);
+    return meta_layout(G).data + worst_data_bytes(G);
+}
+
+size_t dwkv_workspace_bytes(const dwkv_config* cfg, int32_t n_seqs) {
+    if (check_cfg(cfg) != DWKV_OK || n_seqs < 0) return 0;
+    const Geom G = make_geom(cfg);
+    return (size_t)std::max(n_seqs, 1) * G.Hkv * kMaxSplits * rec_floats_of(G, true) * sizeof(float);
+}
+
+dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes, const void* basis_k,
+                        const void* basis_v, void* stream, dwkv_handle* out) {
+    dwkv_status st;
+    if (!out) return fail(DWKV_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if ((st = dwkv_config_check(cfg)) != DWKV_OK) return st;
+    if (!arena || !basis_k || !basis_v) return fail(DWKV_ERR_INVALID_ARG, "arena and bases must be non-NULL");
+    if (reinterpret_cast<uintptr_t>(arena) % 256) return fail(DWKV_ERR_INVALID_ARG, "arena must be 256-byte aligned");
+    const Geom G = make_geom(cfg);
+    const MetaLayout M = meta_layout(G);
+    uint32_t big = 0;
+    for (int k = 0; k < G.ntiers; ++k) big = std::max(big, G.page_units[k]);
+    if (arena_bytes < M.data + (size_t)big * kUnit)
+        return fail(DWKV_ERR_CAPACITY, "arena of %zu bytes is below the metadata (%zu) plus one page (%zu)",
+                    arena_bytes, M.data, (size_t)big * kUnit);
+    if ((arena_bytes - M.data) / kUnit >= (1ull << 32))
+        return fail(DWKV_ERR_UNSUPPORTED, "page pool above 512 GiB");
+    int dev = 0;
+    DWKV_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    cudaPointerAttributes pa{};
+    DWKV_CUDA(cudaPointerGetAttributes(&pa, arena), "cudaPointerGetAttributes(arena)");
+    if (pa.type != cudaMemoryTypeDevice || pa.device != dev)
+        return fail(DWKV_ERR_INVALID_ARG, "arena must be device memory of the current device %d", dev);
+    auto* h = new dwkv_ctx();
+    h->cfg = *cfg;
+    h->geom = G;
+    h->meta = M;
+    h->arena = static_cast<uint8_t*>(arena);
+    h->arena_bytes = arena_bytes;
+    h->st = make_state(h->arena, M, arena_bytes);
+    h->device = dev;
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    h->num_sms = v > 0 ? v : 1;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    h->smem_optin = (size_t)v;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    h->smem_per_sm = (size_t)v;
+    h->len.assign((size_t)G.max_batch * G.L, 0);
+    h->placed.assign((size_t)G.max_batch * G.G, 0);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bbytes = (size_t)2 * G.G * G.Hkv * G.d * G.r_max;
+    cudaError_t e = cudaMemsetAsync(h->arena, 0, M.basis_k, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(h->arena + M.basis_k, basis_k, bbytes, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(h->arena + M.basis_v, basis_v, bbytes, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) {
+        const int maxs = (int)h->smem_optin;
+        e = cudaFuncSetAttribute(decode_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel<8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
+    }
+    if (e != cudaSuccess) {
+        delete h;
+        return cuda_fail(e, "dwkv_create");
+    }
+    size_t sm = 0;
+    if (decode_stages(h, true, &sm) < kConsumerWarps) {
+        delete h;
+        return fail(DWKV_ERR_UNSUPPORTED, "decode pipeline does not fit in shared memory for this geometry");
+    }
+    *out = h;
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_destroy(dwkv_handle h) {
+    if (!h) return fail(DWKV_ERR_INVALID_ARG, "handle is NULL");
+    delete h;
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t waves, int32_t stages) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if (ctas_per_sm < 1 || ctas_per_sm > 2 || waves < 1 || waves > 8 || stages < 0 || stages > 32 ||
+        stages % kConsumerWarps)
+        return fail(DWKV_ERR_INVALID_ARG, "tuning out of range (ctas 1-2, waves 1-8, stages 0 or multiple of 4 <= 32)");
+    const int oc = h->dec_ctas_per_sm, ow = h->dec_waves, os = h->dec_stages_req;
+    h->dec_ctas_per_sm = ctas_per_sm;
+    h->dec_waves = waves;
+    h->dec_stages_req = stages;
+    size_t sm = 0;
+    if (decode_stages(h, true, &sm) < kConsumerWarps) {
+        h->dec_ctas_per_sm = oc; h->dec_waves = ow; h->dec_stages_req = os;
+        return fail(DWKV_ERR_INVALID_ARG, "tuning leaves no room for a 4-stage pipeline");
+    }
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_seq_length(dwkv_handle h, int32_t seq, int32_t layer, int32_t* len) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if ((st = check_layer(h, layer)) != DWKV_OK) return st;
+    if (seq < 0 || seq >= h->geom.max_batch) return fail(DWKV_ERR_INVALID_ARG, "sequence id %d out of range", seq);
+    if (!len) return fail(DWKV_ERR_INVALID_ARG, "len is NULL");
+    *len = h->len[(size_t)seq * h->geom.L + layer];
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_reset_sequence(dwkv_handle h, int32_t seq, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    const Geom& G = h->geom;
+    if (seq < 0 || seq >= G.max_batch) return fail(DWKV_ERR_INVALID_ARG, "sequence id %d out of range", seq);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    reset_kernel<<<1, 256, 0, s>>>(G, h->st, seq);
+    DWKV_CUDA(cudaGetLastError(), "reset_kernel launch");
+    DWKV_CUDA(cudaMemsetAsync(h->st.slot_map + slot_index(G, seq, 0, 0, 0), 0,
+                              (size_t)4 * G.G * G.Hkv * G.max_context, s),
+              "cudaMemsetAsync(slot map)");
+    std::fill(h->len.begin() + (size_t)seq * G.L, h->len.begin() + (size_t)(seq + 1) * G.L, 0);
+    std::fill(h->placed.begin() + (size_t)seq * G.G, h->placed.begin() + (size_t)(seq + 1) * G.G, 0);
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const int32_t* n_new,
+                        const void* k_new, const void* v_new, const uint8_t* tier_idx, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    AppendCall C;
+    if ((st = prepare_call(h, layer, n_seqs, seq_ids, n_new, C, true, tier_idx)) != DWKV_OK) return st;
+    if (C.total == 0) return DWKV_OK;
+    if (!k_new || !v_new) return fail(DWKV_ERR_INVALID_ARG, "k_new and v_new must be non-NULL");
+    const Geom& G = h->geom;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    bool any = false;
+    for (int i = 0; i < C.n; ++i) any |= C.na[i] > 0;
+    if (any) {
+        place_kernel<<<dim3(C.n, G.Hkv), 256, 0, s>>>(G, h->st, C, tier_idx);
+        DWKV_CUDA(cudaGetLastError(), "place_kernel launch");
+    }
+    const dim3 grid(grid_rows(h, C.total), G.Hkv);
+    const size_t sm = encode_smem(G);
+    if (G.bits == 8)
+        encode_kernel<8><<<grid, 256, sm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
+                                                static_cast<const __nv_bfloat16*>(v_new));
+    else
+        encode_kernel<4><<<grid, 256, sm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
+                                                static_cast<const __nv_bfloat16*>(v_new));
+    DWKV_CUDA(cudaGetLastError(), "encode_kernel launch");
+    commit_call(h, C, n_new);
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_append_compressed(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                                   const int32_t* n_new, const uint8_t* tier_idx, const void* coeff,
+                                   const uint8_t* idx, const int8_t* codes, const void* scales, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    AppendCall C;
+    if ((st = prepare_call(h, layer, n_seqs, seq_ids, n_new, C, true, tier_idx)) != DWKV_OK) return st;
+    if (C.total == 0) return DWKV_OK;
+    const Geom& G = h->geom;
+    if (!coeff || !scales || (G.s > 0 && (!idx || !codes)))
+        return fail(DWKV_ERR_INVALID_ARG, "coeff, idx, codes and scales must be non-NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    bool any = false;
+    for (int i = 0; i < C.n; ++i) any |= C.na[i] > 0;
+    if (any) {
+        place_kernel<<<dim3(C.n, G.Hkv), 256, 0, s>>>(G, h->st, C, tier_idx);
+        DWKV_CUDA(cudaGetLastError(), "place_kernel launch");
+    }
+    const dim3 grid(grid_rows(h, C.total), G.Hkv);
+    if (G.bits == 8)
+        import_kernel<8><<<grid, 256, 0, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(coeff), idx, codes,
+                                              static_cast<const __half*>(scales));
+    else
+        import_kernel<4><<<grid, 256, 0, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(coeff), idx, codes,
+                                              static_cast<const __half*>(scales));
+    DWKV_CUDA(cudaGetLastError(), "import_kernel launch");
+    commit_call(h, C, n_new);
+    return DWKV_OK;
+}
+
+static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const void* q,
+                              float* out, float* err, float* out_full, void* workspace, size_t ws_bytes,
+                              void* stream, bool probe) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if ((st = check_layer(h, layer)) != DWKV_OK) return st;
+    if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
+    if (n_seqs == 0) return DWKV_OK;
+    const Geom& G = h->geom;
+    if (!q) return fail(DWKV_ERR_INVALID_ARG, "q is NULL");
+    if (!probe && !out) return fail(DWKV_ERR_INVALID_ARG, "out is NULL");
+    if (probe && !err) return fail(DWKV_ERR_INVALID_ARG, "err is NULL");
+    if (!workspace) return fail(DWKV_ERR_INVALID_ARG, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(workspace) % 16) return fail(DWKV_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    const size_t need = dwkv_workspace_bytes(&h->cfg, n_seqs);
+    if (ws_bytes < need) return fail(DWKV_ERR_CAPACITY, "workspace of %zu bytes is below the %zu needed", ws_bytes, need);
+    const int g = layer / G.LPG;
+    long long tot = 0;
+    for (int i = 0; i < n_seqs; ++i) {
+        const int s = seq_ids[i];
+        const int len = h->len[(size_t)s * G.L + layer], pl = h->placed[(size_t)s * G.G + g];
+        if (len != pl)
+            return fail(DWKV_ERR_INVALID_ARG, "sequence %d holds %d positions at layer %d but its group placed %d; "
+                                              "append every layer of the group before decoding it", s, len, layer, pl);
+        tot += len;
+    }
+    DecodeCall C;
+    memset(&C, 0, sizeof(C));
+    C.n = n_seqs;
+    C.layer = layer;
+    C.g = g;
+    C.lig = layer % G.LPG;
+    const long long target = (long long)h->num_sms * h->dec_ctas_per_sm * h->dec_waves;
+    int total = 0;
+    for (int i = 0; i < n_seqs; ++i) {
+        const int s = seq_ids[i];
+        const long long len = h->len[(size_t)s * G.L + layer];
+        long long sp = tot > 0 ? (target * len) / (tot * G.Hkv) : 1;
+        const long long pages = std::max(1ll, (len + kPage - 1) / kPage);
+        sp = std::max(1ll, std::min({sp, (long long)kMaxSplits, pages}));
+        C.seq[i] = s;
+        C.split_begin[i] = total;
+        total += (int)sp;
+    }
+    C.split_begin[n_seqs] = total;
+    C.total_splits = total;
+    size_t smem = 0;
+    C.stages = decode_stages(h, probe, &smem);
+    C.rec_floats = rec_floats_of(G, probe);
+    C.q = static_cast<const __nv_bfloat16*>(q);
+    C.out = out;
+    C.out_full = out_full;
+    C.err = err;
+    C.ws = static_cast<float*>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 grid(total, G.Hkv);
+    if (!probe) {
+        if (G.bits == 8) decode_kernel<8, false><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C);
+        else decode_kernel<4, false><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C);
+    } else {
+        if (G.bits == 8) decode_kernel<8, true><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C);
+        else decode_kernel<4, true><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C);
+    }
+    DWKV_CUDA(cudaGetLastError(), probe ? "probe kernel launch" : "decode kernel launch");
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_decode_attention(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                                  const void* q, float* out, void* workspace, size_t ws_bytes, void* stream) {
+    return run_decode(h, layer, n_seqs, seq_ids, q, out, nullptr, nullptr, workspace, ws_bytes, stream, false);
+}
+
+dwkv_status dwkv_probe(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const void* q,
+                       float* err, float* out_full, void* workspace, size_t ws_bytes, void* stream) {
+    return run_decode(h, layer, n_seqs, seq_ids, q, nullptr, err, out_full, workspace, ws_bytes, stream, true);
+}
+
+dwkv_status dwkv_export(dwkv_handle h, int32_t layer, int32_t seq, int32_t t0, int32_t n, uint8_t* tier_idx,
+                        void* coeff, uint8_t* idx, int8_t* codes, void* scales, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if ((st = check_layer(h, layer)) != DWKV_OK) return st;
+    const Geom& G = h->geom;
+    if (seq < 0 || seq >= G.max_batch) return fail(DWKV_ERR_INVALID_ARG, "sequence id %d out of range", seq);
+    const int len = h->len[(size_t)seq * G.L + layer];
+    if (t0 < 0 || n < 0 || (long long)t0 + n > len)
+        return fail(DWKV_ERR_INVALID_ARG, "positions [%d, %lld) outside the %d held", t0, (long long)t0 + n, len);
+    if (n == 0) return DWKV_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int grid = (int)std::min<long long>(((long long)n * G.Hkv + 7) / 8, 4096);
+    if (G.bits == 8)
+        export_kernel<8><<<grid, 256, 0, s>>>(G, h->st, layer, seq, t0, n, tier_idx,
+                                              static_cast<__nv_bfloat16*>(coeff), idx, codes, static_cast<__half*>(scales));
+    else
+        export_kernel<4><<<grid, 256, 0, s>>>(G, h->st, layer, seq, t0, n, tier_idx,
+                                              static_cast<__nv_bfloat16*>(coeff), idx, codes, static_cast<__half*>(scales));
+    DWKV_CUDA(cudaGetLastError(), "export_kernel launch");
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_pool_usage(dwkv_handle h, void* stream, dwkv_pool_stats* out) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if (!out) return fail(DWKV_ERR_INVALID_ARG, "out is NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DWKV_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+    unsigned long long bump = 0;
+    uint32_t hd[kMaxTiers], tl[kMaxTiers];
+    DWKV_CUDA(cudaMemcpy(&bump, h->st.bump, 8, cudaMemcpyDeviceToHost), "read pool");
+    DWKV_CUDA(cudaMemcpy(hd, h->st.free_head, sizeof(hd), cudaMemcpyDeviceToHost), "read pool");
+    DWKV_CUDA(cudaMemcpy(tl, h->st.free_tail, sizeof(tl), cudaMemcpyDeviceToHost), "read pool");
+    memset(out, 0, sizeof(*out));
+    out->data_bytes_total = (uint64_t)h->st.data_units * kUnit;
+    out->data_bytes_reserved = std::min<uint64_t>(bump, h->st.data_units) * kUnit;
+    for (int k = 0; k < h->geom.ntiers; ++k) out->free_pages[k] = (int)(tl[k] - hd[k]) > 0 ? tl[k] - hd[k] : 0;
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_sync_status(dwkv_handle h, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DWKV_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+    uint32_t w[3] = {0, 0, 0};
+    DWKV_CUDA(cudaMemcpy(w, h->st.err, sizeof(w), cudaMemcpyDeviceToHost), "read device error word");
+    if (w[0] == 0) return DWKV_OK;
+    DWKV_CUDA(cudaMemset(h->st.err, 0, sizeof(w)), "clear device error word");
+    static const char* names[] = {"none", "page pool exhausted", "tier index out of range",
+                                  "residual channel index out of range", "int4 code outside [-8, 7]",
+                                  "position never placed by its group", "bounded wait timed out",
+                                  "free-page ring overflow"};
+    const char* nm = w[0] < sizeof(names) / sizeof(names[0]) ? names[w[0]] : "unknown";
+    return fail(DWKV_ERR_DEVICE_CHECK, "device check failed: %s (code %u, info %u, %u)", nm, w[0], w[1], w[2]);
+}
+
+}  // extern "C"

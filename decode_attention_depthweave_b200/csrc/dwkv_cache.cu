@@ -1,0 +1,467 @@
+// dwkv_cache.cu -- page placement, encode/append, import, export and reset kernels.
+//
+// Encode follows "DepthWeave-KV: Token-Adaptive Cross-Layer Residual Factorization for
+// Long-Context KV Cache Compression", §3 Method (coefficients are the projection of the
+// original vector onto the current basis; the residual is quantised and kept only on the
+// routed channels), in this library's fixed fp32 operation order, which makes the
+// stored bytes reproducible bit for bit:
+//   1. c_j  = fma chain over i = 0..d-1 of B[i][j] * x_i from +0            (j < r_t)
+//   2. cb_j = bf16_rn(c_j)                                                 (stored)
+//   3. r_i  = x_i - a_i, a_i = fma chain over j = 0..r_t-1 of B[i][j] * cb_j from +0
+//   4. the s largest |r_i|, ties to the lower channel, stored in ascending channel order
+//   5. scale = fp16_rn(max |r_sel| / qmax) with IEEE division, qmax = 127 (int8) / 7 (int4)
+//   6. code  = clamp(rint(r / float(scale)), -qmax, qmax), all zero when scale == 0
+#include "dwkv_common.cuh"
+
+namespace dwkv {
+
+// ------------------------------------------------------------------------------------
+// Slot placement for the group's first layer that appends a position.  One block per
+// (sequence in call, kv-head).  Slots inside a tier are numbered in position order; new
+// pages come from the tier's free ring first, then from the pool's bump pointer.
+// ------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) place_kernel(const Geom G, const State S, const AppendCall C,
+                                                    const uint8_t* __restrict__ tier_idx) {
+    const int i = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int na = C.na[i];
+    if (na <= 0) return;
+    const int seq = C.seq[i], a0 = C.a0[i];
+    const int rowbase = C.tok0[i] + (a0 - C.pos0[i]);
+    __shared__ uint32_t s_cnt[kMaxTiers], s_old[kMaxTiers], s_run[kMaxTiers], s_fail;
+    __shared__ uint32_t s_warp[8][kMaxTiers];
+    const size_t ci = cnt_index(G, seq, C.g, h);
+    if (tid < kMaxTiers) {
+        s_cnt[tid] = 0;
+        s_old[tid] = tid < G.ntiers ? S.counts[ci + tid] : 0u;
+    }
+    if (tid == 0) s_fail = 0;
+    __syncthreads();
+    for (int p = tid; p < na; p += blockDim.x) {
+        uint32_t k = tier_idx[(size_t)(rowbase + p) * G.Hkv + h];
+        if (k < (uint32_t)G.ntiers) atomicAdd(&s_cnt[k], 1u);
+        else set_dev_error(S, 2u /*DWKV_DEV_BAD_TIER*/, (uint32_t)seq, (uint32_t)(a0 + p));
+    }
+    __syncthreads();
+    if (tid < G.ntiers) {
+        const int k = tid;
+        const uint32_t old = s_old[k], nw = old + s_cnt[k];
+        const uint32_t po = (old + kPage - 1) / kPage, pn = (nw + kPage - 1) / kPage;
+        const size_t pi = page_index(G, seq, C.g, h, k);
+        if (pn > (uint32_t)G.max_pages) {
+            set_dev_error(S, 1u /*DWKV_DEV_POOL_EXHAUSTED*/, (uint32_t)seq, (uint32_t)h);
+            s_fail = 1;
+        } else if (pn > po) {
+            const uint32_t need = pn - po;
+            const uint32_t t = atomicAdd(&S.free_head[k], need);
+            const uint32_t tail = *((volatile uint32_t*)&S.free_tail[k]);
+            const int avail = (int)(tail - t);
+            const uint32_t take = avail <= 0 ? 0u : ((uint32_t)avail < need ? (uint32_t)avail : need);
+            for (uint32_t q = 0; q < take; ++q)
+                S.pages[pi + po + q] = S.free_list[(size_t)k * G.free_cap + ((t + q) & (G.free_cap - 1))];
+            const uint32_t rest = need - take;
+            if (rest) {
+                const unsigned long long units = (unsigned long long)rest * G.page_units[k];
+                const unsigned long long base = atomicAdd(S.bump, units);
+                if (base + units > S.data_units) {
+                    set_dev_error(S, 1u /*DWKV_DEV_POOL_EXHAUSTED*/, (uint32_t)seq, (uint32_t)h);
+                    s_fail = 1;
+                } else {
+                    for (uint32_t q = 0; q < rest; ++q)
+                        S.pages[pi + po + take + q] = (uint32_t)(base + (unsigned long long)q * G.page_units[k]);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    const size_t si = slot_index(G, seq, C.g, h, a0);
+    if (s_fail) {
+        for (int p = tid; p < na; p += blockDim.x) S.slot_map[si + p] = 0u;
+        return;
+    }
+    if (tid < kMaxTiers) s_run[tid] = s_old[tid];
+    __syncthreads();
+    for (int base = 0; base < na; base += blockDim.x) {
+        const int p = base + tid;
+        uint32_t k = 0xffu;
+        if (p < na) {
+            k = tier_idx[(size_t)(rowbase + p) * G.Hkv + h];
+            if (k >= (uint32_t)G.ntiers) k = 0xffu;
+        }
+        uint32_t rank = 0;
+        for (int kk = 0; kk < G.ntiers; ++kk) {
+            const uint32_t m = __ballot_sync(0xffffffffu, k == (uint32_t)kk);
+            if (k == (uint32_t)kk) rank = __popc(m & ((1u << lane) - 1u));
+            if (lane == 0) s_warp[warp][kk] = __popc(m);
+        }
+        __syncthreads();
+        if (p < na) {
+            if (k != 0xffu) {
+                uint32_t off = s_run[k];
+                for (int w = 0; w < warp; ++w) off += s_warp[w][k];
+                S.slot_map[si + p] = ((k + 1u) << 24) | (off + rank);
+            } else {
+                S.slot_map[si + p] = 0u;
+            }
+        }
+        __syncthreads();
+        if (tid < G.ntiers) {
+            uint32_t tot = 0;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += s_warp[w][tid];
+            s_run[tid] += tot;
+        }
+        __syncthreads();
+    }
+    if (tid < G.ntiers) S.counts[ci + tid] = s_old[tid] + s_cnt[tid];
+}
+
+// Row of the call's input arrays -> (index in call, sequence, position).
+__device__ __forceinline__ int call_index_of(const AppendCall& C, int row) {
+    int lo = 0, hi = C.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (C.tok0[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Destination block of (sequence, group, kv-head, position) at a layer, or nullptr.
+struct Dest {
+    uint8_t* blk;   // K block; V block = blk + blk_bytes
+    int k, row, R;
+};
+__device__ __forceinline__ bool find_dest(const Geom& G, const State& S, int seq, int g, int lig, int h,
+                                          int pos, Dest& d) {
+    const uint32_t sm = S.slot_map[slot_index(G, seq, g, h, pos)];
+    if (sm == 0u) return false;
+    const int k = (int)(sm >> 24) - 1;
+    const uint32_t slot = sm & 0xffffffu;
+    const uint32_t unit = S.pages[page_index(G, seq, g, h, k) + slot / kPage];
+    d.k = k;
+    d.row = (int)(slot % kPage);
+    d.R = G.tiers[k];
+    d.blk = S.data + (size_t)unit * kUnit + (size_t)lig * G.chunk_bytes[k];
+    return true;
+}
+
+// ------------------------------------------------------------------------------------
+// Encode kernel: one warp per token (keys and values together), block per kv-head slice.
+// The (group, kv-head) bases sit in shared memory as bf16 with a padded row pitch so that
+// both the projection (lanes along j) and the residual (lanes along i) are conflict-free.
+// ------------------------------------------------------------------------------------
+template <int BITS>
+__global__ void __launch_bounds__(256) encode_kernel(const Geom G, const State S, const AppendCall C,
+                                                     const __nv_bfloat16* __restrict__ k_new,
+                                                     const __nv_bfloat16* __restrict__ v_new) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int RM = G.r_max, P = G.r_max + 2, s = G.s;
+    __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem);              // [2][d][P]
+    float* ws_all = reinterpret_cast<float*>(smem + (size_t)2 * kD * P * 2);  // per warp
+    const int wfl = 2 * kD + 2 * RM;                                          // floats per warp
+    float* xs = ws_all + (size_t)warp * (wfl + 64);      // [2][d]
+    float* cs = xs + 2 * kD;                             // [2][r_max]
+    int8_t* cstage = reinterpret_cast<int8_t*>(cs + 2 * RM);  // [2][128] code staging
+
+    const size_t boff = ((size_t)C.g * G.Hkv + h) * kD * RM;
+    for (int e = tid; e < kD * RM; e += blockDim.x) {
+        const int i = e / RM, j = e % RM;
+        bs[i * P + j] = S.basis_k[boff + e];
+        bs[kD * P + i * P + j] = S.basis_v[boff + e];
+    }
+    __syncthreads();
+
+    const float qmax = BITS == 8 ? 127.f : 7.f;
+    const int nw = blockDim.x >> 5;
+    for (int row = blockIdx.x * nw + warp; row < C.total; row += gridDim.x * nw) {
+        const int ci = call_index_of(C, row);
+        const int seq = C.seq[ci];
+        const int pos = C.pos0[ci] + (row - C.tok0[ci]);
+        Dest dst;
+        if (!find_dest(G, S, seq, C.g, C.lig, h, pos, dst)) {
+            // a0..a0+na were placed by place_kernel; a zero entry means placement failed
+            // (already reported) or the group never placed this position.
+            if (lane == 0 && !(pos >= C.a0[ci] && pos < C.a0[ci] + C.na[ci]))
+                set_dev_error(S, 5u /*DWKV_DEV_NO_SLOT*/, (uint32_t)seq, (uint32_t)pos);
+            continue;
+        }
+        const int R = dst.R;
+        // ---- load x (keys at z=0, values at z=1)
+        float xr[2][4];
+        const __nv_bfloat16* src[2] = {k_new + ((size_t)row * G.Hkv + h) * kD,
+                                       v_new + ((size_t)row * G.Hkv + h) * kD};
+#pragma unroll
+        for (int z = 0; z < 2; ++z)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                xr[z][m] = __bfloat162float(src[z][lane + 32 * m]);
+                xs[z * kD + lane + 32 * m] = xr[z][m];
+            }
+        __syncwarp();
+        // ---- 1-2: projection, bf16 rounding, coefficient store
+        for (int j = lane; j < R; j += 32) {
+            float a0 = 0.f, a1 = 0.f;
+            const __nv_bfloat16* b0 = bs + j;
+            const __nv_bfloat16* b1 = bs + kD * P + j;
+#pragma unroll 8
+            for (int i = 0; i < kD; ++i) {
+                a0 = __fmaf_rn(__bfloat162float(b0[i * P]), xs[i], a0);
+                a1 = __fmaf_rn(__bfloat162float(b1[i * P]), xs[kD + i], a1);
+            }
+            const __nv_bfloat16 c0 = __float2bfloat16_rn(a0), c1 = __float2bfloat16_rn(a1);
+            cs[j] = __bfloat162float(c0);
+            cs[RM + j] = __bfloat162float(c1);
+            const size_t co = (size_t)(j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2;
+            *reinterpret_cast<__nv_bfloat16*>(dst.blk + co) = c0;
+            *reinterpret_cast<__nv_bfloat16*>(dst.blk + G.blk_bytes[dst.k] + co) = c1;
+        }
+        __syncwarp();
+        // ---- 3: residual against the stored coefficients
+        float r[2][4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int i = lane + 32 * m;
+            float a0 = 0.f, a1 = 0.f;
+            const __nv_bfloat16* b0 = bs + i * P;
+            const __nv_bfloat16* b1 = bs + kD * P + i * P;
+            for (int j = 0; j < R; ++j) {
+                a0 = __fmaf_rn(__bfloat162float(b0[j]), cs[j], a0);
+                a1 = __fmaf_rn(__bfloat162float(b1[j]), cs[RM + j], a1);
+            }
+            r[0][m] = __fsub_rn(xr[0][m], a0);
+            r[1][m] = __fsub_rn(xr[1][m], a1);
+        }
+        // ---- 4: top-s by magnitude, ties to the lower channel (channel = lane + 32 m)
+        uint32_t key[2][4], sel[2] = {0u, 0u};
+#pragma unroll
+        for (int z = 0; z < 2; ++z)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) key[z][m] = __float_as_uint(fabsf(r[z][m])) + 1u;
+        for (int it = 0; it < s; ++it) {
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+                uint32_t best = 0u, bm = 0u;
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    if (!((sel[z] >> m) & 1u) && key[z][m] > best) { best = key[z][m]; bm = (uint32_t)m; }
+                const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
+                const uint32_t cand = (best == wmax && best != 0u) ? (bm * 32u + (uint32_t)lane) : 0xffffffffu;
+                const uint32_t wch = __reduce_min_sync(0xffffffffu, cand);
+                if ((int)(wch & 31u) == lane) sel[z] |= 1u << (wch >> 5);
+            }
+        }
+        // ---- 5-6: scale and codes; ranks give ascending channel order
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+            uint32_t mx = 0u;
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                if ((sel[z] >> m) & 1u) mx = max(mx, key[z][m] - 1u);
+            const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, mx));
+            const __half sh = __float2half_rn(__fdiv_rn(amax, qmax));
+            const float sf = __half2float(sh);
+            uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
+            uint32_t before = 0u;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const bool on = (sel[z] >> m) & 1u;
+                const uint32_t bal = __ballot_sync(0xffffffffu, on);
+                if (on) {
+                    const int rank = (int)(before + __popc(bal & ((1u << lane) - 1u)));
+                    float c = 0.f;
+                    if (sf != 0.f) c = fminf(fmaxf(rintf(__fdiv_rn(r[z][m], sf)), -qmax), qmax);
+                    blk[off_idx_of(R) + dst.row * s + rank] = (uint8_t)(lane + 32 * m);
+                    if (BITS == 8) blk[off_codes_of(R, s) + dst.row * s + rank] = (uint8_t)(int8_t)c;
+                    else cstage[z * 128 + rank] = (int8_t)c;
+                }
+                before += __popc(bal);
+            }
+            if (lane == 0) *reinterpret_cast<__half*>(blk + off_scales_of(R, s, BITS) + dst.row * 2) = sh;
+        }
+        if (BITS == 4) {
+            __syncwarp();
+            for (int e = lane; e < s; e += 32) {        // e indexes (z, byte) pairs: s/2 bytes per z
+                const int z = e / (s / 2), b = e % (s / 2);
+                const uint8_t lo = (uint8_t)cstage[z * 128 + 2 * b] & 0xfu;
+                const uint8_t hi = (uint8_t)cstage[z * 128 + 2 * b + 1] & 0xfu;
+                uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
+                blk[off_codes_of(R, s) + dst.row * (s / 2) + b] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Import of already compressed tokens: one warp per token row (keys and values).
+// ------------------------------------------------------------------------------------
+template <int BITS>
+__global__ void __launch_bounds__(256) import_kernel(const Geom G, const State S, const AppendCall C,
+                                                     const __nv_bfloat16* __restrict__ coeff,
+                                                     const uint8_t* __restrict__ idx,
+                                                     const int8_t* __restrict__ codes,
+                                                     const __half* __restrict__ scales) {
+    const int h = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nw = blockDim.x >> 5, s = G.s, RM = G.r_max;
+    for (int row = blockIdx.x * nw + warp; row < C.total; row += gridDim.x * nw) {
+        const int ci = call_index_of(C, row);
+        const int seq = C.seq[ci];
+        const int pos = C.pos0[ci] + (row - C.tok0[ci]);
+        Dest dst;
+        if (!find_dest(G, S, seq, C.g, C.lig, h, pos, dst)) {
+            if (lane == 0 && !(pos >= C.a0[ci] && pos < C.a0[ci] + C.na[ci]))
+                set_dev_error(S, 5u, (uint32_t)seq, (uint32_t)pos);
+            continue;
+        }
+        const int R = dst.R;
+        for (int z = 0; z < 2; ++z) {
+            const size_t src = ((size_t)row * G.Hkv + h) * 2 + z;
+            uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
+            for (int j = lane; j < R; j += 32)
+                *reinterpret_cast<__nv_bfloat16*>(blk + (j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2) =
+                    coeff[src * RM + j];
+            for (int e = lane; e < s; e += 32) {
+                const uint8_t ch = idx[src * s + e];
+                if (ch >= kD) set_dev_error(S, 3u /*DWKV_DEV_BAD_CHANNEL*/, (uint32_t)seq, (uint32_t)pos);
+                blk[off_idx_of(R) + dst.row * s + e] = ch;
+                if (BITS == 8) blk[off_codes_of(R, s) + dst.row * s + e] = (uint8_t)codes[src * s + e];
+            }
+            if (BITS == 4) {
+                for (int b = lane; b < s / 2; b += 32) {
+                    const int c0 = codes[src * s + 2 * b], c1 = codes[src * s + 2 * b + 1];
+                    if (c0 < -8 || c0 > 7 || c1 < -8 || c1 > 7)
+                        set_dev_error(S, 4u /*DWKV_DEV_BAD_CODE*/, (uint32_t)seq, (uint32_t)pos);
+                    blk[off_codes_of(R, s) + dst.row * (s / 2) + b] =
+                        (uint8_t)(((uint32_t)c0 & 0xfu) | (((uint32_t)c1 & 0xfu) << 4));
+                }
+            }
+            if (lane == 0)
+                *reinterpret_cast<__half*>(blk + off_scales_of(R, s, BITS) + dst.row * 2) = scales[src];
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Export of positions [t0, t0+n) of (layer, seq), token-ordered.  One warp per (token, h).
+// ------------------------------------------------------------------------------------
+template <int BITS>
+__global__ void __launch_bounds__(256) export_kernel(const Geom G, const State S, int layer, int seq, int t0,
+                                                     int n, uint8_t* tier_out, __nv_bfloat16* coeff_out,
+                                                     uint8_t* idx_out, int8_t* codes_out, __half* scales_out) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int g = layer / G.LPG, lig = layer % G.LPG, s = G.s, RM = G.r_max;
+    for (int w = blockIdx.x * nw + warp; w < n * G.Hkv; w += gridDim.x * nw) {
+        const int t = w / G.Hkv, h = w % G.Hkv;
+        Dest dst;
+        const bool ok = find_dest(G, S, seq, g, lig, h, t0 + t, dst);
+        if (tier_out && lane == 0) tier_out[w] = ok ? (uint8_t)dst.k : (uint8_t)0xff;
+        for (int z = 0; z < 2; ++z) {
+            const size_t o = (size_t)w * 2 + z;
+            const uint8_t* blk = ok ? dst.blk + (z ? G.blk_bytes[dst.k] : 0u) : nullptr;
+            const int R = ok ? dst.R : 0;
+            if (coeff_out)
+                for (int j = lane; j < RM; j += 32)
+                    coeff_out[o * RM + j] = j < R ? *reinterpret_cast<const __nv_bfloat16*>(
+                                                        blk + (j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2)
+                                                  : __float2bfloat16_rn(0.f);
+            for (int e = lane; e < s; e += 32) {
+                if (idx_out) idx_out[o * s + e] = ok ? blk[off_idx_of(R) + dst.row * s + e] : 0;
+                if (codes_out) {
+                    int c = 0;
+                    if (ok) {
+                        if (BITS == 8) c = (int8_t)blk[off_codes_of(R, s) + dst.row * s + e];
+                        else {
+                            const uint32_t byte = blk[off_codes_of(R, s) + dst.row * (s / 2) + e / 2];
+                            const uint32_t nib = (e & 1) ? (byte >> 4) : (byte & 0xfu);
+                            c = (int)(nib ^ 8u) - 8;
+                        }
+                    }
+                    codes_out[o * s + e] = (int8_t)c;
+                }
+            }
+            if (scales_out && lane == 0)
+                scales_out[o] = ok ? *reinterpret_cast<const __half*>(blk + off_scales_of(R, s, BITS) + dst.row * 2)
+                                   : __float2half_rn(0.f);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Reset of one sequence: its pages go to the tiers' free rings, its counts go to zero.
+// Single block; stream-ordered with every other kernel, so no pop runs concurrently.
+// ------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) reset_kernel(const Geom G, const State S, int seq) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ uint32_t s_head, s_tail, s_warp[8], s_total;
+    const int pairs = G.G * G.Hkv;
+    for (int k = 0; k < G.ntiers; ++k) {
+        if (tid == 0) {
+            uint32_t hd = S.free_head[k], tl = S.free_tail[k];
+            if ((int)(hd - tl) > 0) hd = tl;        // pops overshot: the ring was empty
+            s_head = hd;
+            s_tail = tl;
+        }
+        __syncthreads();
+        for (int base = 0; base < pairs; base += blockDim.x) {
+            const int pr = base + tid;
+            uint32_t np = 0;
+            int g = 0, h = 0;
+            if (pr < pairs) {
+                g = pr / G.Hkv;
+                h = pr % G.Hkv;
+                np = (S.counts[cnt_index(G, seq, g, h) + k] + kPage - 1) / kPage;
+            }
+            uint32_t incl = np;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (lane == 31) s_warp[warp] = incl;
+            __syncthreads();
+            if (tid == 0) {
+                uint32_t acc = 0;
+                for (int w = 0; w < (int)(blockDim.x >> 5); ++w) { const uint32_t v = s_warp[w]; s_warp[w] = acc; acc += v; }
+                s_total = acc;
+            }
+            __syncthreads();
+            const uint32_t excl = s_warp[warp] + incl - np;
+            const bool room = (s_tail - s_head) + s_total <= G.free_cap;
+            if (pr < pairs && np) {
+                if (room) {
+                    const size_t pi = page_index(G, seq, g, h, k);
+                    for (uint32_t q = 0; q < np; ++q)
+                        S.free_list[(size_t)k * G.free_cap + ((s_tail + excl + q) & (G.free_cap - 1))] = S.pages[pi + q];
+                } else {
+                    set_dev_error(S, 7u /*DWKV_DEV_FREE_LIST*/, (uint32_t)seq, (uint32_t)k);
+                }
+            }
+            __syncthreads();
+            if (tid == 0 && room) s_tail += s_total;
+            __syncthreads();
+        }
+        if (tid == 0) {
+            S.free_head[k] = s_head;
+            S.free_tail[k] = s_tail;
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < pairs * kMaxTiers; e += blockDim.x)
+        S.counts[cnt_index(G, seq, 0, 0) + e] = 0u;
+}
+
+}  // namespace dwkv
+
+namespace dwkv {
+template __global__ void encode_kernel<8>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
+                                          const __nv_bfloat16*);
+template __global__ void encode_kernel<4>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
+                                          const __nv_bfloat16*);
+template __global__ void import_kernel<8>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
+                                          const uint8_t*, const int8_t*, const __half*);
+template __global__ void import_kernel<4>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
+                                          const uint8_t*, const int8_t*, const __half*);
+template __global__ void export_kernel<8>(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*,
+                                          uint8_t*, int8_t*, __half*);
+template __global__ void export_kernel<4>(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*,
+                                          uint8_t*, int8_t*, __half*);
+}  // namespace dwkv

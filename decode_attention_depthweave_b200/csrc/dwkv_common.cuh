@@ -1,0 +1,216 @@
+// dwkv_common.cuh -- geometry, device state and low-level helpers shared by the libdwkv
+// kernels and host code.  Product code; no test-only code includes it.
+//
+// Storage ("DepthWeave-KV: Token-Adaptive Cross-Layer Residual Factorization for
+// Long-Context KV Cache Compression", §3 Method, Eq. (1); tier-bucketed layout of this
+// library):
+//   * A page holds 64 tokens of ONE rank tier for one (sequence, group, kv-head).  Its
+//     bytes are [layer-in-group][K|V] blocks; decode of one layer reads one contiguous
+//     chunk (the K block then the V block) per page.
+//   * A block of tier rank R with s residual channels and b-bit codes is
+//       coeff  [R/8][64][8] bf16     128*R bytes  (8-coefficient columns, 16 B per token:
+//                                                  the tcgen05 / ldmatrix "core matrix"
+//                                                  order, conflict-free for per-token reads)
+//       idx    [64][s]    uint8      64*s
+//       codes  [64][s*b/8]           8*s*b        (int4: even slot in the low nibble)
+//       scales [64]       fp16       128
+//     Every part is a multiple of 128 bytes, so pages are 128-byte aligned and every page
+//     chunk is a legal bulk-copy (TMA) source.
+//   * The page pool is handed out in 128-byte units by a device bump pointer plus one
+//     free ring per tier (filled by sequence resets).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace dwkv {
+
+constexpr int kPage = 64;          // tokens per page
+constexpr int kD = 128;            // head dimension supported by the kernels
+constexpr int kGQ = 4;             // query heads per kv head supported by the kernels
+constexpr int kUnit = 128;         // page-pool granularity in bytes
+constexpr int kMaxTiers = 8;
+constexpr int kMaxSeqs = 256;      // sequences per call
+constexpr int kMaxSplits = 64;     // decode splits per (sequence, kv-head)
+constexpr int kDecodeThreads = 160;// 4 consumer warps + 1 producer warp
+constexpr int kConsumerWarps = 4;
+
+struct Geom {
+    int L, LPG, G, Hq, Hkv, d, r_max, ntiers, s, bits, max_batch, max_context, max_pages;
+    int tiers[kMaxTiers];
+    float tau;                       // softmax scale
+    uint32_t blk_bytes[kMaxTiers];   // one (layer, K or V) block of a page
+    uint32_t chunk_bytes[kMaxTiers]; // one layer of a page: K block + V block
+    uint32_t page_units[kMaxTiers];  // whole page, in kUnit
+    uint32_t free_cap;               // entries per free ring (power of two)
+    uint32_t stage_bytes;            // largest chunk, rounded to 128
+};
+
+struct State {
+    uint32_t* err;                   // [0] code, [1] info a, [2] info b
+    unsigned long long* bump;        // next free pool unit
+    uint32_t* free_head;             // [kMaxTiers] ring read index (monotonic)
+    uint32_t* free_tail;             // [kMaxTiers] ring write index (monotonic)
+    uint32_t* free_list;             // [kMaxTiers][free_cap] page units
+    uint32_t* counts;                // [max_batch][G][Hkv][kMaxTiers] slots placed
+    uint32_t* pages;                 // [max_batch][G][Hkv][kMaxTiers][max_pages] unit offsets
+    uint32_t* slot_map;              // [max_batch][G][Hkv][max_context]: ((tier+1)<<24)|slot
+    uint32_t* tickets;               // [max_batch][Hkv] split-combine tickets
+    const __nv_bfloat16* basis_k;    // [G][Hkv][d][r_max]
+    const __nv_bfloat16* basis_v;
+    uint8_t* data;                   // page pool
+    unsigned long long data_units;
+};
+
+// Per-call sequence table of append / import (passed by value as a kernel parameter, so
+// captured graphs replay it exactly).
+struct AppendCall {
+    int n, layer, g, lig, total;
+    int seq[kMaxSeqs];
+    int pos0[kMaxSeqs];      // first position appended at this layer
+    int tok0[kMaxSeqs + 1];  // prefix of n_new: first input row of each sequence
+    int a0[kMaxSeqs];        // first position that needs a slot (group's first placement)
+    int na[kMaxSeqs];        // positions that need a slot
+};
+
+struct DecodeCall {
+    int n, layer, g, lig, total_splits, stages, rec_floats;
+    int seq[kMaxSeqs];
+    int split_begin[kMaxSeqs + 1];
+    const __nv_bfloat16* q;  // [n][Hq][d]
+    float* out;              // [n][Hq][d]
+    float* out_full;         // probe: optional [n][Hq][d]
+    float* err;              // probe: [n][Hkv]
+    float* ws;               // partial records
+};
+
+// ------------------------------------------------------------------------------ layout
+__host__ __device__ inline uint32_t blk_bytes_of(int R, int s, int bits) {
+    return 128u * R + 64u * s + 8u * s * bits + 128u;
+}
+__host__ __device__ inline uint32_t off_idx_of(int R) { return 128u * R; }
+__host__ __device__ inline uint32_t off_codes_of(int R, int s) { return 128u * R + 64u * s; }
+__host__ __device__ inline uint32_t off_scales_of(int R, int s, int bits) {
+    return 128u * R + 64u * s + 8u * s * bits;
+}
+__host__ __device__ inline size_t cnt_index(const Geom& G, int seq, int g, int h) {
+    return (((size_t)seq * G.G + g) * G.Hkv + h) * kMaxTiers;
+}
+__host__ __device__ inline size_t page_index(const Geom& G, int seq, int g, int h, int k) {
+    return ((((size_t)seq * G.G + g) * G.Hkv + h) * kMaxTiers + k) * (size_t)G.max_pages;
+}
+__host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int h, int pos) {
+    return (((size_t)seq * G.G + g) * G.Hkv + h) * (size_t)G.max_context + pos;
+}
+
+// Decode shared-memory layout (identical on host and device).
+struct DecodeSmem {
+    uint32_t stages, basis, qt, q, warp, warp_stride, p, p2, accc, accc2, accr, bars, misc, total;
+};
+__host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, int NS, bool probe) {
+    DecodeSmem L;
+    uint32_t o = 0;
+    L.stages = o;  o += (uint32_t)NS * G.stage_bytes;
+    L.basis = o;   o += (uint32_t)G.d * G.r_max * 2;           o = (o + 127) & ~127u;
+    L.qt = o;      o += (uint32_t)G.r_max * 16;
+    L.q = o;       o += (uint32_t)G.d * 16;
+    L.warp = o;
+    uint32_t w = 0;
+    L.p = w;       w += kPage * 16;
+    L.p2 = w;      w += probe ? kPage * 16 : 0;
+    L.accc = w;    w += (uint32_t)G.r_max * 16;
+    L.accc2 = w;   w += probe ? (uint32_t)G.r_max * 16 : 0;
+    L.accr = w;    w += (uint32_t)kGQ * G.d * 4;
+    L.warp_stride = (w + 127) & ~127u;
+    o += kConsumerWarps * L.warp_stride;
+    L.bars = o;    o += (2 * NS + 2) * 8;
+    L.misc = o;    o += 512;
+    L.total = (o + 127) & ~127u;
+    return L;
+}
+
+// Floats in one decode partial record: m[4] l[4] (m2[4] l2[4]) acc_c[4][r_max]
+// (acc_c2[4][r_max]) acc_r[4][d].  The probe layout is used for both kernels' sizing.
+__host__ __device__ inline int rec_floats_of(const Geom& G, bool probe) {
+    return (probe ? 16 : 8) + (probe ? 8 : 4) * G.r_max + kGQ * G.d;
+}
+
+// ------------------------------------------------------------------------------ device
+#ifdef __CUDACC__
+__device__ __forceinline__ void set_dev_error(const State& S, uint32_t code, uint32_t a, uint32_t b) {
+    if (atomicCAS(S.err, 0u, code) == 0u) {
+        S.err[1] = a;
+        S.err[2] = b;
+    }
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase of parity `parity` to complete: gives up after 2 s of wall
+// time (checked every 256 polls); the caller then records DWKV_DEV_TIMEOUT and stops
+// instead of spinning forever.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0u && global_ns() - t0 > 2000000000ull) return false;
+    }
+}
+
+// One bulk (non-tensor) global -> shared copy completing on an mbarrier.  Both addresses
+// 16-byte aligned, bytes a multiple of 16.  No cluster multicast.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+#endif
+
+}  // namespace dwkv

@@ -1,0 +1,225 @@
+/*
+ * dwkv.h -- C ABI of libdwkv: decode attention read directly from a DepthWeave-KV
+ * compressed KV cache, on one NVIDIA B200 (sm_100a).
+ *
+ * Method: "DepthWeave-KV: Token-Adaptive Cross-Layer Residual Factorization for
+ * Long-Context KV Cache Compression" (arXiv 2607.06523), cited as [DW].
+ *
+ *  - [DW] §3 Method, Eq. (1): the key / value of token t at layer l of depth window m,
+ *    kv-head h, is rebuilt as  X^ = A B_{m,h} + g R.  This library stores
+ *      * per (group m, kv-head h) a basis B in bf16, d x r_max, column j = basis vector j
+ *        (one for keys, one for values; [DW] §3: "independently per head and separately
+ *        for keys and values");
+ *      * per (layer, kv-head, token) the first r_t coefficients of A in bf16, r_t being the
+ *        token's rank tier (the router's output, [DW] §3 Eq. (2));
+ *      * per (layer, kv-head, token) a sparse residual R of s channels: channel indices
+ *        (uint8), symmetric integer codes (int8, or int4 two's complement with the even
+ *        slot in the low nibble) and one fp16 scale.  The gate g is 1.
+ *  - [DW] §3, data path paragraph: decode fuses basis lookup, residual dequantisation,
+ *    coefficient multiply and the attention score, and never writes the reconstructed
+ *    keys / values to memory.  dwkv_decode_attention does that: it projects the query
+ *    into basis space once, scores every token from its coefficients plus its residual,
+ *    runs an online softmax, accumulates values in coefficient space and residual space,
+ *    and applies the value basis once at the end.
+ *  - [DW] §3 Eq. (3): the attention-output probe.  dwkv_probe returns, per (sequence,
+ *    kv-head), ||o_full - o_nores||_2 / (||o_full||_2 + 1e-6) where o_full uses the
+ *    residual and o_nores does not; the norm runs over the kv-head's query heads x d.
+ *  - [DW] §3, coefficient paragraph: new keys / values are projected onto the current
+ *    basis.  dwkv_append encodes them (projection, residual against the stored bf16
+ *    coefficients, s largest |residual| channels with ties to the lower channel,
+ *    fp16 scale = amax / qmax, codes = clamp(rint(r / scale))).
+ *
+ * Conventions for every call:
+ *  - Ownership: the caller allocates and owns every buffer (arena, workspace, inputs,
+ *    outputs).  The library never allocates or frees device memory.
+ *  - Pointers named "device" must be device memory of the handle's GPU; pointers named
+ *    "host" are host memory.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *  - All work is stream-ordered and asynchronous.  Arguments are validated on the host
+ *    before anything is launched; on any error nothing is launched and the call returns
+ *    a non-zero status.  dwkv_last_error() gives a message for the calling thread.
+ *  - Checks that need device data (tier indices, residual channels, pool capacity) run
+ *    inside the kernels; a failed check sets a device error word instead of faulting and
+ *    the affected tokens are skipped.  dwkv_sync_status() reports it.
+ *  - A handle is not thread-safe; issue its calls from one thread, on one stream.
+ *  - All kernels read the cache state from device memory, so a sequence of calls may be
+ *    captured in a CUDA graph and replayed; the host's own per-sequence length mirror
+ *    (used only for argument checks) then advances only at capture time.
+ */
+#ifndef DWKV_H
+#define DWKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DWKV_MAX_TIERS 8
+#define DWKV_MAX_SEQS_PER_CALL 256
+#define DWKV_PAGE_TOKENS 64
+
+typedef struct dwkv_ctx* dwkv_handle;
+
+typedef enum {
+    DWKV_OK = 0,
+    DWKV_ERR_INVALID_ARG = 1,   /* bad pointer, size, index or call order               */
+    DWKV_ERR_CAPACITY = 2,      /* context, arena or workspace too small                */
+    DWKV_ERR_CUDA = 3,          /* a CUDA runtime call failed (message has the reason)  */
+    DWKV_ERR_DEVICE_CHECK = 4,  /* a kernel-side check failed (see dwkv_sync_status)    */
+    DWKV_ERR_UNSUPPORTED = 5    /* valid configuration this build has no kernel for     */
+} dwkv_status;
+
+/* Device error codes recorded by kernels (first error wins). */
+#define DWKV_DEV_POOL_EXHAUSTED 1   /* no page left in the arena                         */
+#define DWKV_DEV_BAD_TIER 2         /* tier index >= num_tiers                           */
+#define DWKV_DEV_BAD_CHANNEL 3      /* residual channel index >= head_dim                */
+#define DWKV_DEV_BAD_CODE 4         /* code outside the int4 range [-8, 7]                */
+#define DWKV_DEV_NO_SLOT 5          /* a layer appended a position its group never placed */
+#define DWKV_DEV_TIMEOUT 6          /* a bounded wait in a kernel ran out                 */
+#define DWKV_DEV_FREE_LIST 7        /* free-page ring overflow on reset                   */
+
+/* Cache geometry.  Supported by this build: head_dim == 128; num_q_heads == 4 *
+ * num_kv_heads; tiers drawn from {8, 16, 32, 64, 128}, strictly ascending, each <= r_max;
+ * r_max in {8, 16, 32, 64, 128}; resid_channels s a multiple of 8 with 0 <= s <= 128;
+ * resid_bits 8 or 4; num_layers a multiple of layers_per_group. */
+typedef struct {
+    int32_t num_layers;        /* L                                                     */
+    int32_t layers_per_group;  /* w: adjacent layers sharing one basis ([DW] §3)        */
+    int32_t num_q_heads;       /* Hq                                                    */
+    int32_t num_kv_heads;      /* Hkv                                                   */
+    int32_t head_dim;          /* d                                                     */
+    int32_t r_max;             /* basis columns per (group, kv-head, K/V)               */
+    int32_t num_tiers;         /* 1..DWKV_MAX_TIERS                                     */
+    int32_t tiers[DWKV_MAX_TIERS]; /* coefficient rank of each tier                     */
+    int32_t resid_channels;    /* s                                                     */
+    int32_t resid_bits;        /* 8 (codes in [-127,127]) or 4 (codes in [-7,7])        */
+    int32_t max_batch;         /* sequence slots: ids 0 .. max_batch-1                  */
+    int32_t max_context;       /* tokens per sequence                                   */
+    float softmax_scale;       /* <= 0 selects 1/sqrt(head_dim)                         */
+} dwkv_config;
+
+/* Library version string. */
+const char* dwkv_version(void);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* dwkv_last_error(void);
+
+/* Validates a configuration without touching the GPU. */
+dwkv_status dwkv_config_check(const dwkv_config* cfg);
+
+/* Bytes of one stored token (one layer, one kv-head, keys + values) at tier index
+ * `tier`: 2 * (2*r + s + s*bits/8 + 2).  0 if the arguments are invalid. */
+size_t dwkv_token_bytes(const dwkv_config* cfg, int32_t tier);
+
+/* Bytes of one page of tier `tier`: DWKV_PAGE_TOKENS tokens of one (sequence, group,
+ * kv-head), all layers of the group, keys and values.  0 if invalid. */
+size_t dwkv_page_bytes(const dwkv_config* cfg, int32_t tier);
+
+/* Bytes of the arena's fixed part (bases, page tables, slot maps, counters). */
+size_t dwkv_metadata_bytes(const dwkv_config* cfg);
+
+/* Arena bytes that can hold max_batch sequences of max_context tokens in every layer
+ * even if every token takes the largest tier.  0 if cfg is invalid.  A smaller arena
+ * (at least dwkv_metadata_bytes + one largest page) is accepted: the page pool is then
+ * smaller and running out of it is a device-side DWKV_DEV_POOL_EXHAUSTED error. */
+size_t dwkv_arena_bytes(const dwkv_config* cfg);
+
+/* Workspace bytes that decode / probe need for a call over n_seqs sequences. */
+size_t dwkv_workspace_bytes(const dwkv_config* cfg, int32_t n_seqs);
+
+/* Creates a cache inside `arena` (device, caller-owned, 256-byte aligned, at least
+ * dwkv_metadata_bytes(cfg) + one page) on the current CUDA device.  basis_k / basis_v:
+ * device bf16 [G][Hkv][head_dim][r_max] (G = num_layers / layers_per_group), copied into
+ * the arena; they need not outlive the call.  The arena's metadata is cleared on
+ * `stream`.  Writes the handle to *out. */
+dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
+                        const void* basis_k, const void* basis_v, void* stream,
+                        dwkv_handle* out);
+
+/* Releases the host-side handle (no device memory is freed; the arena stays the
+ * caller's).  Waits for nothing: finish or synchronise the handle's stream first. */
+dwkv_status dwkv_destroy(dwkv_handle h);
+
+/* Empties sequence `seq` in every layer and returns its pages to the free pool. */
+dwkv_status dwkv_reset_sequence(dwkv_handle h, int32_t seq, void* stream);
+
+/* Host-side length of `seq` at `layer` (tokens appended so far through this handle). */
+dwkv_status dwkv_seq_length(dwkv_handle h, int32_t seq, int32_t layer, int32_t* len);
+
+/* Encodes and appends n_new[i] tokens to each listed sequence at `layer`.
+ *   seq_ids, n_new : host int32 [n_seqs]; distinct ids; n_new[i] >= 0
+ *   k_new, v_new   : device bf16 [sum(n_new)][Hkv][head_dim], sequences in list order
+ *   tier_idx       : device uint8 [sum(n_new)][Hkv], index into cfg.tiers.  A token's
+ *                    tier is fixed by the first layer of its group that appends it
+ *                    ([DW] §3 Eq. (2): rho_{m,h,t} has no layer index); later layers of
+ *                    the group reuse it and ignore this array (which may then be NULL).
+ * The positions appended are [len, len + n_new[i]) where len is the sequence's current
+ * length at this layer.  Capacity: len + n_new[i] <= max_context. */
+dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                        const int32_t* n_new, const void* k_new, const void* v_new,
+                        const uint8_t* tier_idx, void* stream);
+
+/* Appends tokens that are already in compressed form (import of a prepared cache).
+ * Same sequence / position rules as dwkv_append.  Device arrays, tokens in list order,
+ * K at [..][0][..] and V at [..][1][..]:
+ *   coeff  bf16  [sum(n_new)][Hkv][2][r_max]   (entries at j >= r_t are ignored)
+ *   idx    uint8 [sum(n_new)][Hkv][2][s]       (each < head_dim)
+ *   codes  int8  [sum(n_new)][Hkv][2][s]       (int4 caches: each in [-8, 7])
+ *   scales fp16  [sum(n_new)][Hkv][2] */
+dwkv_status dwkv_append_compressed(dwkv_handle h, int32_t layer, int32_t n_seqs,
+                                   const int32_t* seq_ids, const int32_t* n_new,
+                                   const uint8_t* tier_idx, const void* coeff,
+                                   const uint8_t* idx, const int8_t* codes, const void* scales,
+                                   void* stream);
+
+/* Decode attention at `layer` for one query token per listed sequence, over every token
+ * the sequence holds at that layer ([DW] §3 Eq. (1) inside softmax attention).
+ *   seq_ids   : host int32 [n_seqs], distinct
+ *   q         : device bf16 [n_seqs][Hq][head_dim]
+ *   out       : device fp32 [n_seqs][Hq][head_dim]; an empty sequence gives zeros
+ *   workspace : device, >= dwkv_workspace_bytes(cfg, n_seqs) bytes, 16-byte aligned
+ * Every layer of a group must hold the same positions when one of them is decoded
+ * (append each layer of the group before decoding it). */
+dwkv_status dwkv_decode_attention(dwkv_handle h, int32_t layer, int32_t n_seqs,
+                                  const int32_t* seq_ids, const void* q, float* out,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* Probe ([DW] §3 Eq. (3), two caches read as with / without the residual) in one pass
+ * over the cache.  err: device fp32 [n_seqs][Hkv].  out_full: NULL or device fp32
+ * [n_seqs][Hq][head_dim] (the decode output).  Other arguments as decode. */
+dwkv_status dwkv_probe(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                       const void* q, float* err, float* out_full, void* workspace,
+                       size_t ws_bytes, void* stream);
+
+/* Reads positions [t0, t0 + n) of (layer, seq) back in token order, as stored:
+ *   tier_idx uint8 [n][Hkv]; coeff bf16 [n][Hkv][2][r_max] (zeros at j >= r_t);
+ *   idx uint8 [n][Hkv][2][s]; codes int8 [n][Hkv][2][s]; scales fp16 [n][Hkv][2].
+ * All device pointers; any of them may be NULL to skip that array. */
+dwkv_status dwkv_export(dwkv_handle h, int32_t layer, int32_t seq, int32_t t0, int32_t n,
+                        uint8_t* tier_idx, void* coeff, uint8_t* idx, int8_t* codes,
+                        void* scales, void* stream);
+
+/* Pool usage, read synchronously (the stream is synchronised first). */
+typedef struct {
+    uint64_t data_bytes_total;     /* page pool size                                    */
+    uint64_t data_bytes_reserved;  /* bytes ever handed out from the pool               */
+    uint32_t free_pages[DWKV_MAX_TIERS]; /* pages waiting in each tier's free ring     */
+} dwkv_pool_stats;
+dwkv_status dwkv_pool_usage(dwkv_handle h, void* stream, dwkv_pool_stats* out);
+
+/* Synchronises `stream`, then returns DWKV_ERR_DEVICE_CHECK if a kernel recorded an
+ * error since the last call (the message names it; the word is then cleared), or
+ * DWKV_ERR_CUDA if the stream reported a CUDA error. */
+dwkv_status dwkv_sync_status(dwkv_handle h, void* stream);
+
+/* Launch tuning (for measurement sweeps): decode CTAs per SM (1 or 2), split waves per
+ * decode (>= 1) and pipeline stages per CTA (0 = largest that fits).  Returns
+ * DWKV_ERR_INVALID_ARG for values out of range. */
+dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t waves,
+                                   int32_t stages);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DWKV_H */

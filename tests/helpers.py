@@ -82,3 +82,70 @@ def rel_l2(a, b) -> float:
 
 def tau_of(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+# ----------------------------------------------------------------------------- GPU cache
+def cfg_for(wl, max_batch=None, max_context=None, softmax_scale=0.0):
+    import decode_attention_depthweave_b200 as dw
+    return dw.config_from(
+        num_layers=wl.num_layers, layers_per_group=wl.layers_per_group, num_q_heads=wl.num_q_heads,
+        num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, r_max=wl.r_max, tiers=wl.tiers,
+        resid_channels=wl.resid_channels, resid_bits=wl.resid_bits,
+        max_batch=max_batch or wl.batch, max_context=max_context or wl.context, softmax_scale=softmax_scale)
+
+
+def to_dev(d: dict, device="cuda") -> dict:
+    return {k: v.to(device).contiguous() for k, v in d.items()}
+
+
+def import_workload(cache, wl, lengths, gen_device="cpu", garbage=False, seed=None, layers=None):
+    """Import synthetic compressed tokens of every (sequence, layer) into ``cache``.
+    Returns {(seq, layer): (tier_idx, comp)} on the generation device."""
+    data = {}
+    layers = range(wl.num_layers) if layers is None else layers
+    for seq, T in enumerate(lengths):
+        tiers_by_group = {}
+        for layer in layers:
+            g = layer // wl.layers_per_group
+            if g not in tiers_by_group:
+                tiers_by_group[g] = synth.make_tiers(wl, seq, g, T, device=gen_device, seed=seed)
+            tiers = tiers_by_group[g]
+            comp = synth.make_compressed(wl, seq, layer, tiers, device=gen_device, seed=seed, garbage_tail=garbage)
+            c = to_dev(comp)
+            cache.append_compressed(layer, [seq], [T], tiers.to("cuda").contiguous(), c["coeff"], c["idx"],
+                                    c["codes"], c["scales"])
+            data[(seq, layer)] = (tiers, comp)
+    return data
+
+
+def check_close(got, ref, max_abs=2e-3, rel=1e-3, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    ma = float(np.max(np.abs(got - ref))) if got.size else 0.0
+    rl = rel_l2(got, ref) if np.linalg.norm(ref) > 0 else float(np.linalg.norm(got))
+    assert ma <= max_abs and rl <= rel, f"{what}: max_abs {ma:.3e} rel_l2 {rl:.3e}"
+    return ma, rl
+
+
+def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None) -> dict:
+    """The oracle's encoding of dense rows k, v (bf16 [n][Hkv][d]) at their tiers, in the
+    token-ordered compressed format of ``synth.make_compressed`` (CPU tensors)."""
+    g = layer // wl.layers_per_group
+    k, v, tier_idx = k.cpu(), v.cpu(), tier_idx.cpu()
+    n, H, s = k.shape[0], wl.num_kv_heads, wl.resid_channels
+    ranks = synth.ranks_of(wl, tier_idx)
+    coeff = np.zeros((n, H, 2, wl.r_max), np.uint16)
+    idx = np.zeros((n, H, 2, s), np.uint8)
+    codes = np.zeros((n, H, 2, s), np.int8)
+    scales = np.zeros((n, H, 2), np.uint16)
+    for h in range(H):
+        for z, x in enumerate((k, v)):
+            r = oracle.encode_many(bases[z][g, h], x[:, h], ranks[:, h], s, wl.resid_bits, nthreads=nthreads)
+            coeff[:, h, z], idx[:, h, z], codes[:, h, z], scales[:, h, z] = r["coeff"], r["idx"], r["codes"], r["scale"]
+    return {"coeff": torch.from_numpy(coeff.view(np.int16)).view(torch.bfloat16),
+            "idx": torch.from_numpy(idx), "codes": torch.from_numpy(codes),
+            "scales": torch.from_numpy(scales.view(np.int16)).view(torch.float16)}
+
+
+def cat_comp(a: dict, b: dict) -> dict:
+    return {key: torch.cat([a[key].cpu(), b[key].cpu()]) for key in a}

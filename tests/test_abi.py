@@ -1,0 +1,99 @@
+"""The C-ABI library loads, exports every symbol its header declares, and validates
+arguments on the host before touching a GPU (these tests run without one)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+import torch
+
+import decode_attention_depthweave_b200 as dw
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "dwkv.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dwkv_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declarations_are_exported():
+    L = C.CDLL(dw.LIB_PATH)
+    names = _declared()
+    assert "dwkv_decode_attention" in names and "dwkv_probe" in names and "dwkv_create" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(dw.EXPORTED_SYMBOLS) == names
+
+
+def _cfg(wl, **over):
+    kw = dict(num_layers=wl.num_layers, layers_per_group=wl.layers_per_group, num_q_heads=wl.num_q_heads,
+              num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, r_max=wl.r_max, tiers=wl.tiers,
+              resid_channels=wl.resid_channels, resid_bits=wl.resid_bits, max_batch=wl.batch,
+              max_context=wl.context + 64)
+    kw.update(over)
+    return dw.config_from(**kw)
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_workload_configs_are_supported(name):
+    assert dw.dwkv_config_check(_cfg(synth.workload(name))) == 0, dw.dwkv_last_error()
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(num_layers=3), 1), (dict(head_dim=64), 5), (dict(num_q_heads=16), 5), (dict(r_max=12), 1),
+    (dict(r_max=48, tiers=(16, 32)), 5), (dict(tiers=(16, 16)), 1), (dict(tiers=(8, 24)), 5), (dict(tiers=(16, 128)), 1),
+    (dict(resid_channels=12), 1), (dict(resid_bits=2), 1), (dict(max_batch=0), 1),
+    (dict(max_context=1 << 24), 1),
+])
+def test_invalid_configs_are_rejected(over, status):
+    cfg = _cfg(synth.workload("llama8b_64k"), **over)
+    assert dw.dwkv_config_check(cfg) == status
+    assert dw.dwkv_last_error()
+
+
+def test_token_and_page_bytes():
+    cfg = _cfg(synth.workload("llama8b_64k"))
+    # one token, one layer, one kv-head, K + V: 2 * (2 r + s + s*bits/8 + 2)
+    assert [dw.dwkv_token_bytes(cfg, k) for k in range(3)] == [2 * (2 * r + 16 + 8 + 2) for r in (16, 32, 64)]
+    assert dw.dwkv_token_bytes(cfg, 3) == 0
+    for k, r in enumerate((16, 32, 64)):
+        assert dw.dwkv_page_bytes(cfg, k) == 2 * 2 * (128 * r + 64 * 16 + 8 * 16 * 4 + 128)
+        assert dw.dwkv_page_bytes(cfg, k) % 128 == 0
+    meta = dw.dwkv_metadata_bytes(cfg)
+    assert 0 < meta < dw.dwkv_arena_bytes(cfg)
+    assert dw.dwkv_workspace_bytes(cfg, 8) == 8 * dw.dwkv_workspace_bytes(cfg, 1)
+
+
+def test_create_rejects_bad_arguments_without_a_gpu():
+    cfg = _cfg(synth.workload("tiny_1k"))
+    h = C.c_void_p()
+    L = dw.lib()
+    assert L.dwkv_create(C.byref(cfg), None, 0, None, None, None, C.byref(h)) == 1
+    assert "non-NULL" in dw.dwkv_last_error()
+    bad = _cfg(synth.workload("tiny_1k"), resid_bits=3)
+    assert L.dwkv_create(C.byref(bad), C.c_void_p(256), 1 << 20, C.c_void_p(256), C.c_void_p(256), None,
+                         C.byref(h)) == 1
+    assert L.dwkv_create(C.byref(cfg), C.c_void_p(257), 1 << 20, C.c_void_p(256), C.c_void_p(256), None,
+                         C.byref(h)) == 1
+    assert "aligned" in dw.dwkv_last_error()
+    assert h.value is None
+
+
+def test_null_handle_calls_fail_cleanly():
+    L = dw.lib()
+    assert L.dwkv_destroy(None) == 1
+    assert L.dwkv_sync_status(None, None) == 1
+    assert L.dwkv_decode_attention(None, 0, 0, None, None, None, None, 0, None) == 1
+    assert L.dwkv_append(None, 0, 0, None, None, None, None, None, None) == 1
+
+
+def test_product_package_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "decode_attention_depthweave_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower(), f
