@@ -239,10 +239,9 @@ size_t encode_smem(const Geom& G) {
     return (size_t)2 * kD * (G.r_max + 2) * 2 + (size_t)8 * (2 * kD + 2 * G.r_max + 64) * 4;
 }
 
-int decode_stages(dwkv_handle h, bool probe, size_t* smem_out) {
+int decode_stages_for(dwkv_handle h, bool probe, int ctas_per_sm, size_t* smem_out) {
     const Geom& G = h->geom;
-    const size_t budget = h->dec_ctas_per_sm == 1 ? h->smem_optin
-                                                  : std::min(h->smem_optin, h->smem_per_sm / 2 - 1024);
+    const size_t budget = ctas_per_sm == 1 ? h->smem_optin : std::min(h->smem_optin, h->smem_per_sm / 2 - 1024);
     int best = 0;
     const int cap = h->dec_stages_req > 0 ? h->dec_stages_req : 16;
     for (int ns = kConsumerWarps; ns <= cap; ns += kConsumerWarps) {
@@ -250,6 +249,19 @@ int decode_stages(dwkv_handle h, bool probe, size_t* smem_out) {
         if (L.total <= budget) { best = ns; *smem_out = L.total; }
     }
     return best;
+}
+
+// Stages for the configured CTAs per SM; the probe (larger per-warp state) falls back to one
+// CTA per SM when two do not fit.  *ctas_out receives the CTAs per SM actually used.
+int decode_stages(dwkv_handle h, bool probe, size_t* smem_out, int* ctas_out = nullptr) {
+    int c = h->dec_ctas_per_sm;
+    int ns = decode_stages_for(h, probe, c, smem_out);
+    if (ns < kConsumerWarps && c > 1) {
+        c = 1;
+        ns = decode_stages_for(h, probe, c, smem_out);
+    }
+    if (ctas_out) *ctas_out = c;
+    return ns;
 }
 
 dwkv_status prepare_call(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
@@ -439,7 +451,7 @@ dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t w
     h->dec_waves = waves;
     h->dec_stages_req = stages;
     size_t sm = 0;
-    if (decode_stages(h, true, &sm) < kConsumerWarps) {
+    if (decode_stages_for(h, false, ctas_per_sm, &sm) < kConsumerWarps) {
         h->dec_ctas_per_sm = oc; h->dec_waves = ow; h->dec_stages_req = os;
         return fail(DWKV_ERR_INVALID_ARG, "tuning leaves no room for a 4-stage pipeline");
     }
@@ -563,7 +575,11 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     C.layer = layer;
     C.g = g;
     C.lig = layer % G.LPG;
-    const long long target = (long long)h->num_sms * h->dec_ctas_per_sm * h->dec_waves;
+    size_t smem = 0;
+    int ctas = 1;
+    const int stages = decode_stages(h, probe, &smem, &ctas);
+    if (stages < kConsumerWarps) return fail(DWKV_ERR_UNSUPPORTED, "decode pipeline does not fit in shared memory");
+    const long long target = (long long)h->num_sms * ctas * h->dec_waves;
     int total = 0;
     for (int i = 0; i < n_seqs; ++i) {
         const int s = seq_ids[i];
@@ -577,8 +593,7 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     }
     C.split_begin[n_seqs] = total;
     C.total_splits = total;
-    size_t smem = 0;
-    C.stages = decode_stages(h, probe, &smem);
+    C.stages = stages;
     C.rec_floats = rec_floats_of(G, probe);
     C.q = static_cast<const __nv_bfloat16*>(q);
     C.out = out;
