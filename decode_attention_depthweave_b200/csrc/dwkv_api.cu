@@ -22,7 +22,7 @@ template <int BITS>
 __global__ void export_kernel(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*, uint8_t*,
                               int8_t*, __half*);
 __global__ void reset_kernel(const Geom, const State, int);
-template <int BITS, bool PROBE>
+template <int BITS, bool PROBE, int RMAX>
 __global__ void decode_kernel(const Geom, const State, const DecodeCall);
 }  // namespace dwkv
 
@@ -244,7 +244,7 @@ int decode_stages_for(dwkv_handle h, bool probe, int ctas_per_sm, size_t* smem_o
     const size_t budget = ctas_per_sm == 1 ? h->smem_optin : std::min(h->smem_optin, h->smem_per_sm / 2 - 1024);
     int best = 0;
     const int cap = h->dec_stages_req > 0 ? h->dec_stages_req : 16;
-    for (int ns = kConsumerWarps; ns <= cap; ns += kConsumerWarps) {
+    for (int ns = kPairs; ns <= cap; ns += kPairs) {
         const DecodeSmem L = decode_smem_layout(G, ns, probe);
         if (L.total <= budget) { best = ns; *smem_out = L.total; }
     }
@@ -256,7 +256,7 @@ int decode_stages_for(dwkv_handle h, bool probe, int ctas_per_sm, size_t* smem_o
 int decode_stages(dwkv_handle h, bool probe, size_t* smem_out, int* ctas_out = nullptr) {
     int c = h->dec_ctas_per_sm;
     int ns = decode_stages_for(h, probe, c, smem_out);
-    if (ns < kConsumerWarps && c > 1) {
+    if (ns < kPairs && c > 1) {
         c = 1;
         ns = decode_stages_for(h, probe, c, smem_out);
     }
@@ -414,19 +414,23 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e == cudaSuccess) {
         const int maxs = (int)h->smem_optin;
-        e = cudaFuncSetAttribute(decode_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel<8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
+        const void* kernels[] = {
+            (const void*)decode_kernel<8, false, 32>, (const void*)decode_kernel<8, false, 64>,
+            (const void*)decode_kernel<8, false, 128>, (const void*)decode_kernel<4, false, 32>,
+            (const void*)decode_kernel<4, false, 64>, (const void*)decode_kernel<4, false, 128>,
+            (const void*)decode_kernel<8, true, 32>, (const void*)decode_kernel<8, true, 64>,
+            (const void*)decode_kernel<8, true, 128>, (const void*)decode_kernel<4, true, 32>,
+            (const void*)decode_kernel<4, true, 64>, (const void*)decode_kernel<4, true, 128>,
+            (const void*)encode_kernel<8>, (const void*)encode_kernel<4>};
+        for (const void* k : kernels)
+            if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
     }
     if (e != cudaSuccess) {
         delete h;
         return cuda_fail(e, "dwkv_create");
     }
     size_t sm = 0;
-    if (decode_stages(h, true, &sm) < kConsumerWarps) {
+    if (decode_stages(h, true, &sm) < kPairs) {
         delete h;
         return fail(DWKV_ERR_UNSUPPORTED, "decode pipeline does not fit in shared memory for this geometry");
     }
@@ -443,15 +447,15 @@ dwkv_status dwkv_destroy(dwkv_handle h) {
 dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t waves, int32_t stages) {
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
-    if (ctas_per_sm < 1 || ctas_per_sm > 2 || waves < 1 || waves > 8 || stages < 0 || stages > 32 ||
-        stages % kConsumerWarps)
-        return fail(DWKV_ERR_INVALID_ARG, "tuning out of range (ctas 1-2, waves 1-8, stages 0 or multiple of 4 <= 32)");
+    if (ctas_per_sm != 1 || waves < 1 || waves > 8 || stages < 0 || stages > 32 ||
+        stages % kPairs)
+        return fail(DWKV_ERR_INVALID_ARG, "tuning out of range (ctas_per_sm 1, waves 1-8, stages 0 or a multiple of 4 up to 32)");
     const int oc = h->dec_ctas_per_sm, ow = h->dec_waves, os = h->dec_stages_req;
     h->dec_ctas_per_sm = ctas_per_sm;
     h->dec_waves = waves;
     h->dec_stages_req = stages;
     size_t sm = 0;
-    if (decode_stages_for(h, false, ctas_per_sm, &sm) < kConsumerWarps) {
+    if (decode_stages_for(h, false, ctas_per_sm, &sm) < kPairs) {
         h->dec_ctas_per_sm = oc; h->dec_waves = ow; h->dec_stages_req = os;
         return fail(DWKV_ERR_INVALID_ARG, "tuning leaves no room for a 4-stage pipeline");
     }
@@ -578,7 +582,7 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     size_t smem = 0;
     int ctas = 1;
     const int stages = decode_stages(h, probe, &smem, &ctas);
-    if (stages < kConsumerWarps) return fail(DWKV_ERR_UNSUPPORTED, "decode pipeline does not fit in shared memory");
+    if (stages < kPairs) return fail(DWKV_ERR_UNSUPPORTED, "decode pipeline does not fit in shared memory");
     const long long target = (long long)h->num_sms * ctas * h->dec_waves;
     int total = 0;
     for (int i = 0; i < n_seqs; ++i) {
@@ -602,13 +606,19 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     C.ws = static_cast<float*>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(total, G.Hkv);
+    const int rm = G.r_max <= 32 ? 32 : (G.r_max <= 64 ? 64 : 128);
+#define DWKV_LAUNCH(B, P, R) decode_kernel<B, P, R><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C)
+#define DWKV_LAUNCH_R(B, P) \
+    do { if (rm == 32) DWKV_LAUNCH(B, P, 32); else if (rm == 64) DWKV_LAUNCH(B, P, 64); else DWKV_LAUNCH(B, P, 128); } while (0)
     if (!probe) {
-        if (G.bits == 8) decode_kernel<8, false><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C);
-        else decode_kernel<4, false><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C);
+        if (G.bits == 8) DWKV_LAUNCH_R(8, false);
+        else DWKV_LAUNCH_R(4, false);
     } else {
-        if (G.bits == 8) decode_kernel<8, true><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C);
-        else decode_kernel<4, true><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C);
+        if (G.bits == 8) DWKV_LAUNCH_R(8, true);
+        else DWKV_LAUNCH_R(4, true);
     }
+#undef DWKV_LAUNCH_R
+#undef DWKV_LAUNCH
     DWKV_CUDA(cudaGetLastError(), probe ? "probe kernel launch" : "decode kernel launch");
     return DWKV_OK;
 }

@@ -33,8 +33,10 @@ constexpr int kUnit = 128;         // page-pool granularity in bytes
 constexpr int kMaxTiers = 8;
 constexpr int kMaxSeqs = 256;      // sequences per call
 constexpr int kMaxSplits = 64;     // decode splits per (sequence, kv-head)
-constexpr int kDecodeThreads = 160;// 4 consumer warps + 1 producer warp
-constexpr int kConsumerWarps = 4;
+constexpr int kConsumerWarps = 8;  // 4 pairs; a pair shares one page (32 tokens per warp)
+constexpr int kPairs = kConsumerWarps / 2;
+constexpr int kDecodeThreads = 32 * (kConsumerWarps + 1);  // + 1 producer warp
+constexpr int kRdBytes = 128 * 16 * 2;                     // dense residual tile: 128 ch x 16 tokens bf16
 
 struct Geom {
     int L, LPG, G, Hq, Hkv, d, r_max, ntiers, s, bits, max_batch, max_context, max_pages;
@@ -105,27 +107,30 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 }
 
 // Decode shared-memory layout (identical on host and device).
+//   stages  NS page chunks (NS a multiple of kPairs: stage <-> pair is fixed)
+//   rd      per consumer warp, one dense residual tile (also holds B_K during the prologue)
+//   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W[32][8] bf16, P2[32][8]
+//   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  zero line
 struct DecodeSmem {
-    uint32_t stages, basis, qt, q, warp, warp_stride, p, p2, accc, accc2, accr, bars, misc, total;
+    uint32_t stages, rd, small, small_stride, S, P, W, P2, qt, q, zero, bars, misc, total;
 };
 __host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, int NS, bool probe) {
     DecodeSmem L;
     uint32_t o = 0;
     L.stages = o;  o += (uint32_t)NS * G.stage_bytes;
-    L.basis = o;   o += (uint32_t)G.d * G.r_max * 2;           o = (o + 127) & ~127u;
-    L.qt = o;      o += (uint32_t)G.r_max * 16;
-    L.q = o;       o += (uint32_t)G.d * 16;
-    L.warp = o;
+    L.rd = o;      o += kConsumerWarps * kRdBytes;
     uint32_t w = 0;
-    L.p = w;       w += kPage * 16;
-    L.p2 = w;      w += probe ? kPage * 16 : 0;
-    L.accc = w;    w += (uint32_t)G.r_max * 16;
-    L.accc2 = w;   w += probe ? (uint32_t)G.r_max * 16 : 0;
-    L.accr = w;    w += (uint32_t)kGQ * G.d * 4;
-    L.warp_stride = (w + 127) & ~127u;
-    o += kConsumerWarps * L.warp_stride;
+    L.S = w;       w += 32 * 16;
+    L.P = w;       w += 32 * 16;
+    L.W = w;       w += 32 * 16;
+    L.P2 = w;      w += probe ? 32 * 16 : 0;
+    L.small_stride = w;
+    L.small = o;   o += kConsumerWarps * w;
+    L.qt = o;      o += (uint32_t)(G.r_max < 16 ? 16 : G.r_max) * 16;
+    L.q = o;       o += (uint32_t)G.d * 16;
+    L.zero = o;    o += 128;
     L.bars = o;    o += (2 * NS + 2) * 8;
-    L.misc = o;    o += 512;
+    L.misc = o;    o += 1024;
     L.total = (o + 127) & ~127u;
     return L;
 }

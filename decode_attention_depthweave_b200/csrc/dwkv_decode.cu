@@ -5,19 +5,27 @@
 // never writing reconstructed keys / values (Eq. (1) evaluated inside attention); the
 // probe is Eq. (3) with the with-residual output as the reference.
 //
-// For one query head q of kv-head h (tau folded with log2 e so exp2 can be used):
-//   qt = B_K^T q                                 (once per CTA, from B_K in shared memory)
-//   s_t = qt[:r_t] . c^K_t + scale^K_t * sum_i q[idx^K_ti] code^K_ti
-//   online softmax over t;  acc_c += p_t c^V_t (coefficient space);
-//   acc_r[idx^V_ti] += p_t scale^V_t code^V_ti (residual space)
-//   o = (B_V acc_c + acc_r) / l                 (B_V applied once, in the combine)
+// For the 4 query heads q_h of kv-head h (tau * log2 e folded into q so exp2 can be used):
+//   qt = B_K^T q                                   (once per CTA, B_K bulk-copied to smem)
+//   s_t = qt[:r_t] . c^K_t + scale^K_t sum_i q[idx^K_ti] code^K_ti
+//   online softmax over t;  acc_c += C^V^T p (coefficient space);
+//   acc_r += R^V^T (p * scale^V) (residual space, R^V the dense residual codes)
+//   o = (B_V acc_c + acc_r) / l                   (B_V applied once, in the combine)
+//
+// Tensor cores take the dense, tier-homogeneous coefficient blocks: the page's 64 x r_t
+// coefficient tile against q~ (scores) and against p (values), and the value residual
+// after it is expanded into a dense 128-channel x 16-token tile in shared memory.  The
+// operands that are not exact in bf16 (q~, p, p * scale) are split into bf16 hi + lo
+// halves (two MMA columns each), so products keep ~16 significant bits and accumulate in
+// fp32.  The key residual is a gather-dot on the CUDA cores.
 //
 // Work split: a CTA takes a byte-balanced run of one (sequence, kv-head)'s pages (pages are
-// tier-homogeneous; tiers are visited in order).  Warp 4 lane 0 streams page chunks into
-// a ring of shared-memory stages with cp.async.bulk (no multicast); warps 0-3 consume
-// pages round-robin, each keeping its own softmax state; the CTA merges its 4 states into
-// one partial record, and the last CTA of the (sequence, kv-head) (atomic ticket, no
-// waiting) merges all partial records and writes the output.
+// tier-homogeneous; tiers are visited in order).  Warp 8 lane 0 streams page chunks into a
+// ring of shared-memory stages with cp.async.bulk (no multicast).  Warps 0-7 form 4 pairs;
+// pair p consumes every 4th page and each warp of the pair takes 32 of its 64 tokens with
+// its own softmax state.  The CTA merges its 8 states into one partial record, and the
+// last CTA of the (sequence, kv-head) (atomic ticket, no waiting) merges all records and
+// writes the output.
 #include "dwkv_common.cuh"
 
 namespace dwkv {
@@ -27,12 +35,40 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleSlack = 8.0f;   // keep a stale max while the new one is < 2^8 larger
 
-struct WarpState {
-    float m[kGQ], l[kGQ];          // running max (log2 domain) and per-lane partial sums
-    float acc[kGQ][4];             // per-lane coefficient-space partials (tier mapping)
-    float m2[kGQ], l2[kGQ];        // probe: no-residual state
-    float acc2[kGQ][4];
-};
+// ------------------------------------------------------------------ warp-level MMA pieces
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t (&r)[2]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(addr));
+}
+// D (16x8 f32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+// x ~= hi + lo with both halves bf16 (about 16 significant bits together)
+__device__ __forceinline__ void split_bf16(float x, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    hi = (uint32_t)__bfloat16_as_ushort(h);
+    lo = bf16_bits(x - __bfloat162float(h));
+}
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -45,7 +81,7 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// signed int8 / int4 code -> float (exact) by biasing into a float's mantissa
+// signed int8 / int4 code -> float (exact), by biasing into a float's mantissa
 __device__ __forceinline__ float code8(uint32_t word, int e) {
     const uint32_t b = (word >> (8 * e)) & 0xffu;
     return __uint_as_float(0x4B400000u | (b ^ 0x80u)) - 12583040.0f;   // 2^23 + 2^22 + 128
@@ -55,255 +91,283 @@ __device__ __forceinline__ float code4(uint32_t word, int e) {
     return __uint_as_float(0x4B400000u | (b ^ 0x8u)) - 12582920.0f;    // 2^23 + 2^22 + 8
 }
 
-// Sum the per-lane partials of a tier mapping into the warp's shared accumulator.
-template <int R, bool PROBE>
-__device__ __forceinline__ void flush(WarpState& w, float4* accc, float4* accc2, int lane) {
-    constexpr int NG = R / 4;
+template <int RMAX, bool PROBE>
+struct WarpAcc {
+    float c[RMAX / 16][4];                 // coefficient-space values, D layout (row j, col n)
+    float r[8][4];                         // residual-space values, D layout (row channel, col n)
+    float c2[PROBE ? RMAX / 16 : 1][4];    // probe: no-residual coefficient-space values
+    float m[kGQ], l[kGQ], m2[kGQ], l2[kGQ];
+};
+
+// Rescale the D-layout accumulators: lane column pair (2c, 2c+1) holds heads (2c)&3, (2c+1)&3.
+template <int N>
+__device__ __forceinline__ void rescale_d(float (&d)[N][4], float a0, float a1) {
 #pragma unroll
-    for (int o = NG; o < 32; o <<= 1)
+    for (int i = 0; i < N; ++i) { d[i][0] *= a0; d[i][1] *= a1; d[i][2] *= a0; d[i][3] *= a1; }
+}
+
+// Address inside a warp's dense residual tile (128 channels x 16 tokens, bf16, 32 B per
+// channel; the 16-byte half is swapped every 4 channels so ldmatrix rows are conflict-free).
+__device__ __forceinline__ uint32_t rd_off(uint32_t ch, uint32_t t) {
+    return ch * 32u + ((((t >> 3) & 1u) ^ ((ch >> 2) & 1u)) << 4) + (t & 7u) * 2u;
+}
+
+// One warp's half of a tier-R page: tokens [32*half, 32*half + 32) of the page's 64 slots,
+// `nv` of them live.  `K` points at the page chunk's key block.
+template <int R, int BITS, bool PROBE, int RMAX>
+__device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int half, int nv, int s,
+                                          const uint32_t (&qb)[RMAX / 16][2], const float4* __restrict__ qs,
+                                          uint8_t* small, uint8_t* rd, uint32_t zero_addr, WarpAcc<RMAX, PROBE>& A,
+                                          int lane) {
+    constexpr int KS = R >= 16 ? R / 16 : 1;         // 16-wide coefficient steps
+    const uint32_t blk = 128u * R + 64u * s + 8u * s * BITS + 128u;
+    const uint32_t off_idx = 128u * R, off_codes = 128u * R + 64u * s, off_sc = off_codes + 8u * s * BITS;
+    const uint8_t* V = K + blk;
+    const int tb = 32 * half;
+    const uint32_t kaddr = smem_addr(K), vaddr = smem_addr(V);
+    float* Ssm = reinterpret_cast<float*>(small);
+    uint8_t* Psm = small + 32 * 16;
+    uint8_t* Wsm = small + 64 * 16;
+    uint8_t* P2sm = small + 96 * 16;
+    const int g = lane >> 2, c = lane & 3, mi = lane >> 3, rr = lane & 7;
+
+    // ---------------- 1. coefficient scores: [32 tokens x R] . [R x 8] on the tensor cores
+    {
+        float d[2][4];
 #pragma unroll
-        for (int h = 0; h < kGQ; ++h)
+        for (int mt = 0; mt < 2; ++mt) {
+            d[mt][0] = d[mt][1] = d[mt][2] = d[mt][3] = 0.f;
+            const uint32_t tok = tb + 16 * mt + (mi & 1) * 8 + rr;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                w.acc[h][c] += __shfl_xor_sync(0xffffffffu, w.acc[h][c], o);
-                if (PROBE) w.acc2[h][c] += __shfl_xor_sync(0xffffffffu, w.acc2[h][c], o);
+            for (int ks = 0; ks < KS; ++ks) {
+                const uint32_t kc = 2 * ks + (mi >> 1);
+                const uint32_t addr = (kc * 8 < (uint32_t)R) ? kaddr + kc * 1024 + tok * 16 : zero_addr;
+                uint32_t a[4];
+                ldsm_x4(addr, a);
+                mma_bf16(d[mt], a, qb[ks]);
             }
-    if (lane < NG) {
+        }
+        // hi + lo columns: lanes c and c^2 hold (hi, lo) of the same two heads
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float4 v = accc[4 * lane + c];
-            v.x += w.acc[0][c]; v.y += w.acc[1][c]; v.z += w.acc[2][c]; v.w += w.acc[3][c];
-            accc[4 * lane + c] = v;
-            if (PROBE) {
-                float4 u = accc2[4 * lane + c];
-                u.x += w.acc2[0][c]; u.y += w.acc2[1][c]; u.z += w.acc2[2][c]; u.w += w.acc2[3][c];
-                accc2[4 * lane + c] = u;
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d[mt][e] += __shfl_xor_sync(0xffffffffu, d[mt][e], 2);
+        if (c < 2) {
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                *reinterpret_cast<float2*>(Ssm + (16 * mt + g) * 4 + 2 * c) = make_float2(d[mt][0], d[mt][1]);
+                *reinterpret_cast<float2*>(Ssm + (16 * mt + g + 8) * 4 + 2 * c) = make_float2(d[mt][2], d[mt][3]);
             }
         }
     }
-#pragma unroll
-    for (int h = 0; h < kGQ; ++h)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) { w.acc[h][c] = 0.f; w.acc2[h][c] = 0.f; }
     __syncwarp();
-}
 
-__device__ __forceinline__ void flush_any(int R, WarpState& w, float4* accc, float4* accc2, int lane, bool probe) {
-    if (probe) {
-        switch (R) {
-            case 8: flush<8, true>(w, accc, accc2, lane); break;
-            case 16: flush<16, true>(w, accc, accc2, lane); break;
-            case 32: flush<32, true>(w, accc, accc2, lane); break;
-            case 64: flush<64, true>(w, accc, accc2, lane); break;
-            case 128: flush<128, true>(w, accc, accc2, lane); break;
-            default: break;
-        }
-    } else {
-        switch (R) {
-            case 8: flush<8, false>(w, accc, accc2, lane); break;
-            case 16: flush<16, false>(w, accc, accc2, lane); break;
-            case 32: flush<32, false>(w, accc, accc2, lane); break;
-            case 64: flush<64, false>(w, accc, accc2, lane); break;
-            case 128: flush<128, false>(w, accc, accc2, lane); break;
-            default: break;
-        }
-    }
-}
-
-// Rescale one softmax state (registers + the warp's shared accumulators) by alpha per head.
-__device__ __forceinline__ void rescale_state(float (&l)[kGQ], float (&acc)[kGQ][4], float4* accc,
-                                              float* accr, const float (&alpha)[kGQ], int r_max, int lane) {
+    // ---------------- 2. key residual gather-dot and the full scores (lane = token)
+    const int t = tb + lane;
+    const bool live = lane < nv;
+    float sc[kGQ], sc2[kGQ];
+    {
 #pragma unroll
-    for (int h = 0; h < kGQ; ++h) {
-        l[h] *= alpha[h];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[h][c] *= alpha[h];
-    }
-    for (int j = lane; j < r_max; j += 32) {
-        float4 v = accc[j];
-        v.x *= alpha[0]; v.y *= alpha[1]; v.z *= alpha[2]; v.w *= alpha[3];
-        accc[j] = v;
-    }
-    if (accr) {
-#pragma unroll
-        for (int h = 0; h < kGQ; ++h)
-#pragma unroll
-            for (int m = 0; m < 4; ++m) accr[h * kD + lane + 32 * m] *= alpha[h];
-    }
-}
-
-// One tier-homogeneous page of 64 token slots (nvalid of them live) for one warp.
-template <int R, int BITS, bool PROBE>
-__device__ __forceinline__ void page_step(const uint8_t* __restrict__ K, int nvalid, int s,
-                                          const float4* __restrict__ qt, const float4* __restrict__ qs,
-                                          float4* p_s, float4* p2_s, float4* accc, float4* accc2, float* accr,
-                                          WarpState& w, int r_max, int lane) {
-    constexpr uint32_t kCo = 128u * R;
-    const uint32_t off_idx = kCo, off_codes = kCo + 64u * s, off_sc = kCo + 64u * s + 8u * s * BITS;
-    const uint8_t* __restrict__ V = K + off_sc + 128u;
-    float sc[2][kGQ], sc2[2][kGQ];
-    // ---------------- scores (keys): coefficient dot + residual gather-dot
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt) {
-        const int t = lane + 32 * tt;
-#pragma unroll
-        for (int h = 0; h < kGQ; ++h) { sc[tt][h] = -INFINITY; sc2[tt][h] = -INFINITY; }
-        if (t < nvalid) {
-            float a[kGQ] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kc = 0; kc < R / 8; ++kc) {
-                const uint4 cw = *reinterpret_cast<const uint4*>(K + kc * 1024 + t * 16);
-                const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float c0 = bf16lo(wv[e]), c1 = bf16hi(wv[e]);
-                    const float4 q0 = qt[kc * 8 + 2 * e], q1 = qt[kc * 8 + 2 * e + 1];
-                    a[0] = fmaf(q0.x, c0, a[0]); a[1] = fmaf(q0.y, c0, a[1]);
-                    a[2] = fmaf(q0.z, c0, a[2]); a[3] = fmaf(q0.w, c0, a[3]);
-                    a[0] = fmaf(q1.x, c1, a[0]); a[1] = fmaf(q1.y, c1, a[1]);
-                    a[2] = fmaf(q1.z, c1, a[2]); a[3] = fmaf(q1.w, c1, a[3]);
-                }
-            }
+        for (int h = 0; h < kGQ; ++h) { sc[h] = -INFINITY; sc2[h] = -INFINITY; }
+        if (live) {
+            const float4 sv = *reinterpret_cast<const float4*>(Ssm + lane * 4);
             float ra[kGQ] = {0.f, 0.f, 0.f, 0.f};
             for (int ch = 0; ch < s; ch += 8) {
                 const uint2 ix = *reinterpret_cast<const uint2*>(K + off_idx + t * s + ch);
                 uint32_t cw0, cw1 = 0;
                 if (BITS == 8) {
-                    const uint2 c = *reinterpret_cast<const uint2*>(K + off_codes + t * s + ch);
-                    cw0 = c.x; cw1 = c.y;
+                    const uint2 cc = *reinterpret_cast<const uint2*>(K + off_codes + t * s + ch);
+                    cw0 = cc.x;
+                    cw1 = cc.y;
                 } else {
                     cw0 = *reinterpret_cast<const uint32_t*>(K + off_codes + t * (s / 2) + ch / 2);
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const uint32_t i = ((e < 4 ? ix.x : ix.y) >> (8 * (e & 3))) & 0xffu;
-                    const float c = BITS == 8 ? code8(e < 4 ? cw0 : cw1, e & 3) : code4(cw0, e);
+                    const float cf = BITS == 8 ? code8(e < 4 ? cw0 : cw1, e & 3) : code4(cw0, e);
                     const float4 q = qs[i];
-                    ra[0] = fmaf(q.x, c, ra[0]); ra[1] = fmaf(q.y, c, ra[1]);
-                    ra[2] = fmaf(q.z, c, ra[2]); ra[3] = fmaf(q.w, c, ra[3]);
+                    ra[0] = fmaf(q.x, cf, ra[0]);
+                    ra[1] = fmaf(q.y, cf, ra[1]);
+                    ra[2] = fmaf(q.z, cf, ra[2]);
+                    ra[3] = fmaf(q.w, cf, ra[3]);
                 }
             }
             const float scale = __half2float(*reinterpret_cast<const __half*>(K + off_sc + t * 2));
-#pragma unroll
-            for (int h = 0; h < kGQ; ++h) {
-                sc[tt][h] = fmaf(scale, ra[h], a[h]);
-                sc2[tt][h] = a[h];
-            }
+            sc[0] = fmaf(scale, ra[0], sv.x);
+            sc[1] = fmaf(scale, ra[1], sv.y);
+            sc[2] = fmaf(scale, ra[2], sv.z);
+            sc[3] = fmaf(scale, ra[3], sv.w);
+            sc2[0] = sv.x; sc2[1] = sv.y; sc2[2] = sv.z; sc2[3] = sv.w;
         }
     }
-    // ---------------- online softmax (per warp; lazily rescaled)
-    float p[2][kGQ], p2[2][kGQ];
+
+    // ---------------- 3. online softmax (lazy rescale), p and p * scale^V as bf16 hi/lo rows
     {
-        float mloc[kGQ], alpha[kGQ];
+        float alpha[kGQ];
         bool any = false;
 #pragma unroll
         for (int h = 0; h < kGQ; ++h) {
-            mloc[h] = warp_max(fmaxf(sc[0][h], sc[1][h]));
+            const float ml = warp_max(sc[h]);
             alpha[h] = 1.f;
-            if (mloc[h] > w.m[h] + kRescaleSlack) {
-                alpha[h] = exp2f(w.m[h] - mloc[h]);
-                w.m[h] = mloc[h];
+            if (ml > A.m[h] + kRescaleSlack) {
+                alpha[h] = exp2f(A.m[h] - ml);
+                A.m[h] = ml;
                 any = true;
             }
         }
-        if (any) rescale_state(w.l, w.acc, accc, accr, alpha, r_max, lane);
+        if (any) {
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt)
+            for (int h = 0; h < kGQ; ++h) A.l[h] *= alpha[h];
+            const float a0 = alpha[(2 * c) & 3], a1 = alpha[(2 * c + 1) & 3];
+            rescale_d(A.c, a0, a1);
+            rescale_d(A.r, a0, a1);
+        }
+        float p[kGQ];
 #pragma unroll
-            for (int h = 0; h < kGQ; ++h) {
-                p[tt][h] = exp2f(sc[tt][h] - w.m[h]);     // -inf -> 0 for dead slots
-                w.l[h] += p[tt][h];
-            }
+        for (int h = 0; h < kGQ; ++h) {
+            p[h] = exp2f(sc[h] - A.m[h]);      // dead lanes: exp2(-inf) = 0
+            A.l[h] += p[h];
+        }
+        const float scv = live ? __half2float(*reinterpret_cast<const __half*>(V + off_sc + t * 2)) : 0.f;
+        uint32_t ph[4], pl[4], wh[4], wl[4];
+#pragma unroll
+        for (int h = 0; h < kGQ; ++h) {
+            split_bf16(p[h], ph[h], pl[h]);
+            split_bf16(p[h] * scv, wh[h], wl[h]);
+        }
+        *reinterpret_cast<uint4*>(Psm + lane * 16) =
+            make_uint4(ph[0] | (ph[1] << 16), ph[2] | (ph[3] << 16), pl[0] | (pl[1] << 16), pl[2] | (pl[3] << 16));
+        *reinterpret_cast<uint4*>(Wsm + lane * 16) =
+            make_uint4(wh[0] | (wh[1] << 16), wh[2] | (wh[3] << 16), wl[0] | (wl[1] << 16), wl[2] | (wl[3] << 16));
         if (PROBE) {
             bool any2 = false;
 #pragma unroll
             for (int h = 0; h < kGQ; ++h) {
-                mloc[h] = warp_max(fmaxf(sc2[0][h], sc2[1][h]));
+                const float ml = warp_max(sc2[h]);
                 alpha[h] = 1.f;
-                if (mloc[h] > w.m2[h] + kRescaleSlack) {
-                    alpha[h] = exp2f(w.m2[h] - mloc[h]);
-                    w.m2[h] = mloc[h];
+                if (ml > A.m2[h] + kRescaleSlack) {
+                    alpha[h] = exp2f(A.m2[h] - ml);
+                    A.m2[h] = ml;
                     any2 = true;
                 }
             }
-            if (any2) rescale_state(w.l2, w.acc2, accc2, nullptr, alpha, r_max, lane);
+            if (any2) {
 #pragma unroll
-            for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-                for (int h = 0; h < kGQ; ++h) {
-                    p2[tt][h] = exp2f(sc2[tt][h] - w.m2[h]);
-                    w.l2[h] += p2[tt][h];
-                }
-        }
-    }
-    // ---------------- residual-space values: scatter p * scale * code
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt) {
-        const int t = lane + 32 * tt;
-        if (t < nvalid) {
-            p_s[t] = make_float4(p[tt][0], p[tt][1], p[tt][2], p[tt][3]);
-            if (PROBE) p2_s[t] = make_float4(p2[tt][0], p2[tt][1], p2[tt][2], p2[tt][3]);
-            const float scale = __half2float(*reinterpret_cast<const __half*>(V + off_sc + t * 2));
-            float wt[kGQ];
-#pragma unroll
-            for (int h = 0; h < kGQ; ++h) wt[h] = p[tt][h] * scale;
-            for (int ch = 0; ch < s; ch += 8) {
-                const uint2 ix = *reinterpret_cast<const uint2*>(V + off_idx + t * s + ch);
-                uint32_t cw0, cw1 = 0;
-                if (BITS == 8) {
-                    const uint2 c = *reinterpret_cast<const uint2*>(V + off_codes + t * s + ch);
-                    cw0 = c.x; cw1 = c.y;
-                } else {
-                    cw0 = *reinterpret_cast<const uint32_t*>(V + off_codes + t * (s / 2) + ch / 2);
-                }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint32_t i = ((e < 4 ? ix.x : ix.y) >> (8 * (e & 3))) & 0xffu;
-                    const float c = BITS == 8 ? code8(e < 4 ? cw0 : cw1, e & 3) : code4(cw0, e);
-#pragma unroll
-                    for (int h = 0; h < kGQ; ++h) atomicAdd(&accr[h * kD + i], wt[h] * c);
-                }
+                for (int h = 0; h < kGQ; ++h) A.l2[h] *= alpha[h];
+                rescale_d(A.c2, alpha[(2 * c) & 3], alpha[(2 * c + 1) & 3]);
             }
+#pragma unroll
+            for (int h = 0; h < kGQ; ++h) {
+                p[h] = exp2f(sc2[h] - A.m2[h]);
+                A.l2[h] += p[h];
+                split_bf16(p[h], ph[h], pl[h]);
+            }
+            *reinterpret_cast<uint4*>(P2sm + lane * 16) =
+                make_uint4(ph[0] | (ph[1] << 16), ph[2] | (ph[3] << 16), pl[0] | (pl[1] << 16), pl[2] | (pl[3] << 16));
         }
     }
     __syncwarp();
-    // ---------------- coefficient-space values: lane = (4-column group, token subset)
-    {
-        constexpr int NG = R / 4, NSUB = 32 / NG;
-        const int g4 = lane % NG, sub = lane / NG;
-        const uint8_t* vb = V + (g4 >> 1) * 1024 + (g4 & 1) * 8;
-#pragma unroll 4
-        for (int t = sub; t < nvalid; t += NSUB) {
-            const uint2 cw = *reinterpret_cast<const uint2*>(vb + t * 16);
-            const float v[4] = {bf16lo(cw.x), bf16hi(cw.x), bf16lo(cw.y), bf16hi(cw.y)};
-            const float4 pp = p_s[t];
+
+    // ---------------- 4. coefficient-space values: acc_c[j][n] += sum_t C^V[t][j] P[t][n]
+    const uint32_t paddr = smem_addr(Psm), waddr = smem_addr(Wsm), p2addr = smem_addr(P2sm);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                w.acc[0][c] = fmaf(pp.x, v[c], w.acc[0][c]);
-                w.acc[1][c] = fmaf(pp.y, v[c], w.acc[1][c]);
-                w.acc[2][c] = fmaf(pp.z, v[c], w.acc[2][c]);
-                w.acc[3][c] = fmaf(pp.w, v[c], w.acc[3][c]);
-            }
-            if (PROBE) {
-                const float4 qq = p2_s[t];
+    for (int ks = 0; ks < 2; ++ks) {
+        uint32_t b[2], b2[2];
+        ldsm_x2_t(paddr + (16 * ks + (lane & 15)) * 16, b);
+        if (PROBE) ldsm_x2_t(p2addr + (16 * ks + (lane & 15)) * 16, b2);
+        const uint32_t tloc = 16 * ks + (mi >> 1) * 8 + rr;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    w.acc2[0][c] = fmaf(qq.x, v[c], w.acc2[0][c]);
-                    w.acc2[1][c] = fmaf(qq.y, v[c], w.acc2[1][c]);
-                    w.acc2[2][c] = fmaf(qq.z, v[c], w.acc2[2][c]);
-                    w.acc2[3][c] = fmaf(qq.w, v[c], w.acc2[3][c]);
+        for (int mt = 0; mt < KS; ++mt) {
+            const uint32_t kc = 2 * mt + (mi & 1);
+            const bool ok = (kc * 8 < (uint32_t)R) && ((int)tloc < nv);
+            uint32_t a[4];
+            ldsm_x4_t(ok ? vaddr + kc * 1024 + (tb + tloc) * 16 : zero_addr, a);
+            mma_bf16(A.c[mt], a, b);
+            if (PROBE) mma_bf16(A.c2[mt], a, b2);
+        }
+    }
+
+    // ---------------- 5. residual-space values through a dense 128 x 16 code tile
+    const uint32_t rdaddr = smem_addr(rd);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const int tl = 16 * ks + (lane & 15);       // token within the half
+        if (tl < nv) {
+            const int tok = tb + tl;
+            const int e0 = (lane >> 4) * (s / 2);
+            for (int e = e0; e < e0 + s / 2; e += 4) {
+                const uint32_t ix = *reinterpret_cast<const uint32_t*>(V + off_idx + tok * s + e);
+                uint32_t cw;
+                if (BITS == 8) cw = *reinterpret_cast<const uint32_t*>(V + off_codes + tok * s + e);
+                else cw = *reinterpret_cast<const uint16_t*>(V + off_codes + tok * (s / 2) + e / 2);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t ch = (ix >> (8 * q)) & 0xffu;
+                    const float cf = BITS == 8 ? code8(cw, q) : code4(cw, q);
+                    *reinterpret_cast<uint16_t*>(rd + rd_off(ch, (uint32_t)(lane & 15))) =
+                        (uint16_t)(__float_as_uint(cf) >> 16);      // small integers are exact in bf16
                 }
             }
         }
+        __syncwarp();
+        uint32_t b[2];
+        ldsm_x2_t(waddr + (16 * ks + (lane & 15)) * 16, b);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const uint32_t ch = 16 * mt + (mi & 1) * 8 + rr;
+            const uint32_t off = ch * 32u + ((((uint32_t)(mi >> 1)) ^ ((ch >> 2) & 1u)) << 4);
+            uint32_t a[4];
+            ldsm_x4(rdaddr + off, a);
+            mma_bf16(A.r[mt], a, b);
+        }
+        __syncwarp();
+        uint4* z = reinterpret_cast<uint4*>(rd);
+#pragma unroll
+        for (int i = 0; i < kRdBytes / 16 / 32; ++i) z[lane + 32 * i] = make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
     }
-    __syncwarp();
+}
+
+template <int BITS, bool PROBE, int RMAX>
+__device__ __forceinline__ void run_page(int R, const uint8_t* K, int half, int nv, int s,
+                                         const uint32_t (&qb)[RMAX / 16][2], const float4* qs, uint8_t* small,
+                                         uint8_t* rd, uint32_t zero_addr, WarpAcc<RMAX, PROBE>& A, int lane) {
+    switch (R) {
+        case 8: half_page<8, BITS, PROBE, RMAX>(K, half, nv, s, qb, qs, small, rd, zero_addr, A, lane); break;
+        case 16: half_page<16, BITS, PROBE, RMAX>(K, half, nv, s, qb, qs, small, rd, zero_addr, A, lane); break;
+        case 32: half_page<32, BITS, PROBE, RMAX>(K, half, nv, s, qb, qs, small, rd, zero_addr, A, lane); break;
+        case 64:
+            if constexpr (RMAX >= 64) half_page<64, BITS, PROBE, RMAX>(K, half, nv, s, qb, qs, small, rd, zero_addr, A, lane);
+            break;
+        case 128:
+            if constexpr (RMAX >= 128) half_page<128, BITS, PROBE, RMAX>(K, half, nv, s, qb, qs, small, rd, zero_addr, A, lane);
+            break;
+        default: break;
+    }
+}
+
+// Sum hi + lo columns of a D-layout accumulator and store acc[j][h] (float4 per row j).
+template <int N>
+__device__ __forceinline__ void store_d(float (&d)[N][4], float* dst, int rows, int lane) {
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d[i][e] += __shfl_xor_sync(0xffffffffu, d[i][e], 2);
+        if (c < 2) {
+            const int j0 = 16 * i + g, j1 = j0 + 8;
+            if (j0 < rows) *reinterpret_cast<float2*>(dst + j0 * 4 + 2 * c) = make_float2(d[i][0], d[i][1]);
+            if (j1 < rows) *reinterpret_cast<float2*>(dst + j1 * 4 + 2 * c) = make_float2(d[i][2], d[i][3]);
+        }
+    }
 }
 
 }  // namespace
 
-template <int BITS, bool PROBE>
+template <int BITS, bool PROBE, int RMAX>
 __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G, const State S, const DecodeCall C) {
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y;
     const int NS = C.stages;
@@ -312,13 +376,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + NS), basis_bar = smem_addr(bars + 2 * NS);
     float4* qt = reinterpret_cast<float4*>(smem + L.qt);
     float4* qs = reinterpret_cast<float4*>(smem + L.q);
-    // per-CTA tier table
     uint32_t* m_cnt = reinterpret_cast<uint32_t*>(smem + L.misc);      // [8]
     uint32_t* m_P = m_cnt + 8;                                          // [9] page prefix
     uint32_t* m_R = m_P + 9;                                            // [8]
     uint32_t* m_chunk = m_R + 8;                                        // [8]
-    uint32_t* m_misc = m_chunk + 8;                                     // p_begin p_end last flag
-    float* m_state = reinterpret_cast<float*>(m_misc + 8);              // [4 warps][16]
+    uint32_t* m_misc = m_chunk + 8;                                     // p_begin p_end last
+    float* m_state = reinterpret_cast<float*>(m_misc + 8);              // [8 warps][16]
+    float* mf = m_state + kConsumerWarps * 16;                          // [2][8 warps][4] factors
 
     // ---- which sequence / split
     int ci = 0;
@@ -336,43 +400,36 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
 
     if (tid == 0) {
         const uint32_t* cnt = S.counts + cnt_index(G, seq, C.g, h);
-        unsigned long long Bs[kMaxTiers + 1];
         uint32_t P = 0;
         unsigned long long B = 0;
         for (int k = 0; k < G.ntiers; ++k) {
-            const uint32_t c = cnt[k], np = (c + kPage - 1) / kPage;
-            m_cnt[k] = c;
+            const uint32_t cc = cnt[k], np = (cc + kPage - 1) / kPage;
+            m_cnt[k] = cc;
             m_P[k] = P;
             m_R[k] = (uint32_t)G.tiers[k];
             m_chunk[k] = G.chunk_bytes[k];
-            Bs[k] = B;
             P += np;
             B += (unsigned long long)np * G.chunk_bytes[k];
         }
         m_P[G.ntiers] = P;
-        Bs[G.ntiers] = B;
         // byte-balanced page range: pages whose first byte lies in [lo, hi)
         const unsigned long long lo = B * (unsigned long long)split / nsplit;
         const unsigned long long hi = B * (unsigned long long)(split + 1) / nsplit;
         uint32_t pb = P, pe = P;
+        unsigned long long Bk = B;
         for (int k = G.ntiers - 1; k >= 0; --k) {
             const uint32_t np = m_P[k + 1] - m_P[k];
-            if (!np) continue;
             const unsigned long long ch = G.chunk_bytes[k];
-            if (lo <= Bs[k] + (np - 1) * ch) {
-                const unsigned long long d = lo > Bs[k] ? (lo - Bs[k] + ch - 1) / ch : 0;
-                pb = m_P[k] + (uint32_t)d;
-            }
-            if (hi <= Bs[k] + (np - 1) * ch) {
-                const unsigned long long d = hi > Bs[k] ? (hi - Bs[k] + ch - 1) / ch : 0;
-                pe = m_P[k] + (uint32_t)d;
-            }
+            Bk -= (unsigned long long)np * ch;      // first byte of tier k
+            if (!np) continue;
+            if (lo <= Bk + (np - 1) * ch) pb = m_P[k] + (uint32_t)(lo > Bk ? (lo - Bk + ch - 1) / ch : 0);
+            if (hi <= Bk + (np - 1) * ch) pe = m_P[k] + (uint32_t)(hi > Bk ? (hi - Bk + ch - 1) / ch : 0);
         }
         m_misc[0] = pb;
         m_misc[1] = pe > pb ? pe : pb;
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(full0 + 8 * s, 1);
-            mbar_init(empty0 + 8 * s, 1);
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(full0 + 8 * i, 1);
+            mbar_init(empty0 + 8 * i, 2);     // both warps of the pair release
         }
         mbar_init(basis_bar, 1);
         fence_mbar_init();
@@ -382,22 +439,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     const size_t basis_off = ((size_t)C.g * G.Hkv + h) * kD * G.r_max;
 
     if (warp == kConsumerWarps) {
-        // ================= producer warp: basis, then the page chunks
+        // ================= producer warp: B_K (into the residual tiles), then page chunks
         if (lane == 0) {
             const uint32_t bytes = (uint32_t)kD * G.r_max * 2;
             mbar_arrive_expect_tx(basis_bar, bytes);
-            bulk_g2s(smem_addr(smem + L.basis), S.basis_k + basis_off, bytes, basis_bar);
+            bulk_g2s(smem_addr(smem + L.rd), S.basis_k + basis_off, bytes, basis_bar);
         }
         const uint32_t npages = p_end - p_begin;
         const size_t pbase = page_index(G, seq, C.g, h, 0);
-        const size_t tier_stride = (size_t)G.max_pages;
-        // page units are fetched 32 at a time by the whole warp, one batch ahead
         auto fetch = [&](uint32_t u) -> uint32_t {
             if (u >= npages) return 0u;
             const uint32_t p = p_begin + u;
             int k = 0;
             while (k + 1 < G.ntiers && p >= m_P[k + 1]) ++k;
-            return S.pages[pbase + (size_t)k * tier_stride + (p - m_P[k])];
+            return S.pages[pbase + (size_t)k * G.max_pages + (p - m_P[k])];
         };
         uint32_t next = fetch(lane);
         bool ok = true;
@@ -428,94 +483,126 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         }
     } else {
         // ================= consumer warps
-        uint8_t* wbase = smem + L.warp + warp * L.warp_stride;
-        float4* p_s = reinterpret_cast<float4*>(wbase + L.p);
-        float4* p2_s = reinterpret_cast<float4*>(wbase + L.p2);
-        float4* accc = reinterpret_cast<float4*>(wbase + L.accc);
-        float4* accc2 = reinterpret_cast<float4*>(wbase + L.accc2);
-        float* accr = reinterpret_cast<float*>(wbase + L.accr);
+        uint8_t* rd = smem + L.rd + warp * kRdBytes;
+        uint8_t* small = smem + L.small + warp * L.small_stride;
+        const uint32_t zero_addr = smem_addr(smem + L.zero);
         const float qscale = G.tau * kLog2e;
         if (tid < kD) {
             const __nv_bfloat16* q = C.q + ((size_t)ci * G.Hq + (size_t)h * kGQ) * kD + tid;
             qs[tid] = make_float4(__bfloat162float(q[0]) * qscale, __bfloat162float(q[kD]) * qscale,
                                   __bfloat162float(q[2 * kD]) * qscale, __bfloat162float(q[3 * kD]) * qscale);
         }
-        for (int j = lane; j < G.r_max; j += 32) {
-            accc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (PROBE) accc2[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        for (int e = lane; e < kGQ * kD; e += 32) accr[e] = 0.f;
+        if (tid < 8) reinterpret_cast<uint4*>(smem + L.zero)[tid] = make_uint4(0u, 0u, 0u, 0u);
         named_barrier(1, kConsumerWarps * 32);
         bool ok = mbar_wait(basis_bar, 0);
         if (!ok && lane == 0) set_dev_error(S, 6u, (uint32_t)seq, 0xffffffffu);
-        if (ok && tid < G.r_max) {
-            const __nv_bfloat16* bk = reinterpret_cast<const __nv_bfloat16*>(smem + L.basis) + tid;
+        const int rq = G.r_max < 16 ? 16 : G.r_max;
+        if (tid < rq) {
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (ok && tid < G.r_max) {
+                const __nv_bfloat16* bk = reinterpret_cast<const __nv_bfloat16*>(smem + L.rd) + tid;
 #pragma unroll 8
-            for (int i = 0; i < kD; ++i) {
-                const float b = __bfloat162float(bk[i * G.r_max]);
-                const float4 q = qs[i];
-                a.x = fmaf(b, q.x, a.x); a.y = fmaf(b, q.y, a.y);
-                a.z = fmaf(b, q.z, a.z); a.w = fmaf(b, q.w, a.w);
+                for (int i = 0; i < kD; ++i) {
+                    const float b = __bfloat162float(bk[i * G.r_max]);
+                    const float4 q = qs[i];
+                    a.x = fmaf(b, q.x, a.x); a.y = fmaf(b, q.y, a.y);
+                    a.z = fmaf(b, q.z, a.z); a.w = fmaf(b, q.w, a.w);
+                }
             }
             qt[tid] = a;
         }
         named_barrier(1, kConsumerWarps * 32);
-
-        WarpState w;
+        // q~ as the MMA B operand: column n < 4 = bf16 hi of head n, n >= 4 = lo of head n-4
+        uint32_t qb[RMAX / 16][2];
+        {
+            const int g = lane >> 2, c = lane & 3, n = g & 3;
+            const bool lo_half = g >= 4;
 #pragma unroll
-        for (int hh = 0; hh < kGQ; ++hh) {
-            w.m[hh] = -INFINITY; w.l[hh] = 0.f; w.m2[hh] = -INFINITY; w.l2[hh] = 0.f;
+            for (int ks = 0; ks < RMAX / 16; ++ks) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) { w.acc[hh][c] = 0.f; w.acc2[hh][c] = 0.f; }
+                for (int r2 = 0; r2 < 2; ++r2) {
+                    uint32_t pk = 0;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int k = 16 * ks + 8 * r2 + 2 * c + e;
+                        float v = 0.f;
+                        if (k < rq) {
+                            const float4 t4 = qt[k];
+                            v = n == 0 ? t4.x : n == 1 ? t4.y : n == 2 ? t4.z : t4.w;
+                        }
+                        uint32_t hi, lo;
+                        split_bf16(v, hi, lo);
+                        pk |= (lo_half ? lo : hi) << (16 * e);
+                    }
+                    qb[ks][r2] = pk;
+                }
+            }
         }
-        int curR = 0;
-        const int s = G.s;
-        for (uint32_t u = warp; ok && p_begin + u < p_end; u += kConsumerWarps) {
+        {   // the residual tiles held B_K until now; clear this warp's tile
+            uint4* z = reinterpret_cast<uint4*>(rd);
+            for (int i = lane; i < kRdBytes / 16; i += 32) z[i] = make_uint4(0u, 0u, 0u, 0u);
+            __syncwarp();
+        }
+
+        WarpAcc<RMAX, PROBE> A;
+#pragma unroll
+        for (int i = 0; i < RMAX / 16; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) A.c[i][e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < (PROBE ? RMAX / 16 : 1); ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) A.c2[i][e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) A.r[i][e] = 0.f;
+#pragma unroll
+        for (int hh = 0; hh < kGQ; ++hh) { A.m[hh] = -INFINITY; A.l[hh] = 0.f; A.m2[hh] = -INFINITY; A.l2[hh] = 0.f; }
+
+        const int pair = warp >> 1, half = warp & 1, s = G.s;
+        for (uint32_t u = pair; ok && p_begin + u < p_end; u += kPairs) {
             const uint32_t p = p_begin + u, st = u % NS;
             int k = 0;
             while (k + 1 < G.ntiers && p >= m_P[k + 1]) ++k;
             const int R = (int)m_R[k];
             const uint32_t pit = p - m_P[k], npk = m_P[k + 1] - m_P[k];
             const int nvalid = pit + 1 < npk ? kPage : (int)(m_cnt[k] - pit * kPage);
-            if (R != curR) {
-                flush_any(curR, w, accc, accc2, lane, PROBE);
-                curR = R;
-            }
             if (!mbar_wait(full0 + 8 * st, (u / NS) & 1)) {
                 if (lane == 0) set_dev_error(S, 6u, (uint32_t)seq, u);
                 ok = false;
                 break;
             }
-            const uint8_t* stg = smem + L.stages + (size_t)st * G.stage_bytes;
-            switch (R) {
-                case 8: page_step<8, BITS, PROBE>(stg, nvalid, s, qt, qs, p_s, p2_s, accc, accc2, accr, w, G.r_max, lane); break;
-                case 16: page_step<16, BITS, PROBE>(stg, nvalid, s, qt, qs, p_s, p2_s, accc, accc2, accr, w, G.r_max, lane); break;
-                case 32: page_step<32, BITS, PROBE>(stg, nvalid, s, qt, qs, p_s, p2_s, accc, accc2, accr, w, G.r_max, lane); break;
-                case 64: page_step<64, BITS, PROBE>(stg, nvalid, s, qt, qs, p_s, p2_s, accc, accc2, accr, w, G.r_max, lane); break;
-                case 128: page_step<128, BITS, PROBE>(stg, nvalid, s, qt, qs, p_s, p2_s, accc, accc2, accr, w, G.r_max, lane); break;
-                default: break;
-            }
+            const int nv = min(max(nvalid - 32 * half, 0), 32);
+            if (nv > 0)
+                run_page<BITS, PROBE, RMAX>(R, smem + L.stages + (size_t)st * G.stage_bytes, half, nv, s, qb, qs,
+                                            small, rd, zero_addr, A, lane);
+            __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8 * st);
         }
-        flush_any(curR, w, accc, accc2, lane, PROBE);
+        // ---- per-warp results: acc_c [r_max][4] and acc_r [d][4] into the residual tile,
+        //      the probe's acc_c2 into the small buffers; m / l into m_state
+        float* oc = reinterpret_cast<float*>(rd);
+        float* orr = oc + G.r_max * 4;
+        store_d(A.c, oc, G.r_max, lane);
+        store_d(A.r, orr, kD, lane);
+        if (PROBE) store_d(A.c2, reinterpret_cast<float*>(small), G.r_max, lane);
         float* ms = m_state + warp * 16;
 #pragma unroll
         for (int hh = 0; hh < kGQ; ++hh) {
-            const float l = warp_sum(w.l[hh]);
-            const float l2 = PROBE ? warp_sum(w.l2[hh]) : 0.f;
+            const float l = warp_sum(A.l[hh]);
+            const float l2 = PROBE ? warp_sum(A.l2[hh]) : 0.f;
             if (lane == 0) {
-                ms[hh] = w.m[hh]; ms[4 + hh] = l;
-                ms[8 + hh] = w.m2[hh]; ms[12 + hh] = l2;
+                ms[hh] = A.m[hh]; ms[4 + hh] = l;
+                ms[8 + hh] = A.m2[hh]; ms[12 + hh] = l2;
             }
         }
     }
     __syncthreads();
 
-    // ================= CTA merge of the 4 warp states -> partial record
+    // ================= CTA merge of the 8 warp states -> partial record
     const int nrec = C.total_splits;
     float* rec = C.ws + ((size_t)h * nrec + blockIdx.x) * C.rec_floats;
-    float* mf = reinterpret_cast<float*>(smem + L.stages);   // [2][4 warps][4 heads] factors; stages are idle now
     if (tid < 2 * kGQ) {
         const int which = tid / kGQ, hh = tid % kGQ;
         if (which == 0 || PROBE) {
@@ -525,7 +612,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
                 const float mw = m_state[w2 * 16 + which * 8 + hh];
                 const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                mf[which * 16 + w2 * 4 + hh] = f;
+                mf[which * 32 + w2 * 4 + hh] = f;
                 Lsum += f * m_state[w2 * 16 + which * 8 + 4 + hh];
             }
             rec[which * 8 + hh] = M;
@@ -542,18 +629,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             const int hh = e / G.r_max, j = e % G.r_max;
             float v = 0.f, v2 = 0.f;
             for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
-                const uint8_t* wb = smem + L.warp + w2 * L.warp_stride;
-                v += mf[w2 * 4 + hh] * reinterpret_cast<const float*>(wb + L.accc)[j * 4 + hh];
-                if (PROBE) v2 += mf[16 + w2 * 4 + hh] * reinterpret_cast<const float*>(wb + L.accc2)[j * 4 + hh];
+                v += mf[w2 * 4 + hh] * reinterpret_cast<const float*>(smem + L.rd + w2 * kRdBytes)[j * 4 + hh];
+                if (PROBE)
+                    v2 += mf[32 + w2 * 4 + hh] *
+                          reinterpret_cast<const float*>(smem + L.small + w2 * L.small_stride)[j * 4 + hh];
             }
             rc[e] = v;
             if (PROBE) rc2[e] = v2;
         }
         for (int e = tid; e < kGQ * kD; e += blockDim.x) {
-            const int hh = e / kD;
+            const int hh = e / kD, i = e % kD;
             float v = 0.f;
             for (int w2 = 0; w2 < kConsumerWarps; ++w2)
-                v += mf[w2 * 4 + hh] * reinterpret_cast<const float*>(smem + L.warp + w2 * L.warp_stride + L.accr)[e];
+                v += mf[w2 * 4 + hh] *
+                     reinterpret_cast<const float*>(smem + L.rd + w2 * kRdBytes)[G.r_max * 4 + i * 4 + hh];
             rr[e] = v;
         }
     }
@@ -575,7 +664,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     float* cc2 = cc + kGQ * G.r_max;                                   // [4][r_max]
     float* cr = cc2 + kGQ * G.r_max;                                   // [4][d]
     float* Ls = cr + kGQ * kD;                                         // [2][4]
-    float* red = Ls + 8;                                               // [2][160] reductions
+    float* red = Ls + 8;                                               // [2][threads] reductions
     if (tid < 2 * kGQ) {
         const int which = tid / kGQ, hh = tid % kGQ;
         if (which == 0 || PROBE) {
@@ -653,9 +742,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
 }
 
 // explicit instantiations
-template __global__ void decode_kernel<8, false>(const Geom, const State, const DecodeCall);
-template __global__ void decode_kernel<4, false>(const Geom, const State, const DecodeCall);
-template __global__ void decode_kernel<8, true>(const Geom, const State, const DecodeCall);
-template __global__ void decode_kernel<4, true>(const Geom, const State, const DecodeCall);
+#define DWKV_DECODE_INST(B, P, R) \
+    template __global__ void decode_kernel<B, P, R>(const Geom, const State, const DecodeCall);
+DWKV_DECODE_INST(8, false, 32)
+DWKV_DECODE_INST(8, false, 64)
+DWKV_DECODE_INST(8, false, 128)
+DWKV_DECODE_INST(4, false, 32)
+DWKV_DECODE_INST(4, false, 64)
+DWKV_DECODE_INST(4, false, 128)
+DWKV_DECODE_INST(8, true, 32)
+DWKV_DECODE_INST(8, true, 64)
+DWKV_DECODE_INST(8, true, 128)
+DWKV_DECODE_INST(4, true, 32)
+DWKV_DECODE_INST(4, true, 64)
+DWKV_DECODE_INST(4, true, 128)
+#undef DWKV_DECODE_INST
 
 }  // namespace dwkv

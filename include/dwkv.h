@@ -213,8 +213,9 @@ dwkv_status dwkv_pool_usage(dwkv_handle h, void* stream, dwkv_pool_stats* out);
  * DWKV_ERR_CUDA if the stream reported a CUDA error. */
 dwkv_status dwkv_sync_status(dwkv_handle h, void* stream);
 
-/* Launch tuning (for measurement sweeps): decode CTAs per SM (1 or 2), split waves per
- * decode (>= 1) and pipeline stages per CTA (0 = largest that fits).  Returns
+/* Launch tuning (for measurement sweeps): decode CTAs per SM (1 in this build: one
+ * 288-thread CTA fills an SM's registers), split waves per decode (1..8) and pipeline
+ * stages per CTA (0 = largest that fits, else a multiple of 4).  Returns
  * DWKV_ERR_INVALID_ARG for values out of range. */
 dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t waves,
                                    int32_t stages);

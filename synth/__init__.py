@@ -282,5 +282,5 @@ def make_dense_vectors(wl: Workload, seq: int, layer: int, n: int, bases, device
             for h in range(H):
                 ch = torch.randperm(d, generator=gc)[:k].to(device)
                 x[:, h, ch] += torch.randn(n, k, generator=g, device=device) * math.sqrt(wl.outlier_var)
-        out.append(x.to(torch.bfloat16))
+        out.append(x.to(torch.bfloat16).contiguous())
     return out[0], out[1]
