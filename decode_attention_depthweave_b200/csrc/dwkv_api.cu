@@ -22,7 +22,7 @@ template <int BITS>
 __global__ void export_kernel(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*, uint8_t*,
                               int8_t*, __half*);
 __global__ void reset_kernel(const Geom, const State, int);
-template <int BITS, bool PROBE, int RMAX>
+template <int BITS, bool PROBE, int RMAX, int S>
 __global__ void decode_kernel(const Geom, const State, const DecodeCall);
 }  // namespace dwkv
 
@@ -101,6 +101,8 @@ dwkv_status check_supported(const dwkv_config* c) {
     if (c->num_q_heads != kGQ * c->num_kv_heads)
         return fail(DWKV_ERR_UNSUPPORTED, "this build has kernels for 4 query heads per kv head only");
     if (!is_pow2_rank(c->r_max)) return fail(DWKV_ERR_UNSUPPORTED, "r_max must be one of 8, 16, 32, 64, 128");
+    if (c->resid_channels != 0 && c->resid_channels != 8 && c->resid_channels != 16 && c->resid_channels != 32)
+        return fail(DWKV_ERR_UNSUPPORTED, "this build has kernels for resid_channels 0, 8, 16 or 32");
     for (int k = 0; k < c->num_tiers; ++k)
         if (!is_pow2_rank(c->tiers[k]))
             return fail(DWKV_ERR_UNSUPPORTED, "tier ranks must be among 8, 16, 32, 64, 128");
@@ -187,6 +189,7 @@ struct dwkv_ctx {
     std::vector<int32_t> len;       // [max_batch][L]
     std::vector<int32_t> placed;    // [max_batch][G]
     int dec_ctas_per_sm = 1, dec_waves = 1, dec_stages_req = 0;
+    int dec_tok_weight = 1024;      // split balance: byte-equivalent cost of one token
 };
 
 namespace {
@@ -415,12 +418,12 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
     if (e == cudaSuccess) {
         const int maxs = (int)h->smem_optin;
         const void* kernels[] = {
-            (const void*)decode_kernel<8, false, 32>, (const void*)decode_kernel<8, false, 64>,
-            (const void*)decode_kernel<8, false, 128>, (const void*)decode_kernel<4, false, 32>,
-            (const void*)decode_kernel<4, false, 64>, (const void*)decode_kernel<4, false, 128>,
-            (const void*)decode_kernel<8, true, 32>, (const void*)decode_kernel<8, true, 64>,
-            (const void*)decode_kernel<8, true, 128>, (const void*)decode_kernel<4, true, 32>,
-            (const void*)decode_kernel<4, true, 64>, (const void*)decode_kernel<4, true, 128>,
+#define DWKV_K(B, P) (const void*)decode_kernel<B, P, 64, 0>, (const void*)decode_kernel<B, P, 64, 8>,       \
+                     (const void*)decode_kernel<B, P, 64, 16>, (const void*)decode_kernel<B, P, 64, 32>,     \
+                     (const void*)decode_kernel<B, P, 128, 0>, (const void*)decode_kernel<B, P, 128, 8>,     \
+                     (const void*)decode_kernel<B, P, 128, 16>, (const void*)decode_kernel<B, P, 128, 32>
+            DWKV_K(4, false), DWKV_K(4, true), DWKV_K(8, false), DWKV_K(8, true),
+#undef DWKV_K
             (const void*)encode_kernel<8>, (const void*)encode_kernel<4>};
         for (const void* k : kernels)
             if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
@@ -599,6 +602,7 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     C.total_splits = total;
     C.stages = stages;
     C.rec_floats = rec_floats_of(G, probe);
+    C.tok_weight = h->dec_tok_weight;
     C.q = static_cast<const __nv_bfloat16*>(q);
     C.out = out;
     C.out_full = out_full;
@@ -606,10 +610,19 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     C.ws = static_cast<float*>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(total, G.Hkv);
-    const int rm = G.r_max <= 32 ? 32 : (G.r_max <= 64 ? 64 : 128);
-#define DWKV_LAUNCH(B, P, R) decode_kernel<B, P, R><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C)
+    const bool big = G.r_max > 64;
+#define DWKV_LAUNCH(B, P, R, SS) decode_kernel<B, P, R, SS><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C)
+#define DWKV_LAUNCH_S(B, P, R)                                  \
+    do {                                                        \
+        switch (G.s) {                                          \
+            case 0: DWKV_LAUNCH(B, P, R, 0); break;             \
+            case 8: DWKV_LAUNCH(B, P, R, 8); break;             \
+            case 16: DWKV_LAUNCH(B, P, R, 16); break;           \
+            default: DWKV_LAUNCH(B, P, R, 32); break;           \
+        }                                                       \
+    } while (0)
 #define DWKV_LAUNCH_R(B, P) \
-    do { if (rm == 32) DWKV_LAUNCH(B, P, 32); else if (rm == 64) DWKV_LAUNCH(B, P, 64); else DWKV_LAUNCH(B, P, 128); } while (0)
+    do { if (big) DWKV_LAUNCH_S(B, P, 128); else DWKV_LAUNCH_S(B, P, 64); } while (0)
     if (!probe) {
         if (G.bits == 8) DWKV_LAUNCH_R(8, false);
         else DWKV_LAUNCH_R(4, false);
@@ -618,6 +631,7 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
         else DWKV_LAUNCH_R(4, true);
     }
 #undef DWKV_LAUNCH_R
+#undef DWKV_LAUNCH_S
 #undef DWKV_LAUNCH
     DWKV_CUDA(cudaGetLastError(), probe ? "probe kernel launch" : "decode kernel launch");
     return DWKV_OK;

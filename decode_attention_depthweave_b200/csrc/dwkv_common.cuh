@@ -36,7 +36,7 @@ constexpr int kMaxSplits = 64;     // decode splits per (sequence, kv-head)
 constexpr int kConsumerWarps = 8;  // 4 pairs; a pair shares one page (32 tokens per warp)
 constexpr int kPairs = kConsumerWarps / 2;
 constexpr int kDecodeThreads = 32 * (kConsumerWarps + 1);  // + 1 producer warp
-constexpr int kRdBytes = 128 * 16 * 2;                     // dense residual tile: 128 ch x 16 tokens bf16
+constexpr int kRdBytes = 128 * 48;                         // dense residual tile: 128 ch x (16 tokens bf16 + pad)
 
 struct Geom {
     int L, LPG, G, Hq, Hkv, d, r_max, ntiers, s, bits, max_batch, max_context, max_pages;
@@ -78,6 +78,7 @@ struct AppendCall {
 
 struct DecodeCall {
     int n, layer, g, lig, total_splits, stages, rec_floats;
+    int tok_weight;          // split balance: cost of one token in byte-equivalents
     int seq[kMaxSeqs];
     int split_begin[kMaxSeqs + 1];
     const __nv_bfloat16* q;  // [n][Hq][d]
@@ -130,15 +131,15 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, int NS, 
     L.q = o;       o += (uint32_t)G.d * 16;
     L.zero = o;    o += 128;
     L.bars = o;    o += (2 * NS + 2) * 8;
-    L.misc = o;    o += 1024;
+    L.misc = o;    o += 1536;
     L.total = (o + 127) & ~127u;
     return L;
 }
 
-// Floats in one decode partial record: m[4] l[4] (m2[4] l2[4]) acc_c[4][r_max]
-// (acc_c2[4][r_max]) acc_r[4][d].  The probe layout is used for both kernels' sizing.
+// Floats in one decode partial record: m[4] l[4] (m2[4] l2[4]) o[4][d] (o2[4][d]), where
+// o = B_V acc_c + acc_r of the CTA's tokens (relative to m).  The probe layout sizes both.
 __host__ __device__ inline int rec_floats_of(const Geom& G, bool probe) {
-    return (probe ? 16 : 8) + (probe ? 8 : 4) * G.r_max + kGQ * G.d;
+    return (probe ? 16 : 8) + (probe ? 2 : 1) * kGQ * G.d;
 }
 
 // ------------------------------------------------------------------------------ device

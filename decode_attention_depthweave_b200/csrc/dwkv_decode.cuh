@@ -1,0 +1,866 @@
+// dwkv_decode.cuh -- fused split-K decode attention (and the probe) over the compressed
+// cache.  "DepthWeave-KV: Token-Adaptive Cross-Layer Residual Factorization for
+// Long-Context KV Cache Compression", §3 Method: the fused kernel loads the shared basis,
+// dequantises only the routed residual channels and feeds the attention score directly,
+// never writing reconstructed keys / values (Eq. (1) evaluated inside attention); the
+// probe is Eq. (3) with the with-residual output as the reference.
+//
+// For the 4 query heads q_h of kv-head h (tau * log2 e folded into q so exp2 can be used):
+//   qt = B_K^T q                                   (once per CTA, B_K bulk-copied to smem)
+//   s_t = qt[:r_t] . c^K_t + scale^K_t sum_i q[idx^K_ti] code^K_ti
+//   online softmax over t;  acc_c += C^V^T p (coefficient space);
+//   acc_r += R^V^T (p * scale^V) (residual space, R^V the dense residual codes)
+//   o = (B_V acc_c + acc_r) / l                   (B_V applied once, in the combine)
+//
+// Tensor cores take the dense, tier-homogeneous coefficient blocks: the page's 64 x r_t
+// coefficient tile against q~ (scores) and against p (values), and the value residual
+// after it is expanded into a dense 128-channel x 16-token tile in shared memory.  The
+// operands that are not exact in bf16 (q~, p, p * scale) are split into bf16 hi + lo
+// halves (two MMA columns each), so products keep ~15 significant bits and accumulate in
+// fp32.  The key residual is a gather-dot on the CUDA cores.
+//
+// Work split: a CTA takes a cost-balanced run of one (sequence, kv-head)'s pages (pages are
+// tier-homogeneous; tiers are visited in order; a page costs its bytes plus a per-token
+// weight).  Warp 8 lane 0 builds the CTA's page table and streams page chunks into a ring
+// of shared-memory stages with cp.async.bulk (no multicast).  Warps 0-7 form 4 pairs; pair p
+// consumes every 4th page and each warp of the pair takes 32 of its 64 tokens with its own
+// softmax state.  The CTA merges its 8 states into one partial record, and the last CTA of
+// the (sequence, kv-head) (atomic ticket, no waiting) merges all records and writes the
+// output.
+#pragma once
+#include "dwkv_common.cuh"
+
+namespace dwkv {
+
+namespace decode_detail {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleSlack = 8.0f;   // keep a stale max while the new one is < 2^8 larger
+
+// ------------------------------------------------------------------ warp-level MMA pieces
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t (&r)[2]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(addr));
+}
+// D (16x8 f32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// x ~= hi + lo with both halves bf16, rounding to nearest (prologue only)
+__device__ __forceinline__ void split_bf16_rn(float x, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    hi = (uint32_t)__bfloat16_as_ushort(h);
+    lo = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(h)));
+}
+// Two values as bf16 hi halves (truncated) in one word, and their remainders' hi halves in
+// another: x - trunc16(x) is exact in fp32 and its own truncation leaves < 2^-14 |x|.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+    const float ra = a - __uint_as_float(ua & 0xffff0000u);
+    const float rb = b - __uint_as_float(ub & 0xffff0000u);
+    hi = __byte_perm(ua, ub, 0x7632);
+    lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// signed int8 / int4 code -> float (exact), by biasing into a float's mantissa
+__device__ __forceinline__ float code8(uint32_t word, int e) {
+    const uint32_t b = (word >> (8 * e)) & 0xffu;
+    return __uint_as_float(0x4B400000u | (b ^ 0x80u)) - 12583040.0f;   // 2^23 + 2^22 + 128
+}
+__device__ __forceinline__ float code4(uint32_t word, int e) {
+    const uint32_t b = (word >> (4 * e)) & 0xfu;
+    return __uint_as_float(0x4B400000u | (b ^ 0x8u)) - 12582920.0f;    // 2^23 + 2^22 + 8
+}
+
+template <int RMAX, bool PROBE>
+struct WarpAcc {
+    float c[RMAX / 16][4];                 // coefficient-space values, D layout (row j, col n)
+    float r[8][4];                         // residual-space values, D layout (row channel, col n)
+    float c2[PROBE ? RMAX / 16 : 1][4];    // probe: no-residual coefficient-space values
+    float m[kGQ], l[kGQ], m2[kGQ], l2[kGQ];
+};
+
+// Rescale the D-layout accumulators: lane column pair (2c, 2c+1) holds heads (2c)&3, (2c+1)&3.
+template <int N>
+__device__ __forceinline__ void rescale_d(float (&d)[N][4], float a0, float a1) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) { d[i][0] *= a0; d[i][1] *= a1; d[i][2] *= a0; d[i][3] *= a1; }
+}
+
+// Dense residual tile of one warp: 128 channel rows x 16 tokens (bf16) with a 48-byte row
+// pitch (32 data bytes + 16 pad) -- 8 consecutive rows then hit disjoint banks for ldmatrix.
+constexpr uint32_t kRdPitch = 48;
+
+// One warp's half of a tier-R page: tokens [32*half, 32*half + 32) of the page's 64 slots,
+// `nv` of them live.  `K` points at the page chunk's key block.
+template <int R, int S, int BITS, bool PROBE, int RMAX>
+__device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int half, int nv,
+                                          const uint32_t (&qb)[RMAX / 16][2], const float4* __restrict__ qs,
+                                          uint8_t* small, uint8_t* rd, uint32_t zero_addr, WarpAcc<RMAX, PROBE>& A,
+                                          int lane) {
+    constexpr int KS = R >= 16 ? R / 16 : 1;         // 16-wide coefficient steps
+    constexpr uint32_t kOffIdx = 128u * R, kOffCodes = kOffIdx + 64u * S, kOffSc = kOffCodes + 8u * S * BITS;
+    constexpr uint32_t kBlk = kOffSc + 128u;
+    const uint8_t* V = K + kBlk;
+    const int tb = 32 * half;
+    const uint32_t kaddr = smem_addr(K), vaddr = smem_addr(V);
+    float* Ssm = reinterpret_cast<float*>(small);
+    uint8_t* Psm = small + 32 * 16;
+    uint8_t* Wsm = small + 64 * 16;
+    uint8_t* P2sm = small + 96 * 16;
+    const int g = lane >> 2, c = lane & 3, mi = lane >> 3, rr = lane & 7;
+
+    // ---------------- 1. coefficient scores: [32 tokens x R] . [R x 8] on the tensor cores
+    {
+        float d[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            d[mt][0] = d[mt][1] = d[mt][2] = d[mt][3] = 0.f;
+            const uint32_t tok = tb + 16 * mt + (mi & 1) * 8 + rr;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                const uint32_t kc = 2 * ks + (mi >> 1);
+                const uint32_t addr = (kc * 8 < (uint32_t)R) ? kaddr + kc * 1024 + tok * 16 : zero_addr;
+                uint32_t a[4];
+                ldsm_x4(addr, a);
+                mma_bf16(d[mt], a, qb[ks]);
+            }
+        }
+        // hi + lo columns: lanes c and c^2 hold (hi, lo) of the same two heads
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d[mt][e] += __shfl_xor_sync(0xffffffffu, d[mt][e], 2);
+        if (c < 2) {
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                *reinterpret_cast<float2*>(Ssm + (16 * mt + g) * 4 + 2 * c) = make_float2(d[mt][0], d[mt][1]);
+                *reinterpret_cast<float2*>(Ssm + (16 * mt + g + 8) * 4 + 2 * c) = make_float2(d[mt][2], d[mt][3]);
+            }
+        }
+    }
+    __syncwarp();
+
+    // ---------------- 2. key residual gather-dot and the full scores (lane = token)
+    const int t = tb + lane;
+    const bool live = lane < nv;
+    float sc[kGQ], sc2[kGQ];
+    {
+#pragma unroll
+        for (int h = 0; h < kGQ; ++h) { sc[h] = -INFINITY; sc2[h] = -INFINITY; }
+        if (live) {
+            const float4 sv = *reinterpret_cast<const float4*>(Ssm + lane * 4);
+            float ra[kGQ] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ch = 0; ch < S; ch += 8) {
+                const uint2 ix = *reinterpret_cast<const uint2*>(K + kOffIdx + t * S + ch);
+                uint32_t cw0, cw1 = 0;
+                if (BITS == 8) {
+                    const uint2 cc = *reinterpret_cast<const uint2*>(K + kOffCodes + t * S + ch);
+                    cw0 = cc.x;
+                    cw1 = cc.y;
+                } else {
+                    cw0 = *reinterpret_cast<const uint32_t*>(K + kOffCodes + t * (S / 2) + ch / 2);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint32_t i = ((e < 4 ? ix.x : ix.y) >> (8 * (e & 3))) & 0xffu;
+                    const float cf = BITS == 8 ? code8(e < 4 ? cw0 : cw1, e & 3) : code4(cw0, e);
+                    const float4 q = qs[i];
+                    ra[0] = fmaf(q.x, cf, ra[0]);
+                    ra[1] = fmaf(q.y, cf, ra[1]);
+                    ra[2] = fmaf(q.z, cf, ra[2]);
+                    ra[3] = fmaf(q.w, cf, ra[3]);
+                }
+            }
+            const float scale = S ? __half2float(*reinterpret_cast<const __half*>(K + kOffSc + t * 2)) : 0.f;
+            sc[0] = fmaf(scale, ra[0], sv.x);
+            sc[1] = fmaf(scale, ra[1], sv.y);
+            sc[2] = fmaf(scale, ra[2], sv.z);
+            sc[3] = fmaf(scale, ra[3], sv.w);
+            sc2[0] = sv.x; sc2[1] = sv.y; sc2[2] = sv.z; sc2[3] = sv.w;
+        }
+    }
+
+    // ---------------- 3. online softmax (lazy rescale), p and p * scale^V as bf16 hi/lo rows
+    {
+        // The running max only moves when some score exceeds it by the slack (one vote);
+        // otherwise p = exp2(s - m) <= 2^slack stays safe in fp32.
+        float alpha[kGQ];
+        bool over = false;
+#pragma unroll
+        for (int h = 0; h < kGQ; ++h) over |= sc[h] > A.m[h] + kRescaleSlack;
+        if (__any_sync(0xffffffffu, over)) {
+#pragma unroll
+            for (int h = 0; h < kGQ; ++h) {
+                const float ml = warp_max(sc[h]);
+                alpha[h] = 1.f;
+                if (ml > A.m[h] + kRescaleSlack) {
+                    alpha[h] = exp2f(A.m[h] - ml);
+                    A.m[h] = ml;
+                }
+                A.l[h] *= alpha[h];
+            }
+            const float a0 = alpha[(2 * c) & 3], a1 = alpha[(2 * c + 1) & 3];
+            rescale_d(A.c, a0, a1);
+            rescale_d(A.r, a0, a1);
+        }
+        float p[kGQ];
+#pragma unroll
+        for (int h = 0; h < kGQ; ++h) {
+            p[h] = exp2f(sc[h] - A.m[h]);      // dead lanes: exp2(-inf) = 0
+            A.l[h] += p[h];
+        }
+        uint4 pr;
+        split2(p[0], p[1], pr.x, pr.z);
+        split2(p[2], p[3], pr.y, pr.w);
+        *reinterpret_cast<uint4*>(Psm + lane * 16) = pr;
+        if (S) {
+            const float scv = live ? __half2float(*reinterpret_cast<const __half*>(V + kOffSc + t * 2)) : 0.f;
+            uint4 wr;
+            split2(p[0] * scv, p[1] * scv, wr.x, wr.z);
+            split2(p[2] * scv, p[3] * scv, wr.y, wr.w);
+            *reinterpret_cast<uint4*>(Wsm + lane * 16) = wr;
+        }
+        if (PROBE) {
+            bool over2 = false;
+#pragma unroll
+            for (int h = 0; h < kGQ; ++h) over2 |= sc2[h] > A.m2[h] + kRescaleSlack;
+            if (__any_sync(0xffffffffu, over2)) {
+#pragma unroll
+                for (int h = 0; h < kGQ; ++h) {
+                    const float ml = warp_max(sc2[h]);
+                    alpha[h] = 1.f;
+                    if (ml > A.m2[h] + kRescaleSlack) {
+                        alpha[h] = exp2f(A.m2[h] - ml);
+                        A.m2[h] = ml;
+                    }
+                    A.l2[h] *= alpha[h];
+                }
+                rescale_d(A.c2, alpha[(2 * c) & 3], alpha[(2 * c + 1) & 3]);
+            }
+#pragma unroll
+            for (int h = 0; h < kGQ; ++h) {
+                p[h] = exp2f(sc2[h] - A.m2[h]);
+                A.l2[h] += p[h];
+            }
+            uint4 p2;
+            split2(p[0], p[1], p2.x, p2.z);
+            split2(p[2], p[3], p2.y, p2.w);
+            *reinterpret_cast<uint4*>(P2sm + lane * 16) = p2;
+        }
+    }
+    __syncwarp();
+
+    // ---------------- 4. coefficient-space values: acc_c[j][n] += sum_t C^V[t][j] P[t][n]
+    {
+        const uint32_t paddr = smem_addr(Psm), p2addr = smem_addr(P2sm);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t b[2], b2[2];
+            ldsm_x2_t(paddr + (16 * ks + (lane & 15)) * 16, b);
+            if (PROBE) ldsm_x2_t(p2addr + (16 * ks + (lane & 15)) * 16, b2);
+            const uint32_t tloc = 16 * ks + (mi >> 1) * 8 + rr;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                const uint32_t kc = 2 * mt + (mi & 1);
+                const bool ok = (kc * 8 < (uint32_t)R) && ((int)tloc < nv);
+                uint32_t a[4];
+                ldsm_x4_t(ok ? vaddr + kc * 1024 + (tb + tloc) * 16 : zero_addr, a);
+                mma_bf16(A.c[mt], a, b);
+                if (PROBE) mma_bf16(A.c2[mt], a, b2);
+            }
+        }
+    }
+
+    // ---------------- 5. residual-space values through a dense 128 x 16 code tile
+    if (S) {
+        const uint32_t rdaddr = smem_addr(rd), waddr = smem_addr(Wsm);
+        const uint32_t my_col = (uint32_t)(lane & 15) * 2;              // this lane's token column
+        const uint32_t a_off = ((uint32_t)(mi & 1) * 8 + rr) * kRdPitch + (uint32_t)(mi >> 1) * 16;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const int tl = 16 * ks + (lane & 15);       // token within the half
+            if (tl < nv) {
+                const int tok = tb + tl;
+                constexpr int kHalfS = S / 2;           // entries per lane (two lanes per token)
+                const int e0 = (lane >> 4) * kHalfS;
+#pragma unroll
+                for (int e = 0; e < kHalfS; e += 4) {
+                    const uint32_t ix = *reinterpret_cast<const uint32_t*>(V + kOffIdx + tok * S + e0 + e);
+                    uint32_t cw;
+                    if (BITS == 8) cw = *reinterpret_cast<const uint32_t*>(V + kOffCodes + tok * S + e0 + e);
+                    else cw = *reinterpret_cast<const uint16_t*>(V + kOffCodes + tok * (S / 2) + (e0 + e) / 2);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t ch = (ix >> (8 * q)) & 0xffu;
+                        const float cf = BITS == 8 ? code8(cw, q) : code4(cw, q);
+                        *reinterpret_cast<uint16_t*>(rd + ch * kRdPitch + my_col) =
+                            (uint16_t)(__float_as_uint(cf) >> 16);      // small integers are exact in bf16
+                    }
+                }
+            }
+            __syncwarp();
+            uint32_t b[2];
+            ldsm_x2_t(waddr + (16 * ks + (lane & 15)) * 16, b);
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                uint32_t a[4];
+                ldsm_x4(rdaddr + mt * 16 * kRdPitch + a_off, a);
+                mma_bf16(A.r[mt], a, b);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {               // clear the 128 x 32 data bytes
+                const uint32_t k = lane + 32 * i;
+                *reinterpret_cast<uint4*>(rd + (k >> 1) * kRdPitch + (k & 1) * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncwarp();
+        }
+    }
+}
+
+template <int S, int BITS, bool PROBE, int RMAX>
+__device__ __forceinline__ void run_page(int R, const uint8_t* K, int half, int nv, const uint32_t (&qb)[RMAX / 16][2],
+                                         const float4* qs, uint8_t* small, uint8_t* rd, uint32_t zero_addr,
+                                         WarpAcc<RMAX, PROBE>& A, int lane) {
+    switch (R) {
+        case 8: half_page<8, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane); break;
+        case 16: half_page<16, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane); break;
+        case 32: half_page<32, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane); break;
+        case 64: half_page<64, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane); break;
+        case 128:
+            if constexpr (RMAX >= 128) half_page<128, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane);
+            break;
+        default: break;
+    }
+}
+
+// Sum hi + lo columns of a D-layout accumulator and store acc[j][h] (float4 per row j).
+template <int N>
+__device__ __forceinline__ void store_d(float (&d)[N][4], float* dst, int rows, int lane) {
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d[i][e] += __shfl_xor_sync(0xffffffffu, d[i][e], 2);
+        if (c < 2) {
+            const int j0 = 16 * i + g, j1 = j0 + 8;
+            if (j0 < rows) *reinterpret_cast<float2*>(dst + j0 * 4 + 2 * c) = make_float2(d[i][0], d[i][1]);
+            if (j1 < rows) *reinterpret_cast<float2*>(dst + j1 * 4 + 2 * c) = make_float2(d[i][2], d[i][3]);
+        }
+    }
+}
+
+}  // namespace decode_detail
+
+// BITS: code width; PROBE: second softmax state without the residual; RMAX: accumulator
+// rows (>= r_max); S: residual channels per token (0, 8, 16 or 32).
+template <int BITS, bool PROBE, int RMAX, int S>
+__global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G, const State St, const DecodeCall C) {
+    using namespace decode_detail;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.y;
+    const int NS = C.stages;
+    const DecodeSmem L = decode_smem_layout(G, NS, PROBE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);   // full[NS] empty[NS] basis table
+    const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + NS), basis_bar = smem_addr(bars + 2 * NS),
+                   table_bar = smem_addr(bars + 2 * NS + 1);
+    float4* qt = reinterpret_cast<float4*>(smem + L.qt);
+    float4* qs = reinterpret_cast<float4*>(smem + L.q);
+    uint32_t* m_cnt = reinterpret_cast<uint32_t*>(smem + L.misc);      // [8]
+    uint32_t* m_P = m_cnt + 8;                                          // [9] page prefix
+    uint32_t* m_R = m_P + 9;                                            // [8]
+    uint32_t* m_chunk = m_R + 8;                                        // [8]
+    uint32_t* m_misc = m_chunk + 8;                                     // p_begin p_end last
+    float* m_state = reinterpret_cast<float*>(m_misc + 8);              // [8 warps][16]
+    float* mf = m_state + kConsumerWarps * 16;                          // [2][8 warps][4] factors
+
+    // ---- which sequence / split
+    int ci = 0;
+    {
+        int lo = 0, hi = C.n - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (C.split_begin[mid] <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+        }
+        ci = lo;
+    }
+    const int split = blockIdx.x - C.split_begin[ci];
+    const int nsplit = C.split_begin[ci + 1] - C.split_begin[ci];
+    const int seq = C.seq[ci];
+    const size_t basis_off = ((size_t)C.g * G.Hkv + h) * kD * G.r_max;
+
+    uint32_t cv[kMaxTiers];                 // tier counts (producer lane 0)
+    if (warp == kConsumerWarps && lane == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(full0 + 8 * i, 1);
+            mbar_init(empty0 + 8 * i, 2);     // both warps of the pair release
+        }
+        mbar_init(basis_bar, 1);
+        mbar_init(table_bar, 1);
+        fence_mbar_init();
+        // B_K into the residual tiles (free until the main loop) and the counts, both in
+        // flight across the barrier below
+        const uint32_t bytes = (uint32_t)kD * G.r_max * 2;
+        mbar_arrive_expect_tx(basis_bar, bytes);
+        bulk_g2s(smem_addr(smem + L.rd), St.basis_k + basis_off, bytes, basis_bar);
+        const uint32_t* cnt = St.counts + cnt_index(G, seq, C.g, h);
+#pragma unroll
+        for (int k = 0; k < kMaxTiers; ++k) cv[k] = k < G.ntiers ? __ldcg(cnt + k) : 0u;
+    }
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {
+        // ================= producer warp: B_K, the CTA's page range, then page chunks
+        if (lane == 0) {
+            uint32_t P = 0;
+            unsigned long long W = 0;
+            const unsigned long long tokw = (unsigned long long)C.tok_weight * kPage;
+#pragma unroll
+            for (int k = 0; k < kMaxTiers; ++k) {
+                if (k >= G.ntiers) break;
+                const uint32_t np = (cv[k] + kPage - 1) / kPage;
+                m_cnt[k] = cv[k];
+                m_P[k] = P;
+                m_R[k] = (uint32_t)G.tiers[k];
+                m_chunk[k] = G.chunk_bytes[k];
+                P += np;
+                W += (unsigned long long)np * (G.chunk_bytes[k] + tokw);
+            }
+            m_P[G.ntiers] = P;
+            // cost-balanced page range: pages whose first cost unit lies in [lo, hi)
+            const unsigned long long lo = W * (unsigned long long)split / nsplit;
+            const unsigned long long hi = W * (unsigned long long)(split + 1) / nsplit;
+            uint32_t pb = P, pe = P;
+            unsigned long long Wk = W;
+            for (int k = G.ntiers - 1; k >= 0; --k) {
+                const uint32_t np = m_P[k + 1] - m_P[k];
+                const unsigned long long w = G.chunk_bytes[k] + tokw;
+                Wk -= (unsigned long long)np * w;      // first cost unit of tier k
+                if (!np) continue;
+                if (lo <= Wk + (np - 1) * w) pb = m_P[k] + (uint32_t)(lo > Wk ? (lo - Wk + w - 1) / w : 0);
+                if (hi <= Wk + (np - 1) * w) pe = m_P[k] + (uint32_t)(hi > Wk ? (hi - Wk + w - 1) / w : 0);
+            }
+            m_misc[0] = pb;
+            m_misc[1] = pe > pb ? pe : pb;
+            mbar_arrive(table_bar);
+        }
+        __syncwarp();
+        const uint32_t p_begin = m_misc[0], p_end = m_misc[1];
+        const uint32_t npages = p_end - p_begin;
+        const size_t pbase = page_index(G, seq, C.g, h, 0);
+        // The warp resolves 32 pages at a time (global page ids, byte counts) into a small
+        // table; lane 0 then issues the copies back to back with a running stage / phase.
+        uint32_t* t_src = reinterpret_cast<uint32_t*>(smem + L.misc + 1024);    // [32] pool units
+        uint32_t* t_len = t_src + 32;                                           // [32] bytes
+        uint32_t st = 0, ph = 0;
+        bool ok = true;
+        for (uint32_t b0 = 0; b0 < npages && ok; b0 += 32) {
+            const uint32_t u = b0 + lane;
+            if (u < npages) {
+                const uint32_t p = p_begin + u;
+                int k = 0;
+#pragma unroll
+                for (int kk = 1; kk < kMaxTiers; ++kk)
+                    if (kk < G.ntiers && p >= m_P[kk]) k = kk;
+                t_src[lane] = __ldcg(St.pages + pbase + (size_t)k * G.max_pages + (p - m_P[k]));
+                t_len[lane] = m_chunk[k];
+            }
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t nb = min(32u, npages - b0);
+                for (uint32_t j = 0; j < nb; ++j) {
+                    // stage st is being reused once the pages have wrapped around the ring
+                    if (b0 + j >= (uint32_t)NS && !mbar_wait(empty0 + 8 * st, ph ^ 1u)) {
+                        set_dev_error(St, 6u /*DWKV_DEV_TIMEOUT*/, (uint32_t)seq, b0 + j);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bytes = t_len[j];
+                    mbar_arrive_expect_tx(full0 + 8 * st, bytes);
+                    bulk_g2s(smem_addr(smem + L.stages + (size_t)st * G.stage_bytes),
+                             St.data + (size_t)t_src[j] * kUnit + (size_t)C.lig * bytes, bytes, full0 + 8 * st);
+                    if (++st == (uint32_t)NS) { st = 0; ph ^= 1u; }
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            __syncwarp();
+        }
+    } else {
+        // ================= consumer warps
+        uint8_t* rd = smem + L.rd + warp * kRdBytes;
+        uint8_t* small = smem + L.small + warp * L.small_stride;
+        const uint32_t zero_addr = smem_addr(smem + L.zero);
+        const float qscale = G.tau * kLog2e;
+        if (tid < kD) {
+            const __nv_bfloat16* q = C.q + ((size_t)ci * G.Hq + (size_t)h * kGQ) * kD + tid;
+            qs[tid] = make_float4(__bfloat162float(q[0]) * qscale, __bfloat162float(q[kD]) * qscale,
+                                  __bfloat162float(q[2 * kD]) * qscale, __bfloat162float(q[3 * kD]) * qscale);
+        }
+        if (tid < 8) reinterpret_cast<uint4*>(smem + L.zero)[tid] = make_uint4(0u, 0u, 0u, 0u);
+        named_barrier(1, kConsumerWarps * 32);
+        bool ok = mbar_wait(basis_bar, 0);
+        if (!ok && lane == 0) set_dev_error(St, 6u, (uint32_t)seq, 0xffffffffu);
+        // q~[j] = sum_i B_K[i][j] q[i]: the 256 consumer threads split the rows into
+        // np = 256 / rq parts (a warp reads one row at a time: conflict-free); the parts
+        // are summed through the small buffers.
+        const int rq = G.r_max < 16 ? 16 : G.r_max;
+        {
+            const int np = (kConsumerWarps * 32) / rq, j = tid % rq, part = tid / rq, rows = kD / np;
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (ok && j < G.r_max) {
+                const __nv_bfloat16* bk = reinterpret_cast<const __nv_bfloat16*>(smem + L.rd) + j;
+#pragma unroll 8
+                for (int i = part * rows; i < (part + 1) * rows; ++i) {
+                    const float b = __bfloat162float(bk[i * G.r_max]);
+                    const float4 q = qs[i];
+                    a.x = fmaf(b, q.x, a.x); a.y = fmaf(b, q.y, a.y);
+                    a.z = fmaf(b, q.z, a.z); a.w = fmaf(b, q.w, a.w);
+                }
+            }
+            float4* parts = reinterpret_cast<float4*>(smem + L.small);     // [np][rq]
+            parts[part * rq + j] = a;
+            named_barrier(1, kConsumerWarps * 32);
+            if (tid < rq) {
+                float4 t4 = parts[tid];
+                for (int q2 = 1; q2 < np; ++q2) {
+                    const float4 u = parts[q2 * rq + tid];
+                    t4.x += u.x; t4.y += u.y; t4.z += u.z; t4.w += u.w;
+                }
+                qt[tid] = t4;
+            }
+        }
+        named_barrier(1, kConsumerWarps * 32);
+        // q~ as the MMA B operand: column n < 4 = bf16 hi of head n, n >= 4 = lo of head n-4
+        uint32_t qb[RMAX / 16][2];
+        {
+            const int g = lane >> 2, c = lane & 3, n = g & 3;
+            const bool lo_half = g >= 4;
+#pragma unroll
+            for (int ks = 0; ks < RMAX / 16; ++ks) {
+#pragma unroll
+                for (int r2 = 0; r2 < 2; ++r2) {
+                    uint32_t pk = 0;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int k = 16 * ks + 8 * r2 + 2 * c + e;
+                        float v = 0.f;
+                        if (k < rq) {
+                            const float4 t4 = qt[k];
+                            v = n == 0 ? t4.x : n == 1 ? t4.y : n == 2 ? t4.z : t4.w;
+                        }
+                        uint32_t hi, lo;
+                        split_bf16_rn(v, hi, lo);
+                        pk |= (lo_half ? lo : hi) << (16 * e);
+                    }
+                    qb[ks][r2] = pk;
+                }
+            }
+        }
+        {   // the residual tiles held B_K until now; clear this warp's tile
+            uint4* z = reinterpret_cast<uint4*>(rd);
+            for (int i = lane; i < kRdBytes / 16; i += 32) z[i] = make_uint4(0u, 0u, 0u, 0u);
+            __syncwarp();
+        }
+
+        WarpAcc<RMAX, PROBE> A;
+#pragma unroll
+        for (int i = 0; i < RMAX / 16; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) A.c[i][e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < (PROBE ? RMAX / 16 : 1); ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) A.c2[i][e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) A.r[i][e] = 0.f;
+#pragma unroll
+        for (int hh = 0; hh < kGQ; ++hh) { A.m[hh] = -INFINITY; A.l[hh] = 0.f; A.m2[hh] = -INFINITY; A.l2[hh] = 0.f; }
+
+        if (ok && !mbar_wait(table_bar, 0)) {
+            if (lane == 0) set_dev_error(St, 6u, (uint32_t)seq, 0xfffffffeu);
+            ok = false;
+        }
+        const uint32_t p_begin = m_misc[0], p_end = m_misc[1];
+        const int pair = warp >> 1, half = warp & 1;
+        for (uint32_t u = pair; ok && p_begin + u < p_end; u += kPairs) {
+            const uint32_t p = p_begin + u, st = u % NS;
+            int k = 0;
+            while (k + 1 < G.ntiers && p >= m_P[k + 1]) ++k;
+            const int R = (int)m_R[k];
+            const uint32_t pit = p - m_P[k], npk = m_P[k + 1] - m_P[k];
+            const int nvalid = pit + 1 < npk ? kPage : (int)(m_cnt[k] - pit * kPage);
+            if (!mbar_wait(full0 + 8 * st, (u / NS) & 1)) {
+                if (lane == 0) set_dev_error(St, 6u, (uint32_t)seq, u);
+                ok = false;
+                break;
+            }
+            const int nv = min(max(nvalid - 32 * half, 0), 32);
+            if (nv > 0)
+                run_page<S, BITS, PROBE, RMAX>(R, smem + L.stages + (size_t)st * G.stage_bytes, half, nv, qb, qs,
+                                               small, rd, zero_addr, A, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty0 + 8 * st);
+        }
+        // ---- per-warp results: acc_c [r_max][4] and acc_r [d][4] into the residual tile,
+        //      the probe's acc_c2 into the small buffers; m / l into m_state
+        float* oc = reinterpret_cast<float*>(rd);
+        float* orr = oc + G.r_max * 4;
+        store_d(A.c, oc, G.r_max, lane);
+        store_d(A.r, orr, kD, lane);
+        if (PROBE) store_d(A.c2, reinterpret_cast<float*>(small), G.r_max, lane);
+        float* ms = m_state + warp * 16;
+#pragma unroll
+        for (int hh = 0; hh < kGQ; ++hh) {
+            const float l = warp_sum(A.l[hh]);
+            const float l2 = PROBE ? warp_sum(A.l2[hh]) : 0.f;
+            if (lane == 0) {
+                ms[hh] = A.m[hh]; ms[4 + hh] = l;
+                ms[8 + hh] = A.m2[hh]; ms[12 + hh] = l2;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ================= CTA merge: the 8 warp states -> one partial record
+    //   {M[4], L[4], (M2[4], L2[4]), o[4][d] = B_V acc_c + acc_r, (o2[4][d] = B_V acc_c2)}
+    // B_V is applied here, once per CTA, so the final merge is a weighted sum.
+    const int nrec = C.total_splits;
+    float* rec = C.ws + ((size_t)h * nrec + blockIdx.x) * C.rec_floats;
+    const int hdr = PROBE ? 16 : 8;
+    constexpr int kRowVec = RMAX / 8;
+    const int gi = tid & (kD - 1), ghp = tid >> 7;       // channel and head pair of threads < 2d
+    uint4 bv[kRowVec];                                  // row gi of B_V, requested early
+    if (tid < 2 * kD) {
+        const uint4* row = reinterpret_cast<const uint4*>(St.basis_v + basis_off + (size_t)gi * G.r_max);
+#pragma unroll
+        for (int v = 0; v < kRowVec; ++v) bv[v] = v * 8 < G.r_max ? __ldcg(row + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (tid < 2 * kGQ) {
+        const int which = tid / kGQ, hh = tid % kGQ;
+        if (which == 0 || PROBE) {
+            float M = -INFINITY;
+            for (int w2 = 0; w2 < kConsumerWarps; ++w2) M = fmaxf(M, m_state[w2 * 16 + which * 8 + hh]);
+            float Lsum = 0.f;
+            for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
+                const float mw = m_state[w2 * 16 + which * 8 + hh];
+                const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+                mf[which * 32 + w2 * 4 + hh] = f;
+                Lsum += f * m_state[w2 * 16 + which * 8 + 4 + hh];
+            }
+            rec[which * 8 + hh] = M;
+            rec[which * 8 + 4 + hh] = Lsum;
+        }
+    }
+    __syncthreads();
+    float* cm = reinterpret_cast<float*>(smem + L.stages);          // [(PROBE ? 2 : 1)][4][r_max]
+    for (int e = tid; e < kGQ * G.r_max; e += blockDim.x) {
+        const int hh = e / G.r_max, j = e % G.r_max;
+        float v = 0.f, v2 = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
+            v = fmaf(mf[w2 * 4 + hh], reinterpret_cast<const float*>(smem + L.rd + w2 * kRdBytes)[j * 4 + hh], v);
+            if (PROBE)
+                v2 = fmaf(mf[32 + w2 * 4 + hh],
+                          reinterpret_cast<const float*>(smem + L.small + w2 * L.small_stride)[j * 4 + hh], v2);
+        }
+        cm[e] = v;
+        if (PROBE) cm[kGQ * G.r_max + e] = v2;
+    }
+    __syncthreads();
+    if (tid < 2 * kD) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int hh = 2 * ghp + q;
+            const float* c1 = cm + hh * G.r_max;
+            const float* c2 = cm + kGQ * G.r_max + hh * G.r_max;
+            float a = 0.f, a2 = 0.f;
+#pragma unroll
+            for (int v = 0; v < kRowVec; ++v) {
+                if (v * 8 >= G.r_max) break;
+                const uint32_t w[4] = {bv[v].x, bv[v].y, bv[v].z, bv[v].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = v * 8 + 2 * e;
+                    a = fmaf(bf16lo(w[e]), c1[j], a);
+                    a = fmaf(bf16hi(w[e]), c1[j + 1], a);
+                    if (PROBE) {
+                        a2 = fmaf(bf16lo(w[e]), c2[j], a2);
+                        a2 = fmaf(bf16hi(w[e]), c2[j + 1], a2);
+                    }
+                }
+            }
+            float r = 0.f;
+#pragma unroll
+            for (int w2 = 0; w2 < kConsumerWarps; ++w2)
+                r = fmaf(mf[w2 * 4 + hh],
+                         reinterpret_cast<const float*>(smem + L.rd + w2 * kRdBytes)[G.r_max * 4 + gi * 4 + hh], r);
+            rec[hdr + hh * kD + gi] = a + r;
+            if (PROBE) rec[hdr + kGQ * kD + hh * kD + gi] = a2;
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const uint32_t t = atomicAdd(&St.tickets[(size_t)seq * G.Hkv + h], 1u);
+        m_misc[2] = (t == (uint32_t)(nsplit - 1)) ? 1u : 0u;
+    }
+    __syncthreads();
+    if (!m_misc[2]) return;
+    __threadfence();
+
+    // ================= last CTA of (sequence, kv-head): log-sum-exp merge of the records.
+    // Headers and record bodies are staged into shared memory with cp.async (every request
+    // in flight at once; the pipeline buffers are idle now), then summed from there.
+    const int r0 = C.split_begin[ci];
+    const int RF = C.rec_floats;
+    const float* recs = C.ws + ((size_t)h * nrec + r0) * RF;
+    float* hdrs = reinterpret_cast<float*>(smem + L.small);                       // [nsplit][16]
+    float* wgt = hdrs + kMaxSplits * 16;                                           // [2][kMaxSplits][4]
+    float* Ls = wgt + 2 * kMaxSplits * kGQ;                                        // [2][4]
+    float* red = Ls + 8;                                                           // [2][threads]
+    float* stage_f = reinterpret_cast<float*>(smem + L.stages);
+    const size_t stage_floats = (size_t)NS * G.stage_bytes / 4;
+    const int per_chunk = (int)max((size_t)1, min((size_t)nsplit, stage_floats / (size_t)RF));
+    {
+        for (int i = tid; i < nsplit * 4; i += blockDim.x) {
+            const int j = i >> 2, q4 = i & 3;
+            if (q4 * 4 < hdr) cp_async16(smem_addr(hdrs + j * 16 + q4 * 4), recs + (size_t)j * RF + q4 * 4);
+        }
+        const int n0 = per_chunk * RF / 4;         // first chunk of records
+        for (int i = tid; i < n0; i += blockDim.x) cp_async16(smem_addr(stage_f) + 16 * i, recs + 4 * i);
+        cp_async_wait_all();
+    }
+    __syncthreads();
+    if (tid < 2 * kGQ) {
+        const int which = tid / kGQ, hh = tid % kGQ;
+        if (which == 0 || PROBE) {
+            float M = -INFINITY;
+            for (int j = 0; j < nsplit; ++j) M = fmaxf(M, hdrs[j * 16 + which * 8 + hh]);
+            float Lsum = 0.f;
+            for (int j = 0; j < nsplit; ++j) {
+                const float mj = hdrs[j * 16 + which * 8 + hh];
+                const float f = mj == -INFINITY ? 0.f : exp2f(mj - M);
+                wgt[(which * kMaxSplits + j) * kGQ + hh] = f;
+                Lsum = fmaf(f, hdrs[j * 16 + which * 8 + 4 + hh], Lsum);
+            }
+            Ls[which * 4 + hh] = Lsum;
+        }
+    }
+    __syncthreads();
+    // thread -> output elements q = (head, channel); full and (probe) no-residual sums
+    constexpr int kPer = 2;                        // ceil(4 * 128 / 288)
+    float acc1[kPer], acc2[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) { acc1[k] = 0.f; acc2[k] = 0.f; }
+    for (int j0 = 0; j0 < nsplit; j0 += per_chunk) {
+        const int nj = min(per_chunk, nsplit - j0);
+        if (j0 > 0) {
+            __syncthreads();
+            for (int i = tid; i < nj * RF / 4; i += blockDim.x)
+                cp_async16(smem_addr(stage_f) + 16 * i, recs + (size_t)j0 * RF + 4 * i);
+            cp_async_wait_all();
+            __syncthreads();
+        }
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int q = tid + k * (int)blockDim.x;
+            if (q < kGQ * kD) {
+                const int hh = q / kD;
+                const float* w1 = wgt + hh;
+                const float* w2 = wgt + kMaxSplits * kGQ + hh;
+                float a = acc1[k], b = acc2[k];
+                for (int j = 0; j < nj; ++j) {
+                    a = fmaf(w1[(j0 + j) * kGQ], stage_f[(size_t)j * RF + hdr + q], a);
+                    if (PROBE) b = fmaf(w2[(j0 + j) * kGQ], stage_f[(size_t)j * RF + hdr + kGQ * kD + q], b);
+                }
+                acc1[k] = a;
+                acc2[k] = b;
+            }
+        }
+    }
+    float dn = 0.f, nn = 0.f;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int q = tid + k * (int)blockDim.x;
+        if (q < kGQ * kD) {
+            const int hh = q / kD, i = q % kD;
+            const float L1 = Ls[hh];
+            const float o = L1 > 0.f ? acc1[k] / L1 : 0.f;
+            const size_t oi = ((size_t)ci * G.Hq + (size_t)h * kGQ + hh) * kD + i;
+            if (!PROBE) {
+                C.out[oi] = o;
+            } else {
+                const float L2 = Ls[4 + hh];
+                const float o2 = L2 > 0.f ? acc2[k] / L2 : 0.f;
+                if (C.out_full) C.out_full[oi] = o;
+                dn += (o - o2) * (o - o2);
+                nn += o * o;
+            }
+        }
+    }
+    if (PROBE) {
+        red[tid] = dn;
+        red[kDecodeThreads + tid] = nn;
+        __syncthreads();
+        if (tid == 0) {
+            float a = 0.f, b = 0.f;
+            for (int t = 0; t < (int)blockDim.x; ++t) { a += red[t]; b += red[kDecodeThreads + t]; }
+            C.err[(size_t)ci * G.Hkv + h] = sqrtf(a) / (sqrtf(b) + 1e-6f);
+        }
+    }
+    if (tid == 0) St.tickets[(size_t)seq * G.Hkv + h] = 0u;
+}
+
+}  // namespace dwkv
+
+// Explicit instantiations for one (BITS, PROBE) pair: RMAX in {64, 128}, S in {0, 8, 16, 32}.
+#define DWKV_DECODE_INSTANTIATE(B, P)                                                        \
+    namespace dwkv {                                                                          \
+    template __global__ void decode_kernel<B, P, 64, 0>(const Geom, const State, const DecodeCall);   \
+    template __global__ void decode_kernel<B, P, 64, 8>(const Geom, const State, const DecodeCall);   \
+    template __global__ void decode_kernel<B, P, 64, 16>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 64, 32>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 128, 0>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 128, 8>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 128, 16>(const Geom, const State, const DecodeCall); \
+    template __global__ void decode_kernel<B, P, 128, 32>(const Geom, const State, const DecodeCall); \
+    }

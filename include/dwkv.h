@@ -81,8 +81,9 @@ typedef enum {
 
 /* Cache geometry.  Supported by this build: head_dim == 128; num_q_heads == 4 *
  * num_kv_heads; tiers drawn from {8, 16, 32, 64, 128}, strictly ascending, each <= r_max;
- * r_max in {8, 16, 32, 64, 128}; resid_channels s a multiple of 8 with 0 <= s <= 128;
- * resid_bits 8 or 4; num_layers a multiple of layers_per_group. */
+ * r_max in {8, 16, 32, 64, 128}; resid_channels s in {0, 8, 16, 32} ([DW] §3 routes at most
+ * 8 residual channels per token; s is fixed per cache here); resid_bits 8 or 4; num_layers
+ * a multiple of layers_per_group. */
 typedef struct {
     int32_t num_layers;        /* L                                                     */
     int32_t layers_per_group;  /* w: adjacent layers sharing one basis ([DW] §3)        */

@@ -45,7 +45,7 @@ def test_workload_configs_are_supported(name):
 @pytest.mark.parametrize("over,status", [
     (dict(num_layers=3), 1), (dict(head_dim=64), 5), (dict(num_q_heads=16), 5), (dict(r_max=12), 1),
     (dict(r_max=48, tiers=(16, 32)), 5), (dict(tiers=(16, 16)), 1), (dict(tiers=(8, 24)), 5), (dict(tiers=(16, 128)), 1),
-    (dict(resid_channels=12), 1), (dict(resid_bits=2), 1), (dict(max_batch=0), 1),
+    (dict(resid_channels=12), 1), (dict(resid_channels=24), 5), (dict(resid_bits=2), 1), (dict(max_batch=0), 1),
     (dict(max_context=1 << 24), 1),
 ])
 def test_invalid_configs_are_rejected(over, status):
