@@ -21,7 +21,7 @@ __all__ = [
     "dwkv_arena_bytes", "dwkv_workspace_bytes", "dwkv_create", "dwkv_destroy",
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage",
-    "dwkv_sync_status", "dwkv_set_decode_tuning", "Cache", "EXPORTED_SYMBOLS",
+    "dwkv_sync_status", "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "Cache", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -36,7 +36,7 @@ EXPORTED_SYMBOLS = (
     "dwkv_metadata_bytes", "dwkv_arena_bytes", "dwkv_workspace_bytes", "dwkv_create", "dwkv_destroy",
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage", "dwkv_sync_status",
-    "dwkv_set_decode_tuning",
+    "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc",
 )
 
 
@@ -95,6 +95,7 @@ def lib():
             "dwkv_pool_usage": ([vp, vp, C.POINTER(dwkv_pool_stats)], C.c_int),
             "dwkv_sync_status": ([vp, vp], C.c_int),
             "dwkv_set_decode_tuning": ([vp, i32, i32, i32], C.c_int),
+            "dwkv_decode_attention_noalloc": ([vp, i32, i32, vp, vp, vp, vp], C.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -214,6 +215,11 @@ def dwkv_decode_attention(h, layer, seq_ids, q, out, workspace, stream=None):
     _check(lib().dwkv_decode_attention(h, layer, len(seq_ids), _i32(seq_ids), _ptr(q), _ptr(out),
                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _stream(stream)))
+
+
+def dwkv_decode_attention_noalloc(h, layer, seq_ids, q, out, stream=None):
+    _check(lib().dwkv_decode_attention_noalloc(h, layer, len(seq_ids), _i32(seq_ids), _ptr(q), _ptr(out),
+                                               _stream(stream)))
 
 
 def dwkv_probe(h, layer, seq_ids, q, err, out_full, workspace, stream=None):

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -706,3 +707,60 @@ dwkv_status dwkv_sync_status(dwkv_handle h, void* stream) {
 }
 
 }  // extern "C"
+
+// ============================================================ decode without allocation
+// Some callers cannot hand this library any device memory at decode time: plugin hooks of
+// an inference engine that run inside the engine's own enqueue path, or serving loops whose
+// device memory is entirely reserved by their own pool up front.  For them cudaMalloc is not
+// an option (it can synchronise the device, and fails once the pool holds all memory), and
+// they may have no workspace buffer to lend.  dwkv_decode_attention_noalloc runs the same
+// decode with a fixed scratch area that is part of the library image itself.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 8u << 20;   // 8 MiB, held by every GPU that loads the library
+constexpr int kNoAllocMaxDevices = 64;
+
+// Split-K partial records of dwkv_decode_attention_noalloc.  Every call on a device uses
+// this same array, so calls that overlap on the GPU race on it.  Nothing in it has to start
+// at zero: each CTA writes its record before any CTA reads it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+extern "C" dwkv_status dwkv_decode_attention_noalloc(dwkv_handle h, int32_t layer, int32_t n_seqs,
+                                                     const int32_t* seq_ids, const void* q, float* out,
+                                                     void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if (n_seqs < 0 || n_seqs > kMaxSeqs)
+        return fail(DWKV_ERR_INVALID_ARG, "n_seqs %d out of [0, %d]", n_seqs, kMaxSeqs);
+    const size_t need = dwkv_workspace_bytes(&h->cfg, n_seqs);
+    if (need > kNoAllocScratchBytes)
+        return fail(DWKV_ERR_CAPACITY,
+                    "dwkv_decode_attention_noalloc: %d sequences need %zu bytes of scratch but the built-in "
+                    "scratch holds %zu; decode fewer sequences per call or use dwkv_decode_attention with a "
+                    "workspace", n_seqs, need, kNoAllocScratchBytes);
+    int dev = -1;
+    DWKV_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev != h->device)
+        return fail(DWKV_ERR_INVALID_ARG, "the handle's device %d must be current (current is %d)", h->device, dev);
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return fail(DWKV_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kNoAllocMaxDevices - 1);
+    void* scratch = nullptr;
+    {
+        // First call on a device: resolve the device address of the scratch array.  The host
+        // name g_noalloc_scratch is only a stand-in; kernels must get this address instead.
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void* ptr = nullptr;
+            const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+            g_noalloc_ptr[dev] = ptr;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    return dwkv_decode_attention(h, layer, n_seqs, seq_ids, q, out, scratch, kNoAllocScratchBytes, stream);
+}

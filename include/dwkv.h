@@ -221,6 +221,24 @@ dwkv_status dwkv_sync_status(dwkv_handle h, void* stream);
 dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t waves,
                                    int32_t stages);
 
+/* Decode attention without any caller-provided or library-allocated memory: the same
+ * operation as dwkv_decode_attention, but its split-K scratch is a fixed 8 MiB array built
+ * into the library (held by every GPU that loads the library until the process exits).
+ * There is no counterpart in [DW]; it exists for callers that cannot allocate device memory
+ * when they decode (engine plugin hooks, serving loops whose memory pool owns all of HBM) and
+ * have no workspace to lend.  Arguments as dwkv_decode_attention without the workspace.
+ *  - Calls nothing that allocates (no cudaMalloc / cudaFree).
+ *  - Returns DWKV_ERR_CAPACITY when dwkv_workspace_bytes(cfg, n_seqs) exceeds 8 MiB
+ *    (for 8 kv-heads and head_dim 128: up to 3 sequences per call).
+ *  - The first call on a device resolves the scratch array's device address (one
+ *    cudaGetSymbolAddress); make that first call before any stream capture.  The handle's
+ *    device must be current.
+ *  - All calls on a device share the one array: calls that overlap on the GPU (other
+ *    streams, other handles) race on it.  Nothing in it needs clearing between calls. */
+dwkv_status dwkv_decode_attention_noalloc(dwkv_handle h, int32_t layer, int32_t n_seqs,
+                                          const int32_t* seq_ids, const void* q, float* out,
+                                          void* stream);
+
 #ifdef __cplusplus
 }
 #endif
