@@ -113,7 +113,7 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 //   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W[32][8] bf16, P2[32][8]
 //   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  zero line
 struct DecodeSmem {
-    uint32_t stages, rd, small, small_stride, S, P, W, P2, qt, q, zero, bars, misc, total;
+    uint32_t stages, rd, small, small_stride, S, P, W, P2, qt, q, qh, zero, bars, misc, total;
 };
 __host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, int NS, bool probe) {
     DecodeSmem L;
@@ -129,6 +129,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, int NS, 
     L.small = o;   o += kConsumerWarps * w;
     L.qt = o;      o += (uint32_t)(G.r_max < 16 ? 16 : G.r_max) * 16;
     L.q = o;       o += (uint32_t)G.d * 16;
+    L.qh = o;      o += (uint32_t)G.d * 8;
     L.zero = o;    o += 128;
     L.bars = o;    o += (2 * NS + 2) * 8;
     L.misc = o;    o += 1536;

@@ -129,9 +129,9 @@ constexpr uint32_t kRdPitch = 48;
 // `nv` of them live.  `K` points at the page chunk's key block.
 template <int R, int S, int BITS, bool PROBE, int RMAX>
 __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int half, int nv,
-                                          const uint32_t (&qb)[RMAX / 16][2], const float4* __restrict__ qs,
-                                          uint8_t* small, uint8_t* rd, uint32_t zero_addr, WarpAcc<RMAX, PROBE>& A,
-                                          int lane) {
+                                          const uint32_t (&qb)[RMAX / 16][2], const uint2* __restrict__ qh,
+                                          float qscale, uint8_t* small, uint8_t* rd, uint32_t zero_addr,
+                                          WarpAcc<RMAX, PROBE>& A, int lane) {
     constexpr int KS = R >= 16 ? R / 16 : 1;         // 16-wide coefficient steps
     constexpr uint32_t kOffIdx = 128u * R, kOffCodes = kOffIdx + 64u * S, kOffSc = kOffCodes + 8u * S * BITS;
     constexpr uint32_t kBlk = kOffSc + 128u;
@@ -200,14 +200,15 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 for (int e = 0; e < 8; ++e) {
                     const uint32_t i = ((e < 4 ? ix.x : ix.y) >> (8 * (e & 3))) & 0xffu;
                     const float cf = BITS == 8 ? code8(e < 4 ? cw0 : cw1, e & 3) : code4(cw0, e);
-                    const float4 q = qs[i];
-                    ra[0] = fmaf(q.x, cf, ra[0]);
-                    ra[1] = fmaf(q.y, cf, ra[1]);
-                    ra[2] = fmaf(q.z, cf, ra[2]);
-                    ra[3] = fmaf(q.w, cf, ra[3]);
+                    const uint2 q = qh[i];                // the 4 heads' q_i as bf16 (exact)
+                    ra[0] = fmaf(bf16lo(q.x), cf, ra[0]);
+                    ra[1] = fmaf(bf16hi(q.x), cf, ra[1]);
+                    ra[2] = fmaf(bf16lo(q.y), cf, ra[2]);
+                    ra[3] = fmaf(bf16hi(q.y), cf, ra[3]);
                 }
             }
-            const float scale = S ? __half2float(*reinterpret_cast<const __half*>(K + kOffSc + t * 2)) : 0.f;
+            const float scale =
+                S ? __half2float(*reinterpret_cast<const __half*>(K + kOffSc + t * 2)) * qscale : 0.f;
             sc[0] = fmaf(scale, ra[0], sv.x);
             sc[1] = fmaf(scale, ra[1], sv.y);
             sc[2] = fmaf(scale, ra[2], sv.z);
@@ -315,13 +316,15 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
             const int tl = 16 * ks + (lane & 15);       // token within the half
+            constexpr int kHalfS = S / 2;               // entries per lane (two lanes per token)
+            uint32_t ixw[kHalfS >= 4 ? kHalfS / 4 : 1];  // this lane's channels, kept to clear them
             if (tl < nv) {
                 const int tok = tb + tl;
-                constexpr int kHalfS = S / 2;           // entries per lane (two lanes per token)
                 const int e0 = (lane >> 4) * kHalfS;
 #pragma unroll
                 for (int e = 0; e < kHalfS; e += 4) {
                     const uint32_t ix = *reinterpret_cast<const uint32_t*>(V + kOffIdx + tok * S + e0 + e);
+                    ixw[e / 4] = ix;
                     uint32_t cw;
                     if (BITS == 8) cw = *reinterpret_cast<const uint32_t*>(V + kOffCodes + tok * S + e0 + e);
                     else cw = *reinterpret_cast<const uint16_t*>(V + kOffCodes + tok * (S / 2) + (e0 + e) / 2);
@@ -344,10 +347,12 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 mma_bf16(A.r[mt], a, b);
             }
             __syncwarp();
+            if (tl < nv) {                              // clear exactly what this lane wrote
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {               // clear the 128 x 32 data bytes
-                const uint32_t k = lane + 32 * i;
-                *reinterpret_cast<uint4*>(rd + (k >> 1) * kRdPitch + (k & 1) * 16) = make_uint4(0u, 0u, 0u, 0u);
+                for (int w = 0; w < kHalfS / 4; ++w)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint16_t*>(rd + ((ixw[w] >> (8 * q)) & 0xffu) * kRdPitch + my_col) = 0;
             }
             __syncwarp();
         }
@@ -356,15 +361,15 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
 
 template <int S, int BITS, bool PROBE, int RMAX>
 __device__ __forceinline__ void run_page(int R, const uint8_t* K, int half, int nv, const uint32_t (&qb)[RMAX / 16][2],
-                                         const float4* qs, uint8_t* small, uint8_t* rd, uint32_t zero_addr,
+                                         const uint2* qs, float qscale, uint8_t* small, uint8_t* rd, uint32_t zero_addr,
                                          WarpAcc<RMAX, PROBE>& A, int lane) {
     switch (R) {
-        case 8: half_page<8, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane); break;
-        case 16: half_page<16, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane); break;
-        case 32: half_page<32, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane); break;
-        case 64: half_page<64, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane); break;
+        case 8: half_page<8, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane); break;
+        case 16: half_page<16, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane); break;
+        case 32: half_page<32, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane); break;
+        case 64: half_page<64, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane); break;
         case 128:
-            if constexpr (RMAX >= 128) half_page<128, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, small, rd, zero_addr, A, lane);
+            if constexpr (RMAX >= 128) half_page<128, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane);
             break;
         default: break;
     }
@@ -528,10 +533,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         uint8_t* small = smem + L.small + warp * L.small_stride;
         const uint32_t zero_addr = smem_addr(smem + L.zero);
         const float qscale = G.tau * kLog2e;
+        uint2* qh = reinterpret_cast<uint2*>(smem + L.qh);
         if (tid < kD) {
             const __nv_bfloat16* q = C.q + ((size_t)ci * G.Hq + (size_t)h * kGQ) * kD + tid;
-            qs[tid] = make_float4(__bfloat162float(q[0]) * qscale, __bfloat162float(q[kD]) * qscale,
-                                  __bfloat162float(q[2 * kD]) * qscale, __bfloat162float(q[3 * kD]) * qscale);
+            const __nv_bfloat16 q0 = q[0], q1 = q[kD], q2 = q[2 * kD], q3 = q[3 * kD];
+            qs[tid] = make_float4(__bfloat162float(q0) * qscale, __bfloat162float(q1) * qscale,
+                                  __bfloat162float(q2) * qscale, __bfloat162float(q3) * qscale);
+            qh[tid] = make_uint2((uint32_t)__bfloat16_as_ushort(q0) | ((uint32_t)__bfloat16_as_ushort(q1) << 16),
+                                 (uint32_t)__bfloat16_as_ushort(q2) | ((uint32_t)__bfloat16_as_ushort(q3) << 16));
         }
         if (tid < 8) reinterpret_cast<uint4*>(smem + L.zero)[tid] = make_uint4(0u, 0u, 0u, 0u);
         named_barrier(1, kConsumerWarps * 32);
@@ -635,8 +644,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             }
             const int nv = min(max(nvalid - 32 * half, 0), 32);
             if (nv > 0)
-                run_page<S, BITS, PROBE, RMAX>(R, smem + L.stages + (size_t)st * G.stage_bytes, half, nv, qb, qs,
-                                               small, rd, zero_addr, A, lane);
+                run_page<S, BITS, PROBE, RMAX>(R, smem + L.stages + (size_t)st * G.stage_bytes, half, nv, qb, qh,
+                                               qscale, small, rd, zero_addr, A, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8 * st);
         }
