@@ -36,7 +36,7 @@ constexpr int kMaxSplits = 64;     // decode splits per (sequence, kv-head)
 constexpr int kConsumerWarps = 8;  // 4 pairs; a pair shares one page (32 tokens per warp)
 constexpr int kPairs = kConsumerWarps / 2;
 constexpr int kDecodeThreads = 32 * (kConsumerWarps + 1);  // + 1 producer warp
-constexpr int kRdBytes = 128 * 48;                         // dense residual tile: 128 ch x (16 tokens bf16 + pad)
+constexpr int kRdBytes = 128 * 32;                         // dense residual tile: 128 ch x 32 tokens int8
 
 struct Geom {
     int L, LPG, G, Hq, Hkv, d, r_max, ntiers, s, bits, max_batch, max_context, max_pages;

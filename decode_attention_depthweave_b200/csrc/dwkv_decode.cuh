@@ -62,6 +62,15 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// D (16x8 s32) = A (16x32 s8, row) * B (32x8 u8, col) + C
+__device__ __forceinline__ void mma_s8u8(int (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -109,7 +118,7 @@ __device__ __forceinline__ float code4(uint32_t word, int e) {
 template <int RMAX, bool PROBE>
 struct WarpAcc {
     float c[RMAX / 16][4];                 // coefficient-space values, D layout (row j, col n)
-    float r[8][4];                         // residual-space values, D layout (row channel, col n)
+    float r[8][2];                         // residual-space values: channels 16i+g, 16i+g+8 of head c
     float c2[PROBE ? RMAX / 16 : 1][4];    // probe: no-residual coefficient-space values
     float m[kGQ], l[kGQ], m2[kGQ], l2[kGQ];
 };
@@ -121,9 +130,15 @@ __device__ __forceinline__ void rescale_d(float (&d)[N][4], float a0, float a1) 
     for (int i = 0; i < N; ++i) { d[i][0] *= a0; d[i][1] *= a1; d[i][2] *= a0; d[i][3] *= a1; }
 }
 
-// Dense residual tile of one warp: 128 channel rows x 16 tokens (bf16) with a 48-byte row
-// pitch (32 data bytes + 16 pad) -- 8 consecutive rows then hit disjoint banks for ldmatrix.
-constexpr uint32_t kRdPitch = 48;
+// Dense value-residual tile of one warp: 128 channel rows x 32 tokens of int8 codes (zero
+// where a token has no entry).  Row pitch 32 bytes; the two 16-byte halves of a row swap
+// places in rows with bit 2 set, so the 8 rows of every ldmatrix hit disjoint bank groups.
+__device__ __forceinline__ uint32_t rd_off(uint32_t row, uint32_t tok) {
+    return row * 32u + (tok ^ ((row & 4u) << 2));
+}
+// Per-head byte rows of the weight limbs: row n = 2 h + limb, 32 tokens, 48-byte pitch (the
+// eight rows' 4-byte words read by one B-fragment load then fall in distinct banks).
+constexpr uint32_t kWbPitch = 48;
 
 // One warp's half of a tier-R page: tokens [32*half, 32*half + 32) of the page's 64 slots,
 // `nv` of them live.  `K` points at the page chunk's key block.
@@ -217,7 +232,9 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
         }
     }
 
-    // ---------------- 3. online softmax (lazy rescale), p and p * scale^V as bf16 hi/lo rows
+    // ---------------- 3. online softmax (lazy rescale), p as bf16 hi/lo rows, p * scale^V as
+    //                     fixed-point byte limbs
+    float wdq = 0.f;                                   // this lane's head c: value of one limb unit
     {
         // The running max only moves when some score exceeds it by the slack (one vote);
         // otherwise p = exp2(s - m) <= 2^slack stays safe in fp32.
@@ -238,7 +255,9 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
             }
             const float a0 = alpha[(2 * c) & 3], a1 = alpha[(2 * c + 1) & 3];
             rescale_d(A.c, a0, a1);
-            rescale_d(A.r, a0, a1);
+            const float ac = alpha[c];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { A.r[i][0] *= ac; A.r[i][1] *= ac; }
         }
         float p[kGQ];
 #pragma unroll
@@ -251,11 +270,19 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
         split2(p[2], p[3], pr.y, pr.w);
         *reinterpret_cast<uint4*>(Psm + lane * 16) = pr;
         if (S) {
+            // w = p * scale^V as 16-bit fixed point per head, in units of 2^(E-15) with E the
+            // exponent of the half page's largest w: two byte limbs (hi, lo) per head
             const float scv = live ? __half2float(*reinterpret_cast<const __half*>(V + kOffSc + t * 2)) : 0.f;
-            uint4 wr;
-            split2(p[0] * scv, p[1] * scv, wr.x, wr.z);
-            split2(p[2] * scv, p[3] * scv, wr.y, wr.w);
-            *reinterpret_cast<uint4*>(Wsm + lane * 16) = wr;
+#pragma unroll
+            for (int h = 0; h < kGQ; ++h) {
+                const float wv = p[h] * scv;                              // >= 0
+                const uint32_t eb = __reduce_max_sync(0xffffffffu, __float_as_uint(wv) >> 23);
+                uint32_t v = 0;
+                if (eb >= 16u) v = min(__float2uint_rn(wv * __uint_as_float((269u - eb) << 23)), 65535u);
+                Wsm[(2 * h) * kWbPitch + lane] = (uint8_t)(v >> 8);
+                Wsm[(2 * h + 1) * kWbPitch + lane] = (uint8_t)v;
+                if (c == h) wdq = eb >= 16u ? __uint_as_float((eb - 15u) << 23) : 0.f;   // 2^(E-15)
+            }
         }
         if (PROBE) {
             bool over2 = false;
@@ -308,54 +335,47 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
         }
     }
 
-    // ---------------- 5. residual-space values through a dense 128 x 16 code tile
+    // ---------------- 5. residual-space values: acc_r[ch][h] += sum_t R^V[t][ch] w[t][h] as one
+    //                     integer MMA per 16 channels over the half page's 32 tokens
     if (S) {
-        const uint32_t rdaddr = smem_addr(rd), waddr = smem_addr(Wsm);
-        const uint32_t my_col = (uint32_t)(lane & 15) * 2;              // this lane's token column
-        const uint32_t a_off = ((uint32_t)(mi & 1) * 8 + rr) * kRdPitch + (uint32_t)(mi >> 1) * 16;
+        if (lane < nv) {                                // scatter this token's codes (lane = token)
+            const int tok = tb + lane;
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            const int tl = 16 * ks + (lane & 15);       // token within the half
-            constexpr int kHalfS = S / 2;               // entries per lane (two lanes per token)
-            uint32_t ixw[kHalfS >= 4 ? kHalfS / 4 : 1];  // this lane's channels, kept to clear them
-            if (tl < nv) {
-                const int tok = tb + tl;
-                const int e0 = (lane >> 4) * kHalfS;
+            for (int e = 0; e < S; e += 4) {
+                const uint32_t ix = *reinterpret_cast<const uint32_t*>(V + kOffIdx + tok * S + e);
+                uint32_t cw;
+                if (BITS == 8) cw = *reinterpret_cast<const uint32_t*>(V + kOffCodes + tok * S + e);
+                else cw = *reinterpret_cast<const uint16_t*>(V + kOffCodes + tok * (S / 2) + e / 2);
 #pragma unroll
-                for (int e = 0; e < kHalfS; e += 4) {
-                    const uint32_t ix = *reinterpret_cast<const uint32_t*>(V + kOffIdx + tok * S + e0 + e);
-                    ixw[e / 4] = ix;
-                    uint32_t cw;
-                    if (BITS == 8) cw = *reinterpret_cast<const uint32_t*>(V + kOffCodes + tok * S + e0 + e);
-                    else cw = *reinterpret_cast<const uint16_t*>(V + kOffCodes + tok * (S / 2) + (e0 + e) / 2);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t ch = (ix >> (8 * q)) & 0xffu;
-                        const float cf = BITS == 8 ? code8(cw, q) : code4(cw, q);
-                        *reinterpret_cast<uint16_t*>(rd + ch * kRdPitch + my_col) =
-                            (uint16_t)(__float_as_uint(cf) >> 16);      // small integers are exact in bf16
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t ch = (ix >> (8 * q)) & 0xffu;
+                    // the code as a signed byte (int4: sign-extend the nibble)
+                    const uint32_t cb = BITS == 8 ? (cw >> (8 * q)) : (uint32_t)((int32_t)(cw << (28 - 4 * q)) >> 28);
+                    rd[rd_off(ch, (uint32_t)lane)] = (uint8_t)cb;
                 }
             }
-            __syncwarp();
-            uint32_t b[2];
-            ldsm_x2_t(waddr + (16 * ks + (lane & 15)) * 16, b);
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                uint32_t a[4];
-                ldsm_x4(rdaddr + mt * 16 * kRdPitch + a_off, a);
-                mma_bf16(A.r[mt], a, b);
-            }
-            __syncwarp();
-            if (tl < nv) {                              // clear exactly what this lane wrote
-#pragma unroll
-                for (int w = 0; w < kHalfS / 4; ++w)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint16_t*>(rd + ((ixw[w] >> (8 * q)) & 0xffu) * kRdPitch + my_col) = 0;
-            }
-            __syncwarp();
         }
+        __syncwarp();
+        uint32_t b[2];
+        b[0] = *reinterpret_cast<const uint32_t*>(Wsm + g * kWbPitch + 4 * c);
+        b[1] = *reinterpret_cast<const uint32_t*>(Wsm + g * kWbPitch + 16 + 4 * c);
+        const uint32_t rdaddr = smem_addr(rd);
+        const uint32_t arow = (uint32_t)(rr + 8 * (mi & 1));
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            uint32_t a[4];
+            ldsm_x4(rdaddr + rd_off(16u * mt + arow, 16u * (uint32_t)(mi >> 1)), a);
+            int d[4] = {0, 0, 0, 0};
+            mma_s8u8(d, a, b);
+            // |d| <= 32 * 128 * 255, so hi * 256 + lo is exact in int32
+            A.r[mt][0] = fmaf(wdq, (float)(d[0] * 256 + d[1]), A.r[mt][0]);
+            A.r[mt][1] = fmaf(wdq, (float)(d[2] * 256 + d[3]), A.r[mt][1]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i)                     // clear the 4 KB tile for the next half page
+            reinterpret_cast<uint4*>(rd)[lane + 32 * i] = make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
     }
 }
 
@@ -431,6 +451,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     const int seq = C.seq[ci];
     const size_t basis_off = ((size_t)C.g * G.Hkv + h) * kD * G.r_max;
 
+    constexpr int kRowVec = RMAX / 8;
+    const int gi = tid & (kD - 1), ghp = tid >> 7;       // channel and head pair of threads < 2d
+    uint4 bv[kRowVec];                                  // row gi of B_V (consumer threads)
     uint32_t cv[kMaxTiers];                 // tier counts (producer lane 0)
     if (warp == kConsumerWarps && lane == 0) {
         for (int i = 0; i < NS; ++i) {
@@ -439,6 +462,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         }
         mbar_init(basis_bar, 1);
         mbar_init(table_bar, 1);
+        m_misc[3] = 0u;                       // half-page work counter
         fence_mbar_init();
         // B_K into the residual tiles (free until the main loop) and the counts, both in
         // flight across the barrier below
@@ -618,9 +642,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
 #pragma unroll
             for (int e = 0; e < 4; ++e) A.c2[i][e] = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) A.r[i][e] = 0.f;
+        for (int i = 0; i < 8; ++i) { A.r[i][0] = 0.f; A.r[i][1] = 0.f; }
 #pragma unroll
         for (int hh = 0; hh < kGQ; ++hh) { A.m[hh] = -INFINITY; A.l[hh] = 0.f; A.m2[hh] = -INFINITY; A.l2[hh] = 0.f; }
 
@@ -628,10 +650,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             if (lane == 0) set_dev_error(St, 6u, (uint32_t)seq, 0xfffffffeu);
             ok = false;
         }
+        // Work items are half pages, taken in order from a shared counter: item w is half
+        // w & 1 of the CTA's page w >> 1.  Both halves of a page release its stage, so the
+        // stage frees once the second of the two warps is done, whichever warps they are.
         const uint32_t p_begin = m_misc[0], p_end = m_misc[1];
-        const int pair = warp >> 1, half = warp & 1;
-        for (uint32_t u = pair; ok && p_begin + u < p_end; u += kPairs) {
-            const uint32_t p = p_begin + u, st = u % NS;
+        const uint32_t nitems = 2 * (p_end - p_begin);
+        uint32_t* work = m_misc + 3;
+        uint32_t w = 0;
+        if (lane == 0) w = atomicAdd(work, 1u);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        while (ok && w < nitems) {
+            // take the next item now (its latency hides behind this one) unless the run is
+            // nearly over, where an early claim would only unbalance the warps' finish
+            uint32_t wn = 0xffffffffu;
+            if (w + 2 * kConsumerWarps < nitems) {
+                if (lane == 0) wn = atomicAdd(work, 1u);
+                wn = __shfl_sync(0xffffffffu, wn, 0);
+            }
+            const uint32_t u = w >> 1, p = p_begin + u, st = u % NS;
+            const int half = (int)(w & 1);
             int k = 0;
             while (k + 1 < G.ntiers && p >= m_P[k + 1]) ++k;
             const int R = (int)m_R[k];
@@ -648,14 +685,31 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                                                qscale, small, rd, zero_addr, A, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8 * st);
+            if (wn == 0xffffffffu) {
+                if (lane == 0) wn = atomicAdd(work, 1u);
+                wn = __shfl_sync(0xffffffffu, wn, 0);
+            }
+            w = wn;
         }
         // ---- per-warp results: acc_c [r_max][4] and acc_r [d][4] into the residual tile,
         //      the probe's acc_c2 into the small buffers; m / l into m_state
         float* oc = reinterpret_cast<float*>(rd);
         float* orr = oc + G.r_max * 4;
         store_d(A.c, oc, G.r_max, lane);
-        store_d(A.r, orr, kD, lane);
+        {
+            const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                orr[(16 * i + g) * 4 + c] = A.r[i][0];
+                orr[(16 * i + g + 8) * 4 + c] = A.r[i][1];
+            }
+        }
         if (PROBE) store_d(A.c2, reinterpret_cast<float*>(small), G.r_max, lane);
+        {   // B_V row gi for the CTA's GEMV below, requested before waiting for the other warps
+            const uint4* row = reinterpret_cast<const uint4*>(St.basis_v + basis_off + (size_t)gi * G.r_max);
+#pragma unroll
+            for (int v = 0; v < kRowVec; ++v) bv[v] = v * 8 < G.r_max ? __ldcg(row + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
         float* ms = m_state + warp * 16;
 #pragma unroll
         for (int hh = 0; hh < kGQ; ++hh) {
@@ -675,26 +729,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     const int nrec = C.total_splits;
     float* rec = C.ws + ((size_t)h * nrec + blockIdx.x) * C.rec_floats;
     const int hdr = PROBE ? 16 : 8;
-    constexpr int kRowVec = RMAX / 8;
-    const int gi = tid & (kD - 1), ghp = tid >> 7;       // channel and head pair of threads < 2d
-    uint4 bv[kRowVec];                                  // row gi of B_V, requested early
-    if (tid < 2 * kD) {
-        const uint4* row = reinterpret_cast<const uint4*>(St.basis_v + basis_off + (size_t)gi * G.r_max);
+    if (warp < (PROBE ? 2 : 1)) {
+        // lane = (warp w2, head hh): the CTA max and the rescaled sum by shuffles
+        const int which = warp, w2 = lane >> 2, hh = lane & 3;
+        const float m = m_state[w2 * 16 + which * 8 + hh];
+        float M = m;
 #pragma unroll
-        for (int v = 0; v < kRowVec; ++v) bv[v] = v * 8 < G.r_max ? __ldcg(row + v) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (tid < 2 * kGQ) {
-        const int which = tid / kGQ, hh = tid % kGQ;
-        if (which == 0 || PROBE) {
-            float M = -INFINITY;
-            for (int w2 = 0; w2 < kConsumerWarps; ++w2) M = fmaxf(M, m_state[w2 * 16 + which * 8 + hh]);
-            float Lsum = 0.f;
-            for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
-                const float mw = m_state[w2 * 16 + which * 8 + hh];
-                const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                mf[which * 32 + w2 * 4 + hh] = f;
-                Lsum += f * m_state[w2 * 16 + which * 8 + 4 + hh];
-            }
+        for (int o = 4; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float f = m == -INFINITY ? 0.f : exp2f(m - M);
+        mf[which * 32 + w2 * 4 + hh] = f;
+        float Lsum = f * m_state[w2 * 16 + which * 8 + 4 + hh];
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+        if (lane < kGQ) {
             rec[which * 8 + hh] = M;
             rec[which * 8 + 4 + hh] = Lsum;
         }
@@ -721,7 +768,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             const int hh = 2 * ghp + q;
             const float* c1 = cm + hh * G.r_max;
             const float* c2 = cm + kGQ * G.r_max + hh * G.r_max;
-            float a = 0.f, a2 = 0.f;
+            float a = 0.f, a2 = 0.f, b = 0.f, b2 = 0.f;
 #pragma unroll
             for (int v = 0; v < kRowVec; ++v) {
                 if (v * 8 >= G.r_max) break;
@@ -730,13 +777,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                 for (int e = 0; e < 4; ++e) {
                     const int j = v * 8 + 2 * e;
                     a = fmaf(bf16lo(w[e]), c1[j], a);
-                    a = fmaf(bf16hi(w[e]), c1[j + 1], a);
+                    b = fmaf(bf16hi(w[e]), c1[j + 1], b);
                     if (PROBE) {
                         a2 = fmaf(bf16lo(w[e]), c2[j], a2);
-                        a2 = fmaf(bf16hi(w[e]), c2[j + 1], a2);
+                        b2 = fmaf(bf16hi(w[e]), c2[j + 1], b2);
                     }
                 }
             }
+            a += b;
+            a2 += b2;
             float r = 0.f;
 #pragma unroll
             for (int w2 = 0; w2 < kConsumerWarps; ++w2)
@@ -757,79 +806,85 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     __threadfence();
 
     // ================= last CTA of (sequence, kv-head): log-sum-exp merge of the records.
-    // Headers and record bodies are staged into shared memory with cp.async (every request
-    // in flight at once; the pipeline buffers are idle now), then summed from there.
+    // Every thread requests its outputs' values from the first kChunk records at once while
+    // warps 0 (and 1, probe) turn the record headers into weights with shuffles.
     const int r0 = C.split_begin[ci];
     const int RF = C.rec_floats;
     const float* recs = C.ws + ((size_t)h * nrec + r0) * RF;
-    float* hdrs = reinterpret_cast<float*>(smem + L.small);                       // [nsplit][16]
-    float* wgt = hdrs + kMaxSplits * 16;                                           // [2][kMaxSplits][4]
+    float* wgt = reinterpret_cast<float*>(smem + L.small);                        // [2][kMaxSplits][4]
     float* Ls = wgt + 2 * kMaxSplits * kGQ;                                        // [2][4]
-    float* red = Ls + 8;                                                           // [2][threads]
-    float* stage_f = reinterpret_cast<float*>(smem + L.stages);
-    const size_t stage_floats = (size_t)NS * G.stage_bytes / 4;
-    const int per_chunk = (int)max((size_t)1, min((size_t)nsplit, stage_floats / (size_t)RF));
-    {
-        for (int i = tid; i < nsplit * 4; i += blockDim.x) {
-            const int j = i >> 2, q4 = i & 3;
-            if (q4 * 4 < hdr) cp_async16(smem_addr(hdrs + j * 16 + q4 * 4), recs + (size_t)j * RF + q4 * 4);
-        }
-        const int n0 = per_chunk * RF / 4;         // first chunk of records
-        for (int i = tid; i < n0; i += blockDim.x) cp_async16(smem_addr(stage_f) + 16 * i, recs + 4 * i);
-        cp_async_wait_all();
-    }
-    __syncthreads();
-    if (tid < 2 * kGQ) {
-        const int which = tid / kGQ, hh = tid % kGQ;
-        if (which == 0 || PROBE) {
-            float M = -INFINITY;
-            for (int j = 0; j < nsplit; ++j) M = fmaxf(M, hdrs[j * 16 + which * 8 + hh]);
-            float Lsum = 0.f;
-            for (int j = 0; j < nsplit; ++j) {
-                const float mj = hdrs[j * 16 + which * 8 + hh];
-                const float f = mj == -INFINITY ? 0.f : exp2f(mj - M);
-                wgt[(which * kMaxSplits + j) * kGQ + hh] = f;
-                Lsum = fmaf(f, hdrs[j * 16 + which * 8 + 4 + hh], Lsum);
+    float* red = Ls + 8;                                                           // [2][warps]
+    constexpr int kPer = 2;                        // ceil(4 * 128 / 288) outputs per thread
+    constexpr int kChunk = 16;                     // records whose values are held at once
+    float v1[kPer][kChunk], v2[kPer][PROBE ? kChunk : 1];
+    auto load_chunk = [&](int j0) {
+        const int nj = min(kChunk, nsplit - j0);
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int q = tid + k * kDecodeThreads;
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j) {
+                const bool in = q < kGQ * kD && j < nj;
+                v1[k][j] = in ? __ldcg(recs + (size_t)(j0 + j) * RF + hdr + q) : 0.f;
+                if (PROBE) v2[k][j] = in ? __ldcg(recs + (size_t)(j0 + j) * RF + hdr + kGQ * kD + q) : 0.f;
             }
-            Ls[which * 4 + hh] = Lsum;
+        }
+    };
+    load_chunk(0);
+    if (warp < (PROBE ? 2 : 1)) {
+        const int which = warp;
+        float mj[2][kGQ], lj[2][kGQ];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int j = lane + 32 * jj;                 // kMaxSplits = 64
+            float4 m4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY), l4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (j < nsplit) {
+                m4 = __ldcg(reinterpret_cast<const float4*>(recs + (size_t)j * RF + which * 8));
+                l4 = __ldcg(reinterpret_cast<const float4*>(recs + (size_t)j * RF + which * 8 + 4));
+            }
+            mj[jj][0] = m4.x; mj[jj][1] = m4.y; mj[jj][2] = m4.z; mj[jj][3] = m4.w;
+            lj[jj][0] = l4.x; lj[jj][1] = l4.y; lj[jj][2] = l4.z; lj[jj][3] = l4.w;
+        }
+#pragma unroll
+        for (int hh = 0; hh < kGQ; ++hh) {
+            const float M = warp_max(fmaxf(mj[0][hh], mj[1][hh]));
+            float Lsum = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const float f = mj[jj][hh] == -INFINITY ? 0.f : exp2f(mj[jj][hh] - M);
+                if (lane + 32 * jj < nsplit) wgt[(which * kMaxSplits + lane + 32 * jj) * kGQ + hh] = f;
+                Lsum = fmaf(f, lj[jj][hh], Lsum);
+            }
+            Lsum = warp_sum(Lsum);
+            if (lane == 0) Ls[which * 4 + hh] = Lsum;
         }
     }
     __syncthreads();
-    // thread -> output elements q = (head, channel); full and (probe) no-residual sums
-    constexpr int kPer = 2;                        // ceil(4 * 128 / 288)
     float acc1[kPer], acc2[kPer];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) { acc1[k] = 0.f; acc2[k] = 0.f; }
-    for (int j0 = 0; j0 < nsplit; j0 += per_chunk) {
-        const int nj = min(per_chunk, nsplit - j0);
-        if (j0 > 0) {
-            __syncthreads();
-            for (int i = tid; i < nj * RF / 4; i += blockDim.x)
-                cp_async16(smem_addr(stage_f) + 16 * i, recs + (size_t)j0 * RF + 4 * i);
-            cp_async_wait_all();
-            __syncthreads();
-        }
+    for (int j0 = 0; j0 < nsplit; j0 += kChunk) {
+        if (j0 > 0) load_chunk(j0);
+        const int nj = min(kChunk, nsplit - j0);
 #pragma unroll
         for (int k = 0; k < kPer; ++k) {
-            const int q = tid + k * (int)blockDim.x;
-            if (q < kGQ * kD) {
-                const int hh = q / kD;
-                const float* w1 = wgt + hh;
-                const float* w2 = wgt + kMaxSplits * kGQ + hh;
-                float a = acc1[k], b = acc2[k];
-                for (int j = 0; j < nj; ++j) {
-                    a = fmaf(w1[(j0 + j) * kGQ], stage_f[(size_t)j * RF + hdr + q], a);
-                    if (PROBE) b = fmaf(w2[(j0 + j) * kGQ], stage_f[(size_t)j * RF + hdr + kGQ * kD + q], b);
+            const int q = tid + k * kDecodeThreads;
+            const int hh = (q < kGQ * kD ? q : 0) / kD;
+            const float* w1 = wgt + j0 * kGQ + hh;
+            const float* w2 = wgt + (kMaxSplits + j0) * kGQ + hh;
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j) {
+                if (j < nj) {
+                    acc1[k] = fmaf(w1[j * kGQ], v1[k][j], acc1[k]);
+                    if (PROBE) acc2[k] = fmaf(w2[j * kGQ], v2[k][j], acc2[k]);
                 }
-                acc1[k] = a;
-                acc2[k] = b;
             }
         }
     }
     float dn = 0.f, nn = 0.f;
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
-        const int q = tid + k * (int)blockDim.x;
+        const int q = tid + k * kDecodeThreads;
         if (q < kGQ * kD) {
             const int hh = q / kD, i = q % kD;
             const float L1 = Ls[hh];
@@ -847,12 +902,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         }
     }
     if (PROBE) {
-        red[tid] = dn;
-        red[kDecodeThreads + tid] = nn;
+        dn = warp_sum(dn);
+        nn = warp_sum(nn);
+        if (lane == 0) { red[warp] = dn; red[kDecodeThreads / 32 + warp] = nn; }
         __syncthreads();
         if (tid == 0) {
             float a = 0.f, b = 0.f;
-            for (int t = 0; t < (int)blockDim.x; ++t) { a += red[t]; b += red[kDecodeThreads + t]; }
+            for (int t = 0; t < kDecodeThreads / 32; ++t) { a += red[t]; b += red[kDecodeThreads / 32 + t]; }
             C.err[(size_t)ci * G.Hkv + h] = sqrtf(a) / (sqrtf(b) + 1e-6f);
         }
     }
