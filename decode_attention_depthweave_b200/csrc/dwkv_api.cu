@@ -243,29 +243,22 @@ size_t encode_smem(const Geom& G) {
     return (size_t)2 * kD * (G.r_max + 2) * 2 + (size_t)8 * (2 * kD + 2 * G.r_max + 64) * 4;
 }
 
-int decode_stages_for(dwkv_handle h, bool probe, int ctas_per_sm, size_t* smem_out) {
+// Bytes of the decode page ring: what the shared-memory budget leaves after the fixed
+// regions, capped at dec_stages_req x the largest chunk when that is set (but never below
+// the CTA merge's scratch, which reuses it).  0 when fewer than two of the largest chunks fit.
+// *smem_out receives the kernel's dynamic shared memory.
+uint32_t decode_ring_for(dwkv_handle h, bool probe, size_t* smem_out) {
     const Geom& G = h->geom;
-    const size_t budget = ctas_per_sm == 1 ? h->smem_optin : std::min(h->smem_optin, h->smem_per_sm / 2 - 1024);
-    int best = 0;
-    const int cap = h->dec_stages_req > 0 ? h->dec_stages_req : 16;
-    for (int ns = kPairs; ns <= cap; ns += kPairs) {
-        const DecodeSmem L = decode_smem_layout(G, ns, probe);
-        if (L.total <= budget) { best = ns; *smem_out = L.total; }
-    }
-    return best;
-}
-
-// Stages for the configured CTAs per SM; the probe (larger per-warp state) falls back to one
-// CTA per SM when two do not fit.  *ctas_out receives the CTAs per SM actually used.
-int decode_stages(dwkv_handle h, bool probe, size_t* smem_out, int* ctas_out = nullptr) {
-    int c = h->dec_ctas_per_sm;
-    int ns = decode_stages_for(h, probe, c, smem_out);
-    if (ns < kPairs && c > 1) {
-        c = 1;
-        ns = decode_stages_for(h, probe, c, smem_out);
-    }
-    if (ctas_out) *ctas_out = c;
-    return ns;
+    const size_t budget = h->smem_optin;
+    const DecodeSmem L0 = decode_smem_layout(G, 0, probe);
+    const size_t scratch = ((size_t)2 * kGQ * G.r_max + (size_t)kGQ * kD) * sizeof(float);
+    const size_t need = std::max(2 * (size_t)G.stage_bytes, scratch);
+    if ((size_t)L0.total + need > budget) return 0;
+    size_t ring = (budget - L0.total) / 128 * 128;
+    if (h->dec_stages_req > 0) ring = std::min(ring, std::max((size_t)h->dec_stages_req * G.stage_bytes, scratch));
+    if (ring < need) return 0;
+    *smem_out = decode_smem_layout(G, (uint32_t)ring, probe).total;
+    return (uint32_t)ring;
 }
 
 dwkv_status prepare_call(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
@@ -434,7 +427,7 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
         return cuda_fail(e, "dwkv_create");
     }
     size_t sm = 0;
-    if (decode_stages(h, true, &sm) < kPairs) {
+    if (decode_ring_for(h, true, &sm) == 0) {
         delete h;
         return fail(DWKV_ERR_UNSUPPORTED, "decode pipeline does not fit in shared memory for this geometry");
     }
@@ -451,17 +444,16 @@ dwkv_status dwkv_destroy(dwkv_handle h) {
 dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t waves, int32_t stages) {
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
-    if (ctas_per_sm != 1 || waves < 1 || waves > 8 || stages < 0 || stages > 32 ||
-        stages % kPairs)
-        return fail(DWKV_ERR_INVALID_ARG, "tuning out of range (ctas_per_sm 1, waves 1-8, stages 0 or a multiple of 4 up to 32)");
+    if (ctas_per_sm != 1 || waves < 1 || waves > 8 || stages < 0 || stages == 1 || stages > 32)
+        return fail(DWKV_ERR_INVALID_ARG, "tuning out of range (ctas_per_sm 1, waves 1-8, stages 0 or 2-32)");
     const int oc = h->dec_ctas_per_sm, ow = h->dec_waves, os = h->dec_stages_req;
     h->dec_ctas_per_sm = ctas_per_sm;
     h->dec_waves = waves;
     h->dec_stages_req = stages;
     size_t sm = 0;
-    if (decode_stages_for(h, false, ctas_per_sm, &sm) < kPairs) {
+    if (decode_ring_for(h, true, &sm) == 0) {
         h->dec_ctas_per_sm = oc; h->dec_waves = ow; h->dec_stages_req = os;
-        return fail(DWKV_ERR_INVALID_ARG, "tuning leaves no room for a 4-stage pipeline");
+        return fail(DWKV_ERR_INVALID_ARG, "tuning leaves no room for two page chunks");
     }
     return DWKV_OK;
 }
@@ -584,10 +576,9 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     C.g = g;
     C.lig = layer % G.LPG;
     size_t smem = 0;
-    int ctas = 1;
-    const int stages = decode_stages(h, probe, &smem, &ctas);
-    if (stages < kPairs) return fail(DWKV_ERR_UNSUPPORTED, "decode pipeline does not fit in shared memory");
-    const long long target = (long long)h->num_sms * ctas * h->dec_waves;
+    const uint32_t ring = decode_ring_for(h, probe, &smem);
+    if (ring == 0) return fail(DWKV_ERR_UNSUPPORTED, "decode pipeline does not fit in shared memory");
+    const long long target = (long long)h->num_sms * h->dec_waves;
     int total = 0;
     for (int i = 0; i < n_seqs; ++i) {
         const int s = seq_ids[i];
@@ -601,7 +592,7 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     }
     C.split_begin[n_seqs] = total;
     C.total_splits = total;
-    C.stages = stages;
+    C.ring_bytes = (int)ring;
     C.rec_floats = rec_floats_of(G, probe);
     C.tok_weight = h->dec_tok_weight;
     C.q = static_cast<const __nv_bfloat16*>(q);

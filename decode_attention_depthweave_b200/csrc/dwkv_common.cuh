@@ -33,8 +33,8 @@ constexpr int kUnit = 128;         // page-pool granularity in bytes
 constexpr int kMaxTiers = 8;
 constexpr int kMaxSeqs = 256;      // sequences per call
 constexpr int kMaxSplits = 64;     // decode splits per (sequence, kv-head)
-constexpr int kConsumerWarps = 8;  // 4 pairs; a pair shares one page (32 tokens per warp)
-constexpr int kPairs = kConsumerWarps / 2;
+constexpr int kConsumerWarps = 12; // each takes half pages (32 tokens) from a shared queue
+constexpr int kSlots = 32;          // page chunks in flight at most (one full / empty barrier pair each)
 constexpr int kDecodeThreads = 32 * (kConsumerWarps + 1);  // + 1 producer warp
 constexpr int kRdBytes = 128 * 32;                         // dense residual tile: 128 ch x 32 tokens int8
 
@@ -77,7 +77,7 @@ struct AppendCall {
 };
 
 struct DecodeCall {
-    int n, layer, g, lig, total_splits, stages, rec_floats;
+    int n, layer, g, lig, total_splits, ring_bytes, rec_floats;
     int tok_weight;          // split balance: cost of one token in byte-equivalents
     int seq[kMaxSeqs];
     int split_begin[kMaxSeqs + 1];
@@ -108,18 +108,29 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 }
 
 // Decode shared-memory layout (identical on host and device).
-//   stages  NS page chunks (NS a multiple of kPairs: stage <-> pair is fixed)
-//   rd      per consumer warp, one dense residual tile (also holds B_K during the prologue)
-//   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W[32][8] bf16, P2[32][8]
-//   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  zero line
+//   ring    page chunks, packed back to back (a chunk that does not fit before the end
+//           starts again at 0); ring_bytes is chosen by the host
+//   rd      per consumer warp, one 4 KB residual tile (also holds B_K during the prologue)
+//   bv      B_V [d][r_max] bf16, rows padded by 16 bytes (conflict-free ldmatrix)
+//   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W limbs [8][48] u8, P2[32][8]
+//   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  qh bf16 [d][4];  zero line
+//   bars    full[kSlots] empty[kSlots] basis table
+//   misc    tier table, page range, work counter; warp states; page-id batch; slot offsets
 struct DecodeSmem {
-    uint32_t stages, rd, small, small_stride, S, P, W, P2, qt, q, qh, zero, bars, misc, total;
+    uint32_t ring, rd, bv, bv_pitch, small, small_stride, S, P, W, P2, qt, q, qh, zero, bars, misc, total;
 };
-__host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, int NS, bool probe) {
+constexpr uint32_t kMiscState = 256;                               // m_state [warps][16]
+constexpr uint32_t kMiscFactors = kMiscState + kConsumerWarps * 64; // mf [2][warps][4]
+constexpr uint32_t kMiscPages = kMiscFactors + kConsumerWarps * 32; // t_src [32], t_len [32]
+constexpr uint32_t kMiscSlots = kMiscPages + 256;                  // slot offsets [kSlots]
+constexpr uint32_t kMiscBytes = kMiscSlots + kSlots * 4;
+__host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, uint32_t ring_bytes, bool probe) {
     DecodeSmem L;
     uint32_t o = 0;
-    L.stages = o;  o += (uint32_t)NS * G.stage_bytes;
+    L.ring = o;    o += ring_bytes;
     L.rd = o;      o += kConsumerWarps * kRdBytes;
+    L.bv_pitch = (uint32_t)G.r_max * 2 + 16;
+    L.bv = o;      o += (uint32_t)G.d * L.bv_pitch;
     uint32_t w = 0;
     L.S = w;       w += 32 * 16;
     L.P = w;       w += 32 * 16;
@@ -131,8 +142,8 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, int NS, 
     L.q = o;       o += (uint32_t)G.d * 16;
     L.qh = o;      o += (uint32_t)G.d * 8;
     L.zero = o;    o += 128;
-    L.bars = o;    o += (2 * NS + 2) * 8;
-    L.misc = o;    o += 1536;
+    L.bars = o;    o += (2 * kSlots + 2) * 8;
+    L.misc = o;    o += (kMiscBytes + 127) & ~127u;
     L.total = (o + 127) & ~127u;
     return L;
 }

@@ -421,20 +421,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y;
-    const int NS = C.stages;
-    const DecodeSmem L = decode_smem_layout(G, NS, PROBE);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);   // full[NS] empty[NS] basis table
-    const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + NS), basis_bar = smem_addr(bars + 2 * NS),
-                   table_bar = smem_addr(bars + 2 * NS + 1);
+    const DecodeSmem L = decode_smem_layout(G, (uint32_t)C.ring_bytes, PROBE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);   // full[kSlots] empty[kSlots] basis table
+    const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + kSlots),
+                   basis_bar = smem_addr(bars + 2 * kSlots), table_bar = smem_addr(bars + 2 * kSlots + 1);
     float4* qt = reinterpret_cast<float4*>(smem + L.qt);
     float4* qs = reinterpret_cast<float4*>(smem + L.q);
     uint32_t* m_cnt = reinterpret_cast<uint32_t*>(smem + L.misc);      // [8]
     uint32_t* m_P = m_cnt + 8;                                          // [9] page prefix
     uint32_t* m_R = m_P + 9;                                            // [8]
     uint32_t* m_chunk = m_R + 8;                                        // [8]
-    uint32_t* m_misc = m_chunk + 8;                                     // p_begin p_end last
-    float* m_state = reinterpret_cast<float*>(m_misc + 8);              // [8 warps][16]
-    float* mf = m_state + kConsumerWarps * 16;                          // [2][8 warps][4] factors
+    uint32_t* m_misc = m_chunk + 8;                                     // p_begin p_end last work
+    float* m_state = reinterpret_cast<float*>(smem + L.misc + kMiscState);     // [warps][16]
+    float* mf = reinterpret_cast<float*>(smem + L.misc + kMiscFactors);        // [2][warps][4] factors
+    uint32_t* m_slot = reinterpret_cast<uint32_t*>(smem + L.misc + kMiscSlots); // ring offset per slot
 
     // ---- which sequence / split
     int ci = 0;
@@ -451,14 +451,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     const int seq = C.seq[ci];
     const size_t basis_off = ((size_t)C.g * G.Hkv + h) * kD * G.r_max;
 
-    constexpr int kRowVec = RMAX / 8;
-    const int gi = tid & (kD - 1), ghp = tid >> 7;       // channel and head pair of threads < 2d
-    uint4 bv[kRowVec];                                  // row gi of B_V (consumer threads)
     uint32_t cv[kMaxTiers];                 // tier counts (producer lane 0)
     if (warp == kConsumerWarps && lane == 0) {
-        for (int i = 0; i < NS; ++i) {
+        for (int i = 0; i < kSlots; ++i) {
             mbar_init(full0 + 8 * i, 1);
-            mbar_init(empty0 + 8 * i, 2);     // both warps of the pair release
+            mbar_init(empty0 + 8 * i, 2);     // released by the warps of its two halves
         }
         mbar_init(basis_bar, 1);
         mbar_init(table_bar, 1);
@@ -503,8 +500,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                 const unsigned long long w = G.chunk_bytes[k] + tokw;
                 Wk -= (unsigned long long)np * w;      // first cost unit of tier k
                 if (!np) continue;
-                if (lo <= Wk + (np - 1) * w) pb = m_P[k] + (uint32_t)(lo > Wk ? (lo - Wk + w - 1) / w : 0);
-                if (hi <= Wk + (np - 1) * w) pe = m_P[k] + (uint32_t)(hi > Wk ? (hi - Wk + w - 1) / w : 0);
+                // lo - Wk < np * w fits 32 bits, so the divisions stay 32-bit
+                const uint32_t w32 = (uint32_t)w;
+                if (lo <= Wk + (np - 1) * w) pb = m_P[k] + (lo > Wk ? ((uint32_t)(lo - Wk) + w32 - 1) / w32 : 0u);
+                if (hi <= Wk + (np - 1) * w) pe = m_P[k] + (hi > Wk ? ((uint32_t)(hi - Wk) + w32 - 1) / w32 : 0u);
             }
             m_misc[0] = pb;
             m_misc[1] = pe > pb ? pe : pb;
@@ -515,15 +514,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         const uint32_t npages = p_end - p_begin;
         const size_t pbase = page_index(G, seq, C.g, h, 0);
         // The warp resolves 32 pages at a time (global page ids, byte counts) into a small
-        // table; lane 0 then issues the copies back to back with a running stage / phase.
-        uint32_t* t_src = reinterpret_cast<uint32_t*>(smem + L.misc + 1024);    // [32] pool units
-        uint32_t* t_len = t_src + 32;                                           // [32] bytes
-        uint32_t st = 0, ph = 0;
+        // table; lane 0 then places each chunk in the ring and issues its copy.  Chunks are
+        // reclaimed oldest first, so the ring holds pages [tail, u) at any time.
+        uint32_t* t_src = reinterpret_cast<uint32_t*>(smem + L.misc + kMiscPages);   // [32] pool units
+        uint32_t* t_len = t_src + 32;                                                // [32] bytes
+        const uint32_t RB = (uint32_t)C.ring_bytes;
+        const uint32_t ring = smem_addr(smem + L.ring);
+        uint32_t head = 0, tail = 0;
         bool ok = true;
         for (uint32_t b0 = 0; b0 < npages && ok; b0 += 32) {
             const uint32_t u = b0 + lane;
             if (u < npages) {
-                const uint32_t p = p_begin + u;
+                const uint32_t p = p_end - 1 - u;           // highest tier first: cheap pages end the run
                 int k = 0;
 #pragma unroll
                 for (int kk = 1; kk < kMaxTiers; ++kk)
@@ -534,18 +536,35 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             __syncwarp();
             if (lane == 0) {
                 const uint32_t nb = min(32u, npages - b0);
-                for (uint32_t j = 0; j < nb; ++j) {
-                    // stage st is being reused once the pages have wrapped around the ring
-                    if (b0 + j >= (uint32_t)NS && !mbar_wait(empty0 + 8 * st, ph ^ 1u)) {
-                        set_dev_error(St, 6u /*DWKV_DEV_TIMEOUT*/, (uint32_t)seq, b0 + j);
-                        ok = false;
-                        break;
+                for (uint32_t j = 0; j < nb && ok; ++j) {
+                    const uint32_t v = b0 + j, len = t_len[j];
+                    uint32_t off = 0;
+                    for (;;) {
+                        const uint32_t inflight = v - tail;
+                        if (inflight == 0) { off = 0; break; }
+                        if (inflight < (uint32_t)kSlots) {
+                            const uint32_t toff = m_slot[tail % kSlots];
+                            if (head > toff) {                     // occupied [toff, head)
+                                if (head + len <= RB) { off = head; break; }
+                                if (len <= toff) { off = 0; break; }
+                            } else if (head + len <= toff) {       // occupied [toff, end) + [0, head)
+                                off = head;
+                                break;
+                            }
+                        }
+                        if (!mbar_wait(empty0 + 8 * (tail % kSlots), (tail / kSlots) & 1u)) {
+                            set_dev_error(St, 6u /*DWKV_DEV_TIMEOUT*/, (uint32_t)seq, v);
+                            ok = false;
+                            break;
+                        }
+                        ++tail;
                     }
-                    const uint32_t bytes = t_len[j];
-                    mbar_arrive_expect_tx(full0 + 8 * st, bytes);
-                    bulk_g2s(smem_addr(smem + L.stages + (size_t)st * G.stage_bytes),
-                             St.data + (size_t)t_src[j] * kUnit + (size_t)C.lig * bytes, bytes, full0 + 8 * st);
-                    if (++st == (uint32_t)NS) { st = 0; ph ^= 1u; }
+                    if (!ok) break;
+                    const uint32_t sl = v % kSlots;
+                    m_slot[sl] = off;
+                    head = off + len;
+                    mbar_arrive_expect_tx(full0 + 8 * sl, len);
+                    bulk_g2s(ring + off, St.data + (size_t)t_src[j] * kUnit + (size_t)C.lig * len, len, full0 + 8 * sl);
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -558,6 +577,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         const uint32_t zero_addr = smem_addr(smem + L.zero);
         const float qscale = G.tau * kLog2e;
         uint2* qh = reinterpret_cast<uint2*>(smem + L.qh);
+        {   // B_V for the CTA merge, in flight for the whole main loop (16-byte cp.async)
+            const int nch = G.r_max / 8;
+            const uint32_t bvs = smem_addr(smem + L.bv);
+            for (int x = tid; x < kD * nch; x += kConsumerWarps * 32) {
+                const int row = x / nch, ch = x % nch;
+                cp_async16(bvs + row * L.bv_pitch + ch * 16, St.basis_v + basis_off + (size_t)row * G.r_max + ch * 8);
+            }
+        }
         if (tid < kD) {
             const __nv_bfloat16* q = C.q + ((size_t)ci * G.Hq + (size_t)h * kGQ) * kD + tid;
             const __nv_bfloat16 q0 = q[0], q1 = q[kD], q2 = q[2 * kD], q3 = q[3 * kD];
@@ -575,9 +602,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         // are summed through the small buffers.
         const int rq = G.r_max < 16 ? 16 : G.r_max;
         {
-            const int np = (kConsumerWarps * 32) / rq, j = tid % rq, part = tid / rq, rows = kD / np;
+            const int np = 256 / rq, j = tid % rq, part = tid / rq, rows = kD / np;
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (ok && j < G.r_max) {
+            if (ok && tid < 256 && j < G.r_max) {
                 const __nv_bfloat16* bk = reinterpret_cast<const __nv_bfloat16*>(smem + L.rd) + j;
 #pragma unroll 8
                 for (int i = part * rows; i < (part + 1) * rows; ++i) {
@@ -588,7 +615,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                 }
             }
             float4* parts = reinterpret_cast<float4*>(smem + L.small);     // [np][rq]
-            parts[part * rq + j] = a;
+            if (tid < 256) parts[part * rq + j] = a;
             named_barrier(1, kConsumerWarps * 32);
             if (tid < rq) {
                 float4 t4 = parts[tid];
@@ -667,24 +694,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                 if (lane == 0) wn = atomicAdd(work, 1u);
                 wn = __shfl_sync(0xffffffffu, wn, 0);
             }
-            const uint32_t u = w >> 1, p = p_begin + u, st = u % NS;
+            const uint32_t u = w >> 1, p = p_end - 1 - u, sl = u % kSlots;
             const int half = (int)(w & 1);
             int k = 0;
             while (k + 1 < G.ntiers && p >= m_P[k + 1]) ++k;
             const int R = (int)m_R[k];
             const uint32_t pit = p - m_P[k], npk = m_P[k + 1] - m_P[k];
             const int nvalid = pit + 1 < npk ? kPage : (int)(m_cnt[k] - pit * kPage);
-            if (!mbar_wait(full0 + 8 * st, (u / NS) & 1)) {
+            if (!mbar_wait(full0 + 8 * sl, (u / kSlots) & 1)) {
                 if (lane == 0) set_dev_error(St, 6u, (uint32_t)seq, u);
                 ok = false;
                 break;
             }
             const int nv = min(max(nvalid - 32 * half, 0), 32);
             if (nv > 0)
-                run_page<S, BITS, PROBE, RMAX>(R, smem + L.stages + (size_t)st * G.stage_bytes, half, nv, qb, qh,
+                run_page<S, BITS, PROBE, RMAX>(R, smem + L.ring + m_slot[sl], half, nv, qb, qh,
                                                qscale, small, rd, zero_addr, A, lane);
             __syncwarp();
-            if (lane == 0) mbar_arrive(empty0 + 8 * st);
+            if (lane == 0) mbar_arrive(empty0 + 8 * sl);
             if (wn == 0xffffffffu) {
                 if (lane == 0) wn = atomicAdd(work, 1u);
                 wn = __shfl_sync(0xffffffffu, wn, 0);
@@ -705,11 +732,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             }
         }
         if (PROBE) store_d(A.c2, reinterpret_cast<float*>(small), G.r_max, lane);
-        {   // B_V row gi for the CTA's GEMV below, requested before waiting for the other warps
-            const uint4* row = reinterpret_cast<const uint4*>(St.basis_v + basis_off + (size_t)gi * G.r_max);
-#pragma unroll
-            for (int v = 0; v < kRowVec; ++v) bv[v] = v * 8 < G.r_max ? __ldcg(row + v) : make_uint4(0u, 0u, 0u, 0u);
-        }
         float* ms = m_state + warp * 16;
 #pragma unroll
         for (int hh = 0; hh < kGQ; ++hh) {
@@ -723,22 +745,37 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     }
     __syncthreads();
 
-    // ================= CTA merge: the 8 warp states -> one partial record
+    // ================= CTA merge: the warp states -> one partial record
     //   {M[4], L[4], (M2[4], L2[4]), o[4][d] = B_V acc_c + acc_r, (o2[4][d] = B_V acc_c2)}
-    // B_V is applied here, once per CTA, so the final merge is a weighted sum.
+    // B_V is applied here, once per CTA (tensor cores), so the final merge is a weighted sum.
     const int nrec = C.total_splits;
     float* rec = C.ws + ((size_t)h * nrec + blockIdx.x) * C.rec_floats;
     const int hdr = PROBE ? 16 : 8;
+    const int nc = kGQ * G.r_max;
     if (warp < (PROBE ? 2 : 1)) {
-        // lane = (warp w2, head hh): the CTA max and the rescaled sum by shuffles
-        const int which = warp, w2 = lane >> 2, hh = lane & 3;
-        const float m = m_state[w2 * 16 + which * 8 + hh];
-        float M = m;
+        // lane = (warp w2 = lane / 4 + 8 i, head hh): the CTA max and rescaled sum by shuffles
+        const int which = warp, hh = lane & 3;
+        constexpr int kRounds = (kConsumerWarps + 7) / 8;
+        float m[kRounds];
+        float M = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kRounds; ++i) {
+            const int w2 = (lane >> 2) + 8 * i;
+            m[i] = w2 < kConsumerWarps ? m_state[w2 * 16 + which * 8 + hh] : -INFINITY;
+            M = fmaxf(M, m[i]);
+        }
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        const float f = m == -INFINITY ? 0.f : exp2f(m - M);
-        mf[which * 32 + w2 * 4 + hh] = f;
-        float Lsum = f * m_state[w2 * 16 + which * 8 + 4 + hh];
+        float Lsum = 0.f;
+#pragma unroll
+        for (int i = 0; i < kRounds; ++i) {
+            const int w2 = (lane >> 2) + 8 * i;
+            if (w2 < kConsumerWarps) {
+                const float f = m[i] == -INFINITY ? 0.f : exp2f(m[i] - M);
+                mf[which * kConsumerWarps * 4 + w2 * 4 + hh] = f;
+                Lsum = fmaf(f, m_state[w2 * 16 + which * 8 + 4 + hh], Lsum);
+            }
+        }
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
         if (lane < kGQ) {
@@ -747,52 +784,81 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         }
     }
     __syncthreads();
-    float* cm = reinterpret_cast<float*>(smem + L.stages);          // [(PROBE ? 2 : 1)][4][r_max]
-    for (int e = tid; e < kGQ * G.r_max; e += blockDim.x) {
-        const int hh = e / G.r_max, j = e % G.r_max;
-        float v = 0.f, v2 = 0.f;
+    // merged sums into the idle ring: cm [4][r_max], racc [4][d], (cm2 [4][r_max]); each warp's
+    // sums sit in its residual tile ([j][4] then [i][4]) and, for acc_c2, its small buffer
+    float* cm = reinterpret_cast<float*>(smem + L.ring);
+    const int nbody = nc + kGQ * kD + (PROBE ? nc : 0);
+    for (int e = tid; e < nbody; e += blockDim.x) {
+        int hh, off, which = 0;
+        const uint8_t* base = smem + L.rd;
+        uint32_t stride = kRdBytes;
+        if (e < nc) { hh = e / G.r_max; off = (e % G.r_max) * 4 + hh; }
+        else if (e < nc + kGQ * kD) { const int x = e - nc; hh = x / kD; off = G.r_max * 4 + (x % kD) * 4 + hh; }
+        else { const int x = e - nc - kGQ * kD; hh = x / G.r_max; off = (x % G.r_max) * 4 + hh;
+               which = 1; base = smem + L.small; stride = L.small_stride; }
+        float v = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
-            v = fmaf(mf[w2 * 4 + hh], reinterpret_cast<const float*>(smem + L.rd + w2 * kRdBytes)[j * 4 + hh], v);
-            if (PROBE)
-                v2 = fmaf(mf[32 + w2 * 4 + hh],
-                          reinterpret_cast<const float*>(smem + L.small + w2 * L.small_stride)[j * 4 + hh], v2);
-        }
+        for (int w2 = 0; w2 < kConsumerWarps; ++w2)
+            v = fmaf(mf[which * kConsumerWarps * 4 + w2 * 4 + hh],
+                     reinterpret_cast<const float*>(base + w2 * stride)[off], v);
         cm[e] = v;
-        if (PROBE) cm[kGQ * G.r_max + e] = v2;
     }
+    cp_async_wait_all();                                // this thread's B_V pieces
     __syncthreads();
-    if (tid < 2 * kD) {
+    if (warp < kD / 16) {
+        // o[i][h] for the warp's 16 channels: B_V rows (A, ldmatrix) against the merged acc_c as
+        // bf16 hi (columns 0-3) + lo (columns 4-7) halves (B), fp32 accumulation
+        const int g = lane >> 2, c = lane & 3, n = g & 3;
+        const bool lo_half = g >= 4;
+        const float* racc = cm + nc;
+        const float* cm2 = cm + nc + kGQ * kD;
+        float d[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t arow = (uint32_t)(16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1));
+        const uint32_t zero_addr = smem_addr(smem + L.zero);
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int hh = 2 * ghp + q;
-            const float* c1 = cm + hh * G.r_max;
-            const float* c2 = cm + kGQ * G.r_max + hh * G.r_max;
-            float a = 0.f, a2 = 0.f, b = 0.f, b2 = 0.f;
+        for (int ks = 0; ks < RMAX / 16; ++ks) {
+            if (16 * ks >= G.r_max) break;
+            const int kc = 16 * ks + 8 * (lane >> 4);
+            uint32_t a[4];
+            ldsm_x4(kc < G.r_max ? smem_addr(smem + L.bv) + arow * L.bv_pitch + kc * 2 : zero_addr, a);
+            uint32_t b[2], b2[2];
 #pragma unroll
-            for (int v = 0; v < kRowVec; ++v) {
-                if (v * 8 >= G.r_max) break;
-                const uint32_t w[4] = {bv[v].x, bv[v].y, bv[v].z, bv[v].w};
+            for (int r2 = 0; r2 < 2; ++r2) {
+                uint32_t pk = 0, pk2 = 0;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = v * 8 + 2 * e;
-                    a = fmaf(bf16lo(w[e]), c1[j], a);
-                    b = fmaf(bf16hi(w[e]), c1[j + 1], b);
+                for (int e = 0; e < 2; ++e) {
+                    const int k = 16 * ks + 8 * r2 + 2 * c + e;
+                    uint32_t hi, lo;
+                    split_bf16_rn(k < G.r_max ? cm[n * G.r_max + k] : 0.f, hi, lo);
+                    pk |= (lo_half ? lo : hi) << (16 * e);
                     if (PROBE) {
-                        a2 = fmaf(bf16lo(w[e]), c2[j], a2);
-                        b2 = fmaf(bf16hi(w[e]), c2[j + 1], b2);
+                        split_bf16_rn(k < G.r_max ? cm2[n * G.r_max + k] : 0.f, hi, lo);
+                        pk2 |= (lo_half ? lo : hi) << (16 * e);
                     }
                 }
+                b[r2] = pk;
+                b2[r2] = pk2;
             }
-            a += b;
-            a2 += b2;
-            float r = 0.f;
+            mma_bf16(d, a, b);
+            if (PROBE) mma_bf16(d2, a, b2);
+        }
+        // lanes c and c^2 hold the hi and lo columns of heads 2(c&1), 2(c&1)+1
 #pragma unroll
-            for (int w2 = 0; w2 < kConsumerWarps; ++w2)
-                r = fmaf(mf[w2 * 4 + hh],
-                         reinterpret_cast<const float*>(smem + L.rd + w2 * kRdBytes)[G.r_max * 4 + gi * 4 + hh], r);
-            rec[hdr + hh * kD + gi] = a + r;
-            if (PROBE) rec[hdr + kGQ * kD + hh * kD + gi] = a2;
+        for (int e = 0; e < 4; ++e) {
+            d[e] += __shfl_xor_sync(0xffffffffu, d[e], 2);
+            if (PROBE) d2[e] += __shfl_xor_sync(0xffffffffu, d2[e], 2);
+        }
+        if (c < 2) {
+#pragma unroll
+            for (int rr2 = 0; rr2 < 2; ++rr2) {
+                const int i = 16 * warp + g + 8 * rr2;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int hh = 2 * c + q;
+                    rec[hdr + hh * kD + i] = d[2 * rr2 + q] + racc[hh * kD + i];
+                    if (PROBE) rec[hdr + kGQ * kD + hh * kD + i] = d2[2 * rr2 + q];
+                }
+            }
         }
     }
     __threadfence();
@@ -814,8 +880,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     float* wgt = reinterpret_cast<float*>(smem + L.small);                        // [2][kMaxSplits][4]
     float* Ls = wgt + 2 * kMaxSplits * kGQ;                                        // [2][4]
     float* red = Ls + 8;                                                           // [2][warps]
-    constexpr int kPer = 2;                        // ceil(4 * 128 / 288) outputs per thread
-    constexpr int kChunk = 16;                     // records whose values are held at once
+    constexpr int kPer = (kGQ * kD + kDecodeThreads - 1) / kDecodeThreads;   // outputs per thread
+    constexpr int kChunk = PROBE ? 8 : 32;         // records whose values are held at once
     float v1[kPer][kChunk], v2[kPer][PROBE ? kChunk : 1];
     auto load_chunk = [&](int j0) {
         const int nj = min(kChunk, nsplit - j0);
@@ -912,6 +978,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             C.err[(size_t)ci * G.Hkv + h] = sqrtf(a) / (sqrtf(b) + 1e-6f);
         }
     }
+    if (tid == 0) St.tickets[(size_t)seq * G.Hkv + h] = 0u;
     if (tid == 0) St.tickets[(size_t)seq * G.Hkv + h] = 0u;
 }
 

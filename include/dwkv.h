@@ -215,9 +215,10 @@ dwkv_status dwkv_pool_usage(dwkv_handle h, void* stream, dwkv_pool_stats* out);
 dwkv_status dwkv_sync_status(dwkv_handle h, void* stream);
 
 /* Launch tuning (for measurement sweeps): decode CTAs per SM (1 in this build: one
- * 288-thread CTA fills an SM's registers), split waves per decode (1..8) and pipeline
- * stages per CTA (0 = largest that fits, else a multiple of 4).  Returns
- * DWKV_ERR_INVALID_ARG for values out of range. */
+ * 13-warp CTA fills an SM's registers), split waves per decode (1..8) and a cap on the
+ * CTA's page ring in units of the largest page chunk (0 = all the shared memory the other
+ * regions leave, else 2..32).  Returns DWKV_ERR_INVALID_ARG for values out of range or a
+ * ring that cannot hold two chunks. */
 dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t waves,
                                    int32_t stages);
 

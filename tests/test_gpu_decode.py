@@ -110,7 +110,7 @@ def test_sequence_subset_and_order():
         check_close(out[i].cpu().numpy(), oracle.decode_head(head_problem(wl, bases, tiers, comp, q[i], 1, 0)))
 
 
-@pytest.mark.parametrize("ctas,waves,stages", [(1, 1, 0), (1, 2, 0), (1, 3, 4), (1, 1, 8)])
+@pytest.mark.parametrize("ctas,waves,stages", [(1, 1, 0), (1, 2, 0), (1, 3, 4), (1, 1, 8), (1, 1, 2), (1, 2, 3)])
 def test_launch_tunings_agree(ctas, waves, stages):
     wl = synth.workload("llama8b_64k").scaled(num_layers=2, context=5000)
     bases = synth.make_bases(wl)
