@@ -106,7 +106,14 @@ class ClockSampler:
                  "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        time.sleep(0.5)
+        # nvidia-smi's first query can take a while on a fresh box: start timing only once
+        # it is sampling, so its start-up never overlaps the timed region
+        t_end = time.time() + 10.0
+        while self.proc is not None and time.time() < t_end:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
+        time.sleep(0.2)
         return self
 
     def mark_start(self):
