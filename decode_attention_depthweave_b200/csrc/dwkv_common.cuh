@@ -111,13 +111,12 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 //   ring    page chunks, packed back to back (a chunk that does not fit before the end
 //           starts again at 0); ring_bytes is chosen by the host
 //   rd      per consumer warp, one 4 KB residual tile (also holds B_K during the prologue)
-//   bv      B_V [d][r_max] bf16, rows padded by 16 bytes (conflict-free ldmatrix)
 //   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W limbs [8][48] u8, P2[32][8]
 //   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  qh bf16 [d][4];  zero line
 //   bars    full[kSlots] empty[kSlots] basis table
 //   misc    tier table, page range, work counter; warp states; page-id batch; slot offsets
 struct DecodeSmem {
-    uint32_t ring, rd, bv, bv_pitch, small, small_stride, S, P, W, P2, qt, q, qh, zero, bars, misc, total;
+    uint32_t ring, rd, small, small_stride, S, P, W, P2, qt, q, qh, zero, bars, misc, total;
 };
 constexpr uint32_t kMiscState = 256;                               // m_state [warps][16]
 constexpr uint32_t kMiscFactors = kMiscState + kConsumerWarps * 64; // mf [2][warps][4]
@@ -129,8 +128,6 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, uint32_t
     uint32_t o = 0;
     L.ring = o;    o += ring_bytes;
     L.rd = o;      o += kConsumerWarps * kRdBytes;
-    L.bv_pitch = (uint32_t)G.r_max * 2 + 16;
-    L.bv = o;      o += (uint32_t)G.d * L.bv_pitch;
     uint32_t w = 0;
     L.S = w;       w += 32 * 16;
     L.P = w;       w += 32 * 16;

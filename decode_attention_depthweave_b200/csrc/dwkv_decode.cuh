@@ -115,6 +115,16 @@ __device__ __forceinline__ float code4(uint32_t word, int e) {
     return __uint_as_float(0x4B400000u | (b ^ 0x8u)) - 12582920.0f;    // 2^23 + 2^22 + 8
 }
 
+template <int BITS>
+__device__ __forceinline__ uint32_t code_bytes(uint32_t cw) {
+    if (BITS == 8) return cw;
+    const uint32_t y = __byte_perm(cw, 0u, 0x1100);              // bytes b0 b0 b1 b1
+    // bytes 0, 2 from y << 4 (low nibbles moved up), bytes 1, 3 from y; clear the low nibbles
+    const uint32_t z = ((y << 4) & 0x00FF00FFu) | (y & 0xFF00FF00u);
+    return z & 0xF0F0F0F0u;
+}
+constexpr float kCodeUnit4 = 1.0f / 16.0f;              // value of one int4 tile unit
+
 template <int RMAX, bool PROBE>
 struct WarpAcc {
     float c[RMAX / 16][4];                 // coefficient-space values, D layout (row j, col n)
@@ -283,6 +293,7 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 Wsm[(2 * h + 1) * kWbPitch + lane] = (uint8_t)v;
                 if (c == h) wdq = eb >= 16u ? __uint_as_float((eb - 15u) << 23) : 0.f;   // 2^(E-15)
             }
+            if (BITS == 4) wdq *= kCodeUnit4;
         }
         if (PROBE) {
             bool over2 = false;
@@ -343,15 +354,12 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
 #pragma unroll
             for (int e = 0; e < S; e += 4) {
                 const uint32_t ix = *reinterpret_cast<const uint32_t*>(V + kOffIdx + tok * S + e);
-                uint32_t cw;
-                if (BITS == 8) cw = *reinterpret_cast<const uint32_t*>(V + kOffCodes + tok * S + e);
-                else cw = *reinterpret_cast<const uint16_t*>(V + kOffCodes + tok * (S / 2) + e / 2);
+                const uint32_t cbw = code_bytes<BITS>(BITS == 8 ? *reinterpret_cast<const uint32_t*>(V + kOffCodes + tok * S + e)
+                                                                : *reinterpret_cast<const uint16_t*>(V + kOffCodes + tok * (S / 2) + e / 2));
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t ch = (ix >> (8 * q)) & 0xffu;
-                    // the code as a signed byte (int4: sign-extend the nibble)
-                    const uint32_t cb = BITS == 8 ? (cw >> (8 * q)) : (uint32_t)((int32_t)(cw << (28 - 4 * q)) >> 28);
-                    rd[rd_off(ch, (uint32_t)lane)] = (uint8_t)cb;
+                    const uint32_t ch = __byte_perm(ix, 0u, 0x4440 + q);
+                    rd[rd_off(ch, (uint32_t)lane)] = (uint8_t)(cbw >> (8 * q));
                 }
             }
         }
@@ -452,6 +460,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     const size_t basis_off = ((size_t)C.g * G.Hkv + h) * kD * G.r_max;
 
     uint32_t cv[kMaxTiers];                 // tier counts (producer lane 0)
+    uint32_t bvf[RMAX / 16][4];             // B_V mma fragments (consumer warps 0-7, epilogue)
     if (warp == kConsumerWarps && lane == 0) {
         for (int i = 0; i < kSlots; ++i) {
             mbar_init(full0 + 8 * i, 1);
@@ -577,13 +586,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         const uint32_t zero_addr = smem_addr(smem + L.zero);
         const float qscale = G.tau * kLog2e;
         uint2* qh = reinterpret_cast<uint2*>(smem + L.qh);
-        {   // B_V for the CTA merge, in flight for the whole main loop (16-byte cp.async)
-            const int nch = G.r_max / 8;
-            const uint32_t bvs = smem_addr(smem + L.bv);
-            for (int x = tid; x < kD * nch; x += kConsumerWarps * 32) {
-                const int row = x / nch, ch = x % nch;
-                cp_async16(bvs + row * L.bv_pitch + ch * 16, St.basis_v + basis_off + (size_t)row * G.r_max + ch * 8);
-            }
+        {   // B_V, read from registers by the CTA merge at the end: warm it into L2 now
+            const int lines = kD * G.r_max * 2 / 128;
+            for (int x = tid; x < lines; x += kConsumerWarps * 32)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(St.basis_v + basis_off) + 128 * x));
         }
         if (tid < kD) {
             const __nv_bfloat16* q = C.q + ((size_t)ci * G.Hq + (size_t)h * kGQ) * kD + tid;
@@ -732,6 +738,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             }
         }
         if (PROBE) store_d(A.c2, reinterpret_cast<float*>(small), G.r_max, lane);
+        if (warp < kD / 16) {
+            // this warp's 16 B_V rows as mma A fragments (row 16 warp + g (+8), columns
+            // 16 ks + 2c (+1, +8, +9)), requested now so they arrive while the CTA merges
+            const int g = lane >> 2, c = lane & 3;
+            const __nv_bfloat16* b0 = St.basis_v + basis_off + (size_t)(16 * warp + g) * G.r_max + 2 * c;
+#pragma unroll
+            for (int ks = 0; ks < RMAX / 16; ++ks) {
+                const int k0 = 16 * ks, k1 = 16 * ks + 8;
+                bvf[ks][0] = k0 < G.r_max ? __ldg(reinterpret_cast<const unsigned int*>(b0 + k0)) : 0u;
+                bvf[ks][1] = k0 < G.r_max ? __ldg(reinterpret_cast<const unsigned int*>(b0 + 8 * G.r_max + k0)) : 0u;
+                bvf[ks][2] = k1 < G.r_max ? __ldg(reinterpret_cast<const unsigned int*>(b0 + k1)) : 0u;
+                bvf[ks][3] = k1 < G.r_max ? __ldg(reinterpret_cast<const unsigned int*>(b0 + 8 * G.r_max + k1)) : 0u;
+            }
+        }
         float* ms = m_state + warp * 16;
 #pragma unroll
         for (int hh = 0; hh < kGQ; ++hh) {
@@ -803,7 +823,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                      reinterpret_cast<const float*>(base + w2 * stride)[off], v);
         cm[e] = v;
     }
-    cp_async_wait_all();                                // this thread's B_V pieces
     __syncthreads();
     if (warp < kD / 16) {
         // o[i][h] for the warp's 16 channels: B_V rows (A, ldmatrix) against the merged acc_c as
@@ -813,14 +832,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         const float* racc = cm + nc;
         const float* cm2 = cm + nc + kGQ * kD;
         float d[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t arow = (uint32_t)(16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1));
-        const uint32_t zero_addr = smem_addr(smem + L.zero);
 #pragma unroll
         for (int ks = 0; ks < RMAX / 16; ++ks) {
             if (16 * ks >= G.r_max) break;
-            const int kc = 16 * ks + 8 * (lane >> 4);
-            uint32_t a[4];
-            ldsm_x4(kc < G.r_max ? smem_addr(smem + L.bv) + arow * L.bv_pitch + kc * 2 : zero_addr, a);
+            const uint32_t (&a)[4] = bvf[ks];
             uint32_t b[2], b2[2];
 #pragma unroll
             for (int r2 = 0; r2 < 2; ++r2) {
