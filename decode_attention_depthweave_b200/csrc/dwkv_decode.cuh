@@ -531,18 +531,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         const uint32_t ring = smem_addr(smem + L.ring);
         uint32_t head = 0, tail = 0;
         bool ok = true;
-        for (uint32_t b0 = 0; b0 < npages && ok; b0 += 32) {
-            const uint32_t u = b0 + lane;
-            if (u < npages) {
-                const uint32_t p = p_end - 1 - u;           // highest tier first: cheap pages end the run
-                int k = 0;
+        // lane j resolves page b0 + j of each batch; the next batch's ids are requested before
+        // lane 0 issues the current batch, so their latency hides behind the issuing
+        auto page_id = [&](uint32_t u, uint32_t& len) -> uint32_t {
+            const uint32_t p = p_end - 1 - u;               // highest tier first: cheap pages end the run
+            int k = 0;
 #pragma unroll
-                for (int kk = 1; kk < kMaxTiers; ++kk)
-                    if (kk < G.ntiers && p >= m_P[kk]) k = kk;
-                t_src[lane] = __ldcg(St.pages + pbase + (size_t)k * G.max_pages + (p - m_P[k]));
-                t_len[lane] = m_chunk[k];
-            }
+            for (int kk = 1; kk < kMaxTiers; ++kk)
+                if (kk < G.ntiers && p >= m_P[kk]) k = kk;
+            len = m_chunk[k];
+            return __ldcg(St.pages + pbase + (size_t)k * G.max_pages + (p - m_P[k]));
+        };
+        uint32_t nxt_src = 0, nxt_len = 0;
+        if (lane < npages) nxt_src = page_id(lane, nxt_len);
+        for (uint32_t b0 = 0; b0 < npages && ok; b0 += 32) {
+            t_src[lane] = nxt_src;
+            t_len[lane] = nxt_len;
             __syncwarp();
+            if (b0 + 32 + lane < npages) nxt_src = page_id(b0 + 32 + lane, nxt_len);
             if (lane == 0) {
                 const uint32_t nb = min(32u, npages - b0);
                 for (uint32_t j = 0; j < nb && ok; ++j) {
