@@ -105,16 +105,9 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// signed int8 / int4 code -> float (exact), by biasing into a float's mantissa
-__device__ __forceinline__ float code8(uint32_t word, int e) {
-    const uint32_t b = (word >> (8 * e)) & 0xffu;
-    return __uint_as_float(0x4B400000u | (b ^ 0x80u)) - 12583040.0f;   // 2^23 + 2^22 + 128
-}
-__device__ __forceinline__ float code4(uint32_t word, int e) {
-    const uint32_t b = (word >> (4 * e)) & 0xfu;
-    return __uint_as_float(0x4B400000u | (b ^ 0x8u)) - 12582920.0f;    // 2^23 + 2^22 + 8
-}
-
+// Four residual codes as signed bytes in one word (byte j = code j): int8 codes as stored;
+// int4 codes as 16 x code (the nibble moved to the byte's high half, which keeps its sign), the
+// factor 1/16 going into the dequantisation.  `cw` holds the 4 codes in its low 32 / 16 bits.
 template <int BITS>
 __device__ __forceinline__ uint32_t code_bytes(uint32_t cw) {
     if (BITS == 8) return cw;
@@ -141,10 +134,10 @@ __device__ __forceinline__ void rescale_d(float (&d)[N][4], float a0, float a1) 
 }
 
 // Dense value-residual tile of one warp: 128 channel rows x 32 tokens of int8 codes (zero
-// where a token has no entry).  Row pitch 32 bytes; the two 16-byte halves of a row swap
-// places in rows with bit 2 set, so the 8 rows of every ldmatrix hit disjoint bank groups.
+// where a token has no entry), stored as two sub-tiles [128][16] (tokens 0-15, 16-31) with
+// 16-byte rows: the 8 rows of an ldmatrix are then 128 contiguous bytes.
 __device__ __forceinline__ uint32_t rd_off(uint32_t row, uint32_t tok) {
-    return row * 32u + (tok ^ ((row & 4u) << 2));
+    return (tok >> 4) * 2048u + row * 16u + (tok & 15u);
 }
 // Per-head byte rows of the weight limbs: row n = 2 h + limb, 32 tokens, 48-byte pitch (the
 // eight rows' 4-byte words read by one B-fragment load then fall in distinct banks).
@@ -185,17 +178,12 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 mma_bf16(d[mt], a, qb[ks]);
             }
         }
-        // hi + lo columns: lanes c and c^2 hold (hi, lo) of the same two heads
+        // S[token][8]: columns 0-3 the hi parts of heads 0-3, 4-7 the lo parts (summed per token
+        // below); S spans the P buffer too, which is written only after every lane has read S
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d[mt][e] += __shfl_xor_sync(0xffffffffu, d[mt][e], 2);
-        if (c < 2) {
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                *reinterpret_cast<float2*>(Ssm + (16 * mt + g) * 4 + 2 * c) = make_float2(d[mt][0], d[mt][1]);
-                *reinterpret_cast<float2*>(Ssm + (16 * mt + g + 8) * 4 + 2 * c) = make_float2(d[mt][2], d[mt][3]);
-            }
+        for (int mt = 0; mt < 2; ++mt) {
+            *reinterpret_cast<float2*>(Ssm + (16 * mt + g) * 8 + 2 * c) = make_float2(d[mt][0], d[mt][1]);
+            *reinterpret_cast<float2*>(Ssm + (16 * mt + g + 8) * 8 + 2 * c) = make_float2(d[mt][2], d[mt][3]);
         }
     }
     __syncwarp();
@@ -207,24 +195,37 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
     {
 #pragma unroll
         for (int h = 0; h < kGQ; ++h) { sc[h] = -INFINITY; sc2[h] = -INFINITY; }
+        float4 sv;
+        {
+            const float4 s0 = *reinterpret_cast<const float4*>(Ssm + lane * 8);
+            const float4 s1 = *reinterpret_cast<const float4*>(Ssm + lane * 8 + 4);
+            sv = make_float4(s0.x + s1.x, s0.y + s1.y, s0.z + s1.z, s0.w + s1.w);
+        }
+        __syncwarp();                                   // S is dead from here (P overwrites it)
         if (live) {
-            const float4 sv = *reinterpret_cast<const float4*>(Ssm + lane * 4);
             float ra[kGQ] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int ch = 0; ch < S; ch += 8) {
                 const uint2 ix = *reinterpret_cast<const uint2*>(K + kOffIdx + t * S + ch);
-                uint32_t cw0, cw1 = 0;
+                // codes as biased bytes (code + 2^(b-1)), each turned into a float by placing it in
+                // the mantissa of 2^23 and subtracting 2^23 + 2^(b-1)
+                uint32_t cb0, cb1;
                 if (BITS == 8) {
                     const uint2 cc = *reinterpret_cast<const uint2*>(K + kOffCodes + t * S + ch);
-                    cw0 = cc.x;
-                    cw1 = cc.y;
+                    cb0 = cc.x ^ 0x80808080u;
+                    cb1 = cc.y ^ 0x80808080u;
                 } else {
-                    cw0 = *reinterpret_cast<const uint32_t*>(K + kOffCodes + t * (S / 2) + ch / 2);
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(K + kOffCodes + t * (S / 2) + ch / 2) ^ 0x88888888u;
+                    cb0 = w & 0x0F0F0F0Fu;                      // codes 0, 2, 4, 6
+                    cb1 = (w >> 4) & 0x0F0F0F0Fu;               // codes 1, 3, 5, 7
                 }
+                constexpr float kBias = BITS == 8 ? 8388736.0f : 8388616.0f;    // 2^23 + 2^(b-1)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const uint32_t i = ((e < 4 ? ix.x : ix.y) >> (8 * (e & 3))) & 0xffu;
-                    const float cf = BITS == 8 ? code8(e < 4 ? cw0 : cw1, e & 3) : code4(cw0, e);
+                    const uint32_t i = __byte_perm(e < 4 ? ix.x : ix.y, 0u, 0x4440 + (e & 3));
+                    const uint32_t src = BITS == 8 ? (e < 4 ? cb0 : cb1) : ((e & 1) ? cb1 : cb0);
+                    const uint32_t sel = BITS == 8 ? (e & 3) : (e >> 1);
+                    const float cf = __uint_as_float(__byte_perm(src, 0x4B000000u, 0x7440 + sel)) - kBias;
                     const uint2 q = qh[i];                // the 4 heads' q_i as bf16 (exact)
                     ra[0] = fmaf(bf16lo(q.x), cf, ra[0]);
                     ra[1] = fmaf(bf16hi(q.x), cf, ra[1]);
@@ -372,7 +373,7 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
             uint32_t a[4];
-            ldsm_x4(rdaddr + rd_off(16u * mt + arow, 16u * (uint32_t)(mi >> 1)), a);
+            ldsm_x4(rdaddr + (uint32_t)(mi >> 1) * 2048u + (16u * mt + arow) * 16u, a);
             int d[4] = {0, 0, 0, 0};
             mma_s8u8(d, a, b);
             // |d| <= 32 * 128 * 255, so hi * 256 + lo is exact in int32
