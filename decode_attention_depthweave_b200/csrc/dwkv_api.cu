@@ -17,6 +17,9 @@ __global__ void place_kernel(const Geom, const State, const AppendCall, const ui
 template <int BITS>
 __global__ void encode_kernel(const Geom, const State, const AppendCall, const __nv_bfloat16*, const __nv_bfloat16*);
 template <int BITS>
+__global__ void append_small_kernel(const Geom, const State, const AppendCall, const uint8_t*, int,
+                                    const __nv_bfloat16*, const __nv_bfloat16*);
+template <int BITS>
 __global__ void import_kernel(const Geom, const State, const AppendCall, const __nv_bfloat16*, const uint8_t*,
                               const int8_t*, const __half*);
 template <int BITS>
@@ -240,7 +243,7 @@ State make_state(uint8_t* arena, const MetaLayout& M, size_t arena_bytes) {
 }
 
 size_t encode_smem(const Geom& G) {
-    return (size_t)2 * kD * (G.r_max + 2) * 2 + (size_t)8 * (2 * kD + 2 * G.r_max + 64) * 4;
+    return (size_t)2 * kD * (G.r_max + 2) * 2 + (size_t)8 * (kD + kMaxRank + 32) * 4;
 }
 
 // Bytes of the decode page ring: what the shared-memory budget leaves after the fixed
@@ -418,9 +421,15 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
                      (const void*)decode_kernel<B, P, 128, 16>, (const void*)decode_kernel<B, P, 128, 32>
             DWKV_K(4, false), DWKV_K(4, true), DWKV_K(8, false), DWKV_K(8, true),
 #undef DWKV_K
-            (const void*)encode_kernel<8>, (const void*)encode_kernel<4>};
+        };
         for (const void* k : kernels)
             if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
+        // the encode kernels ask for what they use (the fused append also has static smem)
+        const int es = (int)encode_smem(G);
+        const void* enc[] = {(const void*)encode_kernel<8>, (const void*)encode_kernel<4>,
+                             (const void*)append_small_kernel<8>, (const void*)append_small_kernel<4>};
+        for (const void* k : enc)
+            if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, es);
     }
     if (e != cudaSuccess) {
         delete h;
@@ -495,13 +504,32 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
     const Geom& G = h->geom;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     bool any = false;
-    for (int i = 0; i < C.n; ++i) any |= C.na[i] > 0;
+    int most = 0;
+    for (int i = 0; i < C.n; ++i) {
+        any |= C.na[i] > 0;
+        most = std::max(most, n_new[i]);
+    }
+    const size_t sm = encode_smem(G);
+    if (most <= 4) {
+        // decode-sized append: placement and encode in one launch, a block per (sequence, kv-head)
+        const dim3 grid(C.n, G.Hkv);
+        if (G.bits == 8)
+            append_small_kernel<8><<<grid, 256, sm, s>>>(G, h->st, C, tier_idx, any ? 1 : 0,
+                                                         static_cast<const __nv_bfloat16*>(k_new),
+                                                         static_cast<const __nv_bfloat16*>(v_new));
+        else
+            append_small_kernel<4><<<grid, 256, sm, s>>>(G, h->st, C, tier_idx, any ? 1 : 0,
+                                                         static_cast<const __nv_bfloat16*>(k_new),
+                                                         static_cast<const __nv_bfloat16*>(v_new));
+        DWKV_CUDA(cudaGetLastError(), "append_small_kernel launch");
+        commit_call(h, C, n_new);
+        return DWKV_OK;
+    }
     if (any) {
         place_kernel<<<dim3(C.n, G.Hkv), 256, 0, s>>>(G, h->st, C, tier_idx);
         DWKV_CUDA(cudaGetLastError(), "place_kernel launch");
     }
-    const dim3 grid(grid_rows(h, C.total), G.Hkv);
-    const size_t sm = encode_smem(G);
+    const dim3 grid(grid_rows(h, 2ll * C.total), G.Hkv);     // a warp per (row, keys or values)
     if (G.bits == 8)
         encode_kernel<8><<<grid, 256, sm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
                                                 static_cast<const __nv_bfloat16*>(v_new));

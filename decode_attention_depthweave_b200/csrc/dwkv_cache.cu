@@ -20,11 +20,11 @@ namespace dwkv {
 // (sequence in call, kv-head).  Slots inside a tier are numbered in position order; new
 // pages come from the tier's free ring first, then from the pool's bump pointer.
 // ------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) place_kernel(const Geom G, const State S, const AppendCall C,
-                                                    const uint8_t* __restrict__ tier_idx) {
-    const int i = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ __forceinline__ void place_block(const Geom& G, const State& S, const AppendCall& C,
+                                            const uint8_t* __restrict__ tier_idx, int i, int h) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int na = C.na[i];
-    if (na <= 0) return;
+    if (na <= 0) return;                     // uniform across the block
     const int seq = C.seq[i], a0 = C.a0[i];
     const int rowbase = C.tok0[i] + (a0 - C.pos0[i]);
     __shared__ uint32_t s_cnt[kMaxTiers], s_old[kMaxTiers], s_run[kMaxTiers], s_fail;
@@ -114,6 +114,11 @@ __global__ void __launch_bounds__(256) place_kernel(const Geom G, const State S,
     if (tid < G.ntiers) S.counts[ci + tid] = s_old[tid] + s_cnt[tid];
 }
 
+__global__ void __launch_bounds__(256) place_kernel(const Geom G, const State S, const AppendCall C,
+                                                    const uint8_t* __restrict__ tier_idx) {
+    place_block(G, S, C, tier_idx, blockIdx.x, blockIdx.y);
+}
+
 // Row of the call's input arrays -> (index in call, sequence, position).
 __device__ __forceinline__ int call_index_of(const AppendCall& C, int row) {
     int lo = 0, hi = C.n - 1;
@@ -144,35 +149,64 @@ __device__ __forceinline__ bool find_dest(const Geom& G, const State& S, int seq
 }
 
 // ------------------------------------------------------------------------------------
-// Encode kernel: one warp per token (keys and values together), block per kv-head slice.
-// The (group, kv-head) bases sit in shared memory as bf16 with a padded row pitch so that
-// both the projection (lanes along j) and the residual (lanes along i) are conflict-free.
+// Encode kernel: one warp per (token row, keys or values): unit u = 2 row + z.  The block
+// holds both bases of its (group, kv-head) in shared memory as bf16 with a padded row pitch,
+// so that the projection (lanes along j) and the residual (lanes along i) are conflict-free.
+// A single appended token therefore runs its keys and values on two warps side by side.
 // ------------------------------------------------------------------------------------
-template <int BITS>
-__global__ void __launch_bounds__(256) encode_kernel(const Geom G, const State S, const AppendCall C,
-                                                     const __nv_bfloat16* __restrict__ k_new,
-                                                     const __nv_bfloat16* __restrict__ v_new) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int RM = G.r_max, P = G.r_max + 2, s = G.s;
-    __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem);              // [2][d][P]
-    float* ws_all = reinterpret_cast<float*>(smem + (size_t)2 * kD * P * 2);  // per warp
-    const int wfl = 2 * kD + 2 * RM;                                          // floats per warp
-    float* xs = ws_all + (size_t)warp * (wfl + 64);      // [2][d]
-    float* cs = xs + 2 * kD;                             // [2][r_max]
-    int8_t* cstage = reinterpret_cast<int8_t*>(cs + 2 * RM);  // [2][128] code staging
-
-    const size_t boff = ((size_t)C.g * G.Hkv + h) * kD * RM;
-    for (int e = tid; e < kD * RM; e += blockDim.x) {
-        const int i = e / RM, j = e % RM;
-        bs[i * P + j] = S.basis_k[boff + e];
-        bs[kD * P + i * P + j] = S.basis_v[boff + e];
+// Both bases of the block's (group, kv-head) into shared memory: [2][d][P] bf16 with P = r_max + 2.
+// 16-byte loads, all of a thread's requests in flight before its stores.
+__device__ __forceinline__ void load_bases(const Geom& G, const State& S, int g, int h, __nv_bfloat16* bs) {
+    const int tid = threadIdx.x, RM = G.r_max, P = G.r_max + 2;
+    const size_t boff = ((size_t)g * G.Hkv + h) * kD * RM;
+    const int nvec = kD * RM / 8;                         // uint4 per basis
+    const uint4* srck = reinterpret_cast<const uint4*>(S.basis_k + boff);
+    const uint4* srcv = reinterpret_cast<const uint4*>(S.basis_v + boff);
+    constexpr int kBatch = 8;
+    for (int e0 = tid; e0 < 2 * nvec; e0 += kBatch * (int)blockDim.x) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int e = e0 + b * (int)blockDim.x;
+            v[b] = e < 2 * nvec ? __ldg(e < nvec ? srck + e : srcv + (e - nvec)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int e = e0 + b * (int)blockDim.x;
+            if (e >= 2 * nvec) break;
+            const int z = e >= nvec, ev = z ? e - nvec : e;
+            const int i = (ev * 8) / RM, j = (ev * 8) % RM;
+            uint32_t* dst = reinterpret_cast<uint32_t*>(bs + (size_t)z * kD * P + (size_t)i * P + j);
+            dst[0] = v[b].x; dst[1] = v[b].y; dst[2] = v[b].z; dst[3] = v[b].w;
+        }
     }
-    __syncthreads();
+}
 
+// Shared-memory scratch of one encode warp: x [d], stored coefficients [kMaxRank], code staging.
+struct EncScratch {
+    float* xs;
+    float* cs;
+    int8_t* cstage;
+};
+__device__ __forceinline__ EncScratch enc_scratch(const Geom& G, uint8_t* smem, int warp) {
+    float* xs = reinterpret_cast<float*>(smem + (size_t)2 * kD * (G.r_max + 2) * 2) + (size_t)warp * (kD + kMaxRank + 32);
+    return {xs, xs + kD, reinterpret_cast<int8_t*>(xs + kD + kMaxRank)};
+}
+
+// One encode unit (token row, keys z = 0 or values z = 1) on one warp.
+template <int BITS>
+__device__ __forceinline__ void encode_unit(const Geom& G, const State& S, const AppendCall& C,
+                                            const __nv_bfloat16* __restrict__ k_new,
+                                            const __nv_bfloat16* __restrict__ v_new,
+                                            const __nv_bfloat16* bs, const EncScratch& W, int h, int unit) {
+    const int lane = threadIdx.x & 31;
+    const int P = G.r_max + 2, s = G.s;
+    float* xs = W.xs;
+    float* cs = W.cs;
+    int8_t* cstage = W.cstage;
     const float qmax = BITS == 8 ? 127.f : 7.f;
-    const int nw = blockDim.x >> 5;
-    for (int row = blockIdx.x * nw + warp; row < C.total; row += gridDim.x * nw) {
+    do {
+        const int row = unit >> 1, z = unit & 1;
         const int ci = call_index_of(C, row);
         const int seq = C.seq[ci];
         const int pos = C.pos0[ci] + (row - C.tok0[ci]);
@@ -180,98 +214,98 @@ __global__ void __launch_bounds__(256) encode_kernel(const Geom G, const State S
         if (!find_dest(G, S, seq, C.g, C.lig, h, pos, dst)) {
             // a0..a0+na were placed by place_kernel; a zero entry means placement failed
             // (already reported) or the group never placed this position.
-            if (lane == 0 && !(pos >= C.a0[ci] && pos < C.a0[ci] + C.na[ci]))
+            if (lane == 0 && z == 0 && !(pos >= C.a0[ci] && pos < C.a0[ci] + C.na[ci]))
                 set_dev_error(S, 5u /*DWKV_DEV_NO_SLOT*/, (uint32_t)seq, (uint32_t)pos);
-            continue;
+            break;
         }
         const int R = dst.R;
-        // ---- load x (keys at z=0, values at z=1)
-        float xr[2][4];
-        const __nv_bfloat16* src[2] = {k_new + ((size_t)row * G.Hkv + h) * kD,
-                                       v_new + ((size_t)row * G.Hkv + h) * kD};
-#pragma unroll
-        for (int z = 0; z < 2; ++z)
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                xr[z][m] = __bfloat162float(src[z][lane + 32 * m]);
-                xs[z * kD + lane + 32 * m] = xr[z][m];
-            }
-        __syncwarp();
-        // ---- 1-2: projection, bf16 rounding, coefficient store
-        for (int j = lane; j < R; j += 32) {
-            float a0 = 0.f, a1 = 0.f;
-            const __nv_bfloat16* b0 = bs + j;
-            const __nv_bfloat16* b1 = bs + kD * P + j;
-#pragma unroll 8
-            for (int i = 0; i < kD; ++i) {
-                a0 = __fmaf_rn(__bfloat162float(b0[i * P]), xs[i], a0);
-                a1 = __fmaf_rn(__bfloat162float(b1[i * P]), xs[kD + i], a1);
-            }
-            const __nv_bfloat16 c0 = __float2bfloat16_rn(a0), c1 = __float2bfloat16_rn(a1);
-            cs[j] = __bfloat162float(c0);
-            cs[RM + j] = __bfloat162float(c1);
-            const size_t co = (size_t)(j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2;
-            *reinterpret_cast<__nv_bfloat16*>(dst.blk + co) = c0;
-            *reinterpret_cast<__nv_bfloat16*>(dst.blk + G.blk_bytes[dst.k] + co) = c1;
-        }
-        __syncwarp();
-        // ---- 3: residual against the stored coefficients
-        float r[2][4];
+        const __nv_bfloat16* bz = bs + (size_t)z * kD * P;
+        uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
+        // ---- x (channel lane + 32 m)
+        float xr[4];
+        const __nv_bfloat16* src = (z ? v_new : k_new) + ((size_t)row * G.Hkv + h) * kD;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            const int i = lane + 32 * m;
-            float a0 = 0.f, a1 = 0.f;
-            const __nv_bfloat16* b0 = bs + i * P;
-            const __nv_bfloat16* b1 = bs + kD * P + i * P;
-            for (int j = 0; j < R; ++j) {
-                a0 = __fmaf_rn(__bfloat162float(b0[j]), cs[j], a0);
-                a1 = __fmaf_rn(__bfloat162float(b1[j]), cs[RM + j], a1);
+            xr[m] = __bfloat162float(src[lane + 32 * m]);
+            xs[lane + 32 * m] = xr[m];
+        }
+        __syncwarp();
+        // ---- 1-2: projection (fma chain over i from +0), bf16 rounding, coefficient store.
+        //      Lane takes j = lane + 32 jj; the chains of one lane run interleaved.
+        {
+            float acc[kMaxRank / 32];
+#pragma unroll
+            for (int jj = 0; jj < kMaxRank / 32; ++jj) acc[jj] = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < kD; ++i) {
+                const float xi = xs[i];
+                const __nv_bfloat16* brow = bz + (size_t)i * P + lane;
+#pragma unroll
+                for (int jj = 0; jj < kMaxRank / 32; ++jj)
+                    if (lane + 32 * jj < R) acc[jj] = __fmaf_rn(__bfloat162float(brow[32 * jj]), xi, acc[jj]);
             }
-            r[0][m] = __fsub_rn(xr[0][m], a0);
-            r[1][m] = __fsub_rn(xr[1][m], a1);
+#pragma unroll
+            for (int jj = 0; jj < kMaxRank / 32; ++jj) {
+                const int j = lane + 32 * jj;
+                if (j < R) {
+                    const __nv_bfloat16 cb = __float2bfloat16_rn(acc[jj]);
+                    cs[j] = __bfloat162float(cb);
+                    *reinterpret_cast<__nv_bfloat16*>(blk + (size_t)(j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2) = cb;
+                }
+            }
+        }
+        __syncwarp();
+        // ---- 3: residual against the stored coefficients (fma chain over j from +0)
+        float r[4];
+        {
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int j0 = 0; j0 < R; j0 += 8) {           // R is a multiple of 8
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const float cj = cs[j0 + jj];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        a[m] = __fmaf_rn(__bfloat162float(bz[(size_t)(lane + 32 * m) * P + j0 + jj]), cj, a[m]);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) r[m] = __fsub_rn(xr[m], a[m]);
         }
         // ---- 4: top-s by magnitude, ties to the lower channel (channel = lane + 32 m)
-        uint32_t key[2][4], sel[2] = {0u, 0u};
+        uint32_t key[4], sel = 0u;
 #pragma unroll
-        for (int z = 0; z < 2; ++z)
-#pragma unroll
-            for (int m = 0; m < 4; ++m) key[z][m] = __float_as_uint(fabsf(r[z][m])) + 1u;
+        for (int m = 0; m < 4; ++m) key[m] = __float_as_uint(fabsf(r[m])) + 1u;
         for (int it = 0; it < s; ++it) {
+            uint32_t best = 0u, bm = 0u;
 #pragma unroll
-            for (int z = 0; z < 2; ++z) {
-                uint32_t best = 0u, bm = 0u;
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    if (!((sel[z] >> m) & 1u) && key[z][m] > best) { best = key[z][m]; bm = (uint32_t)m; }
-                const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
-                const uint32_t cand = (best == wmax && best != 0u) ? (bm * 32u + (uint32_t)lane) : 0xffffffffu;
-                const uint32_t wch = __reduce_min_sync(0xffffffffu, cand);
-                if ((int)(wch & 31u) == lane) sel[z] |= 1u << (wch >> 5);
-            }
+            for (int m = 0; m < 4; ++m)
+                if (!((sel >> m) & 1u) && key[m] > best) { best = key[m]; bm = (uint32_t)m; }
+            const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
+            const uint32_t cand = (best == wmax && best != 0u) ? (bm * 32u + (uint32_t)lane) : 0xffffffffu;
+            const uint32_t wch = __reduce_min_sync(0xffffffffu, cand);
+            if ((int)(wch & 31u) == lane) sel |= 1u << (wch >> 5);
         }
         // ---- 5-6: scale and codes; ranks give ascending channel order
-#pragma unroll
-        for (int z = 0; z < 2; ++z) {
+        {
             uint32_t mx = 0u;
 #pragma unroll
             for (int m = 0; m < 4; ++m)
-                if ((sel[z] >> m) & 1u) mx = max(mx, key[z][m] - 1u);
+                if ((sel >> m) & 1u) mx = max(mx, key[m] - 1u);
             const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, mx));
             const __half sh = __float2half_rn(__fdiv_rn(amax, qmax));
             const float sf = __half2float(sh);
-            uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
             uint32_t before = 0u;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                const bool on = (sel[z] >> m) & 1u;
+                const bool on = (sel >> m) & 1u;
                 const uint32_t bal = __ballot_sync(0xffffffffu, on);
                 if (on) {
                     const int rank = (int)(before + __popc(bal & ((1u << lane) - 1u)));
                     float c = 0.f;
-                    if (sf != 0.f) c = fminf(fmaxf(rintf(__fdiv_rn(r[z][m], sf)), -qmax), qmax);
+                    if (sf != 0.f) c = fminf(fmaxf(rintf(__fdiv_rn(r[m], sf)), -qmax), qmax);
                     blk[off_idx_of(R) + dst.row * s + rank] = (uint8_t)(lane + 32 * m);
                     if (BITS == 8) blk[off_codes_of(R, s) + dst.row * s + rank] = (uint8_t)(int8_t)c;
-                    else cstage[z * 128 + rank] = (int8_t)c;
+                    else cstage[rank] = (int8_t)c;
                 }
                 before += __popc(bal);
             }
@@ -279,16 +313,57 @@ __global__ void __launch_bounds__(256) encode_kernel(const Geom G, const State S
         }
         if (BITS == 4) {
             __syncwarp();
-            for (int e = lane; e < s; e += 32) {        // e indexes (z, byte) pairs: s/2 bytes per z
-                const int z = e / (s / 2), b = e % (s / 2);
-                const uint8_t lo = (uint8_t)cstage[z * 128 + 2 * b] & 0xfu;
-                const uint8_t hi = (uint8_t)cstage[z * 128 + 2 * b + 1] & 0xfu;
-                uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
+            for (int b = lane; b < s / 2; b += 32) {
+                const uint8_t lo = (uint8_t)cstage[2 * b] & 0xfu;
+                const uint8_t hi = (uint8_t)cstage[2 * b + 1] & 0xfu;
                 blk[off_codes_of(R, s) + dst.row * (s / 2) + b] = (uint8_t)(lo | (hi << 4));
             }
         }
-        __syncwarp();
-    }
+    } while (false);
+    __syncwarp();
+}
+
+// ------------------------------------------------------------------------------------
+// Encode kernel: one warp per (token row, keys or values): unit u = 2 row + z.  The block
+// holds both bases of its (group, kv-head) in shared memory as bf16 with a padded row pitch,
+// so that the projection (lanes along j) and the residual (lanes along i) are conflict-free.
+// ------------------------------------------------------------------------------------
+template <int BITS>
+__global__ void __launch_bounds__(256) encode_kernel(const Geom G, const State S, const AppendCall C,
+                                                     const __nv_bfloat16* __restrict__ k_new,
+                                                     const __nv_bfloat16* __restrict__ v_new) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int h = blockIdx.y, warp = threadIdx.x >> 5;
+    __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem);
+    load_bases(G, S, C.g, h, bs);
+    __syncthreads();
+    const EncScratch W = enc_scratch(G, smem, warp);
+    const int nw = blockDim.x >> 5;
+    for (int unit = blockIdx.x * nw + warp; unit < 2 * C.total; unit += gridDim.x * nw)
+        encode_unit<BITS>(G, S, C, k_new, v_new, bs, W, h, unit);
+}
+
+// ------------------------------------------------------------------------------------
+// Decode-time append (a few tokens per sequence): one block per (sequence in call, kv-head)
+// places the sequence's new positions (when this layer is the group's first to append them)
+// and encodes its rows, in one launch.  The bases load while the placement runs.
+// ------------------------------------------------------------------------------------
+template <int BITS>
+__global__ void __launch_bounds__(256) append_small_kernel(const Geom G, const State S, const AppendCall C,
+                                                           const uint8_t* __restrict__ tier_idx, int place,
+                                                           const __nv_bfloat16* __restrict__ k_new,
+                                                           const __nv_bfloat16* __restrict__ v_new) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int i = blockIdx.x, h = blockIdx.y, warp = threadIdx.x >> 5;
+    __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem);
+    load_bases(G, S, C.g, h, bs);
+    if (place) place_block(G, S, C, tier_idx, i, h);
+    __syncthreads();                         // bases in smem; slots and pages written (block scope)
+    const EncScratch W = enc_scratch(G, smem, warp);
+    const int nw = blockDim.x >> 5;
+    const int u0 = 2 * C.tok0[i], u1 = 2 * C.tok0[i + 1];
+    for (int unit = u0 + warp; unit < u1; unit += nw)
+        encode_unit<BITS>(G, S, C, k_new, v_new, bs, W, h, unit);
 }
 
 // ------------------------------------------------------------------------------------
@@ -456,6 +531,10 @@ template __global__ void encode_kernel<8>(const Geom, const State, const AppendC
                                           const __nv_bfloat16*);
 template __global__ void encode_kernel<4>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
                                           const __nv_bfloat16*);
+template __global__ void append_small_kernel<8>(const Geom, const State, const AppendCall, const uint8_t*, int,
+                                                const __nv_bfloat16*, const __nv_bfloat16*);
+template __global__ void append_small_kernel<4>(const Geom, const State, const AppendCall, const uint8_t*, int,
+                                                const __nv_bfloat16*, const __nv_bfloat16*);
 template __global__ void import_kernel<8>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
                                           const uint8_t*, const int8_t*, const __half*);
 template __global__ void import_kernel<4>(const Geom, const State, const AppendCall, const __nv_bfloat16*,

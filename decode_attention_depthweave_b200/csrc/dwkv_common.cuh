@@ -32,6 +32,7 @@ constexpr int kGQ = 4;             // query heads per kv head supported by the k
 constexpr int kUnit = 128;         // page-pool granularity in bytes
 constexpr int kMaxTiers = 8;
 constexpr int kMaxSeqs = 256;      // sequences per call
+constexpr int kMaxRank = 128;      // largest r_max
 constexpr int kMaxSplits = 64;     // decode splits per (sequence, kv-head)
 constexpr int kConsumerWarps = 12; // each takes half pages (32 tokens) from a shared queue
 constexpr int kSlots = 32;          // page chunks in flight at most (one full / empty barrier pair each)

@@ -86,6 +86,20 @@ def test_chunked_appends_equal_one_shot():
                 assert torch.equal(x[key].view(torch.uint8), y[key].view(torch.uint8)), key
 
 
+def test_decode_sized_appends_bit_exact():
+    """Appends of 1-4 tokens per sequence take the one-launch place + encode path; the stored
+    bytes must equal the oracle's for every row, with sequences joining and leaving calls."""
+    wl = synth.workload("llama8b_ragged_b8").scaled(num_layers=2, num_q_heads=8, num_kv_heads=2, batch=3)
+    lengths = [23, 9, 30]
+    cache, bases, dense = _encode_case(wl, lengths, chunks=(1, 4, 2, 3, 1, 4, 4, 4, None))
+    for b, T in enumerate(lengths):
+        for layer in range(wl.num_layers):
+            got = cache.export(layer, b, 0, T)
+            tiers = dense[(b, "t", layer // wl.layers_per_group)]
+            ref = oracle_encode_rows(wl, bases, layer, dense[(b, layer)][0], dense[(b, layer)][1], tiers)
+            _assert_same(got, ref, tiers, f"small appends seq {b} layer {layer}")
+
+
 def test_exact_planted_vectors_and_zero_vectors():
     """Signed-permutation bases and planted residuals (every encoder step exact), and zero
     vectors (ties at zero go to the lowest channels)."""
