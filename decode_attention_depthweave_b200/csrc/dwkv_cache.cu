@@ -210,6 +210,11 @@ __device__ __forceinline__ void encode_unit(const Geom& G, const State& S, const
         const int ci = call_index_of(C, row);
         const int seq = C.seq[ci];
         const int pos = C.pos0[ci] + (row - C.tok0[ci]);
+        // ---- x (channel lane + 32 m), requested before the slot lookup so both are in flight
+        float xr[4];
+        const __nv_bfloat16* src = (z ? v_new : k_new) + ((size_t)row * G.Hkv + h) * kD;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) xr[m] = __bfloat162float(src[lane + 32 * m]);
         Dest dst;
         if (!find_dest(G, S, seq, C.g, C.lig, h, pos, dst)) {
             // a0..a0+na were placed by place_kernel; a zero entry means placement failed
@@ -221,14 +226,8 @@ __device__ __forceinline__ void encode_unit(const Geom& G, const State& S, const
         const int R = dst.R;
         const __nv_bfloat16* bz = bs + (size_t)z * kD * P;
         uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
-        // ---- x (channel lane + 32 m)
-        float xr[4];
-        const __nv_bfloat16* src = (z ? v_new : k_new) + ((size_t)row * G.Hkv + h) * kD;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            xr[m] = __bfloat162float(src[lane + 32 * m]);
-            xs[lane + 32 * m] = xr[m];
-        }
+        for (int m = 0; m < 4; ++m) xs[lane + 32 * m] = xr[m];
         __syncwarp();
         // ---- 1-2: projection (fma chain over i from +0), bf16 rounding, coefficient store.
         //      Lane takes j = lane + 32 jj; the chains of one lane run interleaved.
