@@ -182,6 +182,36 @@ __device__ __forceinline__ void load_bases(const Geom& G, const State& S, int g,
     }
 }
 
+// The same load in two steps, so that other global round trips overlap its latency: the
+// block's share of both bases into registers (at most 16 x 16 bytes a thread for 256
+// threads), then into shared memory.
+constexpr int kBasisRegs = 2 * kD * kMaxRank / 8 / 256;
+__device__ __forceinline__ void bases_issue(const Geom& G, const State& S, int g, int h, uint4 (&v)[kBasisRegs]) {
+    const int tid = threadIdx.x, RM = G.r_max;
+    const size_t boff = ((size_t)g * G.Hkv + h) * kD * RM;
+    const int nvec = kD * RM / 8;
+    const uint4* srck = reinterpret_cast<const uint4*>(S.basis_k + boff);
+    const uint4* srcv = reinterpret_cast<const uint4*>(S.basis_v + boff);
+#pragma unroll
+    for (int b = 0; b < kBasisRegs; ++b) {
+        const int e = tid + b * 256;
+        v[b] = e < 2 * nvec ? __ldg(e < nvec ? srck + e : srcv + (e - nvec)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+__device__ __forceinline__ void bases_store(const Geom& G, const uint4 (&v)[kBasisRegs], __nv_bfloat16* bs) {
+    const int tid = threadIdx.x, RM = G.r_max, P = G.r_max + 2;
+    const int nvec = kD * RM / 8;
+#pragma unroll
+    for (int b = 0; b < kBasisRegs; ++b) {
+        const int e = tid + b * 256;
+        if (e >= 2 * nvec) break;
+        const int z = e >= nvec, ev = z ? e - nvec : e;
+        const int i = (ev * 8) / RM, j = (ev * 8) % RM;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(bs + (size_t)z * kD * P + (size_t)i * P + j);
+        dst[0] = v[b].x; dst[1] = v[b].y; dst[2] = v[b].z; dst[3] = v[b].w;
+    }
+}
+
 // Shared-memory scratch of one encode warp: x [d], stored coefficients [kMaxRank], code staging.
 struct EncScratch {
     float* xs;
@@ -193,12 +223,37 @@ __device__ __forceinline__ EncScratch enc_scratch(const Geom& G, uint8_t* smem, 
     return {xs, xs + kD, reinterpret_cast<int8_t*>(xs + kD + kMaxRank)};
 }
 
-// One encode unit (token row, keys z = 0 or values z = 1) on one warp.
+// Inputs of one encode unit (token row, keys z = 0 or values z = 1): x (channel lane + 32 m)
+// and the destination block, both requested together.
+struct UnitIn {
+    Dest dst;
+    float xr[4];
+    bool ok;
+};
+__device__ __forceinline__ UnitIn encode_fetch(const Geom& G, const State& S, const AppendCall& C,
+                                               const __nv_bfloat16* __restrict__ k_new,
+                                               const __nv_bfloat16* __restrict__ v_new, int h, int unit) {
+    const int lane = threadIdx.x & 31;
+    const int row = unit >> 1, z = unit & 1;
+    const int ci = call_index_of(C, row);
+    const int seq = C.seq[ci];
+    const int pos = C.pos0[ci] + (row - C.tok0[ci]);
+    UnitIn in;
+    const __nv_bfloat16* src = (z ? v_new : k_new) + ((size_t)row * G.Hkv + h) * kD;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) in.xr[m] = __bfloat162float(src[lane + 32 * m]);
+    in.ok = find_dest(G, S, seq, C.g, C.lig, h, pos, in.dst);
+    // a0..a0+na were placed by the placement; a zero entry means placement failed (already
+    // reported) or the group never placed this position
+    if (!in.ok && lane == 0 && z == 0 && !(pos >= C.a0[ci] && pos < C.a0[ci] + C.na[ci]))
+        set_dev_error(S, 5u /*DWKV_DEV_NO_SLOT*/, (uint32_t)seq, (uint32_t)pos);
+    return in;
+}
+
+// The six encode steps of one unit on one warp.
 template <int BITS>
-__device__ __forceinline__ void encode_unit(const Geom& G, const State& S, const AppendCall& C,
-                                            const __nv_bfloat16* __restrict__ k_new,
-                                            const __nv_bfloat16* __restrict__ v_new,
-                                            const __nv_bfloat16* bs, const EncScratch& W, int h, int unit) {
+__device__ __forceinline__ void encode_body(const Geom& G, const State& S, const __nv_bfloat16* bs,
+                                            const EncScratch& W, int unit, const UnitIn& in) {
     const int lane = threadIdx.x & 31;
     const int P = G.r_max + 2, s = G.s;
     float* xs = W.xs;
@@ -206,23 +261,10 @@ __device__ __forceinline__ void encode_unit(const Geom& G, const State& S, const
     int8_t* cstage = W.cstage;
     const float qmax = BITS == 8 ? 127.f : 7.f;
     do {
-        const int row = unit >> 1, z = unit & 1;
-        const int ci = call_index_of(C, row);
-        const int seq = C.seq[ci];
-        const int pos = C.pos0[ci] + (row - C.tok0[ci]);
-        // ---- x (channel lane + 32 m), requested before the slot lookup so both are in flight
-        float xr[4];
-        const __nv_bfloat16* src = (z ? v_new : k_new) + ((size_t)row * G.Hkv + h) * kD;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) xr[m] = __bfloat162float(src[lane + 32 * m]);
-        Dest dst;
-        if (!find_dest(G, S, seq, C.g, C.lig, h, pos, dst)) {
-            // a0..a0+na were placed by place_kernel; a zero entry means placement failed
-            // (already reported) or the group never placed this position.
-            if (lane == 0 && z == 0 && !(pos >= C.a0[ci] && pos < C.a0[ci] + C.na[ci]))
-                set_dev_error(S, 5u /*DWKV_DEV_NO_SLOT*/, (uint32_t)seq, (uint32_t)pos);
-            break;
-        }
+        const int z = unit & 1;
+        if (!in.ok) break;
+        const Dest& dst = in.dst;
+        float xr[4] = {in.xr[0], in.xr[1], in.xr[2], in.xr[3]};
         const int R = dst.R;
         const __nv_bfloat16* bz = bs + (size_t)z * kD * P;
         uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
@@ -322,6 +364,15 @@ __device__ __forceinline__ void encode_unit(const Geom& G, const State& S, const
     __syncwarp();
 }
 
+template <int BITS>
+__device__ __forceinline__ void encode_unit(const Geom& G, const State& S, const AppendCall& C,
+                                            const __nv_bfloat16* __restrict__ k_new,
+                                            const __nv_bfloat16* __restrict__ v_new,
+                                            const __nv_bfloat16* bs, const EncScratch& W, int h, int unit) {
+    const UnitIn in = encode_fetch(G, S, C, k_new, v_new, h, unit);
+    encode_body<BITS>(G, S, bs, W, unit, in);
+}
+
 // ------------------------------------------------------------------------------------
 // Encode kernel: one warp per (token row, keys or values): unit u = 2 row + z.  The block
 // holds both bases of its (group, kv-head) in shared memory as bf16 with a padded row pitch,
@@ -355,14 +406,22 @@ __global__ void __launch_bounds__(256) append_small_kernel(const Geom G, const S
     extern __shared__ __align__(16) uint8_t smem[];
     const int i = blockIdx.x, h = blockIdx.y, warp = threadIdx.x >> 5;
     __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem);
-    load_bases(G, S, C.g, h, bs);
-    if (place) place_block(G, S, C, tier_idx, i, h);
-    __syncthreads();                         // bases in smem; slots and pages written (block scope)
-    const EncScratch W = enc_scratch(G, smem, warp);
-    const int nw = blockDim.x >> 5;
+    // The global round trips overlap: the bases, this warp's unit (x and, when nothing is
+    // placed, its destination) and the placement are all in flight together.
+    uint4 bv[kBasisRegs];
+    bases_issue(G, S, C.g, h, bv);
     const int u0 = 2 * C.tok0[i], u1 = 2 * C.tok0[i + 1];
-    for (int unit = u0 + warp; unit < u1; unit += nw)
-        encode_unit<BITS>(G, S, C, k_new, v_new, bs, W, h, unit);
+    const int unit = u0 + warp;                    // at most 4 rows: one unit per warp
+    UnitIn in;
+    in.ok = false;
+    if (!place && unit < u1) in = encode_fetch(G, S, C, k_new, v_new, h, unit);
+    if (place) place_block(G, S, C, tier_idx, i, h);
+    bases_store(G, bv, bs);
+    __syncthreads();                         // bases in smem; slots and pages written (block scope)
+    if (unit < u1) {
+        if (place) in = encode_fetch(G, S, C, k_new, v_new, h, unit);
+        encode_body<BITS>(G, S, bs, enc_scratch(G, smem, warp), unit, in);
+    }
 }
 
 // ------------------------------------------------------------------------------------

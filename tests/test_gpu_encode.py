@@ -229,3 +229,34 @@ def test_cuda_graph_replay_of_append_and_decode():
         ref = oracle.decode_head(head_problem(wl, bases, tiers, comp, qs[0], 1, 0))
         check_close(out[0].cpu().numpy(), ref, what=f"replay {step}")
     cache.sync()
+
+
+def test_decode_right_after_one_token_appends_across_page_boundaries():
+    """The decode launched right after a one-token append may start while the append runs
+    (it waits for the placement's counts and reads each tier's last page after the append
+    completes).  Step through page boundaries of every tier, eagerly, checking each step."""
+    wl = synth.workload("tiny_1k")
+    bases = synth.make_bases(wl)
+    T0, steps = 160, 24
+    cache = dw.Cache(cfg_for(wl, max_context=T0 + steps + 8), bases[0], bases[1])
+    from helpers import import_workload
+    data = import_workload(cache, wl, [T0])
+    newk = [synth.make_dense_vectors(wl, 0, l, steps, bases, start=T0) for l in range(2)]
+    newt = synth.make_tiers(wl, 0, 0, steps, start=T0)
+    qs = synth.make_queries(wl, 1, temperature=8.0)
+    tiers, comp = data[(0, 1)]
+    pages0 = [(int((tiers == k).sum()) + 63) // 64 for k in range(len(wl.tiers))]
+    for step in range(steps):
+        for layer in range(2):
+            cache.append(layer, [0], [1], newk[layer][0][step:step + 1].cuda(), newk[layer][1][step:step + 1].cuda(),
+                         newt[step:step + 1].cuda() if layer == 0 else None)
+        out = cache.decode(1, [0], qs.cuda())
+        cache.sync()
+        new = oracle_encode_rows(wl, bases, 1, newk[1][0][step:step + 1], newk[1][1][step:step + 1],
+                                 newt[step:step + 1])
+        tiers = torch.cat([tiers, newt[step:step + 1]])
+        comp = cat_comp(comp, new)
+        ref = oracle.decode_head(head_problem(wl, bases, tiers, comp, qs[0], 1, 0))
+        check_close(out[0].cpu().numpy(), ref, what=f"step {step}")
+    pages1 = [(int((tiers == k).sum()) + 63) // 64 for k in range(len(wl.tiers))]
+    assert pages1 != pages0, "the steps should have opened a new page in some tier"
