@@ -5,28 +5,29 @@
 // never writing reconstructed keys / values (Eq. (1) evaluated inside attention); the
 // probe is Eq. (3) with the with-residual output as the reference.
 //
-// For the 4 query heads q_h of kv-head h (tau * log2 e folded into q so exp2 can be used):
+// For the 4 query heads q_h of kv-head h (tau * log2 e folded in, so exp2 can be used):
 //   qt = B_K^T q                                   (once per CTA, B_K bulk-copied to smem)
 //   s_t = qt[:r_t] . c^K_t + scale^K_t sum_i q[idx^K_ti] code^K_ti
 //   online softmax over t;  acc_c += C^V^T p (coefficient space);
 //   acc_r += R^V^T (p * scale^V) (residual space, R^V the dense residual codes)
-//   o = (B_V acc_c + acc_r) / l                   (B_V applied once, in the combine)
+//   o = (B_V acc_c + acc_r) / l                   (B_V applied once per CTA)
 //
 // Tensor cores take the dense, tier-homogeneous coefficient blocks: the page's 64 x r_t
-// coefficient tile against q~ (scores) and against p (values), and the value residual
-// after it is expanded into a dense 128-channel x 16-token tile in shared memory.  The
-// operands that are not exact in bf16 (q~, p, p * scale) are split into bf16 hi + lo
-// halves (two MMA columns each), so products keep ~15 significant bits and accumulate in
-// fp32.  The key residual is a gather-dot on the CUDA cores.
+// coefficient tile against q~ (scores) and against p (values), with q~ and p split into bf16
+// hi + lo halves (two MMA columns each), so products keep ~16 significant bits and accumulate
+// in fp32.  The value residual is expanded into a dense int8 tile [128 channels x 32 tokens]
+// and multiplied by the weights p * scale^V held as 16-bit fixed point (two byte limbs per
+// head, relative to the half page's largest weight) with integer MMAs.  The key residual is
+// a gather-dot on the CUDA cores (lane = token) from a bf16 table of q.
 //
 // Work split: a CTA takes a cost-balanced run of one (sequence, kv-head)'s pages (pages are
-// tier-homogeneous; tiers are visited in order; a page costs its bytes plus a per-token
-// weight).  Warp 8 lane 0 builds the CTA's page table and streams page chunks into a ring
-// of shared-memory stages with cp.async.bulk (no multicast).  Warps 0-7 form 4 pairs; pair p
-// consumes every 4th page and each warp of the pair takes 32 of its 64 tokens with its own
-// softmax state.  The CTA merges its 8 states into one partial record, and the last CTA of
-// the (sequence, kv-head) (atomic ticket, no waiting) merges all records and writes the
-// output.
+// tier-homogeneous; a page costs its bytes plus a per-token weight), visited from the highest
+// tier down.  The producer warp (lane 0) places the page chunks back to back in a byte ring
+// of shared memory with cp.async.bulk (no multicast); its 32 lanes resolve page ids a batch
+// ahead.  The 12 consumer warps take half pages (32 tokens) from a shared counter, each with
+// its own softmax state.  The CTA merges its warps' states into one partial record {M, L, o},
+// and the last CTA of the (sequence, kv-head) (atomic ticket, no waiting) merges the records
+// and writes the output.
 #pragma once
 #include "dwkv_common.cuh"
 
@@ -69,13 +70,6 @@ __device__ __forceinline__ void mma_s8u8(int (&d)[4], const uint32_t (&a)[4], co
         "{%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // x ~= hi + lo with both halves bf16, rounding to nearest (prologue only)
