@@ -175,9 +175,12 @@ def dist_setup():
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:                                        # host-side runs of the same plumbing
+            dist.init_process_group("gloo", timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
@@ -194,9 +197,15 @@ def max_over_ranks(world, value: float) -> float:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (ms * 1e-3)
 
 
 # ----------------------------------------------------------------------------- oracle sample
@@ -397,7 +406,7 @@ def run_dwkv(args, world, rank, local):
         h2d = sK[0].numel() * 2 + sV[0].numel() * 2 + sQ[0].numel() * 2 + sT[0].numel()
         d2h = out.numel() * 4
         assert torch.isfinite(host_out).all()
-        e2e = {"value": round(world * B / (e2e_ms * 1e-3), 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        e2e = {"value": round(aggregate_rate(world, B, e2e_ms), 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms, 4)}
     cache.sync(stream)
 
@@ -412,7 +421,7 @@ def run_dwkv(args, world, rank, local):
                "sample": f"layer 0, {n_items} kv-heads x {T - 1} cached tokens (fp64 C oracle, {dt:.1f} s wall "
                          f"on {threads} threads), scaled x{wl.num_layers} layers to one step"}
 
-    value = world * B / (ms_per_step * 1e-3)
+    value = aggregate_rate(world, B, ms_per_step)
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
