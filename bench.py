@@ -65,7 +65,7 @@ def measured_peaks() -> dict:
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("dwkv_decode.cuh", "dwkv_common.cuh"):
+    for f in ("dwkv_decode.cuh", "dwkv_common.cuh", "dwkv_encode.cuh"):
         h.update(open(os.path.join(ROOT, "decode_attention_depthweave_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 

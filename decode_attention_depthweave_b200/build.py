@@ -17,7 +17,7 @@ OUT_DIR = os.path.join(HERE, "_lib")
 LIB = os.path.join(OUT_DIR, "libdwkv.so")
 SOURCES = ["dwkv_api.cu", "dwkv_cache.cu", "dwkv_decode_b4.cu", "dwkv_decode_b4p.cu", "dwkv_decode_b8.cu",
            "dwkv_decode_b8p.cu"]
-HEADERS = ["dwkv_common.cuh", "dwkv_decode.cuh"]
+HEADERS = ["dwkv_common.cuh", "dwkv_decode.cuh", "dwkv_encode.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
