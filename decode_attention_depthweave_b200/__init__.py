@@ -21,7 +21,8 @@ __all__ = [
     "dwkv_arena_bytes", "dwkv_workspace_bytes", "dwkv_create", "dwkv_destroy",
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage",
-    "dwkv_sync_status", "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "Cache", "EXPORTED_SYMBOLS",
+    "dwkv_sync_status", "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
+    "Cache", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -36,7 +37,7 @@ EXPORTED_SYMBOLS = (
     "dwkv_metadata_bytes", "dwkv_arena_bytes", "dwkv_workspace_bytes", "dwkv_create", "dwkv_destroy",
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage", "dwkv_sync_status",
-    "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc",
+    "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
 )
 
 
@@ -90,6 +91,7 @@ def lib():
             "dwkv_append": ([vp, i32, i32, vp, vp, vp, vp, vp, vp], C.c_int),
             "dwkv_append_compressed": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], C.c_int),
             "dwkv_decode_attention": ([vp, i32, i32, vp, vp, vp, vp, sz, vp], C.c_int),
+            "dwkv_append_decode_attention": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
             "dwkv_probe": ([vp, i32, i32, vp, vp, vp, vp, vp, sz, vp], C.c_int),
             "dwkv_export": ([vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], C.c_int),
             "dwkv_pool_usage": ([vp, vp, C.POINTER(dwkv_pool_stats)], C.c_int),
@@ -217,6 +219,12 @@ def dwkv_decode_attention(h, layer, seq_ids, q, out, workspace, stream=None):
                                        _stream(stream)))
 
 
+def dwkv_append_decode_attention(h, layer, seq_ids, k_new, v_new, tier_idx, q, out, workspace, stream=None):
+    _check(lib().dwkv_append_decode_attention(h, layer, len(seq_ids), _i32(seq_ids), _ptr(k_new), _ptr(v_new),
+                                              _ptr(tier_idx), _ptr(q), _ptr(out), _ptr(workspace),
+                                              workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def dwkv_decode_attention_noalloc(h, layer, seq_ids, q, out, stream=None):
     _check(lib().dwkv_decode_attention_noalloc(h, layer, len(seq_ids), _i32(seq_ids), _ptr(q), _ptr(out),
                                                _stream(stream)))
@@ -287,6 +295,13 @@ class Cache:
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
         dwkv_decode_attention(self.h, layer, seq_ids, q, out, self.workspace, stream)
+        return out
+
+    def append_decode(self, layer, seq_ids, k_new, v_new, tier_idx, q, out=None, stream=None):
+        """One new token per sequence appended and attended in one launch."""
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        dwkv_append_decode_attention(self.h, layer, seq_ids, k_new, v_new, tier_idx, q, out, self.workspace, stream)
         return out
 
     def probe(self, layer, seq_ids, q, want_out=False, stream=None):

@@ -194,6 +194,7 @@ struct dwkv_ctx {
     std::vector<int32_t> placed;    // [max_batch][G]
     int dec_ctas_per_sm = 1, dec_waves = 1, dec_stages_req = 0;
     int dec_tok_weight = 1024;      // split balance: byte-equivalent cost of one token
+    int dec_owner_share = 192;      // fused append: the encoding CTA's share of a split, of 256
 };
 
 namespace {
@@ -571,9 +572,23 @@ dwkv_status dwkv_append_compressed(dwkv_handle h, int32_t layer, int32_t n_seqs,
     return DWKV_OK;
 }
 
+// One new token per sequence appended by the decode launch itself (see the decode kernel).
+struct FusedAppend {
+    const void* k_new;
+    const void* v_new;
+    const uint8_t* tier_idx;
+    const AppendCall* call;          // positions and which sequences this layer places
+};
+
+// Shared memory the fused append borrows from the page ring: both bases with padded rows,
+// and two encode warps' scratch.
+size_t fused_ring_need(const Geom& G) {
+    return (size_t)2 * kD * (G.r_max + 2) * 2 + (size_t)2 * (kD + kMaxRank + 32) * 4;
+}
+
 static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const void* q,
                               float* out, float* err, float* out_full, void* workspace, size_t ws_bytes,
-                              void* stream, bool probe) {
+                              void* stream, bool probe, const FusedAppend* fa = nullptr) {
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
     if ((st = check_layer(h, layer)) != DWKV_OK) return st;
@@ -623,6 +638,18 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     C.ring_bytes = (int)ring;
     C.rec_floats = rec_floats_of(G, probe);
     C.tok_weight = h->dec_tok_weight;
+    C.owner_share = 256;
+    if (fa) {
+        C.fused = 1;
+        C.owner_share = h->dec_owner_share;
+        C.k_new = static_cast<const __nv_bfloat16*>(fa->k_new);
+        C.v_new = static_cast<const __nv_bfloat16*>(fa->v_new);
+        C.tier_idx = fa->tier_idx;
+        for (int i = 0; i < n_seqs; ++i) {
+            C.pos[i] = fa->call->pos0[i];
+            C.place[i] = fa->call->na[i] > 0 ? 1 : 0;
+        }
+    }
     C.q = static_cast<const __nv_bfloat16*>(q);
     C.out = out;
     C.out_full = out_full;
@@ -660,6 +687,36 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
 dwkv_status dwkv_decode_attention(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
                                   const void* q, float* out, void* workspace, size_t ws_bytes, void* stream) {
     return run_decode(h, layer, n_seqs, seq_ids, q, out, nullptr, nullptr, workspace, ws_bytes, stream, false);
+}
+
+dwkv_status dwkv_append_decode_attention(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                                         const void* k_new, const void* v_new, const uint8_t* tier_idx,
+                                         const void* q, float* out, void* workspace, size_t ws_bytes,
+                                         void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if ((st = check_layer(h, layer)) != DWKV_OK) return st;
+    if (n_seqs < 0 || n_seqs > kMaxSeqs) return fail(DWKV_ERR_INVALID_ARG, "n_seqs %d out of range", n_seqs);
+    if (n_seqs == 0) return DWKV_OK;
+    if (!k_new || !v_new) return fail(DWKV_ERR_INVALID_ARG, "k_new and v_new must be non-NULL");
+    if (!q || !out || !workspace) return fail(DWKV_ERR_INVALID_ARG, "q, out and workspace must be non-NULL");
+    if (reinterpret_cast<uintptr_t>(workspace) % 16) return fail(DWKV_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    const size_t need = dwkv_workspace_bytes(&h->cfg, n_seqs);
+    if (ws_bytes < need) return fail(DWKV_ERR_CAPACITY, "workspace of %zu bytes is below the %zu needed", ws_bytes, need);
+    std::vector<int32_t> ones((size_t)n_seqs, 1);
+    AppendCall A;
+    if ((st = prepare_call(h, layer, n_seqs, seq_ids, ones.data(), A, true, tier_idx)) != DWKV_OK) return st;
+    const Geom& G = h->geom;
+    size_t smem = 0;
+    if (decode_ring_for(h, false, &smem) < fused_ring_need(G)) {
+        // the ring is capped below what the fused append borrows: two launches instead
+        if ((st = dwkv_append(h, layer, n_seqs, seq_ids, ones.data(), k_new, v_new, tier_idx, stream)) != DWKV_OK)
+            return st;
+        return dwkv_decode_attention(h, layer, n_seqs, seq_ids, q, out, workspace, ws_bytes, stream);
+    }
+    commit_call(h, A, ones.data());          // the decode below attends to the new positions
+    const FusedAppend fa{k_new, v_new, tier_idx, &A};
+    return run_decode(h, layer, n_seqs, seq_ids, q, out, nullptr, nullptr, workspace, ws_bytes, stream, false, &fa);
 }
 
 dwkv_status dwkv_probe(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const void* q,

@@ -80,6 +80,15 @@ struct AppendCall {
 struct DecodeCall {
     int n, layer, g, lig, total_splits, ring_bytes, rec_floats;
     int tok_weight;          // split balance: cost of one token in byte-equivalents
+    // One new token per sequence appended in the same launch (0 = plain decode).  The first CTA
+    // of each (sequence, kv-head) places and encodes it and attends to it directly; every CTA
+    // attends to the pages without it.  `owner_share` (of 256) is that CTA's share of a split.
+    int fused, owner_share;
+    const __nv_bfloat16* k_new;      // [n][Hkv][d] bf16 (fused)
+    const __nv_bfloat16* v_new;
+    const uint8_t* tier_idx;         // [n][Hkv] tier of the new token (read where it is placed)
+    int pos[kMaxSeqs];               // the new token's position (fused)
+    uint8_t place[kMaxSeqs];         // 1: this layer places it (its group's first to append it)
     int seq[kMaxSeqs];
     int split_begin[kMaxSeqs + 1];
     const __nv_bfloat16* q;  // [n][Hq][d]
@@ -117,7 +126,7 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 //   bars    full[kSlots] empty[kSlots] basis table
 //   misc    tier table, page range, work counter; warp states; page-id batch; slot offsets
 struct DecodeSmem {
-    uint32_t ring, rd, small, small_stride, S, P, W, P2, qt, q, qh, zero, bars, misc, total;
+    uint32_t ring, rd, small, small_stride, S, P, W, P2, qt, q, qh, zero, bars, misc, tok, total;
 };
 constexpr uint32_t kMiscState = 256;                               // m_state [warps][16]
 constexpr uint32_t kMiscFactors = kMiscState + kConsumerWarps * 64; // mf [2][warps][4]
@@ -142,6 +151,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, uint32_t
     L.zero = o;    o += 128;
     L.bars = o;    o += (2 * kSlots + 2) * 8;
     L.misc = o;    o += (kMiscBytes + 127) & ~127u;
+    L.tok = o;     o += 64;                 // the new token's destination (fused append)
     L.total = (o + 127) & ~127u;
     return L;
 }

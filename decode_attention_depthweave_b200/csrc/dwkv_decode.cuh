@@ -29,7 +29,7 @@
 // and the last CTA of the (sequence, kv-head) (atomic ticket, no waiting) merges the records
 // and writes the output.
 #pragma once
-#include "dwkv_common.cuh"
+#include "dwkv_encode.cuh"
 
 namespace dwkv {
 
@@ -414,6 +414,158 @@ __device__ __forceinline__ void store_d(float (&d)[N][4], float* dst, int rows, 
     }
 }
 
+// The fused append's new token, as the CTA that placed and encoded it sees it.
+struct TokDest {
+    Dest d;
+    int ok;
+};
+
+// First CTA of a (sequence, kv-head) in a fused append: place the sequence's new position (when
+// this layer is its group's first to append it; the counts are left for the last CTA), then
+// encode the token's keys (warp 0) and values (warp 1) with both bases staged in the still
+// empty page ring.  All threads; ends with the CTA synchronised.
+template <int BITS>
+__device__ __forceinline__ void owner_append(const Geom& G, const State& St, const DecodeCall& C, int ci, int seq,
+                                             int h, uint8_t* ring, TokDest* td) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        Dest d{};
+        bool ok;
+        if (C.place[ci]) {
+            const uint32_t k = C.tier_idx[(size_t)ci * G.Hkv + h];
+            ok = k < (uint32_t)G.ntiers;
+            if (!ok) set_dev_error(St, 2u /*DWKV_DEV_BAD_TIER*/, (uint32_t)seq, (uint32_t)C.pos[ci]);
+            else ok = place_one(G, St, seq, C.g, h, C.pos[ci], k, d, C.lig);
+        } else {
+            ok = find_dest(G, St, seq, C.g, C.lig, h, C.pos[ci], d);
+            if (!ok) set_dev_error(St, 5u /*DWKV_DEV_NO_SLOT*/, (uint32_t)seq, (uint32_t)C.pos[ci]);
+        }
+        td->d = d;
+        td->ok = ok ? 1 : 0;
+    }
+    // both bases, padded rows, at the start of the ring
+    {
+        const int RM = G.r_max, P = G.r_max + 2;
+        const size_t boff = ((size_t)C.g * G.Hkv + h) * kD * RM;
+        const int nvec = kD * RM / 8;
+        const uint4* srck = reinterpret_cast<const uint4*>(St.basis_k + boff);
+        const uint4* srcv = reinterpret_cast<const uint4*>(St.basis_v + boff);
+        __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(ring);
+        for (int e = tid; e < 2 * nvec; e += blockDim.x) {
+            const uint4 v = __ldg(e < nvec ? srck + e : srcv + (e - nvec));
+            const int z = e >= nvec, ev = z ? e - nvec : e;
+            const int i = (ev * 8) / RM, j = (ev * 8) % RM;
+            uint32_t* dst = reinterpret_cast<uint32_t*>(bs + (size_t)z * kD * P + (size_t)i * P + j);
+            dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+        }
+    }
+    __syncthreads();
+    if (warp < 2 && td->ok) {
+        UnitIn in;
+        in.dst = td->d;
+        in.ok = true;
+        const __nv_bfloat16* src = (warp ? C.v_new : C.k_new) + ((size_t)ci * G.Hkv + h) * kD;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) in.xr[m] = __bfloat162float(src[lane + 32 * m]);
+        encode_body<BITS>(G, St, reinterpret_cast<const __nv_bfloat16*>(ring), enc_scratch(G, ring, warp), warp, in);
+    }
+    __syncthreads();
+}
+
+// Consumer warp 0 of that CTA, after its pages: attend to the new token from its stored bytes
+// (the score over its coefficients and residual, the online-softmax update, and its value in
+// both spaces), so no other CTA waits for it.
+template <int S, int BITS, int RMAX>
+__device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, const float4* qt, const float4* qs,
+                                              WarpAcc<RMAX, false>& A, int lane) {
+    const Dest& d = td.d;
+    const int R = d.R, row = d.row;
+    const uint32_t offIdx = off_idx_of(R), offCodes = off_codes_of(R, S), offSc = off_scales_of(R, S, BITS);
+    const uint8_t* Kb = d.blk;
+    const uint8_t* Vb = d.blk + G.blk_bytes[d.k];
+    auto coeff = [&](const uint8_t* blk, int j) {
+        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(blk + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2));
+    };
+    auto code = [&](const uint8_t* blk, int e) -> float {
+        if (BITS == 8) return (float)(int8_t)blk[offCodes + row * S + e];
+        const uint32_t b = blk[offCodes + row * (S / 2) + e / 2];
+        return (float)((int32_t)(b << (28 - 4 * (e & 1))) >> 28);
+    };
+    // score (log2 units: q~ and q carry tau log2 e)
+    float sc[kGQ] = {0.f, 0.f, 0.f, 0.f}, rs[kGQ] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = lane; j < R; j += 32) {
+        const float c = coeff(Kb, j);
+        const float4 t = qt[j];
+        sc[0] = fmaf(t.x, c, sc[0]); sc[1] = fmaf(t.y, c, sc[1]);
+        sc[2] = fmaf(t.z, c, sc[2]); sc[3] = fmaf(t.w, c, sc[3]);
+    }
+    if (S && lane < S) {
+        const float cf = code(Kb, lane);
+        const float4 q = qs[Kb[offIdx + row * S + lane]];
+        rs[0] = q.x * cf; rs[1] = q.y * cf; rs[2] = q.z * cf; rs[3] = q.w * cf;
+    }
+    const float scK = S ? __half2float(*reinterpret_cast<const __half*>(Kb + offSc + row * 2)) : 0.f;
+    float s_t[kGQ];
+#pragma unroll
+    for (int hh = 0; hh < kGQ; ++hh) s_t[hh] = fmaf(scK, warp_sum(rs[hh]), warp_sum(sc[hh]));
+    // online softmax: move the max when the token exceeds it by the slack, as the pages do
+    float alpha[kGQ];
+    bool over = false;
+#pragma unroll
+    for (int hh = 0; hh < kGQ; ++hh) {
+        alpha[hh] = 1.f;
+        if (s_t[hh] > A.m[hh] + kRescaleSlack) {
+            alpha[hh] = exp2f(A.m[hh] - s_t[hh]);
+            A.m[hh] = s_t[hh];
+            over = true;
+        }
+        A.l[hh] *= alpha[hh];
+    }
+    const int g = lane >> 2, c = lane & 3;
+    if (over) {
+        rescale_d(A.c, alpha[(2 * c) & 3], alpha[(2 * c + 1) & 3]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { A.r[i][0] *= alpha[c]; A.r[i][1] *= alpha[c]; }
+    }
+    float p[kGQ];
+#pragma unroll
+    for (int hh = 0; hh < kGQ; ++hh) {
+        p[hh] = exp2f(s_t[hh] - A.m[hh]);
+        if (lane == 0) A.l[hh] += p[hh];               // A.l is summed over the lanes later
+    }
+    // values, coefficient space: rows j = 16 i + g (+8), hi columns (lanes c < 2: heads 2c, 2c+1)
+    if (c < 2) {
+#pragma unroll
+        for (int i = 0; i < RMAX / 16; ++i) {
+            const int j0 = 16 * i + g, j1 = j0 + 8;
+            if (j0 < R) {
+                const float v = coeff(Vb, j0);
+                A.c[i][0] = fmaf(p[2 * c], v, A.c[i][0]);
+                A.c[i][1] = fmaf(p[2 * c + 1], v, A.c[i][1]);
+            }
+            if (j1 < R) {
+                const float v = coeff(Vb, j1);
+                A.c[i][2] = fmaf(p[2 * c], v, A.c[i][2]);
+                A.c[i][3] = fmaf(p[2 * c + 1], v, A.c[i][3]);
+            }
+        }
+    }
+    // values, residual space: channel ch sits in row (ch & 15) of tile ch >> 4, at lanes g = ch & 7
+    if (S) {
+        const float scV = __half2float(*reinterpret_cast<const __half*>(Vb + offSc + row * 2));
+        const float pc = p[c] * scV;
+        for (int e = 0; e < S; ++e) {
+            const int ch = Vb[offIdx + row * S + e];
+            if ((ch & 7) != g) continue;
+            const float v = pc * code(Vb, e);
+            const int mt = ch >> 4, r2 = (ch >> 3) & 1;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i == mt) { if (r2) A.r[i][1] += v; else A.r[i][0] += v; }
+        }
+    }
+}
+
 }  // namespace decode_detail
 
 // BITS: code width; PROBE: second softmax state without the residual; RMAX: accumulator
@@ -453,6 +605,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     const int nsplit = C.split_begin[ci + 1] - C.split_begin[ci];
     const int seq = C.seq[ci];
     const size_t basis_off = ((size_t)C.g * G.Hkv + h) * kD * G.r_max;
+    TokDest* tokd = reinterpret_cast<TokDest*>(smem + L.tok);
+    const bool owner = !PROBE && C.fused && split == 0;
+    if (owner) owner_append<BITS>(G, St, C, ci, seq, h, smem + L.ring, tokd);
 
     uint32_t cv[kMaxTiers];                 // tier counts (producer lane 0)
     uint32_t bvf[RMAX / 16][4];             // B_V mma fragments (consumer warps 0-7, epilogue)
@@ -473,6 +628,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         const uint32_t* cnt = St.counts + cnt_index(G, seq, C.g, h);
 #pragma unroll
         for (int k = 0; k < kMaxTiers; ++k) cv[k] = k < G.ntiers ? __ldcg(cnt + k) : 0u;
+        // fused append: the pages are attended without the new token.  Where it was placed by
+        // an earlier layer of the group the counts include it (it is the last slot of its tier);
+        // where this launch places it they do not yet (the last CTA adds it).
+        if (C.fused && !C.place[ci]) {
+            const uint32_t sm = __ldcg(St.slot_map + slot_index(G, seq, C.g, h, C.pos[ci]));
+            const uint32_t kt = (sm >> 24) - 1u;
+#pragma unroll
+            for (int k = 0; k < kMaxTiers; ++k)
+                if (sm != 0u && (uint32_t)k == kt && cv[k] > 0u) cv[k] -= 1u;
+        }
     }
     __syncthreads();
 
@@ -494,9 +659,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                 W += (unsigned long long)np * (G.chunk_bytes[k] + tokw);
             }
             m_P[G.ntiers] = P;
-            // cost-balanced page range: pages whose first cost unit lies in [lo, hi)
-            const unsigned long long lo = W * (unsigned long long)split / nsplit;
-            const unsigned long long hi = W * (unsigned long long)(split + 1) / nsplit;
+            // cost-balanced page range: pages whose first cost unit lies in [lo, hi).  With a
+            // fused append, split 0 (which also encodes the token) takes owner_share / 256 of a
+            // share: boundary s sits at W (256 (s - 1) + owner_share) / (256 (nsplit - 1) + owner_share).
+            const unsigned long long fs = (unsigned long long)C.owner_share;
+            const unsigned long long den = 256ull * (nsplit - 1) + fs;
+            auto bound = [&](int sidx) -> unsigned long long {
+                return sidx == 0 ? 0ull : W * (256ull * (sidx - 1) + fs) / den;
+            };
+            const unsigned long long lo = bound(split);
+            const unsigned long long hi = split + 1 == nsplit ? W : bound(split + 1);
             uint32_t pb = P, pe = P;
             unsigned long long Wk = W;
             for (int k = G.ntiers - 1; k >= 0; --k) {
@@ -724,6 +896,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                 wn = __shfl_sync(0xffffffffu, wn, 0);
             }
             w = wn;
+        }
+        if constexpr (!PROBE) {
+            if (owner && warp == 0 && tokd->ok)
+                add_new_token<S, BITS, RMAX>(G, *tokd, reinterpret_cast<const float4*>(smem + L.qt), qs, A, lane);
         }
         // ---- per-warp results: acc_c [r_max][4] and acc_r [d][4] into the residual tile,
         //      the probe's acc_c2 into the small buffers; m / l into m_state
@@ -995,7 +1171,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         }
     }
     if (tid == 0) St.tickets[(size_t)seq * G.Hkv + h] = 0u;
-    if (tid == 0) St.tickets[(size_t)seq * G.Hkv + h] = 0u;
+    if (tid == 0) {
+        St.tickets[(size_t)seq * G.Hkv + h] = 0u;
+        if (C.fused && C.place[ci]) {
+            // every CTA has read the counts: add the position placed by the first CTA
+            const uint32_t k = C.tier_idx[(size_t)ci * G.Hkv + h];
+            if (k < (uint32_t)G.ntiers) St.counts[cnt_index(G, seq, C.g, h) + k] += 1u;
+        }
+    }
 }
 
 }  // namespace dwkv

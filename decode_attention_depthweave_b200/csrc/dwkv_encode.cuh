@@ -34,6 +34,43 @@ __device__ __forceinline__ bool find_dest(const Geom& G, const State& S, int seq
     return true;
 }
 
+// Slot of one new position of (seq, group g, kv-head h) in tier k, the counts left as they are
+// (the caller adds the position to them later): the tier's next slot, and a fresh page when the
+// slot opens one (the tier's free ring first, then the pool's bump pointer).  Single thread.
+__device__ __forceinline__ bool place_one(const Geom& G, const State& S, int seq, int g, int h, int pos,
+                                          uint32_t k, Dest& d, int lig) {
+    const uint32_t old = __ldcg(S.counts + cnt_index(G, seq, g, h) + k);
+    const uint32_t pi = old / kPage;
+    if (pi >= (uint32_t)G.max_pages) {
+        set_dev_error(S, 1u /*DWKV_DEV_POOL_EXHAUSTED*/, (uint32_t)seq, (uint32_t)h);
+        return false;
+    }
+    uint32_t unit;
+    if (old % kPage == 0) {
+        const uint32_t t = atomicAdd(&S.free_head[k], 1u);
+        const uint32_t tail = *((volatile uint32_t*)&S.free_tail[k]);
+        if ((int)(tail - t) > 0) {
+            unit = S.free_list[(size_t)k * G.free_cap + (t & (G.free_cap - 1))];
+        } else {
+            const unsigned long long base = atomicAdd(S.bump, (unsigned long long)G.page_units[k]);
+            if (base + G.page_units[k] > S.data_units) {
+                set_dev_error(S, 1u /*DWKV_DEV_POOL_EXHAUSTED*/, (uint32_t)seq, (uint32_t)h);
+                return false;
+            }
+            unit = (uint32_t)base;
+        }
+        S.pages[page_index(G, seq, g, h, k) + pi] = unit;
+    } else {
+        unit = __ldcg(S.pages + page_index(G, seq, g, h, k) + pi);
+    }
+    S.slot_map[slot_index(G, seq, g, h, pos)] = ((k + 1u) << 24) | old;
+    d.k = (int)k;
+    d.row = (int)(old % kPage);
+    d.R = G.tiers[k];
+    d.blk = S.data + (size_t)unit * kUnit + (size_t)lig * G.chunk_bytes[k];
+    return true;
+}
+
 // Shared-memory scratch of one encode warp: x [d], stored coefficients [kMaxRank], code staging.
 struct EncScratch {
     float* xs;

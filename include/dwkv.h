@@ -186,6 +186,23 @@ dwkv_status dwkv_decode_attention(dwkv_handle h, int32_t layer, int32_t n_seqs,
                                   const int32_t* seq_ids, const void* q, float* out,
                                   void* workspace, size_t ws_bytes, void* stream);
 
+/* One decode step of `layer` in a single launch: appends one new token to each listed
+ * sequence (exactly as dwkv_append with n_new = 1 each: same placement, same stored bytes)
+ * and runs dwkv_decode_attention over every token the sequence then holds, the new one
+ * included ([DW] §3: the new token is compressed with the current basis, then attended
+ * through Eq. (1) with the rest).  Arguments as dwkv_append and dwkv_decode_attention:
+ *   k_new, v_new : device bf16 [n_seqs][Hkv][head_dim]
+ *   tier_idx     : device uint8 [n_seqs][Hkv]; read where this layer is the group's first
+ *                  to append the position, else may be NULL
+ *   q, out, workspace as dwkv_decode_attention.
+ * Same errors as the two calls.  When a tuning cap leaves the page ring too small for the
+ * launch to stage both bases, it runs the two calls instead (same results). */
+dwkv_status dwkv_append_decode_attention(dwkv_handle h, int32_t layer, int32_t n_seqs,
+                                         const int32_t* seq_ids, const void* k_new,
+                                         const void* v_new, const uint8_t* tier_idx,
+                                         const void* q, float* out, void* workspace,
+                                         size_t ws_bytes, void* stream);
+
 /* Probe ([DW] §3 Eq. (3), two caches read as with / without the residual) in one pass
  * over the cache.  err: device fp32 [n_seqs][Hkv].  out_full: NULL or device fp32
  * [n_seqs][Hq][head_dim] (the decode output).  Other arguments as decode. */
