@@ -288,17 +288,18 @@ def run_dwkv(args, world, rank, local):
     lpg = wl.layers_per_group
 
     def step(s, ev=None):
+        # per layer, one launch: append the step's token and attend over the whole context
         for layer in range(wl.num_layers):
             g = layer // lpg
-            dw.dwkv_append(h, layer, [0], [1], Kn[layer][s], Vn[layer][s], Tn[g][s] if layer % lpg == 0 else None,
-                           stream)
             if ev is not None:
                 ev[layer][0].record(stream)
-            dw.dwkv_decode_attention(h, layer, [0], Qs[layer][s], out[layer], ws, stream)
+            dw.dwkv_append_decode_attention(h, layer, [0], Kn[layer][s], Vn[layer][s],
+                                            Tn[g][s] if layer % lpg == 0 else None, Qs[layer][s], out[layer], ws,
+                                            stream)
             if ev is not None:
                 ev[layer][1].record(stream)
 
-    launches_per_step = wl.num_layers * 2 + wl.num_groups      # encode + decode per layer, place per group
+    launches_per_step = wl.num_layers                          # one fused append + decode per layer
 
     # ---- warm-up (graph of W steps, replayed once)
     torch.cuda.synchronize(dev)
@@ -384,8 +385,8 @@ def run_dwkv(args, world, rank, local):
         with torch.cuda.graph(g_e2e, stream=stream):
             for layer in range(wl.num_layers):
                 g = layer // lpg
-                dw.dwkv_append(h, layer, [0], [1], dK[layer], dV[layer], dT[g] if layer % lpg == 0 else None, stream)
-                dw.dwkv_decode_attention(h, layer, [0], dQ[layer], out[layer], ws, stream)
+                dw.dwkv_append_decode_attention(h, layer, [0], dK[layer], dV[layer],
+                                                dT[g] if layer % lpg == 0 else None, dQ[layer], out[layer], ws, stream)
         torch.cuda.synchronize(dev)
         barrier(world)
         a0 = torch.cuda.Event(enable_timing=True)
