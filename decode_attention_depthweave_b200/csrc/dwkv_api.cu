@@ -194,7 +194,7 @@ struct dwkv_ctx {
     std::vector<int32_t> placed;    // [max_batch][G]
     int dec_ctas_per_sm = 1, dec_waves = 1, dec_stages_req = 0;
     int dec_tok_weight = 1024;      // split balance: byte-equivalent cost of one token
-    int dec_owner_share = 192;      // fused append: the encoding CTA's share of a split, of 256
+    int dec_owner_share = 160;      // fused append: the encoding CTA's share of a split, of 256
 };
 
 namespace {
