@@ -6,17 +6,23 @@ two-layer groups, 32 query heads / 8 kv heads, head_dim 128, batch 1, 64K contex
 bases r_max = 64 per (group, kv-head, K/V); tiers {16, 32, 64} with probabilities
 0.6 / 0.3 / 0.1; residual s = 16 int4 channels with an fp16 scale.  The cache holds
 65535 compressed tokens (synthetic, seeded, imported before timing).  One step = for
-each of the 32 layers: encode + append one new token (dwkv_append), then fused decode
-attention over the whole context (dwkv_decode_attention).  Metric: decode tokens/s
-(batch / step time) and the compressed-KV bytes/s of the decode kernel against the
-measured HBM copy bandwidth.  Attention only (no projections / MLP: no weights exist).
+each of the 32 layers one launch of dwkv_append_decode_attention: encode + append the
+step's new token, then fused decode attention over the whole context.  Metric: decode
+tokens/s (batch / step time) and the compressed-KV bytes/s of the decode kernel against
+the measured HBM copy bandwidth.  Attention only (no projections / MLP: no weights exist).
 
 Timing: W warm-up steps, then K steps captured in one CUDA graph and replayed once,
 bracketed by a barrier + synchronize, timed with CUDA events; max over ranks.  Each
-step streams ~2.6 GB of pages (> 126 MB L2), so no L2 flush is needed.  A second
-replay of the same K steps with an external event around every decode launch gives the
-decode kernel's average duration for the roofline.  ``e2e`` repeats the step with host
+step streams ~2.6 GB of pages (> 126 MB L2), so no L2 flush is needed.  Every launch
+in the timed region is the fused decode kernel, so its average launch duration is the
+region's time over its launches (the roofline); a second replay with an external event
+around every launch is reported beside it.  The probe (dwkv_probe, one launch per layer)
+is timed over the same cache after the steps.  ``e2e`` repeats the step with host
 (pinned) inputs copied in and the outputs copied out inside the timed region.
+
+``--workload llama8b_encode_16k`` measures bulk encode instead: 4 sequences x 16384 new
+dense tokens per layer through dwkv_append (32 layers a step, the sequences reset between
+steps), then one decode step and one probe pass over the encoded cache.
 
 ``--impl reference`` times the CPU oracle (plain fp64 C, all host cores) on a bounded
 sample of the same workload and reports the same metric.
@@ -352,6 +358,26 @@ def run_dwkv(args, world, rank, local):
     dec_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(args.profile_steps) for l in range(wl.num_layers)]
     dec_ms_mean = statistics.mean(dec_ms)
 
+    # ---- probe (with / without residual, one launch per layer) over the same cache
+    err = torch.empty(wl.num_layers, 1, wl.num_kv_heads, dtype=torch.float32, device=dev)
+    g_probe = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_probe, stream=stream):
+        for layer in range(wl.num_layers):
+            dw.dwkv_probe(h, layer, [0], Qs[layer][args.warmup], err[layer], None, ws, stream)
+    p0 = torch.cuda.Event(enable_timing=True)
+    p1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g_probe.replay()
+        p0.record(stream)
+        for _ in range(args.profile_steps):
+            g_probe.replay()
+        p1.record(stream)
+    torch.cuda.synchronize(dev)
+    cache.sync(stream)
+    assert torch.isfinite(err).all()
+    probe_launch_ms = p0.elapsed_time(p1) / (args.profile_steps * wl.num_layers)
+    held_probe = T - 1 + args.warmup + args.steps + args.profile_steps
+
     # ---- algorithmic bytes: every stored byte of the attended tokens (per-token bytes of
     #      its tier), plus the two bases, the query and the output of each launch
     held = T - 1 + args.warmup + args.steps                  # tokens per head after the timed steps
@@ -372,6 +398,7 @@ def run_dwkv(args, world, rank, local):
     alg_bytes = layer_bytes(ctx_timed)
     achieved = alg_bytes / (launch_ms * 1e-3) / 1e9
     traffic = profiled_traffic(args.workload)
+    probe_bytes = layer_bytes(held_probe) - wl.num_q_heads * wl.head_dim * 4 + wl.num_kv_heads * 4
 
     # ---- e2e: host inputs in, host outputs out, one step per graph replay
     e2e = None
@@ -451,9 +478,171 @@ def run_dwkv(args, world, rank, local):
                      "launch_ms_bracketed": round(dec_ms_mean, 5),
                      "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
                      "frac_of_8tbs_spec": round(achieved / 8000.0, 4)},
+        "probe": {"kernel": f"dwkv::decode_kernel<{wl.resid_bits},true>", "launch_ms": round(probe_launch_ms, 5),
+                  "context": held_probe,
+                  "achieved_gbs": round(probe_bytes / (probe_launch_ms * 1e-3) / 1e9, 1),
+                  "frac": round(probe_bytes / (probe_launch_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                  "timing": f"graph of {wl.num_layers} probe launches, {args.profile_steps} replays after one warm-up"},
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
+    }
+    cache.close()
+    return res
+
+
+def fp32_alu_peak_tflops(sm_mhz: float, sms: int = 148) -> float:
+    """FP32 FMA peak: 128 fp32 lanes per SM, one FMA (2 flops) per lane per clock."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def run_encode(args, world, rank, local):
+    """Bulk encode (a7) at the encode workload's sizes: per step, every layer compresses
+    ``batch`` sequences x ``new_tokens`` dense K/V tokens through dwkv_append (placement +
+    encode kernels); the sequences are reset before each step, outside the timed events.
+    Then one fused decode step and one probe pass over the encoded cache."""
+    import torch
+
+    import decode_attention_depthweave_b200 as dw
+    import synth
+
+    wl = synth.workload(args.workload)
+    if args.layers:
+        wl = wl.scaled(num_layers=args.layers)
+    dev = torch.device("cuda", local)
+    B, N = wl.batch, wl.new_tokens
+    lpg = wl.layers_per_group
+    bases = synth.make_bases(wl)
+    cfg = dw.config_from(num_layers=wl.num_layers, layers_per_group=lpg, num_q_heads=wl.num_q_heads,
+                         num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, r_max=wl.r_max, tiers=wl.tiers,
+                         resid_channels=wl.resid_channels, resid_bits=wl.resid_bits, max_batch=B,
+                         max_context=N + 64)
+    stream = torch.cuda.Stream(device=dev)
+    cache = dw.Cache(cfg, bases[0], bases[1], device=dev, ws_seqs=B, stream=stream)
+    h = cache.h
+    seqs = list(range(B))
+    K, V, Tg = [], [], {}
+    tier_counts = torch.zeros(len(wl.tiers), dtype=torch.int64)
+    with torch.cuda.stream(stream):
+        for layer in range(wl.num_layers):
+            g = layer // lpg
+            if g not in Tg:
+                Tg[g] = torch.cat([synth.make_tiers(wl, rank * B + b, g, N, device=dev) for b in seqs])
+                for k in range(len(wl.tiers)):
+                    tier_counts[k] += int((Tg[g] == k).sum())
+            kv = [synth.make_dense_vectors(wl, rank * B + b, layer, N, bases, device=dev) for b in seqs]
+            K.append(torch.cat([x[0] for x in kv]))
+            V.append(torch.cat([x[1] for x in kv]))
+            del kv
+    torch.cuda.synchronize(dev)
+
+    def encode_step():
+        for layer in range(wl.num_layers):
+            dw.dwkv_append(h, layer, seqs, [N] * B, K[layer], V[layer], Tg[layer // lpg], stream)
+
+    def reset():
+        for b in seqs:
+            dw.dwkv_reset_sequence(h, b, stream)
+
+    for _ in range(args.warmup):
+        reset()
+        encode_step()
+    torch.cuda.synchronize(dev)
+    cache.sync(stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        clk.mark_start()
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                reset()
+                ev[i][0].record(stream)
+                encode_step()
+                ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        clk.mark_end()
+    barrier(world)
+    cache.sync(stream)
+    ms_steps = [a.elapsed_time(b) for a, b in ev]
+    ms_per_step = max_over_ranks(world, statistics.mean(ms_steps))
+    clocks = clk.summary()
+
+    # ---- algorithmic work per step: every vector reads its dense bf16 row and writes its
+    #      stored bytes; 2 d r_t fp32 FMAs (projection onto the first r_t basis columns, and
+    #      the residual against the stored coefficients)
+    vecs_tier = tier_counts.double() * 2 * lpg       # (seq, head, token) entries x K and V x layers of a group
+    n_vec = float(vecs_tier.sum())
+    stored = sum(float(tier_counts[k]) * lpg * token_bytes(r, wl.resid_channels, wl.resid_bits)   # K + V bytes
+                 for k, r in enumerate(wl.tiers))
+    dense = n_vec * wl.head_dim * 2
+    flops = sum(float(vecs_tier[k]) * 4 * wl.head_dim * r for k, r in enumerate(wl.tiers))
+    step_s = ms_per_step * 1e-3
+    peaks = measured_peaks()
+    sm_mhz = float(clocks.get("sm_max_mhz") or 1965.0) if isinstance(clocks, dict) else 1965.0
+    alu_peak = fp32_alu_peak_tflops(sm_mhz)
+
+    # ---- one decode step (append 1 token per sequence + attend, every layer) and one probe pass
+    kn = [synth.make_dense_vectors(wl, rank * B + b, 0, 1, bases, device=dev, start=N) for b in seqs]
+    k1 = torch.cat([x[0] for x in kn])
+    v1 = torch.cat([x[1] for x in kn])
+    t1 = torch.cat([synth.make_tiers(wl, rank * B + b, 0, 1, device=dev, start=N) for b in seqs])
+    q = [synth.make_queries(wl, layer, batch=B, device=dev) for layer in range(wl.num_layers)]
+    out = torch.empty(wl.num_layers, B, wl.num_q_heads, wl.head_dim, dtype=torch.float32, device=dev)
+    err = torch.empty(wl.num_layers, B, wl.num_kv_heads, dtype=torch.float32, device=dev)
+    ws = cache.workspace
+    d0, d1, p0, p1 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+    with torch.cuda.stream(stream):
+        d0.record(stream)
+        for layer in range(wl.num_layers):
+            dw.dwkv_append_decode_attention(h, layer, seqs, k1, v1, t1 if layer % lpg == 0 else None, q[layer],
+                                            out[layer], ws, stream)
+        d1.record(stream)
+        for layer in range(wl.num_layers):                                    # warm
+            dw.dwkv_probe(h, layer, seqs, q[layer], err[layer], None, ws, stream)
+        p0.record(stream)
+        for layer in range(wl.num_layers):
+            dw.dwkv_probe(h, layer, seqs, q[layer], err[layer], None, ws, stream)
+        p1.record(stream)
+    torch.cuda.synchronize(dev)
+    cache.sync(stream)
+    assert torch.isfinite(out).all() and torch.isfinite(err).all()
+    held = N + 1
+    dec_bytes = (float(tier_counts.double() @ torch.tensor([token_bytes(r, wl.resid_channels, wl.resid_bits)
+                                                             for r in wl.tiers], dtype=torch.float64))
+                 * lpg)                                                         # every layer; K + V bytes
+    dec_ms = d0.elapsed_time(d1)
+    probe_ms = p0.elapsed_time(p1)
+
+    value = aggregate_rate(world, dense / 1e9, ms_per_step)
+    res = {
+        "metric": "bulk encode: dense bf16 K/V GB/s compressed (a7)", "value": round(value, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 math",
+        "data": "synthetic (seeded dense K/V: basis span + outliers + noise; no model weights)",
+        "config": {"workload": args.workload, "layers": wl.num_layers, "kv_heads": wl.num_kv_heads,
+                   "head_dim": wl.head_dim, "batch_per_gpu": B, "new_tokens": N, "r_max": wl.r_max,
+                   "tiers": list(wl.tiers), "tier_probs": list(wl.tier_probs), "resid_channels": wl.resid_channels,
+                   "resid_bits": wl.resid_bits, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (8.6 GB of dense K/V a step); no flush",
+                   "timing": "eager launches, CUDA events around each step's appends (resets outside)"},
+        "gpu_launches": 2 * wl.num_layers * args.steps,
+        "vectors_per_s": round(aggregate_rate(world, n_vec, ms_per_step), 1),
+        "roofline": {"bound": "alu", "achieved": round(flops / step_s / 1e12, 3), "unit": "TFLOP/s",
+                     "peak": round(alu_peak, 2), "frac": round(flops / step_s / 1e12 / alu_peak, 4),
+                     "traffic": None, "kernel": f"dwkv::encode_kernel<{wl.resid_bits}>",
+                     "peak_source": f"148 SMs x 128 fp32 lanes x 2 flops x {sm_mhz:.0f} MHz (sampled max SM clock)",
+                     "flops_per_step": flops},
+        "hbm": {"bytes_per_step": dense + stored, "achieved_gbs": round((dense + stored) / step_s / 1e9, 1),
+                "frac": round((dense + stored) / step_s / 1e9 / peaks["hbm_gbs"], 4)},
+        "decode_step": {"context": held, "batch": B, "ms": round(dec_ms, 4),
+                        "tok_s": round(B / (dec_ms * 1e-3), 1),
+                        "compressed_gbs": round(dec_bytes / (dec_ms * 1e-3) / 1e9, 1),
+                        "timing": "one eager step (32 fused append + decode launches)"},
+        "probe": {"ms_all_layers": round(probe_ms, 4),
+                  "achieved_gbs": round(dec_bytes / (probe_ms * 1e-3) / 1e9, 1),
+                  "frac": round(dec_bytes / (probe_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+        "clocks": clocks,
     }
     cache.close()
     return res
@@ -520,6 +709,8 @@ def main():
             if rank != 0:
                 return
             res = run_reference(args, world, rank, local)
+        elif args.workload == "llama8b_encode_16k":
+            res = run_encode(args, world, rank, local)
         else:
             res = run_dwkv(args, world, rank, local)
         if rank == 0:

@@ -22,7 +22,7 @@ __all__ = [
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage",
     "dwkv_sync_status", "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
-    "Cache", "EXPORTED_SYMBOLS",
+    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "Cache", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -38,6 +38,7 @@ EXPORTED_SYMBOLS = (
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage", "dwkv_sync_status",
     "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
+    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals",
 )
 
 
@@ -98,6 +99,8 @@ def lib():
             "dwkv_sync_status": ([vp, vp], C.c_int),
             "dwkv_set_decode_tuning": ([vp, i32, i32, i32], C.c_int),
             "dwkv_decode_attention_noalloc": ([vp, i32, i32, vp, vp, vp, vp], C.c_int),
+            "dwkv_quantize_work_bytes": ([i32, i32, i32], sz),
+            "dwkv_quantize_residuals": ([i32, i32, i32, vp, vp, vp, vp, vp, sz, vp], C.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -233,6 +236,24 @@ def dwkv_decode_attention_noalloc(h, layer, seq_ids, q, out, stream=None):
 def dwkv_probe(h, layer, seq_ids, q, err, out_full, workspace, stream=None):
     _check(lib().dwkv_probe(h, layer, len(seq_ids), _i32(seq_ids), _ptr(q), _ptr(err), _ptr(out_full),
                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dwkv_quantize_work_bytes(n, s, bits) -> int:
+    return int(lib().dwkv_quantize_work_bytes(n, s, bits))
+
+
+def dwkv_quantize_residuals(r, s, bits, stream=None):
+    """Encode steps 4-6 on residuals r (device fp32 [n][128]): (idx uint8 [n][s], codes int8
+    [n][s], scales fp16 bits as int16 [n]), all on r's device."""
+    n = r.shape[0]
+    dev = r.device
+    idx = torch.empty(n, s, dtype=torch.uint8, device=dev)
+    codes = torch.empty(n, s, dtype=torch.int8, device=dev)
+    scales = torch.empty(n, dtype=torch.int16, device=dev)
+    work = torch.empty(max(dwkv_quantize_work_bytes(n, s, bits), 16), dtype=torch.uint8, device=dev)
+    _check(lib().dwkv_quantize_residuals(n, s, bits, _ptr(r), _ptr(idx), _ptr(codes), _ptr(scales), _ptr(work),
+                                         work.numel(), _stream(stream)))
+    return idx, codes, scales
 
 
 def dwkv_export(h, layer, seq, t0, n, tier_idx=None, coeff=None, idx=None, codes=None, scales=None, stream=None):

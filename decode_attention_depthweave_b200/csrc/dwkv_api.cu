@@ -11,11 +11,14 @@
 
 #include "dwkv.h"
 #include "dwkv_common.cuh"
+#include "dwkv_encode.cuh"
 
 namespace dwkv {
 __global__ void place_kernel(const Geom, const State, const AppendCall, const uint8_t*);
 template <int BITS>
 __global__ void encode_kernel(const Geom, const State, const AppendCall, const __nv_bfloat16*, const __nv_bfloat16*);
+template <int BITS>
+__global__ void quantize_test_kernel(int, int, const float*, uint8_t*, int8_t*, uint16_t*, uint8_t*, uint32_t);
 template <int BITS>
 __global__ void append_small_kernel(const Geom, const State, const AppendCall, const uint8_t*, int,
                                     const __nv_bfloat16*, const __nv_bfloat16*);
@@ -246,6 +249,7 @@ State make_state(uint8_t* arena, const MetaLayout& M, size_t arena_bytes) {
 size_t encode_smem(const Geom& G) {
     return (size_t)2 * kD * (G.r_max + 2) * 2 + (size_t)8 * (kD + kMaxRank + 32) * 4;
 }
+size_t encode_tile_smem(const Geom& G) { return enc_tile_layout(G.r_max).total; }
 
 // Bytes of the decode page ring: what the shared-memory budget leaves after the fixed
 // regions, capped at dec_stages_req x the largest chunk when that is set (but never below
@@ -426,11 +430,13 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
         for (const void* k : kernels)
             if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
         // the encode kernels ask for what they use (the fused append also has static smem)
-        const int es = (int)encode_smem(G);
-        const void* enc[] = {(const void*)encode_kernel<8>, (const void*)encode_kernel<4>,
-                             (const void*)append_small_kernel<8>, (const void*)append_small_kernel<4>};
+        const int es = (int)encode_smem(G), ets = (int)encode_tile_smem(G);
+        const void* enc[] = {(const void*)append_small_kernel<8>, (const void*)append_small_kernel<4>};
         for (const void* k : enc)
             if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, es);
+        const void* tiles[] = {(const void*)encode_kernel<8>, (const void*)encode_kernel<4>};
+        for (const void* k : tiles)
+            if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ets);
     }
     if (e != cudaSuccess) {
         delete h;
@@ -502,6 +508,8 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
     if ((st = prepare_call(h, layer, n_seqs, seq_ids, n_new, C, true, tier_idx)) != DWKV_OK) return st;
     if (C.total == 0) return DWKV_OK;
     if (!k_new || !v_new) return fail(DWKV_ERR_INVALID_ARG, "k_new and v_new must be non-NULL");
+    if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15u)
+        return fail(DWKV_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
     const Geom& G = h->geom;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     bool any = false;
@@ -530,13 +538,17 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
         place_kernel<<<dim3(C.n, G.Hkv), 256, 0, s>>>(G, h->st, C, tier_idx);
         DWKV_CUDA(cudaGetLastError(), "place_kernel launch");
     }
-    const dim3 grid(grid_rows(h, 2ll * C.total), G.Hkv);     // a warp per (row, keys or values)
+    // a block per (kv-head, K or V) and share of the tiles; two blocks fit an SM
+    const long long ntiles = (C.total + kEncTile - 1) / kEncTile;
+    const long long per = std::max(1, h->num_sms / std::max(1, G.Hkv));
+    const dim3 grid((unsigned)std::min(ntiles, per), G.Hkv, 2);
+    const size_t tsm = encode_tile_smem(G);
     if (G.bits == 8)
-        encode_kernel<8><<<grid, 256, sm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
-                                                static_cast<const __nv_bfloat16*>(v_new));
+        encode_kernel<8><<<grid, 256, tsm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
+                                                 static_cast<const __nv_bfloat16*>(v_new));
     else
-        encode_kernel<4><<<grid, 256, sm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
-                                                static_cast<const __nv_bfloat16*>(v_new));
+        encode_kernel<4><<<grid, 256, tsm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
+                                                 static_cast<const __nv_bfloat16*>(v_new));
     DWKV_CUDA(cudaGetLastError(), "encode_kernel launch");
     commit_call(h, C, n_new);
     return DWKV_OK;
@@ -780,6 +792,40 @@ dwkv_status dwkv_sync_status(dwkv_handle h, void* stream) {
                                   "free-page ring overflow"};
     const char* nm = w[0] < sizeof(names) / sizeof(names[0]) ? names[w[0]] : "unknown";
     return fail(DWKV_ERR_DEVICE_CHECK, "device check failed: %s (code %u, info %u, %u)", nm, w[0], w[1], w[2]);
+}
+
+static uint32_t quantize_stride(int32_t s, int32_t bits) {
+    return (off_scales_of(0, s, bits) + 2u + 15u) & ~15u;
+}
+
+size_t dwkv_quantize_work_bytes(int32_t n, int32_t s, int32_t bits) {
+    if (n < 0 || s < 0 || s > kD || (bits != 8 && bits != 4)) return 0;
+    return (size_t)n * quantize_stride(s, bits);
+}
+
+dwkv_status dwkv_quantize_residuals(int32_t n, int32_t s, int32_t bits, const float* r, uint8_t* idx,
+                                    int8_t* codes, uint16_t* scales, void* work, size_t work_bytes,
+                                    void* stream) {
+    if (n < 0) return fail(DWKV_ERR_INVALID_ARG, "n = %d must be >= 0", n);
+    if (s < 0 || s > kD || s % 8) return fail(DWKV_ERR_INVALID_ARG, "s = %d must be a multiple of 8 in 0..%d", s, kD);
+    if (bits != 8 && bits != 4) return fail(DWKV_ERR_INVALID_ARG, "bits = %d must be 8 or 4", bits);
+    if (n == 0) return DWKV_OK;
+    if (!r || !scales || !work || (s > 0 && (!idx || !codes)))
+        return fail(DWKV_ERR_INVALID_ARG, "r, idx, codes, scales and work must be non-NULL");
+    if (work_bytes < dwkv_quantize_work_bytes(n, s, bits))
+        return fail(DWKV_ERR_INVALID_ARG, "work holds %zu bytes, needs %zu", work_bytes,
+                    dwkv_quantize_work_bytes(n, s, bits));
+    if (reinterpret_cast<uintptr_t>(work) % 16) return fail(DWKV_ERR_INVALID_ARG, "work must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned grid = (unsigned)((n + 7) / 8);
+    if (bits == 8)
+        quantize_test_kernel<8><<<grid, 256, 0, st>>>(n, s, r, idx, codes, scales, static_cast<uint8_t*>(work),
+                                                       quantize_stride(s, bits));
+    else
+        quantize_test_kernel<4><<<grid, 256, 0, st>>>(n, s, r, idx, codes, scales, static_cast<uint8_t*>(work),
+                                                       quantize_stride(s, bits));
+    DWKV_CUDA(cudaGetLastError(), "quantize_test_kernel launch");
+    return DWKV_OK;
 }
 
 }  // extern "C"

@@ -120,40 +120,8 @@ __device__ __forceinline__ int call_index_of(const AppendCall& C, int row) {
 
 
 // ------------------------------------------------------------------------------------
-// Encode kernel: one warp per (token row, keys or values): unit u = 2 row + z.  The block
-// holds both bases of its (group, kv-head) in shared memory as bf16 with a padded row pitch,
-// so that the projection (lanes along j) and the residual (lanes along i) are conflict-free.
-// A single appended token therefore runs its keys and values on two warps side by side.
-// ------------------------------------------------------------------------------------
-// Both bases of the block's (group, kv-head) into shared memory: [2][d][P] bf16 with P = r_max + 2.
-// 16-byte loads, all of a thread's requests in flight before its stores.
-__device__ __forceinline__ void load_bases(const Geom& G, const State& S, int g, int h, __nv_bfloat16* bs) {
-    const int tid = threadIdx.x, RM = G.r_max, P = G.r_max + 2;
-    const size_t boff = ((size_t)g * G.Hkv + h) * kD * RM;
-    const int nvec = kD * RM / 8;                         // uint4 per basis
-    const uint4* srck = reinterpret_cast<const uint4*>(S.basis_k + boff);
-    const uint4* srcv = reinterpret_cast<const uint4*>(S.basis_v + boff);
-    constexpr int kBatch = 8;
-    for (int e0 = tid; e0 < 2 * nvec; e0 += kBatch * (int)blockDim.x) {
-        uint4 v[kBatch];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int e = e0 + b * (int)blockDim.x;
-            v[b] = e < 2 * nvec ? __ldg(e < nvec ? srck + e : srcv + (e - nvec)) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int e = e0 + b * (int)blockDim.x;
-            if (e >= 2 * nvec) break;
-            const int z = e >= nvec, ev = z ? e - nvec : e;
-            const int i = (ev * 8) / RM, j = (ev * 8) % RM;
-            uint32_t* dst = reinterpret_cast<uint32_t*>(bs + (size_t)z * kD * P + (size_t)i * P + j);
-            dst[0] = v[b].x; dst[1] = v[b].y; dst[2] = v[b].z; dst[3] = v[b].w;
-        }
-    }
-}
-
-// The same load in two steps, so that other global round trips overlap its latency: the
+// Both bases of the block's (group, kv-head) into shared memory, [2][d][P] bf16 with
+// P = r_max + 2, in two steps so that other global round trips overlap its latency: the
 // block's share of both bases into registers (at most 16 x 16 bytes a thread for 256
 // threads), then into shared memory.
 constexpr int kBasisRegs = 2 * kD * kMaxRank / 8 / 256;
@@ -203,33 +171,254 @@ __device__ __forceinline__ UnitIn encode_fetch(const Geom& G, const State& S, co
     return in;
 }
 
+// ------------------------------------------------------------------------------------
+// Bulk encode kernel.  A block per (kv-head, keys or values) strides over tiles of kEncTile
+// input rows and runs the six encode steps on all of a tile's vectors together, so that
+// every shared-memory load feeds several fma chains:
+//   1. the rows' destinations (slot map), counted by tier and given slots in descending
+//      tier order; each row's x enters shared memory (fp32, [channel][slot]) at its slot;
+//   2. projection items of 32 slots x 16 coefficients: each lane runs the full i = 0..d-1
+//      chains of 8 slots x 2 coefficients (x of 8 slots and a bf16 coefficient pair per
+//      step); the group's chains run to the largest rank among its 32 slots (the first
+//      slot, by the sort), and the coefficients past a slot's own rank are neither stored
+//      nor kept: they enter its residual as exact zeros;
+//   3. residual items of 8 slots, lane = channels lane + 32 m: the chains over j run to the
+//      largest rank of the 8 slots; a zero coefficient adds an exact +-0 to an accumulator
+//      that started at +0, which leaves it unchanged, so every slot gets the residual of
+//      its own-length chain; then steps 4-6 per slot (quantize_store).
+// The arithmetic per vector is the same operations in the same order as encode_body, so
+// the stored bytes are identical to the per-warp encoders'.
+// ------------------------------------------------------------------------------------
 template <int BITS>
-__device__ __forceinline__ void encode_unit(const Geom& G, const State& S, const AppendCall& C,
-                                            const __nv_bfloat16* __restrict__ k_new,
-                                            const __nv_bfloat16* __restrict__ v_new,
-                                            const __nv_bfloat16* bs, const EncScratch& W, int h, int unit) {
-    const UnitIn in = encode_fetch(G, S, C, k_new, v_new, h, unit);
-    encode_body<BITS>(G, S, bs, W, unit, in);
+__global__ void __launch_bounds__(256, 2) encode_kernel(const Geom G, const State S, const AppendCall C,
+                                                        const __nv_bfloat16* __restrict__ k_new,
+                                                        const __nv_bfloat16* __restrict__ v_new) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const EncTileLayout L = enc_tile_layout(G.r_max);
+    const int h = blockIdx.y, z = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem + L.bs);
+    float* xs = reinterpret_cast<float*>(smem + L.xs);
+    float* cs = reinterpret_cast<float*>(smem + L.cs);
+    uint8_t** sblk = reinterpret_cast<uint8_t**>(smem + L.sblk);
+    int* sR = reinterpret_cast<int*>(smem + L.sR);
+    int* sprow = reinterpret_cast<int*>(smem + L.sprow);
+    int* rslot = reinterpret_cast<int*>(smem + L.rslot);
+    int* cnt = reinterpret_cast<int*>(smem + L.misc);
+    int* base = cnt + kMaxTiers;
+    int* nvalid_p = base + kMaxTiers;
+    float* rstage = reinterpret_cast<float*>(smem + L.cst + warp * kEncStage);
+    uint8_t* chstage = reinterpret_cast<uint8_t*>(rstage + kD);
+    const int RM = G.r_max, PB = L.PB, npass = L.RP / 16;
+
+    // ---- this (group, kv-head, K or V) basis: bf16 [kD][PB], the columns past r_max zero
+    {
+        const __nv_bfloat16* src = (z ? S.basis_v : S.basis_k) + ((size_t)C.g * G.Hkv + h) * kD * RM;
+        uint16_t* b16 = reinterpret_cast<uint16_t*>(bs);
+        const int padc = PB - RM;
+        for (int e = tid; e < kD * padc; e += blockDim.x) b16[(e / padc) * PB + RM + e % padc] = 0;
+        const int nvec = kD * RM / 8;
+        for (int e = tid; e < nvec; e += blockDim.x) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + e);
+            const int i = (e * 8) / RM, j = (e * 8) % RM;
+            uint32_t* dst = reinterpret_cast<uint32_t*>(bs + (size_t)i * PB + j);
+            dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+        }
+    }
+
+    const __nv_bfloat16* xin = z ? v_new : k_new;
+    const int ntiles = (C.total + kEncTile - 1) / kEncTile;
+    const int trow = tid & (kEncTile - 1), q = tid / kEncTile;      // 4 threads a row, 32 channels each
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        // ---- 1: x into registers (requested first), destinations, tier counts
+        const int row = tile * kEncTile + trow;
+        const bool in_range = row < C.total;
+        uint4 xv[4];
+        if (in_range) {
+            const uint4* src = reinterpret_cast<const uint4*>(xin + ((size_t)row * G.Hkv + h) * kD + 32 * q);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) xv[b] = __ldg(src + b);
+        }
+        if (tid < kMaxTiers) cnt[tid] = 0;
+        __syncthreads();                        // counts cleared; the previous tile is done
+        Dest d;
+        bool ok = false;
+        int within = 0;
+        if (q == 0 && in_range) {
+            const int ci = call_index_of(C, row);
+            const int seq = C.seq[ci];
+            const int pos = C.pos0[ci] + (row - C.tok0[ci]);
+            ok = find_dest(G, S, seq, C.g, C.lig, h, pos, d);
+            // a0..a0+na were placed by the placement; a zero entry means placement failed
+            // (already reported) or the group never placed this position
+            if (!ok && z == 0 && !(pos >= C.a0[ci] && pos < C.a0[ci] + C.na[ci]))
+                set_dev_error(S, 5u /*DWKV_DEV_NO_SLOT*/, (uint32_t)seq, (uint32_t)pos);
+            if (ok) within = atomicAdd(&cnt[d.k], 1);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int acc = 0;
+            for (int k = kMaxTiers - 1; k >= 0; --k) {
+                base[k] = acc;
+                acc += cnt[k];
+            }
+            *nvalid_p = acc;
+        }
+        __syncthreads();
+        const int nvalid = *nvalid_p;
+        if (q == 0) {
+            int slot = -1;
+            if (ok) {
+                slot = base[d.k] + within;
+                sblk[slot] = d.blk + (z ? G.blk_bytes[d.k] : 0u);
+                sR[slot] = d.R;
+                sprow[slot] = d.row;
+            }
+            rslot[trow] = slot;
+        }
+        if (tid >= nvalid && tid < kEncTile) sR[tid] = 0;          // empty slots
+        __syncthreads();
+        {
+            const int slot = rslot[trow];
+            if (slot >= 0) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const uint32_t w[4] = {xv[b].x, xv[b].y, xv[b].z, xv[b].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 32 * q + 8 * b + 2 * e;
+                        xs[i * kEncXP + slot] = __uint_as_float(w[e] << 16);
+                        xs[(i + 1) * kEncXP + slot] = __uint_as_float(w[e] & 0xffff0000u);
+                    }
+                }
+            }
+            const int nempty = kEncTile - nvalid;
+            for (int e = tid; e < nempty * kD; e += blockDim.x) xs[(e / nempty) * kEncXP + nvalid + e % nempty] = 0.f;
+        }
+        __syncthreads();
+
+        // ---- 2: projection, bf16 rounding, coefficient stores
+        const int ngroups = (nvalid + 31) >> 5;
+        for (int it = warp; it < ngroups * npass; it += (int)(blockDim.x >> 5)) {
+            const int g = it / npass, p = it % npass;
+            if (16 * p >= sR[32 * g]) continue;
+            const int s0 = 32 * g + 8 * (lane >> 3), j0 = 16 * p + 2 * (lane & 7);
+            float acc[8][2];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) acc[t][0] = acc[t][1] = 0.f;
+            const float* xp = xs + s0;
+            const uint32_t* bp = reinterpret_cast<const uint32_t*>(bs + j0);
+#pragma unroll 4
+            for (int i = 0; i < kD; ++i) {
+                const float4 xa = *reinterpret_cast<const float4*>(xp + i * kEncXP);
+                const float4 xb = *reinterpret_cast<const float4*>(xp + i * kEncXP + 4);
+                const uint32_t bb = bp[i * (PB >> 1)];
+                const float b0 = __uint_as_float(bb << 16), b1 = __uint_as_float(bb & 0xffff0000u);
+                const float x8[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    acc[t][0] = __fmaf_rn(b0, x8[t], acc[t][0]);
+                    acc[t][1] = __fmaf_rn(b1, x8[t], acc[t][1]);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const int sl = s0 + t;
+                const bool on = j0 < sR[sl];           // ranks are multiples of 8: j0 + 1 too
+                const __nv_bfloat16 c0 = __float2bfloat16_rn(acc[t][0]), c1 = __float2bfloat16_rn(acc[t][1]);
+                cs[j0 * kEncXP + sl] = on ? __bfloat162float(c0) : 0.f;
+                cs[(j0 + 1) * kEncXP + sl] = on ? __bfloat162float(c1) : 0.f;
+                if (on) {
+                    __nv_bfloat162 pr;
+                    pr.x = c0;
+                    pr.y = c1;
+                    *reinterpret_cast<__nv_bfloat162*>(sblk[sl] + (size_t)(j0 >> 3) * 1024 + sprow[sl] * 16 +
+                                                       (j0 & 7) * 2) = pr;
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- 3: residual against the stored coefficients, then steps 4-6 per slot
+        for (int u = warp; 8 * u < nvalid; u += (int)(blockDim.x >> 5)) {
+            const int s0 = 8 * u, Ru = sR[s0];
+            float a[8][4];
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+#pragma unroll
+                for (int m = 0; m < 4; ++m) a[t][m] = 0.f;
+            for (int j = 0; j < Ru; j += 2) {          // ranks are multiples of 8
+                const float4 c0a = *reinterpret_cast<const float4*>(cs + j * kEncXP + s0);
+                const float4 c0b = *reinterpret_cast<const float4*>(cs + j * kEncXP + s0 + 4);
+                const float4 c1a = *reinterpret_cast<const float4*>(cs + (j + 1) * kEncXP + s0);
+                const float4 c1b = *reinterpret_cast<const float4*>(cs + (j + 1) * kEncXP + s0 + 4);
+                const float c0[8] = {c0a.x, c0a.y, c0a.z, c0a.w, c0b.x, c0b.y, c0b.z, c0b.w};
+                const float c1[8] = {c1a.x, c1a.y, c1a.z, c1a.w, c1b.x, c1b.y, c1b.z, c1b.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const uint32_t bb = *reinterpret_cast<const uint32_t*>(bs + (size_t)(lane + 32 * m) * PB + j);
+                    const float b0 = __uint_as_float(bb << 16), b1 = __uint_as_float(bb & 0xffff0000u);
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        a[t][m] = __fmaf_rn(b0, c0[t], a[t][m]);
+                        a[t][m] = __fmaf_rn(b1, c1[t], a[t][m]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 xa = *reinterpret_cast<const float4*>(xs + (lane + 32 * m) * kEncXP + s0);
+                const float4 xb = *reinterpret_cast<const float4*>(xs + (lane + 32 * m) * kEncXP + s0 + 4);
+                const float x8[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                for (int t = 0; t < 8; ++t) a[t][m] = __fsub_rn(x8[t], a[t][m]);
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const int sl = s0 + t;
+                if (sl >= nvalid) break;
+                const float r4[4] = {a[t][0], a[t][1], a[t][2], a[t][3]};
+                quantize_store<BITS>(G, r4, sblk[sl], sR[sl], sprow[sl], rstage, chstage);
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------------------------------------
-// Encode kernel: one warp per (token row, keys or values): unit u = 2 row + z.  The block
-// holds both bases of its (group, kv-head) in shared memory as bf16 with a padded row pitch,
-// so that the projection (lanes along j) and the residual (lanes along i) are conflict-free.
+// Steps 4-6 alone on given residuals (test support): a warp per vector runs quantize_store
+// into a page-layout block of its own in `work` (rank 0, row 0), then copies the indices,
+// codes (int4 unpacked, sign-extended) and the scale out into plain arrays.
 // ------------------------------------------------------------------------------------
 template <int BITS>
-__global__ void __launch_bounds__(256) encode_kernel(const Geom G, const State S, const AppendCall C,
-                                                     const __nv_bfloat16* __restrict__ k_new,
-                                                     const __nv_bfloat16* __restrict__ v_new) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int h = blockIdx.y, warp = threadIdx.x >> 5;
-    __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem);
-    load_bases(G, S, C.g, h, bs);
-    __syncthreads();
-    const EncScratch W = enc_scratch(G, smem, warp);
-    const int nw = blockDim.x >> 5;
-    for (int unit = blockIdx.x * nw + warp; unit < 2 * C.total; unit += gridDim.x * nw)
-        encode_unit<BITS>(G, S, C, k_new, v_new, bs, W, h, unit);
+__global__ void __launch_bounds__(256) quantize_test_kernel(int n, int s, const float* __restrict__ r,
+                                                            uint8_t* idx, int8_t* codes, uint16_t* scales,
+                                                            uint8_t* work, uint32_t stride) {
+    __shared__ __align__(16) uint8_t stage[8 * kEncStage];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int v = blockIdx.x * 8 + warp;
+    if (v >= n) return;                         // whole warps
+    Geom G{};
+    G.s = s;                                    // the only field the steps read
+    float rr[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) rr[m] = r[(size_t)v * kD + lane + 32 * m];
+    uint8_t* blk = work + (size_t)v * stride;
+    float* rstage = reinterpret_cast<float*>(stage + warp * kEncStage);
+    quantize_store<BITS>(G, rr, blk, 0, 0, rstage, reinterpret_cast<uint8_t*>(rstage + kD));
+    __syncwarp();
+    for (int b = lane; b < s; b += 32) {
+        idx[(size_t)v * s + b] = blk[off_idx_of(0) + b];
+        int c;
+        if (BITS == 8) {
+            c = (int8_t)blk[off_codes_of(0, s) + b];
+        } else {
+            const uint32_t byte = blk[off_codes_of(0, s) + (b >> 1)];
+            c = (int)(((b & 1) ? byte >> 4 : byte) & 0xfu);
+            c = (c ^ 8) - 8;
+        }
+        codes[(size_t)v * s + b] = (int8_t)c;
+    }
+    if (lane == 0) scales[v] = *reinterpret_cast<const uint16_t*>(blk + off_scales_of(0, s, BITS));
 }
 
 // ------------------------------------------------------------------------------------
@@ -428,6 +617,10 @@ template __global__ void encode_kernel<8>(const Geom, const State, const AppendC
                                           const __nv_bfloat16*);
 template __global__ void encode_kernel<4>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
                                           const __nv_bfloat16*);
+template __global__ void quantize_test_kernel<8>(int, int, const float*, uint8_t*, int8_t*, uint16_t*, uint8_t*,
+                                                  uint32_t);
+template __global__ void quantize_test_kernel<4>(int, int, const float*, uint8_t*, int8_t*, uint16_t*, uint8_t*,
+                                                  uint32_t);
 template __global__ void append_small_kernel<8>(const Geom, const State, const AppendCall, const uint8_t*, int,
                                                 const __nv_bfloat16*, const __nv_bfloat16*);
 template __global__ void append_small_kernel<4>(const Geom, const State, const AppendCall, const uint8_t*, int,

@@ -71,6 +71,35 @@ __device__ __forceinline__ bool place_one(const Geom& G, const State& S, int seq
     return true;
 }
 
+// Shared memory of the bulk encode kernel (one tile of kEncTile rows, one of K or V):
+// the basis bf16 [kD][PB] (PB = RP + 2, RP = r_max rounded up to 16; the odd word pitch
+// makes column reads conflict-free), x and the stored coefficients fp32 [.][kEncXP] by slot,
+// per-slot destinations, tier counts, and each warp's code staging.
+constexpr int kEncTile = 64;
+constexpr int kEncXP = kEncTile + 4;
+constexpr int kEncStage = kD * 4 + kD;   // per warp: residuals and channels in rank order
+struct EncTileLayout {
+    uint32_t bs, xs, cs, sblk, sR, sprow, rslot, misc, cst, total;
+    int RP, PB;
+};
+__host__ __device__ inline EncTileLayout enc_tile_layout(int r_max) {
+    EncTileLayout L;
+    L.RP = (r_max + 15) / 16 * 16;
+    L.PB = L.RP + 2;
+    uint32_t o = 0;
+    L.bs = o;    o += (uint32_t)kD * L.PB * 2;  o = (o + 15u) & ~15u;
+    L.xs = o;    o += (uint32_t)kD * kEncXP * 4;
+    L.cs = o;    o += (uint32_t)L.RP * kEncXP * 4;
+    L.sblk = o;  o += kEncTile * 8;
+    L.sR = o;    o += kEncTile * 4;
+    L.sprow = o; o += kEncTile * 4;
+    L.rslot = o; o += kEncTile * 4;
+    L.misc = o;  o += 128;
+    L.cst = o;   o += 8 * kEncStage;
+    L.total = o;
+    return L;
+}
+
 // Shared-memory scratch of one encode warp: x [d], stored coefficients [kMaxRank], code staging.
 struct EncScratch {
     float* xs;
@@ -90,16 +119,129 @@ struct UnitIn {
     bool ok;
 };
 
+// Step 4 by its definition: s rounds of "largest remaining |r|, ties to the lower channel"
+// (channel = lane + 32 m).  Returns the selected channels as a bit mask over m.
+static __device__ __noinline__ uint32_t select_exact(float r0, float r1, float r2, float r3, int s) {
+    const int lane = threadIdx.x & 31;
+    const float r[4] = {r0, r1, r2, r3};
+    uint32_t key[4], sel = 0u;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) key[m] = __float_as_uint(fabsf(r[m])) + 1u;
+    for (int it = 0; it < s; ++it) {
+        uint32_t best = 0u, bm = 0u;
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            if (!((sel >> m) & 1u) && key[m] > best) { best = key[m]; bm = (uint32_t)m; }
+        const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
+        const uint32_t cand = (best == wmax && best != 0u) ? (bm * 32u + (uint32_t)lane) : 0xffffffffu;
+        const uint32_t wch = __reduce_min_sync(0xffffffffu, cand);
+        if ((int)(wch & 31u) == lane) sel |= 1u << (wch >> 5);
+    }
+    return sel;
+}
+
+// Steps 4-6 of one vector on one warp, from its residual r (channel lane + 32 m): top-s
+// selection, scale, codes, and the stores of indices, codes and scale into the vector's block
+// (blk: this vector's K or V block, row: its row in the page).  rstage / chstage: s floats
+// and s bytes of the warp's shared memory.
+//
+// Selection: each channel gets a 32-bit key, its |r| with the 7 lowest mantissa bits replaced
+// by 127 - channel.  The keys are distinct, and ordering them orders |r| at 2^-16 relative
+// resolution with ties to the lower channel.  The s largest keys come out of a warp merge of
+// each lane's 4 keys (sorted in registers) with one max-reduction per round.  If the s-th and
+// (s+1)-th largest keys differ above the 7 replaced bits, every selected |r| exceeds every
+// other one, so the set equals the exact top-s; otherwise (a near-tie at the boundary, e.g.
+// exact zeros) the selection is redone by its definition (select_exact).
+template <int BITS>
+__device__ __forceinline__ void quantize_store(const Geom& G, const float (&r)[4], uint8_t* blk, int R, int row,
+                                               float* rstage, uint8_t* chstage) {
+    const int lane = threadIdx.x & 31;
+    const int s = G.s;
+    const float qmax = BITS == 8 ? 127.f : 7.f;
+    uint32_t sel = 0u, mxb = 0u;
+    if (s > 0) {
+        uint32_t kk[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t b = __float_as_uint(fabsf(r[m]));
+            mxb = max(mxb, b);
+            kk[m] = (b & ~0x7fu) | (uint32_t)(127 - lane - 32 * m);
+        }
+        // the lane's keys, descending (distinct, so min / max order them fully)
+        uint32_t h0 = max(kk[0], kk[1]), h1 = min(kk[0], kk[1]);
+        uint32_t h2 = max(kk[2], kk[3]), h3 = min(kk[2], kk[3]);
+        {
+            const uint32_t a0 = max(h0, h2), a2 = min(h0, h2), a1 = max(h1, h3), a3 = min(h1, h3);
+            h0 = a0;
+            h1 = max(a1, a2);
+            h2 = min(a1, a2);
+            h3 = a3;
+        }
+        uint32_t K = 0u;
+        for (int it = 0; it < s; ++it) {
+            K = __reduce_max_sync(0xffffffffu, h0);
+            if (h0 == K) {
+                h0 = h1;
+                h1 = h2;
+                h2 = h3;
+                h3 = 0u;
+            }
+        }
+        const uint32_t K1 = s < kD ? __reduce_max_sync(0xffffffffu, h0) : 0u;
+        if (s < kD && ((K ^ K1) >> 7) == 0u) {
+            sel = select_exact(r[0], r[1], r[2], r[3], s);
+        } else {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) sel |= (kk[m] >= K ? 1u : 0u) << m;
+        }
+    }
+    // ---- 5-6: scale from the largest selected |r| (the largest of all), codes by rank
+    //      (ascending channel order); lane b takes rank b
+    const float amax = s > 0 ? __uint_as_float(__reduce_max_sync(0xffffffffu, mxb)) : 0.f;
+    const __half sh = __float2half_rn(__fdiv_rn(amax, qmax));
+    const float sf = __half2float(sh);
+    uint32_t before = 0u;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const bool on = (sel >> m) & 1u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, on);
+        if (on) {
+            const int rank = (int)(before + __popc(bal & ((1u << lane) - 1u)));
+            rstage[rank] = r[m];
+            chstage[rank] = (uint8_t)(lane + 32 * m);
+        }
+        before += __popc(bal);
+    }
+    if (lane == 0) *reinterpret_cast<__half*>(blk + off_scales_of(R, s, BITS) + row * 2) = sh;
+    __syncwarp();
+    for (int b0 = 0; b0 < s; b0 += 32) {
+        const int b = b0 + lane;
+        int code = 0;
+        if (b < s) {
+            float c = 0.f;
+            if (sf != 0.f) c = fminf(fmaxf(rintf(__fdiv_rn(rstage[b], sf)), -qmax), qmax);
+            code = (int)c;
+            blk[off_idx_of(R) + row * s + b] = chstage[b];
+            if (BITS == 8) blk[off_codes_of(R, s) + row * s + b] = (uint8_t)(int8_t)code;
+        }
+        if (BITS == 4) {
+            const int hi = __shfl_down_sync(0xffffffffu, code, 1);
+            if (b < s && !(b & 1))
+                blk[off_codes_of(R, s) + row * (s / 2) + (b >> 1)] = (uint8_t)((code & 0xf) | ((hi & 0xf) << 4));
+        }
+    }
+    __syncwarp();
+}
+
 // The six encode steps of one unit on one warp.
 template <int BITS>
 __device__ __forceinline__ void encode_body(const Geom& G, const State& S, const __nv_bfloat16* bs,
                                             const EncScratch& W, int unit, const UnitIn& in) {
     const int lane = threadIdx.x & 31;
-    const int P = G.r_max + 2, s = G.s;
+    const int P = G.r_max + 2;
     float* xs = W.xs;
     float* cs = W.cs;
     int8_t* cstage = W.cstage;
-    const float qmax = BITS == 8 ? 127.f : 7.f;
     do {
         const int z = unit & 1;
         if (!in.ok) break;
@@ -152,54 +294,7 @@ __device__ __forceinline__ void encode_body(const Geom& G, const State& S, const
 #pragma unroll
             for (int m = 0; m < 4; ++m) r[m] = __fsub_rn(xr[m], a[m]);
         }
-        // ---- 4: top-s by magnitude, ties to the lower channel (channel = lane + 32 m)
-        uint32_t key[4], sel = 0u;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) key[m] = __float_as_uint(fabsf(r[m])) + 1u;
-        for (int it = 0; it < s; ++it) {
-            uint32_t best = 0u, bm = 0u;
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-                if (!((sel >> m) & 1u) && key[m] > best) { best = key[m]; bm = (uint32_t)m; }
-            const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
-            const uint32_t cand = (best == wmax && best != 0u) ? (bm * 32u + (uint32_t)lane) : 0xffffffffu;
-            const uint32_t wch = __reduce_min_sync(0xffffffffu, cand);
-            if ((int)(wch & 31u) == lane) sel |= 1u << (wch >> 5);
-        }
-        // ---- 5-6: scale and codes; ranks give ascending channel order
-        {
-            uint32_t mx = 0u;
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-                if ((sel >> m) & 1u) mx = max(mx, key[m] - 1u);
-            const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, mx));
-            const __half sh = __float2half_rn(__fdiv_rn(amax, qmax));
-            const float sf = __half2float(sh);
-            uint32_t before = 0u;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const bool on = (sel >> m) & 1u;
-                const uint32_t bal = __ballot_sync(0xffffffffu, on);
-                if (on) {
-                    const int rank = (int)(before + __popc(bal & ((1u << lane) - 1u)));
-                    float c = 0.f;
-                    if (sf != 0.f) c = fminf(fmaxf(rintf(__fdiv_rn(r[m], sf)), -qmax), qmax);
-                    blk[off_idx_of(R) + dst.row * s + rank] = (uint8_t)(lane + 32 * m);
-                    if (BITS == 8) blk[off_codes_of(R, s) + dst.row * s + rank] = (uint8_t)(int8_t)c;
-                    else cstage[rank] = (int8_t)c;
-                }
-                before += __popc(bal);
-            }
-            if (lane == 0) *reinterpret_cast<__half*>(blk + off_scales_of(R, s, BITS) + dst.row * 2) = sh;
-        }
-        if (BITS == 4) {
-            __syncwarp();
-            for (int b = lane; b < s / 2; b += 32) {
-                const uint8_t lo = (uint8_t)cstage[2 * b] & 0xfu;
-                const uint8_t hi = (uint8_t)cstage[2 * b + 1] & 0xfu;
-                blk[off_codes_of(R, s) + dst.row * (s / 2) + b] = (uint8_t)(lo | (hi << 4));
-            }
-        }
+        quantize_store<BITS>(G, r, blk, R, dst.row, xs, reinterpret_cast<uint8_t*>(cstage));
     } while (false);
     __syncwarp();
 }

@@ -150,7 +150,8 @@ dwkv_status dwkv_seq_length(dwkv_handle h, int32_t seq, int32_t layer, int32_t* 
 
 /* Encodes and appends n_new[i] tokens to each listed sequence at `layer`.
  *   seq_ids, n_new : host int32 [n_seqs]; distinct ids; n_new[i] >= 0
- *   k_new, v_new   : device bf16 [sum(n_new)][Hkv][head_dim], sequences in list order
+ *   k_new, v_new   : device bf16 [sum(n_new)][Hkv][head_dim], sequences in list order,
+ *                    16-byte aligned (DWKV_ERR_INVALID_ARG otherwise)
  *   tier_idx       : device uint8 [sum(n_new)][Hkv], index into cfg.tiers.  A token's
  *                    tier is fixed by the first layer of its group that appends it
  *                    ([DW] §3 Eq. (2): rho_{m,h,t} has no layer index); later layers of
@@ -256,6 +257,22 @@ dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t w
 dwkv_status dwkv_decode_attention_noalloc(dwkv_handle h, int32_t layer, int32_t n_seqs,
                                           const int32_t* seq_ids, const void* q, float* out,
                                           void* stream);
+
+/* Test support: encode steps 4-6 on given residuals ([DW] §3: the residual is kept only on the
+ * routed channels, quantised), through the same device code the encoders use.  For each of n
+ * vectors: the s channels with the largest |r_i| (ties to the lower channel) in ascending
+ * channel order, the fp16 scale round(max |r_sel| / qmax) (qmax 127 or 7) and the codes
+ * clamp(rint(r_i / scale), -qmax, qmax) (all 0 when the scale is 0).
+ *   r      : device fp32 [n][head_dim] (head_dim = 128)
+ *   s      : 0..128, a multiple of 8;  bits : 8 or 4
+ *   idx    : device uint8 [n][s];  codes : device int8 [n][s] (one code per byte, int4 too)
+ *   scales : device fp16 bits [n]
+ *   work   : device scratch of at least dwkv_quantize_work_bytes(n, s, bits) bytes
+ * DWKV_ERR_INVALID_ARG for arguments out of range or NULL pointers (n > 0 and s > 0). */
+size_t dwkv_quantize_work_bytes(int32_t n, int32_t s, int32_t bits);
+dwkv_status dwkv_quantize_residuals(int32_t n, int32_t s, int32_t bits, const float* r, uint8_t* idx,
+                                    int8_t* codes, uint16_t* scales, void* work, size_t work_bytes,
+                                    void* stream);
 
 #ifdef __cplusplus
 }

@@ -39,6 +39,8 @@ def lib():
         L.oracle_decode_many.restype = i
         L.oracle_encode_vector.argtypes = [i, i, p, p, i, i, i, p, p, p, p, p, p]
         L.oracle_encode_vector.restype = i
+        L.oracle_quantize_residual.argtypes = [i, i, i, p, p, p, p]
+        L.oracle_quantize_residual.restype = i
         L.oracle_encode_many.argtypes = [i, i, i, p, p, p, i, i, p, p, p, p, p, i]
         L.oracle_encode_many.restype = i
         L.oracle_reconstruct.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, p]
@@ -225,6 +227,18 @@ def encode_vector(basis, x, r_t, s, bits):
     if rc != 0:
         raise ValueError("oracle_encode_vector: bad arguments")
     return {"coeff": coeff, "c32": c32, "idx": idx, "codes": codes, "scale": scale[0], "resid": resid}
+
+
+def quantize_residual(r, s, bits):
+    """Encode steps 4-6 on a given fp32 residual [d]: dict of idx (ascending), codes, scale (fp16 bits)."""
+    rv = _arr(r, np.float32).reshape(-1)
+    idx = np.zeros(s, np.uint8)
+    codes = np.zeros(s, np.int8)
+    scale = np.zeros(1, np.uint16)
+    rc = lib().oracle_quantize_residual(rv.shape[0], int(s), int(bits), _p(rv), _p(idx), _p(codes), _p(scale))
+    if rc != 0:
+        raise ValueError("oracle_quantize_residual: bad arguments")
+    return {"idx": idx, "codes": codes, "scale": scale[0]}
 
 
 def encode_many(basis, x, ranks, s, bits, nthreads=None, want_c32=False):

@@ -244,33 +244,13 @@ static int oracle_cmp_int(const void* pa, const void* pb) {
     return (a > b) - (a < b);
 }
 
-int oracle_encode_vector(int d, int r_max, const uint16_t* basis, const uint16_t* x, int r_t,
-                         int s, int bits, uint16_t* coeff, float* c32, uint8_t* idx, int8_t* codes,
-                         uint16_t* scale, float* resid) {
-    if (d <= 0 || d > 256 || r_t < 0 || r_t > r_max || s < 0 || s > d || (bits != 8 && bits != 4))
-        return -1;
-    float xf[256], cb[256], r[256];
+/* Steps 4-6 on a given residual r fp32 [d]: the s channels with the largest |r_i| (ties to the
+ * lower channel) in ascending channel order, the fp16 scale and the codes. */
+int oracle_quantize_residual(int d, int s, int bits, const float* r, uint8_t* idx, int8_t* codes,
+                             uint16_t* scale) {
+    if (d <= 0 || d > 256 || s < 0 || s > d || (bits != 8 && bits != 4)) return -1;
     oracle_rank_item items[256];
     int sel[256];
-    for (int i = 0; i < d; ++i) xf[i] = (float)oracle_bf16_to_f64(x[i]);
-    for (int j = 0; j < r_max; ++j) { coeff[j] = 0; if (c32) c32[j] = 0.0f; }
-    /* 1-2: projection and bf16 rounding */
-    for (int j = 0; j < r_t; ++j) {
-        float acc = 0.0f;
-        for (int i = 0; i < d; ++i)
-            acc = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), xf[i], acc);
-        if (c32) c32[j] = acc;
-        coeff[j] = oracle_f32_to_bf16_rn(acc);
-        cb[j] = (float)oracle_bf16_to_f64(coeff[j]);
-    }
-    /* 3: residual against the stored coefficients */
-    for (int i = 0; i < d; ++i) {
-        float a = 0.0f;
-        for (int j = 0; j < r_t; ++j)
-            a = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), cb[j], a);
-        r[i] = xf[i] - a;
-        if (resid) resid[i] = r[i];
-    }
     /* 4: top-s by magnitude, ties to the lower channel, then ascending channel order */
     for (int i = 0; i < d; ++i) { items[i].mag = fabsf(r[i]); items[i].ch = i; }
     qsort(items, (size_t)d, sizeof(items[0]), oracle_cmp_mag_desc);
@@ -293,6 +273,35 @@ int oracle_encode_vector(int d, int r_max, const uint16_t* basis, const uint16_t
         }
         codes[k] = (int8_t)c;
     }
+    return 0;
+}
+
+int oracle_encode_vector(int d, int r_max, const uint16_t* basis, const uint16_t* x, int r_t,
+                         int s, int bits, uint16_t* coeff, float* c32, uint8_t* idx, int8_t* codes,
+                         uint16_t* scale, float* resid) {
+    if (d <= 0 || d > 256 || r_t < 0 || r_t > r_max || s < 0 || s > d || (bits != 8 && bits != 4))
+        return -1;
+    float xf[256], cb[256], r[256];
+    for (int i = 0; i < d; ++i) xf[i] = (float)oracle_bf16_to_f64(x[i]);
+    for (int j = 0; j < r_max; ++j) { coeff[j] = 0; if (c32) c32[j] = 0.0f; }
+    /* 1-2: projection and bf16 rounding */
+    for (int j = 0; j < r_t; ++j) {
+        float acc = 0.0f;
+        for (int i = 0; i < d; ++i)
+            acc = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), xf[i], acc);
+        if (c32) c32[j] = acc;
+        coeff[j] = oracle_f32_to_bf16_rn(acc);
+        cb[j] = (float)oracle_bf16_to_f64(coeff[j]);
+    }
+    /* 3: residual against the stored coefficients */
+    for (int i = 0; i < d; ++i) {
+        float a = 0.0f;
+        for (int j = 0; j < r_t; ++j)
+            a = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), cb[j], a);
+        r[i] = xf[i] - a;
+        if (resid) resid[i] = r[i];
+    }
+    oracle_quantize_residual(d, s, bits, r, idx, codes, scale);
     return 0;
 }
 

@@ -28,7 +28,7 @@ import torch
 __all__ = [
     "Workload", "WORKLOADS", "workload", "seed_for", "make_bases", "make_context_lengths",
     "make_tiers", "make_compressed", "make_queries", "make_dense_vectors",
-    "ranks_of", "qmax_of",
+    "ranks_of", "qmax_of", "make_residual_cases",
 ]
 
 
@@ -284,3 +284,57 @@ def make_dense_vectors(wl: Workload, seq: int, layer: int, n: int, bases, device
                 x[:, h, ch] += torch.randn(n, k, generator=g, device=device) * math.sqrt(wl.outlier_var)
         out.append(x.to(torch.bfloat16).contiguous())
     return out[0], out[1]
+
+
+RESIDUAL_CASE_KINDS = ("gaussian", "boundary_ulp", "boundary_tie", "top_tie", "few_nonzero", "zeros",
+                       "subnormal", "huge", "half_steps")
+
+
+def make_residual_cases(n: int, d: int = 128, s: int = 16, seed: int = 77):
+    """Residual vectors fp32 ``[n][d]`` (numpy) for the selection / quantiser steps alone, made
+    to stress their boundaries; kind ``v % 9`` per vector (``RESIDUAL_CASE_KINDS``):
+    gaussian N(0, 1); the (s+1)-th largest magnitude moved to one ulp above or below the s-th;
+    a group of equal magnitudes (random signs) straddling rank s; equal magnitudes at the top;
+    fewer than s nonzero entries (the rest +0 / -0); all +0 / -0; subnormal magnitudes;
+    magnitudes so large that the fp16 scale overflows; values on exact half steps of a
+    power-of-two scale (an int4 scale of exactly 2^e: round-half-even cases).  Inputs only:
+    no selection happens here."""
+    import numpy as np
+    rng = np.random.default_rng(seed_for(seed, "resid_cases", n, d, s) & 0xFFFFFFFF)
+    out = rng.standard_normal((n, d)).astype(np.float32)
+    for v in range(n):
+        kind = v % len(RESIDUAL_CASE_KINDS)
+        r = out[v]
+        if kind == 1 and s < d:
+            order = np.argsort(-np.abs(r), kind="stable")
+            a, b = order[s - 1], order[s]
+            up = rng.integers(0, 2) == 1
+            mag = np.nextafter(np.abs(r[a]), np.float32(np.inf) if up else np.float32(0))
+            r[b] = np.float32(mag) * np.float32(1 if rng.integers(0, 2) else -1)
+        elif kind == 2 and s < d:
+            order = np.argsort(-np.abs(r), kind="stable")
+            lo, hi = max(0, s - 3), min(d, s + 3)
+            mag = np.abs(r[order[lo]])
+            for c in order[lo:hi]:
+                r[c] = mag * np.float32(1 if rng.integers(0, 2) else -1)
+        elif kind == 3:
+            ch = rng.choice(d, size=min(d, 5), replace=False)
+            r[ch] = np.float32(4.0) * np.where(rng.integers(0, 2, size=ch.size) == 1, 1, -1).astype(np.float32)
+        elif kind == 4:
+            k = int(rng.integers(0, max(1, s)))
+            keep = rng.choice(d, size=k, replace=False)
+            z = np.where(rng.integers(0, 2, size=d) == 1, np.float32(0.0), np.float32(-0.0))
+            z[keep] = r[keep]
+            out[v] = z
+        elif kind == 5:
+            out[v] = np.where(rng.integers(0, 2, size=d) == 1, np.float32(0.0), np.float32(-0.0))
+        elif kind == 6:
+            out[v] = (r * np.float32(1e-39)).astype(np.float32)
+        elif kind == 7:
+            out[v] = (r * np.float32(1e6)).astype(np.float32)
+        elif kind == 8:                 # int4: scale exactly 2^e, so r / scale lands on halves
+            e = int(rng.integers(-6, 3))
+            steps = rng.integers(-14, 15, size=d).astype(np.float32)
+            steps[int(rng.integers(0, d))] = np.float32(14 if rng.integers(0, 2) else -14)
+            out[v] = (steps * np.float32(0.5) * np.float32(2.0 ** e)).astype(np.float32)
+    return out
