@@ -192,6 +192,7 @@ struct dwkv_ctx {
     uint8_t* arena;
     size_t arena_bytes;
     int device, num_sms;
+    int enc_blocks_per_sm = 1;      // bulk encode kernel occupancy
     size_t smem_optin, smem_per_sm;
     std::vector<int32_t> len;       // [max_batch][L]
     std::vector<int32_t> placed;    // [max_batch][G]
@@ -437,6 +438,11 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
         const void* tiles[] = {(const void*)encode_kernel<8>, (const void*)encode_kernel<4>};
         for (const void* k : tiles)
             if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ets);
+        // bulk encode blocks resident per SM at this geometry's shared memory
+        int occ = 0;
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tiles[G.bits == 8 ? 0 : 1], 256, ets);
+        h->enc_blocks_per_sm = std::max(1, occ);
     }
     if (e != cudaSuccess) {
         delete h;
@@ -538,9 +544,9 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
         place_kernel<<<dim3(C.n, G.Hkv), 256, 0, s>>>(G, h->st, C, tier_idx);
         DWKV_CUDA(cudaGetLastError(), "place_kernel launch");
     }
-    // a block per (kv-head, K or V) and share of the tiles; two blocks fit an SM
+    // a block per (kv-head, K or V) and share of the tiles, one wave of resident blocks
     const long long ntiles = (C.total + kEncTile - 1) / kEncTile;
-    const long long per = std::max(1, h->num_sms / std::max(1, G.Hkv));
+    const long long per = std::max(1, h->enc_blocks_per_sm * h->num_sms / std::max(1, 2 * G.Hkv));
     const dim3 grid((unsigned)std::min(ntiles, per), G.Hkv, 2);
     const size_t tsm = encode_tile_smem(G);
     if (G.bits == 8)

@@ -190,7 +190,7 @@ __device__ __forceinline__ UnitIn encode_fetch(const Geom& G, const State& S, co
 // the stored bytes are identical to the per-warp encoders'.
 // ------------------------------------------------------------------------------------
 template <int BITS>
-__global__ void __launch_bounds__(256, 2) encode_kernel(const Geom G, const State S, const AppendCall C,
+__global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const State S, const AppendCall C,
                                                         const __nv_bfloat16* __restrict__ k_new,
                                                         const __nv_bfloat16* __restrict__ v_new) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -339,42 +339,40 @@ __global__ void __launch_bounds__(256, 2) encode_kernel(const Geom G, const Stat
         }
         __syncthreads();
 
-        // ---- 3: residual against the stored coefficients, then steps 4-6 per slot
-        for (int u = warp; 8 * u < nvalid; u += (int)(blockDim.x >> 5)) {
-            const int s0 = 8 * u, Ru = sR[s0];
-            float a[8][4];
+        // ---- 3: residual against the stored coefficients, then steps 4-6 per slot; items of
+        //      4 slots (16 a tile, taken w, w + 8, ...: a costly item with a cheaper one)
+        for (int u = warp; 4 * u < nvalid; u += (int)(blockDim.x >> 5)) {
+            const int s0 = 4 * u, Ru = sR[s0];
+            float a[4][4];
 #pragma unroll
-            for (int t = 0; t < 8; ++t)
+            for (int t = 0; t < 4; ++t)
 #pragma unroll
                 for (int m = 0; m < 4; ++m) a[t][m] = 0.f;
             for (int j = 0; j < Ru; j += 2) {          // ranks are multiples of 8
-                const float4 c0a = *reinterpret_cast<const float4*>(cs + j * kEncXP + s0);
-                const float4 c0b = *reinterpret_cast<const float4*>(cs + j * kEncXP + s0 + 4);
-                const float4 c1a = *reinterpret_cast<const float4*>(cs + (j + 1) * kEncXP + s0);
-                const float4 c1b = *reinterpret_cast<const float4*>(cs + (j + 1) * kEncXP + s0 + 4);
-                const float c0[8] = {c0a.x, c0a.y, c0a.z, c0a.w, c0b.x, c0b.y, c0b.z, c0b.w};
-                const float c1[8] = {c1a.x, c1a.y, c1a.z, c1a.w, c1b.x, c1b.y, c1b.z, c1b.w};
+                const float4 c0 = *reinterpret_cast<const float4*>(cs + j * kEncXP + s0);
+                const float4 c1 = *reinterpret_cast<const float4*>(cs + (j + 1) * kEncXP + s0);
+                const float c0v[4] = {c0.x, c0.y, c0.z, c0.w};
+                const float c1v[4] = {c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     const uint32_t bb = *reinterpret_cast<const uint32_t*>(bs + (size_t)(lane + 32 * m) * PB + j);
                     const float b0 = __uint_as_float(bb << 16), b1 = __uint_as_float(bb & 0xffff0000u);
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        a[t][m] = __fmaf_rn(b0, c0[t], a[t][m]);
-                        a[t][m] = __fmaf_rn(b1, c1[t], a[t][m]);
+                    for (int t = 0; t < 4; ++t) {
+                        a[t][m] = __fmaf_rn(b0, c0v[t], a[t][m]);
+                        a[t][m] = __fmaf_rn(b1, c1v[t], a[t][m]);
                     }
                 }
             }
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const float4 xa = *reinterpret_cast<const float4*>(xs + (lane + 32 * m) * kEncXP + s0);
-                const float4 xb = *reinterpret_cast<const float4*>(xs + (lane + 32 * m) * kEncXP + s0 + 4);
-                const float x8[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                const float x4[4] = {xa.x, xa.y, xa.z, xa.w};
 #pragma unroll
-                for (int t = 0; t < 8; ++t) a[t][m] = __fsub_rn(x8[t], a[t][m]);
+                for (int t = 0; t < 4; ++t) a[t][m] = __fsub_rn(x4[t], a[t][m]);
             }
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
+            for (int t = 0; t < 4; ++t) {
                 const int sl = s0 + t;
                 if (sl >= nvalid) break;
                 const float r4[4] = {a[t][0], a[t][1], a[t][2], a[t][3]};
