@@ -698,6 +698,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         const uint32_t ring = smem_addr(smem + L.ring);
         uint32_t head = 0, tail = 0;
         bool ok = true;
+        const uint64_t pol = l2_evict_first_policy();        // pages are read once a launch
         // lane j resolves page b0 + j of each batch; the next batch's ids are requested before
         // lane 0 issues the current batch, so their latency hides behind the issuing
         auto page_id = [&](uint32_t u, uint32_t& len) -> uint32_t {
@@ -746,7 +747,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                     m_slot[sl] = off;
                     head = off + len;
                     mbar_arrive_expect_tx(full0 + 8 * sl, len);
-                    bulk_g2s(ring + off, St.data + (size_t)t_src[j] * kUnit + (size_t)C.lig * len, len, full0 + 8 * sl);
+                    bulk_g2s_hint(ring + off, St.data + (size_t)t_src[j] * kUnit + (size_t)C.lig * len, len,
+                                  full0 + 8 * sl, pol);
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -1170,7 +1172,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             C.err[(size_t)ci * G.Hkv + h] = sqrtf(a) / (sqrtf(b) + 1e-6f);
         }
     }
-    if (tid == 0) St.tickets[(size_t)seq * G.Hkv + h] = 0u;
     if (tid == 0) {
         St.tickets[(size_t)seq * G.Hkv + h] = 0u;
         if (C.fused && C.place[ci]) {
