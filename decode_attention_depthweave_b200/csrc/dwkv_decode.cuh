@@ -1055,15 +1055,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             }
         }
     }
-    __threadfence();
     __syncthreads();
     if (tid == 0) {
-        const uint32_t t = atomicAdd(&St.tickets[(size_t)seq * G.Hkv + h], 1u);
+        // one acq_rel ticket: it releases the CTA's record (ordered before this thread by the
+        // barrier) at GPU scope, and the last CTA acquires every other CTA's record with it
+        uint32_t t;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(t) : "l"(St.tickets + (size_t)seq * G.Hkv + h) : "memory");
         m_misc[2] = (t == (uint32_t)(nsplit - 1)) ? 1u : 0u;
     }
     __syncthreads();
     if (!m_misc[2]) return;
-    __threadfence();
 
     // ================= last CTA of (sequence, kv-head): log-sum-exp merge of the records.
     // Every thread requests its outputs' values from the first kChunk records at once while
