@@ -18,7 +18,9 @@ in the timed region is the fused decode kernel, so its average launch duration i
 region's time over its launches (the roofline); a second replay with an external event
 around every launch is reported beside it.  The probe (dwkv_probe, one launch per layer)
 is timed over the same cache after the steps.  ``e2e`` repeats the step with host
-(pinned) inputs copied in and the outputs copied out inside the timed region.
+(pinned) inputs copied in (one block a step) and the outputs copied out inside the timed
+region.  ``step_distribution`` gives the median / p90 of up to 50 steps timed one by one
+(an event node between steps) and the eager (no graph) time of a step.
 
 ``--workload llama8b_encode_16k`` measures bulk encode instead: 4 sequences x 16384 new
 dense tokens per layer through dwkv_append (32 layers a step, the sequences reset between
@@ -215,15 +217,27 @@ def aggregate_rate(world: int, units_per_rank: float, ms: float) -> float:
 
 
 # ----------------------------------------------------------------------------- oracle sample
-def cpu_oracle_sample(wl, comp, tiers, bases, q, layer, t_sample, threads):
-    """Time the CPU oracle on the kv-heads of one layer over the first ``t_sample`` cached
-    tokens, on ``threads`` host threads.  Decode cost is linear in the context, so
-    seconds per full step = measured x (T / t_sample) x layers.  Returns (wall s, items)."""
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_oracle_sample(wl, comp, tiers, bases, q, layer, t_sample, threads, heads=None):
+    """Time the CPU oracle on the kv-heads of one layer (the first ``heads`` of them, default
+    all) over the first ``t_sample`` cached tokens, on ``threads`` host threads.  Decode cost
+    is linear in the context, so seconds per full step = measured x (T / t_sample) x layers.
+    Returns (wall s, items)."""
     import oracle
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from helpers import head_problem
     part = {k: v[:t_sample] for k, v in comp.items()}
-    items = [head_problem(wl, bases, tiers[:t_sample], part, q, layer, h) for h in range(wl.num_kv_heads)]
+    items = [head_problem(wl, bases, tiers[:t_sample], part, q, layer, h)
+             for h in range(wl.num_kv_heads if heads is None else heads)]
     t0 = time.perf_counter()
     oracle.decode_many(items, nthreads=threads)
     return time.perf_counter() - t0, len(items)
@@ -242,7 +256,9 @@ def run_dwkv(args, world, rank, local):
     dev = torch.device("cuda", local)
     T = args.context or wl.context
     n_steps = args.warmup + args.steps + args.e2e_steps
-    extra = args.profile_steps + 64
+    n_dist = min(args.steps, 50)                 # steps timed one by one (median / p90)
+    n_eager = 5                                  # steps launched without a graph
+    extra = args.profile_steps + n_dist + n_eager + 64
     B = 1
     bases = synth.make_bases(wl)
     cfg = dw.config_from(num_layers=wl.num_layers, layers_per_group=wl.layers_per_group,
@@ -403,14 +419,24 @@ def run_dwkv(args, world, rank, local):
     # ---- e2e: host inputs in, host outputs out, one step per graph replay
     e2e = None
     if args.e2e_steps > 0:
-        sK = torch.stack([Kn[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1).cpu().pin_memory()
-        sV = torch.stack([Vn[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1).cpu().pin_memory()
-        sQ = torch.stack([Qs[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1).cpu().pin_memory()
-        sT = torch.stack([Tn[g][args.warmup + args.steps:] for g in range(wl.num_groups)], 1).cpu().pin_memory()
-        dK = torch.empty_like(sK[0], device=dev)
-        dV = torch.empty_like(sV[0], device=dev)
-        dQ = torch.empty_like(sQ[0], device=dev)
-        dT = torch.empty_like(sT[0], device=dev)
+        sK = torch.stack([Kn[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1)
+        sV = torch.stack([Vn[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1)
+        sQ = torch.stack([Qs[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1)
+        sT = torch.stack([Tn[g][args.warmup + args.steps:] for g in range(wl.num_groups)], 1)
+        # one pinned host block per step (K | V | Q | tiers, each 16-byte aligned), one copy in
+        parts = [x.reshape(args.e2e_steps, -1).view(torch.uint8) for x in (sK, sV, sQ, sT)]
+        sizes = [x.shape[1] for x in parts]
+        offs = [0]
+        for n_ in sizes[:-1]:
+            offs.append(offs[-1] + (n_ + 15) // 16 * 16)
+        host_in = torch.zeros(args.e2e_steps, offs[-1] + sizes[-1], dtype=torch.uint8).pin_memory()
+        for x, o, n_ in zip(parts, offs, sizes):
+            host_in[:, o:o + n_] = x.cpu()
+        stage = torch.empty(host_in.shape[1], dtype=torch.uint8, device=dev)
+        dK = stage[offs[0]:offs[0] + sizes[0]].view(torch.bfloat16).view(sK.shape[1:])
+        dV = stage[offs[1]:offs[1] + sizes[1]].view(torch.bfloat16).view(sV.shape[1:])
+        dQ = stage[offs[2]:offs[2] + sizes[2]].view(torch.bfloat16).view(sQ.shape[1:])
+        dT = stage[offs[3]:offs[3] + sizes[3]].view(sT.shape[1:])
         host_out = torch.empty((args.e2e_steps,) + tuple(out.shape), dtype=torch.float32).pin_memory()
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e, stream=stream):
@@ -425,22 +451,50 @@ def run_dwkv(args, world, rank, local):
         with torch.cuda.stream(stream):
             a0.record(stream)
             for i in range(args.e2e_steps):
-                dK.copy_(sK[i], non_blocking=True)
-                dV.copy_(sV[i], non_blocking=True)
-                dQ.copy_(sQ[i], non_blocking=True)
-                dT.copy_(sT[i], non_blocking=True)
+                stage.copy_(host_in[i], non_blocking=True)
                 g_e2e.replay()
                 host_out[i].copy_(out, non_blocking=True)
             a1.record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
         e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / args.e2e_steps
-        h2d = sK[0].numel() * 2 + sV[0].numel() * 2 + sQ[0].numel() * 2 + sT[0].numel()
+        h2d = host_in.shape[1]
         d2h = out.numel() * 4
         assert torch.isfinite(host_out).all()
         e2e = {"value": round(aggregate_rate(world, B, e2e_ms), 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms, 4)}
     cache.sync(stream)
+
+    # ---- per-step distribution (one graph of n_dist steps, an event between steps) and the
+    #      eager time (the same launches without a graph); inputs of the timed steps reused
+    dist = None
+    if n_dist > 0:
+        sev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_dist + 1)]
+        g_dist = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_dist, stream=stream):
+            for i in range(n_dist):
+                sev[i].record(stream)
+                step(args.warmup + i % args.steps)
+            sev[n_dist].record(stream)
+        with torch.cuda.stream(stream):
+            g_dist.replay()
+        torch.cuda.synchronize(dev)
+        per = sorted(sev[i].elapsed_time(sev[i + 1]) for i in range(n_dist))
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for i in range(n_eager):
+                step(args.warmup + i % args.steps)
+            ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        cache.sync(stream)
+        dist = {"steps": n_dist, "ms_p50": round(statistics.median(per), 5),
+                "ms_p90": round(per[min(n_dist - 1, int(math.ceil(0.9 * n_dist)) - 1)], 5),
+                "ms_min": round(per[0], 5), "ms_max": round(per[-1], 5),
+                "eager_ms_per_step": round(ev0.elapsed_time(ev1) / n_eager, 5),
+                "timing": "graph of the steps with an event node between steps; eager: 32 launches a step "
+                          "from Python, no graph"}
 
     # ---- CPU oracle baseline (rank 0, N = 1 only): the 8 kv-heads of layer 0 at full context
     cpu = None
@@ -449,9 +503,16 @@ def run_dwkv(args, world, rank, local):
         dt, n_items = cpu_oracle_sample(wl, comp_cpu[0], tiers_cpu[0], bases, Qs[0][args.warmup][0].cpu(), 0,
                                         T - 1, threads)
         step_s = dt * wl.num_layers * wl.num_kv_heads / n_items
+        dt1, n1 = cpu_oracle_sample(wl, comp_cpu[0], tiers_cpu[0], bases, Qs[0][args.warmup][0].cpu(), 0,
+                                    T - 1, 1, heads=1)
+        step1_s = dt1 * wl.num_layers * wl.num_kv_heads / n1
         cpu = {"value": round(B / step_s, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"layer 0, {n_items} kv-heads x {T - 1} cached tokens (fp64 C oracle, {dt:.1f} s wall "
-                         f"on {threads} threads), scaled x{wl.num_layers} layers to one step"}
+                         f"on {threads} threads), scaled x{wl.num_layers} layers to one step",
+               "single_thread_value": round(B / step1_s, 6),
+               "single_thread_sample": f"layer 0, 1 kv-head x {T - 1} cached tokens on 1 thread ({dt1:.1f} s), "
+                                       f"scaled x{wl.num_kv_heads} heads x{wl.num_layers} layers",
+               "nproc": os.cpu_count(), "cpu_model": cpu_model()}
 
     value = aggregate_rate(world, B, ms_per_step)
     res = {
@@ -483,6 +544,7 @@ def run_dwkv(args, world, rank, local):
                   "achieved_gbs": round(probe_bytes / (probe_launch_ms * 1e-3) / 1e9, 1),
                   "frac": round(probe_bytes / (probe_launch_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                   "timing": f"graph of {wl.num_layers} probe launches, {args.profile_steps} replays after one warm-up"},
+        "step_distribution": dist,
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
