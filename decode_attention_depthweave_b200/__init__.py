@@ -22,7 +22,7 @@ __all__ = [
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage",
     "dwkv_sync_status", "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
-    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "Cache", "EXPORTED_SYMBOLS",
+    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "Cache", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -38,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage", "dwkv_sync_status",
     "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
-    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals",
+    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait",
 )
 
 
@@ -101,6 +101,7 @@ def lib():
             "dwkv_decode_attention_noalloc": ([vp, i32, i32, vp, vp, vp, vp], C.c_int),
             "dwkv_quantize_work_bytes": ([i32, i32, i32], sz),
             "dwkv_quantize_residuals": ([i32, i32, i32, vp, vp, vp, vp, vp, sz, vp], C.c_int),
+            "dwkv_check_bounded_wait": ([vp, C.c_uint32, vp], C.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -236,6 +237,10 @@ def dwkv_decode_attention_noalloc(h, layer, seq_ids, q, out, stream=None):
 def dwkv_probe(h, layer, seq_ids, q, err, out_full, workspace, stream=None):
     _check(lib().dwkv_probe(h, layer, len(seq_ids), _i32(seq_ids), _ptr(q), _ptr(err), _ptr(out_full),
                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dwkv_check_bounded_wait(h, limit_us, stream=None):
+    _check(lib().dwkv_check_bounded_wait(h, int(limit_us), _stream(stream)))
 
 
 def dwkv_quantize_work_bytes(n, s, bits) -> int:

@@ -29,6 +29,7 @@ template <int BITS>
 __global__ void export_kernel(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*, uint8_t*,
                               int8_t*, __half*);
 __global__ void reset_kernel(const Geom, const State, int);
+__global__ void wait_timeout_kernel(const State, uint64_t);
 template <int BITS, bool PROBE, int RMAX, int S>
 __global__ void decode_kernel(const Geom, const State, const DecodeCall);
 }  // namespace dwkv
@@ -798,6 +799,16 @@ dwkv_status dwkv_sync_status(dwkv_handle h, void* stream) {
                                   "free-page ring overflow"};
     const char* nm = w[0] < sizeof(names) / sizeof(names[0]) ? names[w[0]] : "unknown";
     return fail(DWKV_ERR_DEVICE_CHECK, "device check failed: %s (code %u, info %u, %u)", nm, w[0], w[1], w[2]);
+}
+
+dwkv_status dwkv_check_bounded_wait(dwkv_handle h, uint32_t limit_us, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if (limit_us < 1 || limit_us > 2000000u)
+        return fail(DWKV_ERR_INVALID_ARG, "limit_us = %u must be in 1..2000000", limit_us);
+    wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(h->st, (uint64_t)limit_us * 1000ull);
+    DWKV_CUDA(cudaGetLastError(), "wait_timeout_kernel launch");
+    return DWKV_OK;
 }
 
 static uint32_t quantize_stride(int32_t s, int32_t bits) {

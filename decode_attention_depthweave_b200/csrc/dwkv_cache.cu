@@ -383,6 +383,20 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
 }
 
 // ------------------------------------------------------------------------------------
+// The kernels' bounded wait, exercised (test support): one thread waits on a shared-memory
+// barrier that nothing arrives at; the wait runs out after limit_ns and the kernel records
+// DWKV_DEV_TIMEOUT in the device error word, as every kernel does, then returns.
+// ------------------------------------------------------------------------------------
+__global__ void wait_timeout_kernel(const State S, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = smem_addr(&bar);
+    mbar_init(b, 1);
+    fence_mbar_init();
+    if (!mbar_wait_for(b, 0, limit_ns)) set_dev_error(S, 6u /*DWKV_DEV_TIMEOUT*/, 0xfffffffeu, 0u);
+}
+
+// ------------------------------------------------------------------------------------
 // Steps 4-6 alone on given residuals (test support): a warp per vector runs quantize_store
 // into a page-layout block of its own in `work` (rank 0, row 0), then copies the indices,
 // codes (int4 unpacked, sign-extended) and the scale out into plain arrays.

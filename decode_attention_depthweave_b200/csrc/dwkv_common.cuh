@@ -210,16 +210,20 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-// Bounded wait for the phase of parity `parity` to complete: gives up after 2 s of wall
+// Bounded wait for the phase of parity `parity` to complete: gives up after limit_ns of wall
 // time (checked every 256 polls); the caller then records DWKV_DEV_TIMEOUT and stops
-// instead of spinning forever.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// instead of spinning forever.  The kernels use a 2 s limit.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0u && global_ns() - t0 > 2000000000ull) return false;
+        if ((it & 255u) == 0u && global_ns() - t0 > limit_ns) return false;
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // One bulk (non-tensor) global -> shared copy completing on an mbarrier.  Both addresses

@@ -258,6 +258,14 @@ dwkv_status dwkv_decode_attention_noalloc(dwkv_handle h, int32_t layer, int32_t 
                                           const int32_t* seq_ids, const void* q, float* out,
                                           void* stream);
 
+/* Test support for the kernels' bounded waits (every wait on a barrier, flag or copy gives up
+ * after a time limit, records DWKV_DEV_TIMEOUT in the handle's device error word and returns):
+ * launches one thread that waits on a shared-memory barrier nothing arrives at, through the
+ * same bounded-wait routine, with a limit of limit_us microseconds (1..2,000,000).  The wait
+ * runs out and the kernel returns; the context stays usable, and dwkv_sync_status then reports
+ * DWKV_ERR_DEVICE_CHECK ("bounded wait timed out") and clears the word. */
+dwkv_status dwkv_check_bounded_wait(dwkv_handle h, uint32_t limit_us, void* stream);
+
 /* Test support: encode steps 4-6 on given residuals ([DW] §3: the residual is kept only on the
  * routed channels, quantised), through the same device code the encoders use.  For each of n
  * vectors: the s channels with the largest |r_i| (ties to the lower channel) in ascending

@@ -150,3 +150,25 @@ def test_host_side_checks():
         cache.export(0, 0, 40, 20)
     cache.decode(0, [], q[:0])                      # empty call is a no-op
     cache.sync()
+
+
+def test_bounded_wait_runs_out_reports_and_leaves_the_context_usable():
+    """A wait that nothing ends: the kernels' bounded-wait routine gives up after its limit
+    (20 ms here), the error word says so through dwkv_sync_status, and decoding afterwards is
+    unaffected (the word is cleared by the report)."""
+    wl = synth.workload("tiny_1k")
+    bases = synth.make_bases(wl)
+    cache = dw.Cache(cfg_for(wl), bases[0], bases[1])
+    data = import_workload(cache, wl, [500])
+    cache.sync()
+    dw.dwkv_check_bounded_wait(cache.h, 20000)
+    with pytest.raises(dw.DwkvError, match="bounded wait timed out"):
+        cache.sync()
+    cache.sync()                                    # cleared
+    q = synth.make_queries(wl, 0, temperature=8.0)
+    out = cache.decode(0, [0], q.cuda())
+    cache.sync()
+    tiers, comp = data[(0, 0)]
+    check_close(out[0].cpu().numpy(), oracle.decode_head(head_problem(wl, bases, tiers, comp, q[0], 0, 0)))
+    with pytest.raises(dw.DwkvError, match="limit_us"):
+        dw.dwkv_check_bounded_wait(cache.h, 0)
