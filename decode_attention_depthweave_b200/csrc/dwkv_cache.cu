@@ -182,12 +182,14 @@ __device__ __forceinline__ UnitIn encode_fetch(const Geom& G, const State& S, co
 //      step); the group's chains run to the largest rank among its 32 slots (the first
 //      slot, by the sort), and the coefficients past a slot's own rank are neither stored
 //      nor kept: they enter its residual as exact zeros;
-//   3. residual items of 8 slots, lane = channels lane + 32 m: the chains over j run to the
-//      largest rank of the 8 slots; a zero coefficient adds an exact +-0 to an accumulator
+//   3. residual items of 4 slots, lane = channels lane + 32 m: the chains over j run to the
+//      largest rank of the 4 slots; a zero coefficient adds an exact +-0 to an accumulator
 //      that started at +0, which leaves it unchanged, so every slot gets the residual of
 //      its own-length chain; then steps 4-6 per slot (quantize_store).
 // The arithmetic per vector is the same operations in the same order as encode_body, so
-// the stored bytes are identical to the per-warp encoders'.
+// the stored bytes are identical to the per-warp encoders'.  Three 256-thread blocks fit an
+// SM (80 registers, ~72 KB of shared memory at r_max 64).  The kernel has no waits of its own
+// beyond block barriers.
 // ------------------------------------------------------------------------------------
 template <int BITS>
 __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const State S, const AppendCall C,
