@@ -189,3 +189,26 @@ def test_llama8b_64k_full_context_sampled_heads():
     for h in (0, 5):
         ref = oracle.decode_head(head_problem(wl, bases, tt, full, q[0].cpu(), 1, h))
         check_close(out[0, h * 4:(h + 1) * 4], ref, what=f"64K head {h}")
+
+
+# ------------------------------------------------------------------------------ residual widths
+@pytest.mark.parametrize("s,bits", [(0, 8), (0, 4), (32, 8), (32, 4)])
+def test_residual_channel_counts_decode_and_probe(s, bits):
+    """No residual at all (pure low-rank: the degenerate case of Eq. 1) and the widest
+    residual the kernels take; the probe is exactly 0 without a residual."""
+    wl = synth.workload("tiny_1k").scaled(resid_channels=s, resid_bits=bits, num_q_heads=8, num_kv_heads=2)
+    bases = synth.make_bases(wl)
+    cache = dw.Cache(cfg_for(wl), bases[0], bases[1])
+    data = import_workload(cache, wl, [700])
+    for layer in range(wl.num_layers):
+        _decode_and_check(wl, cache, data, [700], layer, temp=8.0, what=f"s={s} bits={bits}")
+    q = synth.make_queries(wl, 1, temperature=8.0)
+    err = cache.probe(1, [0], q.cuda())
+    cache.sync()
+    err = err.cpu().numpy()
+    tiers, comp = data[(0, 1)]
+    for h in range(wl.num_kv_heads):
+        e_ref, _, _ = oracle.probe_head(head_problem(wl, bases, tiers, comp, q[0], 1, h))
+        assert abs(err[0, h] - e_ref) <= 2e-3, (h, err[0, h], e_ref)
+    if s == 0:
+        assert float(np.abs(err).max()) == 0.0

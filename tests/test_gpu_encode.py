@@ -260,3 +260,18 @@ def test_decode_right_after_one_token_appends_across_page_boundaries():
         check_close(out[0].cpu().numpy(), ref, what=f"step {step}")
     pages1 = [(int((tiers == k).sum()) + 63) // 64 for k in range(len(wl.tiers))]
     assert pages1 != pages0, "the steps should have opened a new page in some tier"
+
+
+@pytest.mark.parametrize("s,bits", [(0, 8), (32, 4), (32, 8)])
+def test_encode_bit_exact_residual_counts(s, bits):
+    """Bulk encode with no residual and with the widest one, bit for bit against the oracle."""
+    wl = synth.workload("tiny_1k").scaled(resid_channels=s, resid_bits=bits, num_q_heads=8, num_kv_heads=2,
+                                          batch=2)
+    lengths = [300, 77]
+    cache, bases, dense = _encode_case(wl, lengths)
+    for b, T in enumerate(lengths):
+        for layer in range(wl.num_layers):
+            got = cache.export(layer, b, 0, T)
+            tiers = dense[(b, "t", layer // wl.layers_per_group)]
+            ref = oracle_encode_rows(wl, bases, layer, dense[(b, layer)][0], dense[(b, layer)][1], tiers)
+            _assert_same(got, ref, tiers, f"s={s} bits={bits} seq {b} layer {layer}")

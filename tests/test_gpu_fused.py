@@ -135,3 +135,12 @@ def test_fused_falls_back_to_two_launches_when_the_ring_is_capped():
     cache.sync()
     assert np.isfinite(out.cpu().numpy()).all()
     assert cache.seq_length(0, 0) == 101
+
+
+@pytest.mark.parametrize("s,bits", [(0, 4), (32, 8)])
+def test_fused_steps_residual_counts(s, bits):
+    wl = synth.workload("tiny_1k").scaled(resid_channels=s, resid_bits=bits)
+    T0, steps = 120, 10
+    fused, _ = _steps(wl, [T0], steps, fused=True)
+    plain, _ = _steps(wl, [T0], steps, fused=False, check=False)
+    _assert_same_bytes(fused, plain, wl, [T0 + steps])
