@@ -424,14 +424,8 @@ def run_dwkv(args, world, rank, local):
         sQ = torch.stack([Qs[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1)
         sT = torch.stack([Tn[g][args.warmup + args.steps:] for g in range(wl.num_groups)], 1)
         # one pinned host block per step (K | V | Q | tiers, each 16-byte aligned), one copy in
-        parts = [x.reshape(args.e2e_steps, -1).view(torch.uint8) for x in (sK, sV, sQ, sT)]
-        sizes = [x.shape[1] for x in parts]
-        offs = [0]
-        for n_ in sizes[:-1]:
-            offs.append(offs[-1] + (n_ + 15) // 16 * 16)
-        host_in = torch.zeros(args.e2e_steps, offs[-1] + sizes[-1], dtype=torch.uint8).pin_memory()
-        for x, o, n_ in zip(parts, offs, sizes):
-            host_in[:, o:o + n_] = x.cpu()
+        host_in, offs, sizes = pack_step_inputs((sK, sV, sQ, sT))
+        host_in = host_in.pin_memory()
         stage = torch.empty(host_in.shape[1], dtype=torch.uint8, device=dev)
         dK = stage[offs[0]:offs[0] + sizes[0]].view(torch.bfloat16).view(sK.shape[1:])
         dV = stage[offs[1]:offs[1] + sizes[1]].view(torch.bfloat16).view(sV.shape[1:])
@@ -551,6 +545,22 @@ def run_dwkv(args, world, rank, local):
     }
     cache.close()
     return res
+
+
+def pack_step_inputs(tensors):
+    """Per-step inputs packed for one host -> device copy a step: ``tensors`` are [steps, ...]
+    arrays of any dtype; returns (uint8 [steps, bytes] block, offsets, sizes), every part at a
+    16-byte-aligned offset (the library's alignment rule for k_new / v_new)."""
+    import torch
+    parts = [x.reshape(x.shape[0], -1).contiguous().view(torch.uint8) for x in tensors]
+    sizes = [x.shape[1] for x in parts]
+    offs = [0]
+    for n_ in sizes[:-1]:
+        offs.append(offs[-1] + (n_ + 15) // 16 * 16)
+    block = torch.zeros(parts[0].shape[0], offs[-1] + sizes[-1], dtype=torch.uint8)
+    for x, o, n_ in zip(parts, offs, sizes):
+        block[:, o:o + n_] = x.cpu()
+    return block, offs, sizes
 
 
 def fp32_alu_peak_tflops(sm_mhz: float, sms: int = 148) -> float:

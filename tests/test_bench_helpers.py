@@ -25,3 +25,27 @@ def test_token_bytes_of_the_64k_workload():
 def test_measured_peaks_is_read():
     p = bench.measured_peaks()
     assert p["hbm_gbs"] > 1000
+
+
+def test_pack_step_inputs_round_trips_with_aligned_parts():
+    import torch
+    steps = 3
+    k = torch.randn(steps, 4, 1, 8, 128).to(torch.bfloat16)
+    q = torch.randn(steps, 4, 1, 32, 128).to(torch.bfloat16)
+    t = torch.randint(0, 3, (steps, 2, 1, 5), dtype=torch.uint8)       # 10 bytes: forces padding
+    c = torch.randn(steps, 3).to(torch.bfloat16)
+    block, offs, sizes = bench.pack_step_inputs((k, t, q, c))
+    assert all(o % 16 == 0 for o in offs)
+    assert block.shape == (steps, offs[-1] + sizes[-1])
+    for i in range(steps):
+        row = block[i]
+        assert torch.equal(row[offs[0]:offs[0] + sizes[0]].view(torch.bfloat16).view(k.shape[1:]), k[i])
+        assert torch.equal(row[offs[1]:offs[1] + sizes[1]].view(t.shape[1:]), t[i])
+        assert torch.equal(row[offs[2]:offs[2] + sizes[2]].view(torch.bfloat16).view(q.shape[1:]), q[i])
+        assert torch.equal(row[offs[3]:offs[3] + sizes[3]].view(torch.bfloat16).view(c.shape[1:]), c[i])
+
+
+def test_fp32_alu_peak_from_unit_counts_and_clock():
+    # 148 SMs x 128 fp32 lanes x 2 flops (one FMA) x 1965 MHz
+    assert abs(bench.fp32_alu_peak_tflops(1965.0) - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
+    assert abs(bench.fp32_alu_peak_tflops(1965.0) - 74.45) < 0.01
