@@ -97,3 +97,25 @@ def test_product_package_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower(), f
+
+
+def test_test_support_entries_validate_on_the_host():
+    """The test-support calls refuse bad arguments before any launch (so without a GPU)."""
+    L = dw.lib()
+    assert L.dwkv_check_bounded_wait(None, 1000, None) == 1
+    r = C.c_void_p(256)
+    # s must be a multiple of 8 in 0..128, bits 8 or 4, pointers non-NULL, work large enough
+    assert L.dwkv_quantize_residuals(4, 12, 8, r, r, r, r, r, 1 << 20, None) == 1
+    assert "multiple of 8" in dw.dwkv_last_error()
+    assert L.dwkv_quantize_residuals(4, 16, 6, r, r, r, r, r, 1 << 20, None) == 1
+    assert L.dwkv_quantize_residuals(4, 16, 8, None, r, r, r, r, 1 << 20, None) == 1
+    need = dw.dwkv_quantize_work_bytes(4, 16, 8)
+    assert need > 0 and need % 16 == 0
+    assert L.dwkv_quantize_residuals(4, 16, 8, r, r, r, r, r, need - 16, None) == 1
+    assert "needs" in dw.dwkv_last_error()
+    assert L.dwkv_quantize_residuals(0, 16, 8, None, None, None, None, None, 0, None) == 0   # nothing to do
+    # one page-layout block a vector: s idx bytes, then the codes at 64 s, the scale at 64 s + 8 s b
+    for s, b in ((16, 4), (32, 8), (0, 8)):
+        per = (64 * s + 8 * s * b + 2 + 15) // 16 * 16
+        assert dw.dwkv_quantize_work_bytes(3, s, b) == 3 * per
+    assert dw.dwkv_quantize_work_bytes(3, 16, 5) == 0
