@@ -99,11 +99,37 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, uuid: str | None = None):
         self.gpu = gpu_index
+        self.uuid = uuid
         self.proc = None
         self.path = None
         self.t0 = self.t1 = None
+        self.nvml = []                  # (t, sm_mhz, max_mhz, reasons bitmask) every ~1 ms
+        self._stop = None
+        self._thread = None
+
+    def _nvml_loop(self):
+        """SM clock and clock-event reasons read through NVML about every millisecond, so that
+        a timed region of a few tens of ms still holds many samples."""
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                hd = pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else None
+            except pynvml.NVMLError:
+                hd = None
+            if hd is None:
+                hd = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(hd, pynvml.NVML_CLOCK_SM)
+            reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons",
+                              getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+            while not self._stop.is_set():
+                self.nvml.append((time.time(), pynvml.nvmlDeviceGetClockInfo(hd, pynvml.NVML_CLOCK_SM), mx,
+                                  int(reasons(hd)) if reasons else 0))
+                time.sleep(0.001)
+        except Exception:              # no NVML: the nvidia-smi samples stand alone
+            pass
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
@@ -121,6 +147,10 @@ class ClockSampler:
             if os.path.getsize(self.path) > 0:
                 break
             time.sleep(0.05)
+        import threading
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._nvml_loop, daemon=True)
+        self._thread.start()
         time.sleep(0.2)
         return self
 
@@ -131,6 +161,9 @@ class ClockSampler:
         self.t1 = time.time()
 
     def __exit__(self, *exc):
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
         if self.proc is not None:
             time.sleep(0.1)
             self.proc.terminate()
@@ -163,14 +196,23 @@ class ClockSampler:
 
         inside = [r for r in rows if self.t0 and ts(r[0]) is not None and self.t0 - 0.01 <= ts(r[0]) <= self.t1 + 0.01]
         use = inside if inside else rows
-        if not use:
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        # NVML reason bits of the same four events (nvmlClocksEventReason*)
+        bits = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+        nv_in = [x for x in self.nvml if self.t0 and self.t0 <= x[0] <= self.t1]
+        if not use and not nv_in:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         sm = [num(r[2]) for r in use if num(r[2]) is not None]
         mx = [num(r[3]) for r in use if num(r[3]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in use for i in range(4) if r[6 + i].lower().startswith("active")})
+        reasons = {names[i] for r in use for i in range(4) if r[6 + i].lower().startswith("active")}
+        if nv_in:
+            sm = [float(x[1]) for x in nv_in]
+            mx = mx + [float(x[2]) for x in nv_in]
+            reasons |= {n for n in names for x in nv_in if x[3] & bits[n]}
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(use), "samples_in_region": len(inside)}
+                "reasons": sorted(reasons), "samples": len(use) + len(nv_in),
+                "samples_in_region": len(inside) + len(nv_in),
+                "sources": {"nvidia_smi_20ms_in_region": len(inside), "nvml_1ms_in_region": len(nv_in)}}
 
 
 # ----------------------------------------------------------------------------- dist
@@ -227,95 +269,112 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_oracle_sample(wl, comp, tiers, bases, q, layer, t_sample, threads, heads=None):
-    """Time the CPU oracle on the kv-heads of one layer (the first ``heads`` of them, default
-    all) over the first ``t_sample`` cached tokens, on ``threads`` host threads.  Decode cost
-    is linear in the context, so seconds per full step = measured x (T / t_sample) x layers.
-    Returns (wall s, items)."""
+def cpu_oracle_sample(wl, probs_in, threads):
+    """Time the CPU oracle on the given (layer, kv-head) problems on ``threads`` host threads.
+    ``probs_in`` is a list of (bases, tier_idx, comp, q, layer, head).  Returns wall seconds."""
     import oracle
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from helpers import head_problem
-    part = {k: v[:t_sample] for k, v in comp.items()}
-    items = [head_problem(wl, bases, tiers[:t_sample], part, q, layer, h)
-             for h in range(wl.num_kv_heads if heads is None else heads)]
+    items = [oracle.head_problem(wl, b, t, c, q, layer, h) for (b, t, c, q, layer, h) in probs_in]
     t0 = time.perf_counter()
     oracle.decode_many(items, nthreads=threads)
-    return time.perf_counter() - t0, len(items)
+    return time.perf_counter() - t0
+
+
+def oracle_layers_for(wl, cores: int) -> int:
+    """Layers whose kv-heads give every host core at least one (layer, kv-head) problem."""
+    return max(1, min(wl.num_layers, -(-cores // wl.num_kv_heads)))
 
 
 # ----------------------------------------------------------------------------- main path
-def run_dwkv(args, world, rank, local):
+def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e2e_steps=None, light=False):
+    """One decode workload: import the synthetic compressed cache of every sequence, then time
+    K steps of (per layer) one fused append + decode launch over all sequences.  ``light``
+    skips the per-step distribution and the event-bracketed replay (extra workloads of the
+    default run)."""
     import torch
 
     import decode_attention_depthweave_b200 as dw
     import synth
 
-    wl = synth.workload(args.workload)
+    name = workload or args.workload
+    steps = args.steps if steps is None else steps
+    warmup = args.warmup if warmup is None else warmup
+    e2e_steps = args.e2e_steps if e2e_steps is None else e2e_steps
+    wl = synth.workload(name)
     if args.layers:
         wl = wl.scaled(num_layers=args.layers)
     dev = torch.device("cuda", local)
-    T = args.context or wl.context
-    n_steps = args.warmup + args.steps + args.e2e_steps
-    n_dist = min(args.steps, 50)                 # steps timed one by one (median / p90)
-    n_eager = 5                                  # steps launched without a graph
-    extra = args.profile_steps + n_dist + n_eager + 64
-    B = 1
+    B = wl.batch
+    lengths = [args.context] * B if args.context else synth.make_context_lengths(wl)
+    seqs = list(range(B))
+    sid = [rank * B + b for b in seqs]                 # seed index of each sequence (replicas differ)
+    n_steps = warmup + steps + e2e_steps
+    n_dist = 0 if light else min(steps, 50)           # steps timed one by one (median / p90)
+    n_eager = 0 if light else 5                        # steps launched without a graph
+    prof_steps = 0 if light else args.profile_steps
+    extra = prof_steps + n_dist + n_eager + 64
     bases = synth.make_bases(wl)
     cfg = dw.config_from(num_layers=wl.num_layers, layers_per_group=wl.layers_per_group,
                          num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim,
                          r_max=wl.r_max, tiers=wl.tiers, resid_channels=wl.resid_channels,
-                         resid_bits=wl.resid_bits, max_batch=B, max_context=T + n_steps + extra)
+                         resid_bits=wl.resid_bits, max_batch=B, max_context=max(lengths) + n_steps + extra)
     stream = torch.cuda.Stream(device=dev)
     cache = dw.Cache(cfg, bases[0], bases[1], device=dev, ws_seqs=B, stream=stream)
     if args.tuning:
         c, w_, s_ = (int(x) for x in args.tuning.split(","))
         cache.set_decode_tuning(c, w_, s_)
     h = cache.h
-
-    # ---- import the T-1 cached tokens (seeded synthetic compressed form)
-    keep_layers = {0} if (rank == 0 and world == 1 and not args.no_cpu_baseline) else set()
-    tiers_dev, comp_cpu, tiers_cpu = {}, {}, {}
-    tier_counts = torch.zeros(wl.num_groups, wl.num_kv_heads, len(wl.tiers), dtype=torch.int64)
-    with torch.cuda.stream(stream):
-        for layer in range(wl.num_layers):
-            g = layer // wl.layers_per_group
-            if g not in tiers_dev:
-                tiers_dev[g] = synth.make_tiers(wl, rank, g, T - 1, device=dev)
-                for k in range(len(wl.tiers)):
-                    tier_counts[g, :, k] = (tiers_dev[g] == k).sum(0).cpu()
-            comp = synth.make_compressed(wl, rank, layer, tiers_dev[g], device=dev)
-            cache.append_compressed(layer, [0], [T - 1], tiers_dev[g], comp["coeff"], comp["idx"],
-                                    comp["codes"], comp["scales"], stream=stream)
-            if layer in keep_layers:
-                comp_cpu[layer] = {k: v.cpu() for k, v in comp.items()}
-                tiers_cpu[g] = tiers_dev[g].cpu()
-            del comp
-    cache.sync(stream)
-
-    # ---- per-step inputs, resident in HBM
-    Kn, Vn, Qs = [], [], []
-    Tn = {}
-    for layer in range(wl.num_layers):
-        k, v = synth.make_dense_vectors(wl, rank, layer, n_steps, bases, device=dev, start=T - 1)
-        Kn.append(k.view(n_steps, 1, wl.num_kv_heads, wl.head_dim))
-        Vn.append(v.view(n_steps, 1, wl.num_kv_heads, wl.head_dim))
-        Qs.append(synth.make_queries(wl, layer, batch=n_steps, device=dev).view(n_steps, 1, wl.num_q_heads, wl.head_dim))
-        g = layer // wl.layers_per_group
-        if g not in Tn:
-            Tn[g] = synth.make_tiers(wl, rank, g, n_steps, device=dev, start=T - 1).view(n_steps, 1, wl.num_kv_heads)
-            for k_ in range(len(wl.tiers)):
-                tier_counts[g, :, k_] += (Tn[g][: args.warmup + args.steps] == k_).sum((0, 1)).cpu()
-    out = torch.empty(wl.num_layers, 1, wl.num_q_heads, wl.head_dim, dtype=torch.float32, device=dev)
-    ws = cache.workspace
     lpg = wl.layers_per_group
 
+    # ---- import the T_b - 1 cached tokens of every sequence (seeded synthetic compressed form)
+    do_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    cores = os.cpu_count() or 1
+    keep_layers = set(range(oracle_layers_for(wl, cores))) if do_cpu else set()
+    comp_cpu, tiers_cpu = {}, {}
+    tier_counts = torch.zeros(len(wl.tiers), dtype=torch.int64)
+    with torch.cuda.stream(stream):
+        for b in seqs:
+            tiers_dev = {}
+            for layer in range(wl.num_layers):
+                g = layer // lpg
+                if g not in tiers_dev:
+                    tiers_dev[g] = synth.make_tiers(wl, sid[b], g, lengths[b] - 1, device=dev)
+                    tier_counts += torch.bincount(tiers_dev[g].reshape(-1).long(), minlength=len(wl.tiers)).cpu()
+                comp = synth.make_compressed(wl, sid[b], layer, tiers_dev[g], device=dev)
+                cache.append_compressed(layer, [b], [lengths[b] - 1], tiers_dev[g], comp["coeff"], comp["idx"],
+                                        comp["codes"], comp["scales"], stream=stream)
+                if b == 0 and layer in keep_layers:
+                    comp_cpu[layer] = {k: v.cpu() for k, v in comp.items()}
+                    tiers_cpu[layer] = tiers_dev[g].cpu()
+                del comp
+            del tiers_dev
+    cache.sync(stream)
+
+    # ---- per-step inputs of every sequence, resident in HBM: [steps][B][...]
+    Kn, Vn, Qs, Tn = [], [], [], {}
+    for layer in range(wl.num_layers):
+        kv = [synth.make_dense_vectors(wl, sid[b], layer, n_steps, bases, device=dev, start=lengths[b] - 1)
+              for b in seqs]
+        Kn.append(torch.stack([x[0] for x in kv], 1).contiguous())
+        Vn.append(torch.stack([x[1] for x in kv], 1).contiguous())
+        del kv
+        Qs.append(synth.make_queries(wl, layer, batch=n_steps * B, device=dev, step=rank)
+                  .view(n_steps, B, wl.num_q_heads, wl.head_dim))
+        g = layer // lpg
+        if g not in Tn:
+            Tn[g] = torch.stack([synth.make_tiers(wl, sid[b], g, n_steps, device=dev, start=lengths[b] - 1)
+                                 for b in seqs], 1).contiguous()
+            tier_counts += torch.bincount(Tn[g][: warmup + steps].reshape(-1).long(), minlength=len(wl.tiers)).cpu()
+    out = torch.empty(wl.num_layers, B, wl.num_q_heads, wl.head_dim, dtype=torch.float32, device=dev)
+    ws = cache.workspace
+
     def step(s, ev=None):
-        # per layer, one launch: append the step's token and attend over the whole context
+        # per layer, one launch: append the step's token of every sequence and attend over
+        # each sequence's whole context
         for layer in range(wl.num_layers):
             g = layer // lpg
             if ev is not None:
                 ev[layer][0].record(stream)
-            dw.dwkv_append_decode_attention(h, layer, [0], Kn[layer][s], Vn[layer][s],
+            dw.dwkv_append_decode_attention(h, layer, seqs, Kn[layer][s], Vn[layer][s],
                                             Tn[g][s] if layer % lpg == 0 else None, Qs[layer][s], out[layer], ws,
                                             stream)
             if ev is not None:
@@ -327,7 +386,7 @@ def run_dwkv(args, world, rank, local):
     torch.cuda.synchronize(dev)
     g_warm = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_warm, stream=stream):
-        for s in range(args.warmup):
+        for s in range(warmup):
             step(s)
     with torch.cuda.stream(stream):
         g_warm.replay()
@@ -337,13 +396,13 @@ def run_dwkv(args, world, rank, local):
     # ---- timed: K steps in one graph, replayed once
     g_main = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_main, stream=stream):
-        for s in range(args.warmup, args.warmup + args.steps):
+        for s in range(warmup, warmup + steps):
             step(s)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, gpu_uuid(local)) as clk:
         clk.mark_start()
         with torch.cuda.stream(stream):
             e0.record(stream)
@@ -355,57 +414,60 @@ def run_dwkv(args, world, rank, local):
     ms_total = e0.elapsed_time(e1)
     cache.sync(stream)
     ms_total = max_over_ranks(world, ms_total)
-    ms_per_step = ms_total / args.steps
+    ms_per_step = ms_total / steps
     clocks = clk.summary()
+    del g_warm
 
-    # ---- per-launch durations bracketed by CUDA events, for reference: same K steps (state
-    #      rewound is not needed: a re-run appends K more tokens, which changes the work by
-    #      < 0.1 %).  The event nodes between launches add their own gaps, so the roofline
-    #      below uses the timed region instead, where every launch is this kernel.
-    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-            for _ in range(wl.num_layers)] for _ in range(args.profile_steps)]
-    g_prof = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_prof, stream=stream):
-        for i in range(args.profile_steps):
-            step(args.warmup + i, evs[i])
-    with torch.cuda.stream(stream):
-        g_prof.replay()
-    torch.cuda.synchronize(dev)
-    dec_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(args.profile_steps) for l in range(wl.num_layers)]
-    dec_ms_mean = statistics.mean(dec_ms)
+    # ---- per-launch durations bracketed by CUDA events, for reference (re-running the timed
+    #      steps appends more tokens, which changes the work by < 0.1 %).  The event nodes
+    #      between launches add their own gaps, so the roofline below uses the timed region.
+    dec_ms_mean = None
+    if prof_steps:
+        evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+                for _ in range(wl.num_layers)] for _ in range(prof_steps)]
+        g_prof = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_prof, stream=stream):
+            for i in range(prof_steps):
+                step(warmup + i, evs[i])
+        with torch.cuda.stream(stream):
+            g_prof.replay()
+        torch.cuda.synchronize(dev)
+        dec_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(prof_steps) for l in range(wl.num_layers)]
+        dec_ms_mean = statistics.mean(dec_ms)
 
     # ---- probe (with / without residual, one launch per layer) over the same cache
-    err = torch.empty(wl.num_layers, 1, wl.num_kv_heads, dtype=torch.float32, device=dev)
+    err = torch.empty(wl.num_layers, B, wl.num_kv_heads, dtype=torch.float32, device=dev)
     g_probe = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_probe, stream=stream):
         for layer in range(wl.num_layers):
-            dw.dwkv_probe(h, layer, [0], Qs[layer][args.warmup], err[layer], None, ws, stream)
+            dw.dwkv_probe(h, layer, seqs, Qs[layer][warmup], err[layer], None, ws, stream)
     p0 = torch.cuda.Event(enable_timing=True)
     p1 = torch.cuda.Event(enable_timing=True)
+    probe_reps = max(prof_steps, 1)
     with torch.cuda.stream(stream):
         g_probe.replay()
         p0.record(stream)
-        for _ in range(args.profile_steps):
+        for _ in range(probe_reps):
             g_probe.replay()
         p1.record(stream)
     torch.cuda.synchronize(dev)
     cache.sync(stream)
     assert torch.isfinite(err).all()
-    probe_launch_ms = p0.elapsed_time(p1) / (args.profile_steps * wl.num_layers)
-    held_probe = T - 1 + args.warmup + args.steps + args.profile_steps
+    probe_launch_ms = p0.elapsed_time(p1) / (probe_reps * wl.num_layers)
+    held_probe = sum(lengths) - B + B * (warmup + steps + prof_steps)
 
     # ---- algorithmic bytes: every stored byte of the attended tokens (per-token bytes of
-    #      its tier), plus the two bases, the query and the output of each launch
-    held = T - 1 + args.warmup + args.steps                  # tokens per head after the timed steps
+    #      its tier), plus the two bases, the queries and the outputs of each launch
+    held = sum(lengths) - B + B * (warmup + steps)            # tokens per head after the timed steps
     tok_bytes = torch.tensor([token_bytes(r, wl.resid_channels, wl.resid_bits) for r in wl.tiers], dtype=torch.float64)
     bytes_per_tok_head = float((tier_counts.double() * tok_bytes).sum()) / (wl.num_groups * wl.num_kv_heads * held)
     basis_bytes = 2 * wl.num_kv_heads * wl.head_dim * wl.r_max * 2
-    io_bytes = wl.num_q_heads * wl.head_dim * (2 + 4)
+    io_bytes = B * wl.num_q_heads * wl.head_dim * (2 + 4)
 
     def layer_bytes(ctx):
         return bytes_per_tok_head * wl.num_kv_heads * ctx + basis_bytes + io_bytes
 
-    ctx_timed = T - 1 + args.warmup + (args.steps + 1) / 2.0   # mean attended context in the timed steps
+    ctx_timed = sum(lengths) - B + B * (warmup + (steps + 1) / 2.0)   # attended tokens of all sequences, mean over the timed steps
     comp_bytes_layer = bytes_per_tok_head * wl.num_kv_heads * ctx_timed
     peaks = measured_peaks()
     # the timed region holds nothing but the fused decode kernel (one launch per layer): its
@@ -413,30 +475,33 @@ def run_dwkv(args, world, rank, local):
     launch_ms = ms_per_step / launches_per_step
     alg_bytes = layer_bytes(ctx_timed)
     achieved = alg_bytes / (launch_ms * 1e-3) / 1e9
-    traffic = profiled_traffic(args.workload)
-    probe_bytes = layer_bytes(held_probe) - wl.num_q_heads * wl.head_dim * 4 + wl.num_kv_heads * 4
+    traffic = profiled_traffic(name)
+    probe_bytes = layer_bytes(held_probe) - B * wl.num_q_heads * wl.head_dim * 4 + B * wl.num_kv_heads * 4
 
     # ---- e2e: host inputs in, host outputs out, one step per graph replay
     e2e = None
-    if args.e2e_steps > 0:
-        sK = torch.stack([Kn[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1)
-        sV = torch.stack([Vn[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1)
-        sQ = torch.stack([Qs[l][args.warmup + args.steps:] for l in range(wl.num_layers)], 1)
-        sT = torch.stack([Tn[g][args.warmup + args.steps:] for g in range(wl.num_groups)], 1)
+    if e2e_steps > 0:
+        s0 = warmup + steps
+        sK = torch.stack([Kn[l][s0:] for l in range(wl.num_layers)], 1)
+        sV = torch.stack([Vn[l][s0:] for l in range(wl.num_layers)], 1)
+        sQ = torch.stack([Qs[l][s0:] for l in range(wl.num_layers)], 1)
+        sT = torch.stack([Tn[g][s0:] for g in range(wl.num_groups)], 1)
         # one pinned host block per step (K | V | Q | tiers, each 16-byte aligned), one copy in
         host_in, offs, sizes = pack_step_inputs((sK, sV, sQ, sT))
+        del sK, sV, sQ, sT
         host_in = host_in.pin_memory()
         stage = torch.empty(host_in.shape[1], dtype=torch.uint8, device=dev)
-        dK = stage[offs[0]:offs[0] + sizes[0]].view(torch.bfloat16).view(sK.shape[1:])
-        dV = stage[offs[1]:offs[1] + sizes[1]].view(torch.bfloat16).view(sV.shape[1:])
-        dQ = stage[offs[2]:offs[2] + sizes[2]].view(torch.bfloat16).view(sQ.shape[1:])
-        dT = stage[offs[3]:offs[3] + sizes[3]].view(sT.shape[1:])
-        host_out = torch.empty((args.e2e_steps,) + tuple(out.shape), dtype=torch.float32).pin_memory()
+        shp = lambda *t: (wl.num_layers,) + t                                       # noqa: E731
+        dK = stage[offs[0]:offs[0] + sizes[0]].view(torch.bfloat16).view(shp(B, wl.num_kv_heads, wl.head_dim))
+        dV = stage[offs[1]:offs[1] + sizes[1]].view(torch.bfloat16).view(shp(B, wl.num_kv_heads, wl.head_dim))
+        dQ = stage[offs[2]:offs[2] + sizes[2]].view(torch.bfloat16).view(shp(B, wl.num_q_heads, wl.head_dim))
+        dT = stage[offs[3]:offs[3] + sizes[3]].view(wl.num_groups, B, wl.num_kv_heads)
+        host_out = torch.empty((e2e_steps,) + tuple(out.shape), dtype=torch.float32).pin_memory()
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e, stream=stream):
             for layer in range(wl.num_layers):
                 g = layer // lpg
-                dw.dwkv_append_decode_attention(h, layer, [0], dK[layer], dV[layer],
+                dw.dwkv_append_decode_attention(h, layer, seqs, dK[layer], dV[layer],
                                                 dT[g] if layer % lpg == 0 else None, dQ[layer], out[layer], ws, stream)
         torch.cuda.synchronize(dev)
         barrier(world)
@@ -444,19 +509,20 @@ def run_dwkv(args, world, rank, local):
         a1 = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             a0.record(stream)
-            for i in range(args.e2e_steps):
+            for i in range(e2e_steps):
                 stage.copy_(host_in[i], non_blocking=True)
                 g_e2e.replay()
                 host_out[i].copy_(out, non_blocking=True)
             a1.record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
-        e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / args.e2e_steps
+        e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / e2e_steps
         h2d = host_in.shape[1]
         d2h = out.numel() * 4
         assert torch.isfinite(host_out).all()
         e2e = {"value": round(aggregate_rate(world, B, e2e_ms), 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms, 4)}
+        del g_e2e
     cache.sync(stream)
 
     # ---- per-step distribution (one graph of n_dist steps, an event between steps) and the
@@ -468,7 +534,7 @@ def run_dwkv(args, world, rank, local):
         with torch.cuda.graph(g_dist, stream=stream):
             for i in range(n_dist):
                 sev[i].record(stream)
-                step(args.warmup + i % args.steps)
+                step(warmup + i % steps)
             sev[n_dist].record(stream)
         with torch.cuda.stream(stream):
             g_dist.replay()
@@ -479,7 +545,7 @@ def run_dwkv(args, world, rank, local):
         with torch.cuda.stream(stream):
             ev0.record(stream)
             for i in range(n_eager):
-                step(args.warmup + i % args.steps)
+                step(warmup + i % steps)
             ev1.record(stream)
         torch.cuda.synchronize(dev)
         cache.sync(stream)
@@ -487,41 +553,45 @@ def run_dwkv(args, world, rank, local):
                 "ms_p90": round(per[min(n_dist - 1, int(math.ceil(0.9 * n_dist)) - 1)], 5),
                 "ms_min": round(per[0], 5), "ms_max": round(per[-1], 5),
                 "eager_ms_per_step": round(ev0.elapsed_time(ev1) / n_eager, 5),
-                "timing": "graph of the steps with an event node between steps; eager: 32 launches a step "
-                          "from Python, no graph"}
+                "timing": f"graph of the steps with an event node between steps; eager: {wl.num_layers} launches a "
+                          "step from Python, no graph"}
 
-    # ---- CPU oracle baseline (rank 0, N = 1 only): the 8 kv-heads of layer 0 at full context
+    # ---- CPU oracle baseline (rank 0, N = 1 only): every kv-head of the first layers of
+    #      sequence 0 at its full context, one problem per host core, scaled to the step
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and comp_cpu:
-        threads = min(os.cpu_count() or 1, wl.num_kv_heads)
-        dt, n_items = cpu_oracle_sample(wl, comp_cpu[0], tiers_cpu[0], bases, Qs[0][args.warmup][0].cpu(), 0,
-                                        T - 1, threads)
-        step_s = dt * wl.num_layers * wl.num_kv_heads / n_items
-        dt1, n1 = cpu_oracle_sample(wl, comp_cpu[0], tiers_cpu[0], bases, Qs[0][args.warmup][0].cpu(), 0,
-                                    T - 1, 1, heads=1)
-        step1_s = dt1 * wl.num_layers * wl.num_kv_heads / n1
-        cpu = {"value": round(B / step_s, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"layer 0, {n_items} kv-heads x {T - 1} cached tokens (fp64 C oracle, {dt:.1f} s wall "
-                         f"on {threads} threads), scaled x{wl.num_layers} layers to one step",
+    if do_cpu and comp_cpu:
+        probs_in = [(bases, tiers_cpu[l], comp_cpu[l], Qs[l][warmup][0].cpu(), l, hh)
+                    for l in sorted(comp_cpu) for hh in range(wl.num_kv_heads)]
+        dt = cpu_oracle_sample(wl, probs_in, cores)
+        scale = (wl.num_layers * wl.num_kv_heads / len(probs_in)) * (sum(lengths) - B) / (lengths[0] - 1)
+        step_s = dt * scale
+        dt1 = cpu_oracle_sample(wl, probs_in[:1], 1)
+        step1_s = dt1 * wl.num_layers * wl.num_kv_heads * (sum(lengths) - B) / (lengths[0] - 1)
+        cpu = {"value": round(B / step_s, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"sequence 0, layers 0-{len(comp_cpu) - 1} x {wl.num_kv_heads} kv-heads = {len(probs_in)} "
+                         f"problems of {lengths[0] - 1} cached tokens (fp64 C oracle, OpenMP over the problems, "
+                         f"{dt:.1f} s wall on {cores} threads), scaled x{scale:.2f} to one step of all "
+                         f"{B} sequence(s) and {wl.num_layers} layers",
                "single_thread_value": round(B / step1_s, 6),
-               "single_thread_sample": f"layer 0, 1 kv-head x {T - 1} cached tokens on 1 thread ({dt1:.1f} s), "
-                                       f"scaled x{wl.num_kv_heads} heads x{wl.num_layers} layers",
-               "nproc": os.cpu_count(), "cpu_model": cpu_model()}
+               "single_thread_sample": f"one problem (layer 0, kv-head 0, {lengths[0] - 1} tokens) on 1 thread "
+                                       f"({dt1:.1f} s), scaled to the step",
+               "nproc": cores, "cpu_model": cpu_model()}
 
     value = aggregate_rate(world, B, ms_per_step)
     res = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16 storage, fp32 math",
         "data": "synthetic (seeded compressed cache; no model weights)",
-        "config": {"workload": args.workload, "layers": wl.num_layers, "groups": wl.num_groups,
+        "config": {"workload": name, "layers": wl.num_layers, "groups": wl.num_groups,
                    "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
-                   "batch_per_gpu": B, "context": T, "r_max": wl.r_max, "tiers": list(wl.tiers),
-                   "tier_probs": list(wl.tier_probs), "resid_channels": wl.resid_channels,
+                   "batch_per_gpu": B, "context": lengths[0] if B == 1 else lengths, "r_max": wl.r_max,
+                   "tiers": list(wl.tiers), "tier_probs": list(wl.tier_probs), "resid_channels": wl.resid_channels,
                    "resid_bits": wl.resid_bits, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (~2.6 GB of pages per step); no flush",
+                   "l2": f"inputs larger than L2 (~{comp_bytes_layer * wl.num_layers / 1e9:.1f} GB of pages per step); "
+                         "no flush",
                    "graph": "CUDA graph of K steps, replayed once"},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step * steps,
         "compressed_gb_per_step": round(comp_bytes_layer * wl.num_layers / 1e9, 4),
         "compressed_tb_s": round(comp_bytes_layer * wl.num_layers / (ms_per_step * 1e-3) / 1e12, 4),
         "dense_bf16_gb_per_step": round(dense_kv_bytes(wl.num_layers, wl.num_kv_heads, wl.head_dim, int(ctx_timed)) / 1e9, 4),
@@ -530,21 +600,34 @@ def run_dwkv(args, world, rank, local):
                      "traffic": traffic, "kernel": f"dwkv::decode_kernel<{wl.resid_bits},false>",
                      "alg_bytes_per_launch": int(alg_bytes), "launch_ms": round(launch_ms, 5),
                      "launch_ms_source": "timed region / launches (CUDA events on the launching stream)",
-                     "launch_ms_bracketed": round(dec_ms_mean, 5),
+                     "launch_ms_bracketed": None if dec_ms_mean is None else round(dec_ms_mean, 5),
                      "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
                      "frac_of_8tbs_spec": round(achieved / 8000.0, 4)},
         "probe": {"kernel": f"dwkv::decode_kernel<{wl.resid_bits},true>", "launch_ms": round(probe_launch_ms, 5),
                   "context": held_probe,
                   "achieved_gbs": round(probe_bytes / (probe_launch_ms * 1e-3) / 1e9, 1),
                   "frac": round(probe_bytes / (probe_launch_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                  "timing": f"graph of {wl.num_layers} probe launches, {args.profile_steps} replays after one warm-up"},
+                  "timing": f"graph of {wl.num_layers} probe launches, {probe_reps} replay(s) after one warm-up"},
         "step_distribution": dist,
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
     }
     cache.close()
+    del cache, Kn, Vn, Qs, Tn, out, err, g_main, g_probe
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
     return res
+
+
+def gpu_uuid(local: int):
+    """NVML-style UUID of cuda:local (for the clock sampler), or None."""
+    try:
+        import torch
+        u = str(torch.cuda.get_device_properties(local).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
 
 
 def pack_step_inputs(tensors):
@@ -624,7 +707,7 @@ def run_encode(args, world, rank, local):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, gpu_uuid(local)) as clk:
         clk.mark_start()
         with torch.cuda.stream(stream):
             for i in range(args.steps):
@@ -686,6 +769,27 @@ def run_encode(args, world, rank, local):
     dec_ms = d0.elapsed_time(d1)
     probe_ms = p0.elapsed_time(p1)
 
+    # ---- CPU oracle baseline (rank 0, N = 1 only): the oracle's encode of sequence 0's keys
+    #      and values of layer 0, kv-head 0 (2 N vectors), OpenMP over the vectors on all cores
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import numpy as np
+
+        import oracle
+        cores = os.cpu_count() or 1
+        ranks0 = np.asarray(wl.tiers, np.int32)[Tg[0][:N, 0].long().cpu().numpy()]
+        t0 = time.perf_counter()
+        for z, X in enumerate((K[0], V[0])):
+            oracle.encode_many(bases[z][0, 0], X[:N, 0].cpu(), ranks0, wl.resid_channels, wl.resid_bits,
+                               nthreads=cores)
+        dt = time.perf_counter() - t0
+        gbs = 2 * N * wl.head_dim * 2 / dt / 1e9
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"sequence 0, layer 0, kv-head 0: {2 * N} key and value vectors encoded by the fp32 C "
+                         f"oracle (OpenMP over the vectors, {dt:.2f} s wall on {cores} threads); GB/s of dense "
+                         "bf16 input, the rate the step's vectors would see",
+               "nproc": cores, "cpu_model": cpu_model()}
+
     value = aggregate_rate(world, dense / 1e9, ms_per_step)
     res = {
         "metric": "bulk encode: dense bf16 K/V GB/s compressed (a7)", "value": round(value, 2), "unit": "GB/s",
@@ -715,49 +819,70 @@ def run_encode(args, world, rank, local):
                   "achieved_gbs": round(dec_bytes / (probe_ms * 1e-3) / 1e9, 1),
                   "frac": round(dec_bytes / (probe_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
         "clocks": clocks,
+        "cpu_baseline": cpu,
     }
     cache.close()
+    del cache, K, V
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
     return res
 
 
 def run_reference(args, world, rank, local):
-    """The CPU oracle, as it stands, timed on a bounded sample of the same workload: per
-    step, the 8 kv-heads of one layer over a prefix of the context, scaled linearly to the
-    full context and to all layers."""
+    """The CPU oracle, as it stands, timed on the host cores over a bounded sample of the same
+    workload.  One bench step here is one sample: every kv-head of the first layers of
+    sequence 0 (one (layer, kv-head) problem per core at least) at the sequence's full
+    context, fp64, OpenMP over the problems on all cores.  ``value`` scales the sample's
+    time to a whole decode step of the workload (all sequences, all layers); ``ms_per_step``
+    is the sample's own measured time."""
     import synth
     wl = synth.workload(args.workload)
-    T = args.context or wl.context
-    bases = synth.make_bases(wl.scaled(num_layers=wl.layers_per_group))
-    tiers = synth.make_tiers(wl, 0, 0, T - 1)
-    comp = synth.make_compressed(wl, 0, 0, tiers)
-    q = synth.make_queries(wl, 0, batch=1)[0]
-    threads = os.cpu_count() or 1
-    # calibrate: seconds per cached token for the 8 heads, then size the per-step prefix
-    dt, n = cpu_oracle_sample(wl, comp, tiers, bases, q, 0, 2048, min(threads, wl.num_kv_heads))
-    per_tok = dt / 2048
-    budget = min(20.0, 150.0 / max(args.steps + args.warmup, 1))
-    t_s = int(max(512, min(T - 1, budget / max(per_tok, 1e-9))))
+    B = wl.batch
+    lengths = [args.context] * B if args.context else synth.make_context_lengths(wl)
+    cores = os.cpu_count() or 1
+    nl = oracle_layers_for(wl, cores)
+    bases = synth.make_bases(wl)
+    probs_in = []
+    tiers_g = {}
+    for layer in range(nl):
+        g = layer // wl.layers_per_group
+        if g not in tiers_g:
+            tiers_g[g] = synth.make_tiers(wl, 0, g, lengths[0] - 1)
+        comp = synth.make_compressed(wl, 0, layer, tiers_g[g])
+        q = synth.make_queries(wl, layer, batch=1)[0]
+        probs_in += [(bases, tiers_g[g], comp, q, layer, hh) for hh in range(wl.num_kv_heads)]
+    scale = (wl.num_layers * wl.num_kv_heads / len(probs_in)) * (sum(lengths) - B) / (lengths[0] - 1)
     for _ in range(args.warmup):
-        cpu_oracle_sample(wl, comp, tiers, bases, q, 0, t_s, min(threads, wl.num_kv_heads))
-    times = []
-    for _ in range(args.steps):
-        dt, n = cpu_oracle_sample(wl, comp, tiers, bases, q, 0, t_s, min(threads, wl.num_kv_heads))
-        times.append(dt * ((T - 1) / t_s) * wl.num_layers * wl.num_kv_heads / n)
-    ms = statistics.mean(times) * 1e3
-    value = 1.0 / (ms * 1e-3)
-    used = min(threads, wl.num_kv_heads)
-    sample = (f"per step: layer 0, {n} kv-heads over the first {t_s} of {T - 1} cached tokens (fp64 C oracle on "
-              f"{used} threads), scaled linearly to the full context and x{wl.num_layers} layers")
+        cpu_oracle_sample(wl, probs_in, cores)
+    times = [cpu_oracle_sample(wl, probs_in, cores) for _ in range(args.steps)]
+    sample_s = statistics.mean(times)
+    value = B / (sample_s * scale)
+    sample = (f"per step: sequence 0, layers 0-{nl - 1} x {wl.num_kv_heads} kv-heads = {len(probs_in)} problems of "
+              f"{lengths[0] - 1} cached tokens (fp64 C oracle, OpenMP over the problems on {cores} threads); value "
+              f"scales the step's time x{scale:.2f} to a whole decode step ({B} sequence(s), {wl.num_layers} layers)")
     return {
         "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded compressed cache)",
+        "warmup": args.warmup, "ms_per_step": round(sample_s * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded compressed cache)",
         "config": {"workload": args.workload, "layers": wl.num_layers, "kv_heads": wl.num_kv_heads,
-                   "context": T, "batch_per_gpu": 1},
+                   "context": lengths[0] if B == 1 else lengths, "batch_per_gpu": B},
         "impl": "reference",
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample},
+        "ms_per_full_step_scaled": round(sample_s * scale * 1e3, 1),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                         "nproc": cores, "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+EXTRA_WORKLOADS = ("llama8b_ragged_b8", "llama8b_131k_deep", "llama8b_encode_16k")
+
+
+def summary_of(res: dict) -> dict:
+    """The keys of a workload's line that the default run repeats for the extra workloads."""
+    keep = ("metric", "value", "unit", "ms_per_step", "steps", "warmup", "config", "gpu_launches", "roofline",
+            "compressed_gb_per_step", "compressed_tb_s", "probe", "e2e", "cpu_baseline", "clocks", "hbm",
+            "decode_step", "vectors_per_s")
+    return {k: res[k] for k in keep if k in res}
 
 
 def main():
@@ -773,6 +898,7 @@ def main():
     ap.add_argument("--profile-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tuning", default="", help="ctas_per_sm,waves,stages")
+    ap.add_argument("--headline-only", action="store_true", help="skip the other workloads of the default run")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 1)
     world, rank, local = dist_setup()
@@ -785,6 +911,20 @@ def main():
             res = run_encode(args, world, rank, local)
         else:
             res = run_dwkv(args, world, rank, local)
+            # the default single-GPU run also measures the other workloads, each with its own
+            # roofline, e2e and CPU baseline, in fewer steps (the headline stays the 64K line)
+            if world == 1 and args.workload == "llama8b_64k" and not args.headline_only and not args.layers:
+                extra = {}
+                for wname in EXTRA_WORKLOADS:
+                    if wname == "llama8b_encode_16k":
+                        sub = argparse.Namespace(**vars(args))
+                        sub.workload, sub.steps, sub.warmup = wname, 2, 1
+                        extra[wname] = summary_of(run_encode(sub, world, rank, local))
+                    else:
+                        extra[wname] = summary_of(run_dwkv(args, world, rank, local, workload=wname,
+                                                           steps=min(args.steps, 10), warmup=3, e2e_steps=2,
+                                                           light=True))
+                res["workloads"] = extra
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

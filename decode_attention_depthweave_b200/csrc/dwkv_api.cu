@@ -176,6 +176,12 @@ MetaLayout meta_layout(const Geom& G) {
     return M;
 }
 
+// Split-K records a decode (probe = false) or probe launch over n_seqs sequences can write:
+// at most kMaxSplits per (sequence, kv-head), each rec_floats_of(G, probe) floats.
+size_t ws_need(const Geom& G, int n_seqs, bool probe) {
+    return (size_t)std::max(n_seqs, 1) * G.Hkv * kMaxSplits * rec_floats_of(G, probe) * sizeof(float);
+}
+
 size_t worst_data_bytes(const Geom& G) {
     uint32_t big = 0;
     for (int k = 0; k < G.ntiers; ++k) big = std::max(big, G.page_units[k]);
@@ -369,8 +375,7 @@ size_t dwkv_arena_bytes(const dwkv_config* cfg) {
 
 size_t dwkv_workspace_bytes(const dwkv_config* cfg, int32_t n_seqs) {
     if (check_cfg(cfg) != DWKV_OK || n_seqs < 0) return 0;
-    const Geom G = make_geom(cfg);
-    return (size_t)std::max(n_seqs, 1) * G.Hkv * kMaxSplits * rec_floats_of(G, true) * sizeof(float);
+    return ws_need(make_geom(cfg), n_seqs, true);
 }
 
 dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes, const void* basis_k,
@@ -605,6 +610,44 @@ size_t fused_ring_need(const Geom& G) {
     return (size_t)2 * kD * (G.r_max + 2) * 2 + (size_t)2 * (kD + kMaxRank + 32) * 4;
 }
 
+// Splits (CTAs per kv-head) of each sequence of a decode launch.  The launch aims at
+// SMs x waves CTAs in all, i.e. S = SMs x waves / Hkv splits per kv-head, apportioned to the
+// sequences in proportion to the tokens they hold (a sequence's bytes are its tokens times
+// the mean bytes of its tiers, which the host does not know; the tiers are i.i.d. across
+// sequences, so tokens stand in for bytes) by largest remainders.  Every sequence gets at
+// least one split (an empty one writes zeros) and at most min(kMaxSplits, its pages).
+void split_counts(dwkv_handle h, int layer, int n_seqs, const int32_t* seq_ids, long long tot, int* sp) {
+    const Geom& G = h->geom;
+    const long long S = std::max(1ll, (long long)h->num_sms * h->dec_waves / G.Hkv);
+    std::vector<long long> len(n_seqs), cap(n_seqs), rem(n_seqs);
+    long long used = 0;
+    for (int i = 0; i < n_seqs; ++i) {
+        len[i] = h->len[(size_t)seq_ids[i] * G.L + layer];
+        cap[i] = std::max(1ll, std::min((long long)kMaxSplits, (len[i] + kPage - 1) / kPage));
+        const long long q = tot > 0 ? S * len[i] / tot : 0;      // ideal share S len / tot, floored
+        rem[i] = tot > 0 ? S * len[i] % tot : 0;
+        sp[i] = (int)std::max(1ll, std::min(q, cap[i]));
+        used += sp[i];
+    }
+    // the splits left over go to the largest remainders first (ties to the earlier sequence),
+    // then, while some remain (caps cut a share), to the sequence with most tokens per split
+    std::vector<int> order(n_seqs);
+    for (int i = 0; i < n_seqs; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return rem[a] > rem[b]; });
+    for (int i : order) {
+        if (used >= S) break;
+        if (sp[i] < cap[i]) { ++sp[i]; ++used; }
+    }
+    while (used < S) {
+        int best = -1;
+        for (int i = 0; i < n_seqs; ++i)
+            if (sp[i] < cap[i] && (best < 0 || len[i] * sp[best] > len[best] * sp[i])) best = i;
+        if (best < 0) break;
+        ++sp[best];
+        ++used;
+    }
+}
+
 static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const void* q,
                               float* out, float* err, float* out_full, void* workspace, size_t ws_bytes,
                               void* stream, bool probe, const FusedAppend* fa = nullptr) {
@@ -619,7 +662,7 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     if (probe && !err) return fail(DWKV_ERR_INVALID_ARG, "err is NULL");
     if (!workspace) return fail(DWKV_ERR_INVALID_ARG, "workspace is NULL");
     if (reinterpret_cast<uintptr_t>(workspace) % 16) return fail(DWKV_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
-    const size_t need = dwkv_workspace_bytes(&h->cfg, n_seqs);
+    const size_t need = ws_need(G, n_seqs, probe);
     if (ws_bytes < need) return fail(DWKV_ERR_CAPACITY, "workspace of %zu bytes is below the %zu needed", ws_bytes, need);
     const int g = layer / G.LPG;
     long long tot = 0;
@@ -640,17 +683,13 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     size_t smem = 0;
     const uint32_t ring = decode_ring_for(h, probe, &smem);
     if (ring == 0) return fail(DWKV_ERR_UNSUPPORTED, "decode pipeline does not fit in shared memory");
-    const long long target = (long long)h->num_sms * h->dec_waves;
+    std::vector<int> sp(n_seqs);
+    split_counts(h, layer, n_seqs, seq_ids, tot, sp.data());
     int total = 0;
     for (int i = 0; i < n_seqs; ++i) {
-        const int s = seq_ids[i];
-        const long long len = h->len[(size_t)s * G.L + layer];
-        long long sp = tot > 0 ? (target * len) / (tot * G.Hkv) : 1;
-        const long long pages = std::max(1ll, (len + kPage - 1) / kPage);
-        sp = std::max(1ll, std::min({sp, (long long)kMaxSplits, pages}));
-        C.seq[i] = s;
+        C.seq[i] = seq_ids[i];
         C.split_begin[i] = total;
-        total += (int)sp;
+        total += sp[i];
     }
     C.split_begin[n_seqs] = total;
     C.total_splits = total;
@@ -720,7 +759,7 @@ dwkv_status dwkv_append_decode_attention(dwkv_handle h, int32_t layer, int32_t n
     if (!k_new || !v_new) return fail(DWKV_ERR_INVALID_ARG, "k_new and v_new must be non-NULL");
     if (!q || !out || !workspace) return fail(DWKV_ERR_INVALID_ARG, "q, out and workspace must be non-NULL");
     if (reinterpret_cast<uintptr_t>(workspace) % 16) return fail(DWKV_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
-    const size_t need = dwkv_workspace_bytes(&h->cfg, n_seqs);
+    const size_t need = ws_need(h->geom, n_seqs, false);
     if (ws_bytes < need) return fail(DWKV_ERR_CAPACITY, "workspace of %zu bytes is below the %zu needed", ws_bytes, need);
     std::vector<int32_t> ones((size_t)n_seqs, 1);
     AppendCall A;
@@ -876,7 +915,7 @@ extern "C" dwkv_status dwkv_decode_attention_noalloc(dwkv_handle h, int32_t laye
     if ((st = check_handle(h)) != DWKV_OK) return st;
     if (n_seqs < 0 || n_seqs > kMaxSeqs)
         return fail(DWKV_ERR_INVALID_ARG, "n_seqs %d out of [0, %d]", n_seqs, kMaxSeqs);
-    const size_t need = dwkv_workspace_bytes(&h->cfg, n_seqs);
+    const size_t need = ws_need(h->geom, n_seqs, false);
     if (need > kNoAllocScratchBytes)
         return fail(DWKV_ERR_CAPACITY,
                     "dwkv_decode_attention_noalloc: %d sequences need %zu bytes of scratch but the built-in "

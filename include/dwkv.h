@@ -126,7 +126,9 @@ size_t dwkv_metadata_bytes(const dwkv_config* cfg);
  * smaller and running out of it is a device-side DWKV_DEV_POOL_EXHAUSTED error. */
 size_t dwkv_arena_bytes(const dwkv_config* cfg);
 
-/* Workspace bytes that decode / probe need for a call over n_seqs sequences. */
+/* Workspace bytes that decode and probe need for a call over n_seqs sequences (the probe's
+ * split-K records are twice as large; decode alone accepts a workspace of half this size:
+ * n_seqs * Hkv * 64 records of 8 + 4 * head_dim floats). */
 size_t dwkv_workspace_bytes(const dwkv_config* cfg, int32_t n_seqs);
 
 /* Creates a cache inside `arena` (device, caller-owned, 256-byte aligned, at least
@@ -180,7 +182,8 @@ dwkv_status dwkv_append_compressed(dwkv_handle h, int32_t layer, int32_t n_seqs,
  *   seq_ids   : host int32 [n_seqs], distinct
  *   q         : device bf16 [n_seqs][Hq][head_dim]
  *   out       : device fp32 [n_seqs][Hq][head_dim]; an empty sequence gives zeros
- *   workspace : device, >= dwkv_workspace_bytes(cfg, n_seqs) bytes, 16-byte aligned
+ *   workspace : device, 16-byte aligned, >= dwkv_workspace_bytes(cfg, n_seqs) bytes (half of
+ *               that suffices for decode, see dwkv_workspace_bytes)
  * Every layer of a group must hold the same positions when one of them is decoded
  * (append each layer of the group before decoding it). */
 dwkv_status dwkv_decode_attention(dwkv_handle h, int32_t layer, int32_t n_seqs,
@@ -247,8 +250,9 @@ dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t w
  * when they decode (engine plugin hooks, serving loops whose memory pool owns all of HBM) and
  * have no workspace to lend.  Arguments as dwkv_decode_attention without the workspace.
  *  - Calls nothing that allocates (no cudaMalloc / cudaFree).
- *  - Returns DWKV_ERR_CAPACITY when dwkv_workspace_bytes(cfg, n_seqs) exceeds 8 MiB
- *    (for 8 kv-heads and head_dim 128: up to 3 sequences per call).
+ *  - Returns DWKV_ERR_CAPACITY when the call's split-K records, n_seqs * Hkv * 64 records of
+ *    (8 + 4 * head_dim) floats, exceed 8 MiB (for 8 kv-heads and head_dim 128: up to 7
+ *    sequences per call).
  *  - The first call on a device resolves the scratch array's device address (one
  *    cudaGetSymbolAddress); make that first call before any stream capture.  The handle's
  *    device must be current.

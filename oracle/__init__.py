@@ -162,6 +162,24 @@ class HeadProblem:
                 _p(self.sk), _p(self.cv), _p(self.iv), _p(self.qv), _p(self.sv), _p(self.q)]
 
 
+def head_problem(wl, bases, tier_idx, comp, q, layer, head) -> HeadProblem:
+    """The decode problem of one (layer, kv-head) of one sequence, sliced from token-ordered
+    arrays: ``wl`` a workload (tiers, layers_per_group, gqa), ``bases`` the (K, V) bases
+    bf16 [G][Hkv][d][r_max], ``tier_idx`` uint8 [T][Hkv] (index into ``wl.tiers``), ``comp``
+    the stored arrays (coeff [T][Hkv][2][r_max], idx / codes [T][Hkv][2][s], scales
+    [T][Hkv][2]; K at [..][0], V at [..][1]) and ``q`` bf16 [Hq][d], every query head of the
+    sequence."""
+    g = layer // wl.layers_per_group
+    gq = wl.gqa
+    ti = _arr(tier_idx, np.int64)[:, head]
+    ranks = np.asarray(wl.tiers, np.int32)[ti]
+    sl = lambda key, z: comp[key][:, head, z]   # noqa: E731
+    return HeadProblem(bases[0][g, head], bases[1][g, head], ranks,
+                       sl("coeff", 0), sl("idx", 0), sl("codes", 0), comp["scales"][:, head, 0],
+                       sl("coeff", 1), sl("idx", 1), sl("codes", 1), comp["scales"][:, head, 1],
+                       _bits16(q)[head * gq:(head + 1) * gq])
+
+
 def decode_head(prob: HeadProblem, tau=None, with_residual=True, want_p=False):
     """fp64 attention output [gq][d] (and softmax weights [gq][T] when ``want_p``)."""
     tau = default_tau(prob.d) if tau is None else tau

@@ -20,20 +20,8 @@ def bf16_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().to(torch.float64).numpy()
 
 
-def head_problem(wl, bases, tier_idx, comp, q, layer, head) -> oracle.HeadProblem:
-    """Oracle problem for one (layer, kv-head) from token-ordered synthetic arrays.
-
-    ``tier_idx`` uint8 [T][Hkv]; ``comp`` the dict of ``synth.make_compressed``; ``q`` bf16
-    [Hq][d] (all query heads of the sequence)."""
-    g = layer // wl.layers_per_group
-    gq = wl.gqa
-    ranks = synth.ranks_of(wl, tier_idx.cpu())[:, head]
-    c = {k: v.cpu() for k, v in comp.items()}
-    return oracle.HeadProblem(
-        bases[0][g, head], bases[1][g, head], ranks,
-        c["coeff"][:, head, 0], c["idx"][:, head, 0], c["codes"][:, head, 0], c["scales"][:, head, 0],
-        c["coeff"][:, head, 1], c["idx"][:, head, 1], c["codes"][:, head, 1], c["scales"][:, head, 1],
-        q.cpu()[head * gq:(head + 1) * gq])
+# One (layer, kv-head) decode problem of the oracle, sliced from token-ordered arrays.
+head_problem = oracle.head_problem
 
 
 def np_reconstruct(basis, ranks, coeff, idx, codes, scales, with_residual=True) -> np.ndarray:

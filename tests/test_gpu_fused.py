@@ -144,30 +144,3 @@ def test_fused_steps_residual_counts(s, bits):
     fused, _ = _steps(wl, [T0], steps, fused=True)
     plain, _ = _steps(wl, [T0], steps, fused=False, check=False)
     _assert_same_bytes(fused, plain, wl, [T0 + steps])
-
-
-@pytest.mark.slow
-def test_llama8b_64k_full_context_fused_step_sampled_heads():
-    """The bench's launch configuration: one sequence, 8 kv-heads, 64K context, one fused
-    append + decode per layer of a two-layer group (the first layer places the token, the
-    second finds it placed); sampled heads of both layers against the oracle, which encodes
-    the appended token itself."""
-    wl = synth.workload("llama8b_64k").scaled(num_layers=2)
-    T = wl.context
-    bases = synth.make_bases(wl)
-    cache = dw.Cache(cfg_for(wl, max_context=T + 64), bases[0], bases[1])
-    data = import_workload(cache, wl, [T - 1], gen_device="cuda")
-    tn = synth.make_tiers(wl, 0, 0, 1, device="cuda", start=T - 1)
-    for layer in range(2):
-        kn, vn = synth.make_dense_vectors(wl, 0, layer, 1, bases, device="cuda", start=T - 1)
-        q = synth.make_queries(wl, layer, batch=1, device="cuda", temperature=8.0)
-        out = cache.append_decode(layer, [0], kn, vn, tn if layer == 0 else None, q)
-        cache.sync()
-        out = out.cpu().numpy()
-        tiers, comp = data[(0, layer)]
-        new = oracle_encode_rows(wl, bases, layer, kn, vn, tn)
-        tt = torch.cat([tiers.cpu(), tn.cpu()])
-        full = cat_comp(comp, new)
-        for h in (0, 5) if layer else (3,):
-            ref = oracle.decode_head(head_problem(wl, bases, tt, full, q[0].cpu(), layer, h))
-            check_close(out[0, h * 4:(h + 1) * 4], ref, what=f"64K fused layer {layer} head {h}")
