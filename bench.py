@@ -322,6 +322,7 @@ def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e
     if args.tuning:
         c, w_, s_ = (int(x) for x in args.tuning.split(","))
         cache.set_decode_tuning(c, w_, s_)
+    cache.set_decode_overlap(not args.no_overlap)
     h = cache.h
     lpg = wl.layers_per_group
 
@@ -590,7 +591,8 @@ def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e
                    "resid_bits": wl.resid_bits, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2 (~{comp_bytes_layer * wl.num_layers / 1e9:.1f} GB of pages per step); "
                          "no flush",
-                   "graph": "CUDA graph of K steps, replayed once"},
+                   "graph": "CUDA graph of K steps, replayed once",
+                   "launch_overlap": not args.no_overlap},
         "gpu_launches": launches_per_step * steps,
         "compressed_gb_per_step": round(comp_bytes_layer * wl.num_layers / 1e9, 4),
         "compressed_tb_s": round(comp_bytes_layer * wl.num_layers / (ms_per_step * 1e-3) / 1e12, 4),
@@ -899,6 +901,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tuning", default="", help="ctas_per_sm,waves,stages")
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads of the default run")
+    ap.add_argument("--no-overlap", action="store_true", help="serialise the decode launches (measurement)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 1)
     world, rank, local = dist_setup()

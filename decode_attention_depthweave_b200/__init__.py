@@ -22,7 +22,8 @@ __all__ = [
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage",
     "dwkv_sync_status", "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
-    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "Cache", "EXPORTED_SYMBOLS",
+    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
+    "Cache", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -38,7 +39,7 @@ EXPORTED_SYMBOLS = (
     "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage", "dwkv_sync_status",
     "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
-    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait",
+    "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
 )
 
 
@@ -102,6 +103,7 @@ def lib():
             "dwkv_quantize_work_bytes": ([i32, i32, i32], sz),
             "dwkv_quantize_residuals": ([i32, i32, i32, vp, vp, vp, vp, vp, sz, vp], C.c_int),
             "dwkv_check_bounded_wait": ([vp, C.c_uint32, vp], C.c_int),
+            "dwkv_set_decode_overlap": ([vp, i32], C.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -281,6 +283,10 @@ def dwkv_set_decode_tuning(h, ctas_per_sm=1, waves=1, stages=0):
     _check(lib().dwkv_set_decode_tuning(h, ctas_per_sm, waves, stages))
 
 
+def dwkv_set_decode_overlap(h, enable):
+    _check(lib().dwkv_set_decode_overlap(h, int(enable)))
+
+
 # ------------------------------------------------------------------------------ plumbing
 class Cache:
     """Owns the torch allocations around one handle (arena and workspace) and exposes the
@@ -366,3 +372,6 @@ class Cache:
 
     def set_decode_tuning(self, ctas_per_sm=1, waves=1, stages=0):
         dwkv_set_decode_tuning(self.h, ctas_per_sm, waves, stages)
+
+    def set_decode_overlap(self, enable: bool):
+        dwkv_set_decode_overlap(self.h, 1 if enable else 0)

@@ -206,6 +206,7 @@ struct dwkv_ctx {
     int dec_ctas_per_sm = 1, dec_waves = 1, dec_stages_req = 0;
     int dec_tok_weight = 1024;      // split balance: byte-equivalent cost of one token
     int dec_owner_share = 160;      // fused append: the encoding CTA's share of a split, of 256
+    int dec_overlap = 1;            // launch decodes with programmatic stream serialisation
 };
 
 namespace {
@@ -486,6 +487,14 @@ dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t w
     return DWKV_OK;
 }
 
+dwkv_status dwkv_set_decode_overlap(dwkv_handle h, int32_t enable) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if (enable != 0 && enable != 1) return fail(DWKV_ERR_INVALID_ARG, "enable must be 0 or 1 (got %d)", enable);
+    h->dec_overlap = enable;
+    return DWKV_OK;
+}
+
 dwkv_status dwkv_seq_length(dwkv_handle h, int32_t seq, int32_t layer, int32_t* len) {
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
@@ -648,6 +657,25 @@ void split_counts(dwkv_handle h, int layer, int n_seqs, const int32_t* seq_ids, 
     }
 }
 
+// One decode-kernel launch.  With `overlap` it is launched with programmatic stream
+// serialisation: its CTAs may start on SMs the previous kernel of the stream has left, set up
+// their pipeline and stream their first pages before waiting for that kernel (the kernel
+// waits before it reads q, the new token or anything a decode writes).
+cudaError_t launch_decode(void (*k)(const Geom, const State, const DecodeCall), dim3 grid, size_t smem,
+                          cudaStream_t s, bool overlap, const Geom& G, const State& St, const DecodeCall& C) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = dim3(kDecodeThreads);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = overlap ? 1 : 0;
+    return cudaLaunchKernelEx(&lc, k, G, St, C);
+}
+
 static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const void* q,
                               float* out, float* err, float* out_full, void* workspace, size_t ws_bytes,
                               void* stream, bool probe, const FusedAppend* fa = nullptr) {
@@ -689,6 +717,7 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     for (int i = 0; i < n_seqs; ++i) {
         C.seq[i] = seq_ids[i];
         C.split_begin[i] = total;
+        C.expect[i] = h->len[(size_t)seq_ids[i] * G.L + layer];   // positions the group has placed
         total += sp[i];
     }
     C.split_begin[n_seqs] = total;
@@ -706,6 +735,8 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
         for (int i = 0; i < n_seqs; ++i) {
             C.pos[i] = fa->call->pos0[i];
             C.place[i] = fa->call->na[i] > 0 ? 1 : 0;
+            // the placing launch counts its token only at its end; a later layer finds it counted
+            C.expect[i] = C.place[i] ? C.pos[i] : C.pos[i] + 1;
         }
     }
     C.q = static_cast<const __nv_bfloat16*>(q);
@@ -716,7 +747,8 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(total, G.Hkv);
     const bool big = G.r_max > 64;
-#define DWKV_LAUNCH(B, P, R, SS) decode_kernel<B, P, R, SS><<<grid, kDecodeThreads, smem, s>>>(G, h->st, C)
+    cudaError_t lerr = cudaSuccess;
+#define DWKV_LAUNCH(B, P, R, SS) lerr = launch_decode(decode_kernel<B, P, R, SS>, grid, smem, s, h->dec_overlap != 0, G, h->st, C)
 #define DWKV_LAUNCH_S(B, P, R)                                  \
     do {                                                        \
         switch (G.s) {                                          \
@@ -738,6 +770,7 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
 #undef DWKV_LAUNCH_R
 #undef DWKV_LAUNCH_S
 #undef DWKV_LAUNCH
+    if (lerr != cudaSuccess) return cuda_fail(lerr, probe ? "probe kernel launch" : "decode kernel launch");
     DWKV_CUDA(cudaGetLastError(), probe ? "probe kernel launch" : "decode kernel launch");
     return DWKV_OK;
 }

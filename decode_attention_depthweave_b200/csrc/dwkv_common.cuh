@@ -89,6 +89,10 @@ struct DecodeCall {
     const uint8_t* tier_idx;         // [n][Hkv] tier of the new token (read where it is placed)
     int pos[kMaxSeqs];               // the new token's position (fused)
     uint8_t place[kMaxSeqs];         // 1: this layer places it (its group's first to append it)
+    // Sum of the tier counts of each (sequence, kv-head) once every earlier kernel of the stream
+    // has completed.  A CTA that reads exactly this sum before waiting on the previous kernel
+    // (programmatic dependent launch) knows the counts are final; otherwise it waits first.
+    int expect[kMaxSeqs];
     int seq[kMaxSeqs];
     int split_begin[kMaxSeqs + 1];
     const __nv_bfloat16* q;  // [n][Hq][d]
@@ -254,6 +258,28 @@ __device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void* src, uin
 
 __device__ __forceinline__ void named_barrier(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialisation
+// may start while the previous kernel of its stream still runs; grid_dep_wait() returns once
+// that kernel has completed and its memory operations are visible (at once when there is no
+// such kernel).  grid_dep_launch() lets the next such kernel start once every CTA of this one
+// has issued it or exited.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_add_u32(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Orders this thread's earlier generic-proxy view of global memory before its later bulk
+// (async-proxy) copies.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -112,6 +112,33 @@ __device__ __forceinline__ uint32_t code_bytes(uint32_t cw) {
 }
 constexpr float kCodeUnit4 = 1.0f / 16.0f;              // value of one int4 tile unit
 
+// A row of NB bytes (NB a multiple of 4, the address aligned to the widest access used) as
+// 32-bit words, in as few shared-memory accesses as the size allows.
+template <int NB>
+__device__ __forceinline__ void ld_row(const uint8_t* p, uint32_t (&w)[NB / 4 > 0 ? NB / 4 : 1]) {
+    if constexpr (NB % 16 == 0) {
+#pragma unroll
+        for (int i = 0; i < NB / 16; ++i) {
+            const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+    } else if constexpr (NB % 8 == 0) {
+#pragma unroll
+        for (int i = 0; i < NB / 8; ++i) {
+            const uint2 v = reinterpret_cast<const uint2*>(p)[i];
+            w[2 * i] = v.x; w[2 * i + 1] = v.y;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < NB / 4; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+    }
+}
+
+// Score buffer of a half page: the hi and lo column halves as two [32 tokens][4 heads] fp32
+// blocks, the second 16 floats further on so that the stores of both halves from one MMA
+// fragment fall in distinct banks.
+constexpr int kSLo = 32 * 4 + 16;
+
 template <int RMAX, bool PROBE>
 struct WarpAcc {
     float c[RMAX / 16][4];                 // coefficient-space values, D layout (row j, col n)
@@ -172,12 +199,14 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 mma_bf16(d[mt], a, qb[ks]);
             }
         }
-        // S[token][8]: columns 0-3 the hi parts of heads 0-3, 4-7 the lo parts (summed per token
-        // below); S spans the P buffer too, which is written only after every lane has read S
+        // S: MMA columns 0-3 (the hi parts of heads 0-3) at [token][head], columns 4-7 (the lo
+        // parts) kSLo floats on (summed per token below); S spans the P buffer and the start of
+        // the W buffer too, both written only after every lane has read S
+        float* sp = Ssm + (c >> 1) * kSLo + 2 * (c & 1);
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
-            *reinterpret_cast<float2*>(Ssm + (16 * mt + g) * 8 + 2 * c) = make_float2(d[mt][0], d[mt][1]);
-            *reinterpret_cast<float2*>(Ssm + (16 * mt + g + 8) * 8 + 2 * c) = make_float2(d[mt][2], d[mt][3]);
+            *reinterpret_cast<float2*>(sp + (16 * mt + g) * 4) = make_float2(d[mt][0], d[mt][1]);
+            *reinterpret_cast<float2*>(sp + (16 * mt + g + 8) * 4) = make_float2(d[mt][2], d[mt][3]);
         }
     }
     __syncwarp();
@@ -191,25 +220,31 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
         for (int h = 0; h < kGQ; ++h) { sc[h] = -INFINITY; sc2[h] = -INFINITY; }
         float4 sv;
         {
-            const float4 s0 = *reinterpret_cast<const float4*>(Ssm + lane * 8);
-            const float4 s1 = *reinterpret_cast<const float4*>(Ssm + lane * 8 + 4);
+            const float4 s0 = *reinterpret_cast<const float4*>(Ssm + lane * 4);
+            const float4 s1 = *reinterpret_cast<const float4*>(Ssm + kSLo + lane * 4);
             sv = make_float4(s0.x + s1.x, s0.y + s1.y, s0.z + s1.z, s0.w + s1.w);
         }
         __syncwarp();                                   // S is dead from here (P overwrites it)
         if (live) {
             float ra[kGQ] = {0.f, 0.f, 0.f, 0.f};
+            // the token's channel indices and codes, each row in one or two vector loads
+            constexpr int kCB = S * BITS / 8;
+            uint32_t ixw[S / 4 > 0 ? S / 4 : 1], cw[kCB / 4 > 0 ? kCB / 4 : 1];
+            if (S) {
+                ld_row<S>(K + kOffIdx + t * S, ixw);
+                ld_row<kCB>(K + kOffCodes + t * kCB, cw);
+            }
 #pragma unroll
             for (int ch = 0; ch < S; ch += 8) {
-                const uint2 ix = *reinterpret_cast<const uint2*>(K + kOffIdx + t * S + ch);
+                const uint2 ix = make_uint2(ixw[ch / 4], ixw[ch / 4 + 1]);
                 // codes as biased bytes (code + 2^(b-1)), each turned into a float by placing it in
                 // the mantissa of 2^23 and subtracting 2^23 + 2^(b-1)
                 uint32_t cb0, cb1;
                 if (BITS == 8) {
-                    const uint2 cc = *reinterpret_cast<const uint2*>(K + kOffCodes + t * S + ch);
-                    cb0 = cc.x ^ 0x80808080u;
-                    cb1 = cc.y ^ 0x80808080u;
+                    cb0 = cw[ch / 4] ^ 0x80808080u;
+                    cb1 = cw[ch / 4 + 1] ^ 0x80808080u;
                 } else {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(K + kOffCodes + t * (S / 2) + ch / 2) ^ 0x88888888u;
+                    const uint32_t w = cw[ch / 8] ^ 0x88888888u;
                     cb0 = w & 0x0F0F0F0Fu;                      // codes 0, 2, 4, 6
                     cb1 = (w >> 4) & 0x0F0F0F0Fu;               // codes 1, 3, 5, 7
                 }
@@ -346,11 +381,14 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
     if (S) {
         if (lane < nv) {                                // scatter this token's codes (lane = token)
             const int tok = tb + lane;
+            constexpr int kCB = S * BITS / 8;
+            uint32_t ixw[S / 4 > 0 ? S / 4 : 1], cw[kCB / 4 > 0 ? kCB / 4 : 1];
+            ld_row<S>(V + kOffIdx + tok * S, ixw);
+            ld_row<kCB>(V + kOffCodes + tok * kCB, cw);
 #pragma unroll
             for (int e = 0; e < S; e += 4) {
-                const uint32_t ix = *reinterpret_cast<const uint32_t*>(V + kOffIdx + tok * S + e);
-                const uint32_t cbw = code_bytes<BITS>(BITS == 8 ? *reinterpret_cast<const uint32_t*>(V + kOffCodes + tok * S + e)
-                                                                : *reinterpret_cast<const uint16_t*>(V + kOffCodes + tok * (S / 2) + e / 2));
+                const uint32_t ix = ixw[e / 4];
+                const uint32_t cbw = code_bytes<BITS>(BITS == 8 ? cw[e / 4] : (cw[e / 8] >> (16 * ((e / 4) & 1))) & 0xffffu);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const uint32_t ch = __byte_perm(ix, 0u, 0x4440 + q);
@@ -607,7 +645,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     const size_t basis_off = ((size_t)C.g * G.Hkv + h) * kD * G.r_max;
     TokDest* tokd = reinterpret_cast<TokDest*>(smem + L.tok);
     const bool owner = !PROBE && C.fused && split == 0;
-    if (owner) owner_append<BITS>(G, St, C, ci, seq, h, smem + L.ring, tokd);
+    if (owner) {
+        // the new token's keys, values and tier may come from the previous kernel
+        grid_dep_wait();
+        owner_append<BITS>(G, St, C, ci, seq, h, smem + L.ring, tokd);
+    }
 
     uint32_t cv[kMaxTiers];                 // tier counts (producer lane 0)
     uint32_t bvf[RMAX / 16][4];             // B_V mma fragments (consumer warps 0-7, epilogue)
@@ -625,9 +667,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         const uint32_t bytes = (uint32_t)kD * G.r_max * 2;
         mbar_arrive_expect_tx(basis_bar, bytes);
         bulk_g2s(smem_addr(smem + L.rd), St.basis_k + basis_off, bytes, basis_bar);
+        // Until this CTA waits on the previous kernel (programmatic dependent launch), that
+        // kernel may still be running: the counts are final only if they sum to what the host
+        // expects once every earlier kernel has completed (the one count a fused decode adds
+        // at its end is the only change in flight).  Acquired together with the writes that
+        // precede that addition, so the slot map and pages read below are complete; otherwise
+        // wait, then read them again.
         const uint32_t* cnt = St.counts + cnt_index(G, seq, C.g, h);
+        uint32_t sum = 0;
 #pragma unroll
-        for (int k = 0; k < kMaxTiers; ++k) cv[k] = k < G.ntiers ? __ldcg(cnt + k) : 0u;
+        for (int k = 0; k < kMaxTiers; ++k) {
+            cv[k] = k < G.ntiers ? ld_acquire_u32(cnt + k) : 0u;
+            sum += cv[k];
+        }
+        if (sum != (uint32_t)C.expect[ci]) {
+            grid_dep_wait();
+#pragma unroll
+            for (int k = 0; k < kMaxTiers; ++k) cv[k] = k < G.ntiers ? ld_acquire_u32(cnt + k) : 0u;
+        }
+        fence_proxy_async_global();            // page bytes written before them, read by bulk copies
         // fused append: the pages are attended without the new token.  Where it was placed by
         // an earlier layer of the group the counts include it (it is the last slot of its tier);
         // where this launch places it they do not yet (the last CTA adds it).
@@ -766,6 +824,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             for (int x = tid; x < lines; x += kConsumerWarps * 32)
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(St.basis_v + basis_off) + 128 * x));
         }
+        // q may come from the previous kernel, and so may everything this CTA writes from here
+        // on (records, tickets, outputs); the next decode may start once every CTA is past here
+        grid_dep_wait();
+        grid_dep_launch();
         if (tid < kD) {
             const __nv_bfloat16* q = C.q + ((size_t)ci * G.Hq + (size_t)h * kGQ) * kD + tid;
             const __nv_bfloat16 q0 = q[0], q1 = q[kD], q2 = q[2 * kD], q3 = q[3 * kD];
@@ -1179,7 +1241,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         if (C.fused && C.place[ci]) {
             // every CTA has read the counts: add the position placed by the first CTA
             const uint32_t k = C.tier_idx[(size_t)ci * G.Hkv + h];
-            if (k < (uint32_t)G.ntiers) St.counts[cnt_index(G, seq, C.g, h) + k] += 1u;
+            if (k < (uint32_t)G.ntiers) red_release_add_u32(St.counts + cnt_index(G, seq, C.g, h) + k, 1u);
         }
     }
 }

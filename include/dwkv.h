@@ -243,6 +243,15 @@ dwkv_status dwkv_sync_status(dwkv_handle h, void* stream);
 dwkv_status dwkv_set_decode_tuning(dwkv_handle h, int32_t ctas_per_sm, int32_t waves,
                                    int32_t stages);
 
+/* Launch overlap of decode and probe (enable 1, the default, or 0).  With it, each launch
+ * may start while the previous kernel of its stream still runs: its CTAs take the SMs that
+ * kernel leaves, set up and start streaming their pages, and wait for that kernel to
+ * complete before they read q, the new token or the tier indices, or write anything.  The
+ * cache state they read early is read only once its tier counts show that no earlier
+ * decode's placement is still in flight.  Results are the same either way; 0 serialises
+ * the launches (for measurement).  DWKV_ERR_INVALID_ARG for other values. */
+dwkv_status dwkv_set_decode_overlap(dwkv_handle h, int32_t enable);
+
 /* Decode attention without any caller-provided or library-allocated memory: the same
  * operation as dwkv_decode_attention, but its split-K scratch is a fixed 8 MiB array built
  * into the library (held by every GPU that loads the library until the process exits).
