@@ -695,7 +695,7 @@ def run_encode(args, world, rank, local):
 
     def encode_step():
         for layer in range(wl.num_layers):
-            dw.dwkv_append(h, layer, seqs, [N] * B, K[layer], V[layer], Tg[layer // lpg], stream)
+            dw.dwkv_append(h, layer, seqs, [N] * B, K[layer], V[layer], Tg[layer // lpg], stream=stream)
 
     def reset():
         for b in seqs:

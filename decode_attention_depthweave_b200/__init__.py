@@ -23,7 +23,9 @@ __all__ = [
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage",
     "dwkv_sync_status", "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
     "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
-    "Cache", "EXPORTED_SYMBOLS",
+    "dwkv_retier", "dwkv_tier_policy", "dwkv_tier_controller_create", "dwkv_tier_controller_destroy",
+    "dwkv_tier_controller_due", "dwkv_tier_controller_threshold", "dwkv_tier_controller_observe",
+    "dwkv_tier_controller_route", "Cache", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,6 +42,8 @@ EXPORTED_SYMBOLS = (
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage", "dwkv_sync_status",
     "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
     "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
+    "dwkv_retier", "dwkv_tier_controller_create", "dwkv_tier_controller_destroy", "dwkv_tier_controller_due",
+    "dwkv_tier_controller_threshold", "dwkv_tier_controller_observe", "dwkv_tier_controller_route",
 )
 
 
@@ -57,6 +61,12 @@ class dwkv_config(C.Structure):
         ("resid_bits", C.c_int32), ("max_batch", C.c_int32), ("max_context", C.c_int32),
         ("softmax_scale", C.c_float),
     ]
+
+
+class dwkv_tier_policy(C.Structure):
+    _fields_ = [("tol", C.c_float), ("tau_init", C.c_float), ("tau_min", C.c_float), ("tau_max", C.c_float),
+                ("tau_step_down", C.c_float), ("tau_step_up", C.c_float), ("quiet_intervals", C.c_int32),
+                ("probe_every", C.c_int32)]
 
 
 class dwkv_pool_stats(C.Structure):
@@ -90,7 +100,7 @@ def lib():
             "dwkv_destroy": ([vp], C.c_int),
             "dwkv_reset_sequence": ([vp, i32, vp], C.c_int),
             "dwkv_seq_length": ([vp, i32, i32, C.POINTER(i32)], C.c_int),
-            "dwkv_append": ([vp, i32, i32, vp, vp, vp, vp, vp, vp], C.c_int),
+            "dwkv_append": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp], C.c_int),
             "dwkv_append_compressed": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], C.c_int),
             "dwkv_decode_attention": ([vp, i32, i32, vp, vp, vp, vp, sz, vp], C.c_int),
             "dwkv_append_decode_attention": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
@@ -104,6 +114,13 @@ def lib():
             "dwkv_quantize_residuals": ([i32, i32, i32, vp, vp, vp, vp, vp, sz, vp], C.c_int),
             "dwkv_check_bounded_wait": ([vp, C.c_uint32, vp], C.c_int),
             "dwkv_set_decode_overlap": ([vp, i32], C.c_int),
+            "dwkv_retier": ([vp, i32, i32, vp, vp, vp, vp, vp], C.c_int),
+            "dwkv_tier_controller_create": ([C.POINTER(dwkv_tier_policy), i32, C.POINTER(vp)], C.c_int),
+            "dwkv_tier_controller_destroy": ([vp], C.c_int),
+            "dwkv_tier_controller_due": ([vp, C.c_int64], i32),
+            "dwkv_tier_controller_threshold": ([vp, i32, C.POINTER(C.c_float)], C.c_int),
+            "dwkv_tier_controller_observe": ([vp, i32, C.c_float, C.POINTER(i32)], C.c_int),
+            "dwkv_tier_controller_route": ([vp, i32, i32, vp, vp, i32, vp], C.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -209,9 +226,9 @@ def dwkv_seq_length(h, seq, layer) -> int:
     return v.value
 
 
-def dwkv_append(h, layer, seq_ids, n_new, k_new, v_new, tier_idx, stream=None):
+def dwkv_append(h, layer, seq_ids, n_new, k_new, v_new, tier_idx, coeff_dbg=None, stream=None):
     _check(lib().dwkv_append(h, layer, len(seq_ids), _i32(seq_ids), _i32(n_new), _ptr(k_new), _ptr(v_new),
-                             _ptr(tier_idx), _stream(stream)))
+                             _ptr(tier_idx), _ptr(coeff_dbg), _stream(stream)))
 
 
 def dwkv_append_compressed(h, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream=None):
@@ -287,6 +304,49 @@ def dwkv_set_decode_overlap(h, enable):
     _check(lib().dwkv_set_decode_overlap(h, int(enable)))
 
 
+def dwkv_retier(h, group, seq_ids, n_tok, positions, new_tier, stream=None):
+    _check(lib().dwkv_retier(h, group, len(seq_ids), _i32(seq_ids), _i32(n_tok), _ptr(positions), _ptr(new_tier),
+                             _stream(stream)))
+
+
+def dwkv_tier_controller_create(policy: dwkv_tier_policy, num_groups: int) -> C.c_void_p:
+    c = C.c_void_p()
+    _check(lib().dwkv_tier_controller_create(C.byref(policy), num_groups, C.byref(c)))
+    return c
+
+
+def dwkv_tier_controller_destroy(c):
+    _check(lib().dwkv_tier_controller_destroy(c))
+
+
+def dwkv_tier_controller_due(c, step) -> bool:
+    return bool(lib().dwkv_tier_controller_due(c, int(step)))
+
+
+def dwkv_tier_controller_threshold(c, group) -> float:
+    v = C.c_float()
+    _check(lib().dwkv_tier_controller_threshold(c, group, C.byref(v)))
+    return v.value
+
+
+def dwkv_tier_controller_observe(c, group, err) -> bool:
+    low = C.c_int32()
+    _check(lib().dwkv_tier_controller_observe(c, group, float(err), C.byref(low)))
+    return bool(low.value)
+
+
+def dwkv_tier_controller_route(c, group, salience, base_tier, high_tier):
+    """Host arrays: salience float32 [n], base_tier uint8 [n] -> tier uint8 [n] (numpy)."""
+    import numpy as np
+    sal = np.ascontiguousarray(salience, np.float32)
+    base = np.ascontiguousarray(base_tier, np.uint8)
+    out = np.empty_like(base)
+    _check(lib().dwkv_tier_controller_route(c, group, sal.size, sal.ctypes.data_as(C.c_void_p),
+                                            base.ctypes.data_as(C.c_void_p), int(high_tier),
+                                            out.ctypes.data_as(C.c_void_p)))
+    return out
+
+
 # ------------------------------------------------------------------------------ plumbing
 class Cache:
     """Owns the torch allocations around one handle (arena and workspace) and exposes the
@@ -317,8 +377,8 @@ class Cache:
         except Exception:
             pass
 
-    def append(self, layer, seq_ids, n_new, k_new, v_new, tier_idx, stream=None):
-        dwkv_append(self.h, layer, seq_ids, n_new, k_new, v_new, tier_idx, stream)
+    def append(self, layer, seq_ids, n_new, k_new, v_new, tier_idx, stream=None, coeff_dbg=None):
+        dwkv_append(self.h, layer, seq_ids, n_new, k_new, v_new, tier_idx, coeff_dbg, stream)
 
     def append_compressed(self, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream=None):
         dwkv_append_compressed(self.h, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream)
@@ -375,3 +435,6 @@ class Cache:
 
     def set_decode_overlap(self, enable: bool):
         dwkv_set_decode_overlap(self.h, 1 if enable else 0)
+
+    def retier(self, group, seq_ids, n_tok, positions, new_tier, stream=None):
+        dwkv_retier(self.h, group, seq_ids, n_tok, positions, new_tier, stream)

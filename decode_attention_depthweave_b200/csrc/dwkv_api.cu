@@ -16,12 +16,13 @@
 namespace dwkv {
 __global__ void place_kernel(const Geom, const State, const AppendCall, const uint8_t*);
 template <int BITS>
-__global__ void encode_kernel(const Geom, const State, const AppendCall, const __nv_bfloat16*, const __nv_bfloat16*);
+__global__ void encode_kernel(const Geom, const State, const AppendCall, const __nv_bfloat16*, const __nv_bfloat16*,
+                              float*);
 template <int BITS>
 __global__ void quantize_test_kernel(int, int, const float*, uint8_t*, int8_t*, uint16_t*, uint8_t*, uint32_t);
 template <int BITS>
 __global__ void append_small_kernel(const Geom, const State, const AppendCall, const uint8_t*, int,
-                                    const __nv_bfloat16*, const __nv_bfloat16*);
+                                    const __nv_bfloat16*, const __nv_bfloat16*, float*);
 template <int BITS>
 __global__ void import_kernel(const Geom, const State, const AppendCall, const __nv_bfloat16*, const uint8_t*,
                               const int8_t*, const __half*);
@@ -29,6 +30,9 @@ template <int BITS>
 __global__ void export_kernel(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*, uint8_t*,
                               int8_t*, __half*);
 __global__ void reset_kernel(const Geom, const State, int);
+template <int BITS>
+__global__ void retier_kernel(const Geom, const State, const AppendCall, const int32_t*, const uint8_t*);
+__global__ void retier_release_kernel(const Geom, const State, const AppendCall);
 __global__ void wait_timeout_kernel(const State, uint64_t);
 template <int BITS, bool PROBE, int RMAX, int S>
 __global__ void decode_kernel(const Geom, const State, const DecodeCall);
@@ -37,8 +41,14 @@ __global__ void decode_kernel(const Geom, const State, const DecodeCall);
 using namespace dwkv;
 
 namespace {
-
 thread_local std::string g_err;
+}  // namespace
+
+namespace dwkv {
+void set_last_error(const char* msg) { g_err = msg; }
+}  // namespace dwkv
+
+namespace {
 
 dwkv_status fail(dwkv_status st, const char* fmt, ...) {
     char buf[512];
@@ -118,7 +128,7 @@ dwkv_status check_supported(const dwkv_config* c) {
 }
 
 struct MetaLayout {
-    size_t err, bump, free_head, free_tail, free_list, counts, pages, slot_map, tickets, basis_k, basis_v, data;
+    size_t err, bump, free_head, free_tail, free_list, counts, owned, pages, slot_map, tickets, basis_k, basis_v, data;
     uint32_t free_cap;
 };
 
@@ -144,7 +154,7 @@ Geom make_geom(const dwkv_config* c) {
             G.tiers[k] = c->tiers[k];
             G.blk_bytes[k] = blk_bytes_of(c->tiers[k], G.s, G.bits);
             G.chunk_bytes[k] = 2 * G.blk_bytes[k];
-            G.page_units[k] = G.LPG * G.chunk_bytes[k] / kUnit;
+            G.page_units[k] = (G.LPG * G.chunk_bytes[k] + kPosBlockBytes) / kUnit;
             stage = std::max(stage, G.chunk_bytes[k]);
         } else {
             G.tiers[k] = 0;
@@ -167,6 +177,7 @@ MetaLayout meta_layout(const Geom& G) {
     M.free_tail = take(4 * kMaxTiers);
     M.free_list = take((size_t)4 * kMaxTiers * G.free_cap);
     M.counts = take((size_t)4 * G.max_batch * G.G * G.Hkv * kMaxTiers);
+    M.owned = take((size_t)4 * G.max_batch * G.G * G.Hkv * kMaxTiers);
     M.pages = take((size_t)4 * G.max_batch * G.G * G.Hkv * kMaxTiers * G.max_pages);
     M.slot_map = take((size_t)4 * G.max_batch * G.G * G.Hkv * G.max_context);
     M.tickets = take((size_t)4 * G.max_batch * G.Hkv);
@@ -245,6 +256,7 @@ State make_state(uint8_t* arena, const MetaLayout& M, size_t arena_bytes) {
     S.free_tail = reinterpret_cast<uint32_t*>(arena + M.free_tail);
     S.free_list = reinterpret_cast<uint32_t*>(arena + M.free_list);
     S.counts = reinterpret_cast<uint32_t*>(arena + M.counts);
+    S.owned = reinterpret_cast<uint32_t*>(arena + M.owned);
     S.pages = reinterpret_cast<uint32_t*>(arena + M.pages);
     S.slot_map = reinterpret_cast<uint32_t*>(arena + M.slot_map);
     S.tickets = reinterpret_cast<uint32_t*>(arena + M.tickets);
@@ -439,7 +451,8 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
             if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs);
         // the encode kernels ask for what they use (the fused append also has static smem)
         const int es = (int)encode_smem(G), ets = (int)encode_tile_smem(G);
-        const void* enc[] = {(const void*)append_small_kernel<8>, (const void*)append_small_kernel<4>};
+        const void* enc[] = {(const void*)append_small_kernel<8>, (const void*)append_small_kernel<4>,
+                             (const void*)retier_kernel<8>, (const void*)retier_kernel<4>};
         for (const void* k : enc)
             if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, es);
         const void* tiles[] = {(const void*)encode_kernel<8>, (const void*)encode_kernel<4>};
@@ -522,7 +535,8 @@ dwkv_status dwkv_reset_sequence(dwkv_handle h, int32_t seq, void* stream) {
 }
 
 dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const int32_t* n_new,
-                        const void* k_new, const void* v_new, const uint8_t* tier_idx, void* stream) {
+                        const void* k_new, const void* v_new, const uint8_t* tier_idx, float* coeff_dbg,
+                        void* stream) {
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
     AppendCall C;
@@ -546,11 +560,11 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
         if (G.bits == 8)
             append_small_kernel<8><<<grid, 256, sm, s>>>(G, h->st, C, tier_idx, any ? 1 : 0,
                                                          static_cast<const __nv_bfloat16*>(k_new),
-                                                         static_cast<const __nv_bfloat16*>(v_new));
+                                                         static_cast<const __nv_bfloat16*>(v_new), coeff_dbg);
         else
             append_small_kernel<4><<<grid, 256, sm, s>>>(G, h->st, C, tier_idx, any ? 1 : 0,
                                                          static_cast<const __nv_bfloat16*>(k_new),
-                                                         static_cast<const __nv_bfloat16*>(v_new));
+                                                         static_cast<const __nv_bfloat16*>(v_new), coeff_dbg);
         DWKV_CUDA(cudaGetLastError(), "append_small_kernel launch");
         commit_call(h, C, n_new);
         return DWKV_OK;
@@ -566,10 +580,10 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
     const size_t tsm = encode_tile_smem(G);
     if (G.bits == 8)
         encode_kernel<8><<<grid, 256, tsm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
-                                                 static_cast<const __nv_bfloat16*>(v_new));
+                                                 static_cast<const __nv_bfloat16*>(v_new), coeff_dbg);
     else
         encode_kernel<4><<<grid, 256, tsm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
-                                                 static_cast<const __nv_bfloat16*>(v_new));
+                                                 static_cast<const __nv_bfloat16*>(v_new), coeff_dbg);
     DWKV_CUDA(cudaGetLastError(), "encode_kernel launch");
     commit_call(h, C, n_new);
     return DWKV_OK;
@@ -801,7 +815,8 @@ dwkv_status dwkv_append_decode_attention(dwkv_handle h, int32_t layer, int32_t n
     size_t smem = 0;
     if (decode_ring_for(h, false, &smem) < fused_ring_need(G)) {
         // the ring is capped below what the fused append borrows: two launches instead
-        if ((st = dwkv_append(h, layer, n_seqs, seq_ids, ones.data(), k_new, v_new, tier_idx, stream)) != DWKV_OK)
+        if ((st = dwkv_append(h, layer, n_seqs, seq_ids, ones.data(), k_new, v_new, tier_idx, nullptr, stream)) !=
+            DWKV_OK)
             return st;
         return dwkv_decode_attention(h, layer, n_seqs, seq_ids, q, out, workspace, ws_bytes, stream);
     }
@@ -813,6 +828,49 @@ dwkv_status dwkv_append_decode_attention(dwkv_handle h, int32_t layer, int32_t n
 dwkv_status dwkv_probe(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const void* q,
                        float* err, float* out_full, void* workspace, size_t ws_bytes, void* stream) {
     return run_decode(h, layer, n_seqs, seq_ids, q, nullptr, err, out_full, workspace, ws_bytes, stream, true);
+}
+
+dwkv_status dwkv_retier(dwkv_handle h, int32_t group, int32_t n_seqs, const int32_t* seq_ids, const int32_t* n_tok,
+                        const int32_t* positions, const uint8_t* new_tier, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    const Geom& G = h->geom;
+    if (group < 0 || group >= G.G) return fail(DWKV_ERR_INVALID_ARG, "group %d out of [0, %d)", group, G.G);
+    if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
+    if (n_seqs && !n_tok) return fail(DWKV_ERR_INVALID_ARG, "n_tok is NULL");
+    AppendCall C;
+    memset(&C, 0, sizeof(C));
+    C.n = n_seqs;
+    C.g = group;
+    C.layer = group * G.LPG;
+    long long total = 0;
+    for (int i = 0; i < n_seqs; ++i) {
+        const int s = seq_ids[i];
+        const int pl = h->placed[(size_t)s * G.G + group];
+        for (int l = group * G.LPG; l < (group + 1) * G.LPG; ++l)
+            if (h->len[(size_t)s * G.L + l] != pl)
+                return fail(DWKV_ERR_INVALID_ARG, "sequence %d: layer %d holds %d positions but its group placed %d; "
+                                                  "re-tier only when every layer of the group holds the same positions",
+                            s, l, h->len[(size_t)s * G.L + l], pl);
+        if (n_tok[i] < 0 || n_tok[i] > pl)
+            return fail(DWKV_ERR_INVALID_ARG, "n_tok[%d] = %d out of [0, %d]", i, n_tok[i], pl);
+        C.seq[i] = s;
+        C.tok0[i] = (int)total;
+        total += n_tok[i];
+    }
+    C.tok0[n_seqs] = (int)total;
+    C.total = (int)total;
+    if (total == 0) return DWKV_OK;
+    if (!positions || !new_tier) return fail(DWKV_ERR_INVALID_ARG, "positions and new_tier must be non-NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 grid(n_seqs, G.Hkv);
+    const size_t sm = encode_smem(G);
+    if (G.bits == 8) retier_kernel<8><<<grid, 256, sm, s>>>(G, h->st, C, positions, new_tier);
+    else retier_kernel<4><<<grid, 256, sm, s>>>(G, h->st, C, positions, new_tier);
+    DWKV_CUDA(cudaGetLastError(), "retier_kernel launch");
+    retier_release_kernel<<<1, 256, 0, s>>>(G, h->st, C);
+    DWKV_CUDA(cudaGetLastError(), "retier_release_kernel launch");
+    return DWKV_OK;
 }
 
 dwkv_status dwkv_export(dwkv_handle h, int32_t layer, int32_t seq, int32_t t0, int32_t n, uint8_t* tier_idx,

@@ -34,7 +34,9 @@ __device__ __forceinline__ void place_block(const Geom& G, const State& S, const
     if (tid < G.ntiers) {
         const int k = tid;
         const uint32_t old = s_old[k], nw = old + s_cnt[k];
-        const uint32_t po = (old + kPage - 1) / kPage, pn = (nw + kPage - 1) / kPage;
+        const uint32_t pn = (nw + kPage - 1) / kPage;
+        // pages the tier already holds (emptied by re-tiering, or partly filled) are reused
+        const uint32_t po = S.owned[ci + k];
         const size_t pi = page_index(G, seq, C.g, h, k);
         if (pn > (uint32_t)G.max_pages) {
             set_dev_error(S, 1u /*DWKV_DEV_POOL_EXHAUSTED*/, (uint32_t)seq, (uint32_t)h);
@@ -59,6 +61,7 @@ __device__ __forceinline__ void place_block(const Geom& G, const State& S, const
                         S.pages[pi + po + take + q] = (uint32_t)(base + (unsigned long long)q * G.page_units[k]);
                 }
             }
+            if (!s_fail) S.owned[ci + k] = pn;
         }
     }
     __syncthreads();
@@ -87,7 +90,10 @@ __device__ __forceinline__ void place_block(const Geom& G, const State& S, const
             if (k != 0xffu) {
                 uint32_t off = s_run[k];
                 for (int w = 0; w < warp; ++w) off += s_warp[w][k];
-                S.slot_map[si + p] = ((k + 1u) << 24) | (off + rank);
+                const uint32_t slot = off + rank;
+                S.slot_map[si + p] = ((k + 1u) << 24) | slot;
+                const uint32_t unit = S.pages[page_index(G, seq, C.g, h, k) + slot / kPage];
+                reinterpret_cast<int32_t*>(S.data + (size_t)unit * kUnit + pos_block_of(G, k))[slot % kPage] = a0 + p;
             } else {
                 S.slot_map[si + p] = 0u;
             }
@@ -153,7 +159,8 @@ __device__ __forceinline__ void bases_store(const Geom& G, const uint4 (&v)[kBas
 
 __device__ __forceinline__ UnitIn encode_fetch(const Geom& G, const State& S, const AppendCall& C,
                                                const __nv_bfloat16* __restrict__ k_new,
-                                               const __nv_bfloat16* __restrict__ v_new, int h, int unit) {
+                                               const __nv_bfloat16* __restrict__ v_new, int h, int unit,
+                                               float* coeff_dbg) {
     const int lane = threadIdx.x & 31;
     const int row = unit >> 1, z = unit & 1;
     const int ci = call_index_of(C, row);
@@ -164,6 +171,7 @@ __device__ __forceinline__ UnitIn encode_fetch(const Geom& G, const State& S, co
 #pragma unroll
     for (int m = 0; m < 4; ++m) in.xr[m] = __bfloat162float(src[lane + 32 * m]);
     in.ok = find_dest(G, S, seq, C.g, C.lig, h, pos, in.dst);
+    in.dbg = coeff_dbg ? coeff_dbg + (((size_t)row * G.Hkv + h) * 2 + z) * G.r_max : nullptr;
     // a0..a0+na were placed by the placement; a zero entry means placement failed (already
     // reported) or the group never placed this position
     if (!in.ok && lane == 0 && z == 0 && !(pos >= C.a0[ci] && pos < C.a0[ci] + C.na[ci]))
@@ -173,58 +181,71 @@ __device__ __forceinline__ UnitIn encode_fetch(const Geom& G, const State& S, co
 
 // ------------------------------------------------------------------------------------
 // Bulk encode kernel.  A block per (kv-head, keys or values) strides over tiles of kEncTile
-// input rows and runs the six encode steps on all of a tile's vectors together, so that
-// every shared-memory load feeds several fma chains:
+// input rows and runs the encode steps on all of a tile's vectors together:
 //   1. the rows' destinations (slot map), counted by tier and given slots in descending
-//      tier order; each row's x enters shared memory (fp32, [channel][slot]) at its slot;
-//   2. projection items of 32 slots x 16 coefficients: each lane runs the full i = 0..d-1
-//      chains of 8 slots x 2 coefficients (x of 8 slots and a bf16 coefficient pair per
-//      step); the group's chains run to the largest rank among its 32 slots (the first
-//      slot, by the sort), and the coefficients past a slot's own rank are neither stored
-//      nor kept: they enter its residual as exact zeros;
-//   3. residual items of 4 slots, lane = channels lane + 32 m: the chains over j run to the
-//      largest rank of the 4 slots; a zero coefficient adds an exact +-0 to an accumulator
-//      that started at +0, which leaves it unchanged, so every slot gets the residual of
-//      its own-length chain; then steps 4-6 per slot (quantize_store).
-// The arithmetic per vector is the same operations in the same order as encode_body, so
-// the stored bytes are identical to the per-warp encoders'.  Three 256-thread blocks fit an
-// SM (80 registers, ~72 KB of shared memory at r_max 64).  The kernel has no waits of its own
-// beyond block barriers.
+//      tier order; each row's x enters shared memory as bf16 [slot][channel];
+//   2. the projection on the tensor cores: a warp takes 16 slots (one MMA row tile) and half
+//      of their coefficient tiles, c = X B as bf16 x bf16 products accumulated in fp32 (within
+//      1e-5 |x| of the fp64 projection; the order of the accumulation is the tensor core's),
+//      up to the largest rank among its slots (the first slot, by the sort); then the bf16
+//      rounding and the coefficient stores (a slot's coefficients past its own rank are
+//      neither stored nor kept: they enter its residual as exact zeros), and the fp32
+//      projection exported when asked (coeff_dbg);
+//   3. residual items of 4 slots, lane = channels lane + 32 m: the fixed-order fma chains
+//      over j of step 3 run to the largest rank of the 4 slots; a zero coefficient adds an
+//      exact +-0 to an accumulator that started at +0, which leaves it unchanged, so every
+//      slot gets the residual of its own-length chain; then steps 4-6 per slot (quantize_store).
+// Steps 2 (rounding) to 6 are the same operations in the same order as encode_body's, so the
+// stored bytes follow from the exported projection bit for bit.  Three 256-thread blocks fit
+// an SM at r_max 64 (~76 KB of shared memory).  The kernel has no waits of its own beyond
+// block barriers.
 // ------------------------------------------------------------------------------------
 template <int BITS>
 __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const State S, const AppendCall C,
                                                         const __nv_bfloat16* __restrict__ k_new,
-                                                        const __nv_bfloat16* __restrict__ v_new) {
+                                                        const __nv_bfloat16* __restrict__ v_new,
+                                                        float* __restrict__ coeff_dbg) {
     extern __shared__ __align__(16) uint8_t smem[];
     const EncTileLayout L = enc_tile_layout(G.r_max);
     const int h = blockIdx.y, z = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem + L.bs);
-    float* xs = reinterpret_cast<float*>(smem + L.xs);
+    __nv_bfloat16* bt = reinterpret_cast<__nv_bfloat16*>(smem + L.bt);
+    __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(smem + L.xb);
     float* cs = reinterpret_cast<float*>(smem + L.cs);
     uint8_t** sblk = reinterpret_cast<uint8_t**>(smem + L.sblk);
     int* sR = reinterpret_cast<int*>(smem + L.sR);
     int* sprow = reinterpret_cast<int*>(smem + L.sprow);
+    int* srow = reinterpret_cast<int*>(smem + L.srow);
     int* rslot = reinterpret_cast<int*>(smem + L.rslot);
     int* cnt = reinterpret_cast<int*>(smem + L.misc);
     int* base = cnt + kMaxTiers;
     int* nvalid_p = base + kMaxTiers;
     float* rstage = reinterpret_cast<float*>(smem + L.cst + warp * kEncStage);
     uint8_t* chstage = reinterpret_cast<uint8_t*>(rstage + kD);
-    const int RM = G.r_max, PB = L.PB, npass = L.RP / 16;
+    const int RM = G.r_max, PB = L.PB;
 
-    // ---- this (group, kv-head, K or V) basis: bf16 [kD][PB], the columns past r_max zero
+    // ---- this (group, kv-head, K or V) basis: bf16 [kD][PB] and transposed [RP][kEncXB],
+    //      the columns past r_max zero
     {
         const __nv_bfloat16* src = (z ? S.basis_v : S.basis_k) + ((size_t)C.g * G.Hkv + h) * kD * RM;
         uint16_t* b16 = reinterpret_cast<uint16_t*>(bs);
+        uint16_t* t16 = reinterpret_cast<uint16_t*>(bt);
         const int padc = PB - RM;
         for (int e = tid; e < kD * padc; e += blockDim.x) b16[(e / padc) * PB + RM + e % padc] = 0;
+        for (int e = tid; e < (L.RP - RM) * kD; e += blockDim.x) t16[(RM + e / kD) * kEncXB + e % kD] = 0;
         const int nvec = kD * RM / 8;
         for (int e = tid; e < nvec; e += blockDim.x) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + e);
             const int i = (e * 8) / RM, j = (e * 8) % RM;
             uint32_t* dst = reinterpret_cast<uint32_t*>(bs + (size_t)i * PB + j);
             dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                t16[(j + 2 * q) * kEncXB + i] = (uint16_t)(w4[q] & 0xffffu);
+                t16[(j + 2 * q + 1) * kEncXB + i] = (uint16_t)(w4[q] >> 16);
+            }
         }
     }
 
@@ -275,6 +296,7 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
                 sblk[slot] = d.blk + (z ? G.blk_bytes[d.k] : 0u);
                 sR[slot] = d.R;
                 sprow[slot] = d.row;
+                srow[slot] = row;
             }
             rslot[trow] = slot;
         }
@@ -283,59 +305,65 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
         {
             const int slot = rslot[trow];
             if (slot >= 0) {
+                uint4* dst = reinterpret_cast<uint4*>(xb + (size_t)slot * kEncXB + 32 * q);
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const uint32_t w[4] = {xv[b].x, xv[b].y, xv[b].z, xv[b].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 32 * q + 8 * b + 2 * e;
-                        xs[i * kEncXP + slot] = __uint_as_float(w[e] << 16);
-                        xs[(i + 1) * kEncXP + slot] = __uint_as_float(w[e] & 0xffff0000u);
-                    }
-                }
+                for (int b = 0; b < 4; ++b) dst[b] = xv[b];
             }
-            const int nempty = kEncTile - nvalid;
-            for (int e = tid; e < nempty * kD; e += blockDim.x) xs[(e / nempty) * kEncXP + nvalid + e % nempty] = 0.f;
         }
         __syncthreads();
 
-        // ---- 2: projection, bf16 rounding, coefficient stores
-        const int ngroups = (nvalid + 31) >> 5;
-        for (int it = warp; it < ngroups * npass; it += (int)(blockDim.x >> 5)) {
-            const int g = it / npass, p = it % npass;
-            if (16 * p >= sR[32 * g]) continue;
-            const int s0 = 32 * g + 8 * (lane >> 3), j0 = 16 * p + 2 * (lane & 7);
-            float acc[8][2];
+        // ---- 2: projection on the tensor cores, bf16 rounding, coefficient stores
+        {
+            const int mt = warp & 3, nh = warp >> 2;
+            const int Rm = 16 * mt < nvalid ? sR[16 * mt] : 0;
+            if (Rm > 0) {
+                const int g = lane >> 2, c = lane & 3;
+                const uint32_t xaddr = smem_addr(xb + (size_t)(16 * mt + (lane & 15)) * kEncXB + 8 * (lane >> 4));
+                const uint32_t baddr = smem_addr(bt + (size_t)(lane & 7) * kEncXB + 8 * ((lane >> 3) & 1));
+                const int ntl = Rm / 8;                        // coefficient tiles of 8; this warp: nh, nh + 2, ...
+                for (int u0 = nh; u0 < ntl; u0 += 8) {         // up to 4 tiles at a time
+                    float dd[4][4];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) acc[t][0] = acc[t][1] = 0.f;
-            const float* xp = xs + s0;
-            const uint32_t* bp = reinterpret_cast<const uint32_t*>(bs + j0);
-#pragma unroll 4
-            for (int i = 0; i < kD; ++i) {
-                const float4 xa = *reinterpret_cast<const float4*>(xp + i * kEncXP);
-                const float4 xb = *reinterpret_cast<const float4*>(xp + i * kEncXP + 4);
-                const uint32_t bb = bp[i * (PB >> 1)];
-                const float b0 = __uint_as_float(bb << 16), b1 = __uint_as_float(bb & 0xffff0000u);
-                const float x8[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                    for (int u = 0; u < 4; ++u) dd[u][0] = dd[u][1] = dd[u][2] = dd[u][3] = 0.f;
 #pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    acc[t][0] = __fmaf_rn(b0, x8[t], acc[t][0]);
-                    acc[t][1] = __fmaf_rn(b1, x8[t], acc[t][1]);
-                }
-            }
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        uint32_t af[4];
+                        ldsm_x4(xaddr + 32u * ks, af);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const int sl = s0 + t;
-                const bool on = j0 < sR[sl];           // ranks are multiples of 8: j0 + 1 too
-                const __nv_bfloat16 c0 = __float2bfloat16_rn(acc[t][0]), c1 = __float2bfloat16_rn(acc[t][1]);
-                cs[j0 * kEncXP + sl] = on ? __bfloat162float(c0) : 0.f;
-                cs[(j0 + 1) * kEncXP + sl] = on ? __bfloat162float(c1) : 0.f;
-                if (on) {
-                    __nv_bfloat162 pr;
-                    pr.x = c0;
-                    pr.y = c1;
-                    *reinterpret_cast<__nv_bfloat162*>(sblk[sl] + (size_t)(j0 >> 3) * 1024 + sprow[sl] * 16 +
-                                                       (j0 & 7) * 2) = pr;
+                        for (int u = 0; u < 4; ++u) {
+                            const int nt = u0 + 2 * u;
+                            if (nt < ntl) {
+                                uint32_t b[2];
+                                ldsm_x2(baddr + (uint32_t)(8 * nt) * (kEncXB * 2) + 32u * ks, b);
+                                mma_bf16(dd[u], af, b);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int nt = u0 + 2 * u;
+                        if (nt >= ntl) break;
+                        const int j0 = 8 * nt + 2 * c;
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int sl = 16 * mt + g + 8 * hf;
+                            const float v0 = dd[u][2 * hf], v1 = dd[u][2 * hf + 1];
+                            const bool on = j0 < sR[sl];           // ranks are multiples of 8: j0 + 1 too
+                            const __nv_bfloat16 c0 = __float2bfloat16_rn(v0), c1 = __float2bfloat16_rn(v1);
+                            cs[j0 * kEncXP + sl] = on ? __bfloat162float(c0) : 0.f;
+                            cs[(j0 + 1) * kEncXP + sl] = on ? __bfloat162float(c1) : 0.f;
+                            if (on) {
+                                __nv_bfloat162 pr;
+                                pr.x = c0;
+                                pr.y = c1;
+                                *reinterpret_cast<__nv_bfloat162*>(sblk[sl] + (size_t)(j0 >> 3) * 1024 + sprow[sl] * 16 +
+                                                                   (j0 & 7) * 2) = pr;
+                                if (coeff_dbg)
+                                    *reinterpret_cast<float2*>(coeff_dbg + (((size_t)srow[sl] * G.Hkv + h) * 2 + z) * RM +
+                                                               j0) = make_float2(v0, v1);
+                            }
+                        }
+                    }
                 }
             }
         }
@@ -367,11 +395,11 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
                 }
             }
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 xa = *reinterpret_cast<const float4*>(xs + (lane + 32 * m) * kEncXP + s0);
-                const float x4[4] = {xa.x, xa.y, xa.z, xa.w};
+            for (int t = 0; t < 4; ++t) {
+                const int sl = s0 + t;
 #pragma unroll
-                for (int t = 0; t < 4; ++t) a[t][m] = __fsub_rn(x4[t], a[t][m]);
+                for (int m = 0; m < 4; ++m)
+                    a[t][m] = __fsub_rn(__bfloat162float(xb[(size_t)sl * kEncXB + lane + 32 * m]), a[t][m]);
             }
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
@@ -444,7 +472,8 @@ template <int BITS>
 __global__ void __launch_bounds__(256) append_small_kernel(const Geom G, const State S, const AppendCall C,
                                                            const uint8_t* __restrict__ tier_idx, int place,
                                                            const __nv_bfloat16* __restrict__ k_new,
-                                                           const __nv_bfloat16* __restrict__ v_new) {
+                                                           const __nv_bfloat16* __restrict__ v_new,
+                                                           float* coeff_dbg) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int i = blockIdx.x, h = blockIdx.y, warp = threadIdx.x >> 5;
     __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem);
@@ -456,12 +485,12 @@ __global__ void __launch_bounds__(256) append_small_kernel(const Geom G, const S
     const int unit = u0 + warp;                    // at most 4 rows: one unit per warp
     UnitIn in;
     in.ok = false;
-    if (!place && unit < u1) in = encode_fetch(G, S, C, k_new, v_new, h, unit);
+    if (!place && unit < u1) in = encode_fetch(G, S, C, k_new, v_new, h, unit, coeff_dbg);
     if (place) place_block(G, S, C, tier_idx, i, h);
     bases_store(G, bv, bs);
     __syncthreads();                         // bases in smem; slots and pages written (block scope)
     if (unit < u1) {
-        if (place) in = encode_fetch(G, S, C, k_new, v_new, h, unit);
+        if (place) in = encode_fetch(G, S, C, k_new, v_new, h, unit, coeff_dbg);
         encode_body<BITS>(G, S, bs, enc_scratch(G, smem, warp), unit, in);
     }
 }
@@ -583,7 +612,7 @@ __global__ void __launch_bounds__(256) reset_kernel(const Geom G, const State S,
             if (pr < pairs) {
                 g = pr / G.Hkv;
                 h = pr % G.Hkv;
-                np = (S.counts[cnt_index(G, seq, g, h) + k] + kPage - 1) / kPage;
+                np = S.owned[cnt_index(G, seq, g, h) + k];
             }
             uint32_t incl = np;
 #pragma unroll
@@ -620,25 +649,222 @@ __global__ void __launch_bounds__(256) reset_kernel(const Geom G, const State S,
         }
         __syncthreads();
     }
-    for (int e = tid; e < pairs * kMaxTiers; e += blockDim.x)
+    for (int e = tid; e < pairs * kMaxTiers; e += blockDim.x) {
         S.counts[cnt_index(G, seq, 0, 0) + e] = 0u;
+        S.owned[cnt_index(G, seq, 0, 0) + e] = 0u;
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Re-tiering ("DepthWeave-KV ...", §3, Eq. (2)-(3) paragraphs: the probe's feedback moves the
+// router threshold, so a token's rank tier changes).  One block per (sequence in call,
+// kv-head) takes the call's tokens of its sequence in order; for each token whose tier
+// changes:
+//   1. a slot at the end of the new tier (place_one: slot map and page position updated);
+//   2. every layer's keys and values re-encoded there from the token's reconstruction, a_i =
+//      fma chain over j < r_old of B[i][j] cb_j from +0, plus scale * code on its residual
+//      channels, rounded to bf16 (the dense vector is not kept), by the six encode steps at
+//      the new rank (encode_body: the same operations as every encoder);
+//   3. the old tier's last slot moved into the token's old slot (all layers' rows and the
+//      page position; the moved token's slot-map entry follows), and both counts updated.
+// Softmax is order-free, so the order of slots within a tier does not matter; a page the old
+// tier empties stays with the tier (owned) until retier_release_kernel returns it.
+// ------------------------------------------------------------------------------------
+template <int BITS>
+__global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S, const AppendCall C,
+                                                     const int32_t* __restrict__ positions,
+                                                     const uint8_t* __restrict__ new_tier) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int i = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem);
+    {
+        uint4 bv[kBasisRegs];
+        bases_issue(G, S, C.g, h, bv);
+        bases_store(G, bv, bs);
+    }
+    __shared__ int s_go, s_kold, s_knew, s_slot, s_last;
+    __shared__ uint32_t s_unit_old, s_unit_last;
+    __shared__ Dest s_dst;
+    const int seq = C.seq[i], P = G.r_max + 2;
+    const size_t ci = cnt_index(G, seq, C.g, h);
+    for (int t = C.tok0[i]; t < C.tok0[i + 1]; ++t) {
+        __syncthreads();                               // the previous token is done
+        if (tid == 0) {
+            int go = 0;
+            const int pos = positions[t];
+            const uint32_t knew = new_tier[(size_t)t * G.Hkv + h];
+            const uint32_t sm = (pos >= 0 && pos < G.max_context) ? S.slot_map[slot_index(G, seq, C.g, h, pos)] : 0u;
+            if (sm == 0u) {
+                set_dev_error(S, 5u /*DWKV_DEV_NO_SLOT*/, (uint32_t)seq, (uint32_t)pos);
+            } else if (knew >= (uint32_t)G.ntiers) {
+                set_dev_error(S, 2u /*DWKV_DEV_BAD_TIER*/, (uint32_t)seq, (uint32_t)pos);
+            } else {
+                const uint32_t kold = (sm >> 24) - 1u, slot = sm & 0xffffffu;
+                Dest d;
+                if (kold != knew && place_one(G, S, seq, C.g, h, pos, knew, d, 0)) {
+                    const size_t po = page_index(G, seq, C.g, h, (int)kold);
+                    const uint32_t last = S.counts[ci + kold] - 1u;
+                    s_kold = (int)kold;
+                    s_knew = (int)knew;
+                    s_slot = (int)slot;
+                    s_last = (int)last;
+                    s_unit_old = S.pages[po + slot / kPage];
+                    s_unit_last = S.pages[po + last / kPage];
+                    s_dst = d;
+                    go = 1;
+                }
+            }
+            s_go = go;
+        }
+        __syncthreads();
+        if (!s_go) continue;
+        const int kold = s_kold, knew = s_knew, slot = s_slot, last = s_last;
+        const int Rold = G.tiers[kold], row = slot % kPage;
+        // ---- 2: re-encode every (layer, K / V) unit of the token, a warp each
+        for (int u = warp; u < 2 * G.LPG; u += (int)(blockDim.x >> 5)) {
+            const int lig = u >> 1, z = u & 1;
+            const uint8_t* ob = S.data + (size_t)s_unit_old * kUnit + (size_t)lig * G.chunk_bytes[kold] +
+                                (z ? G.blk_bytes[kold] : 0u);
+            const __nv_bfloat16* bz = bs + (size_t)z * kD * P;
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int j = 0; j < Rold; ++j) {
+                const float cj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                    ob + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2));
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    a[m] = __fmaf_rn(__bfloat162float(bz[(size_t)(lane + 32 * m) * P + j]), cj, a[m]);
+            }
+            if (G.s > 0) {
+                const float sf = __half2float(*reinterpret_cast<const __half*>(ob + off_scales_of(Rold, G.s, BITS) + row * 2));
+                for (int e = 0; e < G.s; ++e) {
+                    const int ch = ob[off_idx_of(Rold) + row * G.s + e];
+                    int code;
+                    if (BITS == 8) {
+                        code = (int8_t)ob[off_codes_of(Rold, G.s) + row * G.s + e];
+                    } else {
+                        const uint32_t byte = ob[off_codes_of(Rold, G.s) + row * (G.s / 2) + (e >> 1)];
+                        code = (int)(((e & 1) ? byte >> 4 : byte) & 0xfu);
+                        code = (code ^ 8) - 8;
+                    }
+                    if ((ch & 31) == lane && ch < kD) {
+                        const float v = __fmul_rn(sf, (float)code);       // exact: 11 x 7 significant bits
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            if ((ch >> 5) == m) a[m] = __fadd_rn(a[m], v);
+                    }
+                }
+            }
+            UnitIn in;
+            in.ok = true;
+            in.dbg = nullptr;
+            in.dst = s_dst;
+            in.dst.blk = s_dst.blk + (size_t)lig * G.chunk_bytes[knew];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) in.xr[m] = __bfloat162float(__float2bfloat16_rn(a[m]));
+            encode_body<BITS>(G, S, bs, enc_scratch(G, smem, warp), z, in);
+        }
+        __syncthreads();
+        // ---- 3: the old tier's last slot into the token's old slot
+        if (slot != last) {
+            const int lrow = last % kPage;
+            const uint32_t blk = G.blk_bytes[kold];
+            const uint32_t coff = off_idx_of(Rold);
+            const uint32_t nidx = (uint32_t)G.s, ncode = (uint32_t)G.s * BITS / 8;
+            for (int u = warp; u < 2 * G.LPG; u += (int)(blockDim.x >> 5)) {
+                const int lig = u >> 1, z = u & 1;
+                uint8_t* dst = S.data + (size_t)s_unit_old * kUnit + (size_t)lig * G.chunk_bytes[kold] + (z ? blk : 0u);
+                const uint8_t* src = S.data + (size_t)s_unit_last * kUnit + (size_t)lig * G.chunk_bytes[kold] + (z ? blk : 0u);
+                for (int c = lane; c < Rold / 8; c += 32)       // 8-coefficient columns, 16 bytes a token
+                    *reinterpret_cast<uint4*>(dst + (size_t)c * 1024 + row * 16) =
+                        *reinterpret_cast<const uint4*>(src + (size_t)c * 1024 + lrow * 16);
+                for (uint32_t b = lane; b < nidx; b += 32) dst[coff + row * nidx + b] = src[coff + lrow * nidx + b];
+                const uint32_t qo = off_codes_of(Rold, G.s);
+                for (uint32_t b = lane; b < ncode; b += 32) dst[qo + row * ncode + b] = src[qo + lrow * ncode + b];
+                if (lane == 0) {
+                    const uint32_t so = off_scales_of(Rold, G.s, BITS);
+                    *reinterpret_cast<uint16_t*>(dst + so + row * 2) = *reinterpret_cast<const uint16_t*>(src + so + lrow * 2);
+                }
+            }
+            if (tid == 0) {
+                const int32_t* lp = reinterpret_cast<const int32_t*>(S.data + (size_t)s_unit_last * kUnit + pos_block_of(G, kold));
+                int32_t* sp = reinterpret_cast<int32_t*>(S.data + (size_t)s_unit_old * kUnit + pos_block_of(G, kold));
+                const int32_t moved = lp[lrow];
+                sp[row] = moved;
+                S.slot_map[slot_index(G, seq, C.g, h, moved)] = ((uint32_t)(kold + 1) << 24) | (uint32_t)slot;
+            }
+        }
+        if (tid == 0) {
+            S.counts[ci + kold] = (uint32_t)last;
+            S.counts[ci + knew] += 1u;
+        }
+    }
+}
+
+// After re-tiering: the pages a tier holds beyond ceil(count / 64) go back to the tier's free
+// ring.  One block for the whole call (no other kernel takes from the rings meanwhile).
+__global__ void __launch_bounds__(256) retier_release_kernel(const Geom G, const State S, const AppendCall C) {
+    const int tid = threadIdx.x;
+    __shared__ uint32_t s_tail[kMaxTiers], s_total[kMaxTiers], s_over[kMaxTiers];
+    if (tid < kMaxTiers) {
+        s_total[tid] = 0u;
+        s_over[tid] = 0u;
+        s_tail[tid] = tid < G.ntiers ? S.free_tail[tid] : 0u;
+    }
+    __syncthreads();
+    const int pairs = C.n * G.Hkv;
+    // 1: how many pages each tier gives back
+    for (int e = tid; e < pairs * G.ntiers; e += blockDim.x) {
+        const int k = e % G.ntiers, pr = e / G.ntiers;
+        const size_t ci = cnt_index(G, C.seq[pr / G.Hkv], C.g, pr % G.Hkv);
+        const uint32_t keep = (S.counts[ci + k] + kPage - 1) / kPage, ow = S.owned[ci + k];
+        if (ow > keep) atomicAdd(&s_total[k], ow - keep);
+    }
+    __syncthreads();
+    if (tid < G.ntiers) {
+        uint32_t hd = S.free_head[tid];
+        if ((int)(hd - s_tail[tid]) > 0) hd = s_tail[tid];
+        if ((s_tail[tid] - hd) + s_total[tid] > G.free_cap) {
+            s_over[tid] = 1u;
+            set_dev_error(S, 7u /*DWKV_DEV_FREE_LIST*/, 0xffffffffu, (uint32_t)tid);
+        }
+        s_total[tid] = 0u;
+    }
+    __syncthreads();
+    // 2: push them (ring order does not matter)
+    for (int e = tid; e < pairs * G.ntiers; e += blockDim.x) {
+        const int k = e % G.ntiers, pr = e / G.ntiers;
+        const int seq = C.seq[pr / G.Hkv], h = pr % G.Hkv;
+        const size_t ci = cnt_index(G, seq, C.g, h);
+        const uint32_t keep = (S.counts[ci + k] + kPage - 1) / kPage, ow = S.owned[ci + k];
+        if (ow > keep && !s_over[k]) {
+            const uint32_t at = atomicAdd(&s_total[k], ow - keep);
+            const size_t pi = page_index(G, seq, C.g, h, k);
+            for (uint32_t q = keep; q < ow; ++q)
+                S.free_list[(size_t)k * G.free_cap + ((s_tail[k] + at + q - keep) & (G.free_cap - 1))] = S.pages[pi + q];
+            S.owned[ci + k] = keep;
+        }
+    }
+    __syncthreads();
+    if (tid < G.ntiers && !s_over[tid]) S.free_tail[tid] = s_tail[tid] + s_total[tid];
 }
 
 }  // namespace dwkv
 
 namespace dwkv {
+template __global__ void retier_kernel<8>(const Geom, const State, const AppendCall, const int32_t*, const uint8_t*);
+template __global__ void retier_kernel<4>(const Geom, const State, const AppendCall, const int32_t*, const uint8_t*);
 template __global__ void encode_kernel<8>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
-                                          const __nv_bfloat16*);
+                                          const __nv_bfloat16*, float*);
 template __global__ void encode_kernel<4>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
-                                          const __nv_bfloat16*);
+                                          const __nv_bfloat16*, float*);
 template __global__ void quantize_test_kernel<8>(int, int, const float*, uint8_t*, int8_t*, uint16_t*, uint8_t*,
                                                   uint32_t);
 template __global__ void quantize_test_kernel<4>(int, int, const float*, uint8_t*, int8_t*, uint16_t*, uint8_t*,
                                                   uint32_t);
 template __global__ void append_small_kernel<8>(const Geom, const State, const AppendCall, const uint8_t*, int,
-                                                const __nv_bfloat16*, const __nv_bfloat16*);
+                                                const __nv_bfloat16*, const __nv_bfloat16*, float*);
 template __global__ void append_small_kernel<4>(const Geom, const State, const AppendCall, const uint8_t*, int,
-                                                const __nv_bfloat16*, const __nv_bfloat16*);
+                                                const __nv_bfloat16*, const __nv_bfloat16*, float*);
 template __global__ void import_kernel<8>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
                                           const uint8_t*, const int8_t*, const __half*);
 template __global__ void import_kernel<4>(const Geom, const State, const AppendCall, const __nv_bfloat16*,

@@ -16,6 +16,9 @@
 //       scales [64]       fp16       128
 //     Every part is a multiple of 128 bytes, so pages are 128-byte aligned and every page
 //     chunk is a legal bulk-copy (TMA) source.
+//   * After the layers' chunks a page holds the position of each of its 64 slots (int32), so
+//     a slot can be moved within its tier (re-tiering) with its slot-map entry; decode never
+//     reads it.
 //   * The page pool is handed out in 128-byte units by a device bump pointer plus one
 //     free ring per tier (filled by sequence resets).
 #pragma once
@@ -57,6 +60,8 @@ struct State {
     uint32_t* free_tail;             // [kMaxTiers] ring write index (monotonic)
     uint32_t* free_list;             // [kMaxTiers][free_cap] page units
     uint32_t* counts;                // [max_batch][G][Hkv][kMaxTiers] slots placed
+    uint32_t* owned;                 // [max_batch][G][Hkv][kMaxTiers] pages held (>= ceil(counts / 64);
+                                     //   re-tiering can empty a page the tier keeps for reuse)
     uint32_t* pages;                 // [max_batch][G][Hkv][kMaxTiers][max_pages] unit offsets
     uint32_t* slot_map;              // [max_batch][G][Hkv][max_context]: ((tier+1)<<24)|slot
     uint32_t* tickets;               // [max_batch][Hkv] split-combine tickets
@@ -111,6 +116,10 @@ __host__ __device__ inline uint32_t off_codes_of(int R, int s) { return 128u * R
 __host__ __device__ inline uint32_t off_scales_of(int R, int s, int bits) {
     return 128u * R + 64u * s + 8u * s * bits;
 }
+// Byte offset of a page's slot-position block (after the layers' chunks).
+__host__ __device__ inline uint32_t pos_block_of(const Geom& G, int k) { return (uint32_t)G.LPG * G.chunk_bytes[k]; }
+constexpr uint32_t kPosBlockBytes = kPage * 4;
+
 __host__ __device__ inline size_t cnt_index(const Geom& G, int seq, int g, int h) {
     return (((size_t)seq * G.G + g) * G.Hkv + h) * kMaxTiers;
 }
@@ -280,6 +289,46 @@ __device__ __forceinline__ void red_release_add_u32(uint32_t* p, uint32_t v) {
 // (async-proxy) copies.
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ warp-level MMA pieces (sm_80+ forms)
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t (&r)[2]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(addr));
+}
+// D (16x8 f32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// D (16x8 s32) = A (16x32 s8, row) * B (32x8 u8, col) + C
+__device__ __forceinline__ void mma_s8u8(int (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(addr));
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

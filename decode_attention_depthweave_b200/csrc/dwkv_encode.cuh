@@ -35,8 +35,10 @@ __device__ __forceinline__ bool find_dest(const Geom& G, const State& S, int seq
 }
 
 // Slot of one new position of (seq, group g, kv-head h) in tier k, the counts left as they are
-// (the caller adds the position to them later): the tier's next slot, and a fresh page when the
-// slot opens one (the tier's free ring first, then the pool's bump pointer).  Single thread.
+// (the caller adds the position to them later): the tier's next slot, and, when the slot opens
+// a page, a page the tier already holds or else a fresh one (the tier's free ring first, then
+// the pool's bump pointer).  Records the slot in the slot map and the position in the page.
+// Single thread.
 __device__ __forceinline__ bool place_one(const Geom& G, const State& S, int seq, int g, int h, int pos,
                                           uint32_t k, Dest& d, int lig) {
     const uint32_t old = __ldcg(S.counts + cnt_index(G, seq, g, h) + k);
@@ -46,7 +48,9 @@ __device__ __forceinline__ bool place_one(const Geom& G, const State& S, int seq
         return false;
     }
     uint32_t unit;
-    if (old % kPage == 0) {
+    if (old % kPage == 0 && pi < __ldcg(S.owned + cnt_index(G, seq, g, h) + k)) {
+        unit = __ldcg(S.pages + page_index(G, seq, g, h, k) + pi);
+    } else if (old % kPage == 0) {
         const uint32_t t = atomicAdd(&S.free_head[k], 1u);
         const uint32_t tail = *((volatile uint32_t*)&S.free_tail[k]);
         if ((int)(tail - t) > 0) {
@@ -60,10 +64,12 @@ __device__ __forceinline__ bool place_one(const Geom& G, const State& S, int seq
             unit = (uint32_t)base;
         }
         S.pages[page_index(G, seq, g, h, k) + pi] = unit;
+        S.owned[cnt_index(G, seq, g, h) + k] = pi + 1;
     } else {
         unit = __ldcg(S.pages + page_index(G, seq, g, h, k) + pi);
     }
     S.slot_map[slot_index(G, seq, g, h, pos)] = ((k + 1u) << 24) | old;
+    reinterpret_cast<int32_t*>(S.data + (size_t)unit * kUnit + pos_block_of(G, (int)k))[old % kPage] = pos;
     d.k = (int)k;
     d.row = (int)(old % kPage);
     d.R = G.tiers[k];
@@ -73,13 +79,17 @@ __device__ __forceinline__ bool place_one(const Geom& G, const State& S, int seq
 
 // Shared memory of the bulk encode kernel (one tile of kEncTile rows, one of K or V):
 // the basis bf16 [kD][PB] (PB = RP + 2, RP = r_max rounded up to 16; the odd word pitch
-// makes column reads conflict-free), x and the stored coefficients fp32 [.][kEncXP] by slot,
-// per-slot destinations, tier counts, and each warp's code staging.
+// makes column reads conflict-free) for the residual step, the basis transposed bf16
+// [RP][kEncXB] and the tile's x bf16 [kEncTile][kEncXB] by slot (the tensor-core operands of
+// the projection; a 272-byte row pitch keeps ldmatrix conflict-free), the stored
+// coefficients fp32 [RP][kEncXP] by slot, per-slot destinations and input rows, tier counts,
+// and each warp's code staging.
 constexpr int kEncTile = 64;
 constexpr int kEncXP = kEncTile + 4;
+constexpr int kEncXB = kD + 8;
 constexpr int kEncStage = kD * 4 + kD;   // per warp: residuals and channels in rank order
 struct EncTileLayout {
-    uint32_t bs, xs, cs, sblk, sR, sprow, rslot, misc, cst, total;
+    uint32_t bs, bt, xb, cs, sblk, sR, sprow, srow, rslot, misc, cst, total;
     int RP, PB;
 };
 __host__ __device__ inline EncTileLayout enc_tile_layout(int r_max) {
@@ -88,11 +98,13 @@ __host__ __device__ inline EncTileLayout enc_tile_layout(int r_max) {
     L.PB = L.RP + 2;
     uint32_t o = 0;
     L.bs = o;    o += (uint32_t)kD * L.PB * 2;  o = (o + 15u) & ~15u;
-    L.xs = o;    o += (uint32_t)kD * kEncXP * 4;
+    L.bt = o;    o += (uint32_t)L.RP * kEncXB * 2;
+    L.xb = o;    o += (uint32_t)kEncTile * kEncXB * 2;
     L.cs = o;    o += (uint32_t)L.RP * kEncXP * 4;
     L.sblk = o;  o += kEncTile * 8;
     L.sR = o;    o += kEncTile * 4;
     L.sprow = o; o += kEncTile * 4;
+    L.srow = o;  o += kEncTile * 4;
     L.rslot = o; o += kEncTile * 4;
     L.misc = o;  o += 128;
     L.cst = o;   o += 8 * kEncStage;
@@ -117,6 +129,7 @@ struct UnitIn {
     Dest dst;
     float xr[4];
     bool ok;
+    float* dbg;      // nullable: the unit's fp32 projection c[j], j < r_t (coefficient export)
 };
 
 // Step 4 by its definition: s rounds of "largest remaining |r|, ties to the lower channel"
@@ -271,6 +284,7 @@ __device__ __forceinline__ void encode_body(const Geom& G, const State& S, const
             for (int jj = 0; jj < kMaxRank / 32; ++jj) {
                 const int j = lane + 32 * jj;
                 if (j < R) {
+                    if (in.dbg) in.dbg[j] = acc[jj];
                     const __nv_bfloat16 cb = __float2bfloat16_rn(acc[jj]);
                     cs[j] = __bfloat162float(cb);
                     *reinterpret_cast<__nv_bfloat16*>(blk + (size_t)(j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2) = cb;

@@ -158,11 +158,21 @@ dwkv_status dwkv_seq_length(dwkv_handle h, int32_t seq, int32_t layer, int32_t* 
  *                    tier is fixed by the first layer of its group that appends it
  *                    ([DW] §3 Eq. (2): rho_{m,h,t} has no layer index); later layers of
  *                    the group reuse it and ignore this array (which may then be NULL).
+ *   coeff_dbg      : NULL, or device fp32 [sum(n_new)][Hkv][2][r_max]: the projection c_j
+ *                    (j < r_t; entries past r_t are not written) that the stored bf16
+ *                    coefficients round, for checking steps 2-6 against a reference fed the
+ *                    same c.  Calls with at most 4 tokens per sequence compute c as an fp32
+ *                    fma chain over i = 0..d-1 from +0 (the fused decode step does too); larger
+ *                    calls compute it on the tensor cores (bf16 products, fp32 accumulation in
+ *                    the tensor core's order), within 1e-5 |x| of the exact projection.
+ * Steps 2-6 (bf16 rounding, the residual against the stored coefficients as an fp32 fma
+ * chain over j from +0, the top-s selection, scale and codes) are the same operations on
+ * every path, so the stored bytes follow from c bit for bit.
  * The positions appended are [len, len + n_new[i]) where len is the sequence's current
  * length at this layer.  Capacity: len + n_new[i] <= max_context. */
 dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
                         const int32_t* n_new, const void* k_new, const void* v_new,
-                        const uint8_t* tier_idx, void* stream);
+                        const uint8_t* tier_idx, float* coeff_dbg, void* stream);
 
 /* Appends tokens that are already in compressed form (import of a prepared cache).
  * Same sequence / position rules as dwkv_append.  Device arrays, tokens in list order,
@@ -213,6 +223,61 @@ dwkv_status dwkv_append_decode_attention(dwkv_handle h, int32_t layer, int32_t n
 dwkv_status dwkv_probe(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
                        const void* q, float* err, float* out_full, void* workspace,
                        size_t ws_bytes, void* stream);
+
+/* Moves stored tokens to other rank tiers ([DW] §3, Eq. (2)-(3) paragraphs: the probe's
+ * feedback lowers or raises the router threshold tau_m of a depth window, which changes the
+ * rank level its tokens are kept at).  For each listed sequence i, its n_tok[i] positions
+ * (device int32 positions[], sequences in list order, distinct within a sequence) and every
+ * kv-head h, the token takes tier new_tier[t][h] (device uint8 [sum(n_tok)][Hkv], an index
+ * into cfg.tiers) in every layer of `group`, keys and values:
+ *   - a token already at its new tier is left as it is;
+ *   - otherwise it is re-encoded at the new rank from its reconstruction (Eq. (1), g = 1),
+ *     since the dense vector is not kept: a_i = fp32 fma chain over j < r_old of
+ *     B[i][j] * c_j from +0, plus scale * code on its residual channels, rounded to bf16,
+ *     then the encode steps of dwkv_append; the stored bytes equal dwkv_append's for that
+ *     bf16 vector.
+ * Every layer of the group must hold the same positions (call between decode steps, not
+ * between the layers of one step); DWKV_ERR_INVALID_ARG otherwise.  Positions the group has
+ * not placed, or tier indices >= num_tiers, set a device error (DWKV_DEV_NO_SLOT,
+ * DWKV_DEV_BAD_TIER) and are skipped.  Decoding after the call sees the new tiers; the
+ * sequence's length is unchanged.  Pages a tier empties return to the pool's free ring. */
+dwkv_status dwkv_retier(dwkv_handle h, int32_t group, int32_t n_seqs, const int32_t* seq_ids,
+                        const int32_t* n_tok, const int32_t* positions, const uint8_t* new_tier,
+                        void* stream);
+
+/* Probe-driven threshold of the router, per depth window ([DW] §3, Eq. (2) and the Eq. (3)
+ * paragraph).  Host code only; it holds no device state.
+ *  - dwkv_tier_controller_due(c, step): 1 when decode step `step` (>= 0) is a probe step
+ *    (every probe_every steps, step 0 included), else 0.
+ *  - dwkv_tier_controller_observe(c, group, err, &lowered): one probe interval's result for
+ *    the group, err = the largest probe error (dwkv_probe) over its layers and kv-heads.  If
+ *    err > tol: tau = max(tau_min, tau - tau_step_down), the quiet count restarts and
+ *    *lowered = 1 (the caller may then promote stored tokens, dwkv_retier).  Otherwise the
+ *    quiet count grows; when it reaches quiet_intervals, tau = min(tau_max, tau + tau_step_up)
+ *    and the count restarts.  NaN err: DWKV_ERR_INVALID_ARG.
+ *  - dwkv_tier_controller_route(c, group, n, salience, base_tier, high_tier, tier_out): the
+ *    router's two-level rule with the group's current threshold, on host arrays of n tokens:
+ *    tier_out[t] = high_tier if salience[t] > tau and base_tier[t] < high_tier, else
+ *    base_tier[t].  The salience scores (the router's sigma(u^T phi)) are the caller's.
+ *  - dwkv_tier_controller_threshold(c, group, &tau): the group's current threshold. */
+typedef struct {
+    float tol;                 /* probe error above which tau is lowered                    */
+    float tau_init, tau_min, tau_max;
+    float tau_step_down, tau_step_up;
+    int32_t quiet_intervals;   /* probes in a row at or below tol before tau rises (>= 1)   */
+    int32_t probe_every;       /* decode steps between probes (>= 1)                        */
+} dwkv_tier_policy;
+typedef struct dwkv_tier_ctrl* dwkv_tier_controller;
+dwkv_status dwkv_tier_controller_create(const dwkv_tier_policy* policy, int32_t num_groups,
+                                        dwkv_tier_controller* out);
+dwkv_status dwkv_tier_controller_destroy(dwkv_tier_controller c);
+int32_t dwkv_tier_controller_due(dwkv_tier_controller c, int64_t step);
+dwkv_status dwkv_tier_controller_threshold(dwkv_tier_controller c, int32_t group, float* tau);
+dwkv_status dwkv_tier_controller_observe(dwkv_tier_controller c, int32_t group, float err,
+                                         int32_t* lowered);
+dwkv_status dwkv_tier_controller_route(dwkv_tier_controller c, int32_t group, int32_t n,
+                                       const float* salience, const uint8_t* base_tier,
+                                       int32_t high_tier, uint8_t* tier_out);
 
 /* Reads positions [t0, t0 + n) of (layer, seq) back in token order, as stored:
  *   tier_idx uint8 [n][Hkv]; coeff bf16 [n][Hkv][2][r_max] (zeros at j >= r_t);

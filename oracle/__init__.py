@@ -43,6 +43,10 @@ def lib():
         L.oracle_quantize_residual.restype = i
         L.oracle_encode_many.argtypes = [i, i, i, p, p, p, i, i, p, p, p, p, p, i]
         L.oracle_encode_many.restype = i
+        L.oracle_encode_many_from_coeffs.argtypes = [i, i, i, p, p, p, p, i, i, p, p, p, p, i]
+        L.oracle_encode_many_from_coeffs.restype = i
+        L.oracle_reencode_vector.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, i, p, p, p, p, p]
+        L.oracle_reencode_vector.restype = i
         L.oracle_reconstruct.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, p]
         L.oracle_reconstruct.restype = None
         for name in ("oracle_f32_to_bf16_rn_many", "oracle_f32_to_fp16_rn_many",
@@ -280,3 +284,45 @@ def encode_many(basis, x, ranks, s, bits, nthreads=None, want_c32=False):
     if want_c32:
         out["c32"] = c32
     return out
+
+
+def reencode_vector(basis, r_old, coeff, idx, codes, scale, r_new, bits):
+    """Re-tier one stored vector: re-encode its bf16-rounded reconstruction at rank r_new
+    (``oracle_reencode_vector``).  Returns the encode dict plus ``xh`` (bf16 bits [d])."""
+    b = _bits16(basis)
+    d, r_max = b.shape
+    c = _bits16(coeff).reshape(r_max)
+    ix = _arr(idx, np.uint8).reshape(-1)
+    cd = _arr(codes, np.int8).reshape(-1)
+    s = ix.size
+    sc = int(_bits16(scale).reshape(-1)[0])
+    out_c = np.zeros(r_max, np.uint16)
+    out_i = np.zeros(s, np.uint8)
+    out_q = np.zeros(s, np.int8)
+    out_s = np.zeros(1, np.uint16)
+    xh = np.zeros(d, np.uint16)
+    rc = lib().oracle_reencode_vector(d, r_max, _p(b), int(r_old), _p(c), s, _p(ix), _p(cd), sc, int(r_new), int(bits),
+                                      _p(out_c), _p(out_i), _p(out_q), _p(out_s), _p(xh))
+    if rc != 0:
+        raise ValueError("oracle_reencode_vector: bad arguments")
+    return {"coeff": out_c, "idx": out_i, "codes": out_q, "scale": out_s[0], "xh": xh}
+
+
+def encode_many_from_coeffs(basis, x, c32, ranks, s, bits, nthreads=None):
+    """Encode steps 2-6 of n vectors [n][d] sharing one basis, from given fp32 projections
+    c32 [n][r_max] (only [:r_t] read): the stored bytes of an encoder that computed c32."""
+    b = _bits16(basis)
+    d, r_max = b.shape
+    xv = _bits16(x).reshape(-1, d)
+    n = xv.shape[0]
+    cv = _arr(c32, np.float32).reshape(n, r_max)
+    rk = _arr(ranks, np.int32).reshape(n)
+    coeff = np.zeros((n, r_max), np.uint16)
+    idx = np.zeros((n, s), np.uint8)
+    codes = np.zeros((n, s), np.int8)
+    scale = np.zeros(n, np.uint16)
+    rc = lib().oracle_encode_many_from_coeffs(n, d, r_max, _p(b), _p(xv), _p(cv), _p(rk), int(s), int(bits), _p(coeff),
+                                              _p(idx), _p(codes), _p(scale), int(nthreads or os.cpu_count() or 1))
+    if rc != 0:
+        raise ValueError("oracle_encode_many_from_coeffs: bad arguments")
+    return {"coeff": coeff, "idx": idx, "codes": codes, "scale": scale}

@@ -276,21 +276,20 @@ int oracle_quantize_residual(int d, int s, int bits, const float* r, uint8_t* id
     return 0;
 }
 
-int oracle_encode_vector(int d, int r_max, const uint16_t* basis, const uint16_t* x, int r_t,
-                         int s, int bits, uint16_t* coeff, float* c32, uint8_t* idx, int8_t* codes,
-                         uint16_t* scale, float* resid) {
+/* Steps 2-6 on a given fp32 projection c (c[j] for j < r_t): what an encoder stores once it
+ * has its coefficients, whatever arithmetic produced them.  Arguments as oracle_encode_vector,
+ * with c32 the input. */
+int oracle_encode_from_coeffs(int d, int r_max, const uint16_t* basis, const uint16_t* x, const float* c32,
+                              int r_t, int s, int bits, uint16_t* coeff, uint8_t* idx, int8_t* codes,
+                              uint16_t* scale, float* resid) {
     if (d <= 0 || d > 256 || r_t < 0 || r_t > r_max || s < 0 || s > d || (bits != 8 && bits != 4))
         return -1;
     float xf[256], cb[256], r[256];
     for (int i = 0; i < d; ++i) xf[i] = (float)oracle_bf16_to_f64(x[i]);
-    for (int j = 0; j < r_max; ++j) { coeff[j] = 0; if (c32) c32[j] = 0.0f; }
-    /* 1-2: projection and bf16 rounding */
+    for (int j = 0; j < r_max; ++j) coeff[j] = 0;
+    /* 2: bf16 rounding of the coefficients kept */
     for (int j = 0; j < r_t; ++j) {
-        float acc = 0.0f;
-        for (int i = 0; i < d; ++i)
-            acc = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), xf[i], acc);
-        if (c32) c32[j] = acc;
-        coeff[j] = oracle_f32_to_bf16_rn(acc);
+        coeff[j] = oracle_f32_to_bf16_rn(c32[j]);
         cb[j] = (float)oracle_bf16_to_f64(coeff[j]);
     }
     /* 3: residual against the stored coefficients */
@@ -305,6 +304,39 @@ int oracle_encode_vector(int d, int r_max, const uint16_t* basis, const uint16_t
     return 0;
 }
 
+int oracle_encode_vector(int d, int r_max, const uint16_t* basis, const uint16_t* x, int r_t,
+                         int s, int bits, uint16_t* coeff, float* c32, uint8_t* idx, int8_t* codes,
+                         uint16_t* scale, float* resid) {
+    if (d <= 0 || d > 256 || r_t < 0 || r_t > r_max || s < 0 || s > d || (bits != 8 && bits != 4))
+        return -1;
+    float xf[256], c[256];
+    for (int i = 0; i < d; ++i) xf[i] = (float)oracle_bf16_to_f64(x[i]);
+    /* 1: projection, an fma chain over i = 0..d-1 from +0 */
+    for (int j = 0; j < r_max; ++j) c[j] = 0.0f;
+    for (int j = 0; j < r_t; ++j) {
+        float acc = 0.0f;
+        for (int i = 0; i < d; ++i)
+            acc = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), xf[i], acc);
+        c[j] = acc;
+    }
+    if (c32) for (int j = 0; j < r_max; ++j) c32[j] = c[j];
+    /* 2-6 */
+    return oracle_encode_from_coeffs(d, r_max, basis, x, c, r_t, s, bits, coeff, idx, codes, scale, resid);
+}
+
+/* Steps 2-6 for many vectors that share one basis, from given projections c32 [n][r_max]. */
+int oracle_encode_many_from_coeffs(int n, int d, int r_max, const uint16_t* basis, const uint16_t* x,
+                                   const float* c32, const int32_t* rank, int s, int bits, uint16_t* coeff,
+                                   uint8_t* idx, int8_t* codes, uint16_t* scale, int nthreads) {
+    int bad = 0;
+#pragma omp parallel for schedule(static) num_threads(nthreads) reduction(| : bad)
+    for (int k = 0; k < n; ++k)
+        bad |= (oracle_encode_from_coeffs(d, r_max, basis, x + (size_t)k * d, c32 + (size_t)k * r_max, rank[k], s,
+                                          bits, coeff + (size_t)k * r_max, idx + (size_t)k * s, codes + (size_t)k * s,
+                                          scale + k, NULL) != 0);
+    return bad ? -1 : 0;
+}
+
 /* Encode many vectors that share one basis (token-ordered): x [n][d], rank [n]. */
 int oracle_encode_many(int n, int d, int r_max, const uint16_t* basis, const uint16_t* x,
                        const int32_t* rank, int s, int bits, uint16_t* coeff, float* c32,
@@ -316,6 +348,45 @@ int oracle_encode_many(int n, int d, int r_max, const uint16_t* basis, const uin
                                      coeff + (size_t)k * r_max, c32 ? c32 + (size_t)k * r_max : NULL,
                                      idx + (size_t)k * s, codes + (size_t)k * s, scale + k, NULL) != 0);
     return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Re-tiering a stored vector ([DW] §3, Eq. (2)-(3) paragraphs: the probe feedback lowers   */
+/* the router threshold, so tokens move to another rank tier).  The dense vector is not     */
+/* kept, so the token is re-encoded from its reconstruction (Eq. (1), g = 1), rounded to    */
+/* bf16 like any input vector, at the new rank:                                            */
+/*   a_i  = fma chain over j = 0..r_old-1 of B[i][j] * cb_j from +0      (fp32)            */
+/*   xh_i = bf16_rn(a_i + scale * code_i) for the stored residual channels, bf16_rn(a_i)    */
+/*          for the others (scale * code is exact in fp32; one rounding in the add)         */
+/* then the six encode steps of oracle_encode_vector on xh at rank r_new.                  */
+/* Inputs: the stored coeff (bf16 [r_max], entries >= r_old ignored), idx / codes [s],      */
+/* scale (fp16 bits).  Outputs as oracle_encode_vector; xh_out (nullable) bf16 bits [d].    */
+/* ------------------------------------------------------------------------------------ */
+int oracle_reencode_vector(int d, int r_max, const uint16_t* basis, int r_old, const uint16_t* coeff_old,
+                           int s, const uint8_t* idx_old, const int8_t* codes_old, uint16_t scale_old,
+                           int r_new, int bits, uint16_t* coeff, uint8_t* idx, int8_t* codes,
+                           uint16_t* scale, uint16_t* xh_out) {
+    if (d <= 0 || d > 256 || r_old < 0 || r_old > r_max || r_new < 0 || r_new > r_max || s < 0 || s > d)
+        return -1;
+    float a[256];
+    uint16_t xh[256];
+    for (int i = 0; i < d; ++i) {
+        float acc = 0.0f;
+        for (int j = 0; j < r_old; ++j)
+            acc = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), (float)oracle_bf16_to_f64(coeff_old[j]),
+                       acc);
+        a[i] = acc;
+    }
+    const float sf = (float)oracle_fp16_to_f64(scale_old);
+    for (int k = 0; k < s; ++k) {
+        if (idx_old[k] >= d) return -1;
+        a[idx_old[k]] = a[idx_old[k]] + sf * (float)codes_old[k];
+    }
+    for (int i = 0; i < d; ++i) {
+        xh[i] = oracle_f32_to_bf16_rn(a[i]);
+        if (xh_out) xh_out[i] = xh[i];
+    }
+    return oracle_encode_vector(d, r_max, basis, xh, r_new, s, bits, coeff, NULL, idx, codes, scale, NULL);
 }
 
 /* Element-wise format conversions over arrays (used to pin the converters). */

@@ -115,9 +115,11 @@ def check_close(got, ref, max_abs=2e-3, rel=1e-3, what=""):
     return ma, rl
 
 
-def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None) -> dict:
+def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None, c32=None) -> dict:
     """The oracle's encoding of dense rows k, v (bf16 [n][Hkv][d]) at their tiers, in the
-    token-ordered compressed format of ``synth.make_compressed`` (CPU tensors)."""
+    token-ordered compressed format of ``synth.make_compressed`` (CPU tensors).  With ``c32``
+    (fp32 [n][Hkv][2][r_max], an encoder's exported projection) the oracle runs encode steps
+    2-6 on those coefficients instead of its own step 1."""
     g = layer // wl.layers_per_group
     k, v, tier_idx = k.cpu(), v.cpu(), tier_idx.cpu()
     n, H, s = k.shape[0], wl.num_kv_heads, wl.resid_channels
@@ -126,9 +128,15 @@ def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None) -> dict:
     idx = np.zeros((n, H, 2, s), np.uint8)
     codes = np.zeros((n, H, 2, s), np.int8)
     scales = np.zeros((n, H, 2), np.uint16)
+    if c32 is not None:
+        c32 = np.nan_to_num(np.asarray(c32.cpu() if hasattr(c32, "cpu") else c32, np.float32))
     for h in range(H):
         for z, x in enumerate((k, v)):
-            r = oracle.encode_many(bases[z][g, h], x[:, h], ranks[:, h], s, wl.resid_bits, nthreads=nthreads)
+            if c32 is not None:
+                r = oracle.encode_many_from_coeffs(bases[z][g, h], x[:, h], c32[:, h, z], ranks[:, h], s, wl.resid_bits,
+                                                   nthreads=nthreads)
+            else:
+                r = oracle.encode_many(bases[z][g, h], x[:, h], ranks[:, h], s, wl.resid_bits, nthreads=nthreads)
             coeff[:, h, z], idx[:, h, z], codes[:, h, z], scales[:, h, z] = r["coeff"], r["idx"], r["codes"], r["scale"]
     return {"coeff": torch.from_numpy(coeff.view(np.int16)).view(torch.bfloat16),
             "idx": torch.from_numpy(idx), "codes": torch.from_numpy(codes),

@@ -60,7 +60,8 @@ def test_token_and_page_bytes():
     assert [dw.dwkv_token_bytes(cfg, k) for k in range(3)] == [2 * (2 * r + 16 + 8 + 2) for r in (16, 32, 64)]
     assert dw.dwkv_token_bytes(cfg, 3) == 0
     for k, r in enumerate((16, 32, 64)):
-        assert dw.dwkv_page_bytes(cfg, k) == 2 * 2 * (128 * r + 64 * 16 + 8 * 16 * 4 + 128)
+        # two layers x (K + V) blocks, then the 64 slots' positions (int32)
+        assert dw.dwkv_page_bytes(cfg, k) == 2 * 2 * (128 * r + 64 * 16 + 8 * 16 * 4 + 128) + 64 * 4
         assert dw.dwkv_page_bytes(cfg, k) % 128 == 0
     meta = dw.dwkv_metadata_bytes(cfg)
     assert 0 < meta < dw.dwkv_arena_bytes(cfg)
@@ -87,7 +88,7 @@ def test_null_handle_calls_fail_cleanly():
     assert L.dwkv_destroy(None) == 1
     assert L.dwkv_sync_status(None, None) == 1
     assert L.dwkv_decode_attention(None, 0, 0, None, None, None, None, 0, None) == 1
-    assert L.dwkv_append(None, 0, 0, None, None, None, None, None, None) == 1
+    assert L.dwkv_append(None, 0, 0, None, None, None, None, None, None, None) == 1
 
 
 def test_product_package_never_imports_the_oracle():

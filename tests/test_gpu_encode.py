@@ -1,7 +1,10 @@
 """GPU encode/append (through the C ABI) against the oracle's encoder, bit for bit:
 stored bf16 coefficients, channel indices, integer codes and fp16 scales, plus the
-tier each token was placed in.  Then decode over an encoded cache against the oracle
-decoding the oracle's own encoding."""
+tier each token was placed in.  Appends of up to 4 tokens per sequence project with the
+fp32 fma chain the oracle runs, so their bytes and exported projections equal the oracle's
+own; larger appends project on the tensor cores, so their projection is checked against the
+fp64 projection (within 1e-5 |x|) and their bytes against the oracle's steps 2-6 on the
+exported projection.  Then decode over an encoded cache against the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -24,10 +27,30 @@ def _assert_same(got: dict, ref: dict, tiers, what=""):
     assert torch.equal(got["scales"].cpu().view(torch.int16), ref["scales"].view(torch.int16)), what + " scales"
 
 
+def _check_projection(wl, bases, layer, k, v, tiers, c32, what=""):
+    """The exported fp32 projection against the fp64 one (numpy matmul of the exact bf16
+    values), within 1e-5 |x| for every kept coefficient."""
+    g = layer // wl.layers_per_group
+    ranks = synth.ranks_of(wl, tiers.cpu()).numpy()
+    c32 = np.asarray(c32.cpu(), np.float64)
+    for z, x in enumerate((k, v)):
+        xf = x.cpu().to(torch.float64).numpy()                     # [n][H][d]
+        for h in range(wl.num_kv_heads):
+            Bm = bases[z][g, h].to(torch.float64).numpy()            # [d][r_max]
+            exact = xf[:, h] @ Bm                                    # [n][r_max]
+            keep = np.arange(wl.r_max)[None, :] < ranks[:, h][:, None]
+            err = np.abs(np.where(keep, c32[:, h, z] - exact, 0.0)).max(axis=1)
+            assert np.all(err <= 1e-5 * np.linalg.norm(xf[:, h], axis=1) + 1e-30), what
+
+
 def _encode_case(wl, lengths, chunks=(None,), gen_device="cpu"):
+    """Appends the dense rows in chunks; returns the cache, the bases, the inputs and, per
+    (sequence, layer), the projection each row's append exported (fp32 [T][H][2][r_max])."""
     bases = synth.make_bases(wl)
     cache = dw.Cache(cfg_for(wl, max_batch=len(lengths), max_context=max(lengths) + 8), bases[0], bases[1])
     dense = {}
+    c32 = {(b, layer): torch.full((T, wl.num_kv_heads, 2, wl.r_max), float("nan"))
+           for b, T in enumerate(lengths) for layer in range(wl.num_layers)}
     for b, T in enumerate(lengths):
         for layer in range(wl.num_layers):
             dense[(b, layer)] = synth.make_dense_vectors(wl, b, layer, T, bases, device=gen_device)
@@ -52,10 +75,17 @@ def _encode_case(wl, lengths, chunks=(None,), gen_device="cpu"):
                     ts.append(dense[(b, "t", g)][a:e])
             if seqs:
                 lay0 = layer % wl.layers_per_group == 0
+                dbg = torch.full((sum(ns), wl.num_kv_heads, 2, wl.r_max), float("nan"), device="cuda")
                 cache.append(layer, seqs, ns, torch.cat(ks).cuda(), torch.cat(vs).cuda(),
-                             torch.cat(ts).cuda() if lay0 else None)
+                             torch.cat(ts).cuda() if lay0 else None, coeff_dbg=dbg)
+                dbg = dbg.cpu()
+                o = 0
+                for b, n_ in zip(seqs, ns):
+                    a = bounds[b][step]
+                    c32[(b, layer)][a:a + n_] = dbg[o:o + n_]
+                    o += n_
     cache.sync()
-    return cache, bases, dense
+    return cache, bases, dense, c32
 
 
 @pytest.mark.parametrize("name", ["llama8b_encode_16k", "llama8b_ragged_b8", "llama8b_131k_deep", "tiny_1k"])
@@ -65,25 +95,43 @@ def test_encode_bit_exact(name):
     wl = wl.scaled(num_layers=lpg, num_q_heads=8 if wl.num_kv_heads > 1 else 4,
                    num_kv_heads=2 if wl.num_kv_heads > 1 else 1, batch=2)
     lengths = [300, 77]
-    cache, bases, dense = _encode_case(wl, lengths)
+    cache, bases, dense, c32 = _encode_case(wl, lengths)
     for b, T in enumerate(lengths):
         for layer in range(wl.num_layers):
             got = cache.export(layer, b, 0, T)
             tiers = dense[(b, "t", layer // lpg)]
-            ref = oracle_encode_rows(wl, bases, layer, dense[(b, layer)][0], dense[(b, layer)][1], tiers)
+            k, v = dense[(b, layer)]
+            _check_projection(wl, bases, layer, k, v, tiers, c32[(b, layer)], f"{name} seq {b} layer {layer}")
+            ref = oracle_encode_rows(wl, bases, layer, k, v, tiers, c32=c32[(b, layer)])
             _assert_same(got, ref, tiers, f"{name} seq {b} layer {layer}")
 
 
-def test_chunked_appends_equal_one_shot():
+def test_chunked_appends_bit_exact_on_both_paths():
+    """Chunks of 1 and 4 tokens take the fp32-chain path (bytes and projection equal the
+    oracle's own), the others the tensor-core path (bytes equal the oracle's steps 2-6 on the
+    exported projection)."""
     wl = synth.workload("llama8b_encode_16k").scaled(num_layers=2, num_q_heads=8, num_kv_heads=2, batch=2)
     lengths = [200, 131]
-    c1, bases, dense = _encode_case(wl, lengths)
-    c2, _, _ = _encode_case(wl, lengths, chunks=(1, 1, 37, 64, 5, None))
+    chunks = (1, 1, 37, 4, 64, 5, None)
+    cache, bases, dense, c32 = _encode_case(wl, lengths, chunks=chunks)
     for b, T in enumerate(lengths):
+        small = np.zeros(T, bool)
+        a = 0
+        for c in chunks:
+            e = T if c is None else min(T, a + c)
+            if c is not None and c <= 4:
+                small[a:e] = True
+            a = e
         for layer in range(2):
-            x, y = c1.export(layer, b, 0, T), c2.export(layer, b, 0, T)
-            for key in x:
-                assert torch.equal(x[key].view(torch.uint8), y[key].view(torch.uint8)), key
+            got = cache.export(layer, b, 0, T)
+            tiers = dense[(b, "t", 0)]
+            k, v = dense[(b, layer)]
+            _check_projection(wl, bases, layer, k, v, tiers, c32[(b, layer)], f"seq {b} layer {layer}")
+            _assert_same(got, oracle_encode_rows(wl, bases, layer, k, v, tiers, c32=c32[(b, layer)]), tiers,
+                         f"seq {b} layer {layer}")
+            own = oracle_encode_rows(wl, bases, layer, k[small], v[small], tiers[small])
+            _assert_same({key: val.cpu()[torch.from_numpy(small)] for key, val in got.items()}, own, tiers[small],
+                         f"chain rows seq {b} layer {layer}")
 
 
 def test_decode_sized_appends_bit_exact():
@@ -91,13 +139,23 @@ def test_decode_sized_appends_bit_exact():
     bytes must equal the oracle's for every row, with sequences joining and leaving calls."""
     wl = synth.workload("llama8b_ragged_b8").scaled(num_layers=2, num_q_heads=8, num_kv_heads=2, batch=3)
     lengths = [23, 9, 30]
-    cache, bases, dense = _encode_case(wl, lengths, chunks=(1, 4, 2, 3, 1, 4, 4, 4, None))
+    cache, bases, dense, c32 = _encode_case(wl, lengths, chunks=(1, 4, 2, 3, 1, 4, 4, 4, 4, 4))
+    g = 0
     for b, T in enumerate(lengths):
         for layer in range(wl.num_layers):
             got = cache.export(layer, b, 0, T)
             tiers = dense[(b, "t", layer // wl.layers_per_group)]
             ref = oracle_encode_rows(wl, bases, layer, dense[(b, layer)][0], dense[(b, layer)][1], tiers)
             _assert_same(got, ref, tiers, f"small appends seq {b} layer {layer}")
+            # the exported projection is the oracle's fp32 chain, bit for bit
+            ranks = synth.ranks_of(wl, tiers.cpu())
+            for h in range(wl.num_kv_heads):
+                for z in range(2):
+                    x = dense[(b, layer)][z][:, h]
+                    for t in range(T):
+                        r = int(ranks[t, h])
+                        own = oracle.encode_vector(bases[z][g, h], x[t], r, wl.resid_channels, wl.resid_bits)["c32"]
+                        assert np.array_equal(c32[(b, layer)][t, h, z, :r].numpy(), own[:r]), (b, layer, t, h, z)
 
 
 def test_exact_planted_vectors_and_zero_vectors():
@@ -123,8 +181,8 @@ def test_exact_planted_vectors_and_zero_vectors():
         x[t, 0, ch] = torch.randint(-7, 8, (5,), generator=g).float() * 2.0 ** -6
     k = x.to(torch.bfloat16)
     v = (x * 0.5).to(torch.bfloat16)
-    cache.append(0, [0], [n], k.cuda(), v.cuda(), tiers.cuda())
-    cache.append(1, [0], [n], v.cuda(), k.cuda(), None)
+    cache.append(0, [0], [n], k.cuda(), v.cuda(), tiers.cuda())          # tensor-core projection:
+    cache.append(1, [0], [n], v.cuda(), k.cuda(), None)                  # one nonzero term, exact
     cache.sync()
     for layer, (kk, vv) in enumerate(((k, v), (v, k))):
         got = cache.export(layer, 0, 0, n)
@@ -154,8 +212,10 @@ def test_encode_full_size_sampled():
                 tiers[b] = synth.make_tiers(wl, b, 0, n, device="cuda")
             ts.append(tiers[b])
             dense[(b, layer)] = (k, v)
+        dbg = torch.full((wl.batch * n, wl.num_kv_heads, 2, wl.r_max), float("nan"), device="cuda")
         cache.append(layer, list(range(wl.batch)), [n] * wl.batch, torch.cat(ks), torch.cat(vs),
-                     torch.cat(ts) if layer == 0 else None)
+                     torch.cat(ts) if layer == 0 else None, coeff_dbg=dbg)
+        dense[("dbg", layer)] = dbg.cpu()
     cache.sync()
     sel = torch.randperm(n, generator=torch.Generator().manual_seed(1))[:512].sort().values
     for b in (0, 3):
@@ -163,14 +223,16 @@ def test_encode_full_size_sampled():
             got = cache.export(layer, b, 0, n)
             got = {key: val.cpu()[sel] for key, val in got.items()}
             k, v = dense[(b, layer)]
-            ref = oracle_encode_rows(wl, bases, layer, k.cpu()[sel], v.cpu()[sel], tiers[b].cpu()[sel])
+            c = dense[("dbg", layer)][b * n:(b + 1) * n][sel]
+            _check_projection(wl, bases, layer, k.cpu()[sel], v.cpu()[sel], tiers[b].cpu()[sel], c, f"full seq {b}")
+            ref = oracle_encode_rows(wl, bases, layer, k.cpu()[sel], v.cpu()[sel], tiers[b].cpu()[sel], c32=c)
             _assert_same(got, ref, tiers[b].cpu()[sel], f"full seq {b} layer {layer}")
 
 
 def test_decode_over_encoded_cache():
     wl = synth.workload("llama8b_encode_16k").scaled(num_layers=2, num_q_heads=8, num_kv_heads=2, batch=2)
     lengths = [900, 257]
-    cache, bases, dense = _encode_case(wl, lengths, chunks=(500, None))
+    cache, bases, dense, c32 = _encode_case(wl, lengths, chunks=(500, None))
     q = synth.make_queries(wl, 1, batch=2, temperature=8.0)
     out = cache.decode(1, [0, 1], q.cuda())
     err = cache.probe(1, [0, 1], q.cuda())
@@ -178,7 +240,7 @@ def test_decode_over_encoded_cache():
     out, err = out.cpu().numpy(), err.cpu().numpy()
     for b in range(2):
         tiers = dense[(b, "t", 0)]
-        comp = oracle_encode_rows(wl, bases, 1, dense[(b, 1)][0], dense[(b, 1)][1], tiers)
+        comp = oracle_encode_rows(wl, bases, 1, dense[(b, 1)][0], dense[(b, 1)][1], tiers, c32=c32[(b, 1)])
         for h in range(2):
             prob = head_problem(wl, bases, tiers, comp, q[b], 1, h)
             check_close(out[b, h * 4:(h + 1) * 4], oracle.decode_head(prob), what=f"seq {b} head {h}")
@@ -268,10 +330,11 @@ def test_encode_bit_exact_residual_counts(s, bits):
     wl = synth.workload("tiny_1k").scaled(resid_channels=s, resid_bits=bits, num_q_heads=8, num_kv_heads=2,
                                           batch=2)
     lengths = [300, 77]
-    cache, bases, dense = _encode_case(wl, lengths)
+    cache, bases, dense, c32 = _encode_case(wl, lengths)
     for b, T in enumerate(lengths):
         for layer in range(wl.num_layers):
             got = cache.export(layer, b, 0, T)
             tiers = dense[(b, "t", layer // wl.layers_per_group)]
-            ref = oracle_encode_rows(wl, bases, layer, dense[(b, layer)][0], dense[(b, layer)][1], tiers)
+            ref = oracle_encode_rows(wl, bases, layer, dense[(b, layer)][0], dense[(b, layer)][1], tiers,
+                                     c32=c32[(b, layer)])
             _assert_same(got, ref, tiers, f"s={s} bits={bits} seq {b} layer {layer}")
