@@ -7,27 +7,37 @@ bases r_max = 64 per (group, kv-head, K/V); tiers {16, 32, 64} with probabilitie
 0.6 / 0.3 / 0.1; residual s = 16 int4 channels with an fp16 scale.  The cache holds
 65535 compressed tokens (synthetic, seeded, imported before timing).  One step = for
 each of the 32 layers one launch of dwkv_append_decode_attention: encode + append the
-step's new token, then fused decode attention over the whole context.  Metric: decode
-tokens/s (batch / step time) and the compressed-KV bytes/s of the decode kernel against
-the measured HBM copy bandwidth.  Attention only (no projections / MLP: no weights exist).
+step's new token of every sequence, then fused decode attention over each whole context.
+Metric: decode tokens/s (batch / step time) and the compressed-KV bytes/s of the decode
+kernel against the measured HBM copy bandwidth.  Attention only (no projections / MLP: no
+weights exist).  ``--workload llama8b_ragged_b8`` (8 sequences of 16K-32K tokens, int8) and
+``--workload llama8b_131k_deep`` (131072 tokens, 4-layer groups, r_max 128) run the same
+step on the other decode workloads.
 
 Timing: W warm-up steps, then K steps captured in one CUDA graph and replayed once,
 bracketed by a barrier + synchronize, timed with CUDA events; max over ranks.  Each
-step streams ~2.6 GB of pages (> 126 MB L2), so no L2 flush is needed.  Every launch
-in the timed region is the fused decode kernel, so its average launch duration is the
-region's time over its launches (the roofline); a second replay with an external event
-around every launch is reported beside it.  The probe (dwkv_probe, one launch per layer)
-is timed over the same cache after the steps.  ``e2e`` repeats the step with host
-(pinned) inputs copied in (one block a step) and the outputs copied out inside the timed
-region.  ``step_distribution`` gives the median / p90 of up to 50 steps timed one by one
-(an event node between steps) and the eager (no graph) time of a step.
+step streams GBs of pages (> 126 MB L2), so no L2 flush is needed.  Every launch in the
+timed region is the fused decode kernel, so its average launch duration is the region's
+time over its launches (the roofline); a second replay with an external event around every
+launch is reported beside it.  Decode launches overlap their predecessor (programmatic
+dependent launch) unless ``--no-overlap``.  The probe (dwkv_probe, one launch per layer) is
+timed over the same cache after the steps.  ``e2e`` repeats the step with host (pinned)
+inputs copied in (one block a step) and the outputs copied out inside the timed region.
+``step_distribution`` gives the median / p90 of up to 50 steps timed one by one (an event
+node between steps) and the eager (no graph) time of a step.  Clocks: nvidia-smi every 20 ms
+and NVML every ~1 ms during the timed region.
+
+The default single-GPU run also measures, in fewer steps, the ragged batch-8 and 131K
+workloads and the bulk encode (below), each with its own roofline, e2e and CPU baseline,
+under ``workloads`` in the same JSON line (``--headline-only`` skips them).
 
 ``--workload llama8b_encode_16k`` measures bulk encode instead: 4 sequences x 16384 new
 dense tokens per layer through dwkv_append (32 layers a step, the sequences reset between
 steps), then one decode step and one probe pass over the encoded cache.
 
-``--impl reference`` times the CPU oracle (plain fp64 C, all host cores) on a bounded
-sample of the same workload and reports the same metric.
+``cpu_baseline`` / ``--impl reference``: the CPU oracle (plain fp64 C) on every host core,
+OpenMP over (layer, kv-head) problems of sequence 0 at its full context (at least one problem
+per core), scaled to the whole step.
 
 Multi-GPU (torchrun): every rank runs an independent replica (the path shards by
 sequence with no exchange); value = total tokens of all ranks / max-over-ranks time.

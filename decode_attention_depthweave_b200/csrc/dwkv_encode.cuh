@@ -129,7 +129,7 @@ struct UnitIn {
     Dest dst;
     float xr[4];
     bool ok;
-    float* dbg;      // nullable: the unit's fp32 projection c[j], j < r_t (coefficient export)
+    float* dbg = nullptr;   // the unit's fp32 projection c[j], j < r_t (coefficient export), or none
 };
 
 // Step 4 by its definition: s rounds of "largest remaining |r|, ties to the lower channel"

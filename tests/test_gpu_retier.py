@@ -27,6 +27,9 @@ def _expected_after(wl, bases, data, moves):
         g = layer // wl.layers_per_group
         c = {k: v.clone().cpu() for k, v in comp.items()}
         t = tiers.clone().cpu()
+        # the cache stores (and exports) +0 past each token's rank, whatever the input held there
+        keep = torch.arange(wl.r_max).view(1, 1, 1, -1) < synth.ranks_of(wl, t).view(t.shape[0], -1, 1, 1)
+        c["coeff"] = torch.where(keep, c["coeff"], torch.zeros_like(c["coeff"]))
         if b in moves:
             pos, nt = moves[b]
             for n, p in enumerate(pos.tolist()):
@@ -36,6 +39,7 @@ def _expected_after(wl, bases, data, moves):
                     if k_old == k_new:
                         continue
                     for z in range(2):
+                        c["coeff"][p, h, z] = 0
                         r = oracle.reencode_vector(bases[z][g, h], wl.tiers[k_old], comp["coeff"][p, h, z],
                                                    comp["idx"][p, h, z], comp["codes"][p, h, z], comp["scales"][p, h, z],
                                                    wl.tiers[k_new], wl.resid_bits)
