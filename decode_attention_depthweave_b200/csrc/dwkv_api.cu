@@ -31,8 +31,8 @@ __global__ void export_kernel(const Geom, const State, int, int, int, int, uint8
                               int8_t*, __half*);
 __global__ void reset_kernel(const Geom, const State, int);
 template <int BITS>
-__global__ void retier_kernel(const Geom, const State, const AppendCall, const int32_t*, const uint8_t*);
-__global__ void retier_release_kernel(const Geom, const State, const AppendCall);
+__global__ void retier_kernel(const Geom, const State, const RetierCall, const int32_t*, const uint8_t*);
+__global__ void retier_release_kernel(const Geom, const State, const RetierCall);
 __global__ void wait_timeout_kernel(const State, uint64_t);
 template <int BITS, bool PROBE, int RMAX, int S>
 __global__ void decode_kernel(const Geom, const State, const DecodeCall);
@@ -218,6 +218,9 @@ struct dwkv_ctx {
     int dec_tok_weight = 1024;      // split balance: byte-equivalent cost of one token
     int dec_owner_share = 160;      // fused append: the encoding CTA's share of a split, of 256
     int dec_overlap = 1;            // launch decodes with programmatic stream serialisation
+    // The last launch on the handle when it was a fused decode step (else layer -1): a decode
+    // launched right after it may start while it runs, and must not read early what it writes.
+    int last_fused_layer = -1, last_fused_placed = 0;
 };
 
 namespace {
@@ -226,6 +229,10 @@ dwkv_status check_handle(dwkv_handle h) {
     if (!h) return fail(DWKV_ERR_INVALID_ARG, "handle is NULL");
     return DWKV_OK;
 }
+
+// A launch without programmatic serialisation starts after everything before it on the
+// stream has completed, so the next decode may read the cache early again.
+void note_plain_launch(dwkv_handle h) { h->last_fused_layer = -1; }
 
 dwkv_status check_layer(dwkv_handle h, int32_t layer) {
     if (layer < 0 || layer >= h->geom.L)
@@ -526,6 +533,7 @@ dwkv_status dwkv_reset_sequence(dwkv_handle h, int32_t seq, void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     reset_kernel<<<1, 256, 0, s>>>(G, h->st, seq);
     DWKV_CUDA(cudaGetLastError(), "reset_kernel launch");
+    note_plain_launch(h);
     DWKV_CUDA(cudaMemsetAsync(h->st.slot_map + slot_index(G, seq, 0, 0, 0), 0,
                               (size_t)4 * G.G * G.Hkv * G.max_context, s),
               "cudaMemsetAsync(slot map)");
@@ -566,12 +574,14 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
                                                          static_cast<const __nv_bfloat16*>(k_new),
                                                          static_cast<const __nv_bfloat16*>(v_new), coeff_dbg);
         DWKV_CUDA(cudaGetLastError(), "append_small_kernel launch");
+        note_plain_launch(h);
         commit_call(h, C, n_new);
         return DWKV_OK;
     }
     if (any) {
         place_kernel<<<dim3(C.n, G.Hkv), 256, 0, s>>>(G, h->st, C, tier_idx);
         DWKV_CUDA(cudaGetLastError(), "place_kernel launch");
+        note_plain_launch(h);
     }
     // a block per (kv-head, K or V) and share of the tiles, one wave of resident blocks
     const long long ntiles = (C.total + kEncTile - 1) / kEncTile;
@@ -585,6 +595,7 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
         encode_kernel<4><<<grid, 256, tsm, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(k_new),
                                                  static_cast<const __nv_bfloat16*>(v_new), coeff_dbg);
     DWKV_CUDA(cudaGetLastError(), "encode_kernel launch");
+    note_plain_launch(h);
     commit_call(h, C, n_new);
     return DWKV_OK;
 }
@@ -606,6 +617,7 @@ dwkv_status dwkv_append_compressed(dwkv_handle h, int32_t layer, int32_t n_seqs,
     if (any) {
         place_kernel<<<dim3(C.n, G.Hkv), 256, 0, s>>>(G, h->st, C, tier_idx);
         DWKV_CUDA(cudaGetLastError(), "place_kernel launch");
+        note_plain_launch(h);
     }
     const dim3 grid(grid_rows(h, C.total), G.Hkv);
     if (G.bits == 8)
@@ -615,6 +627,7 @@ dwkv_status dwkv_append_compressed(dwkv_handle h, int32_t layer, int32_t n_seqs,
         import_kernel<4><<<grid, 256, 0, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(coeff), idx, codes,
                                               static_cast<const __half*>(scales));
     DWKV_CUDA(cudaGetLastError(), "import_kernel launch");
+    note_plain_launch(h);
     commit_call(h, C, n_new);
     return DWKV_OK;
 }
@@ -731,8 +744,15 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     for (int i = 0; i < n_seqs; ++i) {
         C.seq[i] = seq_ids[i];
         C.split_begin[i] = total;
-        C.expect[i] = h->len[(size_t)seq_ids[i] * G.L + layer];   // positions the group has placed
         total += sp[i];
+    }
+    // cache state written by the previous launch, if that was a fused step of this group: a
+    // placing launch adds its token's count at its end; every fused launch writes its token's
+    // bytes of its layer
+    {
+        const int pl = h->last_fused_layer;
+        const bool same_group = pl >= 0 && pl / G.LPG == g;
+        C.early = (same_group && (h->last_fused_placed || pl == layer)) ? 0 : 1;
     }
     C.split_begin[n_seqs] = total;
     C.total_splits = total;
@@ -749,8 +769,6 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
         for (int i = 0; i < n_seqs; ++i) {
             C.pos[i] = fa->call->pos0[i];
             C.place[i] = fa->call->na[i] > 0 ? 1 : 0;
-            // the placing launch counts its token only at its end; a later layer finds it counted
-            C.expect[i] = C.place[i] ? C.pos[i] : C.pos[i] + 1;
         }
     }
     C.q = static_cast<const __nv_bfloat16*>(q);
@@ -786,6 +804,10 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
 #undef DWKV_LAUNCH
     if (lerr != cudaSuccess) return cuda_fail(lerr, probe ? "probe kernel launch" : "decode kernel launch");
     DWKV_CUDA(cudaGetLastError(), probe ? "probe kernel launch" : "decode kernel launch");
+    h->last_fused_layer = fa ? layer : -1;
+    h->last_fused_placed = 0;
+    if (fa)
+        for (int i = 0; i < n_seqs; ++i) h->last_fused_placed |= C.place[i];
     return DWKV_OK;
 }
 
@@ -838,12 +860,7 @@ dwkv_status dwkv_retier(dwkv_handle h, int32_t group, int32_t n_seqs, const int3
     if (group < 0 || group >= G.G) return fail(DWKV_ERR_INVALID_ARG, "group %d out of [0, %d)", group, G.G);
     if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
     if (n_seqs && !n_tok) return fail(DWKV_ERR_INVALID_ARG, "n_tok is NULL");
-    AppendCall C;
-    memset(&C, 0, sizeof(C));
-    C.n = n_seqs;
-    C.g = group;
-    C.layer = group * G.LPG;
-    long long total = 0;
+    std::vector<int> first(n_seqs + 1, 0);
     for (int i = 0; i < n_seqs; ++i) {
         const int s = seq_ids[i];
         const int pl = h->placed[(size_t)s * G.G + group];
@@ -854,22 +871,35 @@ dwkv_status dwkv_retier(dwkv_handle h, int32_t group, int32_t n_seqs, const int3
                             s, l, h->len[(size_t)s * G.L + l], pl);
         if (n_tok[i] < 0 || n_tok[i] > pl)
             return fail(DWKV_ERR_INVALID_ARG, "n_tok[%d] = %d out of [0, %d]", i, n_tok[i], pl);
-        C.seq[i] = s;
-        C.tok0[i] = (int)total;
-        total += n_tok[i];
+        first[i + 1] = first[i] + n_tok[i];
     }
-    C.tok0[n_seqs] = (int)total;
-    C.total = (int)total;
-    if (total == 0) return DWKV_OK;
+    if (first[n_seqs] == 0) return DWKV_OK;
     if (!positions || !new_tier) return fail(DWKV_ERR_INVALID_ARG, "positions and new_tier must be non-NULL");
+    // Rounds of at most one page of tokens per sequence, each followed by the release of the
+    // pages the moves emptied: a round needs at most a page or two more per tier than the
+    // tokens it moves, so a cache sized by dwkv_arena_bytes has room for any number of moves.
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const dim3 grid(n_seqs, G.Hkv);
     const size_t sm = encode_smem(G);
-    if (G.bits == 8) retier_kernel<8><<<grid, 256, sm, s>>>(G, h->st, C, positions, new_tier);
-    else retier_kernel<4><<<grid, 256, sm, s>>>(G, h->st, C, positions, new_tier);
-    DWKV_CUDA(cudaGetLastError(), "retier_kernel launch");
-    retier_release_kernel<<<1, 256, 0, s>>>(G, h->st, C);
-    DWKV_CUDA(cudaGetLastError(), "retier_release_kernel launch");
+    for (int r0 = 0;; r0 += kPage) {
+        RetierCall C;
+        memset(&C, 0, sizeof(C));
+        C.g = group;
+        for (int i = 0; i < n_seqs; ++i) {
+            if (n_tok[i] <= r0) continue;
+            C.seq[C.n] = seq_ids[i];
+            C.begin[C.n] = first[i] + r0;
+            C.end[C.n] = first[i] + std::min(n_tok[i], r0 + kPage);
+            ++C.n;
+        }
+        if (C.n == 0) break;
+        const dim3 grid(C.n, G.Hkv);
+        if (G.bits == 8) retier_kernel<8><<<grid, 256, sm, s>>>(G, h->st, C, positions, new_tier);
+        else retier_kernel<4><<<grid, 256, sm, s>>>(G, h->st, C, positions, new_tier);
+        DWKV_CUDA(cudaGetLastError(), "retier_kernel launch");
+        retier_release_kernel<<<1, 256, 0, s>>>(G, h->st, C);
+        DWKV_CUDA(cudaGetLastError(), "retier_release_kernel launch");
+    }
+    note_plain_launch(h);
     return DWKV_OK;
 }
 
@@ -893,6 +923,7 @@ dwkv_status dwkv_export(dwkv_handle h, int32_t layer, int32_t seq, int32_t t0, i
         export_kernel<4><<<grid, 256, 0, s>>>(G, h->st, layer, seq, t0, n, tier_idx,
                                               static_cast<__nv_bfloat16*>(coeff), idx, codes, static_cast<__half*>(scales));
     DWKV_CUDA(cudaGetLastError(), "export_kernel launch");
+    note_plain_launch(h);
     return DWKV_OK;
 }
 
@@ -938,6 +969,7 @@ dwkv_status dwkv_check_bounded_wait(dwkv_handle h, uint32_t limit_us, void* stre
         return fail(DWKV_ERR_INVALID_ARG, "limit_us = %u must be in 1..2000000", limit_us);
     wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(h->st, (uint64_t)limit_us * 1000ull);
     DWKV_CUDA(cudaGetLastError(), "wait_timeout_kernel launch");
+    note_plain_launch(h);
     return DWKV_OK;
 }
 

@@ -671,7 +671,7 @@ __global__ void __launch_bounds__(256) reset_kernel(const Geom G, const State S,
 // tier empties stays with the tier (owned) until retier_release_kernel returns it.
 // ------------------------------------------------------------------------------------
 template <int BITS>
-__global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S, const AppendCall C,
+__global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S, const RetierCall C,
                                                      const int32_t* __restrict__ positions,
                                                      const uint8_t* __restrict__ new_tier) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -687,7 +687,7 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
     __shared__ Dest s_dst;
     const int seq = C.seq[i], P = G.r_max + 2;
     const size_t ci = cnt_index(G, seq, C.g, h);
-    for (int t = C.tok0[i]; t < C.tok0[i + 1]; ++t) {
+    for (int t = C.begin[i]; t < C.end[i]; ++t) {
         __syncthreads();                               // the previous token is done
         if (tid == 0) {
             int go = 0;
@@ -802,7 +802,7 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
 
 // After re-tiering: the pages a tier holds beyond ceil(count / 64) go back to the tier's free
 // ring.  One block for the whole call (no other kernel takes from the rings meanwhile).
-__global__ void __launch_bounds__(256) retier_release_kernel(const Geom G, const State S, const AppendCall C) {
+__global__ void __launch_bounds__(256) retier_release_kernel(const Geom G, const State S, const RetierCall C) {
     const int tid = threadIdx.x;
     __shared__ uint32_t s_tail[kMaxTiers], s_total[kMaxTiers], s_over[kMaxTiers];
     if (tid < kMaxTiers) {
@@ -851,8 +851,8 @@ __global__ void __launch_bounds__(256) retier_release_kernel(const Geom G, const
 }  // namespace dwkv
 
 namespace dwkv {
-template __global__ void retier_kernel<8>(const Geom, const State, const AppendCall, const int32_t*, const uint8_t*);
-template __global__ void retier_kernel<4>(const Geom, const State, const AppendCall, const int32_t*, const uint8_t*);
+template __global__ void retier_kernel<8>(const Geom, const State, const RetierCall, const int32_t*, const uint8_t*);
+template __global__ void retier_kernel<4>(const Geom, const State, const RetierCall, const int32_t*, const uint8_t*);
 template __global__ void encode_kernel<8>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
                                           const __nv_bfloat16*, float*);
 template __global__ void encode_kernel<4>(const Geom, const State, const AppendCall, const __nv_bfloat16*,

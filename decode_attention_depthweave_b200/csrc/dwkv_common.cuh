@@ -82,6 +82,15 @@ struct AppendCall {
     int na[kMaxSeqs];        // positions that need a slot
 };
 
+// One round of a re-tier call: for each listed sequence, the tokens [begin, end) of the call's
+// positions / new-tier arrays.
+struct RetierCall {
+    int n, g;
+    int seq[kMaxSeqs];
+    int begin[kMaxSeqs];
+    int end[kMaxSeqs];
+};
+
 struct DecodeCall {
     int n, layer, g, lig, total_splits, ring_bytes, rec_floats;
     int tok_weight;          // split balance: cost of one token in byte-equivalents
@@ -94,10 +103,12 @@ struct DecodeCall {
     const uint8_t* tier_idx;         // [n][Hkv] tier of the new token (read where it is placed)
     int pos[kMaxSeqs];               // the new token's position (fused)
     uint8_t place[kMaxSeqs];         // 1: this layer places it (its group's first to append it)
-    // Sum of the tier counts of each (sequence, kv-head) once every earlier kernel of the stream
-    // has completed.  A CTA that reads exactly this sum before waiting on the previous kernel
-    // (programmatic dependent launch) knows the counts are final; otherwise it waits first.
-    int expect[kMaxSeqs];
+    // 1: the tier counts, page tables and page bytes this launch reads are final before it waits
+    // on the previous kernel (programmatic dependent launch), so its producer may read them and
+    // stream pages at once; 0: it waits first.  The host sets 0 when the previous launch on the
+    // handle was a fused step of the same group that still writes them (a placing launch adds
+    // its token's count at its end; every fused launch writes its token's bytes of its layer).
+    int early;
     int seq[kMaxSeqs];
     int split_begin[kMaxSeqs + 1];
     const __nv_bfloat16* q;  // [n][Hq][d]
@@ -276,20 +287,6 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
 // has issued it or exited.
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void red_release_add_u32(uint32_t* p, uint32_t v) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// Orders this thread's earlier generic-proxy view of global memory before its later bulk
-// (async-proxy) copies.
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 
 // ------------------------------------------------------------------ warp-level MMA pieces (sm_80+ forms)
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {

@@ -634,24 +634,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         mbar_arrive_expect_tx(basis_bar, bytes);
         bulk_g2s(smem_addr(smem + L.rd), St.basis_k + basis_off, bytes, basis_bar);
         // Until this CTA waits on the previous kernel (programmatic dependent launch), that
-        // kernel may still be running: the counts are final only if they sum to what the host
-        // expects once every earlier kernel has completed (the one count a fused decode adds
-        // at its end is the only change in flight).  Acquired together with the writes that
-        // precede that addition, so the slot map and pages read below are complete; otherwise
-        // wait, then read them again.
+        // kernel may still be running; the host says whether the cache state read from here on
+        // (counts, slot map, page tables, page bytes) is already final.
+        if (!C.early) grid_dep_wait();
         const uint32_t* cnt = St.counts + cnt_index(G, seq, C.g, h);
-        uint32_t sum = 0;
 #pragma unroll
-        for (int k = 0; k < kMaxTiers; ++k) {
-            cv[k] = k < G.ntiers ? ld_acquire_u32(cnt + k) : 0u;
-            sum += cv[k];
-        }
-        if (sum != (uint32_t)C.expect[ci]) {
-            grid_dep_wait();
-#pragma unroll
-            for (int k = 0; k < kMaxTiers; ++k) cv[k] = k < G.ntiers ? ld_acquire_u32(cnt + k) : 0u;
-        }
-        fence_proxy_async_global();            // page bytes written before them, read by bulk copies
+        for (int k = 0; k < kMaxTiers; ++k) cv[k] = k < G.ntiers ? __ldcg(cnt + k) : 0u;
         // fused append: the pages are attended without the new token.  Where it was placed by
         // an earlier layer of the group the counts include it (it is the last slot of its tier);
         // where this launch places it they do not yet (the last CTA adds it).
@@ -1207,7 +1195,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         if (C.fused && C.place[ci]) {
             // every CTA has read the counts: add the position placed by the first CTA
             const uint32_t k = C.tier_idx[(size_t)ci * G.Hkv + h];
-            if (k < (uint32_t)G.ntiers) red_release_add_u32(St.counts + cnt_index(G, seq, C.g, h) + k, 1u);
+            if (k < (uint32_t)G.ntiers) St.counts[cnt_index(G, seq, C.g, h) + k] += 1u;
         }
     }
 }

@@ -1,9 +1,10 @@
 """Decode launches that overlap their predecessor (programmatic dependent launch): a launch
 may start, read the tier counts and page tables and stream pages while the previous decode of
-the stream still runs, and waits for it only before reading its inputs or writing.  Results
-must not depend on it: overlapped and serialised launches give bit-identical outputs and
-stored bytes, and both match the oracle, including back-to-back launches that place tokens
-in the same group (a one-layer model) and probes between decode steps."""
+the stream still runs, and waits for it only before reading its inputs or writing (and before
+reading the cache when the previous launch was a fused step of the same group).  Results must
+not depend on it: overlapped and serialised launches store identical bytes and agree to fp32
+rounding, and both match the oracle, including back-to-back launches that place tokens in the
+same group (a one-layer model), probes between decode steps, and graph replays."""
 import os
 
 import numpy as np
@@ -74,12 +75,15 @@ def _oracle_at(wl, bases, state, Q, b, l, st, h, probe=False):
     return oracle.probe_head(prob)[0] if probe else oracle.decode_head(prob)
 
 
-def test_overlapped_and_serialised_launches_are_bit_identical():
+def test_overlapped_and_serialised_launches_agree():
+    """Stored bytes bit for bit; outputs to fp32 rounding (warps take half pages from a shared
+    queue, so the order of a CTA's fp32 sums differs from run to run either way)."""
     wl = synth.workload("llama8b_64k").scaled(num_layers=4, context=3000, batch=2)
     T0s, steps = [2900, 1700], 5
     c_on, o_on, _, st_on, bases, Q = _run_steps(wl, T0s, steps, True)
     c_off, o_off, _, _, _, _ = _run_steps(wl, T0s, steps, False)
-    assert torch.equal(o_on, o_off)
+    d = (o_on - o_off).abs().max().item()
+    assert d <= 1e-6 * max(o_off.abs().max().item(), 1.0), d
     for b, T0 in enumerate(T0s):
         for l in range(wl.num_layers):
             x, y = c_on.export(l, b, 0, T0 + steps), c_off.export(l, b, 0, T0 + steps)
