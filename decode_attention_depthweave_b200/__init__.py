@@ -25,7 +25,7 @@ __all__ = [
     "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
     "dwkv_retier", "dwkv_tier_policy", "dwkv_tier_controller_create", "dwkv_tier_controller_destroy",
     "dwkv_tier_controller_due", "dwkv_tier_controller_threshold", "dwkv_tier_controller_observe",
-    "dwkv_tier_controller_route", "Cache", "EXPORTED_SYMBOLS",
+    "dwkv_tier_controller_route", "dwkv_arena_bytes_all_tiers", "Cache", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,6 +44,7 @@ EXPORTED_SYMBOLS = (
     "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
     "dwkv_retier", "dwkv_tier_controller_create", "dwkv_tier_controller_destroy", "dwkv_tier_controller_due",
     "dwkv_tier_controller_threshold", "dwkv_tier_controller_observe", "dwkv_tier_controller_route",
+    "dwkv_arena_bytes_all_tiers",
 )
 
 
@@ -95,6 +96,7 @@ def lib():
             "dwkv_page_bytes": ([cfgp, i32], sz),
             "dwkv_metadata_bytes": ([cfgp], sz),
             "dwkv_arena_bytes": ([cfgp], sz),
+            "dwkv_arena_bytes_all_tiers": ([cfgp], sz),
             "dwkv_workspace_bytes": ([cfgp, i32], sz),
             "dwkv_create": ([cfgp, vp, sz, vp, vp, vp, C.POINTER(vp)], C.c_int),
             "dwkv_destroy": ([vp], C.c_int),
@@ -197,6 +199,10 @@ def dwkv_metadata_bytes(cfg) -> int:
 
 def dwkv_arena_bytes(cfg) -> int:
     return lib().dwkv_arena_bytes(C.byref(cfg))
+
+
+def dwkv_arena_bytes_all_tiers(cfg) -> int:
+    return lib().dwkv_arena_bytes_all_tiers(C.byref(cfg))
 
 
 def dwkv_workspace_bytes(cfg, n_seqs) -> int:

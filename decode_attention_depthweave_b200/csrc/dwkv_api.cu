@@ -393,6 +393,14 @@ size_t dwkv_arena_bytes(const dwkv_config* cfg) {
     return meta_layout(G).data + worst_data_bytes(G);
 }
 
+size_t dwkv_arena_bytes_all_tiers(const dwkv_config* cfg) {
+    if (check_cfg(cfg) != DWKV_OK) return 0;
+    const Geom G = make_geom(cfg);
+    size_t per_head = 0;
+    for (int k = 0; k < G.ntiers; ++k) per_head += ((size_t)G.max_pages + 1) * G.page_units[k] * kUnit;
+    return meta_layout(G).data + (size_t)G.max_batch * G.G * G.Hkv * per_head;
+}
+
 size_t dwkv_workspace_bytes(const dwkv_config* cfg, int32_t n_seqs) {
     if (check_cfg(cfg) != DWKV_OK || n_seqs < 0) return 0;
     return ws_need(make_geom(cfg), n_seqs, true);

@@ -126,6 +126,12 @@ size_t dwkv_metadata_bytes(const dwkv_config* cfg);
  * smaller and running out of it is a device-side DWKV_DEV_POOL_EXHAUSTED error. */
 size_t dwkv_arena_bytes(const dwkv_config* cfg);
 
+/* Arena bytes for a cache whose tokens change tier (dwkv_retier): a page that moves empty is
+ * kept for reuse by its own tier (pages differ in size between tiers), so every tier may hold
+ * max_context tokens' worth of pages at once: the metadata plus, for every (sequence, group,
+ * kv-head) and tier, (max_pages + 1) pages of that tier.  0 if cfg is invalid. */
+size_t dwkv_arena_bytes_all_tiers(const dwkv_config* cfg);
+
 /* Workspace bytes that decode and probe need for a call over n_seqs sequences (the probe's
  * split-K records are twice as large; decode alone accepts a workspace of half this size:
  * n_seqs * Hkv * 64 records of 8 + 4 * head_dim floats). */
@@ -240,7 +246,9 @@ dwkv_status dwkv_probe(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32
  * between the layers of one step); DWKV_ERR_INVALID_ARG otherwise.  Positions the group has
  * not placed, or tier indices >= num_tiers, set a device error (DWKV_DEV_NO_SLOT,
  * DWKV_DEV_BAD_TIER) and are skipped.  Decoding after the call sees the new tiers; the
- * sequence's length is unchanged.  Pages a tier empties return to the pool's free ring. */
+ * sequence's length is unchanged.  Pages a tier empties return to that tier's free ring and
+ * serve that tier's later placements; an arena sized by dwkv_arena_bytes_all_tiers has room
+ * for any sequence of moves (dwkv_arena_bytes assumes tokens keep their tier). */
 dwkv_status dwkv_retier(dwkv_handle h, int32_t group, int32_t n_seqs, const int32_t* seq_ids,
                         const int32_t* n_tok, const int32_t* positions, const uint8_t* new_tier,
                         void* stream);

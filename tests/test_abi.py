@@ -63,6 +63,12 @@ def test_token_and_page_bytes():
         # two layers x (K + V) blocks, then the 64 slots' positions (int32)
         assert dw.dwkv_page_bytes(cfg, k) == 2 * 2 * (128 * r + 64 * 16 + 8 * 16 * 4 + 128) + 64 * 4
         assert dw.dwkv_page_bytes(cfg, k) % 128 == 0
+    # room for every tier at its largest (re-tiering): metadata + pages of every tier
+    G = cfg.num_layers // cfg.layers_per_group
+    pages = (cfg.max_context + 63) // 64 + 1
+    want = dw.dwkv_metadata_bytes(cfg) + cfg.max_batch * G * cfg.num_kv_heads * pages * sum(
+        dw.dwkv_page_bytes(cfg, k) for k in range(cfg.num_tiers))
+    assert dw.dwkv_arena_bytes_all_tiers(cfg) == want
     meta = dw.dwkv_metadata_bytes(cfg)
     assert 0 < meta < dw.dwkv_arena_bytes(cfg)
     assert dw.dwkv_workspace_bytes(cfg, 8) == 8 * dw.dwkv_workspace_bytes(cfg, 1)

@@ -105,7 +105,8 @@ def test_repeated_moves_reuse_pages_and_fused_steps_continue():
     wl = synth.workload("tiny_1k").scaled(num_q_heads=8, num_kv_heads=2)
     T0 = 600
     bases = synth.make_bases(wl)
-    cache = dw.Cache(cfg_for(wl, max_context=T0 + 16), bases[0], bases[1])
+    cfg = cfg_for(wl, max_context=T0 + 16)
+    cache = dw.Cache(cfg, bases[0], bases[1], arena_bytes=dw.dwkv_arena_bytes_all_tiers(cfg))
     data = import_workload(cache, wl, [T0])
     state = {(0, l): data[(0, l)] for l in range(2)}
     reserved = []
