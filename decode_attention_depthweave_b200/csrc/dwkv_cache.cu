@@ -821,8 +821,13 @@ __global__ void __launch_bounds__(256) retier_release_kernel(const Geom G, const
     }
     __syncthreads();
     if (tid < G.ntiers) {
+        // pops on an empty ring move the head past the tail; no kernel pops meanwhile, so bring
+        // it back before the pushes (as the reset does)
         uint32_t hd = S.free_head[tid];
-        if ((int)(hd - s_tail[tid]) > 0) hd = s_tail[tid];
+        if ((int)(hd - s_tail[tid]) > 0) {
+            hd = s_tail[tid];
+            S.free_head[tid] = hd;
+        }
         if ((s_tail[tid] - hd) + s_total[tid] > G.free_cap) {
             s_over[tid] = 1u;
             set_dev_error(S, 7u /*DWKV_DEV_FREE_LIST*/, 0xffffffffu, (uint32_t)tid);
