@@ -31,19 +31,19 @@ def lib():
         p = C.c_void_p
         i = C.c_int
         d = C.c_double
-        L.oracle_decode_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, i, p, p]
+        L.oracle_decode_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, i, p, p, p]
         L.oracle_decode_head.restype = i
-        L.oracle_probe_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, d, p, p, p]
+        L.oracle_probe_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, d, p, p, p, p]
         L.oracle_probe_head.restype = i
-        L.oracle_decode_many.argtypes = [i, i, i, i, i, p] + [p] * 12 + [d, p, i]
+        L.oracle_decode_many.argtypes = [i, i, i, i, i, p] + [p] * 12 + [d, p, i, p]
         L.oracle_decode_many.restype = i
         L.oracle_encode_vector.argtypes = [i, i, p, p, i, i, i, p, p, p, p, p, p]
         L.oracle_encode_vector.restype = i
         L.oracle_quantize_residual.argtypes = [i, i, i, p, p, p, p]
         L.oracle_quantize_residual.restype = i
-        L.oracle_encode_many.argtypes = [i, i, i, p, p, p, i, i, p, p, p, p, p, i]
+        L.oracle_encode_many.argtypes = [i, i, i, p, p, p, i, i, p, p, p, p, p, i, p]
         L.oracle_encode_many.restype = i
-        L.oracle_encode_many_from_coeffs.argtypes = [i, i, i, p, p, p, p, i, i, p, p, p, p, i]
+        L.oracle_encode_many_from_coeffs.argtypes = [i, i, i, p, p, p, p, i, i, p, p, p, p, i, p]
         L.oracle_encode_many_from_coeffs.restype = i
         L.oracle_reencode_vector.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, i, p, p, p, p, p]
         L.oracle_reencode_vector.restype = i
@@ -142,7 +142,7 @@ class HeadProblem:
     """Token-ordered inputs of one (sequence, layer, kv-head) decode problem."""
 
     def __init__(self, basis_k, basis_v, ranks, coeff_k, idx_k, codes_k, scale_k,
-                 coeff_v, idx_v, codes_v, scale_v, q):
+                 coeff_v, idx_v, codes_v, scale_v, q, nres=None):
         self.bk = _bits16(basis_k)
         self.bv = _bits16(basis_v)
         self.d, self.r_max = self.bk.shape
@@ -160,6 +160,8 @@ class HeadProblem:
         self.sv = _bits16(scale_v).reshape(self.T)
         self.q = _bits16(q).reshape(-1, self.d)
         self.gq = self.q.shape[0]
+        # per-token residual counts (each <= s), or None: every token keeps s entries
+        self.nres = None if nres is None else _arr(nres, np.int32).reshape(self.T)
 
     def _ptrs(self):
         return [_p(self.bk), _p(self.bv), _p(self.rank), _p(self.ck), _p(self.ik), _p(self.qk),
@@ -168,7 +170,8 @@ class HeadProblem:
 
 def head_problem(wl, bases, tier_idx, comp, q, layer, head) -> HeadProblem:
     """The decode problem of one (layer, kv-head) of one sequence, sliced from token-ordered
-    arrays: ``wl`` a workload (tiers, layers_per_group, gqa), ``bases`` the (K, V) bases
+    arrays: ``wl`` a workload (tiers, optional per-tier residual counts ``tier_resid``,
+    layers_per_group, gqa), ``bases`` the (K, V) bases
     bf16 [G][Hkv][d][r_max], ``tier_idx`` uint8 [T][Hkv] (index into ``wl.tiers``), ``comp``
     the stored arrays (coeff [T][Hkv][2][r_max], idx / codes [T][Hkv][2][s], scales
     [T][Hkv][2]; K at [..][0], V at [..][1]) and ``q`` bf16 [Hq][d], every query head of the
@@ -177,11 +180,13 @@ def head_problem(wl, bases, tier_idx, comp, q, layer, head) -> HeadProblem:
     gq = wl.gqa
     ti = _arr(tier_idx, np.int64)[:, head]
     ranks = np.asarray(wl.tiers, np.int32)[ti]
+    tr = getattr(wl, "tier_resid", ())
+    nres = np.asarray(tr, np.int32)[ti] if tr else None
     sl = lambda key, z: comp[key][:, head, z]   # noqa: E731
     return HeadProblem(bases[0][g, head], bases[1][g, head], ranks,
                        sl("coeff", 0), sl("idx", 0), sl("codes", 0), comp["scales"][:, head, 0],
                        sl("coeff", 1), sl("idx", 1), sl("codes", 1), comp["scales"][:, head, 1],
-                       _bits16(q)[head * gq:(head + 1) * gq])
+                       _bits16(q)[head * gq:(head + 1) * gq], nres=nres)
 
 
 def decode_head(prob: HeadProblem, tau=None, with_residual=True, want_p=False):
@@ -191,7 +196,7 @@ def decode_head(prob: HeadProblem, tau=None, with_residual=True, want_p=False):
     pw = np.empty((prob.gq, max(prob.T, 1)), np.float64) if want_p else None
     rc = lib().oracle_decode_head(prob.d, prob.r_max, prob.T, prob.gq, prob.s, *prob._ptrs(),
                                   float(tau), 1 if with_residual else 0, _p(out),
-                                  _p(pw) if want_p else None)
+                                  _p(pw) if want_p else None, _p(prob.nres) if prob.nres is not None else None)
     if rc != 0:
         raise MemoryError("oracle_decode_head failed")
     if want_p:
@@ -206,7 +211,8 @@ def probe_head(prob: HeadProblem, tau=None, eps=1e-6):
     of = np.empty((prob.gq, prob.d), np.float64)
     on = np.empty((prob.gq, prob.d), np.float64)
     rc = lib().oracle_probe_head(prob.d, prob.r_max, prob.T, prob.gq, prob.s, *prob._ptrs(),
-                                 float(tau), float(eps), _p(err), _p(of), _p(on))
+                                 float(tau), float(eps), _p(err), _p(of), _p(on),
+                                 _p(prob.nres) if prob.nres is not None else None)
     if rc != 0:
         raise MemoryError("oracle_probe_head failed")
     return float(err[0]), of, on
@@ -225,8 +231,12 @@ def decode_many(problems, tau=None, nthreads=None):
     arrs = [(C.c_void_p * n)(*col) for col in cols]
     outs = [np.empty((pr.gq, pr.d), np.float64) for pr in problems]
     oarr = (C.c_void_p * n)(*[_p(o) for o in outs])
+    narr = None
+    if any(pr.nres is not None for pr in problems):
+        full = [pr.nres if pr.nres is not None else np.full(pr.T, pr.s, np.int32) for pr in problems]
+        narr = (C.c_void_p * n)(*[_p(a) for a in full])
     rc = lib().oracle_decode_many(n, p0.d, p0.r_max, p0.gq, p0.s, _p(T), *arrs, float(tau), oarr,
-                                  int(nthreads))
+                                  int(nthreads), narr)
     if rc != 0:
         raise MemoryError("oracle_decode_many failed")
     return outs
@@ -263,8 +273,9 @@ def quantize_residual(r, s, bits):
     return {"idx": idx, "codes": codes, "scale": scale[0]}
 
 
-def encode_many(basis, x, ranks, s, bits, nthreads=None, want_c32=False):
-    """Encode n vectors [n][d] sharing one basis; arrays token-ordered."""
+def encode_many(basis, x, ranks, s, bits, nthreads=None, want_c32=False, nres=None):
+    """Encode n vectors [n][d] sharing one basis; arrays token-ordered.  ``nres`` (optional,
+    int [n], each <= s): per-vector residual counts; entries past them stay zero."""
     b = _bits16(basis)
     d, r_max = b.shape
     xv = _bits16(x).reshape(-1, d)
@@ -275,9 +286,10 @@ def encode_many(basis, x, ranks, s, bits, nthreads=None, want_c32=False):
     idx = np.zeros((n, s), np.uint8)
     codes = np.zeros((n, s), np.int8)
     scale = np.zeros(n, np.uint16)
+    nr = None if nres is None else _arr(nres, np.int32).reshape(n)
     rc = lib().oracle_encode_many(n, d, r_max, _p(b), _p(xv), _p(rk), int(s), int(bits), _p(coeff),
                                   _p(c32) if want_c32 else None, _p(idx), _p(codes), _p(scale),
-                                  int(nthreads or os.cpu_count() or 1))
+                                  int(nthreads or os.cpu_count() or 1), _p(nr) if nr is not None else None)
     if rc != 0:
         raise ValueError("oracle_encode_many: bad arguments")
     out = {"coeff": coeff, "idx": idx, "codes": codes, "scale": scale}
@@ -308,7 +320,7 @@ def reencode_vector(basis, r_old, coeff, idx, codes, scale, r_new, bits):
     return {"coeff": out_c, "idx": out_i, "codes": out_q, "scale": out_s[0], "xh": xh}
 
 
-def encode_many_from_coeffs(basis, x, c32, ranks, s, bits, nthreads=None):
+def encode_many_from_coeffs(basis, x, c32, ranks, s, bits, nthreads=None, nres=None):
     """Encode steps 2-6 of n vectors [n][d] sharing one basis, from given fp32 projections
     c32 [n][r_max] (only [:r_t] read): the stored bytes of an encoder that computed c32."""
     b = _bits16(basis)
@@ -321,8 +333,10 @@ def encode_many_from_coeffs(basis, x, c32, ranks, s, bits, nthreads=None):
     idx = np.zeros((n, s), np.uint8)
     codes = np.zeros((n, s), np.int8)
     scale = np.zeros(n, np.uint16)
+    nr = None if nres is None else _arr(nres, np.int32).reshape(n)
     rc = lib().oracle_encode_many_from_coeffs(n, d, r_max, _p(b), _p(xv), _p(cv), _p(rk), int(s), int(bits), _p(coeff),
-                                              _p(idx), _p(codes), _p(scale), int(nthreads or os.cpu_count() or 1))
+                                              _p(idx), _p(codes), _p(scale), int(nthreads or os.cpu_count() or 1),
+                                              _p(nr) if nr is not None else None)
     if rc != 0:
         raise ValueError("oracle_encode_many_from_coeffs: bad arguments")
     return {"coeff": coeff, "idx": idx, "codes": codes, "scale": scale}

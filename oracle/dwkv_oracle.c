@@ -111,6 +111,8 @@ void oracle_reconstruct(int d, int r_max, const uint16_t* basis, int r_t, const 
 /*   reconstructed cache; the reconstruction is never stored).                            */
 /* Token arrays are token-ordered: rank[T]; ck/cv [T][r_max] bf16; ik/iv [T][s] u8;       */
 /* qk/qv [T][s] i8 codes; sk/sv [T] fp16.  q: bf16 [gq][d].  out: [gq][d].                 */
+/* nres (nullable): token t keeps only its first nres[t] <= s residual entries ([DW] §3     */
+/* Eq. (2): the router's level is the number of retained residual channels).               */
 /* p_out (nullable): softmax weights [gq][T].  Returns 0, or -1 on allocation failure.    */
 /* T == 0 gives a zero output (attention over an empty cache).                            */
 /* ------------------------------------------------------------------------------------ */
@@ -119,7 +121,7 @@ int oracle_decode_head(int d, int r_max, int T, int gq, int s,
                        const uint16_t* ck, const uint8_t* ik, const int8_t* qk, const uint16_t* sk,
                        const uint16_t* cv, const uint8_t* iv, const int8_t* qv, const uint16_t* sv,
                        const uint16_t* q, double tau, int with_residual,
-                       double* out, double* p_out) {
+                       double* out, double* p_out, const int32_t* nres) {
     for (int h = 0; h < gq * d; ++h) out[h] = 0.0;
     if (T <= 0) return 0;
     double* score = (double*)malloc(sizeof(double) * (size_t)T * gq);
@@ -130,7 +132,7 @@ int oracle_decode_head(int d, int r_max, int T, int gq, int s,
 
     /* scores: tau * q . K^_t */
     for (int t = 0; t < T; ++t) {
-        oracle_reconstruct(d, r_max, bk, rank[t], ck + (size_t)t * r_max, s,
+        oracle_reconstruct(d, r_max, bk, rank[t], ck + (size_t)t * r_max, nres ? nres[t] : s,
                            ik + (size_t)t * s, qk + (size_t)t * s, sk[t], with_residual, x);
         for (int h = 0; h < gq; ++h) {
             double dot = 0.0;
@@ -151,7 +153,7 @@ int oracle_decode_head(int d, int r_max, int T, int gq, int s,
     }
     /* o = sum_t p_t V^_t */
     for (int t = 0; t < T; ++t) {
-        oracle_reconstruct(d, r_max, bv, rank[t], cv + (size_t)t * r_max, s,
+        oracle_reconstruct(d, r_max, bv, rank[t], cv + (size_t)t * r_max, nres ? nres[t] : s,
                            iv + (size_t)t * s, qv + (size_t)t * s, sv[t], with_residual, x);
         for (int h = 0; h < gq; ++h) {
             double p = score[(size_t)t * gq + h];
@@ -175,15 +177,15 @@ int oracle_probe_head(int d, int r_max, int T, int gq, int s,
                       const uint16_t* ck, const uint8_t* ik, const int8_t* qk, const uint16_t* sk,
                       const uint16_t* cv, const uint8_t* iv, const int8_t* qv, const uint16_t* sv,
                       const uint16_t* q, double tau, double eps,
-                      double* err, double* o_full, double* o_nores) {
+                      double* err, double* o_full, double* o_nores, const int32_t* nres) {
     double* a = (double*)malloc(sizeof(double) * (size_t)gq * d);
     double* b = (double*)malloc(sizeof(double) * (size_t)gq * d);
     if (!a || !b) { free(a); free(b); return -1; }
     int rc = oracle_decode_head(d, r_max, T, gq, s, bk, bv, rank, ck, ik, qk, sk, cv, iv, qv, sv,
-                                q, tau, 1, a, NULL);
+                                q, tau, 1, a, NULL, nres);
     if (rc == 0)
         rc = oracle_decode_head(d, r_max, T, gq, s, bk, bv, rank, ck, ik, qk, sk, cv, iv, qv, sv,
-                                q, tau, 0, b, NULL);
+                                q, tau, 0, b, NULL, nres);
     if (rc == 0) {
         double num = 0.0, den = 0.0;
         for (int k = 0; k < gq * d; ++k) { num += (a[k] - b[k]) * (a[k] - b[k]); den += a[k] * a[k]; }
@@ -205,12 +207,14 @@ int oracle_decode_many(int n, int d, int r_max, int gq, int s, const int32_t* T,
                        const uint16_t* const* sk,
                        const uint16_t* const* cv, const uint8_t* const* iv, const int8_t* const* qv,
                        const uint16_t* const* sv,
-                       const uint16_t* const* q, double tau, double* const* out, int nthreads) {
+                       const uint16_t* const* q, double tau, double* const* out, int nthreads,
+                       const int32_t* const* nres) {
     int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(| : bad)
     for (int k = 0; k < n; ++k)
         bad |= (oracle_decode_head(d, r_max, T[k], gq, s, bk[k], bv[k], rank[k], ck[k], ik[k], qk[k],
-                                   sk[k], cv[k], iv[k], qv[k], sv[k], q[k], tau, 1, out[k], NULL) != 0);
+                                   sk[k], cv[k], iv[k], qv[k], sv[k], q[k], tau, 1, out[k], NULL,
+                                   nres ? nres[k] : NULL) != 0);
     return bad ? -1 : 0;
 }
 
@@ -327,11 +331,13 @@ int oracle_encode_vector(int d, int r_max, const uint16_t* basis, const uint16_t
 /* Steps 2-6 for many vectors that share one basis, from given projections c32 [n][r_max]. */
 int oracle_encode_many_from_coeffs(int n, int d, int r_max, const uint16_t* basis, const uint16_t* x,
                                    const float* c32, const int32_t* rank, int s, int bits, uint16_t* coeff,
-                                   uint8_t* idx, int8_t* codes, uint16_t* scale, int nthreads) {
+                                   uint8_t* idx, int8_t* codes, uint16_t* scale, int nthreads,
+                                   const int32_t* nres) {
     int bad = 0;
 #pragma omp parallel for schedule(static) num_threads(nthreads) reduction(| : bad)
     for (int k = 0; k < n; ++k)
-        bad |= (oracle_encode_from_coeffs(d, r_max, basis, x + (size_t)k * d, c32 + (size_t)k * r_max, rank[k], s,
+        bad |= (oracle_encode_from_coeffs(d, r_max, basis, x + (size_t)k * d, c32 + (size_t)k * r_max, rank[k],
+                                          nres ? nres[k] : s,
                                           bits, coeff + (size_t)k * r_max, idx + (size_t)k * s, codes + (size_t)k * s,
                                           scale + k, NULL) != 0);
     return bad ? -1 : 0;
@@ -340,11 +346,11 @@ int oracle_encode_many_from_coeffs(int n, int d, int r_max, const uint16_t* basi
 /* Encode many vectors that share one basis (token-ordered): x [n][d], rank [n]. */
 int oracle_encode_many(int n, int d, int r_max, const uint16_t* basis, const uint16_t* x,
                        const int32_t* rank, int s, int bits, uint16_t* coeff, float* c32,
-                       uint8_t* idx, int8_t* codes, uint16_t* scale, int nthreads) {
+                       uint8_t* idx, int8_t* codes, uint16_t* scale, int nthreads, const int32_t* nres) {
     int bad = 0;
 #pragma omp parallel for schedule(static) num_threads(nthreads) reduction(| : bad)
     for (int k = 0; k < n; ++k)
-        bad |= (oracle_encode_vector(d, r_max, basis, x + (size_t)k * d, rank[k], s, bits,
+        bad |= (oracle_encode_vector(d, r_max, basis, x + (size_t)k * d, rank[k], nres ? nres[k] : s, bits,
                                      coeff + (size_t)k * r_max, c32 ? c32 + (size_t)k * r_max : NULL,
                                      idx + (size_t)k * s, codes + (size_t)k * s, scale + k, NULL) != 0);
     return bad ? -1 : 0;
