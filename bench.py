@@ -73,6 +73,11 @@ def token_bytes(rank: int, s: int, bits: int) -> int:
     return 2 * (2 * rank + s + s * bits // 8 + 2)
 
 
+def tier_counts_of(wl) -> list:
+    """Residual channels a token of each tier keeps."""
+    return list(wl.tier_resid) if wl.tier_resid else [wl.resid_channels] * len(wl.tiers)
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -326,7 +331,8 @@ def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e
     cfg = dw.config_from(num_layers=wl.num_layers, layers_per_group=wl.layers_per_group,
                          num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim,
                          r_max=wl.r_max, tiers=wl.tiers, resid_channels=wl.resid_channels,
-                         resid_bits=wl.resid_bits, max_batch=B, max_context=max(lengths) + n_steps + extra)
+                         resid_bits=wl.resid_bits, max_batch=B, max_context=max(lengths) + n_steps + extra,
+                         tier_resid=wl.tier_resid or None)
     stream = torch.cuda.Stream(device=dev)
     cache = dw.Cache(cfg, bases[0], bases[1], device=dev, ws_seqs=B, stream=stream)
     if args.tuning:
@@ -470,7 +476,8 @@ def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e
     # ---- algorithmic bytes: every stored byte of the attended tokens (per-token bytes of
     #      its tier), plus the two bases, the queries and the outputs of each launch
     held = sum(lengths) - B + B * (warmup + steps)            # tokens per head after the timed steps
-    tok_bytes = torch.tensor([token_bytes(r, wl.resid_channels, wl.resid_bits) for r in wl.tiers], dtype=torch.float64)
+    tok_bytes = torch.tensor([token_bytes(r, n, wl.resid_bits) for r, n in zip(wl.tiers, tier_counts_of(wl))],
+                             dtype=torch.float64)
     bytes_per_tok_head = float((tier_counts.double() * tok_bytes).sum()) / (wl.num_groups * wl.num_kv_heads * held)
     basis_bytes = 2 * wl.num_kv_heads * wl.head_dim * wl.r_max * 2
     io_bytes = B * wl.num_q_heads * wl.head_dim * (2 + 4)
@@ -598,6 +605,7 @@ def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e
                    "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                    "batch_per_gpu": B, "context": lengths[0] if B == 1 else lengths, "r_max": wl.r_max,
                    "tiers": list(wl.tiers), "tier_probs": list(wl.tier_probs), "resid_channels": wl.resid_channels,
+                   **({"tier_resid": list(wl.tier_resid)} if wl.tier_resid else {}),
                    "resid_bits": wl.resid_bits, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2 (~{comp_bytes_layer * wl.num_layers / 1e9:.1f} GB of pages per step); "
                          "no flush",
@@ -811,6 +819,7 @@ def run_encode(args, world, rank, local):
         "config": {"workload": args.workload, "layers": wl.num_layers, "kv_heads": wl.num_kv_heads,
                    "head_dim": wl.head_dim, "batch_per_gpu": B, "new_tokens": N, "r_max": wl.r_max,
                    "tiers": list(wl.tiers), "tier_probs": list(wl.tier_probs), "resid_channels": wl.resid_channels,
+                   **({"tier_resid": list(wl.tier_resid)} if wl.tier_resid else {}),
                    "resid_bits": wl.resid_bits, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (8.6 GB of dense K/V a step); no flush",
                    "timing": "eager launches, CUDA events around each step's appends (resets outside)"},
@@ -886,7 +895,7 @@ def run_reference(args, world, rank, local):
     }
 
 
-EXTRA_WORKLOADS = ("llama8b_ragged_b8", "llama8b_131k_deep", "llama8b_encode_16k")
+EXTRA_WORKLOADS = ("llama8b_ragged_b8", "llama8b_131k_deep", "llama8b_routed_64k", "llama8b_encode_16k")
 
 
 def summary_of(res: dict) -> dict:

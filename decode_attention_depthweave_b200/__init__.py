@@ -60,7 +60,7 @@ class dwkv_config(C.Structure):
         ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32), ("r_max", C.c_int32),
         ("num_tiers", C.c_int32), ("tiers", C.c_int32 * 8), ("resid_channels", C.c_int32),
         ("resid_bits", C.c_int32), ("max_batch", C.c_int32), ("max_context", C.c_int32),
-        ("softmax_scale", C.c_float),
+        ("softmax_scale", C.c_float), ("resid_routed", C.c_int32), ("tier_resid", C.c_int32 * 8),
     ]
 
 
@@ -160,8 +160,15 @@ def _stream(stream):
 
 
 def config_from(num_layers, layers_per_group, num_q_heads, num_kv_heads, head_dim, r_max, tiers,
-                resid_channels, resid_bits, max_batch, max_context, softmax_scale=0.0) -> dwkv_config:
+                resid_channels, resid_bits, max_batch, max_context, softmax_scale=0.0,
+                tier_resid=None) -> dwkv_config:
+    """tier_resid: per-tier residual channel counts (residual-count routing; every tier then has
+    the same rank and resid_channels is 8), or None for one count, resid_channels, everywhere."""
     c = dwkv_config()
+    if tier_resid is not None:
+        c.resid_routed = 1
+        for k, n in enumerate(tier_resid):
+            c.tier_resid[k] = int(n)
     c.num_layers, c.layers_per_group = num_layers, layers_per_group
     c.num_q_heads, c.num_kv_heads, c.head_dim, c.r_max = num_q_heads, num_kv_heads, head_dim, r_max
     c.num_tiers = len(tiers)

@@ -94,17 +94,30 @@ dwkv_status check_cfg(const dwkv_config* c) {
         return fail(DWKV_ERR_INVALID_ARG, "r_max %d must be a multiple of 8 in [8, head_dim]", c->r_max);
     if (c->num_tiers < 1 || c->num_tiers > DWKV_MAX_TIERS)
         return fail(DWKV_ERR_INVALID_ARG, "num_tiers %d out of [1, %d]", c->num_tiers, DWKV_MAX_TIERS);
+    if (c->resid_routed != 0 && c->resid_routed != 1)
+        return fail(DWKV_ERR_INVALID_ARG, "resid_routed must be 0 or 1 (got %d)", c->resid_routed);
     for (int k = 0; k < c->num_tiers; ++k) {
         if (c->tiers[k] <= 0 || c->tiers[k] % 8 || c->tiers[k] > c->r_max)
             return fail(DWKV_ERR_INVALID_ARG, "tier %d rank %d must be a multiple of 8 in [8, r_max]", k, c->tiers[k]);
-        if (k && c->tiers[k] <= c->tiers[k - 1])
+        if (!c->resid_routed && k && c->tiers[k] <= c->tiers[k - 1])
             return fail(DWKV_ERR_INVALID_ARG, "tiers must be strictly ascending");
+        if (c->resid_routed) {
+            const int t = c->tier_resid[k];
+            if (c->tiers[k] != c->tiers[0])
+                return fail(DWKV_ERR_INVALID_ARG, "with resid_routed every tier has the same rank");
+            if (t != 0 && t != 2 && t != 4 && t != 8)
+                return fail(DWKV_ERR_INVALID_ARG, "tier_resid[%d] = %d must be 0, 2, 4 or 8", k, t);
+            if (k && t <= c->tier_resid[k - 1])
+                return fail(DWKV_ERR_INVALID_ARG, "tier_resid must be strictly ascending");
+        }
     }
     if (c->resid_bits != 8 && c->resid_bits != 4)
         return fail(DWKV_ERR_INVALID_ARG, "resid_bits must be 8 or 4 (got %d)", c->resid_bits);
     if (c->resid_channels < 0 || c->resid_channels > c->head_dim || c->resid_channels % 8)
         return fail(DWKV_ERR_INVALID_ARG, "resid_channels %d must be a multiple of 8 in [0, head_dim]",
                     c->resid_channels);
+    if (c->resid_routed && c->resid_channels != 8)
+        return fail(DWKV_ERR_INVALID_ARG, "with resid_routed, resid_channels must be 8 (the arrays' stride)");
     if (c->max_batch <= 0 || c->max_context <= 0)
         return fail(DWKV_ERR_INVALID_ARG, "max_batch and max_context must be positive");
     if (c->max_context >= (1 << 24))
@@ -143,6 +156,8 @@ Geom make_geom(const dwkv_config* c) {
     G.r_max = c->r_max;
     G.ntiers = c->num_tiers;
     G.s = c->resid_channels;
+    G.routed = c->resid_routed ? 1 : 0;
+    for (int k = 0; k < kMaxTiers; ++k) G.ts[k] = (k < c->num_tiers && G.routed) ? c->tier_resid[k] : G.s;
     G.bits = c->resid_bits;
     G.max_batch = c->max_batch;
     G.max_context = c->max_context;
@@ -152,7 +167,7 @@ Geom make_geom(const dwkv_config* c) {
     for (int k = 0; k < kMaxTiers; ++k) {
         if (k < c->num_tiers) {
             G.tiers[k] = c->tiers[k];
-            G.blk_bytes[k] = blk_bytes_of(c->tiers[k], G.s, G.bits);
+            G.blk_bytes[k] = blk_bytes_of(c->tiers[k], G.ts[k], G.bits);
             G.chunk_bytes[k] = 2 * G.blk_bytes[k];
             G.page_units[k] = (G.LPG * G.chunk_bytes[k] + kPosBlockBytes) / kUnit;
             stage = std::max(stage, G.chunk_bytes[k]);
@@ -372,7 +387,8 @@ dwkv_status dwkv_config_check(const dwkv_config* cfg) {
 
 size_t dwkv_token_bytes(const dwkv_config* cfg, int32_t tier) {
     if (check_cfg(cfg) != DWKV_OK || tier < 0 || tier >= cfg->num_tiers) return 0;
-    const int r = cfg->tiers[tier], s = cfg->resid_channels, b = cfg->resid_bits;
+    const int r = cfg->tiers[tier], s = cfg->resid_routed ? cfg->tier_resid[tier] : cfg->resid_channels;
+    const int b = cfg->resid_bits;
     return (size_t)2 * (2 * r + s + s * b / 8 + 2);
 }
 
@@ -458,7 +474,8 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
 #define DWKV_K(B, P) (const void*)decode_kernel<B, P, 64, 0>, (const void*)decode_kernel<B, P, 64, 8>,       \
                      (const void*)decode_kernel<B, P, 64, 16>, (const void*)decode_kernel<B, P, 64, 32>,     \
                      (const void*)decode_kernel<B, P, 128, 0>, (const void*)decode_kernel<B, P, 128, 8>,     \
-                     (const void*)decode_kernel<B, P, 128, 16>, (const void*)decode_kernel<B, P, 128, 32>
+                     (const void*)decode_kernel<B, P, 128, 16>, (const void*)decode_kernel<B, P, 128, 32>,   \
+                     (const void*)decode_kernel<B, P, 64, -1>, (const void*)decode_kernel<B, P, 128, -1>
             DWKV_K(4, false), DWKV_K(4, true), DWKV_K(8, false), DWKV_K(8, true),
 #undef DWKV_K
         };
@@ -791,7 +808,8 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
 #define DWKV_LAUNCH(B, P, R, SS) lerr = launch_decode(decode_kernel<B, P, R, SS>, grid, smem, s, h->dec_overlap != 0, G, h->st, C)
 #define DWKV_LAUNCH_S(B, P, R)                                  \
     do {                                                        \
-        switch (G.s) {                                          \
+        switch (G.routed ? -1 : G.s) {                          \
+            case -1: DWKV_LAUNCH(B, P, R, -1); break;           \
             case 0: DWKV_LAUNCH(B, P, R, 0); break;             \
             case 8: DWKV_LAUNCH(B, P, R, 8); break;             \
             case 16: DWKV_LAUNCH(B, P, R, 16); break;           \

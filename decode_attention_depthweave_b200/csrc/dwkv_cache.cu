@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
                 slot = base[d.k] + within;
                 sblk[slot] = d.blk + (z ? G.blk_bytes[d.k] : 0u);
                 sR[slot] = d.R;
-                sprow[slot] = d.row;
+                sprow[slot] = d.row | (d.k << 8);          // row in the page, tier
                 srow[slot] = row;
             }
             rslot[trow] = slot;
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
                                 __nv_bfloat162 pr;
                                 pr.x = c0;
                                 pr.y = c1;
-                                *reinterpret_cast<__nv_bfloat162*>(sblk[sl] + (size_t)(j0 >> 3) * 1024 + sprow[sl] * 16 +
+                                *reinterpret_cast<__nv_bfloat162*>(sblk[sl] + (size_t)(j0 >> 3) * 1024 + (sprow[sl] & 0xff) * 16 +
                                                                    (j0 & 7) * 2) = pr;
                                 if (coeff_dbg)
                                     *reinterpret_cast<float2*>(coeff_dbg + (((size_t)srow[sl] * G.Hkv + h) * 2 + z) * RM +
@@ -406,7 +406,7 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
                 const int sl = s0 + t;
                 if (sl >= nvalid) break;
                 const float r4[4] = {a[t][0], a[t][1], a[t][2], a[t][3]};
-                quantize_store<BITS>(G, r4, sblk[sl], sR[sl], sprow[sl], rstage, chstage);
+                quantize_store<BITS>(r4, sblk[sl], sR[sl], sprow[sl] & 0xff, G.ts[sprow[sl] >> 8], rstage, chstage);
             }
         }
     }
@@ -439,14 +439,12 @@ __global__ void __launch_bounds__(256) quantize_test_kernel(int n, int s, const 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int v = blockIdx.x * 8 + warp;
     if (v >= n) return;                         // whole warps
-    Geom G{};
-    G.s = s;                                    // the only field the steps read
     float rr[4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) rr[m] = r[(size_t)v * kD + lane + 32 * m];
     uint8_t* blk = work + (size_t)v * stride;
     float* rstage = reinterpret_cast<float*>(stage + warp * kEncStage);
-    quantize_store<BITS>(G, rr, blk, 0, 0, rstage, reinterpret_cast<uint8_t*>(rstage + kD));
+    quantize_store<BITS>(rr, blk, 0, 0, s, rstage, reinterpret_cast<uint8_t*>(rstage + kD));
     __syncwarp();
     for (int b = lane; b < s; b += 32) {
         idx[(size_t)v * s + b] = blk[off_idx_of(0) + b];
@@ -516,30 +514,30 @@ __global__ void __launch_bounds__(256) import_kernel(const Geom G, const State S
                 set_dev_error(S, 5u, (uint32_t)seq, (uint32_t)pos);
             continue;
         }
-        const int R = dst.R;
+        const int R = dst.R, st = G.ts[dst.k];        // the row's tier keeps st <= s entries
         for (int z = 0; z < 2; ++z) {
             const size_t src = ((size_t)row * G.Hkv + h) * 2 + z;
             uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
             for (int j = lane; j < R; j += 32)
                 *reinterpret_cast<__nv_bfloat16*>(blk + (j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2) =
                     coeff[src * RM + j];
-            for (int e = lane; e < s; e += 32) {
+            for (int e = lane; e < st; e += 32) {
                 const uint8_t ch = idx[src * s + e];
                 if (ch >= kD) set_dev_error(S, 3u /*DWKV_DEV_BAD_CHANNEL*/, (uint32_t)seq, (uint32_t)pos);
-                blk[off_idx_of(R) + dst.row * s + e] = ch;
-                if (BITS == 8) blk[off_codes_of(R, s) + dst.row * s + e] = (uint8_t)codes[src * s + e];
+                blk[off_idx_of(R) + dst.row * st + e] = ch;
+                if (BITS == 8) blk[off_codes_of(R, st) + dst.row * st + e] = (uint8_t)codes[src * s + e];
             }
             if (BITS == 4) {
-                for (int b = lane; b < s / 2; b += 32) {
+                for (int b = lane; b < st / 2; b += 32) {
                     const int c0 = codes[src * s + 2 * b], c1 = codes[src * s + 2 * b + 1];
                     if (c0 < -8 || c0 > 7 || c1 < -8 || c1 > 7)
                         set_dev_error(S, 4u /*DWKV_DEV_BAD_CODE*/, (uint32_t)seq, (uint32_t)pos);
-                    blk[off_codes_of(R, s) + dst.row * (s / 2) + b] =
+                    blk[off_codes_of(R, st) + dst.row * (st / 2) + b] =
                         (uint8_t)(((uint32_t)c0 & 0xfu) | (((uint32_t)c1 & 0xfu) << 4));
                 }
             }
-            if (lane == 0)
-                *reinterpret_cast<__half*>(blk + off_scales_of(R, s, BITS) + dst.row * 2) = scales[src];
+            if (lane == 0 && st)
+                *reinterpret_cast<__half*>(blk + off_scales_of(R, st, BITS) + dst.row * 2) = scales[src];
         }
     }
 }
@@ -561,20 +559,21 @@ __global__ void __launch_bounds__(256) export_kernel(const Geom G, const State S
         for (int z = 0; z < 2; ++z) {
             const size_t o = (size_t)w * 2 + z;
             const uint8_t* blk = ok ? dst.blk + (z ? G.blk_bytes[dst.k] : 0u) : nullptr;
-            const int R = ok ? dst.R : 0;
+            const int R = ok ? dst.R : 0, st = ok ? G.ts[dst.k] : 0;   // entries past st read as 0
             if (coeff_out)
                 for (int j = lane; j < RM; j += 32)
                     coeff_out[o * RM + j] = j < R ? *reinterpret_cast<const __nv_bfloat16*>(
                                                         blk + (j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2)
                                                   : __float2bfloat16_rn(0.f);
             for (int e = lane; e < s; e += 32) {
-                if (idx_out) idx_out[o * s + e] = ok ? blk[off_idx_of(R) + dst.row * s + e] : 0;
+                const bool on = e < st;
+                if (idx_out) idx_out[o * s + e] = on ? blk[off_idx_of(R) + dst.row * st + e] : 0;
                 if (codes_out) {
                     int c = 0;
-                    if (ok) {
-                        if (BITS == 8) c = (int8_t)blk[off_codes_of(R, s) + dst.row * s + e];
+                    if (on) {
+                        if (BITS == 8) c = (int8_t)blk[off_codes_of(R, st) + dst.row * st + e];
                         else {
-                            const uint32_t byte = blk[off_codes_of(R, s) + dst.row * (s / 2) + e / 2];
+                            const uint32_t byte = blk[off_codes_of(R, st) + dst.row * (st / 2) + e / 2];
                             const uint32_t nib = (e & 1) ? (byte >> 4) : (byte & 0xfu);
                             c = (int)(nib ^ 8u) - 8;
                         }
@@ -583,7 +582,7 @@ __global__ void __launch_bounds__(256) export_kernel(const Geom G, const State S
                 }
             }
             if (scales_out && lane == 0)
-                scales_out[o] = ok ? *reinterpret_cast<const __half*>(blk + off_scales_of(R, s, BITS) + dst.row * 2)
+                scales_out[o] = st ? *reinterpret_cast<const __half*>(blk + off_scales_of(R, st, BITS) + dst.row * 2)
                                    : __float2half_rn(0.f);
         }
     }
@@ -719,7 +718,7 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
         __syncthreads();
         if (!s_go) continue;
         const int kold = s_kold, knew = s_knew, slot = s_slot, last = s_last;
-        const int Rold = G.tiers[kold], row = slot % kPage;
+        const int Rold = G.tiers[kold], sold = G.ts[kold], row = slot % kPage;
         // ---- 2: re-encode every (layer, K / V) unit of the token, a warp each
         for (int u = warp; u < 2 * G.LPG; u += (int)(blockDim.x >> 5)) {
             const int lig = u >> 1, z = u & 1;
@@ -734,15 +733,15 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
                 for (int m = 0; m < 4; ++m)
                     a[m] = __fmaf_rn(__bfloat162float(bz[(size_t)(lane + 32 * m) * P + j]), cj, a[m]);
             }
-            if (G.s > 0) {
-                const float sf = __half2float(*reinterpret_cast<const __half*>(ob + off_scales_of(Rold, G.s, BITS) + row * 2));
-                for (int e = 0; e < G.s; ++e) {
-                    const int ch = ob[off_idx_of(Rold) + row * G.s + e];
+            if (sold > 0) {
+                const float sf = __half2float(*reinterpret_cast<const __half*>(ob + off_scales_of(Rold, sold, BITS) + row * 2));
+                for (int e = 0; e < sold; ++e) {
+                    const int ch = ob[off_idx_of(Rold) + row * sold + e];
                     int code;
                     if (BITS == 8) {
-                        code = (int8_t)ob[off_codes_of(Rold, G.s) + row * G.s + e];
+                        code = (int8_t)ob[off_codes_of(Rold, sold) + row * sold + e];
                     } else {
-                        const uint32_t byte = ob[off_codes_of(Rold, G.s) + row * (G.s / 2) + (e >> 1)];
+                        const uint32_t byte = ob[off_codes_of(Rold, sold) + row * (sold / 2) + (e >> 1)];
                         code = (int)(((e & 1) ? byte >> 4 : byte) & 0xfu);
                         code = (code ^ 8) - 8;
                     }
@@ -769,7 +768,7 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
             const int lrow = last % kPage;
             const uint32_t blk = G.blk_bytes[kold];
             const uint32_t coff = off_idx_of(Rold);
-            const uint32_t nidx = (uint32_t)G.s, ncode = (uint32_t)G.s * BITS / 8;
+            const uint32_t nidx = (uint32_t)sold, ncode = (uint32_t)sold * BITS / 8;
             for (int u = warp; u < 2 * G.LPG; u += (int)(blockDim.x >> 5)) {
                 const int lig = u >> 1, z = u & 1;
                 uint8_t* dst = S.data + (size_t)s_unit_old * kUnit + (size_t)lig * G.chunk_bytes[kold] + (z ? blk : 0u);
@@ -778,10 +777,10 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
                     *reinterpret_cast<uint4*>(dst + (size_t)c * 1024 + row * 16) =
                         *reinterpret_cast<const uint4*>(src + (size_t)c * 1024 + lrow * 16);
                 for (uint32_t b = lane; b < nidx; b += 32) dst[coff + row * nidx + b] = src[coff + lrow * nidx + b];
-                const uint32_t qo = off_codes_of(Rold, G.s);
+                const uint32_t qo = off_codes_of(Rold, sold);
                 for (uint32_t b = lane; b < ncode; b += 32) dst[qo + row * ncode + b] = src[qo + lrow * ncode + b];
                 if (lane == 0) {
-                    const uint32_t so = off_scales_of(Rold, G.s, BITS);
+                    const uint32_t so = off_scales_of(Rold, sold, BITS);
                     *reinterpret_cast<uint16_t*>(dst + so + row * 2) = *reinterpret_cast<const uint16_t*>(src + so + lrow * 2);
                 }
             }

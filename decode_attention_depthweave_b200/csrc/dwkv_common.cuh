@@ -12,7 +12,8 @@
 //                                                  the tcgen05 / ldmatrix "core matrix"
 //                                                  order, conflict-free for per-token reads)
 //       idx    [64][s]    uint8      64*s
-//       codes  [64][s*b/8]           8*s*b        (int4: even slot in the low nibble)
+//       codes  [64][s*b/8]           8*s*b        (int4: even slot in the low nibble; the part
+//                                                  padded to 128 bytes when shorter)
 //       scales [64]       fp16       128
 //     Every part is a multiple of 128 bytes, so pages are 128-byte aligned and every page
 //     chunk is a legal bulk-copy (TMA) source.
@@ -45,6 +46,8 @@ constexpr int kRdBytes = 128 * 32;                         // dense residual til
 struct Geom {
     int L, LPG, G, Hq, Hkv, d, r_max, ntiers, s, bits, max_batch, max_context, max_pages;
     int tiers[kMaxTiers];
+    int ts[kMaxTiers];               // residual channels a token of each tier keeps (<= s; s when not routed)
+    int routed;                      // 1: per-tier residual counts (every tier at one basis rank)
     float tau;                       // softmax scale
     uint32_t blk_bytes[kMaxTiers];   // one (layer, K or V) block of a page
     uint32_t chunk_bytes[kMaxTiers]; // one layer of a page: K block + V block
@@ -119,13 +122,15 @@ struct DecodeCall {
 };
 
 // ------------------------------------------------------------------------------ layout
+// The code part rounded up to 128 bytes (only 2 int4 codes a token, 64 bytes, needs it).
+__host__ __device__ inline uint32_t code_part_bytes(int s, int bits) { return (8u * s * bits + 127u) & ~127u; }
 __host__ __device__ inline uint32_t blk_bytes_of(int R, int s, int bits) {
-    return 128u * R + 64u * s + 8u * s * bits + 128u;
+    return 128u * R + 64u * s + code_part_bytes(s, bits) + 128u;
 }
 __host__ __device__ inline uint32_t off_idx_of(int R) { return 128u * R; }
 __host__ __device__ inline uint32_t off_codes_of(int R, int s) { return 128u * R + 64u * s; }
 __host__ __device__ inline uint32_t off_scales_of(int R, int s, int bits) {
-    return 128u * R + 64u * s + 8u * s * bits;
+    return 128u * R + 64u * s + code_part_bytes(s, bits);
 }
 // Byte offset of a page's slot-position block (after the layers' chunks).
 __host__ __device__ inline uint32_t pos_block_of(const Geom& G, int k) { return (uint32_t)G.LPG * G.chunk_bytes[k]; }

@@ -100,6 +100,28 @@ __device__ __forceinline__ void ld_row(const uint8_t* p, uint32_t (&w)[NB / 4 > 
     }
 }
 
+// A row of n in {1, 2, 4, 8} bytes (aligned to its size) into one or two words.
+__device__ __forceinline__ void load_small_row(const uint8_t* p, int n, uint32_t& w0, uint32_t& w1) {
+    if (n == 8) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        w0 = v.x;
+        w1 = v.y;
+    } else if (n == 4) {
+        w0 = *reinterpret_cast<const uint32_t*>(p);
+    } else if (n == 2) {
+        w0 = *reinterpret_cast<const uint16_t*>(p);
+    } else if (n == 1) {
+        w0 = *p;
+    }
+}
+// Code e of a row of at most 8 codes held in (w0, w1): int8 bytes, or int4 nibbles with the
+// even slot low.
+template <int BITS>
+__device__ __forceinline__ float small_code(uint32_t w0, uint32_t w1, int e) {
+    if (BITS == 8) return (float)(int8_t)__byte_perm(e < 4 ? w0 : w1, 0u, 0x4440 + (e & 3));
+    return (float)((int32_t)(w0 << (28 - 4 * e)) >> 28);
+}
+
 // Score buffer of a half page: the hi and lo column halves as two [32 tokens][4 heads] fp32
 // blocks, the second 16 floats further on so that the stores of both halves from one MMA
 // fragment fall in distinct banks.
@@ -132,14 +154,19 @@ constexpr uint32_t kWbPitch = 48;
 
 // One warp's half of a tier-R page: tokens [32*half, 32*half + 32) of the page's 64 slots,
 // `nv` of them live.  `K` points at the page chunk's key block.
+// S >= 0: every token has S residual channels.  S < 0 (routed residual counts): the page's
+// tokens have s_rt in {0, 2, 4, 8}.
 template <int R, int S, int BITS, bool PROBE, int RMAX>
 __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int half, int nv,
                                           const uint32_t (&qb)[RMAX / 16][2], const uint2* __restrict__ qh,
                                           float qscale, uint8_t* small, uint8_t* rd, uint32_t zero_addr,
-                                          WarpAcc<RMAX, PROBE>& A, int lane) {
+                                          WarpAcc<RMAX, PROBE>& A, int lane, int s_rt) {
+    constexpr bool ROUTED = S < 0;
     constexpr int KS = R >= 16 ? R / 16 : 1;         // 16-wide coefficient steps
-    constexpr uint32_t kOffIdx = 128u * R, kOffCodes = kOffIdx + 64u * S, kOffSc = kOffCodes + 8u * S * BITS;
-    constexpr uint32_t kBlk = kOffSc + 128u;
+    const int s_ = ROUTED ? s_rt : S;                // residual channels of this page's tokens
+    const uint32_t kOffIdx = 128u * R, kOffCodes = kOffIdx + 64u * s_;
+    const uint32_t kOffSc = kOffCodes + ((8u * s_ * BITS + 127u) & ~127u);
+    const uint32_t kBlk = kOffSc + 128u;
     const uint8_t* V = K + kBlk;
     const int tb = 32 * half;
     const uint32_t kaddr = smem_addr(K), vaddr = smem_addr(V);
@@ -193,15 +220,36 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
         __syncwarp();                                   // S is dead from here (P overwrites it)
         if (live) {
             float ra[kGQ] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (ROUTED) {
+                // a page of the routed layout: s_ in {0, 2, 4, 8} channels a token, each row in one load
+                if (s_ > 0) {
+                    uint32_t i0 = 0, i1 = 0, c0 = 0, c1 = 0;
+                    load_small_row(K + kOffIdx + t * s_, s_, i0, i1);
+                    load_small_row(K + kOffCodes + t * (s_ * BITS / 8), s_ * BITS / 8, c0, c1);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        if (e < s_) {
+                            const uint32_t i = __byte_perm(e < 4 ? i0 : i1, 0u, 0x4440 + (e & 3));
+                            const float cf = small_code<BITS>(c0, c1, e);
+                            const uint2 q = qh[i];
+                            ra[0] = fmaf(bf16lo(q.x), cf, ra[0]);
+                            ra[1] = fmaf(bf16hi(q.x), cf, ra[1]);
+                            ra[2] = fmaf(bf16lo(q.y), cf, ra[2]);
+                            ra[3] = fmaf(bf16hi(q.y), cf, ra[3]);
+                        }
+                    }
+                }
+            }
             // the token's channel indices and codes, each row in one or two vector loads
-            constexpr int kCB = S * BITS / 8;
-            uint32_t ixw[S / 4 > 0 ? S / 4 : 1], cw[kCB / 4 > 0 ? kCB / 4 : 1];
-            if (S) {
-                ld_row<S>(K + kOffIdx + t * S, ixw);
+            constexpr int SF = ROUTED ? 0 : S;
+            constexpr int kCB = SF * BITS / 8;
+            uint32_t ixw[SF / 4 > 0 ? SF / 4 : 1], cw[kCB / 4 > 0 ? kCB / 4 : 1];
+            if (SF) {
+                ld_row<SF>(K + kOffIdx + t * SF, ixw);
                 ld_row<kCB>(K + kOffCodes + t * kCB, cw);
             }
 #pragma unroll
-            for (int ch = 0; ch < S; ch += 8) {
+            for (int ch = 0; ch < SF; ch += 8) {
                 const uint2 ix = make_uint2(ixw[ch / 4], ixw[ch / 4 + 1]);
                 // codes as biased bytes (code + 2^(b-1)), each turned into a float by placing it in
                 // the mantissa of 2^23 and subtracting 2^23 + 2^(b-1)
@@ -229,7 +277,7 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 }
             }
             const float scale =
-                S ? __half2float(*reinterpret_cast<const __half*>(K + kOffSc + t * 2)) * qscale : 0.f;
+                s_ ? __half2float(*reinterpret_cast<const __half*>(K + kOffSc + t * 2)) * qscale : 0.f;
             sc[0] = fmaf(scale, ra[0], sv.x);
             sc[1] = fmaf(scale, ra[1], sv.y);
             sc[2] = fmaf(scale, ra[2], sv.z);
@@ -275,7 +323,7 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
         split2(p[0], p[1], pr.x, pr.z);
         split2(p[2], p[3], pr.y, pr.w);
         *reinterpret_cast<uint4*>(Psm + lane * 16) = pr;
-        if (S) {
+        if (s_) {
             // w = p * scale^V as 16-bit fixed point per head, in units of 2^(E-15) with E the
             // exponent of the half page's largest w: two byte limbs (hi, lo) per head
             const float scv = live ? __half2float(*reinterpret_cast<const __half*>(V + kOffSc + t * 2)) : 0.f;
@@ -344,15 +392,32 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
 
     // ---------------- 5. residual-space values: acc_r[ch][h] += sum_t R^V[t][ch] w[t][h] as one
     //                     integer MMA per 16 channels over the half page's 32 tokens
-    if (S) {
-        if (lane < nv) {                                // scatter this token's codes (lane = token)
+    if (s_) {
+        if (lane < nv && ROUTED) {                      // scatter this token's codes (lane = token)
             const int tok = tb + lane;
-            constexpr int kCB = S * BITS / 8;
-            uint32_t ixw[S / 4 > 0 ? S / 4 : 1], cw[kCB / 4 > 0 ? kCB / 4 : 1];
-            ld_row<S>(V + kOffIdx + tok * S, ixw);
+            uint32_t i0 = 0, i1 = 0, c0 = 0, c1 = 0;
+            load_small_row(V + kOffIdx + tok * s_, s_, i0, i1);
+            load_small_row(V + kOffCodes + tok * (s_ * BITS / 8), s_ * BITS / 8, c0, c1);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                if (e < s_) {
+                    const uint32_t ch = __byte_perm(e < 4 ? i0 : i1, 0u, 0x4440 + (e & 3));
+                    // int8 codes as stored, int4 codes as 16 x code (see code_bytes)
+                    const uint32_t v = BITS == 8 ? __byte_perm(e < 4 ? c0 : c1, 0u, 0x4440 + (e & 3))
+                                                 : ((c0 >> (4 * e)) & 0xfu) << 4;
+                    rd[rd_off(ch, (uint32_t)lane)] = (uint8_t)v;
+                }
+            }
+        }
+        if (lane < nv && !ROUTED) {                     // scatter this token's codes (lane = token)
+            const int tok = tb + lane;
+            constexpr int SF = ROUTED ? 0 : S;
+            constexpr int kCB = SF * BITS / 8;
+            uint32_t ixw[SF / 4 > 0 ? SF / 4 : 1], cw[kCB / 4 > 0 ? kCB / 4 : 1];
+            ld_row<SF>(V + kOffIdx + tok * SF, ixw);
             ld_row<kCB>(V + kOffCodes + tok * kCB, cw);
 #pragma unroll
-            for (int e = 0; e < S; e += 4) {
+            for (int e = 0; e < SF; e += 4) {
                 const uint32_t ix = ixw[e / 4];
                 const uint32_t cbw = code_bytes<BITS>(BITS == 8 ? cw[e / 4] : (cw[e / 8] >> (16 * ((e / 4) & 1))) & 0xffffu);
 #pragma unroll
@@ -389,14 +454,15 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
 template <int S, int BITS, bool PROBE, int RMAX>
 __device__ __forceinline__ void run_page(int R, const uint8_t* K, int half, int nv, const uint32_t (&qb)[RMAX / 16][2],
                                          const uint2* qs, float qscale, uint8_t* small, uint8_t* rd, uint32_t zero_addr,
-                                         WarpAcc<RMAX, PROBE>& A, int lane) {
+                                         WarpAcc<RMAX, PROBE>& A, int lane, int s_rt) {
     switch (R) {
-        case 8: half_page<8, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane); break;
-        case 16: half_page<16, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane); break;
-        case 32: half_page<32, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane); break;
-        case 64: half_page<64, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane); break;
+        case 8: half_page<8, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt); break;
+        case 16: half_page<16, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt); break;
+        case 32: half_page<32, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt); break;
+        case 64: half_page<64, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt); break;
         case 128:
-            if constexpr (RMAX >= 128) half_page<128, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane);
+            if constexpr (RMAX >= 128)
+                half_page<128, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt);
             break;
         default: break;
     }
@@ -484,15 +550,16 @@ __device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, 
                                               WarpAcc<RMAX, false>& A, int lane) {
     const Dest& d = td.d;
     const int R = d.R, row = d.row;
-    const uint32_t offIdx = off_idx_of(R), offCodes = off_codes_of(R, S), offSc = off_scales_of(R, S, BITS);
+    const int s_ = S < 0 ? G.ts[d.k] : S;            // the token's residual channels
+    const uint32_t offIdx = off_idx_of(R), offCodes = off_codes_of(R, s_), offSc = off_scales_of(R, s_, BITS);
     const uint8_t* Kb = d.blk;
     const uint8_t* Vb = d.blk + G.blk_bytes[d.k];
     auto coeff = [&](const uint8_t* blk, int j) {
         return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(blk + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2));
     };
     auto code = [&](const uint8_t* blk, int e) -> float {
-        if (BITS == 8) return (float)(int8_t)blk[offCodes + row * S + e];
-        const uint32_t b = blk[offCodes + row * (S / 2) + e / 2];
+        if (BITS == 8) return (float)(int8_t)blk[offCodes + row * s_ + e];
+        const uint32_t b = blk[offCodes + row * (s_ / 2) + e / 2];
         return (float)((int32_t)(b << (28 - 4 * (e & 1))) >> 28);
     };
     // score (log2 units: q~ and q carry tau log2 e)
@@ -503,12 +570,12 @@ __device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, 
         sc[0] = fmaf(t.x, c, sc[0]); sc[1] = fmaf(t.y, c, sc[1]);
         sc[2] = fmaf(t.z, c, sc[2]); sc[3] = fmaf(t.w, c, sc[3]);
     }
-    if (S && lane < S) {
+    if (s_ && lane < s_) {
         const float cf = code(Kb, lane);
-        const float4 q = qs[Kb[offIdx + row * S + lane]];
+        const float4 q = qs[Kb[offIdx + row * s_ + lane]];
         rs[0] = q.x * cf; rs[1] = q.y * cf; rs[2] = q.z * cf; rs[3] = q.w * cf;
     }
-    const float scK = S ? __half2float(*reinterpret_cast<const __half*>(Kb + offSc + row * 2)) : 0.f;
+    const float scK = s_ ? __half2float(*reinterpret_cast<const __half*>(Kb + offSc + row * 2)) : 0.f;
     float s_t[kGQ];
 #pragma unroll
     for (int hh = 0; hh < kGQ; ++hh) s_t[hh] = fmaf(scK, warp_sum(rs[hh]), warp_sum(sc[hh]));
@@ -555,11 +622,11 @@ __device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, 
         }
     }
     // values, residual space: channel ch sits in row (ch & 15) of tile ch >> 4, at lanes g = ch & 7
-    if (S) {
+    if (s_) {
         const float scV = __half2float(*reinterpret_cast<const __half*>(Vb + offSc + row * 2));
         const float pc = p[c] * scV;
-        for (int e = 0; e < S; ++e) {
-            const int ch = Vb[offIdx + row * S + e];
+        for (int e = 0; e < s_; ++e) {
+            const int ch = Vb[offIdx + row * s_ + e];
             if ((ch & 7) != g) continue;
             const float v = pc * code(Vb, e);
             const int mt = ch >> 4, r2 = (ch >> 3) & 1;
@@ -573,7 +640,7 @@ __device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, 
 }  // namespace decode_detail
 
 // BITS: code width; PROBE: second softmax state without the residual; RMAX: accumulator
-// rows (>= r_max); S: residual channels per token (0, 8, 16 or 32).
+// rows (>= r_max); S: residual channels per token (0, 8, 16 or 32), or -1 for per-tier counts.
 template <int BITS, bool PROBE, int RMAX, int S>
 __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G, const State St, const DecodeCall C) {
     using namespace decode_detail;
@@ -906,7 +973,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             const int nv = min(max(nvalid - 32 * half, 0), 32);
             if (nv > 0)
                 run_page<S, BITS, PROBE, RMAX>(R, smem + L.ring + m_slot[sl], half, nv, qb, qh,
-                                               qscale, small, rd, zero_addr, A, lane);
+                                               qscale, small, rd, zero_addr, A, lane, G.ts[k]);
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8 * sl);
             if (wn == 0xffffffffu) {
@@ -1202,7 +1269,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
 
 }  // namespace dwkv
 
-// Explicit instantiations for one (BITS, PROBE) pair: RMAX in {64, 128}, S in {0, 8, 16, 32}.
+// Explicit instantiations for one (BITS, PROBE) pair: RMAX in {64, 128}, S in {0, 8, 16, 32}
+// and -1 (routed residual counts).
 #define DWKV_DECODE_INSTANTIATE(B, P)                                                        \
     namespace dwkv {                                                                          \
     template __global__ void decode_kernel<B, P, 64, 0>(const Geom, const State, const DecodeCall);   \
@@ -1213,4 +1281,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     template __global__ void decode_kernel<B, P, 128, 8>(const Geom, const State, const DecodeCall);  \
     template __global__ void decode_kernel<B, P, 128, 16>(const Geom, const State, const DecodeCall); \
     template __global__ void decode_kernel<B, P, 128, 32>(const Geom, const State, const DecodeCall); \
+    template __global__ void decode_kernel<B, P, 64, -1>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 128, -1>(const Geom, const State, const DecodeCall); \
     }

@@ -155,8 +155,8 @@ static __device__ __noinline__ uint32_t select_exact(float r0, float r1, float r
 
 // Steps 4-6 of one vector on one warp, from its residual r (channel lane + 32 m): top-s
 // selection, scale, codes, and the stores of indices, codes and scale into the vector's block
-// (blk: this vector's K or V block, row: its row in the page).  rstage / chstage: s floats
-// and s bytes of the warp's shared memory.
+// (blk: this vector's K or V block, row: its row in the page, s: the residual channels its
+// tier keeps).  rstage / chstage: s floats and s bytes of the warp's shared memory.
 //
 // Selection: each channel gets a 32-bit key, its |r| with the 7 lowest mantissa bits replaced
 // by 127 - channel.  The keys are distinct, and ordering them orders |r| at 2^-16 relative
@@ -166,10 +166,9 @@ static __device__ __noinline__ uint32_t select_exact(float r0, float r1, float r
 // other one, so the set equals the exact top-s; otherwise (a near-tie at the boundary, e.g.
 // exact zeros) the selection is redone by its definition (select_exact).
 template <int BITS>
-__device__ __forceinline__ void quantize_store(const Geom& G, const float (&r)[4], uint8_t* blk, int R, int row,
+__device__ __forceinline__ void quantize_store(const float (&r)[4], uint8_t* blk, int R, int row, int s,
                                                float* rstage, uint8_t* chstage) {
     const int lane = threadIdx.x & 31;
-    const int s = G.s;
     const float qmax = BITS == 8 ? 127.f : 7.f;
     uint32_t sel = 0u, mxb = 0u;
     if (s > 0) {
@@ -308,7 +307,7 @@ __device__ __forceinline__ void encode_body(const Geom& G, const State& S, const
 #pragma unroll
             for (int m = 0; m < 4; ++m) r[m] = __fsub_rn(xr[m], a[m]);
         }
-        quantize_store<BITS>(G, r, blk, R, dst.row, xs, reinterpret_cast<uint8_t*>(cstage));
+        quantize_store<BITS>(r, blk, R, dst.row, G.ts[dst.k], xs, reinterpret_cast<uint8_t*>(cstage));
     } while (false);
     __syncwarp();
 }

@@ -98,6 +98,13 @@ typedef struct {
     int32_t max_batch;         /* sequence slots: ids 0 .. max_batch-1                  */
     int32_t max_context;       /* tokens per sequence                                   */
     float softmax_scale;       /* <= 0 selects 1/sqrt(head_dim)                         */
+    /* Residual-count routing ([DW] §3 Eq. (2): the router's level rho is the number of
+     * residual channels a token keeps, at a fixed basis rank).  0: every tier keeps
+     * resid_channels channels.  1: tier k keeps tier_resid[k] of {0, 2, 4, 8} channels; every
+     * tier then has the same rank (tiers[k] all equal), tier_resid strictly ascending, and
+     * resid_channels == 8 (the stride of the residual arrays of append_compressed / export). */
+    int32_t resid_routed;
+    int32_t tier_resid[DWKV_MAX_TIERS];
 } dwkv_config;
 
 /* Library version string. */
@@ -110,7 +117,8 @@ const char* dwkv_last_error(void);
 dwkv_status dwkv_config_check(const dwkv_config* cfg);
 
 /* Bytes of one stored token (one layer, one kv-head, keys + values) at tier index
- * `tier`: 2 * (2*r + s + s*bits/8 + 2).  0 if the arguments are invalid. */
+ * `tier`: 2 * (2*r + s + s*bits/8 + 2), s the tier's residual channels.  0 if the arguments
+ * are invalid. */
 size_t dwkv_token_bytes(const dwkv_config* cfg, int32_t tier);
 
 /* Bytes of one page of tier `tier`: DWKV_PAGE_TOKENS tokens of one (sequence, group,

@@ -45,7 +45,7 @@ def lib():
         L.oracle_encode_many.restype = i
         L.oracle_encode_many_from_coeffs.argtypes = [i, i, i, p, p, p, p, i, i, p, p, p, p, i, p]
         L.oracle_encode_many_from_coeffs.restype = i
-        L.oracle_reencode_vector.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, i, p, p, p, p, p]
+        L.oracle_reencode_vector.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, i, i, p, p, p, p, p]
         L.oracle_reencode_vector.restype = i
         L.oracle_reconstruct.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, p]
         L.oracle_reconstruct.restype = None
@@ -298,9 +298,10 @@ def encode_many(basis, x, ranks, s, bits, nthreads=None, want_c32=False, nres=No
     return out
 
 
-def reencode_vector(basis, r_old, coeff, idx, codes, scale, r_new, bits):
-    """Re-tier one stored vector: re-encode its bf16-rounded reconstruction at rank r_new
-    (``oracle_reencode_vector``).  Returns the encode dict plus ``xh`` (bf16 bits [d])."""
+def reencode_vector(basis, r_old, coeff, idx, codes, scale, r_new, bits, s_new=None):
+    """Re-tier one stored vector: re-encode its bf16-rounded reconstruction at rank r_new with
+    s_new residual channels (default: as many as stored) (``oracle_reencode_vector``).  Returns
+    the encode dict plus ``xh`` (bf16 bits [d])."""
     b = _bits16(basis)
     d, r_max = b.shape
     c = _bits16(coeff).reshape(r_max)
@@ -308,13 +309,14 @@ def reencode_vector(basis, r_old, coeff, idx, codes, scale, r_new, bits):
     cd = _arr(codes, np.int8).reshape(-1)
     s = ix.size
     sc = int(_bits16(scale).reshape(-1)[0])
+    sn = s if s_new is None else int(s_new)
     out_c = np.zeros(r_max, np.uint16)
-    out_i = np.zeros(s, np.uint8)
-    out_q = np.zeros(s, np.int8)
+    out_i = np.zeros(sn, np.uint8)
+    out_q = np.zeros(sn, np.int8)
     out_s = np.zeros(1, np.uint16)
     xh = np.zeros(d, np.uint16)
-    rc = lib().oracle_reencode_vector(d, r_max, _p(b), int(r_old), _p(c), s, _p(ix), _p(cd), sc, int(r_new), int(bits),
-                                      _p(out_c), _p(out_i), _p(out_q), _p(out_s), _p(xh))
+    rc = lib().oracle_reencode_vector(d, r_max, _p(b), int(r_old), _p(c), s, _p(ix), _p(cd), sc, int(r_new), sn,
+                                      int(bits), _p(out_c), _p(out_i), _p(out_q), _p(out_s), _p(xh))
     if rc != 0:
         raise ValueError("oracle_reencode_vector: bad arguments")
     return {"coeff": out_c, "idx": out_i, "codes": out_q, "scale": out_s[0], "xh": xh}

@@ -364,15 +364,19 @@ int oracle_encode_many(int n, int d, int r_max, const uint16_t* basis, const uin
 /*   a_i  = fma chain over j = 0..r_old-1 of B[i][j] * cb_j from +0      (fp32)            */
 /*   xh_i = bf16_rn(a_i + scale * code_i) for the stored residual channels, bf16_rn(a_i)    */
 /*          for the others (scale * code is exact in fp32; one rounding in the add)         */
-/* then the six encode steps of oracle_encode_vector on xh at rank r_new.                  */
+/* then the six encode steps of oracle_encode_vector on xh at rank r_new with s_new        */
+/* residual channels (a tier of the residual-count routing reading keeps its own count;     */
+/* otherwise s_new = s).                                                                    */
 /* Inputs: the stored coeff (bf16 [r_max], entries >= r_old ignored), idx / codes [s],      */
-/* scale (fp16 bits).  Outputs as oracle_encode_vector; xh_out (nullable) bf16 bits [d].    */
+/* scale (fp16 bits).  Outputs as oracle_encode_vector (idx / codes [s_new]); xh_out        */
+/* (nullable) bf16 bits [d].                                                                */
 /* ------------------------------------------------------------------------------------ */
 int oracle_reencode_vector(int d, int r_max, const uint16_t* basis, int r_old, const uint16_t* coeff_old,
                            int s, const uint8_t* idx_old, const int8_t* codes_old, uint16_t scale_old,
-                           int r_new, int bits, uint16_t* coeff, uint8_t* idx, int8_t* codes,
+                           int r_new, int s_new, int bits, uint16_t* coeff, uint8_t* idx, int8_t* codes,
                            uint16_t* scale, uint16_t* xh_out) {
-    if (d <= 0 || d > 256 || r_old < 0 || r_old > r_max || r_new < 0 || r_new > r_max || s < 0 || s > d)
+    if (d <= 0 || d > 256 || r_old < 0 || r_old > r_max || r_new < 0 || r_new > r_max || s < 0 || s > d ||
+        s_new < 0 || s_new > d)
         return -1;
     float a[256];
     uint16_t xh[256];
@@ -392,7 +396,7 @@ int oracle_reencode_vector(int d, int r_max, const uint16_t* basis, int r_old, c
         xh[i] = oracle_f32_to_bf16_rn(a[i]);
         if (xh_out) xh_out[i] = xh[i];
     }
-    return oracle_encode_vector(d, r_max, basis, xh, r_new, s, bits, coeff, NULL, idx, codes, scale, NULL);
+    return oracle_encode_vector(d, r_max, basis, xh, r_new, s_new, bits, coeff, NULL, idx, codes, scale, NULL);
 }
 
 /* Element-wise format conversions over arrays (used to pin the converters). */

@@ -59,6 +59,7 @@ class Workload:
     outlier_var: float = 0.0
     noise_var: float = 0.0
     resid_var: float = 0.05           # scale drawn from max |N(0, resid_var)| / qmax
+    tier_resid: tuple = ()            # per-tier residual counts (every tier at one rank), or ()
     extra: dict = field(default_factory=dict)
 
     @property
@@ -73,7 +74,7 @@ class Workload:
         return replace(self, **kw)
 
 
-# The five workloads.  Names say what they are; sizes are the full ones.
+# The workloads.  Names say what they are; sizes are the full ones.
 WORKLOADS = {
     "tiny_1k": Workload(
         name="tiny_1k", num_layers=2, layers_per_group=2, num_q_heads=4, num_kv_heads=1,
@@ -95,6 +96,11 @@ WORKLOADS = {
         tier_probs=(0.4, 0.3, 0.15, 0.1, 0.05), resid_channels=8, resid_bits=4, batch=1,
         context=131072, span_tier=4, num_spans=3, span_len=256, base_seed=1004,
         coeff_var_rank=128, noise_var=0.01),
+    "llama8b_routed_64k": Workload(
+        name="llama8b_routed_64k", num_layers=32, layers_per_group=2, num_q_heads=32, num_kv_heads=8,
+        head_dim=128, r_max=32, tiers=(32, 32, 32, 32), tier_probs=(0.4, 0.3, 0.2, 0.1),
+        resid_channels=8, resid_bits=4, batch=1, context=65536, base_seed=1006,
+        coeff_var_rank=32, noise_var=0.01, tier_resid=(0, 2, 4, 8)),
     "llama8b_encode_16k": Workload(
         name="llama8b_encode_16k", num_layers=32, layers_per_group=2, num_q_heads=32,
         num_kv_heads=8, head_dim=128, r_max=64, tiers=(16, 32, 64), tier_probs=(0.6, 0.3, 0.1),
@@ -198,6 +204,14 @@ def ranks_of(wl: Workload, tier_idx: torch.Tensor) -> torch.Tensor:
     return torch.tensor(wl.tiers, dtype=torch.int32, device=tier_idx.device)[tier_idx.long()]
 
 
+def resid_counts_of(wl: Workload, tier_idx: torch.Tensor) -> torch.Tensor:
+    """Residual channels each token keeps (a table lookup, ``int32``): ``wl.tier_resid`` of its
+    tier, or ``wl.resid_channels`` for every token without per-tier counts."""
+    if not wl.tier_resid:
+        return torch.full(tier_idx.shape, wl.resid_channels, dtype=torch.int32, device=tier_idx.device)
+    return torch.tensor(wl.tier_resid, dtype=torch.int32, device=tier_idx.device)[tier_idx.long()]
+
+
 def make_compressed(wl: Workload, seq: int, layer: int, tier_idx: torch.Tensor,
                     device="cpu", seed: int | None = None, garbage_tail: bool = False,
                     start: int = 0) -> dict:
@@ -212,6 +226,10 @@ def make_compressed(wl: Workload, seq: int, layer: int, tier_idx: torch.Tensor,
     * ``codes``  int8 ``[n][Hkv][2][s]``: a discretised Gaussian, round(N(0, (qmax/2.5)^2))
       clipped to [-qmax, qmax].
     * ``scales`` fp16 ``[n][Hkv][2]``: max_i |N(0, resid_var)| over s draws, divided by qmax.
+
+    With per-tier residual counts (``wl.tier_resid``) a token of tier k keeps the first
+    ``tier_resid[k]`` entries of idx / codes; the entries past them are zero (the scale too
+    when the count is 0), or left as drawn with ``garbage_tail`` (they must be ignored).
     """
     seed = wl.base_seed if seed is None else seed
     n = tier_idx.shape[0]
@@ -240,6 +258,12 @@ def make_compressed(wl: Workload, seq: int, layer: int, tier_idx: torch.Tensor,
         idx = torch.zeros(n, H, 2, 0, dtype=torch.uint8, device=device)
         codes = torch.zeros(n, H, 2, 0, dtype=torch.int8, device=device)
         scales = torch.zeros(n, H, 2, dtype=torch.float16, device=device)
+    if wl.tier_resid and not garbage_tail:
+        nres = resid_counts_of(wl, tier_idx)                           # [n][H]
+        on = torch.arange(s, device=device).view(1, 1, 1, s) < nres.view(n, H, 1, 1)
+        idx = idx * on
+        codes = codes * on
+        scales = scales * (nres.view(n, H, 1) > 0)
     return {"coeff": coeff, "idx": idx, "codes": codes, "scales": scales}
 
 

@@ -79,7 +79,8 @@ def cfg_for(wl, max_batch=None, max_context=None, softmax_scale=0.0):
         num_layers=wl.num_layers, layers_per_group=wl.layers_per_group, num_q_heads=wl.num_q_heads,
         num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, r_max=wl.r_max, tiers=wl.tiers,
         resid_channels=wl.resid_channels, resid_bits=wl.resid_bits,
-        max_batch=max_batch or wl.batch, max_context=max_context or wl.context, softmax_scale=softmax_scale)
+        max_batch=max_batch or wl.batch, max_context=max_context or wl.context, softmax_scale=softmax_scale,
+        tier_resid=wl.tier_resid or None)
 
 
 def to_dev(d: dict, device="cuda") -> dict:
@@ -124,6 +125,7 @@ def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None, c32=None
     k, v, tier_idx = k.cpu(), v.cpu(), tier_idx.cpu()
     n, H, s = k.shape[0], wl.num_kv_heads, wl.resid_channels
     ranks = synth.ranks_of(wl, tier_idx)
+    nres = synth.resid_counts_of(wl, tier_idx) if wl.tier_resid else None
     coeff = np.zeros((n, H, 2, wl.r_max), np.uint16)
     idx = np.zeros((n, H, 2, s), np.uint8)
     codes = np.zeros((n, H, 2, s), np.int8)
@@ -134,9 +136,10 @@ def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None, c32=None
         for z, x in enumerate((k, v)):
             if c32 is not None:
                 r = oracle.encode_many_from_coeffs(bases[z][g, h], x[:, h], c32[:, h, z], ranks[:, h], s, wl.resid_bits,
-                                                   nthreads=nthreads)
+                                                   nthreads=nthreads, nres=None if nres is None else nres[:, h])
             else:
-                r = oracle.encode_many(bases[z][g, h], x[:, h], ranks[:, h], s, wl.resid_bits, nthreads=nthreads)
+                r = oracle.encode_many(bases[z][g, h], x[:, h], ranks[:, h], s, wl.resid_bits, nthreads=nthreads,
+                                       nres=None if nres is None else nres[:, h])
             coeff[:, h, z], idx[:, h, z], codes[:, h, z], scales[:, h, z] = r["coeff"], r["idx"], r["codes"], r["scale"]
     return {"coeff": torch.from_numpy(coeff.view(np.int16)).view(torch.bfloat16),
             "idx": torch.from_numpy(idx), "codes": torch.from_numpy(codes),

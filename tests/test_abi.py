@@ -32,7 +32,7 @@ def _cfg(wl, **over):
     kw = dict(num_layers=wl.num_layers, layers_per_group=wl.layers_per_group, num_q_heads=wl.num_q_heads,
               num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, r_max=wl.r_max, tiers=wl.tiers,
               resid_channels=wl.resid_channels, resid_bits=wl.resid_bits, max_batch=wl.batch,
-              max_context=wl.context + 64)
+              max_context=wl.context + 64, tier_resid=wl.tier_resid or None)
     kw.update(over)
     return dw.config_from(**kw)
 
@@ -72,6 +72,28 @@ def test_token_and_page_bytes():
     meta = dw.dwkv_metadata_bytes(cfg)
     assert 0 < meta < dw.dwkv_arena_bytes(cfg)
     assert dw.dwkv_workspace_bytes(cfg, 8) == 8 * dw.dwkv_workspace_bytes(cfg, 1)
+
+
+@pytest.mark.parametrize("over", [
+    dict(tier_resid=(0, 2, 4, 8), tiers=(32, 32, 32, 16)),      # routed tiers share one rank
+    dict(tier_resid=(0, 2, 3, 8)),                              # counts in {0, 2, 4, 8}
+    dict(tier_resid=(0, 4, 2, 8)),                              # strictly ascending
+    dict(tier_resid=(0, 2, 4, 8), resid_channels=16),           # array stride 8
+])
+def test_invalid_routed_configs_are_rejected(over):
+    cfg = _cfg(synth.workload("llama8b_routed_64k"), **over)
+    assert dw.dwkv_config_check(cfg) == 1
+    assert dw.dwkv_last_error()
+
+
+def test_routed_token_and_page_bytes():
+    """Per-tier residual counts: 2 * (2 r + rho + rho * bits / 8 + 2) bytes a token; a page's
+    code part is padded to 128 bytes."""
+    cfg = _cfg(synth.workload("llama8b_routed_64k"))
+    assert [dw.dwkv_token_bytes(cfg, k) for k in range(4)] == [2 * (64 + n + n // 2 + 2) for n in (0, 2, 4, 8)]
+    for k, n in enumerate((0, 2, 4, 8)):
+        code = (8 * n * 4 + 127) // 128 * 128
+        assert dw.dwkv_page_bytes(cfg, k) == 2 * 2 * (128 * 32 + 64 * n + code + 128) + 64 * 4
 
 
 def test_create_rejects_bad_arguments_without_a_gpu():

@@ -23,13 +23,19 @@ def _expected_after(wl, bases, data, moves):
     new_tier [n][H])}, from the oracle's re-encode of the imported values."""
     exp = {}
     tiers_new = {}
+    nres_of = wl.tier_resid or (wl.resid_channels,) * len(wl.tiers)
     for (b, layer), (tiers, comp) in data.items():
         g = layer // wl.layers_per_group
         c = {k: v.clone().cpu() for k, v in comp.items()}
         t = tiers.clone().cpu()
-        # the cache stores (and exports) +0 past each token's rank, whatever the input held there
+        # the cache stores (and exports) +0 past each token's rank, whatever the input held there,
+        # and zeros past its residual count
         keep = torch.arange(wl.r_max).view(1, 1, 1, -1) < synth.ranks_of(wl, t).view(t.shape[0], -1, 1, 1)
         c["coeff"] = torch.where(keep, c["coeff"], torch.zeros_like(c["coeff"]))
+        nres = synth.resid_counts_of(wl, t)
+        on = torch.arange(wl.resid_channels).view(1, 1, 1, -1) < nres.view(t.shape[0], -1, 1, 1)
+        c["idx"], c["codes"] = c["idx"] * on, c["codes"] * on
+        c["scales"] = c["scales"] * (nres.view(t.shape[0], -1, 1) > 0)
         if b in moves:
             pos, nt = moves[b]
             for n, p in enumerate(pos.tolist()):
@@ -38,14 +44,17 @@ def _expected_after(wl, bases, data, moves):
                     t[p, h] = k_new
                     if k_old == k_new:
                         continue
+                    s_old, s_new = int(nres_of[k_old]), int(nres_of[k_new])
                     for z in range(2):
                         c["coeff"][p, h, z] = 0
                         r = oracle.reencode_vector(bases[z][g, h], wl.tiers[k_old], comp["coeff"][p, h, z],
-                                                   comp["idx"][p, h, z], comp["codes"][p, h, z], comp["scales"][p, h, z],
-                                                   wl.tiers[k_new], wl.resid_bits)
+                                                   comp["idx"][p, h, z, :s_old], comp["codes"][p, h, z, :s_old],
+                                                   comp["scales"][p, h, z], wl.tiers[k_new], wl.resid_bits, s_new=s_new)
                         c["coeff"][p, h, z] = torch.from_numpy(r["coeff"].view(np.int16)).view(torch.bfloat16)
-                        c["idx"][p, h, z] = torch.from_numpy(r["idx"])
-                        c["codes"][p, h, z] = torch.from_numpy(r["codes"])
+                        c["idx"][p, h, z] = 0
+                        c["codes"][p, h, z] = 0
+                        c["idx"][p, h, z, :s_new] = torch.from_numpy(r["idx"])
+                        c["codes"][p, h, z, :s_new] = torch.from_numpy(r["codes"])
                         c["scales"][p, h, z] = torch.from_numpy(np.array([r["scale"]], np.uint16).view(np.int16)).view(torch.float16)[0]
         exp[(b, layer)] = (t, c)
         tiers_new[b] = t
@@ -77,7 +86,7 @@ def _retier(cache, wl, group, moves):
     cache.retier(group, seqs, [len(moves[b][0]) for b in seqs], pos, nt)
 
 
-@pytest.mark.parametrize("name", ["llama8b_64k", "llama8b_ragged_b8", "llama8b_131k_deep"])
+@pytest.mark.parametrize("name", ["llama8b_64k", "llama8b_ragged_b8", "llama8b_131k_deep", "llama8b_routed_64k"])
 def test_moved_tokens_are_reencoded_bit_exact_and_decode_matches(name):
     wl = synth.workload(name).scaled(num_q_heads=8, num_kv_heads=2, batch=2)
     wl = wl.scaled(num_layers=wl.layers_per_group)

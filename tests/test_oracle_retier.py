@@ -114,3 +114,45 @@ def test_dense_basis_reconstruction_is_within_bf16_rounding_of_fp64():
         xh = bf16_np(torch.from_numpy(out["xh"].view(np.int16)).view(torch.bfloat16))
         # bf16 rounding (half an ulp, 2^-9 relative) plus the fp32 chain's error
         assert np.all(np.abs(xh - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6 * np.linalg.norm(ref)), seed
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("s_old,s_new", [(8, 2), (2, 8), (4, 0), (0, 4)])
+def test_residual_count_change_at_one_rank(bits, s_old, s_new):
+    """A tier move of the residual-count routing reading (same rank, another residual count)
+    with a signed-permutation basis: the coefficients are kept exactly when the old residual
+    stays off the basis directions, and the new residual is the s_new largest |xh| off the
+    kept directions, ties to the lower channel, codes by the scale of the largest."""
+    d, r_max, r = 128, 64, 32
+    Bm, perm, sign = signed_permutation(d, r_max, 40 + s_old)
+    g = torch.Generator().manual_seed(41 + s_new)
+    c = torch.zeros(r_max)
+    c[:r] = torch.randn(r, generator=g)
+    c = c.to(torch.bfloat16)
+    covered = {int(perm[j]) for j in range(r)}
+    free = [i for i in range(d) if i not in covered]
+    pick = torch.randperm(len(free), generator=g)[:s_old].tolist()
+    idx = torch.tensor(sorted(free[i] for i in pick), dtype=torch.uint8)
+    qmax = synth.qmax_of(bits)
+    codes = torch.randint(-qmax, qmax + 1, (s_old,), generator=g).to(torch.int8)
+    scale = torch.tensor([0.021], dtype=torch.float16)
+    out = oracle.reencode_vector(Bm, r, c, idx, codes, scale, r, bits, s_new=s_new)
+    assert out["idx"].shape == (s_new,) and out["codes"].shape == (s_new,)
+    assert np.array_equal(out["coeff"], c.view(torch.int16).numpy().view(np.uint16))
+    xf = bf16_np(torch.from_numpy(out["xh"].view(np.int16)).view(torch.bfloat16)).astype(np.float64)
+    res = xf.copy()
+    for j in range(r):
+        res[int(perm[j])] = 0.0
+    # the old residual is the only mass off the kept directions
+    assert np.count_nonzero(res) <= s_old
+    order = sorted(range(d), key=lambda i: (-abs(res[i]), i))[:s_new]
+    assert list(out["idx"]) == sorted(order)
+    if s_new:
+        amax = max(abs(res[i]) for i in order)
+        sf = float(np.float16(np.float32(amax) / np.float32(qmax)))
+        assert abs(float(bf16_np(torch.tensor([out["scale"]], dtype=torch.int16).view(torch.float16))[0]) - sf) == 0.0
+        for i, q in zip(out["idx"], out["codes"]):
+            want = 0 if sf == 0 else int(np.clip(np.rint(np.float32(res[int(i)]) / np.float32(sf)), -qmax, qmax))
+            assert int(q) == want, (i, q, want)
+    else:
+        assert out["scale"] == 0
