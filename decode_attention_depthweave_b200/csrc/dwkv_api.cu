@@ -302,7 +302,7 @@ uint32_t decode_ring_for(dwkv_handle h, bool probe, size_t* smem_out) {
     const Geom& G = h->geom;
     const size_t budget = h->smem_optin;
     const DecodeSmem L0 = decode_smem_layout(G, 0, probe);
-    const size_t scratch = ((size_t)2 * kGQ * G.r_max + (size_t)kGQ * kD) * sizeof(float);
+    const size_t scratch = (size_t)kMergeBvOff + (size_t)kD * G.r_max * 2;   // merged sums, then B_V
     const size_t need = std::max(2 * (size_t)G.stage_bytes, scratch);
     if ((size_t)L0.total + need > budget) return 0;
     size_t ring = (budget - L0.total) / 128 * 128;

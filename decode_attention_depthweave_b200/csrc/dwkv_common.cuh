@@ -157,6 +157,8 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 struct DecodeSmem {
     uint32_t ring, rd, small, small_stride, S, P, W, P2, qt, q, qh, zero, bars, misc, tok, total;
 };
+// The CTA merge reuses the idle ring: the merged sums (at most 6 KB) at 0, B_V at kMergeBvOff.
+constexpr uint32_t kMergeBvOff = 8192;
 constexpr uint32_t kMiscState = 256;                               // m_state [warps][16]
 constexpr uint32_t kMiscFactors = kMiscState + kConsumerWarps * 64; // mf [2][warps][4]
 constexpr uint32_t kMiscPages = kMiscFactors + kConsumerWarps * 32; // t_src [32], t_len [32]

@@ -685,7 +685,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     }
 
     uint32_t cv[kMaxTiers];                 // tier counts (producer lane 0)
-    uint32_t bvf[RMAX / 16][4];             // B_V mma fragments (consumer warps 0-7, epilogue)
     if (warp == kConsumerWarps && lane == 0) {
         for (int i = 0; i < kSlots; ++i) {
             mbar_init(full0 + 8 * i, 1);
@@ -840,7 +839,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         const uint32_t zero_addr = smem_addr(smem + L.zero);
         const float qscale = G.tau * kLog2e;
         uint2* qh = reinterpret_cast<uint2*>(smem + L.qh);
-        {   // B_V, read from registers by the CTA merge at the end: warm it into L2 now
+        {   // B_V, copied into the ring for the CTA merge at the end: warm it into L2 now
             const int lines = kD * G.r_max * 2 / 128;
             for (int x = tid; x < lines; x += kConsumerWarps * 32)
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(St.basis_v + basis_off) + 128 * x));
@@ -1000,28 +999,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             }
         }
         if (PROBE) store_d(A.c2, reinterpret_cast<float*>(small), G.r_max, lane);
-        if (warp < kD / 16) {
-            // this warp's 16 B_V rows as mma A fragments (row 16 warp + g (+8), columns
-            // 16 ks + 2c (+1, +8, +9)), requested now so they arrive while the CTA merges
-            const int g = lane >> 2, c = lane & 3;
-            const __nv_bfloat16* b0 = St.basis_v + basis_off + (size_t)(16 * warp + g) * G.r_max + 2 * c;
-#pragma unroll
-            for (int ks = 0; ks < RMAX / 16; ++ks) {
-                const int k0 = 16 * ks, k1 = 16 * ks + 8;
-                bvf[ks][0] = k0 < G.r_max ? __ldg(reinterpret_cast<const unsigned int*>(b0 + k0)) : 0u;
-                bvf[ks][1] = k0 < G.r_max ? __ldg(reinterpret_cast<const unsigned int*>(b0 + 8 * G.r_max + k0)) : 0u;
-                bvf[ks][2] = k1 < G.r_max ? __ldg(reinterpret_cast<const unsigned int*>(b0 + k1)) : 0u;
-                bvf[ks][3] = k1 < G.r_max ? __ldg(reinterpret_cast<const unsigned int*>(b0 + 8 * G.r_max + k1)) : 0u;
-            }
-        }
         float* ms = m_state + warp * 16;
+        float l[kGQ], l2[kGQ];
 #pragma unroll
-        for (int hh = 0; hh < kGQ; ++hh) {
-            const float l = warp_sum(A.l[hh]);
-            const float l2 = PROBE ? warp_sum(A.l2[hh]) : 0.f;
-            if (lane == 0) {
-                ms[hh] = A.m[hh]; ms[4 + hh] = l;
-                ms[8 + hh] = A.m2[hh]; ms[12 + hh] = l2;
+        for (int hh = 0; hh < kGQ; ++hh) { l[hh] = A.l[hh]; l2[hh] = PROBE ? A.l2[hh] : 0.f; }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)             // the heads' sums side by side
+#pragma unroll
+            for (int hh = 0; hh < kGQ; ++hh) {
+                l[hh] += __shfl_xor_sync(0xffffffffu, l[hh], o);
+                if (PROBE) l2[hh] += __shfl_xor_sync(0xffffffffu, l2[hh], o);
+            }
+        if (lane == 0) {
+#pragma unroll
+            for (int hh = 0; hh < kGQ; ++hh) {
+                ms[hh] = A.m[hh]; ms[4 + hh] = l[hh];
+                ms[8 + hh] = A.m2[hh]; ms[12 + hh] = l2[hh];
             }
         }
     }
@@ -1030,10 +1023,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     // ================= CTA merge: the warp states -> one partial record
     //   {M[4], L[4], (M2[4], L2[4]), o[4][d] = B_V acc_c + acc_r, (o2[4][d] = B_V acc_c2)}
     // B_V is applied here, once per CTA (tensor cores), so the final merge is a weighted sum.
+    // Every page has been attended, so the ring is idle: B_V [d][r_max] goes into it (one bulk
+    // copy, in flight while the states merge) after the merged sums' region.
+    const uint32_t bv_bytes = (uint32_t)kD * G.r_max * 2;
+    const __nv_bfloat16* bvs = reinterpret_cast<const __nv_bfloat16*>(smem + L.ring + kMergeBvOff);
+    if (tid == 0) {
+        mbar_arrive_expect_tx(basis_bar, bv_bytes);
+        bulk_g2s(smem_addr(smem + L.ring + kMergeBvOff), St.basis_v + basis_off, bv_bytes, basis_bar);
+    }
     const int nrec = C.total_splits;
     float* rec = C.ws + ((size_t)h * nrec + blockIdx.x) * C.rec_floats;
     const int hdr = PROBE ? 16 : 8;
-    const int nc = kGQ * G.r_max;
     if (warp < (PROBE ? 2 : 1)) {
         // lane = (warp w2 = lane / 4 + 8 i, head hh): the CTA max and rescaled sum by shuffles
         const int which = warp, hh = lane & 3;
@@ -1066,38 +1066,56 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         }
     }
     __syncthreads();
-    // merged sums into the idle ring: cm [4][r_max], racc [4][d], (cm2 [4][r_max]); each warp's
-    // sums sit in its residual tile ([j][4] then [i][4]) and, for acc_c2, its small buffer
+    // merged sums into the idle ring, rows of the 4 heads: cm [r_max][4], racc [d][4],
+    // (cm2 [r_max][4]); each warp's sums sit in its residual tile ([j][4] then [i][4]) and,
+    // for acc_c2, its small buffer.  A thread per row.
     float* cm = reinterpret_cast<float*>(smem + L.ring);
-    const int nbody = nc + kGQ * kD + (PROBE ? nc : 0);
-    for (int e = tid; e < nbody; e += blockDim.x) {
-        int hh, off, which = 0;
-        const uint8_t* base = smem + L.rd;
+    const int nrows = G.r_max + kD + (PROBE ? G.r_max : 0);
+    for (int e = tid; e < nrows; e += blockDim.x) {
+        int which = 0;
+        const uint8_t* base = smem + L.rd + (size_t)e * 16;
         uint32_t stride = kRdBytes;
-        if (e < nc) { hh = e / G.r_max; off = (e % G.r_max) * 4 + hh; }
-        else if (e < nc + kGQ * kD) { const int x = e - nc; hh = x / kD; off = G.r_max * 4 + (x % kD) * 4 + hh; }
-        else { const int x = e - nc - kGQ * kD; hh = x / G.r_max; off = (x % G.r_max) * 4 + hh;
-               which = 1; base = smem + L.small; stride = L.small_stride; }
-        float v = 0.f;
+        if (e >= G.r_max + kD) {
+            which = 1;
+            base = smem + L.small + (size_t)(e - G.r_max - kD) * 16;
+            stride = L.small_stride;
+        }
+        const float4* fw = reinterpret_cast<const float4*>(mf + which * kConsumerWarps * 4);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w2 = 0; w2 < kConsumerWarps; ++w2)
-            v = fmaf(mf[which * kConsumerWarps * 4 + w2 * 4 + hh],
-                     reinterpret_cast<const float*>(base + w2 * stride)[off], v);
-        cm[e] = v;
+        for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
+            const float4 f = fw[w2];
+            const float4 x = *reinterpret_cast<const float4*>(base + w2 * stride);
+            v.x = fmaf(f.x, x.x, v.x);
+            v.y = fmaf(f.y, x.y, v.y);
+            v.z = fmaf(f.z, x.z, v.z);
+            v.w = fmaf(f.w, x.w, v.w);
+        }
+        reinterpret_cast<float4*>(cm)[e] = v;
     }
     __syncthreads();
+    const bool bv_ok = mbar_wait(basis_bar, 1);
+    if (!bv_ok && tid == 0) set_dev_error(St, 6u, (uint32_t)seq, 0xfffffffdu);
     if (warp < kD / 16) {
         // o[i][h] for the warp's 16 channels: B_V rows (A, ldmatrix) against the merged acc_c as
         // bf16 hi (columns 0-3) + lo (columns 4-7) halves (B), fp32 accumulation
         const int g = lane >> 2, c = lane & 3, n = g & 3;
         const bool lo_half = g >= 4;
-        const float* racc = cm + nc;
-        const float* cm2 = cm + nc + kGQ * kD;
+        const float* racc = cm + 4 * G.r_max;
+        const float* cm2 = cm + 4 * (G.r_max + kD);
         float d[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
+        // this warp's 16 B_V rows as mma A fragments: rows 16 warp + g (+8), columns
+        // 16 ks + 2c (+1, +8, +9)
+        const __nv_bfloat16* b0 = bvs + (size_t)(16 * warp + g) * G.r_max + 2 * c;
 #pragma unroll
         for (int ks = 0; ks < RMAX / 16; ++ks) {
             if (16 * ks >= G.r_max) break;
-            const uint32_t (&a)[4] = bvf[ks];
+            const int k0 = 16 * ks, k1 = 16 * ks + 8;
+            uint32_t a[4];
+            a[0] = *reinterpret_cast<const uint32_t*>(b0 + k0);
+            a[1] = *reinterpret_cast<const uint32_t*>(b0 + 8 * G.r_max + k0);
+            a[2] = *reinterpret_cast<const uint32_t*>(b0 + k1);
+            a[3] = *reinterpret_cast<const uint32_t*>(b0 + 8 * G.r_max + k1);
             uint32_t b[2], b2[2];
 #pragma unroll
             for (int r2 = 0; r2 < 2; ++r2) {
@@ -1106,10 +1124,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                 for (int e = 0; e < 2; ++e) {
                     const int k = 16 * ks + 8 * r2 + 2 * c + e;
                     uint32_t hi, lo;
-                    split_bf16_rn(k < G.r_max ? cm[n * G.r_max + k] : 0.f, hi, lo);
+                    split_bf16_rn(k < G.r_max ? cm[k * 4 + n] : 0.f, hi, lo);
                     pk |= (lo_half ? lo : hi) << (16 * e);
                     if (PROBE) {
-                        split_bf16_rn(k < G.r_max ? cm2[n * G.r_max + k] : 0.f, hi, lo);
+                        split_bf16_rn(k < G.r_max ? cm2[k * 4 + n] : 0.f, hi, lo);
                         pk2 |= (lo_half ? lo : hi) << (16 * e);
                     }
                 }
@@ -1132,7 +1150,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const int hh = 2 * c + q;
-                    rec[hdr + hh * kD + i] = d[2 * rr2 + q] + racc[hh * kD + i];
+                    rec[hdr + hh * kD + i] = d[2 * rr2 + q] + racc[i * 4 + hh];
                     if (PROBE) rec[hdr + kGQ * kD + hh * kD + i] = d2[2 * rr2 + q];
                 }
             }
@@ -1175,10 +1193,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             }
         }
     };
-    load_chunk(0);
-    if (warp < (PROBE ? 2 : 1)) {
+    // the headers first: the weights wait on them, the values only at the sums
+    const bool hdr_warp = warp < (PROBE ? 2 : 1);
+    float mj[2][kGQ], lj[2][kGQ];
+    if (hdr_warp) {
         const int which = warp;
-        float mj[2][kGQ], lj[2][kGQ];
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
             const int j = lane + 32 * jj;                 // kMaxSplits = 64
@@ -1190,19 +1209,33 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             mj[jj][0] = m4.x; mj[jj][1] = m4.y; mj[jj][2] = m4.z; mj[jj][3] = m4.w;
             lj[jj][0] = l4.x; lj[jj][1] = l4.y; lj[jj][2] = l4.z; lj[jj][3] = l4.w;
         }
+    }
+    load_chunk(0);
+    if (hdr_warp) {
+        const int which = warp;
+        // the four heads' reductions side by side (independent shuffle chains)
+        float M[kGQ], Lsum[kGQ];
+#pragma unroll
+        for (int hh = 0; hh < kGQ; ++hh) M[hh] = fmaxf(mj[0][hh], mj[1][hh]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int hh = 0; hh < kGQ; ++hh) M[hh] = fmaxf(M[hh], __shfl_xor_sync(0xffffffffu, M[hh], o));
 #pragma unroll
         for (int hh = 0; hh < kGQ; ++hh) {
-            const float M = warp_max(fmaxf(mj[0][hh], mj[1][hh]));
-            float Lsum = 0.f;
+            Lsum[hh] = 0.f;
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
-                const float f = mj[jj][hh] == -INFINITY ? 0.f : exp2f(mj[jj][hh] - M);
+                const float f = mj[jj][hh] == -INFINITY ? 0.f : exp2f(mj[jj][hh] - M[hh]);
                 if (lane + 32 * jj < nsplit) wgt[(which * kMaxSplits + lane + 32 * jj) * kGQ + hh] = f;
-                Lsum = fmaf(f, lj[jj][hh], Lsum);
+                Lsum[hh] = fmaf(f, lj[jj][hh], Lsum[hh]);
             }
-            Lsum = warp_sum(Lsum);
-            if (lane == 0) Ls[which * 4 + hh] = Lsum;
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int hh = 0; hh < kGQ; ++hh) Lsum[hh] += __shfl_xor_sync(0xffffffffu, Lsum[hh], o);
+        if (lane < kGQ) Ls[which * 4 + lane] = lane == 0 ? Lsum[0] : lane == 1 ? Lsum[1] : lane == 2 ? Lsum[2] : Lsum[3];
     }
     __syncthreads();
     float acc1[kPer], acc2[kPer];
