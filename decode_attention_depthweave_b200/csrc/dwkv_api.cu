@@ -34,6 +34,7 @@ template <int BITS>
 __global__ void retier_kernel(const Geom, const State, const RetierCall, const int32_t*, const uint8_t*);
 __global__ void retier_release_kernel(const Geom, const State, const RetierCall);
 __global__ void wait_timeout_kernel(const State, uint64_t);
+__global__ void tile_basis_kernel(const Geom, const State);
 template <int BITS, bool PROBE, int RMAX, int S>
 __global__ void decode_kernel(const Geom, const State, const DecodeCall);
 }  // namespace dwkv
@@ -141,7 +142,8 @@ dwkv_status check_supported(const dwkv_config* c) {
 }
 
 struct MetaLayout {
-    size_t err, bump, free_head, free_tail, free_list, counts, owned, pages, slot_map, tickets, basis_k, basis_v, data;
+    size_t err, bump, free_head, free_tail, free_list, counts, owned, pages, slot_map, tickets, basis_k, basis_v, basis_kt,
+        data;
     uint32_t free_cap;
 };
 
@@ -198,6 +200,7 @@ MetaLayout meta_layout(const Geom& G) {
     M.tickets = take((size_t)4 * G.max_batch * G.Hkv);
     M.basis_k = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
     M.basis_v = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
+    M.basis_kt = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
     M.data = o;
     return M;
 }
@@ -284,6 +287,7 @@ State make_state(uint8_t* arena, const MetaLayout& M, size_t arena_bytes) {
     S.tickets = reinterpret_cast<uint32_t*>(arena + M.tickets);
     S.basis_k = reinterpret_cast<const __nv_bfloat16*>(arena + M.basis_k);
     S.basis_v = reinterpret_cast<const __nv_bfloat16*>(arena + M.basis_v);
+    S.basis_kt = reinterpret_cast<const __nv_bfloat16*>(arena + M.basis_kt);
     S.data = arena + M.data;
     S.data_units = (arena_bytes - M.data) / kUnit;
     return S;
@@ -467,6 +471,10 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
     cudaError_t e = cudaMemsetAsync(h->arena, 0, M.basis_k, s);
     if (e == cudaSuccess) e = cudaMemcpyAsync(h->arena + M.basis_k, basis_k, bbytes, cudaMemcpyDeviceToDevice, s);
     if (e == cudaSuccess) e = cudaMemcpyAsync(h->arena + M.basis_v, basis_v, bbytes, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) {
+        tile_basis_kernel<<<G.G * G.Hkv, 256, 0, s>>>(G, h->st);
+        e = cudaGetLastError();
+    }
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e == cudaSuccess) {
         const int maxs = (int)h->smem_optin;

@@ -413,6 +413,18 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
 }
 
 // ------------------------------------------------------------------------------------
+// The decode's copy of B_K in 8 x 8 tiles (tiled_basis_off), one block per (group, kv-head).
+// ------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) tile_basis_kernel(const Geom G, const State S) {
+    const size_t base = (size_t)blockIdx.x * kD * G.r_max;
+    __nv_bfloat16* dst = const_cast<__nv_bfloat16*>(S.basis_kt) + base;
+    for (int e = threadIdx.x; e < kD * G.r_max; e += blockDim.x) {
+        const int i = e / G.r_max, j = e % G.r_max;
+        dst[tiled_basis_off(i, j, G.r_max)] = S.basis_k[base + e];
+    }
+}
+
+// ------------------------------------------------------------------------------------
 // The kernels' bounded wait, exercised (test support): one thread waits on a shared-memory
 // barrier that nothing arrives at; the wait runs out after limit_ns and the kernel records
 // DWKV_DEV_TIMEOUT in the device error word, as every kernel does, then returns.

@@ -69,6 +69,7 @@ struct State {
     uint32_t* slot_map;              // [max_batch][G][Hkv][max_context]: ((tier+1)<<24)|slot
     uint32_t* tickets;               // [max_batch][Hkv] split-combine tickets
     const __nv_bfloat16* basis_k;    // [G][Hkv][d][r_max]
+    const __nv_bfloat16* basis_kt;   // the same, per (group, kv-head) as 8 x 8 tiles [d/8][r_max/8][8][8]
     const __nv_bfloat16* basis_v;
     uint8_t* data;                   // page pool
     unsigned long long data_units;
@@ -132,6 +133,12 @@ __host__ __device__ inline uint32_t off_codes_of(int R, int s) { return 128u * R
 __host__ __device__ inline uint32_t off_scales_of(int R, int s, int bits) {
     return 128u * R + 64u * s + code_part_bytes(s, bits);
 }
+// Element offset of B_K[i][j] in a tiled basis (basis_kt) of rank r_max: 8 x 8 tiles, the tile
+// rows 16 contiguous bytes, so that an ldmatrix row set (8 rows of one tile) is one 128-byte line.
+__host__ __device__ inline uint32_t tiled_basis_off(int i, int j, int r_max) {
+    return ((uint32_t)(i >> 3) * (uint32_t)(r_max >> 3) + (uint32_t)(j >> 3)) * 64u + (uint32_t)(i & 7) * 8u + (uint32_t)(j & 7);
+}
+
 // Byte offset of a page's slot-position block (after the layers' chunks).
 __host__ __device__ inline uint32_t pos_block_of(const Geom& G, int k) { return (uint32_t)G.LPG * G.chunk_bytes[k]; }
 constexpr uint32_t kPosBlockBytes = kPage * 4;
@@ -151,11 +158,12 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 //           starts again at 0); ring_bytes is chosen by the host
 //   rd      per consumer warp, one 4 KB residual tile (also holds B_K during the prologue)
 //   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W limbs [8][48] u8, P2[32][8]
-//   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  qh bf16 [d][4];  zero line
+//   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  qh bf16 [d][4];  qb: q~ as MMA
+//           B fragments [ks][2][lane];  zero line
 //   bars    full[kSlots] empty[kSlots] basis table
 //   misc    tier table, page range, work counter; warp states; page-id batch; slot offsets
 struct DecodeSmem {
-    uint32_t ring, rd, small, small_stride, S, P, W, P2, qt, q, qh, zero, bars, misc, tok, total;
+    uint32_t ring, rd, small, small_stride, S, P, W, P2, qt, q, qh, qb, zero, bars, misc, tok, total;
 };
 // The CTA merge reuses the idle ring: the merged sums (at most 6 KB) at 0, B_V at kMergeBvOff.
 constexpr uint32_t kMergeBvOff = 8192;
@@ -179,6 +187,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, uint32_t
     L.qt = o;      o += (uint32_t)(G.r_max < 16 ? 16 : G.r_max) * 16;
     L.q = o;       o += (uint32_t)G.d * 16;
     L.qh = o;      o += (uint32_t)G.d * 8;
+    L.qb = o;      o += 32 * 2 * (kMaxRank / 16) * 4;
     L.zero = o;    o += 128;
     L.bars = o;    o += (2 * kSlots + 2) * 8;
     L.misc = o;    o += (kMiscBytes + 127) & ~127u;

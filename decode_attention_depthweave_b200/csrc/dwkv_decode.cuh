@@ -685,20 +685,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     }
 
     uint32_t cv[kMaxTiers];                 // tier counts (producer lane 0)
-    if (warp == kConsumerWarps && lane == 0) {
-        for (int i = 0; i < kSlots; ++i) {
-            mbar_init(full0 + 8 * i, 1);
-            mbar_init(empty0 + 8 * i, 2);     // released by the warps of its two halves
+    static_assert(kSlots == 32, "the producer's lane i sets up ring slot i");
+    if (warp == kConsumerWarps) {
+        mbar_init(full0 + 8 * lane, 1);
+        mbar_init(empty0 + 8 * lane, 2);      // released by the warps of its two halves
+        if (lane == 0) {
+            mbar_init(basis_bar, 1);
+            mbar_init(table_bar, 1);
+            m_misc[3] = 0u;                   // half-page work counter
         }
-        mbar_init(basis_bar, 1);
-        mbar_init(table_bar, 1);
-        m_misc[3] = 0u;                       // half-page work counter
         fence_mbar_init();
+        __syncwarp();
+    }
+    if (warp == kConsumerWarps && lane == 0) {
         // B_K into the residual tiles (free until the main loop) and the counts, both in
         // flight across the barrier below
         const uint32_t bytes = (uint32_t)kD * G.r_max * 2;
         mbar_arrive_expect_tx(basis_bar, bytes);
-        bulk_g2s(smem_addr(smem + L.rd), St.basis_k + basis_off, bytes, basis_bar);
+        bulk_g2s(smem_addr(smem + L.rd), St.basis_kt + basis_off, bytes, basis_bar);
         // Until this CTA waits on the previous kernel (programmatic dependent launch), that
         // kernel may still be running; the host says whether the cache state read from here on
         // (counts, slot map, page tables, page bytes) is already final.
@@ -722,42 +726,56 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
     if (warp == kConsumerWarps) {
         // ================= producer warp: B_K, the CTA's page range, then page chunks
         if (lane == 0) {
-            uint32_t P = 0;
+            // Integer costs; each boundary is computed by the same operations in the two CTAs
+            // that share it, and the divisions are fp32 estimates corrected to the exact result.
+            uint32_t P = 0, rP[kMaxTiers + 1];
             unsigned long long W = 0;
-            const unsigned long long tokw = (unsigned long long)C.tok_weight * kPage;
+            uint32_t rw[kMaxTiers];
+            const uint32_t tokw = (uint32_t)C.tok_weight * kPage;
 #pragma unroll
             for (int k = 0; k < kMaxTiers; ++k) {
-                if (k >= G.ntiers) break;
-                const uint32_t np = (cv[k] + kPage - 1) / kPage;
-                m_cnt[k] = cv[k];
-                m_P[k] = P;
-                m_R[k] = (uint32_t)G.tiers[k];
-                m_chunk[k] = G.chunk_bytes[k];
+                const uint32_t np = k < G.ntiers ? (cv[k] + kPage - 1) / kPage : 0u;
+                rP[k] = P;
+                rw[k] = k < G.ntiers ? G.chunk_bytes[k] + tokw : 1u;
+                if (k < G.ntiers) {
+                    m_cnt[k] = cv[k];
+                    m_P[k] = P;
+                    m_R[k] = (uint32_t)G.tiers[k];
+                    m_chunk[k] = G.chunk_bytes[k];
+                }
                 P += np;
-                W += (unsigned long long)np * (G.chunk_bytes[k] + tokw);
+                W += (unsigned long long)np * rw[k];
             }
+            rP[kMaxTiers] = P;
             m_P[G.ntiers] = P;
             // cost-balanced page range: pages whose first cost unit lies in [lo, hi).  With a
             // fused append, split 0 (which also encodes the token) takes owner_share / 256 of a
             // share: boundary s sits at W (256 (s - 1) + owner_share) / (256 (nsplit - 1) + owner_share).
-            const unsigned long long fs = (unsigned long long)C.owner_share;
-            const unsigned long long den = 256ull * (nsplit - 1) + fs;
+            const float fs = (float)C.owner_share;
+            const float den = 256.f * (float)(nsplit - 1) + fs;
             auto bound = [&](int sidx) -> unsigned long long {
-                return sidx == 0 ? 0ull : W * (256ull * (sidx - 1) + fs) / den;
+                return sidx == 0 ? 0ull
+                                 : (unsigned long long)floor((double)W * (double)((256.f * (float)(sidx - 1) + fs) / den));
+            };
+            // ceil(x / w): an fp32 estimate (within a few units for these sizes), then exact
+            auto cdiv = [](unsigned long long x, uint32_t w) -> uint32_t {
+                uint32_t q = (uint32_t)ceilf(__fdividef((float)x, (float)w));
+                while ((unsigned long long)q * w < x) ++q;
+                while (q > 0u && (unsigned long long)(q - 1u) * w >= x) --q;
+                return q;
             };
             const unsigned long long lo = bound(split);
-            const unsigned long long hi = split + 1 == nsplit ? W : bound(split + 1);
+            const unsigned long long hi = split + 1 == nsplit ? W : min(bound(split + 1), W);
             uint32_t pb = P, pe = P;
             unsigned long long Wk = W;
-            for (int k = G.ntiers - 1; k >= 0; --k) {
-                const uint32_t np = m_P[k + 1] - m_P[k];
-                const unsigned long long w = G.chunk_bytes[k] + tokw;
-                Wk -= (unsigned long long)np * w;      // first cost unit of tier k
+#pragma unroll
+            for (int k = kMaxTiers - 1; k >= 0; --k) {
+                const uint32_t np = rP[k + 1] - rP[k];
+                const uint32_t w = rw[k];
+                Wk -= (unsigned long long)np * w;        // first cost unit of tier k
                 if (!np) continue;
-                // lo - Wk < np * w fits 32 bits, so the divisions stay 32-bit
-                const uint32_t w32 = (uint32_t)w;
-                if (lo <= Wk + (np - 1) * w) pb = m_P[k] + (lo > Wk ? ((uint32_t)(lo - Wk) + w32 - 1) / w32 : 0u);
-                if (hi <= Wk + (np - 1) * w) pe = m_P[k] + (hi > Wk ? ((uint32_t)(hi - Wk) + w32 - 1) / w32 : 0u);
+                if (lo <= Wk + (unsigned long long)(np - 1) * w) pb = rP[k] + (lo > Wk ? cdiv(lo - Wk, w) : 0u);
+                if (hi <= Wk + (unsigned long long)(np - 1) * w) pe = rP[k] + (hi > Wk ? cdiv(hi - Wk, w) : 0u);
             }
             m_misc[0] = pb;
             m_misc[1] = pe > pb ? pe : pb;
@@ -860,61 +878,73 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         named_barrier(1, kConsumerWarps * 32);
         bool ok = mbar_wait(basis_bar, 0);
         if (!ok && lane == 0) set_dev_error(St, 6u, (uint32_t)seq, 0xffffffffu);
-        // q~[j] = sum_i B_K[i][j] q[i]: the 256 consumer threads split the rows into
-        // np = 256 / rq parts (a warp reads one row at a time: conflict-free); the parts
-        // are summed through the small buffers.
+        // q~[j] = qscale sum_i B_K[i][j] q[i] on the tensor cores: warp m < rq / 16 takes rows
+        // j in [16 m, 16 m + 16) as one MMA row tile, A = B_K^T (ldmatrix.trans of the 8 x 8
+        // tiles of B_K in the residual tiles), B = q as bf16 (exact) in columns 0-3, fp32
+        // accumulation.
         const int rq = G.r_max < 16 ? 16 : G.r_max;
-        {
-            const int np = 256 / rq, j = tid % rq, part = tid / rq, rows = kD / np;
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (ok && tid < 256 && j < G.r_max) {
-                const __nv_bfloat16* bk = reinterpret_cast<const __nv_bfloat16*>(smem + L.rd) + j;
-#pragma unroll 8
-                for (int i = part * rows; i < (part + 1) * rows; ++i) {
-                    const float b = __bfloat162float(bk[i * G.r_max]);
-                    const float4 q = qs[i];
-                    a.x = fmaf(b, q.x, a.x); a.y = fmaf(b, q.y, a.y);
-                    a.z = fmaf(b, q.z, a.z); a.w = fmaf(b, q.w, a.w);
+        if (warp < rq / 16) {
+            const int g = lane >> 2, c = lane & 3, mi = lane >> 3, rr = lane & 7;
+            const uint32_t bk = smem_addr(smem + L.rd);
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks) {
+                // matrix mi: rows j 16 warp + 8 (mi & 1) .., columns i 16 ks + 8 (mi >> 1) ..
+                const int i = 16 * ks + 8 * (mi >> 1) + rr, j0 = 16 * warp + 8 * (mi & 1);
+                uint32_t a[4];
+                ldsm_x4_t(bk + tiled_basis_off(i, j0, G.r_max) * 2u, a);
+                uint32_t b[2] = {0u, 0u};
+                if (g < kGQ) {
+#pragma unroll
+                    for (int r2 = 0; r2 < 2; ++r2) {
+                        const int i0 = 16 * ks + 8 * r2 + 2 * c;
+                        const uint2 w0 = qh[i0], w1 = qh[i0 + 1];
+                        const uint32_t x0 = g < 2 ? w0.x : w0.y, x1 = g < 2 ? w1.x : w1.y;
+                        const uint32_t sh = 16u * (uint32_t)(g & 1);
+                        b[r2] = ((x0 >> sh) & 0xffffu) | (((x1 >> sh) & 0xffffu) << 16);
+                    }
                 }
+                mma_bf16(d, a, b);
             }
-            float4* parts = reinterpret_cast<float4*>(smem + L.small);     // [np][rq]
-            if (tid < 256) parts[part * rq + j] = a;
-            named_barrier(1, kConsumerWarps * 32);
-            if (tid < rq) {
-                float4 t4 = parts[tid];
-                for (int q2 = 1; q2 < np; ++q2) {
-                    const float4 u = parts[q2 * rq + tid];
-                    t4.x += u.x; t4.y += u.y; t4.z += u.z; t4.w += u.w;
+            if (c < 2) {                                  // columns 2c, 2c+1 = heads
+#pragma unroll
+                for (int rr2 = 0; rr2 < 2; ++rr2) {
+                    const int j = 16 * warp + g + 8 * rr2;
+                    const bool on = ok && j < G.r_max;
+                    reinterpret_cast<float2*>(qt + j)[c] =
+                        make_float2(on ? d[2 * rr2] * qscale : 0.f, on ? d[2 * rr2 + 1] * qscale : 0.f);
                 }
-                qt[tid] = t4;
             }
         }
         named_barrier(1, kConsumerWarps * 32);
-        // q~ as the MMA B operand: column n < 4 = bf16 hi of head n, n >= 4 = lo of head n-4
-        uint32_t qb[RMAX / 16][2];
-        {
-            const int g = lane >> 2, c = lane & 3, n = g & 3;
+        // q~ as the score MMA's B operand, the same fragments in every warp: built once into
+        // qbs [ks][r2][lane] (column n < 4 = bf16 hi of head n, n >= 4 = lo of head n-4)
+        uint32_t* qbs = reinterpret_cast<uint32_t*>(smem + L.qb);
+        for (int x = tid; x < 32 * 2 * (RMAX / 16); x += kConsumerWarps * 32) {
+            const int ln = x & 31, ks = (x >> 5) >> 1, r2 = (x >> 5) & 1;
+            const int g = ln >> 2, c = ln & 3, n = g & 3;
             const bool lo_half = g >= 4;
+            uint32_t pk = 0;
 #pragma unroll
-            for (int ks = 0; ks < RMAX / 16; ++ks) {
-#pragma unroll
-                for (int r2 = 0; r2 < 2; ++r2) {
-                    uint32_t pk = 0;
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int k = 16 * ks + 8 * r2 + 2 * c + e;
-                        float v = 0.f;
-                        if (k < rq) {
-                            const float4 t4 = qt[k];
-                            v = n == 0 ? t4.x : n == 1 ? t4.y : n == 2 ? t4.z : t4.w;
-                        }
-                        uint32_t hi, lo;
-                        split_bf16_rn(v, hi, lo);
-                        pk |= (lo_half ? lo : hi) << (16 * e);
-                    }
-                    qb[ks][r2] = pk;
+            for (int e = 0; e < 2; ++e) {
+                const int k = 16 * ks + 8 * r2 + 2 * c + e;
+                float v = 0.f;
+                if (k < rq) {
+                    const float4 t4 = qt[k];
+                    v = n == 0 ? t4.x : n == 1 ? t4.y : n == 2 ? t4.z : t4.w;
                 }
+                uint32_t hi, lo;
+                split_bf16_rn(v, hi, lo);
+                pk |= (lo_half ? lo : hi) << (16 * e);
             }
+            qbs[x] = pk;
+        }
+        named_barrier(1, kConsumerWarps * 32);
+        uint32_t qb[RMAX / 16][2];
+#pragma unroll
+        for (int ks = 0; ks < RMAX / 16; ++ks) {
+            qb[ks][0] = qbs[(2 * ks) * 32 + lane];
+            qb[ks][1] = qbs[(2 * ks + 1) * 32 + lane];
         }
         {   // the residual tiles held B_K until now; clear this warp's tile
             uint4* z = reinterpret_cast<uint4*>(rd);
