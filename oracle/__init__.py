@@ -45,7 +45,7 @@ def lib():
         L.oracle_encode_many.restype = i
         L.oracle_encode_many_from_coeffs.argtypes = [i, i, i, p, p, p, p, i, i, p, p, p, p, i, p]
         L.oracle_encode_many_from_coeffs.restype = i
-        L.oracle_reencode_vector.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, i, i, p, p, p, p, p]
+        L.oracle_reencode_vector.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, i, i, p, p, p, p, p, p]
         L.oracle_reencode_vector.restype = i
         L.oracle_reconstruct.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, p]
         L.oracle_reconstruct.restype = None
@@ -298,10 +298,10 @@ def encode_many(basis, x, ranks, s, bits, nthreads=None, want_c32=False, nres=No
     return out
 
 
-def reencode_vector(basis, r_old, coeff, idx, codes, scale, r_new, bits, s_new=None):
+def reencode_vector(basis, r_old, coeff, idx, codes, scale, r_new, bits, s_new=None, basis_new=None):
     """Re-tier one stored vector: re-encode its bf16-rounded reconstruction at rank r_new with
-    s_new residual channels (default: as many as stored) (``oracle_reencode_vector``).  Returns
-    the encode dict plus ``xh`` (bf16 bits [d])."""
+    s_new residual channels (default: as many as stored) on basis_new (default: the same basis)
+    (``oracle_reencode_vector``).  Returns the encode dict plus ``xh`` (bf16 bits [d])."""
     b = _bits16(basis)
     d, r_max = b.shape
     c = _bits16(coeff).reshape(r_max)
@@ -315,8 +315,12 @@ def reencode_vector(basis, r_old, coeff, idx, codes, scale, r_new, bits, s_new=N
     out_q = np.zeros(sn, np.int8)
     out_s = np.zeros(1, np.uint16)
     xh = np.zeros(d, np.uint16)
+    bn = None if basis_new is None else _bits16(basis_new)
+    if bn is not None and bn.shape != b.shape:
+        raise ValueError("basis_new must have the basis' shape")
     rc = lib().oracle_reencode_vector(d, r_max, _p(b), int(r_old), _p(c), s, _p(ix), _p(cd), sc, int(r_new), sn,
-                                      int(bits), _p(out_c), _p(out_i), _p(out_q), _p(out_s), _p(xh))
+                                      int(bits), _p(out_c), _p(out_i), _p(out_q), _p(out_s), _p(xh),
+                                      _p(bn) if bn is not None else None)
     if rc != 0:
         raise ValueError("oracle_reencode_vector: bad arguments")
     return {"coeff": out_c, "idx": out_i, "codes": out_q, "scale": out_s[0], "xh": xh}

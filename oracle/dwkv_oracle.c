@@ -366,7 +366,9 @@ int oracle_encode_many(int n, int d, int r_max, const uint16_t* basis, const uin
 /*          for the others (scale * code is exact in fp32; one rounding in the add)         */
 /* then the six encode steps of oracle_encode_vector on xh at rank r_new with s_new        */
 /* residual channels (a tier of the residual-count routing reading keeps its own count;     */
-/* otherwise s_new = s).                                                                    */
+/* otherwise s_new = s), on basis_new (nullable: the same basis).  A basis update (the     */
+/* shared bases' moving average, [DW] §3) moves a token with basis_new the updated basis    */
+/* and r_new = r_old.                                                                       */
 /* Inputs: the stored coeff (bf16 [r_max], entries >= r_old ignored), idx / codes [s],      */
 /* scale (fp16 bits).  Outputs as oracle_encode_vector (idx / codes [s_new]); xh_out        */
 /* (nullable) bf16 bits [d].                                                                */
@@ -374,7 +376,7 @@ int oracle_encode_many(int n, int d, int r_max, const uint16_t* basis, const uin
 int oracle_reencode_vector(int d, int r_max, const uint16_t* basis, int r_old, const uint16_t* coeff_old,
                            int s, const uint8_t* idx_old, const int8_t* codes_old, uint16_t scale_old,
                            int r_new, int s_new, int bits, uint16_t* coeff, uint8_t* idx, int8_t* codes,
-                           uint16_t* scale, uint16_t* xh_out) {
+                           uint16_t* scale, uint16_t* xh_out, const uint16_t* basis_new) {
     if (d <= 0 || d > 256 || r_old < 0 || r_old > r_max || r_new < 0 || r_new > r_max || s < 0 || s > d ||
         s_new < 0 || s_new > d)
         return -1;
@@ -396,7 +398,8 @@ int oracle_reencode_vector(int d, int r_max, const uint16_t* basis, int r_old, c
         xh[i] = oracle_f32_to_bf16_rn(a[i]);
         if (xh_out) xh_out[i] = xh[i];
     }
-    return oracle_encode_vector(d, r_max, basis, xh, r_new, s_new, bits, coeff, NULL, idx, codes, scale, NULL);
+    return oracle_encode_vector(d, r_max, basis_new ? basis_new : basis, xh, r_new, s_new, bits, coeff, NULL, idx,
+                                codes, scale, NULL);
 }
 
 /* Element-wise format conversions over arrays (used to pin the converters). */
