@@ -25,7 +25,8 @@ __all__ = [
     "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
     "dwkv_retier", "dwkv_tier_policy", "dwkv_tier_controller_create", "dwkv_tier_controller_destroy",
     "dwkv_tier_controller_due", "dwkv_tier_controller_threshold", "dwkv_tier_controller_observe",
-    "dwkv_tier_controller_route", "dwkv_arena_bytes_all_tiers", "Cache", "EXPORTED_SYMBOLS",
+    "dwkv_tier_controller_route", "dwkv_arena_bytes_all_tiers", "dwkv_basis_sketch", "dwkv_basis_update",
+    "dwkv_get_bases", "dwkv_get_moment", "Cache", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,7 +45,7 @@ EXPORTED_SYMBOLS = (
     "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
     "dwkv_retier", "dwkv_tier_controller_create", "dwkv_tier_controller_destroy", "dwkv_tier_controller_due",
     "dwkv_tier_controller_threshold", "dwkv_tier_controller_observe", "dwkv_tier_controller_route",
-    "dwkv_arena_bytes_all_tiers",
+    "dwkv_arena_bytes_all_tiers", "dwkv_basis_sketch", "dwkv_basis_update", "dwkv_get_bases", "dwkv_get_moment",
 )
 
 
@@ -117,6 +118,10 @@ def lib():
             "dwkv_check_bounded_wait": ([vp, C.c_uint32, vp], C.c_int),
             "dwkv_set_decode_overlap": ([vp, i32], C.c_int),
             "dwkv_retier": ([vp, i32, i32, vp, vp, vp, vp, vp], C.c_int),
+            "dwkv_basis_sketch": ([vp, i32, i32, vp, vp, vp, i32, vp, vp], C.c_int),
+            "dwkv_basis_update": ([vp, i32, i32, vp, vp, C.c_float, i32, vp, vp, vp], C.c_int),
+            "dwkv_get_bases": ([vp, i32, vp, vp, vp], C.c_int),
+            "dwkv_get_moment": ([vp, i32, vp, vp], C.c_int),
             "dwkv_tier_controller_create": ([C.POINTER(dwkv_tier_policy), i32, C.POINTER(vp)], C.c_int),
             "dwkv_tier_controller_destroy": ([vp], C.c_int),
             "dwkv_tier_controller_due": ([vp, C.c_int64], i32),
@@ -322,6 +327,24 @@ def dwkv_retier(h, group, seq_ids, n_tok, positions, new_tier, stream=None):
                              _stream(stream)))
 
 
+def dwkv_basis_sketch(h, group, n_rows, k_rows, v_rows, omega, power_steps=2, eigenvalues=None, stream=None):
+    _check(lib().dwkv_basis_sketch(h, group, n_rows, _ptr(k_rows), _ptr(v_rows), _ptr(omega), int(power_steps),
+                                   _ptr(eigenvalues), _stream(stream)))
+
+
+def dwkv_basis_update(h, group, n_rows, k_rows, v_rows, beta, seq_ids, eigenvalues=None, stream=None):
+    _check(lib().dwkv_basis_update(h, group, n_rows, _ptr(k_rows), _ptr(v_rows), float(beta), len(seq_ids),
+                                   _i32(seq_ids), _ptr(eigenvalues), _stream(stream)))
+
+
+def dwkv_get_bases(h, group, basis_k, basis_v, stream=None):
+    _check(lib().dwkv_get_bases(h, group, _ptr(basis_k), _ptr(basis_v), _stream(stream)))
+
+
+def dwkv_get_moment(h, group, moment, stream=None):
+    _check(lib().dwkv_get_moment(h, group, _ptr(moment), _stream(stream)))
+
+
 def dwkv_tier_controller_create(policy: dwkv_tier_policy, num_groups: int) -> C.c_void_p:
     c = C.c_void_p()
     _check(lib().dwkv_tier_controller_create(C.byref(policy), num_groups, C.byref(c)))
@@ -451,3 +474,29 @@ class Cache:
 
     def retier(self, group, seq_ids, n_tok, positions, new_tier, stream=None):
         dwkv_retier(self.h, group, seq_ids, n_tok, positions, new_tier, stream)
+
+    def basis_sketch(self, group, k_rows, v_rows, omega, power_steps=2, stream=None):
+        """k_rows / v_rows: bf16 [layers_per_group][n][Hkv][d]; omega fp32 [d][r_max].  Returns
+        the Rayleigh-Ritz eigenvalues fp32 [Hkv][2][r_max]."""
+        eig = torch.empty(self.cfg.num_kv_heads, 2, self.cfg.r_max, dtype=torch.float32, device=self.device)
+        dwkv_basis_sketch(self.h, group, k_rows.shape[1], k_rows, v_rows, omega, power_steps, eig, stream)
+        return eig
+
+    def basis_update(self, group, k_rows, v_rows, beta, seq_ids, stream=None):
+        eig = torch.empty(self.cfg.num_kv_heads, 2, self.cfg.r_max, dtype=torch.float32, device=self.device)
+        n = 0 if k_rows is None else k_rows.shape[1]
+        dwkv_basis_update(self.h, group, n, k_rows, v_rows, beta, seq_ids, eig, stream)
+        return eig
+
+    def bases(self, group, stream=None):
+        c = self.cfg
+        bk = torch.empty(c.num_kv_heads, c.head_dim, c.r_max, dtype=torch.bfloat16, device=self.device)
+        bv = torch.empty_like(bk)
+        dwkv_get_bases(self.h, group, bk, bv, stream)
+        return bk, bv
+
+    def moment(self, group, stream=None):
+        c = self.cfg
+        m = torch.empty(c.num_kv_heads, 2, c.head_dim, c.head_dim, dtype=torch.float32, device=self.device)
+        dwkv_get_moment(self.h, group, m, stream)
+        return m

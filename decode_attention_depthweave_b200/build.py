@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(HERE, "_lib")
 LIB = os.path.join(OUT_DIR, "libdwkv.so")
-SOURCES = ["dwkv_api.cu", "dwkv_cache.cu", "dwkv_control.cu", "dwkv_decode_b4.cu", "dwkv_decode_b4p.cu",
+SOURCES = ["dwkv_api.cu", "dwkv_basis.cu", "dwkv_cache.cu", "dwkv_control.cu", "dwkv_decode_b4.cu", "dwkv_decode_b4p.cu",
            "dwkv_decode_b8.cu", "dwkv_decode_b8p.cu"]
 HEADERS = ["dwkv_common.cuh", "dwkv_decode.cuh", "dwkv_encode.cuh"]
 

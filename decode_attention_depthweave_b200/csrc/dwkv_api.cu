@@ -35,6 +35,13 @@ __global__ void retier_kernel(const Geom, const State, const RetierCall, const i
 __global__ void retier_release_kernel(const Geom, const State, const RetierCall);
 __global__ void wait_timeout_kernel(const State, uint64_t);
 __global__ void tile_basis_kernel(const Geom, const State);
+__global__ void gram_kernel(const Geom, int, const __nv_bfloat16*, const __nv_bfloat16*, float*, float);
+__global__ void moment_scale_kernel(float*, size_t, float);
+__global__ void basis_kernel(const Geom, const State, int, const float*, const float*, int, float*);
+template <int BITS>
+__global__ void reproject_kernel(const Geom, const State, int, const SeqList, const __nv_bfloat16*,
+                                 const __nv_bfloat16*);
+size_t basis_smem_bytes(int r);
 template <int BITS, bool PROBE, int RMAX, int S>
 __global__ void decode_kernel(const Geom, const State, const DecodeCall);
 }  // namespace dwkv
@@ -143,7 +150,7 @@ dwkv_status check_supported(const dwkv_config* c) {
 
 struct MetaLayout {
     size_t err, bump, free_head, free_tail, free_list, counts, owned, pages, slot_map, tickets, basis_k, basis_v, basis_kt,
-        data;
+        moment, basis_old, data;
     uint32_t free_cap;
 };
 
@@ -201,6 +208,8 @@ MetaLayout meta_layout(const Geom& G) {
     M.basis_k = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
     M.basis_v = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
     M.basis_kt = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
+    M.moment = take((size_t)4 * G.G * G.Hkv * 2 * G.d * G.d);          // fp32 [G][Hkv][K|V][d][d]
+    M.basis_old = take((size_t)2 * 2 * G.Hkv * G.d * G.r_max);         // bf16 [K|V][Hkv][d][r_max]
     M.data = o;
     return M;
 }
@@ -293,9 +302,7 @@ State make_state(uint8_t* arena, const MetaLayout& M, size_t arena_bytes) {
     return S;
 }
 
-size_t encode_smem(const Geom& G) {
-    return (size_t)2 * kD * (G.r_max + 2) * 2 + (size_t)8 * (kD + kMaxRank + 32) * 4;
-}
+size_t encode_smem(const Geom& G) { return encode_smem_bytes(G.r_max); }
 size_t encode_tile_smem(const Geom& G) { return enc_tile_layout(G.r_max).total; }
 
 // Bytes of the decode page ring: what the shared-memory budget leaves after the fixed
@@ -545,6 +552,141 @@ dwkv_status dwkv_set_decode_overlap(dwkv_handle h, int32_t enable) {
     if ((st = check_handle(h)) != DWKV_OK) return st;
     if (enable != 0 && enable != 1) return fail(DWKV_ERR_INVALID_ARG, "enable must be 0 or 1 (got %d)", enable);
     h->dec_overlap = enable;
+    return DWKV_OK;
+}
+
+// ------------------------------------------------------------------------------------
+// Online bases ([DW] §3 Method, the shared-bases paragraph): sketch after prefill, moving-
+// average update with re-projection of the stored tokens.
+// ------------------------------------------------------------------------------------
+namespace {
+dwkv_status check_basis_args(dwkv_handle h, int32_t group, int32_t n_rows, const void* k_rows, const void* v_rows) {
+    const Geom& G = h->geom;
+    if (group < 0 || group >= G.G) return fail(DWKV_ERR_INVALID_ARG, "group %d out of [0, %d)", group, G.G);
+    if (G.r_max > 64) return fail(DWKV_ERR_UNSUPPORTED, "online bases are built for r_max <= 64 (got %d)", G.r_max);
+    if (n_rows < 0) return fail(DWKV_ERR_INVALID_ARG, "n_rows %d is negative", n_rows);
+    if (n_rows > 0 && (!k_rows || !v_rows)) return fail(DWKV_ERR_INVALID_ARG, "k_rows and v_rows must be non-NULL");
+    return DWKV_OK;
+}
+
+dwkv_status launch_gram(dwkv_handle h, int32_t group, int32_t n_rows, const void* k_rows, const void* v_rows,
+                        float scale, cudaStream_t s) {
+    const Geom& G = h->geom;
+    if (n_rows == 0) return DWKV_OK;
+    float* c = reinterpret_cast<float*>(h->arena + h->meta.moment) + (size_t)group * G.Hkv * 2 * kD * kD;
+    const long long rows = (long long)G.LPG * n_rows;
+    const long long want = std::max(1ll, 2ll * h->num_sms / (2 * G.Hkv));
+    const int nblk = (int)std::min(want, (rows + 63) / 64);
+    gram_kernel<<<dim3(nblk, G.Hkv, 2), 256, 0, s>>>(G, n_rows, static_cast<const __nv_bfloat16*>(k_rows),
+                                                     static_cast<const __nv_bfloat16*>(v_rows), c, scale);
+    DWKV_CUDA(cudaGetLastError(), "gram_kernel launch");
+    return DWKV_OK;
+}
+
+dwkv_status launch_basis(dwkv_handle h, int32_t group, const float* omega, int32_t power_steps, float* eig,
+                         cudaStream_t s) {
+    const Geom& G = h->geom;
+    const float* c = reinterpret_cast<const float*>(h->arena + h->meta.moment) + (size_t)group * G.Hkv * 2 * kD * kD;
+    const size_t sm = basis_smem_bytes(G.r_max);
+    DWKV_CUDA(cudaFuncSetAttribute(basis_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm),
+              "basis_kernel shared memory");
+    basis_kernel<<<2 * G.Hkv, 512, sm, s>>>(G, h->st, group, c, omega, power_steps, eig);
+    DWKV_CUDA(cudaGetLastError(), "basis_kernel launch");
+    return DWKV_OK;
+}
+}  // namespace
+
+dwkv_status dwkv_basis_sketch(dwkv_handle h, int32_t group, int32_t n_rows, const void* k_rows, const void* v_rows,
+                              const float* omega, int32_t power_steps, float* eigenvalues, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if ((st = check_basis_args(h, group, n_rows, k_rows, v_rows)) != DWKV_OK) return st;
+    if (n_rows < 1) return fail(DWKV_ERR_INVALID_ARG, "the sketch needs rows (n_rows = %d)", n_rows);
+    if (!omega) return fail(DWKV_ERR_INVALID_ARG, "omega must be non-NULL");
+    if (power_steps < 0 || power_steps > 16) return fail(DWKV_ERR_INVALID_ARG, "power_steps %d out of [0, 16]", power_steps);
+    const Geom& G = h->geom;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* c = reinterpret_cast<float*>(h->arena + h->meta.moment) + (size_t)group * G.Hkv * 2 * kD * kD;
+    DWKV_CUDA(cudaMemsetAsync(c, 0, sizeof(float) * G.Hkv * 2 * kD * kD, s), "clear the window's moment");
+    if ((st = launch_gram(h, group, n_rows, k_rows, v_rows, 1.0f, s)) != DWKV_OK) return st;
+    if ((st = launch_basis(h, group, omega, power_steps, eigenvalues, s)) != DWKV_OK) return st;
+    note_plain_launch(h);
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_basis_update(dwkv_handle h, int32_t group, int32_t n_rows, const void* k_rows, const void* v_rows,
+                              float beta, int32_t n_seqs, const int32_t* seq_ids, float* eigenvalues, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    if ((st = check_basis_args(h, group, n_rows, k_rows, v_rows)) != DWKV_OK) return st;
+    if (!(beta >= 0.f && beta <= 1.f)) return fail(DWKV_ERR_INVALID_ARG, "beta must be in [0, 1]");
+    if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
+    const Geom& G = h->geom;
+    for (int i = 0; i < n_seqs; ++i) {
+        const int sq = seq_ids[i];
+        const int pl = h->placed[(size_t)sq * G.G + group];
+        for (int l = group * G.LPG; l < (group + 1) * G.LPG; ++l)
+            if (h->len[(size_t)sq * G.L + l] != pl)
+                return fail(DWKV_ERR_INVALID_ARG, "sequence %d: layer %d holds %d positions but its group placed %d; "
+                                                  "update the basis only when every layer of the group holds the same "
+                                                  "positions",
+                            sq, l, h->len[(size_t)sq * G.L + l], pl);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* c = reinterpret_cast<float*>(h->arena + h->meta.moment) + (size_t)group * G.Hkv * 2 * kD * kD;
+    const size_t nc = (size_t)G.Hkv * 2 * kD * kD;
+    moment_scale_kernel<<<64, 256, 0, s>>>(c, nc, beta);
+    DWKV_CUDA(cudaGetLastError(), "moment_scale_kernel launch");
+    if ((st = launch_gram(h, group, n_rows, k_rows, v_rows, 1.0f - beta, s)) != DWKV_OK) return st;
+    // the current bases, for the stored tokens' reconstruction
+    const size_t bbytes = (size_t)G.Hkv * kD * G.r_max * 2;
+    uint8_t* old = h->arena + h->meta.basis_old;
+    DWKV_CUDA(cudaMemcpyAsync(old, h->arena + h->meta.basis_k + (size_t)group * bbytes, bbytes,
+                              cudaMemcpyDeviceToDevice, s), "save the K basis");
+    DWKV_CUDA(cudaMemcpyAsync(old + bbytes, h->arena + h->meta.basis_v + (size_t)group * bbytes, bbytes,
+                              cudaMemcpyDeviceToDevice, s), "save the V basis");
+    if ((st = launch_basis(h, group, nullptr, 0, eigenvalues, s)) != DWKV_OK) return st;
+    const size_t sm = encode_smem_bytes(G.r_max) + (size_t)2 * kD * (G.r_max + 2) * 2;
+    auto kern = G.bits == 8 ? reproject_kernel<8> : reproject_kernel<4>;
+    DWKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm),
+              "reproject_kernel shared memory");
+    for (int i0 = 0; i0 < n_seqs; i0 += kMaxSeqs) {
+        SeqList L;
+        memset(&L, 0, sizeof(L));
+        L.n = std::min(kMaxSeqs, n_seqs - i0);
+        for (int i = 0; i < L.n; ++i) L.seq[i] = seq_ids[i0 + i];
+        kern<<<dim3(L.n, G.Hkv), 256, sm, s>>>(G, h->st, group, L, reinterpret_cast<const __nv_bfloat16*>(old),
+                                                 reinterpret_cast<const __nv_bfloat16*>(old + bbytes));
+        DWKV_CUDA(cudaGetLastError(), "reproject_kernel launch");
+    }
+    note_plain_launch(h);
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_get_bases(dwkv_handle h, int32_t group, void* basis_k, void* basis_v, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    const Geom& G = h->geom;
+    if (group < 0 || group >= G.G) return fail(DWKV_ERR_INVALID_ARG, "group %d out of [0, %d)", group, G.G);
+    if (!basis_k || !basis_v) return fail(DWKV_ERR_INVALID_ARG, "basis_k and basis_v must be non-NULL");
+    const size_t bbytes = (size_t)G.Hkv * kD * G.r_max * 2;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DWKV_CUDA(cudaMemcpyAsync(basis_k, h->arena + h->meta.basis_k + (size_t)group * bbytes, bbytes,
+                              cudaMemcpyDefault, s), "copy the K basis");
+    DWKV_CUDA(cudaMemcpyAsync(basis_v, h->arena + h->meta.basis_v + (size_t)group * bbytes, bbytes,
+                              cudaMemcpyDefault, s), "copy the V basis");
+    return DWKV_OK;
+}
+
+dwkv_status dwkv_get_moment(dwkv_handle h, int32_t group, float* moment, void* stream) {
+    dwkv_status st;
+    if ((st = check_handle(h)) != DWKV_OK) return st;
+    const Geom& G = h->geom;
+    if (group < 0 || group >= G.G) return fail(DWKV_ERR_INVALID_ARG, "group %d out of [0, %d)", group, G.G);
+    if (!moment) return fail(DWKV_ERR_INVALID_ARG, "moment must be non-NULL");
+    const size_t nb = sizeof(float) * G.Hkv * 2 * kD * kD;
+    DWKV_CUDA(cudaMemcpyAsync(moment, h->arena + h->meta.moment + (size_t)group * nb, nb, cudaMemcpyDefault,
+                              static_cast<cudaStream_t>(stream)), "copy the moment");
     return DWKV_OK;
 }
 
@@ -991,7 +1133,7 @@ dwkv_status dwkv_sync_status(dwkv_handle h, void* stream) {
     static const char* names[] = {"none", "page pool exhausted", "tier index out of range",
                                   "residual channel index out of range", "int4 code outside [-8, 7]",
                                   "position never placed by its group", "bounded wait timed out",
-                                  "free-page ring overflow"};
+                                  "free-page ring overflow", "basis construction: a sketch column vanished"};
     const char* nm = w[0] < sizeof(names) / sizeof(names[0]) ? names[w[0]] : "unknown";
     return fail(DWKV_ERR_DEVICE_CHECK, "device check failed: %s (code %u, info %u, %u)", nm, w[0], w[1], w[2]);
 }

@@ -95,6 +95,12 @@ struct RetierCall {
     int end[kMaxSeqs];
 };
 
+// Sequences of a call that touches every stored token of theirs (basis re-projection).
+struct SeqList {
+    int n;
+    int32_t seq[kMaxSeqs];
+};
+
 struct DecodeCall {
     int n, layer, g, lig, total_splits, ring_bytes, rec_floats;
     int tok_weight;          // split balance: cost of one token in byte-equivalents

@@ -112,6 +112,12 @@ __host__ __device__ inline EncTileLayout enc_tile_layout(int r_max) {
     return L;
 }
 
+// Shared memory of an 8-warp encoder block: both bases with padded rows, then the warps'
+// scratch (enc_scratch).
+__host__ __device__ inline size_t encode_smem_bytes(int r_max) {
+    return (size_t)2 * kD * (r_max + 2) * 2 + (size_t)8 * (kD + kMaxRank + 32) * 4;
+}
+
 // Shared-memory scratch of one encode warp: x [d], stored coefficients [kMaxRank], code staging.
 struct EncScratch {
     float* xs;

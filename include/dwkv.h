@@ -78,6 +78,7 @@ typedef enum {
 #define DWKV_DEV_NO_SLOT 5          /* a layer appended a position its group never placed */
 #define DWKV_DEV_TIMEOUT 6          /* a bounded wait in a kernel ran out                 */
 #define DWKV_DEV_FREE_LIST 7        /* free-page ring overflow on reset                   */
+#define DWKV_DEV_BASIS 8            /* basis construction: a sketch column vanished        */
 
 /* Cache geometry.  Supported by this build: head_dim == 128; num_q_heads == 4 *
  * num_kv_heads; tiers drawn from {8, 16, 32, 64, 128}, strictly ascending, each <= r_max;
@@ -106,6 +107,51 @@ typedef struct {
     int32_t resid_routed;
     int32_t tier_resid[DWKV_MAX_TIERS];
 } dwkv_config;
+
+/* ---- Online bases ([DW] §3 Method, the shared-bases paragraph: "initialized online from
+ * the first compressed prefix block" by a randomized low-rank sketch of the cached keys and
+ * values after prefill, then "an exponential moving average as generation proceeds", per head
+ * and separately for keys and values).  The pages fix no sketch size or update rule; the build
+ * reads them as follows, per (window, kv-head, K or V):
+ *   C     = sum over the window's layers and rows of x x^T (the channel second moment, fp32);
+ *   sketch: Q = GS(C Omega), then power_steps times Q = GS(C Q) (Gram-Schmidt with
+ *           re-orthogonalisation, columns in order, fp64);
+ *   B     = Q U, U the eigenvectors of Q^T C Q with eigenvalues in descending order (cyclic
+ *           Jacobi), each column's largest-magnitude entry (lowest channel among equals)
+ *           positive, rounded to bf16: a token of rank r_t uses B's first r_t columns;
+ *   update: C <- beta C + (1 - beta) C_rows, then Q = GS(C B) and the same B = Q U.
+ * Online bases need r_max <= 64 (else DWKV_ERR_UNSUPPORTED). */
+
+/* Sketch the bases of window `group` from the dense rows of its layers and replace its K and V
+ * bases.  k_rows / v_rows: device bf16 [layers_per_group][n_rows][num_kv_heads][head_dim]
+ * (rows of any sequences; n_rows >= 1).  omega: device fp32 [head_dim][r_max] test matrix (the
+ * random numbers are the caller's), shared by every head, K and V.  power_steps in [0, 16].
+ * eigenvalues (nullable): device fp32 [num_kv_heads][2][r_max], the Rayleigh-Ritz values in
+ * the basis' column order.  The window's moment is reset to the rows' C.  Tokens already stored
+ * in the window are not re-projected (sketch before storing the window's tokens).  Stream-
+ * ordered; a column that vanishes in the sketch leaves the basis as it was and records
+ * DWKV_DEV_BASIS. */
+dwkv_status dwkv_basis_sketch(dwkv_handle h, int32_t group, int32_t n_rows, const void* k_rows, const void* v_rows,
+                              const float* omega, int32_t power_steps, float* eigenvalues, void* stream);
+
+/* Moving-average update of window `group`'s bases: C <- beta C + (1 - beta) C_rows over the new
+ * dense rows (n_rows >= 0, layout as dwkv_basis_sketch; 0 rows: C is only scaled), the bases
+ * refreshed from C, then every stored token of the listed sequences (host seq_ids) re-projected
+ * onto them: each (token, layer of the window, K / V) is reconstructed on the previous basis
+ * (the fixed-order fp32 chain over its rank plus scale x code, rounded to bf16, as dwkv_retier
+ * does) and encoded on the new basis at its own tier, in place.  Every layer of the window
+ * must hold the same positions for each listed sequence (DWKV_ERR_INVALID_ARG otherwise).
+ * beta in [0, 1].  eigenvalues: as dwkv_basis_sketch.  Tokens of sequences not listed keep
+ * their bytes and are then stale against the new bases: list every sequence that holds tokens
+ * in the window. */
+dwkv_status dwkv_basis_update(dwkv_handle h, int32_t group, int32_t n_rows, const void* k_rows, const void* v_rows,
+                              float beta, int32_t n_seqs, const int32_t* seq_ids, float* eigenvalues, void* stream);
+
+/* Copies of window `group`'s bases (bf16 [num_kv_heads][head_dim][r_max] each; host or device
+ * destinations) and of its second moment (fp32 [num_kv_heads][2][head_dim][head_dim]).
+ * Stream-ordered; synchronise before reading a host copy. */
+dwkv_status dwkv_get_bases(dwkv_handle h, int32_t group, void* basis_k, void* basis_v, void* stream);
+dwkv_status dwkv_get_moment(dwkv_handle h, int32_t group, float* moment, void* stream);
 
 /* Library version string. */
 const char* dwkv_version(void);

@@ -310,6 +310,13 @@ def make_dense_vectors(wl: Workload, seq: int, layer: int, n: int, bases, device
     return out[0], out[1]
 
 
+def make_test_matrix(wl: Workload, seed: int | None = None, device="cpu") -> torch.Tensor:
+    """The basis sketch's Gaussian test matrix, fp32 ``[d][r_max]`` ~ N(0, 1)."""
+    seed = wl.base_seed if seed is None else seed
+    g = _gen("cpu", seed_for(seed, "omega"))
+    return torch.randn(wl.head_dim, wl.r_max, generator=g, dtype=torch.float32).to(device)
+
+
 RESIDUAL_CASE_KINDS = ("gaussian", "boundary_ulp", "boundary_tie", "top_tie", "few_nonzero", "zeros",
                        "subnormal", "huge", "half_steps")
 
