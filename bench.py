@@ -810,6 +810,43 @@ def run_encode(args, world, rank, local):
                          "bf16 input, the rate the step's vectors would see",
                "nproc": cores, "cpu_model": cpu_model()}
 
+    # ---- online bases of window 0 (f2): the moving-average update with the re-projection of
+    #      every stored token of the window (valid: the tokens were encoded on the current
+    #      bases), then a sketch from the window's prefill rows (it replaces the bases; the cache
+    #      is not used after it)
+    online = None
+    if wl.r_max <= 64:
+        L = wl.num_layers
+        n_upd = 1024
+        u0, u1, s0, s1 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+        with torch.cuda.stream(stream):                  # the inputs are made on the launching stream
+            k_upd = torch.stack([K[l][:n_upd] for l in range(L)]).contiguous()
+            v_upd = torch.stack([V[l][:n_upd] for l in range(L)]).contiguous()
+            omega = synth.make_test_matrix(wl, device=dev)
+            u0.record(stream)
+            dw.dwkv_basis_update(h, dw.DWKV_ALL_GROUPS, n_upd, k_upd, v_upd, 0.9, seqs, None, stream)
+            u1.record(stream)
+        torch.cuda.synchronize(dev)
+        del k_upd, v_upd
+        with torch.cuda.stream(stream):
+            k_sk = torch.stack(K).contiguous()
+            v_sk = torch.stack(V).contiguous()
+            s0.record(stream)
+            dw.dwkv_basis_sketch(h, dw.DWKV_ALL_GROUPS, k_sk.shape[1], k_sk, v_sk, omega, 2, None, stream)
+            s1.record(stream)
+        torch.cuda.synchronize(dev)
+        cache.sync(stream)
+        del k_sk, v_sk
+        upd_ms, sk_ms = u0.elapsed_time(u1), s0.elapsed_time(s1)
+        rows = L * B * N                                     # rows a kv-head, all windows
+        moment_flops = 2.0 * rows * wl.head_dim * wl.head_dim * wl.num_kv_heads * 2
+        n_rep = B * held * wl.num_kv_heads * L * 2
+        online = {"sketch_ms": round(sk_ms, 4), "windows": wl.num_groups, "sketch_rows_per_head": rows,
+                  "power_steps": 2, "moment_tflops_lower_bound": round(moment_flops / (sk_ms * 1e-3) / 1e12, 2),
+                  "update_ms": round(upd_ms, 4), "update_rows_per_head": L * n_upd,
+                  "reprojected_vectors": n_rep, "reprojected_vectors_per_s": round(n_rep / (upd_ms * 1e-3), 1),
+                  "timing": "every window in one call each (update first, on the encoded cache), CUDA events"}
+
     value = aggregate_rate(world, dense / 1e9, ms_per_step)
     res = {
         "metric": "bulk encode: dense bf16 K/V GB/s compressed (a7)", "value": round(value, 2), "unit": "GB/s",
@@ -839,6 +876,7 @@ def run_encode(args, world, rank, local):
         "probe": {"ms_all_layers": round(probe_ms, 4),
                   "achieved_gbs": round(dec_bytes / (probe_ms * 1e-3) / 1e9, 1),
                   "frac": round(dec_bytes / (probe_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+        "online_basis": online,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
@@ -902,7 +940,7 @@ def summary_of(res: dict) -> dict:
     """The keys of a workload's line that the default run repeats for the extra workloads."""
     keep = ("metric", "value", "unit", "ms_per_step", "steps", "warmup", "config", "gpu_launches", "roofline",
             "compressed_gb_per_step", "compressed_tb_s", "probe", "e2e", "cpu_baseline", "clocks", "hbm",
-            "decode_step", "vectors_per_s")
+            "decode_step", "vectors_per_s", "online_basis")
     return {k: res[k] for k in keep if k in res}
 
 

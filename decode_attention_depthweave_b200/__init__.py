@@ -26,13 +26,14 @@ __all__ = [
     "dwkv_retier", "dwkv_tier_policy", "dwkv_tier_controller_create", "dwkv_tier_controller_destroy",
     "dwkv_tier_controller_due", "dwkv_tier_controller_threshold", "dwkv_tier_controller_observe",
     "dwkv_tier_controller_route", "dwkv_arena_bytes_all_tiers", "dwkv_basis_sketch", "dwkv_basis_update",
-    "dwkv_get_bases", "dwkv_get_moment", "Cache", "EXPORTED_SYMBOLS",
+    "dwkv_get_bases", "dwkv_get_moment", "DWKV_ALL_GROUPS", "Cache", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libdwkv.so")
 
 DWKV_OK = 0
+DWKV_ALL_GROUPS = -1
 STATUS_NAMES = {0: "DWKV_OK", 1: "DWKV_ERR_INVALID_ARG", 2: "DWKV_ERR_CAPACITY", 3: "DWKV_ERR_CUDA",
                 4: "DWKV_ERR_DEVICE_CHECK", 5: "DWKV_ERR_UNSUPPORTED"}
 
@@ -475,18 +476,24 @@ class Cache:
     def retier(self, group, seq_ids, n_tok, positions, new_tier, stream=None):
         dwkv_retier(self.h, group, seq_ids, n_tok, positions, new_tier, stream)
 
+    def _windows(self, group):
+        return self.cfg.num_layers // self.cfg.layers_per_group if group == DWKV_ALL_GROUPS else 1
+
     def basis_sketch(self, group, k_rows, v_rows, omega, power_steps=2, stream=None):
-        """k_rows / v_rows: bf16 [layers_per_group][n][Hkv][d]; omega fp32 [d][r_max].  Returns
-        the Rayleigh-Ritz eigenvalues fp32 [Hkv][2][r_max]."""
-        eig = torch.empty(self.cfg.num_kv_heads, 2, self.cfg.r_max, dtype=torch.float32, device=self.device)
+        """k_rows / v_rows: bf16 [layers][n][Hkv][d] (the window's layers, or every layer with
+        group = DWKV_ALL_GROUPS); omega fp32 [d][r_max].  Returns the Rayleigh-Ritz eigenvalues
+        fp32 [windows][Hkv][2][r_max] ([Hkv][2][r_max] for one window)."""
+        w = self._windows(group)
+        eig = torch.empty(w, self.cfg.num_kv_heads, 2, self.cfg.r_max, dtype=torch.float32, device=self.device)
         dwkv_basis_sketch(self.h, group, k_rows.shape[1], k_rows, v_rows, omega, power_steps, eig, stream)
-        return eig
+        return eig[0] if group != DWKV_ALL_GROUPS else eig
 
     def basis_update(self, group, k_rows, v_rows, beta, seq_ids, stream=None):
-        eig = torch.empty(self.cfg.num_kv_heads, 2, self.cfg.r_max, dtype=torch.float32, device=self.device)
+        w = self._windows(group)
+        eig = torch.empty(w, self.cfg.num_kv_heads, 2, self.cfg.r_max, dtype=torch.float32, device=self.device)
         n = 0 if k_rows is None else k_rows.shape[1]
         dwkv_basis_update(self.h, group, n, k_rows, v_rows, beta, seq_ids, eig, stream)
-        return eig
+        return eig[0] if group != DWKV_ALL_GROUPS else eig
 
     def bases(self, group, stream=None):
         c = self.cfg

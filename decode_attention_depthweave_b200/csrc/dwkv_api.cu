@@ -209,7 +209,7 @@ MetaLayout meta_layout(const Geom& G) {
     M.basis_v = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
     M.basis_kt = take((size_t)2 * G.G * G.Hkv * G.d * G.r_max);
     M.moment = take((size_t)4 * G.G * G.Hkv * 2 * G.d * G.d);          // fp32 [G][Hkv][K|V][d][d]
-    M.basis_old = take((size_t)2 * 2 * G.Hkv * G.d * G.r_max);         // bf16 [K|V][Hkv][d][r_max]
+    M.basis_old = take((size_t)2 * 2 * G.G * G.Hkv * G.d * G.r_max);   // bf16 [K|V][G][Hkv][d][r_max]
     M.data = o;
     return M;
 }
@@ -478,6 +478,8 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
     cudaError_t e = cudaMemsetAsync(h->arena, 0, M.basis_k, s);
     if (e == cudaSuccess) e = cudaMemcpyAsync(h->arena + M.basis_k, basis_k, bbytes, cudaMemcpyDeviceToDevice, s);
     if (e == cudaSuccess) e = cudaMemcpyAsync(h->arena + M.basis_v, basis_v, bbytes, cudaMemcpyDeviceToDevice, s);
+    // the windows' second moments start at zero (an update before any sketch averages from 0)
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->arena + M.moment, 0, M.basis_old - M.moment, s);
     if (e == cudaSuccess) {
         tile_basis_kernel<<<G.G * G.Hkv, 256, 0, s>>>(G, h->st);
         e = cudaGetLastError();
@@ -560,37 +562,50 @@ dwkv_status dwkv_set_decode_overlap(dwkv_handle h, int32_t enable) {
 // average update with re-projection of the stored tokens.
 // ------------------------------------------------------------------------------------
 namespace {
-dwkv_status check_basis_args(dwkv_handle h, int32_t group, int32_t n_rows, const void* k_rows, const void* v_rows) {
+// Windows [g0, g0 + ng) of a basis call: group >= 0 one window, DWKV_ALL_GROUPS every window.
+dwkv_status basis_windows(dwkv_handle h, int32_t group, int* g0, int* ng) {
     const Geom& G = h->geom;
+    if (group == DWKV_ALL_GROUPS) { *g0 = 0; *ng = G.G; return DWKV_OK; }
     if (group < 0 || group >= G.G) return fail(DWKV_ERR_INVALID_ARG, "group %d out of [0, %d)", group, G.G);
+    *g0 = group;
+    *ng = 1;
+    return DWKV_OK;
+}
+
+dwkv_status check_basis_args(dwkv_handle h, int32_t n_rows, const void* k_rows, const void* v_rows) {
+    const Geom& G = h->geom;
     if (G.r_max > 64) return fail(DWKV_ERR_UNSUPPORTED, "online bases are built for r_max <= 64 (got %d)", G.r_max);
     if (n_rows < 0) return fail(DWKV_ERR_INVALID_ARG, "n_rows %d is negative", n_rows);
     if (n_rows > 0 && (!k_rows || !v_rows)) return fail(DWKV_ERR_INVALID_ARG, "k_rows and v_rows must be non-NULL");
     return DWKV_OK;
 }
 
-dwkv_status launch_gram(dwkv_handle h, int32_t group, int32_t n_rows, const void* k_rows, const void* v_rows,
+float* moment_of(dwkv_handle h, int g) {
+    const Geom& G = h->geom;
+    return reinterpret_cast<float*>(h->arena + h->meta.moment) + (size_t)g * G.Hkv * 2 * kD * kD;
+}
+
+dwkv_status launch_gram(dwkv_handle h, int g0, int ng, int32_t n_rows, const void* k_rows, const void* v_rows,
                         float scale, cudaStream_t s) {
     const Geom& G = h->geom;
     if (n_rows == 0) return DWKV_OK;
-    float* c = reinterpret_cast<float*>(h->arena + h->meta.moment) + (size_t)group * G.Hkv * 2 * kD * kD;
     const long long rows = (long long)G.LPG * n_rows;
-    const long long want = std::max(1ll, 2ll * h->num_sms / (2 * G.Hkv));
+    const long long want = std::max(1ll, 2ll * h->num_sms / (2ll * G.Hkv * ng));
     const int nblk = (int)std::min(want, (rows + 63) / 64);
-    gram_kernel<<<dim3(nblk, G.Hkv, 2), 256, 0, s>>>(G, n_rows, static_cast<const __nv_bfloat16*>(k_rows),
-                                                     static_cast<const __nv_bfloat16*>(v_rows), c, scale);
+    gram_kernel<<<dim3(nblk, G.Hkv * ng, 2), 256, 0, s>>>(G, n_rows, static_cast<const __nv_bfloat16*>(k_rows),
+                                                          static_cast<const __nv_bfloat16*>(v_rows), moment_of(h, g0),
+                                                          scale);
     DWKV_CUDA(cudaGetLastError(), "gram_kernel launch");
     return DWKV_OK;
 }
 
-dwkv_status launch_basis(dwkv_handle h, int32_t group, const float* omega, int32_t power_steps, float* eig,
+dwkv_status launch_basis(dwkv_handle h, int g0, int ng, const float* omega, int32_t power_steps, float* eig,
                          cudaStream_t s) {
     const Geom& G = h->geom;
-    const float* c = reinterpret_cast<const float*>(h->arena + h->meta.moment) + (size_t)group * G.Hkv * 2 * kD * kD;
     const size_t sm = basis_smem_bytes(G.r_max);
     DWKV_CUDA(cudaFuncSetAttribute(basis_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm),
               "basis_kernel shared memory");
-    basis_kernel<<<2 * G.Hkv, 512, sm, s>>>(G, h->st, group, c, omega, power_steps, eig);
+    basis_kernel<<<dim3(2 * G.Hkv, ng), 512, sm, s>>>(G, h->st, g0, moment_of(h, g0), omega, power_steps, eig);
     DWKV_CUDA(cudaGetLastError(), "basis_kernel launch");
     return DWKV_OK;
 }
@@ -600,16 +615,18 @@ dwkv_status dwkv_basis_sketch(dwkv_handle h, int32_t group, int32_t n_rows, cons
                               const float* omega, int32_t power_steps, float* eigenvalues, void* stream) {
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
-    if ((st = check_basis_args(h, group, n_rows, k_rows, v_rows)) != DWKV_OK) return st;
+    int g0 = 0, ng = 0;
+    if ((st = basis_windows(h, group, &g0, &ng)) != DWKV_OK) return st;
+    if ((st = check_basis_args(h, n_rows, k_rows, v_rows)) != DWKV_OK) return st;
     if (n_rows < 1) return fail(DWKV_ERR_INVALID_ARG, "the sketch needs rows (n_rows = %d)", n_rows);
     if (!omega) return fail(DWKV_ERR_INVALID_ARG, "omega must be non-NULL");
     if (power_steps < 0 || power_steps > 16) return fail(DWKV_ERR_INVALID_ARG, "power_steps %d out of [0, 16]", power_steps);
     const Geom& G = h->geom;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    float* c = reinterpret_cast<float*>(h->arena + h->meta.moment) + (size_t)group * G.Hkv * 2 * kD * kD;
-    DWKV_CUDA(cudaMemsetAsync(c, 0, sizeof(float) * G.Hkv * 2 * kD * kD, s), "clear the window's moment");
-    if ((st = launch_gram(h, group, n_rows, k_rows, v_rows, 1.0f, s)) != DWKV_OK) return st;
-    if ((st = launch_basis(h, group, omega, power_steps, eigenvalues, s)) != DWKV_OK) return st;
+    DWKV_CUDA(cudaMemsetAsync(moment_of(h, g0), 0, sizeof(float) * ng * G.Hkv * 2 * kD * kD, s),
+              "clear the windows' moments");
+    if ((st = launch_gram(h, g0, ng, n_rows, k_rows, v_rows, 1.0f, s)) != DWKV_OK) return st;
+    if ((st = launch_basis(h, g0, ng, omega, power_steps, eigenvalues, s)) != DWKV_OK) return st;
     note_plain_launch(h);
     return DWKV_OK;
 }
@@ -618,34 +635,36 @@ dwkv_status dwkv_basis_update(dwkv_handle h, int32_t group, int32_t n_rows, cons
                               float beta, int32_t n_seqs, const int32_t* seq_ids, float* eigenvalues, void* stream) {
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
-    if ((st = check_basis_args(h, group, n_rows, k_rows, v_rows)) != DWKV_OK) return st;
+    int g0 = 0, ng = 0;
+    if ((st = basis_windows(h, group, &g0, &ng)) != DWKV_OK) return st;
+    if ((st = check_basis_args(h, n_rows, k_rows, v_rows)) != DWKV_OK) return st;
     if (!(beta >= 0.f && beta <= 1.f)) return fail(DWKV_ERR_INVALID_ARG, "beta must be in [0, 1]");
     if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
     const Geom& G = h->geom;
     for (int i = 0; i < n_seqs; ++i) {
         const int sq = seq_ids[i];
-        const int pl = h->placed[(size_t)sq * G.G + group];
-        for (int l = group * G.LPG; l < (group + 1) * G.LPG; ++l)
-            if (h->len[(size_t)sq * G.L + l] != pl)
-                return fail(DWKV_ERR_INVALID_ARG, "sequence %d: layer %d holds %d positions but its group placed %d; "
-                                                  "update the basis only when every layer of the group holds the same "
-                                                  "positions",
-                            sq, l, h->len[(size_t)sq * G.L + l], pl);
+        for (int g = g0; g < g0 + ng; ++g) {
+            const int pl = h->placed[(size_t)sq * G.G + g];
+            for (int l = g * G.LPG; l < (g + 1) * G.LPG; ++l)
+                if (h->len[(size_t)sq * G.L + l] != pl)
+                    return fail(DWKV_ERR_INVALID_ARG, "sequence %d: layer %d holds %d positions but its group placed %d; "
+                                                      "update the basis only when every layer of the group holds the "
+                                                      "same positions",
+                                sq, l, h->len[(size_t)sq * G.L + l], pl);
+        }
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    float* c = reinterpret_cast<float*>(h->arena + h->meta.moment) + (size_t)group * G.Hkv * 2 * kD * kD;
-    const size_t nc = (size_t)G.Hkv * 2 * kD * kD;
-    moment_scale_kernel<<<64, 256, 0, s>>>(c, nc, beta);
+    moment_scale_kernel<<<128, 256, 0, s>>>(moment_of(h, g0), (size_t)ng * G.Hkv * 2 * kD * kD, beta);
     DWKV_CUDA(cudaGetLastError(), "moment_scale_kernel launch");
-    if ((st = launch_gram(h, group, n_rows, k_rows, v_rows, 1.0f - beta, s)) != DWKV_OK) return st;
-    // the current bases, for the stored tokens' reconstruction
+    if ((st = launch_gram(h, g0, ng, n_rows, k_rows, v_rows, 1.0f - beta, s)) != DWKV_OK) return st;
+    // the current bases, for the stored tokens' reconstruction: [K|V][window][Hkv][d][r_max]
     const size_t bbytes = (size_t)G.Hkv * kD * G.r_max * 2;
     uint8_t* old = h->arena + h->meta.basis_old;
-    DWKV_CUDA(cudaMemcpyAsync(old, h->arena + h->meta.basis_k + (size_t)group * bbytes, bbytes,
-                              cudaMemcpyDeviceToDevice, s), "save the K basis");
-    DWKV_CUDA(cudaMemcpyAsync(old + bbytes, h->arena + h->meta.basis_v + (size_t)group * bbytes, bbytes,
-                              cudaMemcpyDeviceToDevice, s), "save the V basis");
-    if ((st = launch_basis(h, group, nullptr, 0, eigenvalues, s)) != DWKV_OK) return st;
+    DWKV_CUDA(cudaMemcpyAsync(old, h->arena + h->meta.basis_k + (size_t)g0 * bbytes, ng * bbytes,
+                              cudaMemcpyDeviceToDevice, s), "save the K bases");
+    DWKV_CUDA(cudaMemcpyAsync(old + ng * bbytes, h->arena + h->meta.basis_v + (size_t)g0 * bbytes, ng * bbytes,
+                              cudaMemcpyDeviceToDevice, s), "save the V bases");
+    if ((st = launch_basis(h, g0, ng, nullptr, 0, eigenvalues, s)) != DWKV_OK) return st;
     const size_t sm = encode_smem_bytes(G.r_max) + (size_t)2 * kD * (G.r_max + 2) * 2;
     auto kern = G.bits == 8 ? reproject_kernel<8> : reproject_kernel<4>;
     DWKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm),
@@ -655,9 +674,14 @@ dwkv_status dwkv_basis_update(dwkv_handle h, int32_t group, int32_t n_rows, cons
         memset(&L, 0, sizeof(L));
         L.n = std::min(kMaxSeqs, n_seqs - i0);
         for (int i = 0; i < L.n; ++i) L.seq[i] = seq_ids[i0 + i];
-        kern<<<dim3(L.n, G.Hkv), 256, sm, s>>>(G, h->st, group, L, reinterpret_cast<const __nv_bfloat16*>(old),
-                                                 reinterpret_cast<const __nv_bfloat16*>(old + bbytes));
-        DWKV_CUDA(cudaGetLastError(), "reproject_kernel launch");
+        // blocks per (sequence, kv-head): enough for ~3 blocks per SM over the call
+        const int per = std::max(1, (3 * h->num_sms + L.n * G.Hkv - 1) / (L.n * G.Hkv));
+        for (int g = g0; g < g0 + ng; ++g) {
+            const __nv_bfloat16* ok_ = reinterpret_cast<const __nv_bfloat16*>(old + (size_t)(g - g0) * bbytes);
+            const __nv_bfloat16* ov_ = reinterpret_cast<const __nv_bfloat16*>(old + (size_t)(ng + g - g0) * bbytes);
+            kern<<<dim3(L.n, G.Hkv, per), 256, sm, s>>>(G, h->st, g, L, ok_, ov_);
+            DWKV_CUDA(cudaGetLastError(), "reproject_kernel launch");
+        }
     }
     note_plain_launch(h);
     return DWKV_OK;

@@ -16,8 +16,8 @@
 namespace dwkv {
 
 // ------------------------------------------------------------------------------------
-// Second moment C[h][z] += scale * X^T X over rows [row0, row0 + nrows) of the window's
-// layers (rows = LPG x n_rows, layer-major), on the tensor cores.  A block of 8 warps: warp w
+// Second moment C[w][h][z] += scale * X^T X over the rows of window w's layers (rows = LPG x
+// n_rows, layer-major; blockIdx.y = w Hkv + h), on the tensor cores.  A block of 8 warps: warp w
 // owns channels [16 w, 16 w + 16) of C's rows and all 128 columns (16 n-tiles); chunks of 64
 // rows are staged as bf16 [64][136] (a 272-byte pitch: ldmatrix rows on distinct banks).
 // Partial sums go to C with fp32 atomics, so the order of the sum is not fixed.
@@ -28,10 +28,11 @@ __global__ void __launch_bounds__(256) gram_kernel(const Geom G, int n_rows, con
                                                    const __nv_bfloat16* __restrict__ v_rows, float* __restrict__ cacc,
                                                    float scale) {
     __shared__ __align__(16) __nv_bfloat16 xs[kGramRows * kGramPitch];
-    const int h = blockIdx.y, z = blockIdx.z;
+    const int h = blockIdx.y % G.Hkv, gw = blockIdx.y / G.Hkv, z = blockIdx.z;   // gw: window within the call
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3, mi = lane >> 3, rr = lane & 7;
-    const __nv_bfloat16* src = z ? v_rows : k_rows;
+    const __nv_bfloat16* src = (z ? v_rows : k_rows) + (size_t)gw * G.LPG * n_rows * G.Hkv * kD;
+    cacc += (size_t)gw * G.Hkv * 2 * kD * kD;
     const long long total = (long long)G.LPG * n_rows;
     const long long per = (total + gridDim.x - 1) / gridDim.x;
     const long long r0 = (long long)blockIdx.x * per, r1 = r0 + per < total ? r0 + per : total;
@@ -163,6 +164,8 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
     extern __shared__ __align__(16) uint8_t smem[];
     const int r = G.r_max;
     const int h = blockIdx.x >> 1, z = blockIdx.x & 1;
+    g += blockIdx.y;                                        // all-windows launches: one row of blocks a window
+    moment += (size_t)blockIdx.y * G.Hkv * 2 * kD * kD;
     const int tid = threadIdx.x;
     double* q = reinterpret_cast<double*>(smem);            // [d][r]
     double* w = q + kD * r;                                 // [d][r]; later U [r][r]
@@ -296,7 +299,7 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
             if (m > bm) { bm = m; best = i; }
         }
         dots[tid] = q[best * r + tid] < 0.0 ? -1.0 : 1.0;
-        if (eig_out) eig_out[((size_t)h * 2 + z) * r + tid] = (float)lam[ord[tid]];
+        if (eig_out) eig_out[(((size_t)blockIdx.y * G.Hkv + h) * 2 + z) * r + tid] = (float)lam[ord[tid]];
     }
     __syncthreads();
     __nv_bfloat16* tk = const_cast<__nv_bfloat16*>(S.basis_kt) + boff;
@@ -309,8 +312,9 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
 }
 
 // ------------------------------------------------------------------------------------
-// Re-projection of the stored tokens of a window onto its updated basis: a block per
-// (sequence in the list, kv-head), a warp per (slot, layer of the window, K / V) unit.  Each
+// Re-projection of the stored tokens of a window onto its updated basis: gridDim.z blocks per
+// (sequence in the list, kv-head), a warp per (slot, layer of the window, K / V) unit, the
+// units of a (sequence, kv-head) dealt out over its blocks' warps.  Each
 // unit is reconstructed on the previous basis (old_k / old_v: the fixed-order fp32 chain over
 // its rank, plus scale x code on its residual channels, rounded to bf16, as a re-tier does)
 // and encoded on the new basis at its own tier, in place.  Slots and counts do not change.
@@ -343,7 +347,8 @@ __global__ void __launch_bounds__(256) reproject_kernel(const Geom G, const Stat
     }
     __syncthreads();
     const uint32_t units = s_base[kMaxTiers] * (uint32_t)G.LPG * 2u;
-    for (uint32_t u = warp; u < units; u += blockDim.x >> 5) {
+    const uint32_t nw = (blockDim.x >> 5) * gridDim.z;
+    for (uint32_t u = blockIdx.z * (blockDim.x >> 5) + warp; u < units; u += nw) {
         const uint32_t z = u & 1u, lig = (u >> 1) % (uint32_t)G.LPG, slotg = (u >> 1) / (uint32_t)G.LPG;
         int k = 0;
         while (k + 1 < kMaxTiers && slotg >= s_base[k + 1]) ++k;

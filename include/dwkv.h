@@ -122,19 +122,23 @@ typedef struct {
  *   update: C <- beta C + (1 - beta) C_rows, then Q = GS(C B) and the same B = Q U.
  * Online bases need r_max <= 64 (else DWKV_ERR_UNSUPPORTED). */
 
-/* Sketch the bases of window `group` from the dense rows of its layers and replace its K and V
- * bases.  k_rows / v_rows: device bf16 [layers_per_group][n_rows][num_kv_heads][head_dim]
- * (rows of any sequences; n_rows >= 1).  omega: device fp32 [head_dim][r_max] test matrix (the
+#define DWKV_ALL_GROUPS (-1)
+
+/* Sketch the bases of window `group` (or of every window: DWKV_ALL_GROUPS, in one launch)
+ * from the dense rows of its layers and replace its K and V bases.  k_rows / v_rows: device
+ * bf16 [layers][n_rows][num_kv_heads][head_dim] with layers = layers_per_group for one window,
+ * num_layers for all (rows of any sequences; n_rows >= 1).  omega: device fp32 [head_dim][r_max] test matrix (the
  * random numbers are the caller's), shared by every head, K and V.  power_steps in [0, 16].
- * eigenvalues (nullable): device fp32 [num_kv_heads][2][r_max], the Rayleigh-Ritz values in
- * the basis' column order.  The window's moment is reset to the rows' C.  Tokens already stored
+ * eigenvalues (nullable): device fp32 [windows][num_kv_heads][2][r_max], the Rayleigh-Ritz
+ * values in the basis' column order.  The window's moment is reset to the rows' C.  Tokens already stored
  * in the window are not re-projected (sketch before storing the window's tokens).  Stream-
  * ordered; a column that vanishes in the sketch leaves the basis as it was and records
  * DWKV_DEV_BASIS. */
 dwkv_status dwkv_basis_sketch(dwkv_handle h, int32_t group, int32_t n_rows, const void* k_rows, const void* v_rows,
                               const float* omega, int32_t power_steps, float* eigenvalues, void* stream);
 
-/* Moving-average update of window `group`'s bases: C <- beta C + (1 - beta) C_rows over the new
+/* Moving-average update of window `group`'s bases (or every window's: DWKV_ALL_GROUPS):
+ * C <- beta C + (1 - beta) C_rows over the new
  * dense rows (n_rows >= 0, layout as dwkv_basis_sketch; 0 rows: C is only scaled), the bases
  * refreshed from C, then every stored token of the listed sequences (host seq_ids) re-projected
  * onto them: each (token, layer of the window, K / V) is reconstructed on the previous basis

@@ -208,3 +208,74 @@ def test_basis_calls_refuse_bad_arguments():
     kr = torch.zeros(4, 16, 2, 128, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(dw.DwkvError):
         dw.dwkv_basis_sketch(c2.h, 0, 16, kr, kr, torch.zeros(128, 128, device="cuda"))
+
+
+def test_every_window_in_one_call():
+    """DWKV_ALL_GROUPS: one launch sketches (and updates) every window from all layers' rows;
+    each window's moment and basis match the oracle as for a single window, and the update
+    re-projects the tokens of every window."""
+    wl = _wl(num_layers=4)                                       # two windows of two layers
+    bases = synth.make_bases(wl)
+    cache = dw.Cache(cfg_for(wl, max_context=700), bases[0], bases[1])
+    lengths = [300, 199]
+    per_layer, k_rows, v_rows = _rows(wl, bases, lengths)       # [4][n][H][d]
+    omega = synth.make_test_matrix(wl)
+    eig = cache.basis_sketch(dw.DWKV_ALL_GROUPS, k_rows.cuda(), v_rows.cuda(), omega.cuda(), power_steps=2)
+    cache.sync()
+    assert eig.shape[0] == 2
+    bw = {}
+    for g in range(2):
+        bk, bv = cache.bases(g)
+        mom = cache.moment(g)
+        cache.sync()
+        bw[g] = (bk.cpu(), bv.cpu())
+        for h in range(wl.num_kv_heads):
+            for z, rows in enumerate((k_rows, v_rows)):
+                x = _f64(rows[2 * g:2 * g + 2, :, h].reshape(-1, wl.head_dim))
+                c_gpu = mom[h, z].cpu().numpy().astype(np.float64)
+                c_or = ob.gram(x)
+                assert np.linalg.norm(c_gpu - c_or) <= 1e-5 * np.linalg.norm(c_or), (g, h, z)
+                b_or, w_or = ob.sketch_basis(c_gpu, omega.numpy().astype(np.float64), power_steps=2)
+                _check_basis(_f64(bw[g][z][h]), b_or, w_or, f"window {g} head {h} z {z}")
+    tiers = {g: [synth.make_tiers(wl, b, g, n) for b, n in enumerate(lengths)] for g in range(2)}
+    for layer in range(4):
+        k, v = per_layer[layer]
+        g = layer // 2
+        cache.append(layer, [0, 1], lengths, k.cuda(), v.cuda(), torch.cat(tiers[g]).cuda() if layer % 2 == 0 else None)
+    cache.sync()
+    before = {(b, layer): cache.export(layer, b, 0, lengths[b]) for b in range(2) for layer in (1, 2)}
+    cache.basis_update(dw.DWKV_ALL_GROUPS, k_rows[:, :64].contiguous().cuda(), v_rows[:, :64].contiguous().cuda(),
+                       0.5, [0, 1])
+    cache.sync()
+    new = {g: tuple(t.cpu() for t in cache.bases(g)) for g in range(2)}
+    cache.sync()
+    for (b, layer), old in before.items():
+        g = layer // 2
+        got = cache.export(layer, b, 0, lengths[b])
+        oc = {k_: v_.cpu() for k_, v_ in old.items()}
+        for t in range(0, lengths[b], 23):
+            for h in range(wl.num_kv_heads):
+                r = wl.tiers[int(oc["tier_idx"][t, h])]
+                for z in range(2):
+                    ref = oracle.reencode_vector(bw[g][z][h], r, oc["coeff"][t, h, z], oc["idx"][t, h, z],
+                                                 oc["codes"][t, h, z], oc["scales"][t, h, z], r, wl.resid_bits,
+                                                 basis_new=new[g][z][h])
+                    gc = got["coeff"][t, h, z].cpu().view(torch.int16).numpy().view(np.uint16)
+                    assert np.array_equal(gc, ref["coeff"]), (b, layer, t, h, z)
+                    assert np.array_equal(got["idx"][t, h, z].cpu().numpy(), ref["idx"]), (b, layer, t, h, z)
+
+
+def test_update_before_any_sketch_averages_from_zero():
+    """A window's moment starts at zero: an update without a sketch gives (1 - beta) C_rows."""
+    wl = _wl()
+    bases = synth.make_bases(wl)
+    cache = dw.Cache(cfg_for(wl, max_context=300), bases[0], bases[1])
+    _, k_rows, v_rows = _rows(wl, bases, [200])
+    cache.basis_update(0, k_rows.cuda(), v_rows.cuda(), 0.75, [])
+    mom = cache.moment(0)
+    cache.sync()
+    for h in range(wl.num_kv_heads):
+        for z, rows in enumerate((k_rows, v_rows)):
+            want = 0.25 * ob.gram(_f64(rows[:, :, h].reshape(-1, wl.head_dim)))
+            got = mom[h, z].cpu().numpy().astype(np.float64)
+            assert np.linalg.norm(got - want) <= 1e-5 * np.linalg.norm(want), (h, z)
