@@ -31,11 +31,11 @@ def lib():
         p = C.c_void_p
         i = C.c_int
         d = C.c_double
-        L.oracle_decode_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, i, p, p, p]
+        L.oracle_decode_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, i, p, p, p, p, p]
         L.oracle_decode_head.restype = i
-        L.oracle_probe_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, d, p, p, p, p]
+        L.oracle_probe_head.argtypes = [i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p, d, d, p, p, p, p, p, p]
         L.oracle_probe_head.restype = i
-        L.oracle_decode_many.argtypes = [i, i, i, i, i, p] + [p] * 12 + [d, p, i, p]
+        L.oracle_decode_many.argtypes = [i, i, i, i, i, p] + [p] * 12 + [d, p, i, p, p, p]
         L.oracle_decode_many.restype = i
         L.oracle_encode_vector.argtypes = [i, i, p, p, i, i, i, p, p, p, p, p, p]
         L.oracle_encode_vector.restype = i
@@ -49,6 +49,12 @@ def lib():
         L.oracle_reencode_vector.restype = i
         L.oracle_reconstruct.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, p]
         L.oracle_reconstruct.restype = None
+        L.oracle_quantize_coeffs8.argtypes = [i, i, p, p, p, p]
+        L.oracle_quantize_coeffs8.restype = i
+        L.oracle_encode_vector8.argtypes = [i, i, p, p, p, i, i, i, p, p, p, p, p, p]
+        L.oracle_encode_vector8.restype = i
+        L.oracle_encode_many8.argtypes = [i, i, i, p, p, p, p, i, i, p, p, p, p, p, p, i, p]
+        L.oracle_encode_many8.restype = i
         for name in ("oracle_f32_to_bf16_rn_many", "oracle_f32_to_fp16_rn_many",
                      "oracle_fp16_to_f64_many", "oracle_bf16_to_f64_many"):
             getattr(L, name).argtypes = [C.c_int64, p, p]
@@ -142,7 +148,7 @@ class HeadProblem:
     """Token-ordered inputs of one (sequence, layer, kv-head) decode problem."""
 
     def __init__(self, basis_k, basis_v, ranks, coeff_k, idx_k, codes_k, scale_k,
-                 coeff_v, idx_v, codes_v, scale_v, q, nres=None):
+                 coeff_v, idx_v, codes_v, scale_v, q, nres=None, coeff_k_f=None, coeff_v_f=None):
         self.bk = _bits16(basis_k)
         self.bv = _bits16(basis_v)
         self.d, self.r_max = self.bk.shape
@@ -162,10 +168,17 @@ class HeadProblem:
         self.gq = self.q.shape[0]
         # per-token residual counts (each <= s), or None: every token keeps s entries
         self.nres = None if nres is None else _arr(nres, np.int32).reshape(self.T)
+        # the coefficients as fp64 values [T][r_max] (the 8-bit blockwise form, dequantised),
+        # used instead of coeff_k / coeff_v when given
+        self.ckf = None if coeff_k_f is None else _arr(coeff_k_f, np.float64).reshape(self.T, self.r_max)
+        self.cvf = None if coeff_v_f is None else _arr(coeff_v_f, np.float64).reshape(self.T, self.r_max)
 
     def _ptrs(self):
         return [_p(self.bk), _p(self.bv), _p(self.rank), _p(self.ck), _p(self.ik), _p(self.qk),
                 _p(self.sk), _p(self.cv), _p(self.iv), _p(self.qv), _p(self.sv), _p(self.q)]
+
+    def _fptrs(self):
+        return [_p(self.ckf) if self.ckf is not None else None, _p(self.cvf) if self.cvf is not None else None]
 
 
 def head_problem(wl, bases, tier_idx, comp, q, layer, head) -> HeadProblem:
@@ -174,8 +187,9 @@ def head_problem(wl, bases, tier_idx, comp, q, layer, head) -> HeadProblem:
     layers_per_group, gqa), ``bases`` the (K, V) bases
     bf16 [G][Hkv][d][r_max], ``tier_idx`` uint8 [T][Hkv] (index into ``wl.tiers``), ``comp``
     the stored arrays (coeff [T][Hkv][2][r_max], idx / codes [T][Hkv][2][s], scales
-    [T][Hkv][2]; K at [..][0], V at [..][1]) and ``q`` bf16 [Hq][d], every query head of the
-    sequence."""
+    [T][Hkv][2]; K at [..][0], V at [..][1]; with 8-bit coefficients ``ccodes`` int8
+    [T][Hkv][2][r_max] and ``cscales`` fp16 bits [T][Hkv][2][r_max / 16] instead of coeff) and
+    ``q`` bf16 [Hq][d], every query head of the sequence."""
     g = layer // wl.layers_per_group
     gq = wl.gqa
     ti = _arr(tier_idx, np.int64)[:, head]
@@ -183,6 +197,13 @@ def head_problem(wl, bases, tier_idx, comp, q, layer, head) -> HeadProblem:
     tr = getattr(wl, "tier_resid", ())
     nres = np.asarray(tr, np.int32)[ti] if tr else None
     sl = lambda key, z: comp[key][:, head, z]   # noqa: E731
+    if "ccodes" in comp:
+        cf = [dequant_coeffs8(sl("ccodes", z), sl("cscales", z)) for z in (0, 1)]
+        zero = np.zeros(cf[0].shape, np.uint16)
+        return HeadProblem(bases[0][g, head], bases[1][g, head], ranks,
+                           zero, sl("idx", 0), sl("codes", 0), comp["scales"][:, head, 0],
+                           zero, sl("idx", 1), sl("codes", 1), comp["scales"][:, head, 1],
+                           _bits16(q)[head * gq:(head + 1) * gq], nres=nres, coeff_k_f=cf[0], coeff_v_f=cf[1])
     return HeadProblem(bases[0][g, head], bases[1][g, head], ranks,
                        sl("coeff", 0), sl("idx", 0), sl("codes", 0), comp["scales"][:, head, 0],
                        sl("coeff", 1), sl("idx", 1), sl("codes", 1), comp["scales"][:, head, 1],
@@ -196,7 +217,8 @@ def decode_head(prob: HeadProblem, tau=None, with_residual=True, want_p=False):
     pw = np.empty((prob.gq, max(prob.T, 1)), np.float64) if want_p else None
     rc = lib().oracle_decode_head(prob.d, prob.r_max, prob.T, prob.gq, prob.s, *prob._ptrs(),
                                   float(tau), 1 if with_residual else 0, _p(out),
-                                  _p(pw) if want_p else None, _p(prob.nres) if prob.nres is not None else None)
+                                  _p(pw) if want_p else None, _p(prob.nres) if prob.nres is not None else None,
+                                  *prob._fptrs())
     if rc != 0:
         raise MemoryError("oracle_decode_head failed")
     if want_p:
@@ -212,7 +234,7 @@ def probe_head(prob: HeadProblem, tau=None, eps=1e-6):
     on = np.empty((prob.gq, prob.d), np.float64)
     rc = lib().oracle_probe_head(prob.d, prob.r_max, prob.T, prob.gq, prob.s, *prob._ptrs(),
                                  float(tau), float(eps), _p(err), _p(of), _p(on),
-                                 _p(prob.nres) if prob.nres is not None else None)
+                                 _p(prob.nres) if prob.nres is not None else None, *prob._fptrs())
     if rc != 0:
         raise MemoryError("oracle_probe_head failed")
     return float(err[0]), of, on
@@ -235,8 +257,15 @@ def decode_many(problems, tau=None, nthreads=None):
     if any(pr.nres is not None for pr in problems):
         full = [pr.nres if pr.nres is not None else np.full(pr.T, pr.s, np.int32) for pr in problems]
         narr = (C.c_void_p * n)(*[_p(a) for a in full])
+    farr, keep = [None, None], []
+    for z, key in enumerate(("ckf", "cvf")):
+        if any(getattr(pr, key) is not None for pr in problems):
+            full = [getattr(pr, key) if getattr(pr, key) is not None
+                    else bf16_to_f64(getattr(pr, key[:2])).reshape(pr.T, pr.r_max) for pr in problems]
+            keep.append(full)                       # alive until the call returns
+            farr[z] = (C.c_void_p * n)(*[_p(a) for a in full])
     rc = lib().oracle_decode_many(n, p0.d, p0.r_max, p0.gq, p0.s, _p(T), *arrs, float(tau), oarr,
-                                  int(nthreads), narr)
+                                  int(nthreads), narr, *farr)
     if rc != 0:
         raise MemoryError("oracle_decode_many failed")
     return outs
@@ -346,3 +375,72 @@ def encode_many_from_coeffs(basis, x, c32, ranks, s, bits, nthreads=None, nres=N
     if rc != 0:
         raise ValueError("oracle_encode_many_from_coeffs: bad arguments")
     return {"coeff": coeff, "idx": idx, "codes": codes, "scale": scale}
+
+
+# ----------------------------------------------------------------------------- 8-bit coefficients
+def quantize_coeffs8(c, r_t):
+    """The 8-bit blockwise form of fp32 coefficients c [r_max] (only [:r_t] read, r_t a multiple
+    of 16): dict of codes int8 [r_max], scales (fp16 bits [r_max / 16]) and the dequantised
+    values cbar fp32 [r_max] (``oracle_quantize_coeffs8``)."""
+    cv = _arr(c, np.float32).reshape(-1)
+    r_max = cv.size
+    q = np.zeros(r_max, np.int8)
+    sc = np.zeros(max(r_max // 16, 1), np.uint16)
+    cbar = np.zeros(r_max, np.float32)
+    if lib().oracle_quantize_coeffs8(int(r_t), r_max, _p(cv), _p(q), _p(sc), _p(cbar)) != 0:
+        raise ValueError("oracle_quantize_coeffs8: bad arguments")
+    return {"codes": q, "scales": sc, "cbar": cbar}
+
+
+def dequant_coeffs8(codes, scales) -> np.ndarray:
+    """fp64 values of 8-bit blockwise coefficients: code_j x scale of block j // 16 (exact)."""
+    q = _arr(codes, np.int8)
+    sc = fp16_to_f64(_bits16(scales).reshape(-1)).reshape(_bits16(scales).shape)
+    return q.astype(np.float64) * np.repeat(sc, 16, axis=-1)[..., :q.shape[-1]]
+
+
+def encode_vector8(basis, x, r_t, s, bits, c_in=None):
+    """Encode one bf16 vector with 8-bit blockwise coefficients: dict of ccodes (int8 [r_max]),
+    cscales (fp16 bits [r_max / 16]), c32, idx, codes, scale (fp16 bits)."""
+    b = _bits16(basis)
+    d, r_max = b.shape
+    xv = _bits16(x).reshape(d)
+    ci = None if c_in is None else _arr(c_in, np.float32).reshape(r_max)
+    cc = np.zeros(r_max, np.int8)
+    cs = np.zeros(r_max // 16, np.uint16)
+    c32 = np.zeros(r_max, np.float32)
+    idx = np.zeros(s, np.uint8)
+    codes = np.zeros(s, np.int8)
+    scale = np.zeros(1, np.uint16)
+    rc = lib().oracle_encode_vector8(d, r_max, _p(b), _p(xv), _p(ci) if ci is not None else None, int(r_t), int(s),
+                                     int(bits), _p(cc), _p(cs), _p(c32), _p(idx), _p(codes), _p(scale))
+    if rc != 0:
+        raise ValueError("oracle_encode_vector8: bad arguments")
+    return {"ccodes": cc, "cscales": cs, "c32": c32, "idx": idx, "codes": codes, "scale": scale[0]}
+
+
+def encode_many8(basis, x, ranks, s, bits, c32=None, nthreads=None, nres=None, want_c32=False):
+    """encode_vector8 over n vectors [n][d] sharing one basis, token-ordered; ``c32`` (optional
+    [n][r_max]) the fp32 projections to use instead of step 1; ``nres`` as encode_many."""
+    b = _bits16(basis)
+    d, r_max = b.shape
+    xv = _bits16(x).reshape(-1, d)
+    n = xv.shape[0]
+    rk = _arr(ranks, np.int32).reshape(n)
+    ci = None if c32 is None else _arr(c32, np.float32).reshape(n, r_max)
+    cc = np.zeros((n, r_max), np.int8)
+    cs = np.zeros((n, r_max // 16), np.uint16)
+    co = np.zeros((n, r_max), np.float32) if want_c32 else None
+    idx = np.zeros((n, s), np.uint8)
+    codes = np.zeros((n, s), np.int8)
+    scale = np.zeros(n, np.uint16)
+    nr = None if nres is None else _arr(nres, np.int32).reshape(n)
+    rc = lib().oracle_encode_many8(n, d, r_max, _p(b), _p(xv), _p(ci) if ci is not None else None, _p(rk), int(s),
+                                   int(bits), _p(cc), _p(cs), _p(co) if want_c32 else None, _p(idx), _p(codes),
+                                   _p(scale), int(nthreads or os.cpu_count() or 1), _p(nr) if nr is not None else None)
+    if rc != 0:
+        raise ValueError("oracle_encode_many8: bad arguments")
+    out = {"ccodes": cc, "cscales": cs, "idx": idx, "codes": codes, "scale": scale}
+    if want_c32:
+        out["c32"] = co
+    return out

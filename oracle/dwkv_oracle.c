@@ -22,6 +22,9 @@
  *   - Encoding: project x on the basis, keep r_t coefficients rounded to bf16, take the
  *     residual against the *stored* coefficients, keep the s largest |residual| channels
  *     (ties -> lower channel), quantise symmetrically with one fp16 scale per token.
+ *   - The 8-bit coefficient variant: blocks of 16 coefficients, one fp16 scale a block
+ *     (max |c| / 127), codes rounded to nearest even; the residual is taken against the
+ *     dequantised coefficients.  Decode then reads the coefficients as exact fp64 values.
  *
  * Precision: everything of decode and probe runs in fp64 from the stored values, which
  * convert exactly (bf16, fp16, integer codes).  Encode runs in fp32 with a fully stated
@@ -90,19 +93,28 @@ uint16_t oracle_f32_to_fp16_rn(float x) {
 /*   coeff : bf16 [r_max], only the first r_t entries are part of the token               */
 /*   idx, codes : s residual channels and their integer codes; scale : fp16 bits          */
 /* ------------------------------------------------------------------------------------ */
-void oracle_reconstruct(int d, int r_max, const uint16_t* basis, int r_t, const uint16_t* coeff,
-                        int s, const uint8_t* idx, const int8_t* codes, uint16_t scale,
-                        int with_residual, double* out) {
+/* coeff_f (nullable): the coefficients as exact fp64 values instead of bf16 bits (the 8-bit */
+/* blockwise form, dequantised: code x scale).                                             */
+static void oracle_reconstruct_any(int d, int r_max, const uint16_t* basis, int r_t, const uint16_t* coeff,
+                                   const double* coeff_f, int s, const uint8_t* idx, const int8_t* codes,
+                                   uint16_t scale, int with_residual, double* out) {
     for (int i = 0; i < d; ++i) {
         double acc = 0.0;
         for (int j = 0; j < r_t; ++j)
-            acc += oracle_bf16_to_f64(basis[(size_t)i * r_max + j]) * oracle_bf16_to_f64(coeff[j]);
+            acc += oracle_bf16_to_f64(basis[(size_t)i * r_max + j]) *
+                   (coeff_f ? coeff_f[j] : oracle_bf16_to_f64(coeff[j]));
         out[i] = acc;
     }
     if (with_residual) {
         double sc = oracle_fp16_to_f64(scale);
         for (int k = 0; k < s; ++k) out[idx[k]] += sc * (double)codes[k];
     }
+}
+
+void oracle_reconstruct(int d, int r_max, const uint16_t* basis, int r_t, const uint16_t* coeff,
+                        int s, const uint8_t* idx, const int8_t* codes, uint16_t scale,
+                        int with_residual, double* out) {
+    oracle_reconstruct_any(d, r_max, basis, r_t, coeff, NULL, s, idx, codes, scale, with_residual, out);
 }
 
 /* ------------------------------------------------------------------------------------ */
@@ -114,6 +126,8 @@ void oracle_reconstruct(int d, int r_max, const uint16_t* basis, int r_t, const 
 /* nres (nullable): token t keeps only its first nres[t] <= s residual entries ([DW] §3     */
 /* Eq. (2): the router's level is the number of retained residual channels).               */
 /* p_out (nullable): softmax weights [gq][T].  Returns 0, or -1 on allocation failure.    */
+/* ckf / cvf (nullable): the coefficients as fp64 values [T][r_max], used instead of ck /   */
+/* cv (the 8-bit blockwise coefficients of [DW] §3, dequantised exactly).                  */
 /* T == 0 gives a zero output (attention over an empty cache).                            */
 /* ------------------------------------------------------------------------------------ */
 int oracle_decode_head(int d, int r_max, int T, int gq, int s,
@@ -121,7 +135,7 @@ int oracle_decode_head(int d, int r_max, int T, int gq, int s,
                        const uint16_t* ck, const uint8_t* ik, const int8_t* qk, const uint16_t* sk,
                        const uint16_t* cv, const uint8_t* iv, const int8_t* qv, const uint16_t* sv,
                        const uint16_t* q, double tau, int with_residual,
-                       double* out, double* p_out, const int32_t* nres) {
+                       double* out, double* p_out, const int32_t* nres, const double* ckf, const double* cvf) {
     for (int h = 0; h < gq * d; ++h) out[h] = 0.0;
     if (T <= 0) return 0;
     double* score = (double*)malloc(sizeof(double) * (size_t)T * gq);
@@ -132,8 +146,8 @@ int oracle_decode_head(int d, int r_max, int T, int gq, int s,
 
     /* scores: tau * q . K^_t */
     for (int t = 0; t < T; ++t) {
-        oracle_reconstruct(d, r_max, bk, rank[t], ck + (size_t)t * r_max, nres ? nres[t] : s,
-                           ik + (size_t)t * s, qk + (size_t)t * s, sk[t], with_residual, x);
+        oracle_reconstruct_any(d, r_max, bk, rank[t], ck + (size_t)t * r_max, ckf ? ckf + (size_t)t * r_max : NULL,
+                               nres ? nres[t] : s, ik + (size_t)t * s, qk + (size_t)t * s, sk[t], with_residual, x);
         for (int h = 0; h < gq; ++h) {
             double dot = 0.0;
             for (int i = 0; i < d; ++i) dot += qd[(size_t)h * d + i] * x[i];
@@ -153,8 +167,8 @@ int oracle_decode_head(int d, int r_max, int T, int gq, int s,
     }
     /* o = sum_t p_t V^_t */
     for (int t = 0; t < T; ++t) {
-        oracle_reconstruct(d, r_max, bv, rank[t], cv + (size_t)t * r_max, nres ? nres[t] : s,
-                           iv + (size_t)t * s, qv + (size_t)t * s, sv[t], with_residual, x);
+        oracle_reconstruct_any(d, r_max, bv, rank[t], cv + (size_t)t * r_max, cvf ? cvf + (size_t)t * r_max : NULL,
+                               nres ? nres[t] : s, iv + (size_t)t * s, qv + (size_t)t * s, sv[t], with_residual, x);
         for (int h = 0; h < gq; ++h) {
             double p = score[(size_t)t * gq + h];
             for (int i = 0; i < d; ++i) out[(size_t)h * d + i] += p * x[i];
@@ -177,15 +191,16 @@ int oracle_probe_head(int d, int r_max, int T, int gq, int s,
                       const uint16_t* ck, const uint8_t* ik, const int8_t* qk, const uint16_t* sk,
                       const uint16_t* cv, const uint8_t* iv, const int8_t* qv, const uint16_t* sv,
                       const uint16_t* q, double tau, double eps,
-                      double* err, double* o_full, double* o_nores, const int32_t* nres) {
+                      double* err, double* o_full, double* o_nores, const int32_t* nres,
+                      const double* ckf, const double* cvf) {
     double* a = (double*)malloc(sizeof(double) * (size_t)gq * d);
     double* b = (double*)malloc(sizeof(double) * (size_t)gq * d);
     if (!a || !b) { free(a); free(b); return -1; }
     int rc = oracle_decode_head(d, r_max, T, gq, s, bk, bv, rank, ck, ik, qk, sk, cv, iv, qv, sv,
-                                q, tau, 1, a, NULL, nres);
+                                q, tau, 1, a, NULL, nres, ckf, cvf);
     if (rc == 0)
         rc = oracle_decode_head(d, r_max, T, gq, s, bk, bv, rank, ck, ik, qk, sk, cv, iv, qv, sv,
-                                q, tau, 0, b, NULL, nres);
+                                q, tau, 0, b, NULL, nres, ckf, cvf);
     if (rc == 0) {
         double num = 0.0, den = 0.0;
         for (int k = 0; k < gq * d; ++k) { num += (a[k] - b[k]) * (a[k] - b[k]); den += a[k] * a[k]; }
@@ -208,13 +223,13 @@ int oracle_decode_many(int n, int d, int r_max, int gq, int s, const int32_t* T,
                        const uint16_t* const* cv, const uint8_t* const* iv, const int8_t* const* qv,
                        const uint16_t* const* sv,
                        const uint16_t* const* q, double tau, double* const* out, int nthreads,
-                       const int32_t* const* nres) {
+                       const int32_t* const* nres, const double* const* ckf, const double* const* cvf) {
     int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(| : bad)
     for (int k = 0; k < n; ++k)
         bad |= (oracle_decode_head(d, r_max, T[k], gq, s, bk[k], bv[k], rank[k], ck[k], ik[k], qk[k],
                                    sk[k], cv[k], iv[k], qv[k], sv[k], q[k], tau, 1, out[k], NULL,
-                                   nres ? nres[k] : NULL) != 0);
+                                   nres ? nres[k] : NULL, ckf ? ckf[k] : NULL, cvf ? cvf[k] : NULL) != 0);
     return bad ? -1 : 0;
 }
 
@@ -306,6 +321,88 @@ int oracle_encode_from_coeffs(int d, int r_max, const uint16_t* basis, const uin
     }
     oracle_quantize_residual(d, s, bits, r, idx, codes, scale);
     return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* The 8-bit blockwise coefficient form ([DW] §3 Method, the shared-bases paragraph: the    */
+/* coefficient vector is kept as 8-bit codes, a block at a time).  Reading: blocks of 16    */
+/* coefficients j < r_t (r_t a multiple of 16), each with one fp16 scale, in the residual   */
+/* codec's symmetric form:                                                                   */
+/*   s_b = fp16_rn(max_{j in b} |c_j| / 127)   (IEEE fp32 division)                        */
+/*   q_j = clamp(rint(c_j / float(s_b)), -127, 127); all zero if s_b == 0                  */
+/*   c^_j = q_j * float(s_b)                    (fp32, exact)                              */
+/* q, sc (nullable), cbar: [r_max], [r_max / 16], [r_max], zero past r_t.                  */
+/* ------------------------------------------------------------------------------------ */
+int oracle_quantize_coeffs8(int r_t, int r_max, const float* c, int8_t* q, uint16_t* sc, float* cbar) {
+    if (r_t < 0 || r_t > r_max || r_t % 16 || r_max % 16) return -1;
+    for (int j = 0; j < r_max; ++j) { if (q) q[j] = 0; cbar[j] = 0.0f; }
+    for (int b = 0; b < r_max / 16; ++b) if (sc) sc[b] = 0;
+    for (int b = 0; b < r_t / 16; ++b) {
+        float amax = 0.0f;
+        for (int j = 16 * b; j < 16 * b + 16; ++j) if (fabsf(c[j]) > amax) amax = fabsf(c[j]);
+        const uint16_t sh = oracle_f32_to_fp16_rn(amax / 127.0f);
+        const float sf = (float)oracle_fp16_to_f64(sh);
+        if (sc) sc[b] = sh;
+        for (int j = 16 * b; j < 16 * b + 16; ++j) {
+            float v = 0.0f;
+            if (sf != 0.0f) {
+                v = rintf(c[j] / sf);
+                if (v > 127.0f) v = 127.0f;
+                if (v < -127.0f) v = -127.0f;
+            }
+            if (q) q[j] = (int8_t)v;
+            cbar[j] = v * sf;
+        }
+    }
+    return 0;
+}
+
+/* Encode one vector with 8-bit blockwise coefficients: step 1 of oracle_encode_vector (or   */
+/* the given fp32 projections c_in [r_max], only [:r_t] read, for an encoder that computed  */
+/* them in another order), the coefficients in the 8-bit form above, the residual against   */
+/* their dequantised values c^, then steps 4-6.  Outputs: ccodes int8 [r_max], cscales fp16  */
+/* [r_max / 16], c32 (nullable) the projections, idx / codes / scale as oracle_encode_vector. */
+int oracle_encode_vector8(int d, int r_max, const uint16_t* basis, const uint16_t* x, const float* c_in, int r_t,
+                          int s, int bits, int8_t* ccodes, uint16_t* cscales, float* c32, uint8_t* idx,
+                          int8_t* codes, uint16_t* scale) {
+    if (d <= 0 || d > 256 || r_max > 256 || r_t < 0 || r_t > r_max || r_t % 16 || s < 0 || s > d ||
+        (bits != 8 && bits != 4))
+        return -1;
+    float xf[256], c[256], cbar[256], r[256];
+    for (int i = 0; i < d; ++i) xf[i] = (float)oracle_bf16_to_f64(x[i]);
+    for (int j = 0; j < r_max; ++j) c[j] = 0.0f;
+    for (int j = 0; j < r_t; ++j) {
+        if (c_in) { c[j] = c_in[j]; continue; }
+        float acc = 0.0f;
+        for (int i = 0; i < d; ++i)
+            acc = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), xf[i], acc);
+        c[j] = acc;
+    }
+    if (c32) for (int j = 0; j < r_max; ++j) c32[j] = c[j];
+    if (oracle_quantize_coeffs8(r_t, r_max, c, ccodes, cscales, cbar)) return -1;
+    for (int i = 0; i < d; ++i) {
+        float a = 0.0f;
+        for (int j = 0; j < r_t; ++j)
+            a = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), cbar[j], a);
+        r[i] = xf[i] - a;
+    }
+    return oracle_quantize_residual(d, s, bits, r, idx, codes, scale);
+}
+
+/* Many vectors sharing one basis (token-ordered): x [n][d], rank [n]; c_in (nullable)       */
+/* [n][r_max]; nres (nullable) per-vector residual counts <= s (the arrays' stride stays s).  */
+int oracle_encode_many8(int n, int d, int r_max, const uint16_t* basis, const uint16_t* x, const float* c_in,
+                        const int32_t* rank, int s, int bits, int8_t* ccodes, uint16_t* cscales, float* c32,
+                        uint8_t* idx, int8_t* codes, uint16_t* scale, int nthreads, const int32_t* nres) {
+    if (r_max % 16) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(static) num_threads(nthreads) reduction(| : bad)
+    for (int k = 0; k < n; ++k)
+        bad |= (oracle_encode_vector8(d, r_max, basis, x + (size_t)k * d, c_in ? c_in + (size_t)k * r_max : NULL,
+                                      rank[k], nres ? nres[k] : s, bits, ccodes + (size_t)k * r_max,
+                                      cscales + (size_t)k * (r_max / 16), c32 ? c32 + (size_t)k * r_max : NULL,
+                                      idx + (size_t)k * s, codes + (size_t)k * s, scale + k) != 0);
+    return bad ? -1 : 0;
 }
 
 int oracle_encode_vector(int d, int r_max, const uint16_t* basis, const uint16_t* x, int r_t,
