@@ -68,9 +68,11 @@ def dense_kv_bytes(layers: int, kv_heads: int, head_dim: int, tokens: int, elem_
     return 2 * layers * kv_heads * head_dim * tokens * elem_bytes
 
 
-def token_bytes(rank: int, s: int, bits: int) -> int:
-    """Stored bytes of one token of one (layer, kv-head), keys + values."""
-    return 2 * (2 * rank + s + s * bits // 8 + 2)
+def token_bytes(rank: int, s: int, bits: int, coeff_bits: int = 16) -> int:
+    """Stored bytes of one token of one (layer, kv-head), keys + values: the coefficients (bf16,
+    or 8-bit codes with an fp16 scale per block of 16), s indices, s codes, one fp16 scale."""
+    cb = rank + rank // 8 if coeff_bits == 8 else 2 * rank
+    return 2 * (cb + s + s * bits // 8 + 2)
 
 
 def tier_counts_of(wl) -> list:
@@ -332,7 +334,7 @@ def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e
                          num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim,
                          r_max=wl.r_max, tiers=wl.tiers, resid_channels=wl.resid_channels,
                          resid_bits=wl.resid_bits, max_batch=B, max_context=max(lengths) + n_steps + extra,
-                         tier_resid=wl.tier_resid or None)
+                         tier_resid=wl.tier_resid or None, coeff_bits=wl.coeff_bits)
     stream = torch.cuda.Stream(device=dev)
     cache = dw.Cache(cfg, bases[0], bases[1], device=dev, ws_seqs=B, stream=stream)
     if args.tuning:
@@ -357,7 +359,8 @@ def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e
                     tiers_dev[g] = synth.make_tiers(wl, sid[b], g, lengths[b] - 1, device=dev)
                     tier_counts += torch.bincount(tiers_dev[g].reshape(-1).long(), minlength=len(wl.tiers)).cpu()
                 comp = synth.make_compressed(wl, sid[b], layer, tiers_dev[g], device=dev)
-                cache.append_compressed(layer, [b], [lengths[b] - 1], tiers_dev[g], comp["coeff"], comp["idx"],
+                coeff = (comp["ccodes"], comp["cscales"]) if "ccodes" in comp else comp["coeff"]
+                cache.append_compressed(layer, [b], [lengths[b] - 1], tiers_dev[g], coeff, comp["idx"],
                                         comp["codes"], comp["scales"], stream=stream)
                 if b == 0 and layer in keep_layers:
                     comp_cpu[layer] = {k: v.cpu() for k, v in comp.items()}
@@ -476,7 +479,7 @@ def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e
     # ---- algorithmic bytes: every stored byte of the attended tokens (per-token bytes of
     #      its tier), plus the two bases, the queries and the outputs of each launch
     held = sum(lengths) - B + B * (warmup + steps)            # tokens per head after the timed steps
-    tok_bytes = torch.tensor([token_bytes(r, n, wl.resid_bits) for r, n in zip(wl.tiers, tier_counts_of(wl))],
+    tok_bytes = torch.tensor([token_bytes(r, n, wl.resid_bits, wl.coeff_bits) for r, n in zip(wl.tiers, tier_counts_of(wl))],
                              dtype=torch.float64)
     bytes_per_tok_head = float((tier_counts.double() * tok_bytes).sum()) / (wl.num_groups * wl.num_kv_heads * held)
     basis_bytes = 2 * wl.num_kv_heads * wl.head_dim * wl.r_max * 2
@@ -606,6 +609,7 @@ def run_dwkv(args, world, rank, local, workload=None, steps=None, warmup=None, e
                    "batch_per_gpu": B, "context": lengths[0] if B == 1 else lengths, "r_max": wl.r_max,
                    "tiers": list(wl.tiers), "tier_probs": list(wl.tier_probs), "resid_channels": wl.resid_channels,
                    **({"tier_resid": list(wl.tier_resid)} if wl.tier_resid else {}),
+                   **({"coeff_bits": wl.coeff_bits} if wl.coeff_bits != 16 else {}),
                    "resid_bits": wl.resid_bits, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2 (~{comp_bytes_layer * wl.num_layers / 1e9:.1f} GB of pages per step); "
                          "no flush",
@@ -691,7 +695,7 @@ def run_encode(args, world, rank, local):
     cfg = dw.config_from(num_layers=wl.num_layers, layers_per_group=lpg, num_q_heads=wl.num_q_heads,
                          num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, r_max=wl.r_max, tiers=wl.tiers,
                          resid_channels=wl.resid_channels, resid_bits=wl.resid_bits, max_batch=B,
-                         max_context=N + 64)
+                         max_context=N + 64, tier_resid=wl.tier_resid or None, coeff_bits=wl.coeff_bits)
     stream = torch.cuda.Stream(device=dev)
     cache = dw.Cache(cfg, bases[0], bases[1], device=dev, ws_seqs=B, stream=stream)
     h = cache.h
@@ -748,8 +752,8 @@ def run_encode(args, world, rank, local):
     #      the residual against the stored coefficients)
     vecs_tier = tier_counts.double() * 2 * lpg       # (seq, head, token) entries x K and V x layers of a group
     n_vec = float(vecs_tier.sum())
-    stored = sum(float(tier_counts[k]) * lpg * token_bytes(r, wl.resid_channels, wl.resid_bits)   # K + V bytes
-                 for k, r in enumerate(wl.tiers))
+    stored = sum(float(tier_counts[k]) * lpg * token_bytes(r, n, wl.resid_bits, wl.coeff_bits)   # K + V bytes
+                 for k, (r, n) in enumerate(zip(wl.tiers, tier_counts_of(wl))))
     dense = n_vec * wl.head_dim * 2
     flops = sum(float(vecs_tier[k]) * 4 * wl.head_dim * r for k, r in enumerate(wl.tiers))
     step_s = ms_per_step * 1e-3
@@ -783,8 +787,9 @@ def run_encode(args, world, rank, local):
     cache.sync(stream)
     assert torch.isfinite(out).all() and torch.isfinite(err).all()
     held = N + 1
-    dec_bytes = (float(tier_counts.double() @ torch.tensor([token_bytes(r, wl.resid_channels, wl.resid_bits)
-                                                             for r in wl.tiers], dtype=torch.float64))
+    dec_bytes = (float(tier_counts.double() @ torch.tensor([token_bytes(r, n, wl.resid_bits, wl.coeff_bits)
+                                                             for r, n in zip(wl.tiers, tier_counts_of(wl))],
+                                                            dtype=torch.float64))
                  * lpg)                                                         # every layer; K + V bytes
     dec_ms = d0.elapsed_time(d1)
     probe_ms = p0.elapsed_time(p1)
@@ -857,6 +862,7 @@ def run_encode(args, world, rank, local):
                    "head_dim": wl.head_dim, "batch_per_gpu": B, "new_tokens": N, "r_max": wl.r_max,
                    "tiers": list(wl.tiers), "tier_probs": list(wl.tier_probs), "resid_channels": wl.resid_channels,
                    **({"tier_resid": list(wl.tier_resid)} if wl.tier_resid else {}),
+                   **({"coeff_bits": wl.coeff_bits} if wl.coeff_bits != 16 else {}),
                    "resid_bits": wl.resid_bits, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (8.6 GB of dense K/V a step); no flush",
                    "timing": "eager launches, CUDA events around each step's appends (resets outside)"},
@@ -933,7 +939,7 @@ def run_reference(args, world, rank, local):
     }
 
 
-EXTRA_WORKLOADS = ("llama8b_ragged_b8", "llama8b_131k_deep", "llama8b_routed_64k", "llama8b_encode_16k")
+EXTRA_WORKLOADS = ("llama8b_64k_c8", "llama8b_ragged_b8", "llama8b_131k_deep", "llama8b_routed_64k", "llama8b_encode_16k")
 
 
 def summary_of(res: dict) -> dict:

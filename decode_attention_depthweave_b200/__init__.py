@@ -27,6 +27,7 @@ __all__ = [
     "dwkv_tier_controller_due", "dwkv_tier_controller_threshold", "dwkv_tier_controller_observe",
     "dwkv_tier_controller_route", "dwkv_arena_bytes_all_tiers", "dwkv_basis_sketch", "dwkv_basis_update",
     "dwkv_get_bases", "dwkv_get_moment", "DWKV_ALL_GROUPS", "Cache", "EXPORTED_SYMBOLS",
+    "pack_coeff8", "unpack_coeff8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -63,6 +64,7 @@ class dwkv_config(C.Structure):
         ("num_tiers", C.c_int32), ("tiers", C.c_int32 * 8), ("resid_channels", C.c_int32),
         ("resid_bits", C.c_int32), ("max_batch", C.c_int32), ("max_context", C.c_int32),
         ("softmax_scale", C.c_float), ("resid_routed", C.c_int32), ("tier_resid", C.c_int32 * 8),
+        ("coeff_bits", C.c_int32),
     ]
 
 
@@ -167,10 +169,12 @@ def _stream(stream):
 
 def config_from(num_layers, layers_per_group, num_q_heads, num_kv_heads, head_dim, r_max, tiers,
                 resid_channels, resid_bits, max_batch, max_context, softmax_scale=0.0,
-                tier_resid=None) -> dwkv_config:
+                tier_resid=None, coeff_bits=16) -> dwkv_config:
     """tier_resid: per-tier residual channel counts (residual-count routing; every tier then has
-    the same rank and resid_channels is 8), or None for one count, resid_channels, everywhere."""
+    the same rank and resid_channels is 8), or None for one count, resid_channels, everywhere.
+    coeff_bits: 16 (bf16 coefficients) or 8 (int8 codes with an fp16 scale per block of 16)."""
     c = dwkv_config()
+    c.coeff_bits = int(coeff_bits)
     if tier_resid is not None:
         c.resid_routed = 1
         for k, n in enumerate(tier_resid):
@@ -385,6 +389,18 @@ def dwkv_tier_controller_route(c, group, salience, base_tier, high_tier):
 
 
 # ------------------------------------------------------------------------------ plumbing
+def pack_coeff8(codes: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
+    """Coefficient records of the 8-bit form, uint8 [..][r_max + r_max / 8]: the int8 codes
+    [..][r_max], then the fp16 block scales [..][r_max / 16] (byte marshalling only)."""
+    return torch.cat([codes.contiguous().view(torch.uint8), scales.contiguous().view(torch.uint8)], dim=-1).contiguous()
+
+
+def unpack_coeff8(records: torch.Tensor, r_max: int):
+    """(codes int8 [..][r_max], scales fp16 [..][r_max / 16]) of packed coefficient records."""
+    return (records[..., :r_max].contiguous().view(torch.int8),
+            records[..., r_max:].contiguous().view(torch.float16))
+
+
 class Cache:
     """Owns the torch allocations around one handle (arena and workspace) and exposes the
     C ABI calls with tensors.  Allocation is torch's; computation is libdwkv's."""
@@ -418,6 +434,10 @@ class Cache:
         dwkv_append(self.h, layer, seq_ids, n_new, k_new, v_new, tier_idx, coeff_dbg, stream)
 
     def append_compressed(self, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream=None):
+        """coeff: bf16 [n][Hkv][2][r_max], or with 8-bit coefficients the pair (codes int8
+        [n][Hkv][2][r_max], block scales fp16 [n][Hkv][2][r_max / 16]) or its packed records."""
+        if isinstance(coeff, (tuple, list)):
+            coeff = pack_coeff8(*coeff)
         dwkv_append_compressed(self.h, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream)
 
     def decode(self, layer, seq_ids, q, out=None, stream=None):
@@ -443,9 +463,11 @@ class Cache:
         c = self.cfg
         H, R, s = c.num_kv_heads, c.r_max, c.resid_channels
         dev = self.device
+        c8 = c.coeff_bits == 8
         out = {
             "tier_idx": torch.empty(n, H, dtype=torch.uint8, device=dev),
-            "coeff": torch.empty(n, H, 2, R, dtype=torch.bfloat16, device=dev),
+            "coeff": (torch.empty(n, H, 2, R + R // 8, dtype=torch.uint8, device=dev) if c8
+                      else torch.empty(n, H, 2, R, dtype=torch.bfloat16, device=dev)),
             "idx": torch.empty(n, H, 2, s, dtype=torch.uint8, device=dev),
             "codes": torch.empty(n, H, 2, s, dtype=torch.int8, device=dev),
             "scales": torch.empty(n, H, 2, dtype=torch.float16, device=dev),
@@ -453,6 +475,8 @@ class Cache:
         if n:
             dwkv_export(self.h, layer, seq, t0, n, out["tier_idx"], out["coeff"], out["idx"] if s else None,
                         out["codes"] if s else None, out["scales"], stream)
+        if c8:
+            out["ccodes"], out["cscales"] = unpack_coeff8(out.pop("coeff"), R)
         return out
 
     def reset(self, seq, stream=None):

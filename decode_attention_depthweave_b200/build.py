@@ -16,7 +16,8 @@ INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(HERE, "_lib")
 LIB = os.path.join(OUT_DIR, "libdwkv.so")
 SOURCES = ["dwkv_api.cu", "dwkv_basis.cu", "dwkv_cache.cu", "dwkv_control.cu", "dwkv_decode_b4.cu", "dwkv_decode_b4p.cu",
-           "dwkv_decode_b8.cu", "dwkv_decode_b8p.cu"]
+           "dwkv_decode_b8.cu", "dwkv_decode_b8p.cu", "dwkv_decode_b4c8.cu", "dwkv_decode_b4pc8.cu",
+           "dwkv_decode_b8c8.cu", "dwkv_decode_b8pc8.cu"]
 HEADERS = ["dwkv_common.cuh", "dwkv_decode.cuh", "dwkv_encode.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -24,10 +24,10 @@ template <int BITS>
 __global__ void append_small_kernel(const Geom, const State, const AppendCall, const uint8_t*, int,
                                     const __nv_bfloat16*, const __nv_bfloat16*, float*);
 template <int BITS>
-__global__ void import_kernel(const Geom, const State, const AppendCall, const __nv_bfloat16*, const uint8_t*,
+__global__ void import_kernel(const Geom, const State, const AppendCall, const uint8_t*, const uint8_t*,
                               const int8_t*, const __half*);
 template <int BITS>
-__global__ void export_kernel(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*, uint8_t*,
+__global__ void export_kernel(const Geom, const State, int, int, int, int, uint8_t*, uint8_t*, uint8_t*,
                               int8_t*, __half*);
 __global__ void reset_kernel(const Geom, const State, int);
 template <int BITS>
@@ -42,7 +42,7 @@ template <int BITS>
 __global__ void reproject_kernel(const Geom, const State, int, const SeqList, const __nv_bfloat16*,
                                  const __nv_bfloat16*);
 size_t basis_smem_bytes(int r);
-template <int BITS, bool PROBE, int RMAX, int S>
+template <int BITS, bool PROBE, int RMAX, int S, bool C8>
 __global__ void decode_kernel(const Geom, const State, const DecodeCall);
 }  // namespace dwkv
 
@@ -104,9 +104,16 @@ dwkv_status check_cfg(const dwkv_config* c) {
         return fail(DWKV_ERR_INVALID_ARG, "num_tiers %d out of [1, %d]", c->num_tiers, DWKV_MAX_TIERS);
     if (c->resid_routed != 0 && c->resid_routed != 1)
         return fail(DWKV_ERR_INVALID_ARG, "resid_routed must be 0 or 1 (got %d)", c->resid_routed);
+    if (c->coeff_bits != 0 && c->coeff_bits != 16 && c->coeff_bits != 8)
+        return fail(DWKV_ERR_INVALID_ARG, "coeff_bits must be 16 (or 0) or 8 (got %d)", c->coeff_bits);
+    if (c->coeff_bits == 8 && c->r_max % 16)
+        return fail(DWKV_ERR_INVALID_ARG, "with coeff_bits 8, r_max (%d) must be a multiple of 16", c->r_max);
     for (int k = 0; k < c->num_tiers; ++k) {
         if (c->tiers[k] <= 0 || c->tiers[k] % 8 || c->tiers[k] > c->r_max)
             return fail(DWKV_ERR_INVALID_ARG, "tier %d rank %d must be a multiple of 8 in [8, r_max]", k, c->tiers[k]);
+        if (c->coeff_bits == 8 && c->tiers[k] % 16)
+            return fail(DWKV_ERR_INVALID_ARG, "with coeff_bits 8, tier %d rank %d must be a multiple of 16 (whole blocks)",
+                        k, c->tiers[k]);
         if (!c->resid_routed && k && c->tiers[k] <= c->tiers[k - 1])
             return fail(DWKV_ERR_INVALID_ARG, "tiers must be strictly ascending");
         if (c->resid_routed) {
@@ -166,6 +173,7 @@ Geom make_geom(const dwkv_config* c) {
     G.ntiers = c->num_tiers;
     G.s = c->resid_channels;
     G.routed = c->resid_routed ? 1 : 0;
+    G.c8 = c->coeff_bits == 8 ? 1 : 0;
     for (int k = 0; k < kMaxTiers; ++k) G.ts[k] = (k < c->num_tiers && G.routed) ? c->tier_resid[k] : G.s;
     G.bits = c->resid_bits;
     G.max_batch = c->max_batch;
@@ -176,7 +184,7 @@ Geom make_geom(const dwkv_config* c) {
     for (int k = 0; k < kMaxTiers; ++k) {
         if (k < c->num_tiers) {
             G.tiers[k] = c->tiers[k];
-            G.blk_bytes[k] = blk_bytes_of(c->tiers[k], G.ts[k], G.bits);
+            G.blk_bytes[k] = blk_bytes_of(c->tiers[k], G.ts[k], G.bits, G.c8);
             G.chunk_bytes[k] = 2 * G.blk_bytes[k];
             G.page_units[k] = (G.LPG * G.chunk_bytes[k] + kPosBlockBytes) / kUnit;
             stage = std::max(stage, G.chunk_bytes[k]);
@@ -400,7 +408,8 @@ size_t dwkv_token_bytes(const dwkv_config* cfg, int32_t tier) {
     if (check_cfg(cfg) != DWKV_OK || tier < 0 || tier >= cfg->num_tiers) return 0;
     const int r = cfg->tiers[tier], s = cfg->resid_routed ? cfg->tier_resid[tier] : cfg->resid_channels;
     const int b = cfg->resid_bits;
-    return (size_t)2 * (2 * r + s + s * b / 8 + 2);
+    const int cb = cfg->coeff_bits == 8 ? r + r / 8 : 2 * r;     // int8 codes + an fp16 scale per 16
+    return (size_t)2 * (cb + s + s * b / 8 + 2);
 }
 
 size_t dwkv_page_bytes(const dwkv_config* cfg, int32_t tier) {
@@ -488,12 +497,13 @@ dwkv_status dwkv_create(const dwkv_config* cfg, void* arena, size_t arena_bytes,
     if (e == cudaSuccess) {
         const int maxs = (int)h->smem_optin;
         const void* kernels[] = {
-#define DWKV_K(B, P) (const void*)decode_kernel<B, P, 64, 0>, (const void*)decode_kernel<B, P, 64, 8>,       \
-                     (const void*)decode_kernel<B, P, 64, 16>, (const void*)decode_kernel<B, P, 64, 32>,     \
-                     (const void*)decode_kernel<B, P, 128, 0>, (const void*)decode_kernel<B, P, 128, 8>,     \
-                     (const void*)decode_kernel<B, P, 128, 16>, (const void*)decode_kernel<B, P, 128, 32>,   \
-                     (const void*)decode_kernel<B, P, 64, -1>, (const void*)decode_kernel<B, P, 128, -1>
-            DWKV_K(4, false), DWKV_K(4, true), DWKV_K(8, false), DWKV_K(8, true),
+#define DWKV_K(B, P, C) (const void*)decode_kernel<B, P, 64, 0, C>, (const void*)decode_kernel<B, P, 64, 8, C>,       \
+                     (const void*)decode_kernel<B, P, 64, 16, C>, (const void*)decode_kernel<B, P, 64, 32, C>,     \
+                     (const void*)decode_kernel<B, P, 128, 0, C>, (const void*)decode_kernel<B, P, 128, 8, C>,     \
+                     (const void*)decode_kernel<B, P, 128, 16, C>, (const void*)decode_kernel<B, P, 128, 32, C>,   \
+                     (const void*)decode_kernel<B, P, 64, -1, C>, (const void*)decode_kernel<B, P, 128, -1, C>
+            DWKV_K(4, false, false), DWKV_K(4, true, false), DWKV_K(8, false, false), DWKV_K(8, true, false),
+            DWKV_K(4, false, true), DWKV_K(4, true, true), DWKV_K(8, false, true), DWKV_K(8, true, true),
 #undef DWKV_K
         };
         for (const void* k : kernels)
@@ -641,6 +651,8 @@ dwkv_status dwkv_basis_update(dwkv_handle h, int32_t group, int32_t n_rows, cons
     if (!(beta >= 0.f && beta <= 1.f)) return fail(DWKV_ERR_INVALID_ARG, "beta must be in [0, 1]");
     if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
     const Geom& G = h->geom;
+    if (n_seqs > 0 && G.c8)
+        return fail(DWKV_ERR_UNSUPPORTED, "no re-projection kernel for 8-bit coefficients (update with n_seqs = 0)");
     for (int i = 0; i < n_seqs; ++i) {
         const int sq = seq_ids[i];
         for (int g = g0; g < g0 + ng; ++g) {
@@ -810,6 +822,8 @@ dwkv_status dwkv_append_compressed(dwkv_handle h, int32_t layer, int32_t n_seqs,
     const Geom& G = h->geom;
     if (!coeff || !scales || (G.s > 0 && (!idx || !codes)))
         return fail(DWKV_ERR_INVALID_ARG, "coeff, idx, codes and scales must be non-NULL");
+    if (((uintptr_t)coeff & 1u) || ((uintptr_t)scales & 1u))
+        return fail(DWKV_ERR_INVALID_ARG, "coeff and scales must be 2-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     bool any = false;
     for (int i = 0; i < C.n; ++i) any |= C.na[i] > 0;
@@ -820,10 +834,10 @@ dwkv_status dwkv_append_compressed(dwkv_handle h, int32_t layer, int32_t n_seqs,
     }
     const dim3 grid(grid_rows(h, C.total), G.Hkv);
     if (G.bits == 8)
-        import_kernel<8><<<grid, 256, 0, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(coeff), idx, codes,
+        import_kernel<8><<<grid, 256, 0, s>>>(G, h->st, C, static_cast<const uint8_t*>(coeff), idx, codes,
                                               static_cast<const __half*>(scales));
     else
-        import_kernel<4><<<grid, 256, 0, s>>>(G, h->st, C, static_cast<const __nv_bfloat16*>(coeff), idx, codes,
+        import_kernel<4><<<grid, 256, 0, s>>>(G, h->st, C, static_cast<const uint8_t*>(coeff), idx, codes,
                                               static_cast<const __half*>(scales));
     DWKV_CUDA(cudaGetLastError(), "import_kernel launch");
     note_plain_launch(h);
@@ -979,7 +993,9 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     const dim3 grid(total, G.Hkv);
     const bool big = G.r_max > 64;
     cudaError_t lerr = cudaSuccess;
-#define DWKV_LAUNCH(B, P, R, SS) lerr = launch_decode(decode_kernel<B, P, R, SS>, grid, smem, s, h->dec_overlap != 0, G, h->st, C)
+#define DWKV_LAUNCH(B, P, R, SS)                                                                                        \
+    lerr = G.c8 ? launch_decode(decode_kernel<B, P, R, SS, true>, grid, smem, s, h->dec_overlap != 0, G, h->st, C)      \
+                : launch_decode(decode_kernel<B, P, R, SS, false>, grid, smem, s, h->dec_overlap != 0, G, h->st, C)
 #define DWKV_LAUNCH_S(B, P, R)                                  \
     do {                                                        \
         switch (G.routed ? -1 : G.s) {                          \
@@ -1057,6 +1073,7 @@ dwkv_status dwkv_retier(dwkv_handle h, int32_t group, int32_t n_seqs, const int3
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
     const Geom& G = h->geom;
+    if (G.c8) return fail(DWKV_ERR_UNSUPPORTED, "no re-tier kernel for 8-bit coefficients");
     if (group < 0 || group >= G.G) return fail(DWKV_ERR_INVALID_ARG, "group %d out of [0, %d)", group, G.G);
     if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
     if (n_seqs && !n_tok) return fail(DWKV_ERR_INVALID_ARG, "n_tok is NULL");
@@ -1114,14 +1131,16 @@ dwkv_status dwkv_export(dwkv_handle h, int32_t layer, int32_t seq, int32_t t0, i
     if (t0 < 0 || n < 0 || (long long)t0 + n > len)
         return fail(DWKV_ERR_INVALID_ARG, "positions [%d, %lld) outside the %d held", t0, (long long)t0 + n, len);
     if (n == 0) return DWKV_OK;
+    if (((uintptr_t)coeff & 1u) || ((uintptr_t)scales & 1u))
+        return fail(DWKV_ERR_INVALID_ARG, "coeff and scales must be 2-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int grid = (int)std::min<long long>(((long long)n * G.Hkv + 7) / 8, 4096);
     if (G.bits == 8)
         export_kernel<8><<<grid, 256, 0, s>>>(G, h->st, layer, seq, t0, n, tier_idx,
-                                              static_cast<__nv_bfloat16*>(coeff), idx, codes, static_cast<__half*>(scales));
+                                              static_cast<uint8_t*>(coeff), idx, codes, static_cast<__half*>(scales));
     else
         export_kernel<4><<<grid, 256, 0, s>>>(G, h->st, layer, seq, t0, n, tier_idx,
-                                              static_cast<__nv_bfloat16*>(coeff), idx, codes, static_cast<__half*>(scales));
+                                              static_cast<uint8_t*>(coeff), idx, codes, static_cast<__half*>(scales));
     DWKV_CUDA(cudaGetLastError(), "export_kernel launch");
     note_plain_launch(h);
     return DWKV_OK;

@@ -349,6 +349,14 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
                             const int sl = 16 * mt + g + 8 * hf;
                             const float v0 = dd[u][2 * hf], v1 = dd[u][2 * hf + 1];
                             const bool on = j0 < sR[sl];           // ranks are multiples of 8: j0 + 1 too
+                            if (G.c8) {                                // the projections; blocks below
+                                cs[j0 * kEncXP + sl] = on ? v0 : 0.f;
+                                cs[(j0 + 1) * kEncXP + sl] = on ? v1 : 0.f;
+                                if (on && coeff_dbg)
+                                    *reinterpret_cast<float2*>(coeff_dbg + (((size_t)srow[sl] * G.Hkv + h) * 2 + z) * RM +
+                                                               j0) = make_float2(v0, v1);
+                                continue;
+                            }
                             const __nv_bfloat16 c0 = __float2bfloat16_rn(v0), c1 = __float2bfloat16_rn(v1);
                             cs[j0 * kEncXP + sl] = on ? __bfloat162float(c0) : 0.f;
                             cs[(j0 + 1) * kEncXP + sl] = on ? __bfloat162float(c1) : 0.f;
@@ -368,6 +376,30 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
             }
         }
         __syncthreads();
+
+        // ---- 2 (8-bit coefficients): each half warp quantises one (slot, block of 16) at a
+        //      time, the dequantised values replacing the projections in cs
+        if (G.c8) {
+            const int nbm = L.RP / 16, units = nvalid * nbm, e = lane & 15;
+            for (int u0 = 2 * warp; u0 < units; u0 += 2 * (int)(blockDim.x >> 5)) {
+                const int u = u0 + (lane >> 4);
+                const int sl = u < units ? u / nbm : 0, b = u < units ? u % nbm : 0;
+                const bool on = u < units && 16 * b < sR[sl];   // uniform over the half warp
+                const int j = 16 * b + e;
+                uint16_t sh;
+                int qc;
+                float cb;
+                quantize_coeff8(on ? cs[j * kEncXP + sl] : 0.f, sh, qc, cb);
+                if (on) {
+                    cs[j * kEncXP + sl] = cb;
+                    const int prow = sprow[sl] & 0xff, Rs = sR[sl];
+                    sblk[sl][z ? vc8_code_off(j, prow) : kc8_code_off(j, prow)] = (uint8_t)(int8_t)qc;
+                    if (e == 0)
+                        *reinterpret_cast<uint16_t*>(sblk[sl] + (z ? vc8_scale_off(Rs, b, prow) : kc8_scale_off(Rs, b, prow))) = sh;
+                }
+            }
+            __syncthreads();
+        }
 
         // ---- 3: residual against the stored coefficients, then steps 4-6 per slot; items of
         //      4 slots (16 a tile, taken w, w + 8, ...: a costly item with a cheaper one)
@@ -406,7 +438,7 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
                 const int sl = s0 + t;
                 if (sl >= nvalid) break;
                 const float r4[4] = {a[t][0], a[t][1], a[t][2], a[t][3]};
-                quantize_store<BITS>(r4, sblk[sl], sR[sl], sprow[sl] & 0xff, G.ts[sprow[sl] >> 8], rstage, chstage);
+                quantize_store<BITS>(r4, sblk[sl], sR[sl], sprow[sl] & 0xff, G.ts[sprow[sl] >> 8], rstage, chstage, G.c8);
             }
         }
     }
@@ -456,7 +488,7 @@ __global__ void __launch_bounds__(256) quantize_test_kernel(int n, int s, const 
     for (int m = 0; m < 4; ++m) rr[m] = r[(size_t)v * kD + lane + 32 * m];
     uint8_t* blk = work + (size_t)v * stride;
     float* rstage = reinterpret_cast<float*>(stage + warp * kEncStage);
-    quantize_store<BITS>(rr, blk, 0, 0, s, rstage, reinterpret_cast<uint8_t*>(rstage + kD));
+    quantize_store<BITS>(rr, blk, 0, 0, s, rstage, reinterpret_cast<uint8_t*>(rstage + kD), 0);
     __syncwarp();
     for (int b = lane; b < s; b += 32) {
         idx[(size_t)v * s + b] = blk[off_idx_of(0) + b];
@@ -508,9 +540,15 @@ __global__ void __launch_bounds__(256) append_small_kernel(const Geom G, const S
 // ------------------------------------------------------------------------------------
 // Import of already compressed tokens: one warp per token row (keys and values).
 // ------------------------------------------------------------------------------------
+// Bytes of one coefficient record of the import / export arrays: bf16 [r_max], or int8 codes
+// [r_max] then fp16 block scales [r_max / 16].
+__host__ __device__ inline size_t coeff_record_bytes(const Geom& G) {
+    return G.c8 ? (size_t)G.r_max + G.r_max / 8 : (size_t)2 * G.r_max;
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(256) import_kernel(const Geom G, const State S, const AppendCall C,
-                                                     const __nv_bfloat16* __restrict__ coeff,
+                                                     const uint8_t* __restrict__ coeff,
                                                      const uint8_t* __restrict__ idx,
                                                      const int8_t* __restrict__ codes,
                                                      const __half* __restrict__ scales) {
@@ -527,29 +565,40 @@ __global__ void __launch_bounds__(256) import_kernel(const Geom G, const State S
             continue;
         }
         const int R = dst.R, st = G.ts[dst.k];        // the row's tier keeps st <= s entries
+        const int c8 = G.c8;
+        const size_t crb = coeff_record_bytes(G);
         for (int z = 0; z < 2; ++z) {
             const size_t src = ((size_t)row * G.Hkv + h) * 2 + z;
             uint8_t* blk = dst.blk + (z ? G.blk_bytes[dst.k] : 0u);
-            for (int j = lane; j < R; j += 32)
-                *reinterpret_cast<__nv_bfloat16*>(blk + (j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2) =
-                    coeff[src * RM + j];
+            const uint8_t* rec = coeff + src * crb;
+            if (c8) {
+                for (int j = lane; j < R; j += 32)
+                    blk[z ? vc8_code_off(j, dst.row) : kc8_code_off(j, dst.row)] = rec[j];
+                for (int b = lane; b < R / 16; b += 32)
+                    *reinterpret_cast<uint16_t*>(blk + (z ? vc8_scale_off(R, b, dst.row) : kc8_scale_off(R, b, dst.row))) =
+                        *reinterpret_cast<const uint16_t*>(rec + RM + 2 * b);
+            } else {
+                for (int j = lane; j < R; j += 32)
+                    *reinterpret_cast<uint16_t*>(blk + (j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2) =
+                        reinterpret_cast<const uint16_t*>(rec)[j];
+            }
             for (int e = lane; e < st; e += 32) {
                 const uint8_t ch = idx[src * s + e];
                 if (ch >= kD) set_dev_error(S, 3u /*DWKV_DEV_BAD_CHANNEL*/, (uint32_t)seq, (uint32_t)pos);
-                blk[off_idx_of(R) + dst.row * st + e] = ch;
-                if (BITS == 8) blk[off_codes_of(R, st) + dst.row * st + e] = (uint8_t)codes[src * s + e];
+                blk[off_idx_of(R, c8) + dst.row * st + e] = ch;
+                if (BITS == 8) blk[off_codes_of(R, st, c8) + dst.row * st + e] = (uint8_t)codes[src * s + e];
             }
             if (BITS == 4) {
                 for (int b = lane; b < st / 2; b += 32) {
                     const int c0 = codes[src * s + 2 * b], c1 = codes[src * s + 2 * b + 1];
                     if (c0 < -8 || c0 > 7 || c1 < -8 || c1 > 7)
                         set_dev_error(S, 4u /*DWKV_DEV_BAD_CODE*/, (uint32_t)seq, (uint32_t)pos);
-                    blk[off_codes_of(R, st) + dst.row * (st / 2) + b] =
+                    blk[off_codes_of(R, st, c8) + dst.row * (st / 2) + b] =
                         (uint8_t)(((uint32_t)c0 & 0xfu) | (((uint32_t)c1 & 0xfu) << 4));
                 }
             }
             if (lane == 0 && st)
-                *reinterpret_cast<__half*>(blk + off_scales_of(R, st, BITS) + dst.row * 2) = scales[src];
+                *reinterpret_cast<__half*>(blk + off_scales_of(R, st, BITS, c8) + dst.row * 2) = scales[src];
         }
     }
 }
@@ -559,7 +608,7 @@ __global__ void __launch_bounds__(256) import_kernel(const Geom G, const State S
 // ------------------------------------------------------------------------------------
 template <int BITS>
 __global__ void __launch_bounds__(256) export_kernel(const Geom G, const State S, int layer, int seq, int t0,
-                                                     int n, uint8_t* tier_out, __nv_bfloat16* coeff_out,
+                                                     int n, uint8_t* tier_out, uint8_t* coeff_out,
                                                      uint8_t* idx_out, int8_t* codes_out, __half* scales_out) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int g = layer / G.LPG, lig = layer % G.LPG, s = G.s, RM = G.r_max;
@@ -572,20 +621,33 @@ __global__ void __launch_bounds__(256) export_kernel(const Geom G, const State S
             const size_t o = (size_t)w * 2 + z;
             const uint8_t* blk = ok ? dst.blk + (z ? G.blk_bytes[dst.k] : 0u) : nullptr;
             const int R = ok ? dst.R : 0, st = ok ? G.ts[dst.k] : 0;   // entries past st read as 0
-            if (coeff_out)
-                for (int j = lane; j < RM; j += 32)
-                    coeff_out[o * RM + j] = j < R ? *reinterpret_cast<const __nv_bfloat16*>(
-                                                        blk + (j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2)
-                                                  : __float2bfloat16_rn(0.f);
+            const int c8 = G.c8;
+            if (coeff_out) {
+                uint8_t* rec = coeff_out + o * coeff_record_bytes(G);
+                if (c8) {
+                    for (int j = lane; j < RM; j += 32)
+                        rec[j] = j < R ? blk[z ? vc8_code_off(j, dst.row) : kc8_code_off(j, dst.row)] : 0;
+                    for (int b = lane; b < RM / 16; b += 32)
+                        *reinterpret_cast<uint16_t*>(rec + RM + 2 * b) =
+                            16 * b < R ? *reinterpret_cast<const uint16_t*>(
+                                             blk + (z ? vc8_scale_off(R, b, dst.row) : kc8_scale_off(R, b, dst.row)))
+                                       : (uint16_t)0;
+                } else {
+                    for (int j = lane; j < RM; j += 32)
+                        reinterpret_cast<uint16_t*>(rec)[j] =
+                            j < R ? *reinterpret_cast<const uint16_t*>(blk + (j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2)
+                                  : (uint16_t)0;
+                }
+            }
             for (int e = lane; e < s; e += 32) {
                 const bool on = e < st;
-                if (idx_out) idx_out[o * s + e] = on ? blk[off_idx_of(R) + dst.row * st + e] : 0;
+                if (idx_out) idx_out[o * s + e] = on ? blk[off_idx_of(R, c8) + dst.row * st + e] : 0;
                 if (codes_out) {
                     int c = 0;
                     if (on) {
-                        if (BITS == 8) c = (int8_t)blk[off_codes_of(R, st) + dst.row * st + e];
+                        if (BITS == 8) c = (int8_t)blk[off_codes_of(R, st, c8) + dst.row * st + e];
                         else {
-                            const uint32_t byte = blk[off_codes_of(R, st) + dst.row * (st / 2) + e / 2];
+                            const uint32_t byte = blk[off_codes_of(R, st, c8) + dst.row * (st / 2) + e / 2];
                             const uint32_t nib = (e & 1) ? (byte >> 4) : (byte & 0xfu);
                             c = (int)(nib ^ 8u) - 8;
                         }
@@ -594,7 +656,7 @@ __global__ void __launch_bounds__(256) export_kernel(const Geom G, const State S
                 }
             }
             if (scales_out && lane == 0)
-                scales_out[o] = st ? *reinterpret_cast<const __half*>(blk + off_scales_of(R, st, BITS) + dst.row * 2)
+                scales_out[o] = st ? *reinterpret_cast<const __half*>(blk + off_scales_of(R, st, BITS, c8) + dst.row * 2)
                                    : __float2half_rn(0.f);
         }
     }
@@ -881,12 +943,12 @@ template __global__ void append_small_kernel<8>(const Geom, const State, const A
                                                 const __nv_bfloat16*, const __nv_bfloat16*, float*);
 template __global__ void append_small_kernel<4>(const Geom, const State, const AppendCall, const uint8_t*, int,
                                                 const __nv_bfloat16*, const __nv_bfloat16*, float*);
-template __global__ void import_kernel<8>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
+template __global__ void import_kernel<8>(const Geom, const State, const AppendCall, const uint8_t*,
                                           const uint8_t*, const int8_t*, const __half*);
-template __global__ void import_kernel<4>(const Geom, const State, const AppendCall, const __nv_bfloat16*,
+template __global__ void import_kernel<4>(const Geom, const State, const AppendCall, const uint8_t*,
                                           const uint8_t*, const int8_t*, const __half*);
-template __global__ void export_kernel<8>(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*,
+template __global__ void export_kernel<8>(const Geom, const State, int, int, int, int, uint8_t*, uint8_t*,
                                           uint8_t*, int8_t*, __half*);
-template __global__ void export_kernel<4>(const Geom, const State, int, int, int, int, uint8_t*, __nv_bfloat16*,
+template __global__ void export_kernel<4>(const Geom, const State, int, int, int, int, uint8_t*, uint8_t*,
                                           uint8_t*, int8_t*, __half*);
 }  // namespace dwkv

@@ -48,6 +48,7 @@ struct Geom {
     int tiers[kMaxTiers];
     int ts[kMaxTiers];               // residual channels a token of each tier keeps (<= s; s when not routed)
     int routed;                      // 1: per-tier residual counts (every tier at one basis rank)
+    int c8;                          // 1: coefficients as 8-bit codes with an fp16 scale per block of 16
     float tau;                       // softmax scale
     uint32_t blk_bytes[kMaxTiers];   // one (layer, K or V) block of a page
     uint32_t chunk_bytes[kMaxTiers]; // one layer of a page: K block + V block
@@ -129,15 +130,43 @@ struct DecodeCall {
 };
 
 // ------------------------------------------------------------------------------ layout
+// One (layer, K or V) block of a page of tier rank R, 64 token slots:
+//   coefficients: bf16 [R/8][64][8] (128 R bytes), or with c8 the 8-bit form (72 R bytes, below)
+//   idx u8 [64][s], codes [64][s] (int8, or int4 pairs) padded to 128 bytes, scales fp16 [64].
 // The code part rounded up to 128 bytes (only 2 int4 codes a token, 64 bytes, needs it).
 __host__ __device__ inline uint32_t code_part_bytes(int s, int bits) { return (8u * s * bits + 127u) & ~127u; }
-__host__ __device__ inline uint32_t blk_bytes_of(int R, int s, int bits) {
-    return 128u * R + 64u * s + code_part_bytes(s, bits) + 128u;
+__host__ __device__ inline uint32_t coeff_part_bytes(int R, int c8) { return c8 ? 72u * R : 128u * R; }
+__host__ __device__ inline uint32_t blk_bytes_of(int R, int s, int bits, int c8 = 0) {
+    return coeff_part_bytes(R, c8) + 64u * s + code_part_bytes(s, bits) + 128u;
 }
-__host__ __device__ inline uint32_t off_idx_of(int R) { return 128u * R; }
-__host__ __device__ inline uint32_t off_codes_of(int R, int s) { return 128u * R + 64u * s; }
-__host__ __device__ inline uint32_t off_scales_of(int R, int s, int bits) {
-    return 128u * R + 64u * s + code_part_bytes(s, bits);
+__host__ __device__ inline uint32_t off_idx_of(int R, int c8 = 0) { return coeff_part_bytes(R, c8); }
+__host__ __device__ inline uint32_t off_codes_of(int R, int s, int c8 = 0) { return coeff_part_bytes(R, c8) + 64u * s; }
+__host__ __device__ inline uint32_t off_scales_of(int R, int s, int bits, int c8 = 0) {
+    return coeff_part_bytes(R, c8) + 64u * s + code_part_bytes(s, bits);
+}
+// The 8-bit coefficient form (R a multiple of 16; blocks b of 16 coefficients): codes int8
+// [R/16][1024 bytes], then fp16 scales [R/16][128 bytes].
+//  keys:   token t's 16 codes of block b are the 16 bytes at b 1024 + 16 t, coefficient 16 b + e
+//          at byte kc8_pos(e): bytes 4c..4c+3 hold e = 2c, 2c+1, 2c+8, 2c+9, one lane's two
+//          A-operand pairs of an m16n8k16 MMA row.  The scales of tokens t and t + 8 of a
+//          16-token tile sit side by side (one 32-bit word for an MMA fragment's two rows).
+//  values: coefficient 16 b + e of token t at b 1024 + 64 e + 16 ((t/16) ^ (e/2 mod 4)) + t mod 16:
+//          rows of 64 tokens (the A operand of a tokens-deep integer MMA), the 16-byte chunks
+//          of a row rotated so that the 8 rows an ldmatrix reads fall in distinct banks.  A
+//          token's scales sit together: (R/16) fp16 at (R/16) 1024 + t (R/16) 2.
+__host__ __device__ inline uint32_t kc8_pos(int e) {
+    return e < 8 ? 4u * (uint32_t)(e >> 1) + (uint32_t)(e & 1) : 4u * (uint32_t)((e - 8) >> 1) + 2u + (uint32_t)(e & 1);
+}
+__host__ __device__ inline uint32_t kc8_code_off(int j, int t) { return (uint32_t)(j >> 4) * 1024u + 16u * (uint32_t)t + kc8_pos(j & 15); }
+__host__ __device__ inline uint32_t kc8_scale_off(int R, int b, int t) {
+    return (uint32_t)(R >> 4) * 1024u + (uint32_t)b * 128u + 2u * (16u * (uint32_t)(t >> 4) + 2u * (uint32_t)(t & 7) + (uint32_t)((t >> 3) & 1));
+}
+__host__ __device__ inline uint32_t vc8_code_off(int j, int t) {
+    const int e = j & 15;
+    return (uint32_t)(j >> 4) * 1024u + 64u * (uint32_t)e + 16u * (uint32_t)(((t >> 4) ^ (e >> 1)) & 3) + (uint32_t)(t & 15);
+}
+__host__ __device__ inline uint32_t vc8_scale_off(int R, int b, int t) {
+    return (uint32_t)(R >> 4) * 1024u + (uint32_t)t * (uint32_t)(R >> 4) * 2u + 2u * (uint32_t)b;
 }
 // Element offset of B_K[i][j] in a tiled basis (basis_kt) of rank r_max: 8 x 8 tiles, the tile
 // rows 16 contiguous bytes, so that an ldmatrix row set (8 rows of one tile) is one 128-byte line.
@@ -163,13 +192,14 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 //   ring    page chunks, packed back to back (a chunk that does not fit before the end
 //           starts again at 0); ring_bytes is chosen by the host
 //   rd      per consumer warp, one 4 KB residual tile (also holds B_K during the prologue)
-//   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W limbs [8][48] u8, P2[32][8]
+//   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W limbs [8][48] u8, P2[32][8];
+//           with 8-bit coefficients two more limb tiles CW [8 or 16][48] u8 (ping-pong over blocks)
 //   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  qh bf16 [d][4];  qb: q~ as MMA
 //           B fragments [ks][2][lane];  zero line
 //   bars    full[kSlots] empty[kSlots] basis table
 //   misc    tier table, page range, work counter; warp states; page-id batch; slot offsets
 struct DecodeSmem {
-    uint32_t ring, rd, small, small_stride, S, P, W, P2, qt, q, qh, qb, zero, bars, misc, tok, total;
+    uint32_t ring, rd, small, small_stride, S, P, W, P2, CW, qt, q, qh, qb, zero, bars, misc, tok, total;
 };
 // The CTA merge reuses the idle ring: the merged sums (at most 6 KB) at 0, B_V at kMergeBvOff.
 constexpr uint32_t kMergeBvOff = 8192;
@@ -188,6 +218,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(const Geom& G, uint32_t
     L.P = w;       w += 32 * 16;
     L.W = w;       w += 32 * 16;
     L.P2 = w;      w += probe ? 32 * 16 : 0;
+    L.CW = w;      w += G.c8 ? 2 * (probe ? 768 : 384) : 0;
     L.small_stride = w;
     L.small = o;   o += kConsumerWarps * w;
     L.qt = o;      o += (uint32_t)(G.r_max < 16 ? 16 : G.r_max) * 16;
@@ -337,6 +368,23 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// D (16x8 f32) += A (16x16 f16, row) * B (16x8 f16, col)
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// Two int8 values (bytes lo, lo + 1 of w when hi == 0, bytes 2, 3 when hi == 1) as an f16 pair,
+// exactly: the biased byte (x + 128) in the mantissa of 1024, then 1024 + 128 subtracted.
+__device__ __forceinline__ uint32_t s8x2_to_f16x2(uint32_t w, int hi) {
+    const uint32_t b = __byte_perm(w ^ 0x80808080u, 0x64646464u, hi ? 0x4342u : 0x4140u);
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(b), "r"(0x64806480u));
+    return r;
 }
 
 // D (16x8 s32) = A (16x32 s8, row) * B (32x8 u8, col) + C

@@ -152,19 +152,30 @@ __device__ __forceinline__ uint32_t rd_off(uint32_t row, uint32_t tok) {
 // eight rows' 4-byte words read by one B-fragment load then fall in distinct banks).
 constexpr uint32_t kWbPitch = 48;
 
+// Rescale the 8-bit-coefficient accumulators: [i][0] row g, [i][1] row g + 8, both of head c.
+template <int N>
+__device__ __forceinline__ void rescale_c8(float (&d)[N][4], float a) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) { d[i][0] *= a; d[i][1] *= a; }
+}
+
 // One warp's half of a tier-R page: tokens [32*half, 32*half + 32) of the page's 64 slots,
 // `nv` of them live.  `K` points at the page chunk's key block.
 // S >= 0: every token has S residual channels.  S < 0 (routed residual counts): the page's
 // tokens have s_rt in {0, 2, 4, 8}.
-template <int R, int S, int BITS, bool PROBE, int RMAX>
+// C8: coefficients in the 8-bit blockwise form (kc8_* / vc8_* layouts): qb holds q~ 2^E as
+// f16 hi / lo fragments (kexp = 2^-E), and the A.c / A.c2 accumulators hold rows g, g + 8 of
+// head c at [i][0], [i][1]; cw is the warp's two coefficient limb tiles.
+template <int R, int S, int BITS, bool PROBE, int RMAX, bool C8>
 __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int half, int nv,
                                           const uint32_t (&qb)[RMAX / 16][2], const uint2* __restrict__ qh,
                                           float qscale, uint8_t* small, uint8_t* rd, uint32_t zero_addr,
-                                          WarpAcc<RMAX, PROBE>& A, int lane, int s_rt) {
+                                          WarpAcc<RMAX, PROBE>& A, int lane, int s_rt, uint8_t* cw, float kexp) {
     constexpr bool ROUTED = S < 0;
     constexpr int KS = R >= 16 ? R / 16 : 1;         // 16-wide coefficient steps
+    static_assert(!C8 || R % 16 == 0, "8-bit coefficients come in blocks of 16");
     const int s_ = ROUTED ? s_rt : S;                // residual channels of this page's tokens
-    const uint32_t kOffIdx = 128u * R, kOffCodes = kOffIdx + 64u * s_;
+    const uint32_t kOffIdx = (C8 ? 72u : 128u) * R, kOffCodes = kOffIdx + 64u * s_;
     const uint32_t kOffSc = kOffCodes + ((8u * s_ * BITS + 127u) & ~127u);
     const uint32_t kBlk = kOffSc + 128u;
     const uint8_t* V = K + kBlk;
@@ -179,6 +190,31 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
     // ---------------- 1. coefficient scores: [32 tokens x R] . [R x 8] on the tensor cores
     {
         float d[2][4];
+        if constexpr (C8) {
+            // per block of 16: the codes as exact f16 against q~ 2^E (f16 hi / lo), then the
+            // block's per-token scale (times 2^-E) on the two rows of the fragment
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                d[mt][0] = d[mt][1] = d[mt][2] = d[mt][3] = 0.f;
+                const int t0 = tb + 16 * mt + g;
+#pragma unroll
+                for (int b = 0; b < KS; ++b) {
+                    const uint32_t w0 = *reinterpret_cast<const uint32_t*>(K + b * 1024 + t0 * 16 + 4 * c);
+                    const uint32_t w1 = *reinterpret_cast<const uint32_t*>(K + b * 1024 + (t0 + 8) * 16 + 4 * c);
+                    const uint32_t a[4] = {s8x2_to_f16x2(w0, 0), s8x2_to_f16x2(w1, 0), s8x2_to_f16x2(w0, 1),
+                                           s8x2_to_f16x2(w1, 1)};
+                    float e[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_f16(e, a, qb[b]);
+                    const uint32_t sw = *reinterpret_cast<const uint32_t*>(K + kc8_scale_off(R, b, t0));
+                    const float s0 = __half2float(__ushort_as_half((unsigned short)(sw & 0xffffu))) * kexp;
+                    const float s1 = __half2float(__ushort_as_half((unsigned short)(sw >> 16))) * kexp;
+                    d[mt][0] = fmaf(s0, e[0], d[mt][0]);
+                    d[mt][1] = fmaf(s0, e[1], d[mt][1]);
+                    d[mt][2] = fmaf(s1, e[2], d[mt][2]);
+                    d[mt][3] = fmaf(s1, e[3], d[mt][3]);
+                }
+            }
+        } else {
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
             d[mt][0] = d[mt][1] = d[mt][2] = d[mt][3] = 0.f;
@@ -191,6 +227,7 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 ldsm_x4(addr, a);
                 mma_bf16(d[mt], a, qb[ks]);
             }
+        }
         }
         // S: MMA columns 0-3 (the hi parts of heads 0-3) at [token][head], columns 4-7 (the lo
         // parts) kSLo floats on (summed per token below); S spans the P buffer and the start of
@@ -289,6 +326,7 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
     // ---------------- 3. online softmax (lazy rescale), p as bf16 hi/lo rows, p * scale^V as
     //                     fixed-point byte limbs
     float wdq = 0.f;                                   // this lane's head c: value of one limb unit
+    float p1[kGQ], p2v[PROBE ? kGQ : 1];               // this lane's token weights (with / without residual)
     {
         // The running max only moves when some score exceeds it by the slack (one vote);
         // otherwise p = exp2(s - m) <= 2^slack stays safe in fp32.
@@ -307,9 +345,9 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 }
                 A.l[h] *= alpha[h];
             }
-            const float a0 = alpha[(2 * c) & 3], a1 = alpha[(2 * c + 1) & 3];
-            rescale_d(A.c, a0, a1);
             const float ac = alpha[c];
+            if constexpr (C8) rescale_c8(A.c, ac);
+            else rescale_d(A.c, alpha[(2 * c) & 3], alpha[(2 * c + 1) & 3]);
 #pragma unroll
             for (int i = 0; i < 8; ++i) { A.r[i][0] *= ac; A.r[i][1] *= ac; }
         }
@@ -318,11 +356,14 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
         for (int h = 0; h < kGQ; ++h) {
             p[h] = exp2f(sc[h] - A.m[h]);      // dead lanes: exp2(-inf) = 0
             A.l[h] += p[h];
+            p1[h] = p[h];
         }
-        uint4 pr;
-        split2(p[0], p[1], pr.x, pr.z);
-        split2(p[2], p[3], pr.y, pr.w);
-        *reinterpret_cast<uint4*>(Psm + lane * 16) = pr;
+        if constexpr (!C8) {
+            uint4 pr;
+            split2(p[0], p[1], pr.x, pr.z);
+            split2(p[2], p[3], pr.y, pr.w);
+            *reinterpret_cast<uint4*>(Psm + lane * 16) = pr;
+        }
         if (s_) {
             // w = p * scale^V as 16-bit fixed point per head, in units of 2^(E-15) with E the
             // exponent of the half page's largest w: two byte limbs (hi, lo) per head
@@ -354,23 +395,96 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                     }
                     A.l2[h] *= alpha[h];
                 }
-                rescale_d(A.c2, alpha[(2 * c) & 3], alpha[(2 * c + 1) & 3]);
+                if constexpr (C8) rescale_c8(A.c2, alpha[c]);
+                else rescale_d(A.c2, alpha[(2 * c) & 3], alpha[(2 * c + 1) & 3]);
             }
 #pragma unroll
             for (int h = 0; h < kGQ; ++h) {
                 p[h] = exp2f(sc2[h] - A.m2[h]);
                 A.l2[h] += p[h];
+                p2v[h] = p[h];
             }
-            uint4 p2;
-            split2(p[0], p[1], p2.x, p2.z);
-            split2(p[2], p[3], p2.y, p2.w);
-            *reinterpret_cast<uint4*>(P2sm + lane * 16) = p2;
+            if constexpr (!C8) {
+                uint4 p2;
+                split2(p[0], p[1], p2.x, p2.z);
+                split2(p[2], p[3], p2.y, p2.w);
+                *reinterpret_cast<uint4*>(P2sm + lane * 16) = p2;
+            }
         }
     }
     __syncwarp();
 
     // ---------------- 4. coefficient-space values: acc_c[j][n] += sum_t C^V[t][j] P[t][n]
-    {
+    if constexpr (C8) {
+        // 8-bit form, per block b of 16: acc_c[16 b + e][h] += sum_t code[t][e] w_b[t][h] with
+        // w_b = p scale_b as 16-bit fixed point (two byte limbs, unit 2^(E-15) from the half
+        // page's largest w_b of head h), one integer MMA over the half page's 32 tokens
+        constexpr int NB = R / 16;
+        constexpr uint32_t kTile = PROBE ? 768u : 384u;
+        float svb[NB];
+        {
+            const uint8_t* sp = V + vc8_scale_off(R, 0, live ? t : 0);
+            uint16_t hs[NB];
+            if constexpr (NB == 1) hs[0] = *reinterpret_cast<const uint16_t*>(sp);
+            else if constexpr (NB == 2) { const uint32_t w = *reinterpret_cast<const uint32_t*>(sp); hs[0] = (uint16_t)w; hs[1] = (uint16_t)(w >> 16); }
+            else if constexpr (NB == 4) {
+                const uint2 w = *reinterpret_cast<const uint2*>(sp);
+                hs[0] = (uint16_t)w.x; hs[1] = (uint16_t)(w.x >> 16); hs[2] = (uint16_t)w.y; hs[3] = (uint16_t)(w.y >> 16);
+            } else {
+                const uint4 w = *reinterpret_cast<const uint4*>(sp);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) { hs[2 * q] = (uint16_t)ww[q]; hs[2 * q + 1] = (uint16_t)(ww[q] >> 16); }
+            }
+#pragma unroll
+            for (int b = 0; b < NB; ++b) svb[b] = live ? __half2float(__ushort_as_half(hs[b])) : 0.f;
+        }
+        const int arow = rr + 8 * (mi & 1), tcq = (tb >> 4) + (mi >> 1);
+        const uint32_t aoff = (uint32_t)arow * 64u + 16u * (uint32_t)((tcq ^ (arow >> 1)) & 3);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            uint8_t* tile = cw + (b & 1) * kTile;
+            float wq = 0.f, wq2 = 0.f;
+#pragma unroll
+            for (int h = 0; h < kGQ; ++h) {
+                const float wv = p1[h] * svb[b];                          // >= 0
+                const uint32_t eb = __reduce_max_sync(0xffffffffu, __float_as_uint(wv) >> 23);
+                uint32_t v = 0;
+                if (eb >= 16u) v = min(__float2uint_rn(wv * __uint_as_float((269u - eb) << 23)), 65535u);
+                tile[(2 * h) * kWbPitch + lane] = (uint8_t)(v >> 8);
+                tile[(2 * h + 1) * kWbPitch + lane] = (uint8_t)v;
+                if (c == h) wq = eb >= 16u ? __uint_as_float((eb - 15u) << 23) : 0.f;
+                if constexpr (PROBE) {
+                    const float w2 = p2v[h] * svb[b];
+                    const uint32_t e2 = __reduce_max_sync(0xffffffffu, __float_as_uint(w2) >> 23);
+                    uint32_t v2 = 0;
+                    if (e2 >= 16u) v2 = min(__float2uint_rn(w2 * __uint_as_float((269u - e2) << 23)), 65535u);
+                    tile[(8 + 2 * h) * kWbPitch + lane] = (uint8_t)(v2 >> 8);
+                    tile[(9 + 2 * h) * kWbPitch + lane] = (uint8_t)v2;
+                    if (c == h) wq2 = e2 >= 16u ? __uint_as_float((e2 - 15u) << 23) : 0.f;
+                }
+            }
+            __syncwarp();
+            uint32_t a[4];
+            ldsm_x4(vaddr + (uint32_t)b * 1024u + aoff, a);
+            {
+                const uint32_t bb[2] = {*reinterpret_cast<const uint32_t*>(tile + g * kWbPitch + 4 * c),
+                                        *reinterpret_cast<const uint32_t*>(tile + g * kWbPitch + 16 + 4 * c)};
+                int dd[4] = {0, 0, 0, 0};
+                mma_s8u8(dd, a, bb);
+                A.c[b][0] = fmaf(wq, (float)(dd[0] * 256 + dd[1]), A.c[b][0]);
+                A.c[b][1] = fmaf(wq, (float)(dd[2] * 256 + dd[3]), A.c[b][1]);
+            }
+            if constexpr (PROBE) {
+                const uint32_t bb[2] = {*reinterpret_cast<const uint32_t*>(tile + (8 + g) * kWbPitch + 4 * c),
+                                        *reinterpret_cast<const uint32_t*>(tile + (8 + g) * kWbPitch + 16 + 4 * c)};
+                int dd[4] = {0, 0, 0, 0};
+                mma_s8u8(dd, a, bb);
+                A.c2[b][0] = fmaf(wq2, (float)(dd[0] * 256 + dd[1]), A.c2[b][0]);
+                A.c2[b][1] = fmaf(wq2, (float)(dd[2] * 256 + dd[3]), A.c2[b][1]);
+            }
+        }
+    } else {
         const uint32_t paddr = smem_addr(Psm), p2addr = smem_addr(P2sm);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
@@ -451,20 +565,34 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
     }
 }
 
-template <int S, int BITS, bool PROBE, int RMAX>
+template <int S, int BITS, bool PROBE, int RMAX, bool C8>
 __device__ __forceinline__ void run_page(int R, const uint8_t* K, int half, int nv, const uint32_t (&qb)[RMAX / 16][2],
                                          const uint2* qs, float qscale, uint8_t* small, uint8_t* rd, uint32_t zero_addr,
-                                         WarpAcc<RMAX, PROBE>& A, int lane, int s_rt) {
+                                         WarpAcc<RMAX, PROBE>& A, int lane, int s_rt, uint8_t* cw, float kexp) {
+#define DWKV_HP(RR) half_page<RR, S, BITS, PROBE, RMAX, C8>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt, cw, kexp)
     switch (R) {
-        case 8: half_page<8, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt); break;
-        case 16: half_page<16, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt); break;
-        case 32: half_page<32, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt); break;
-        case 64: half_page<64, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt); break;
+        case 8: if constexpr (!C8) DWKV_HP(8); break;     // 8-bit coefficient tiers are multiples of 16
+        case 16: DWKV_HP(16); break;
+        case 32: DWKV_HP(32); break;
+        case 64: DWKV_HP(64); break;
         case 128:
-            if constexpr (RMAX >= 128)
-                half_page<128, S, BITS, PROBE, RMAX>(K, half, nv, qb, qs, qscale, small, rd, zero_addr, A, lane, s_rt);
+            if constexpr (RMAX >= 128) DWKV_HP(128);
             break;
         default: break;
+    }
+#undef DWKV_HP
+}
+
+// Store the 8-bit-coefficient accumulators ([i][0] row 16 i + g, [i][1] row 16 i + g + 8, head
+// c) as acc[j][h] (float4 per row j).
+template <int N>
+__device__ __forceinline__ void store_c8(const float (&d)[N][4], float* dst, int rows, int lane) {
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int j0 = 16 * i + g, j1 = j0 + 8;
+        if (j0 < rows) dst[j0 * 4 + c] = d[i][0];
+        if (j1 < rows) dst[j1 * 4 + c] = d[i][1];
     }
 }
 
@@ -545,16 +673,22 @@ __device__ __forceinline__ void owner_append(const Geom& G, const State& St, con
 // Consumer warp 0 of that CTA, after its pages: attend to the new token from its stored bytes
 // (the score over its coefficients and residual, the online-softmax update, and its value in
 // both spaces), so no other CTA waits for it.
-template <int S, int BITS, int RMAX>
+template <int S, int BITS, int RMAX, bool C8>
 __device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, const float4* qt, const float4* qs,
                                               WarpAcc<RMAX, false>& A, int lane) {
     const Dest& d = td.d;
     const int R = d.R, row = d.row;
     const int s_ = S < 0 ? G.ts[d.k] : S;            // the token's residual channels
-    const uint32_t offIdx = off_idx_of(R), offCodes = off_codes_of(R, s_), offSc = off_scales_of(R, s_, BITS);
+    const uint32_t offIdx = off_idx_of(R, C8), offCodes = off_codes_of(R, s_, C8), offSc = off_scales_of(R, s_, BITS, C8);
     const uint8_t* Kb = d.blk;
     const uint8_t* Vb = d.blk + G.blk_bytes[d.k];
-    auto coeff = [&](const uint8_t* blk, int j) {
+    auto coeff = [&](const uint8_t* blk, int j) -> float {
+        if constexpr (C8) {
+            const bool key = blk == Kb;
+            const int8_t q = (int8_t)blk[key ? kc8_code_off(j, row) : vc8_code_off(j, row)];
+            const uint32_t so = key ? kc8_scale_off(R, j >> 4, row) : vc8_scale_off(R, j >> 4, row);
+            return (float)q * __half2float(*reinterpret_cast<const __half*>(blk + so));     // exact
+        }
         return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(blk + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2));
     };
     auto code = [&](const uint8_t* blk, int e) -> float {
@@ -594,7 +728,8 @@ __device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, 
     }
     const int g = lane >> 2, c = lane & 3;
     if (over) {
-        rescale_d(A.c, alpha[(2 * c) & 3], alpha[(2 * c + 1) & 3]);
+        if constexpr (C8) rescale_c8(A.c, alpha[c]);
+        else rescale_d(A.c, alpha[(2 * c) & 3], alpha[(2 * c + 1) & 3]);
 #pragma unroll
         for (int i = 0; i < 8; ++i) { A.r[i][0] *= alpha[c]; A.r[i][1] *= alpha[c]; }
     }
@@ -604,8 +739,16 @@ __device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, 
         p[hh] = exp2f(s_t[hh] - A.m[hh]);
         if (lane == 0) A.l[hh] += p[hh];               // A.l is summed over the lanes later
     }
-    // values, coefficient space: rows j = 16 i + g (+8), hi columns (lanes c < 2: heads 2c, 2c+1)
-    if (c < 2) {
+    // values, coefficient space: rows j = 16 i + g (+8), hi columns (lanes c < 2: heads 2c, 2c+1);
+    // 8-bit form: rows j of head c
+    if constexpr (C8) {
+#pragma unroll
+        for (int i = 0; i < RMAX / 16; ++i) {
+            const int j0 = 16 * i + g, j1 = j0 + 8;
+            if (j0 < R) A.c[i][0] = fmaf(p[c], coeff(Vb, j0), A.c[i][0]);
+            if (j1 < R) A.c[i][1] = fmaf(p[c], coeff(Vb, j1), A.c[i][1]);
+        }
+    } else if (c < 2) {
 #pragma unroll
         for (int i = 0; i < RMAX / 16; ++i) {
             const int j0 = 16 * i + g, j1 = j0 + 8;
@@ -640,8 +783,9 @@ __device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, 
 }  // namespace decode_detail
 
 // BITS: code width; PROBE: second softmax state without the residual; RMAX: accumulator
-// rows (>= r_max); S: residual channels per token (0, 8, 16 or 32), or -1 for per-tier counts.
-template <int BITS, bool PROBE, int RMAX, int S>
+// rows (>= r_max); S: residual channels per token (0, 8, 16 or 32), or -1 for per-tier counts;
+// C8: coefficients in the 8-bit blockwise form.
+template <int BITS, bool PROBE, int RMAX, int S, bool C8>
 __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G, const State St, const DecodeCall C) {
     using namespace decode_detail;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -854,6 +998,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         // ================= consumer warps
         uint8_t* rd = smem + L.rd + warp * kRdBytes;
         uint8_t* small = smem + L.small + warp * L.small_stride;
+        uint8_t* cw = small + L.CW;
         const uint32_t zero_addr = smem_addr(smem + L.zero);
         const float qscale = G.tau * kLog2e;
         uint2* qh = reinterpret_cast<uint2*>(smem + L.qh);
@@ -918,7 +1063,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         }
         named_barrier(1, kConsumerWarps * 32);
         // q~ as the score MMA's B operand, the same fragments in every warp: built once into
-        // qbs [ks][r2][lane] (column n < 4 = bf16 hi of head n, n >= 4 = lo of head n-4)
+        // qbs [ks][r2][lane] (column n < 4 = bf16 hi of head n, n >= 4 = lo of head n-4).
+        // 8-bit coefficients: f16 hi / lo of q~ 2^E instead, E putting max |q~| in [2^14, 2^15)
+        // (the f16 range; each warp finds the max itself), and kexp = 2^-E.
+        float qsc = 1.f, kexp = 1.f;
+        if constexpr (C8) {
+            uint32_t mb = 0u;
+            for (int k = lane; k < rq; k += 32) {
+                const float4 t4 = qt[k];
+                mb = max(mb, max(max(__float_as_uint(fabsf(t4.x)), __float_as_uint(fabsf(t4.y))),
+                                 max(__float_as_uint(fabsf(t4.z)), __float_as_uint(fabsf(t4.w)))));
+            }
+            const uint32_t eb = __reduce_max_sync(0xffffffffu, mb) >> 23;      // biased exponent of the max
+            if (eb >= 15u && eb < 255u) {
+                qsc = __uint_as_float((268u - eb) << 23);                       // 2^(141 - eb)
+                kexp = __uint_as_float((eb - 14u) << 23);                       // 2^(eb - 141)
+            }
+        }
         uint32_t* qbs = reinterpret_cast<uint32_t*>(smem + L.qb);
         for (int x = tid; x < 32 * 2 * (RMAX / 16); x += kConsumerWarps * 32) {
             const int ln = x & 31, ks = (x >> 5) >> 1, r2 = (x >> 5) & 1;
@@ -934,7 +1095,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                     v = n == 0 ? t4.x : n == 1 ? t4.y : n == 2 ? t4.z : t4.w;
                 }
                 uint32_t hi, lo;
-                split_bf16_rn(v, hi, lo);
+                if constexpr (C8) {
+                    const float vs = v * qsc;                                   // exact (power of two)
+                    const __half hh = __float2half_rn(vs);
+                    hi = __half_as_ushort(hh);
+                    lo = __half_as_ushort(__float2half_rn(vs - __half2float(hh)));
+                } else {
+                    split_bf16_rn(v, hi, lo);
+                }
                 pk |= (lo_half ? lo : hi) << (16 * e);
             }
             qbs[x] = pk;
@@ -1001,8 +1169,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             }
             const int nv = min(max(nvalid - 32 * half, 0), 32);
             if (nv > 0)
-                run_page<S, BITS, PROBE, RMAX>(R, smem + L.ring + m_slot[sl], half, nv, qb, qh,
-                                               qscale, small, rd, zero_addr, A, lane, G.ts[k]);
+                run_page<S, BITS, PROBE, RMAX, C8>(R, smem + L.ring + m_slot[sl], half, nv, qb, qh,
+                                               qscale, small, rd, zero_addr, A, lane, G.ts[k], cw, kexp);
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8 * sl);
             if (wn == 0xffffffffu) {
@@ -1013,13 +1181,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         }
         if constexpr (!PROBE) {
             if (owner && warp == 0 && tokd->ok)
-                add_new_token<S, BITS, RMAX>(G, *tokd, reinterpret_cast<const float4*>(smem + L.qt), qs, A, lane);
+                add_new_token<S, BITS, RMAX, C8>(G, *tokd, reinterpret_cast<const float4*>(smem + L.qt), qs, A, lane);
         }
         // ---- per-warp results: acc_c [r_max][4] and acc_r [d][4] into the residual tile,
         //      the probe's acc_c2 into the small buffers; m / l into m_state
         float* oc = reinterpret_cast<float*>(rd);
         float* orr = oc + G.r_max * 4;
-        store_d(A.c, oc, G.r_max, lane);
+        if constexpr (C8) store_c8(A.c, oc, G.r_max, lane);
+        else store_d(A.c, oc, G.r_max, lane);
         {
             const int g = lane >> 2, c = lane & 3;
 #pragma unroll
@@ -1028,7 +1197,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                 orr[(16 * i + g + 8) * 4 + c] = A.r[i][1];
             }
         }
-        if (PROBE) store_d(A.c2, reinterpret_cast<float*>(small), G.r_max, lane);
+        if constexpr (PROBE && C8) store_c8(A.c2, reinterpret_cast<float*>(small), G.r_max, lane);
+        else if constexpr (PROBE) store_d(A.c2, reinterpret_cast<float*>(small), G.r_max, lane);
         float* ms = m_state + warp * 16;
         float l[kGQ], l2[kGQ];
 #pragma unroll
@@ -1332,18 +1502,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
 
 }  // namespace dwkv
 
-// Explicit instantiations for one (BITS, PROBE) pair: RMAX in {64, 128}, S in {0, 8, 16, 32}
-// and -1 (routed residual counts).
-#define DWKV_DECODE_INSTANTIATE(B, P)                                                        \
-    namespace dwkv {                                                                          \
-    template __global__ void decode_kernel<B, P, 64, 0>(const Geom, const State, const DecodeCall);   \
-    template __global__ void decode_kernel<B, P, 64, 8>(const Geom, const State, const DecodeCall);   \
-    template __global__ void decode_kernel<B, P, 64, 16>(const Geom, const State, const DecodeCall);  \
-    template __global__ void decode_kernel<B, P, 64, 32>(const Geom, const State, const DecodeCall);  \
-    template __global__ void decode_kernel<B, P, 128, 0>(const Geom, const State, const DecodeCall);  \
-    template __global__ void decode_kernel<B, P, 128, 8>(const Geom, const State, const DecodeCall);  \
-    template __global__ void decode_kernel<B, P, 128, 16>(const Geom, const State, const DecodeCall); \
-    template __global__ void decode_kernel<B, P, 128, 32>(const Geom, const State, const DecodeCall); \
-    template __global__ void decode_kernel<B, P, 64, -1>(const Geom, const State, const DecodeCall);  \
-    template __global__ void decode_kernel<B, P, 128, -1>(const Geom, const State, const DecodeCall); \
+// Explicit instantiations for one (BITS, PROBE, C8) triple: RMAX in {64, 128}, S in {0, 8, 16,
+// 32} and -1 (routed residual counts).
+#define DWKV_DECODE_INSTANTIATE(B, P, C)                                                          \
+    namespace dwkv {                                                                               \
+    template __global__ void decode_kernel<B, P, 64, 0, C>(const Geom, const State, const DecodeCall);   \
+    template __global__ void decode_kernel<B, P, 64, 8, C>(const Geom, const State, const DecodeCall);   \
+    template __global__ void decode_kernel<B, P, 64, 16, C>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 64, 32, C>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 128, 0, C>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 128, 8, C>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 128, 16, C>(const Geom, const State, const DecodeCall); \
+    template __global__ void decode_kernel<B, P, 128, 32, C>(const Geom, const State, const DecodeCall); \
+    template __global__ void decode_kernel<B, P, 64, -1, C>(const Geom, const State, const DecodeCall);  \
+    template __global__ void decode_kernel<B, P, 128, -1, C>(const Geom, const State, const DecodeCall); \
     }

@@ -1,4 +1,4 @@
-// Decode / probe kernels for 8-bit codes, probe variant (one translation unit per pair, built in parallel).
+// Decode / probe kernels for 8-bit codes, probe variant, bf16 coefficients (one translation unit per triple, built in parallel).
 #include "dwkv_decode.cuh"
 
-DWKV_DECODE_INSTANTIATE(8, true)
+DWKV_DECODE_INSTANTIATE(8, true, false)

@@ -10,6 +10,9 @@
 //   4. the s largest |r_i|, ties to the lower channel, stored in ascending channel order
 //   5. scale = fp16_rn(max |r_sel| / qmax) with IEEE division, qmax = 127 (int8) / 7 (int4)
 //   6. code  = clamp(rint(r / float(scale)), -qmax, qmax), all zero when scale == 0
+// With 8-bit coefficients (the blockwise form kept by the pages), step 2 becomes, per block of
+// 16 coefficients: sc = fp16_rn(max |c| / 127) (IEEE division), q_j = clamp(rint(c_j /
+// float(sc)), -127, 127) (0 when sc == 0), cb_j = q_j float(sc) (exact); steps 3-6 as above.
 #pragma once
 #include "dwkv_common.cuh"
 
@@ -173,7 +176,7 @@ static __device__ __noinline__ uint32_t select_exact(float r0, float r1, float r
 // exact zeros) the selection is redone by its definition (select_exact).
 template <int BITS>
 __device__ __forceinline__ void quantize_store(const float (&r)[4], uint8_t* blk, int R, int row, int s,
-                                               float* rstage, uint8_t* chstage) {
+                                               float* rstage, uint8_t* chstage, int c8) {
     const int lane = threadIdx.x & 31;
     const float qmax = BITS == 8 ? 127.f : 7.f;
     uint32_t sel = 0u, mxb = 0u;
@@ -230,7 +233,7 @@ __device__ __forceinline__ void quantize_store(const float (&r)[4], uint8_t* blk
         }
         before += __popc(bal);
     }
-    if (lane == 0) *reinterpret_cast<__half*>(blk + off_scales_of(R, s, BITS) + row * 2) = sh;
+    if (lane == 0) *reinterpret_cast<__half*>(blk + off_scales_of(R, s, BITS, c8) + row * 2) = sh;
     __syncwarp();
     for (int b0 = 0; b0 < s; b0 += 32) {
         const int b = b0 + lane;
@@ -239,16 +242,32 @@ __device__ __forceinline__ void quantize_store(const float (&r)[4], uint8_t* blk
             float c = 0.f;
             if (sf != 0.f) c = fminf(fmaxf(rintf(__fdiv_rn(rstage[b], sf)), -qmax), qmax);
             code = (int)c;
-            blk[off_idx_of(R) + row * s + b] = chstage[b];
-            if (BITS == 8) blk[off_codes_of(R, s) + row * s + b] = (uint8_t)(int8_t)code;
+            blk[off_idx_of(R, c8) + row * s + b] = chstage[b];
+            if (BITS == 8) blk[off_codes_of(R, s, c8) + row * s + b] = (uint8_t)(int8_t)code;
         }
         if (BITS == 4) {
             const int hi = __shfl_down_sync(0xffffffffu, code, 1);
             if (b < s && !(b & 1))
-                blk[off_codes_of(R, s) + row * (s / 2) + (b >> 1)] = (uint8_t)((code & 0xf) | ((hi & 0xf) << 4));
+                blk[off_codes_of(R, s, c8) + row * (s / 2) + (b >> 1)] = (uint8_t)((code & 0xf) | ((hi & 0xf) << 4));
         }
     }
     __syncwarp();
+}
+
+// Step 2 of the 8-bit coefficient form for one value per lane, the lanes of each half warp one
+// block of 16 (every lane of the warp calls it): the block's scale (fp16 bits) and this lane's
+// code and dequantised value.
+__device__ __forceinline__ void quantize_coeff8(float v, uint16_t& sh_out, int& q_out, float& cb_out) {
+    float m = fabsf(v);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const __half sh = __float2half_rn(__fdiv_rn(m, 127.f));
+    const float sf = __half2float(sh);
+    float q = 0.f;
+    if (sf != 0.f) q = fminf(fmaxf(rintf(__fdiv_rn(v, sf)), -127.f), 127.f);
+    sh_out = __half_as_ushort(sh);
+    q_out = (int)q;
+    cb_out = q * sf;
 }
 
 // The six encode steps of one unit on one warp.
@@ -288,7 +307,21 @@ __device__ __forceinline__ void encode_body(const Geom& G, const State& S, const
 #pragma unroll
             for (int jj = 0; jj < kMaxRank / 32; ++jj) {
                 const int j = lane + 32 * jj;
-                if (j < R) {
+                if (G.c8) {
+                    if (32 * jj >= R) break;                       // uniform: R is a multiple of 16
+                    uint16_t sh;
+                    int q;
+                    float cb;
+                    quantize_coeff8(j < R ? acc[jj] : 0.f, sh, q, cb);
+                    if (j < R) {
+                        if (in.dbg) in.dbg[j] = acc[jj];
+                        cs[j] = cb;
+                        blk[z ? vc8_code_off(j, dst.row) : kc8_code_off(j, dst.row)] = (uint8_t)(int8_t)q;
+                        if ((j & 15) == 0)
+                            *reinterpret_cast<uint16_t*>(blk + (z ? vc8_scale_off(R, j >> 4, dst.row)
+                                                                  : kc8_scale_off(R, j >> 4, dst.row))) = sh;
+                    }
+                } else if (j < R) {
                     if (in.dbg) in.dbg[j] = acc[jj];
                     const __nv_bfloat16 cb = __float2bfloat16_rn(acc[jj]);
                     cs[j] = __bfloat162float(cb);
@@ -313,7 +346,7 @@ __device__ __forceinline__ void encode_body(const Geom& G, const State& S, const
 #pragma unroll
             for (int m = 0; m < 4; ++m) r[m] = __fsub_rn(xr[m], a[m]);
         }
-        quantize_store<BITS>(r, blk, R, dst.row, G.ts[dst.k], xs, reinterpret_cast<uint8_t*>(cstage));
+        quantize_store<BITS>(r, blk, R, dst.row, G.ts[dst.k], xs, reinterpret_cast<uint8_t*>(cstage), G.c8);
     } while (false);
     __syncwarp();
 }

@@ -106,6 +106,13 @@ typedef struct {
      * resid_channels == 8 (the stride of the residual arrays of append_compressed / export). */
     int32_t resid_routed;
     int32_t tier_resid[DWKV_MAX_TIERS];
+    /* Coefficient storage ([DW] §3 Method, the shared-bases paragraph: the projection onto the
+     * basis is kept in 8-bit blockwise form).  16 (or 0): bf16.  8: int8 codes in blocks of
+     * 16 coefficients with one fp16 scale a block, scale = fp16(max |c| / 127) and
+     * code = clamp(rint(c / scale), -127, 127); the residual is taken against code * scale.
+     * Needs r_max and every tier rank to be multiples of 16.  Re-tiering and the basis
+     * update's re-projection have no kernels for it (DWKV_ERR_UNSUPPORTED). */
+    int32_t coeff_bits;
 } dwkv_config;
 
 /* ---- Online bases ([DW] §3 Method, the shared-bases paragraph: "initialized online from
@@ -167,8 +174,9 @@ const char* dwkv_last_error(void);
 dwkv_status dwkv_config_check(const dwkv_config* cfg);
 
 /* Bytes of one stored token (one layer, one kv-head, keys + values) at tier index
- * `tier`: 2 * (2*r + s + s*bits/8 + 2), s the tier's residual channels.  0 if the arguments
- * are invalid. */
+ * `tier`: 2 * (C + s + s*bits/8 + 2), s the tier's residual channels, C = 2 r (bf16
+ * coefficients) or r + r/8 (8-bit codes and their block scales).  0 if the arguments are
+ * invalid. */
 size_t dwkv_token_bytes(const dwkv_config* cfg, int32_t tier);
 
 /* Bytes of one page of tier `tier`: DWKV_PAGE_TOKENS tokens of one (sequence, group,
@@ -241,7 +249,9 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
 /* Appends tokens that are already in compressed form (import of a prepared cache).
  * Same sequence / position rules as dwkv_append.  Device arrays, tokens in list order,
  * K at [..][0][..] and V at [..][1][..]:
- *   coeff  bf16  [sum(n_new)][Hkv][2][r_max]   (entries at j >= r_t are ignored)
+ *   coeff  [sum(n_new)][Hkv][2] coefficient records (entries at j >= r_t are ignored):
+ *          bf16 [r_max] (coeff_bits 16), or with coeff_bits 8 r_max + r_max/8 bytes,
+ *          int8 codes [r_max] then fp16 block scales [r_max/16] (2-byte aligned)
  *   idx    uint8 [sum(n_new)][Hkv][2][s]       (each < head_dim)
  *   codes  int8  [sum(n_new)][Hkv][2][s]       (int4 caches: each in [-8, 7])
  *   scales fp16  [sum(n_new)][Hkv][2] */
@@ -346,7 +356,8 @@ dwkv_status dwkv_tier_controller_route(dwkv_tier_controller c, int32_t group, in
                                        int32_t high_tier, uint8_t* tier_out);
 
 /* Reads positions [t0, t0 + n) of (layer, seq) back in token order, as stored:
- *   tier_idx uint8 [n][Hkv]; coeff bf16 [n][Hkv][2][r_max] (zeros at j >= r_t);
+ *   tier_idx uint8 [n][Hkv]; coeff [n][Hkv][2] coefficient records as in
+ *   dwkv_append_compressed (zeros at j >= r_t);
  *   idx uint8 [n][Hkv][2][s]; codes int8 [n][Hkv][2][s]; scales fp16 [n][Hkv][2].
  * All device pointers; any of them may be NULL to skip that array. */
 dwkv_status dwkv_export(dwkv_handle h, int32_t layer, int32_t seq, int32_t t0, int32_t n,

@@ -60,6 +60,7 @@ class Workload:
     noise_var: float = 0.0
     resid_var: float = 0.05           # scale drawn from max |N(0, resid_var)| / qmax
     tier_resid: tuple = ()            # per-tier residual counts (every tier at one rank), or ()
+    coeff_bits: int = 16              # 16: bf16 coefficients; 8: int8 codes + fp16 scale per block of 16
     extra: dict = field(default_factory=dict)
 
     @property
@@ -85,6 +86,11 @@ WORKLOADS = {
         head_dim=128, r_max=64, tiers=(16, 32, 64), tier_probs=(0.6, 0.3, 0.1),
         resid_channels=16, resid_bits=4, batch=1, context=65536, base_seed=1002,
         coeff_var_rank=64, noise_var=0.01),
+    "llama8b_64k_c8": Workload(
+        name="llama8b_64k_c8", num_layers=32, layers_per_group=2, num_q_heads=32, num_kv_heads=8,
+        head_dim=128, r_max=64, tiers=(16, 32, 64), tier_probs=(0.6, 0.3, 0.1),
+        resid_channels=16, resid_bits=4, batch=1, context=65536, base_seed=1007,
+        coeff_var_rank=64, noise_var=0.01, coeff_bits=8),
     "llama8b_ragged_b8": Workload(
         name="llama8b_ragged_b8", num_layers=32, layers_per_group=2, num_q_heads=32,
         num_kv_heads=8, head_dim=128, r_max=64, tiers=(16, 32, 64),
@@ -230,6 +236,14 @@ def make_compressed(wl: Workload, seq: int, layer: int, tier_idx: torch.Tensor,
     With per-tier residual counts (``wl.tier_resid``) a token of tier k keeps the first
     ``tier_resid[k]`` entries of idx / codes; the entries past them are zero (the scale too
     when the count is 0), or left as drawn with ``garbage_tail`` (they must be ignored).
+
+    With 8-bit coefficients (``wl.coeff_bits == 8``) ``coeff`` is replaced by
+
+    * ``ccodes``  int8 ``[n][Hkv][2][r_max]``: round(N(0, (127/2.5)^2)) clipped to [-127, 127];
+    * ``cscales`` fp16 ``[n][Hkv][2][r_max / 16]``: for block b, max |N(0, 1/j)| over its 16
+      rank indices j, divided by 127,
+
+    zero past r_t (blocks past r_t / 16), or N(0, 1)-scaled garbage with ``garbage_tail``.
     """
     seed = wl.base_seed if seed is None else seed
     n = tier_idx.shape[0]
@@ -247,6 +261,21 @@ def make_compressed(wl: Workload, seq: int, layer: int, tier_idx: torch.Tensor,
     else:
         coeff = coeff * keep
     coeff = coeff.to(torch.bfloat16)
+    c8 = None
+    if wl.coeff_bits == 8:
+        nb = R // 16
+        codes8 = (torch.randn(n, H, 2, R, generator=g, device=device) * (127 / 2.5)).round().clamp_(-127, 127)
+        amax = (torch.randn(n, H, 2, nb, 16, generator=g, device=device) * j.view(nb, 16).rsqrt()).abs().amax(-1)
+        sc8 = amax / 127
+        if garbage_tail:
+            junk_c = torch.randint(-128, 128, (n, H, 2, R), generator=g, device=device).float()
+            junk_s = torch.rand(n, H, 2, nb, generator=g, device=device) * 4
+            codes8 = torch.where(keep, codes8, junk_c)
+            sc8 = torch.where(keep[..., ::16], sc8, junk_s)
+        else:
+            codes8 = codes8 * keep
+            sc8 = sc8 * keep[..., ::16]
+        c8 = (codes8.to(torch.int8), sc8.to(torch.float16))
     if s > 0:
         keys = torch.rand(n, H, 2, d, generator=g, device=device)
         idx = keys.topk(s, dim=-1).indices.sort(dim=-1).values.to(torch.uint8)
@@ -264,6 +293,8 @@ def make_compressed(wl: Workload, seq: int, layer: int, tier_idx: torch.Tensor,
         idx = idx * on
         codes = codes * on
         scales = scales * (nres.view(n, H, 1) > 0)
+    if c8 is not None:
+        return {"ccodes": c8[0], "cscales": c8[1], "idx": idx, "codes": codes, "scales": scales}
     return {"coeff": coeff, "idx": idx, "codes": codes, "scales": scales}
 
 

@@ -80,7 +80,7 @@ def cfg_for(wl, max_batch=None, max_context=None, softmax_scale=0.0):
         num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, r_max=wl.r_max, tiers=wl.tiers,
         resid_channels=wl.resid_channels, resid_bits=wl.resid_bits,
         max_batch=max_batch or wl.batch, max_context=max_context or wl.context, softmax_scale=softmax_scale,
-        tier_resid=wl.tier_resid or None)
+        tier_resid=wl.tier_resid or None, coeff_bits=wl.coeff_bits)
 
 
 def to_dev(d: dict, device="cuda") -> dict:
@@ -101,7 +101,8 @@ def import_workload(cache, wl, lengths, gen_device="cpu", garbage=False, seed=No
             tiers = tiers_by_group[g]
             comp = synth.make_compressed(wl, seq, layer, tiers, device=gen_device, seed=seed, garbage_tail=garbage)
             c = to_dev(comp)
-            cache.append_compressed(layer, [seq], [T], tiers.to("cuda").contiguous(), c["coeff"], c["idx"],
+            coeff = (c["ccodes"], c["cscales"]) if "ccodes" in c else c["coeff"]
+            cache.append_compressed(layer, [seq], [T], tiers.to("cuda").contiguous(), coeff, c["idx"],
                                     c["codes"], c["scales"])
             data[(seq, layer)] = (tiers, comp)
     return data
@@ -126,7 +127,10 @@ def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None, c32=None
     n, H, s = k.shape[0], wl.num_kv_heads, wl.resid_channels
     ranks = synth.ranks_of(wl, tier_idx)
     nres = synth.resid_counts_of(wl, tier_idx) if wl.tier_resid else None
+    c8 = wl.coeff_bits == 8
     coeff = np.zeros((n, H, 2, wl.r_max), np.uint16)
+    ccodes = np.zeros((n, H, 2, wl.r_max), np.int8)
+    cscales = np.zeros((n, H, 2, wl.r_max // 16), np.uint16)
     idx = np.zeros((n, H, 2, s), np.uint8)
     codes = np.zeros((n, H, 2, s), np.int8)
     scales = np.zeros((n, H, 2), np.uint16)
@@ -134,16 +138,28 @@ def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None, c32=None
         c32 = np.nan_to_num(np.asarray(c32.cpu() if hasattr(c32, "cpu") else c32, np.float32))
     for h in range(H):
         for z, x in enumerate((k, v)):
-            if c32 is not None:
+            nr = None if nres is None else nres[:, h]
+            if c8:
+                r = oracle.encode_many8(bases[z][g, h], x[:, h], ranks[:, h], s, wl.resid_bits,
+                                        c32=None if c32 is None else c32[:, h, z], nthreads=nthreads, nres=nr)
+                ccodes[:, h, z], cscales[:, h, z] = r["ccodes"], r["cscales"]
+            elif c32 is not None:
                 r = oracle.encode_many_from_coeffs(bases[z][g, h], x[:, h], c32[:, h, z], ranks[:, h], s, wl.resid_bits,
-                                                   nthreads=nthreads, nres=None if nres is None else nres[:, h])
+                                                   nthreads=nthreads, nres=nr)
             else:
                 r = oracle.encode_many(bases[z][g, h], x[:, h], ranks[:, h], s, wl.resid_bits, nthreads=nthreads,
-                                       nres=None if nres is None else nres[:, h])
-            coeff[:, h, z], idx[:, h, z], codes[:, h, z], scales[:, h, z] = r["coeff"], r["idx"], r["codes"], r["scale"]
-    return {"coeff": torch.from_numpy(coeff.view(np.int16)).view(torch.bfloat16),
-            "idx": torch.from_numpy(idx), "codes": torch.from_numpy(codes),
-            "scales": torch.from_numpy(scales.view(np.int16)).view(torch.float16)}
+                                       nres=nr)
+            if not c8:
+                coeff[:, h, z] = r["coeff"]
+            idx[:, h, z], codes[:, h, z], scales[:, h, z] = r["idx"], r["codes"], r["scale"]
+    out = {"idx": torch.from_numpy(idx), "codes": torch.from_numpy(codes),
+           "scales": torch.from_numpy(scales.view(np.int16)).view(torch.float16)}
+    if c8:
+        out["ccodes"] = torch.from_numpy(ccodes)
+        out["cscales"] = torch.from_numpy(cscales.view(np.int16)).view(torch.float16)
+    else:
+        out["coeff"] = torch.from_numpy(coeff.view(np.int16)).view(torch.bfloat16)
+    return out
 
 
 def cat_comp(a: dict, b: dict) -> dict:

@@ -32,7 +32,7 @@ def _cfg(wl, **over):
     kw = dict(num_layers=wl.num_layers, layers_per_group=wl.layers_per_group, num_q_heads=wl.num_q_heads,
               num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, r_max=wl.r_max, tiers=wl.tiers,
               resid_channels=wl.resid_channels, resid_bits=wl.resid_bits, max_batch=wl.batch,
-              max_context=wl.context + 64, tier_resid=wl.tier_resid or None)
+              max_context=wl.context + 64, tier_resid=wl.tier_resid or None, coeff_bits=wl.coeff_bits)
     kw.update(over)
     return dw.config_from(**kw)
 
@@ -94,6 +94,31 @@ def test_routed_token_and_page_bytes():
     for k, n in enumerate((0, 2, 4, 8)):
         code = (8 * n * 4 + 127) // 128 * 128
         assert dw.dwkv_page_bytes(cfg, k) == 2 * 2 * (128 * 32 + 64 * n + code + 128) + 64 * 4
+
+
+@pytest.mark.parametrize("over", [
+    dict(coeff_bits=8, tiers=(8, 16, 32), r_max=32),            # whole blocks of 16
+    dict(coeff_bits=8, tiers=(8,), r_max=8),                    # r_max a multiple of 16
+    dict(coeff_bits=4),
+    dict(coeff_bits=32),
+])
+def test_invalid_coefficient_widths_are_rejected(over):
+    cfg = _cfg(synth.workload("llama8b_64k"), **over)
+    assert dw.dwkv_config_check(cfg) == 1
+    assert dw.dwkv_last_error()
+
+
+def test_8bit_coefficient_token_and_page_bytes():
+    """8-bit coefficients: r codes + r/16 fp16 scales a vector (r + r/8 bytes); a page block
+    holds 72 r bytes of them (1 KB of codes and 128 bytes of scales per block of 16)."""
+    cfg = _cfg(synth.workload("llama8b_64k_c8"))
+    assert cfg.coeff_bits == 8 and dw.dwkv_config_check(cfg) == 0
+    assert [dw.dwkv_token_bytes(cfg, k) for k in range(3)] == [2 * (r + r // 8 + 16 + 8 + 2) for r in (16, 32, 64)]
+    for k, r in enumerate((16, 32, 64)):
+        assert dw.dwkv_page_bytes(cfg, k) == 2 * 2 * (72 * r + 64 * 16 + 8 * 16 * 4 + 128) + 64 * 4
+        assert dw.dwkv_page_bytes(cfg, k) % 128 == 0
+    bf = _cfg(synth.workload("llama8b_64k"))
+    assert all(dw.dwkv_page_bytes(cfg, k) < dw.dwkv_page_bytes(bf, k) for k in range(3))
 
 
 def test_create_rejects_bad_arguments_without_a_gpu():

@@ -3,7 +3,8 @@ one fused append + decode launch per layer of a group over all sequences, every 
 every layer of the group checked against the fp64 oracle (which encodes each step's new token
 itself).  Bars: max-abs <= 2e-3 and relative L2 <= 1e-3.
 
- * 64K: Llama-3-8B shapes, one sequence of 65536 tokens, int4 residual, r_max 64.
+ * 64K: Llama-3-8B shapes, one sequence of 65536 tokens, int4 residual, r_max 64; and the
+   same with 8-bit blockwise coefficients.
  * ragged batch: 8 sequences of 16K-32K tokens (seeded), int8 residual: the split-K
    apportionment across sequences of different lengths.
  * 131K deep: one sequence of 131072 tokens, 4-layer groups, r_max 128 with the full-rank
@@ -63,6 +64,11 @@ def _fused_group_step(wl, lengths, temp=8.0):
 
 def test_llama8b_64k_fused_step_every_head_both_layers():
     wl = synth.workload("llama8b_64k").scaled(num_layers=2)
+    assert _fused_group_step(wl, [wl.context]) == 2 * 8
+
+
+def test_llama8b_64k_8bit_coefficients_fused_step_every_head_both_layers():
+    wl = synth.workload("llama8b_64k_c8").scaled(num_layers=2)
     assert _fused_group_step(wl, [wl.context]) == 2 * 8
 
 
