@@ -192,7 +192,7 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
         float d[2][4];
         if constexpr (C8) {
             // per block of 16: the codes as exact f16 against q~ 2^E (f16 hi / lo), then the
-            // block's per-token scale (times 2^-E) on the two rows of the fragment
+            // block's per-token scale on the two rows of the fragment (2^-E once at the end)
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
                 d[mt][0] = d[mt][1] = d[mt][2] = d[mt][3] = 0.f;
@@ -206,13 +206,15 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                     float e[4] = {0.f, 0.f, 0.f, 0.f};
                     mma_f16(e, a, qb[b]);
                     const uint32_t sw = *reinterpret_cast<const uint32_t*>(K + kc8_scale_off(R, b, t0));
-                    const float s0 = __half2float(__ushort_as_half((unsigned short)(sw & 0xffffu))) * kexp;
-                    const float s1 = __half2float(__ushort_as_half((unsigned short)(sw >> 16))) * kexp;
+                    const float s0 = __half2float(__ushort_as_half((unsigned short)(sw & 0xffffu)));
+                    const float s1 = __half2float(__ushort_as_half((unsigned short)(sw >> 16)));
                     d[mt][0] = fmaf(s0, e[0], d[mt][0]);
                     d[mt][1] = fmaf(s0, e[1], d[mt][1]);
                     d[mt][2] = fmaf(s1, e[2], d[mt][2]);
                     d[mt][3] = fmaf(s1, e[3], d[mt][3]);
                 }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) d[mt][e] *= kexp;           // 2^-E: exact
             }
         } else {
 #pragma unroll
