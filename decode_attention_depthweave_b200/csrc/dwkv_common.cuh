@@ -197,7 +197,7 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 //   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  qh bf16 [d][4];  qb: q~ as MMA
 //           B fragments [ks][2][lane];  zero line
 //   bars    full[kSlots] empty[kSlots] basis table
-//   misc    tier table, page range, work counter; warp states; page-id batch; slot offsets
+//   misc    tier table, page range; warp states; page-id batch; slot offsets
 struct DecodeSmem {
     uint32_t ring, rd, small, small_stride, S, P, W, P2, CW, qt, q, qh, qb, zero, bars, misc, tok, total;
 };

@@ -24,8 +24,8 @@
 // tier-homogeneous; a page costs its bytes plus a per-token weight), visited from the highest
 // tier down.  The producer warp (lane 0) places the page chunks back to back in a byte ring
 // of shared memory with cp.async.bulk (no multicast); its 32 lanes resolve page ids a batch
-// ahead.  The 12 consumer warps take half pages (32 tokens) from a shared counter, each with
-// its own softmax state.  The CTA merges its warps' states into one partial record {M, L, o},
+// ahead.  The 12 consumer warps take the half pages (32 tokens) round robin, each with its
+// own softmax state.  The CTA merges its warps' states into one partial record {M, L, o},
 // and the last CTA of the (sequence, kv-head) (atomic ticket, no waiting) merges the records
 // and writes the output.
 #pragma once
@@ -838,7 +838,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
         if (lane == 0) {
             mbar_init(basis_bar, 1);
             mbar_init(table_bar, 1);
-            m_misc[3] = 0u;                   // half-page work counter
         }
         fence_mbar_init();
         __syncwarp();
@@ -1140,23 +1139,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             if (lane == 0) set_dev_error(St, 6u, (uint32_t)seq, 0xfffffffeu);
             ok = false;
         }
-        // Work items are half pages, taken in order from a shared counter: item w is half
-        // w & 1 of the CTA's page w >> 1.  Both halves of a page release its stage, so the
-        // stage frees once the second of the two warps is done, whichever warps they are.
+        // Work items are half pages, dealt round robin: warp w takes items w, w + 12, ...;
+        // item i is half i & 1 of the CTA's page i >> 1.  Both halves of a page release its
+        // stage, so the stage frees once the second of its two warps is done.  (A warp only
+        // waits for a page the producer will issue: the oldest unreleased page belongs to an
+        // item earlier in some warp's sequence than anything that warp waits for.)  Claims from
+        // a shared counter balanced the warps' finish no better and cost ~430 cycles an item.
         const uint32_t p_begin = m_misc[0], p_end = m_misc[1];
         const uint32_t nitems = 2 * (p_end - p_begin);
-        uint32_t* work = m_misc + 3;
-        uint32_t w = 0;
-        if (lane == 0) w = atomicAdd(work, 1u);
-        w = __shfl_sync(0xffffffffu, w, 0);
+        uint32_t w = (uint32_t)warp;
         while (ok && w < nitems) {
-            // take the next item now (its latency hides behind this one) unless the run is
-            // nearly over, where an early claim would only unbalance the warps' finish
-            uint32_t wn = 0xffffffffu;
-            if (w + 2 * kConsumerWarps < nitems) {
-                if (lane == 0) wn = atomicAdd(work, 1u);
-                wn = __shfl_sync(0xffffffffu, wn, 0);
-            }
+            const uint32_t wn = w + kConsumerWarps;
             const uint32_t u = w >> 1, p = p_end - 1 - u, sl = u % kSlots;
             const int half = (int)(w & 1);
             int k = 0;
@@ -1175,10 +1168,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
                                                qscale, small, rd, zero_addr, A, lane, G.ts[k], cw, kexp);
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8 * sl);
-            if (wn == 0xffffffffu) {
-                if (lane == 0) wn = atomicAdd(work, 1u);
-                wn = __shfl_sync(0xffffffffu, wn, 0);
-            }
             w = wn;
         }
         if constexpr (!PROBE) {
