@@ -251,7 +251,7 @@ struct dwkv_ctx {
     std::vector<int32_t> placed;    // [max_batch][G]
     int dec_ctas_per_sm = 1, dec_waves = 1, dec_stages_req = 0;
     int dec_tok_weight = 1024;      // split balance: byte-equivalent cost of one token
-    int dec_owner_share = 160;      // fused append: the encoding CTA's share of a split, of 256
+    int dec_owner_share = 112;      // fused append: the encoding CTA's share of a split, of 256
     int dec_overlap = 1;            // launch decodes with programmatic stream serialisation
     // The last launch on the handle when it was a fused decode step (else layer -1): a decode
     // launched right after it may start while it runs, and must not read early what it writes.

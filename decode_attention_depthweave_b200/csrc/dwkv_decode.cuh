@@ -672,9 +672,9 @@ __device__ __forceinline__ void owner_append(const Geom& G, const State& St, con
     __syncthreads();
 }
 
-// Consumer warp 0 of that CTA, after its pages: attend to the new token from its stored bytes
-// (the score over its coefficients and residual, the online-softmax update, and its value in
-// both spaces), so no other CTA waits for it.
+// One consumer warp of that CTA (the first to finish its pages), after its pages: attend to the
+// new token from its stored bytes (the score over its coefficients and residual, the
+// online-softmax update, and its value in both spaces), so no other CTA waits for it.
 template <int S, int BITS, int RMAX, bool C8>
 __device__ __forceinline__ void add_new_token(const Geom& G, const TokDest& td, const float4* qt, const float4* qs,
                                               WarpAcc<RMAX, false>& A, int lane) {
@@ -1171,7 +1171,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             w = wn;
         }
         if constexpr (!PROBE) {
-            if (owner && warp == 0 && tokd->ok)
+            // the warp whose last item comes first in the final round (item nitems - 12) is the
+            // first to finish: it attends to the new token
+            if (owner && warp == (int)(nitems % kConsumerWarps) && tokd->ok)
                 add_new_token<S, BITS, RMAX, C8>(G, *tokd, reinterpret_cast<const float4*>(smem + L.qt), qs, A, lane);
         }
         // ---- per-warp results: acc_c [r_max][4] and acc_r [d][4] into the residual tile,
