@@ -192,8 +192,8 @@ __host__ __device__ inline size_t slot_index(const Geom& G, int seq, int g, int 
 //   ring    page chunks, packed back to back (a chunk that does not fit before the end
 //           starts again at 0); ring_bytes is chosen by the host
 //   rd      per consumer warp, one 4 KB residual tile (also holds B_K during the prologue)
-//   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W limbs [8][48] u8, P2[32][8];
-//           with 8-bit coefficients two more limb tiles CW [8 or 16][48] u8 (ping-pong over blocks)
+//   small   per consumer warp: scores S[32][4] f32, P[32][8] bf16, W [4 heads][48] u16, P2[32][8];
+//           with 8-bit coefficients two more weight tiles CW [4 or 8][48] u16 (ping-pong over blocks)
 //   qt      q~ = B_K^T q, fp32 [r_max][4];  q  fp32 [d][4];  qh bf16 [d][4];  qb: q~ as MMA
 //           B fragments [ks][2][lane];  zero line
 //   bars    full[kSlots] empty[kSlots] basis table

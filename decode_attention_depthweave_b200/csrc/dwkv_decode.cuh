@@ -148,9 +148,22 @@ __device__ __forceinline__ void rescale_d(float (&d)[N][4], float a0, float a1) 
 __device__ __forceinline__ uint32_t rd_off(uint32_t row, uint32_t tok) {
     return (tok >> 4) * 2048u + row * 16u + (tok & 15u);
 }
-// Per-head byte rows of the weight limbs: row n = 2 h + limb, 32 tokens, 48-byte pitch (the
-// eight rows' 4-byte words read by one B-fragment load then fall in distinct banks).
-constexpr uint32_t kWbPitch = 48;
+// 16-bit fixed-point weights of a half page: one row of 32 tokens per head, 96-byte pitch.  A
+// token's weight is one 16-bit store; the integer MMA's B operand (column n = 2 h + limb, limb
+// 0 the high byte, 1 the low byte; k = token) is rebuilt from 8-byte loads by byte permutes.
+// With the 96-byte pitch the four heads' rows fall on distinct banks for both fragment loads.
+constexpr uint32_t kWhPitch = 96;
+__device__ __forceinline__ void store_w16(uint8_t* tile, int h, int lane, uint32_t v) {
+    *reinterpret_cast<uint16_t*>(tile + h * kWhPitch + 2 * lane) = (uint16_t)v;
+}
+__device__ __forceinline__ void load_wfrag(const uint8_t* tile, int g, int c, uint32_t (&b)[2]) {
+    const uint8_t* row = tile + (g >> 1) * kWhPitch + 8 * c;
+    const uint2 x0 = *reinterpret_cast<const uint2*>(row);          // tokens 4c .. 4c + 3
+    const uint2 x1 = *reinterpret_cast<const uint2*>(row + 32);     // tokens 16 + 4c ..
+    const uint32_t sel = (g & 1) ? 0x6420u : 0x7531u;               // low bytes : high bytes
+    b[0] = __byte_perm(x0.x, x0.y, sel);
+    b[1] = __byte_perm(x1.x, x1.y, sel);
+}
 
 // Rescale the 8-bit-coefficient accumulators: [i][0] row g, [i][1] row g + 8, both of head c.
 template <int N>
@@ -376,8 +389,7 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 const uint32_t eb = __reduce_max_sync(0xffffffffu, __float_as_uint(wv) >> 23);
                 uint32_t v = 0;
                 if (eb >= 16u) v = min(__float2uint_rn(wv * __uint_as_float((269u - eb) << 23)), 65535u);
-                Wsm[(2 * h) * kWbPitch + lane] = (uint8_t)(v >> 8);
-                Wsm[(2 * h + 1) * kWbPitch + lane] = (uint8_t)v;
+                store_w16(Wsm, h, lane, v);
                 if (c == h) wdq = eb >= 16u ? __uint_as_float((eb - 15u) << 23) : 0.f;   // 2^(E-15)
             }
             if (BITS == 4) wdq *= kCodeUnit4;
@@ -453,16 +465,14 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
                 const uint32_t eb = __reduce_max_sync(0xffffffffu, __float_as_uint(wv) >> 23);
                 uint32_t v = 0;
                 if (eb >= 16u) v = min(__float2uint_rn(wv * __uint_as_float((269u - eb) << 23)), 65535u);
-                tile[(2 * h) * kWbPitch + lane] = (uint8_t)(v >> 8);
-                tile[(2 * h + 1) * kWbPitch + lane] = (uint8_t)v;
+                store_w16(tile, h, lane, v);
                 if (c == h) wq = eb >= 16u ? __uint_as_float((eb - 15u) << 23) : 0.f;
                 if constexpr (PROBE) {
                     const float w2 = p2v[h] * svb[b];
                     const uint32_t e2 = __reduce_max_sync(0xffffffffu, __float_as_uint(w2) >> 23);
                     uint32_t v2 = 0;
                     if (e2 >= 16u) v2 = min(__float2uint_rn(w2 * __uint_as_float((269u - e2) << 23)), 65535u);
-                    tile[(8 + 2 * h) * kWbPitch + lane] = (uint8_t)(v2 >> 8);
-                    tile[(9 + 2 * h) * kWbPitch + lane] = (uint8_t)v2;
+                    store_w16(tile + 4 * kWhPitch, h, lane, v2);
                     if (c == h) wq2 = e2 >= 16u ? __uint_as_float((e2 - 15u) << 23) : 0.f;
                 }
             }
@@ -470,16 +480,16 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
             uint32_t a[4];
             ldsm_x4(vaddr + (uint32_t)b * 1024u + aoff, a);
             {
-                const uint32_t bb[2] = {*reinterpret_cast<const uint32_t*>(tile + g * kWbPitch + 4 * c),
-                                        *reinterpret_cast<const uint32_t*>(tile + g * kWbPitch + 16 + 4 * c)};
+                uint32_t bb[2];
+                load_wfrag(tile, g, c, bb);
                 int dd[4] = {0, 0, 0, 0};
                 mma_s8u8(dd, a, bb);
                 A.c[b][0] = fmaf(wq, (float)(dd[0] * 256 + dd[1]), A.c[b][0]);
                 A.c[b][1] = fmaf(wq, (float)(dd[2] * 256 + dd[3]), A.c[b][1]);
             }
             if constexpr (PROBE) {
-                const uint32_t bb[2] = {*reinterpret_cast<const uint32_t*>(tile + (8 + g) * kWbPitch + 4 * c),
-                                        *reinterpret_cast<const uint32_t*>(tile + (8 + g) * kWbPitch + 16 + 4 * c)};
+                uint32_t bb[2];
+                load_wfrag(tile + 4 * kWhPitch, g, c, bb);
                 int dd[4] = {0, 0, 0, 0};
                 mma_s8u8(dd, a, bb);
                 A.c2[b][0] = fmaf(wq2, (float)(dd[0] * 256 + dd[1]), A.c2[b][0]);
@@ -545,8 +555,7 @@ __device__ __forceinline__ void half_page(const uint8_t* __restrict__ K, int hal
         }
         __syncwarp();
         uint32_t b[2];
-        b[0] = *reinterpret_cast<const uint32_t*>(Wsm + g * kWbPitch + 4 * c);
-        b[1] = *reinterpret_cast<const uint32_t*>(Wsm + g * kWbPitch + 16 + 4 * c);
+        load_wfrag(Wsm, g, c, b);
         const uint32_t rdaddr = smem_addr(rd);
         const uint32_t arow = (uint32_t)(rr + 8 * (mi & 1));
 #pragma unroll
