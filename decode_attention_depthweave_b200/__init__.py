@@ -19,7 +19,7 @@ __all__ = [
     "DwkvError", "dwkv_config", "lib", "config_from", "dwkv_version", "dwkv_last_error",
     "dwkv_config_check", "dwkv_token_bytes", "dwkv_page_bytes", "dwkv_metadata_bytes",
     "dwkv_arena_bytes", "dwkv_workspace_bytes", "dwkv_create", "dwkv_destroy",
-    "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
+    "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_gated", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage",
     "dwkv_sync_status", "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
     "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
@@ -41,7 +41,7 @@ STATUS_NAMES = {0: "DWKV_OK", 1: "DWKV_ERR_INVALID_ARG", 2: "DWKV_ERR_CAPACITY",
 EXPORTED_SYMBOLS = (
     "dwkv_version", "dwkv_last_error", "dwkv_config_check", "dwkv_token_bytes", "dwkv_page_bytes",
     "dwkv_metadata_bytes", "dwkv_arena_bytes", "dwkv_workspace_bytes", "dwkv_create", "dwkv_destroy",
-    "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_compressed",
+    "dwkv_reset_sequence", "dwkv_seq_length", "dwkv_append", "dwkv_append_gated", "dwkv_append_compressed",
     "dwkv_decode_attention", "dwkv_probe", "dwkv_export", "dwkv_pool_usage", "dwkv_sync_status",
     "dwkv_set_decode_tuning", "dwkv_decode_attention_noalloc", "dwkv_append_decode_attention",
     "dwkv_quantize_work_bytes", "dwkv_quantize_residuals", "dwkv_check_bounded_wait", "dwkv_set_decode_overlap",
@@ -107,6 +107,7 @@ def lib():
             "dwkv_reset_sequence": ([vp, i32, vp], C.c_int),
             "dwkv_seq_length": ([vp, i32, i32, C.POINTER(i32)], C.c_int),
             "dwkv_append": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp], C.c_int),
+            "dwkv_append_gated": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], C.c_int),
             "dwkv_append_compressed": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], C.c_int),
             "dwkv_decode_attention": ([vp, i32, i32, vp, vp, vp, vp, sz, vp], C.c_int),
             "dwkv_append_decode_attention": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
@@ -252,6 +253,11 @@ def dwkv_seq_length(h, seq, layer) -> int:
 def dwkv_append(h, layer, seq_ids, n_new, k_new, v_new, tier_idx, coeff_dbg=None, stream=None):
     _check(lib().dwkv_append(h, layer, len(seq_ids), _i32(seq_ids), _i32(n_new), _ptr(k_new), _ptr(v_new),
                              _ptr(tier_idx), _ptr(coeff_dbg), _stream(stream)))
+
+
+def dwkv_append_gated(h, layer, seq_ids, n_new, k_new, v_new, tier_idx, gate, coeff_dbg=None, stream=None):
+    _check(lib().dwkv_append_gated(h, layer, len(seq_ids), _i32(seq_ids), _i32(n_new), _ptr(k_new), _ptr(v_new),
+                                   _ptr(tier_idx), _ptr(gate), _ptr(coeff_dbg), _stream(stream)))
 
 
 def dwkv_append_compressed(h, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream=None):
@@ -430,8 +436,12 @@ class Cache:
         except Exception:
             pass
 
-    def append(self, layer, seq_ids, n_new, k_new, v_new, tier_idx, stream=None, coeff_dbg=None):
-        dwkv_append(self.h, layer, seq_ids, n_new, k_new, v_new, tier_idx, coeff_dbg, stream)
+    def append(self, layer, seq_ids, n_new, k_new, v_new, tier_idx, stream=None, coeff_dbg=None, gate=None):
+        """gate: optional fp32 [sum(n_new)][Hkv][2] residual gates (dwkv_append_gated)."""
+        if gate is not None:
+            dwkv_append_gated(self.h, layer, seq_ids, n_new, k_new, v_new, tier_idx, gate, coeff_dbg, stream)
+        else:
+            dwkv_append(self.h, layer, seq_ids, n_new, k_new, v_new, tier_idx, coeff_dbg, stream)
 
     def append_compressed(self, layer, seq_ids, n_new, tier_idx, coeff, idx, codes, scales, stream=None):
         """coeff: bf16 [n][Hkv][2][r_max], or with 8-bit coefficients the pair (codes int8

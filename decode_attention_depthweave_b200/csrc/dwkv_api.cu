@@ -753,9 +753,9 @@ dwkv_status dwkv_reset_sequence(dwkv_handle h, int32_t seq, void* stream) {
     return DWKV_OK;
 }
 
-dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const int32_t* n_new,
-                        const void* k_new, const void* v_new, const uint8_t* tier_idx, float* coeff_dbg,
-                        void* stream) {
+static dwkv_status append_impl(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                               const int32_t* n_new, const void* k_new, const void* v_new,
+                               const uint8_t* tier_idx, const float* gate, float* coeff_dbg, void* stream) {
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
     AppendCall C;
@@ -764,6 +764,8 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
     if (!k_new || !v_new) return fail(DWKV_ERR_INVALID_ARG, "k_new and v_new must be non-NULL");
     if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15u)
         return fail(DWKV_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(gate) & 3u) return fail(DWKV_ERR_INVALID_ARG, "gate must be 4-byte aligned");
+    C.gate = gate;
     const Geom& G = h->geom;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     bool any = false;
@@ -809,6 +811,19 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
     note_plain_launch(h);
     commit_call(h, C, n_new);
     return DWKV_OK;
+}
+
+dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids, const int32_t* n_new,
+                        const void* k_new, const void* v_new, const uint8_t* tier_idx, float* coeff_dbg,
+                        void* stream) {
+    return append_impl(h, layer, n_seqs, seq_ids, n_new, k_new, v_new, tier_idx, nullptr, coeff_dbg, stream);
+}
+
+dwkv_status dwkv_append_gated(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                              const int32_t* n_new, const void* k_new, const void* v_new, const uint8_t* tier_idx,
+                              const float* gate, float* coeff_dbg, void* stream) {
+    if (!gate) return fail(DWKV_ERR_INVALID_ARG, "gate is NULL (use dwkv_append)");
+    return append_impl(h, layer, n_seqs, seq_ids, n_new, k_new, v_new, tier_idx, gate, coeff_dbg, stream);
 }
 
 dwkv_status dwkv_append_compressed(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,

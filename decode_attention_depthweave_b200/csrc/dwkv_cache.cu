@@ -172,6 +172,7 @@ __device__ __forceinline__ UnitIn encode_fetch(const Geom& G, const State& S, co
     for (int m = 0; m < 4; ++m) in.xr[m] = __bfloat162float(src[lane + 32 * m]);
     in.ok = find_dest(G, S, seq, C.g, C.lig, h, pos, in.dst);
     in.dbg = coeff_dbg ? coeff_dbg + (((size_t)row * G.Hkv + h) * 2 + z) * G.r_max : nullptr;
+    in.gate = C.gate ? C.gate[((size_t)row * G.Hkv + h) * 2 + z] : 1.f;
     // a0..a0+na were placed by the placement; a zero entry means placement failed (already
     // reported) or the group never placed this position
     if (!in.ok && lane == 0 && z == 0 && !(pos >= C.a0[ci] && pos < C.a0[ci] + C.na[ci]))
@@ -438,7 +439,8 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(const Geom G, const Stat
                 const int sl = s0 + t;
                 if (sl >= nvalid) break;
                 const float r4[4] = {a[t][0], a[t][1], a[t][2], a[t][3]};
-                quantize_store<BITS>(r4, sblk[sl], sR[sl], sprow[sl] & 0xff, G.ts[sprow[sl] >> 8], rstage, chstage, G.c8);
+                quantize_store<BITS>(r4, sblk[sl], sR[sl], sprow[sl] & 0xff, G.ts[sprow[sl] >> 8], rstage, chstage, G.c8,
+                                     C.gate ? C.gate[((size_t)srow[sl] * G.Hkv + h) * 2 + z] : 1.f);
             }
         }
     }

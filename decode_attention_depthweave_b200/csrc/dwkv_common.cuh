@@ -85,6 +85,7 @@ struct AppendCall {
     int tok0[kMaxSeqs + 1];  // prefix of n_new: first input row of each sequence
     int a0[kMaxSeqs];        // first position that needs a slot (group's first placement)
     int na[kMaxSeqs];        // positions that need a slot
+    const float* gate;       // nullable: residual gate g [total][Hkv][2], folded into the stored scale
 };
 
 // One round of a re-tier call: for each listed sequence, the tokens [begin, end) of the call's

@@ -10,6 +10,8 @@
 //   4. the s largest |r_i|, ties to the lower channel, stored in ascending channel order
 //   5. scale = fp16_rn(max |r_sel| / qmax) with IEEE division, qmax = 127 (int8) / 7 (int4)
 //   6. code  = clamp(rint(r / float(scale)), -qmax, qmax), all zero when scale == 0
+//      With a residual gate g (Eq. (1)'s g R, folded into the dequantisation): the stored
+//      scale is fp16_rn(g * float(scale)) (an fp32 product); the codes are those of step 6.
 // With 8-bit coefficients (the blockwise form kept by the pages), step 2 becomes, per block of
 // 16 coefficients: sc = fp16_rn(max |c| / 127) (IEEE division), q_j = clamp(rint(c_j /
 // float(sc)), -127, 127) (0 when sc == 0), cb_j = q_j float(sc) (exact); steps 3-6 as above.
@@ -139,6 +141,7 @@ struct UnitIn {
     float xr[4];
     bool ok;
     float* dbg = nullptr;   // the unit's fp32 projection c[j], j < r_t (coefficient export), or none
+    float gate = 1.f;       // residual gate folded into the stored scale
 };
 
 // Step 4 by its definition: s rounds of "largest remaining |r|, ties to the lower channel"
@@ -176,7 +179,7 @@ static __device__ __noinline__ uint32_t select_exact(float r0, float r1, float r
 // exact zeros) the selection is redone by its definition (select_exact).
 template <int BITS>
 __device__ __forceinline__ void quantize_store(const float (&r)[4], uint8_t* blk, int R, int row, int s,
-                                               float* rstage, uint8_t* chstage, int c8) {
+                                               float* rstage, uint8_t* chstage, int c8, float gate = 1.f) {
     const int lane = threadIdx.x & 31;
     const float qmax = BITS == 8 ? 127.f : 7.f;
     uint32_t sel = 0u, mxb = 0u;
@@ -233,7 +236,9 @@ __device__ __forceinline__ void quantize_store(const float (&r)[4], uint8_t* blk
         }
         before += __popc(bal);
     }
-    if (lane == 0) *reinterpret_cast<__half*>(blk + off_scales_of(R, s, BITS, c8) + row * 2) = sh;
+    if (lane == 0)
+        *reinterpret_cast<__half*>(blk + off_scales_of(R, s, BITS, c8) + row * 2) =
+            gate == 1.f ? sh : __float2half_rn(__fmul_rn(gate, sf));
     __syncwarp();
     for (int b0 = 0; b0 < s; b0 += 32) {
         const int b = b0 + lane;
@@ -346,7 +351,7 @@ __device__ __forceinline__ void encode_body(const Geom& G, const State& S, const
 #pragma unroll
             for (int m = 0; m < 4; ++m) r[m] = __fsub_rn(xr[m], a[m]);
         }
-        quantize_store<BITS>(r, blk, R, dst.row, G.ts[dst.k], xs, reinterpret_cast<uint8_t*>(cstage), G.c8);
+        quantize_store<BITS>(r, blk, R, dst.row, G.ts[dst.k], xs, reinterpret_cast<uint8_t*>(cstage), G.c8, in.gate);
     } while (false);
     __syncwarp();
 }

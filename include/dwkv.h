@@ -246,6 +246,17 @@ dwkv_status dwkv_append(dwkv_handle h, int32_t layer, int32_t n_seqs, const int3
                         const int32_t* n_new, const void* k_new, const void* v_new,
                         const uint8_t* tier_idx, float* coeff_dbg, void* stream);
 
+/* dwkv_append with the residual gate of [DW] §3 Eq. (1) (X^ = A B + g R, g in [0, 1]) folded
+ * into the dequantisation: the token's residual is quantised as in dwkv_append and its stored
+ * fp16 scale is fp16_rn(g * scale) (an fp32 product), so decode and probe reconstruct g R.
+ *   gate : device fp32 [sum(n_new)][Hkv][2] (K at [..][0], V at [..][1]), 4-byte aligned,
+ *          non-NULL; values are used as given.
+ * The fused decode step (dwkv_append_decode_attention) appends with g = 1; a re-tiered or
+ * re-projected token is re-encoded from its reconstruction (which includes g R) with g = 1. */
+dwkv_status dwkv_append_gated(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                              const int32_t* n_new, const void* k_new, const void* v_new,
+                              const uint8_t* tier_idx, const float* gate, float* coeff_dbg, void* stream);
+
 /* Appends tokens that are already in compressed form (import of a prepared cache).
  * Same sequence / position rules as dwkv_append.  Device arrays, tokens in list order,
  * K at [..][0][..] and V at [..][1][..]:

@@ -49,6 +49,8 @@ def lib():
         L.oracle_reencode_vector.restype = i
         L.oracle_reconstruct.argtypes = [i, i, p, i, p, i, p, p, C.c_uint16, i, p]
         L.oracle_reconstruct.restype = None
+        L.oracle_gate_scales.argtypes = [C.c_int64, p, p, p]
+        L.oracle_gate_scales.restype = None
         L.oracle_quantize_coeffs8.argtypes = [i, i, p, p, p, p]
         L.oracle_quantize_coeffs8.restype = i
         L.oracle_encode_vector8.argtypes = [i, i, p, p, p, i, i, i, p, p, p, p, p, p]
@@ -443,4 +445,15 @@ def encode_many8(basis, x, ranks, s, bits, c32=None, nthreads=None, nres=None, w
     out = {"ccodes": cc, "cscales": cs, "idx": idx, "codes": codes, "scale": scale}
     if want_c32:
         out["c32"] = co
+    return out
+
+
+# ----------------------------------------------------------------------------- residual gate
+def gate_scales(scales, gates) -> np.ndarray:
+    """Stored residual scales with the gate folded in: fp16_rn(g * scale) elementwise (fp16
+    bits in, fp16 bits out; ``oracle_gate_scale``)."""
+    sc = _bits16(scales)
+    g = _arr(gates, np.float32).reshape(sc.shape)
+    out = np.empty(sc.shape, np.uint16)
+    lib().oracle_gate_scales(sc.size, _p(sc), _p(g), _p(out))
     return out

@@ -12,7 +12,8 @@
  *   [DW] §3 Method, Eq. (3):  e_{l,h} = ||Attn(Q,K,V) - Attn(Q,K^,V^)||_2 / (||Attn(Q,K,V)||_2 + eps)
  *
  * Readings taken where [DW] is silent (each one is listed in the design notes):
- *   - g = 1 (no trained gates exist).  The basis is stored transposed, d x r_max with
+ *   - g = 1 by default (no trained gates exist); a given gate g folds into the stored
+ *     residual scale, fp16_rn(g * scale).  The basis is stored transposed, d x r_max with
  *     columns as basis vectors, so A B becomes sum_{j<r_t} B[:, j] c_t[j].
  *   - The router's rank r_t truncates the coefficient vector; the residual keeps a fixed
  *     number s of channels: R = scale_t * sum_i code_{t,i} e_{idx_{t,i}}.
@@ -321,6 +322,17 @@ int oracle_encode_from_coeffs(int d, int r_max, const uint16_t* basis, const uin
     }
     oracle_quantize_residual(d, s, bits, r, idx, codes, scale);
     return 0;
+}
+
+/* The residual gate g of [DW] §3 Eq. (1) (X^ = A B + g R) folded into the dequantisation:   */
+/* the token's stored residual scale becomes fp16_rn(g * float(scale)), an fp32 product;      */
+/* the codes stay those of step 6.                                                           */
+uint16_t oracle_gate_scale(uint16_t scale, float g) {
+    return oracle_f32_to_fp16_rn(g * (float)oracle_fp16_to_f64(scale));
+}
+
+void oracle_gate_scales(int64_t n, const uint16_t* scale, const float* g, uint16_t* out) {
+    for (int64_t k = 0; k < n; ++k) out[k] = oracle_gate_scale(scale[k], g[k]);
 }
 
 /* ------------------------------------------------------------------------------------ */

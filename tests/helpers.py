@@ -117,7 +117,7 @@ def check_close(got, ref, max_abs=2e-3, rel=1e-3, what=""):
     return ma, rl
 
 
-def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None, c32=None) -> dict:
+def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None, c32=None, gate=None) -> dict:
     """The oracle's encoding of dense rows k, v (bf16 [n][Hkv][d]) at their tiers, in the
     token-ordered compressed format of ``synth.make_compressed`` (CPU tensors).  With ``c32``
     (fp32 [n][Hkv][2][r_max], an encoder's exported projection) the oracle runs encode steps
@@ -152,6 +152,8 @@ def oracle_encode_rows(wl, bases, layer, k, v, tier_idx, nthreads=None, c32=None
             if not c8:
                 coeff[:, h, z] = r["coeff"]
             idx[:, h, z], codes[:, h, z], scales[:, h, z] = r["idx"], r["codes"], r["scale"]
+            if gate is not None:                    # the residual gate folded into the scale
+                scales[:, h, z] = oracle.gate_scales(scales[:, h, z], np.asarray(gate.cpu())[:, h, z])
     out = {"idx": torch.from_numpy(idx), "codes": torch.from_numpy(codes),
            "scales": torch.from_numpy(scales.view(np.int16)).view(torch.float16)}
     if c8:
