@@ -94,11 +94,14 @@ __global__ void __launch_bounds__(256) moment_scale_kernel(float* c, size_t n, f
 // ------------------------------------------------------------------------------------
 // The basis of one (kv-head, K / V) of a window from its second moment: one block of 512
 // threads, fp64 in shared memory (r_max <= 64).  omega (fp32 [d][r_max]) starts a sketch;
-// without it the current basis starts one refresh step.
+// without it the current basis starts one refresh step.  The [.][r] arrays have a row pitch
+// of r + 1 doubles, so the column walks (Gram-Schmidt's dot products, the Jacobi rotations of
+// columns) step across banks instead of hitting one.
 // ------------------------------------------------------------------------------------
 constexpr int kBasisThreads = 512;
 size_t basis_smem_bytes(int r) {
-    return (size_t)2 * kD * r * 8 + (size_t)r * r * 8 + (size_t)(kD + 2 * r + 32) * 8;
+    const size_t rp = (size_t)r + 1;
+    return (2 * kD * rp + (size_t)r * rp + kD + 2 * (size_t)r + 32) * 8;
 }
 
 // Block-wide sum of one double per thread (kBasisThreads threads); every thread gets it.
@@ -114,44 +117,44 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
     return s;
 }
 
-// W = C Q: C fp32 [d][d] (global), Q, W fp64 [d][r] (shared).
-__device__ void moment_times(const float* __restrict__ cm, const double* q, double* w, int r) {
+// W = C Q: C fp32 [d][d] (global), Q, W fp64 [d][r] with row pitch rp (shared).
+__device__ void moment_times(const float* __restrict__ cm, const double* q, double* w, int r, int rp) {
     for (int e = threadIdx.x; e < kD * r; e += blockDim.x) {
         const int i = e / r, j = e % r;
         double a = 0.0;
-        for (int k = 0; k < kD; ++k) a = fma((double)__ldg(cm + (size_t)i * kD + k), q[k * r + j], a);
-        w[e] = a;
+        for (int k = 0; k < kD; ++k) a = fma((double)__ldg(cm + (size_t)i * kD + k), q[k * rp + j], a);
+        w[i * rp + j] = a;
     }
     __syncthreads();
 }
 
-// Gram-Schmidt of the columns of q [d][r] in order, in place, each column orthogonalised
-// twice against the previous ones (classical Gram-Schmidt, twice: orthogonal to rounding for
-// any conditioning).  Returns false if a column vanishes.
-__device__ bool orthonormalize(double* q, int r, double* dots, double* red) {
+// Gram-Schmidt of the columns of q [d][r] (row pitch rp) in order, in place, each column
+// orthogonalised twice against the previous ones (classical Gram-Schmidt, twice: orthogonal
+// to rounding for any conditioning).  Returns false if a column vanishes.
+__device__ bool orthonormalize(double* q, int r, int rp, double* dots, double* red) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int j = 0; j < r; ++j) {
         for (int pass = 0; pass < 2; ++pass) {
             // dots[i] = q[:, i] . q[:, j] for i < j: a warp per i
             for (int i = warp; i < j; i += kBasisThreads / 32) {
                 double a = 0.0;
-                for (int row = lane; row < kD; row += 32) a = fma(q[row * r + i], q[row * r + j], a);
+                for (int row = lane; row < kD; row += 32) a = fma(q[row * rp + i], q[row * rp + j], a);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
                 if (lane == 0) dots[i] = a;
             }
             __syncthreads();
             if (tid < kD) {
-                double v = q[tid * r + j];
-                for (int i = 0; i < j; ++i) v = fma(-dots[i], q[tid * r + i], v);
-                q[tid * r + j] = v;
+                double v = q[tid * rp + j];
+                for (int i = 0; i < j; ++i) v = fma(-dots[i], q[tid * rp + i], v);
+                q[tid * rp + j] = v;
             }
             __syncthreads();
         }
-        const double x = tid < kD ? q[tid * r + j] : 0.0;
+        const double x = tid < kD ? q[tid * rp + j] : 0.0;
         const double n2 = block_sum(x * x, red);
         if (!(n2 > 0.0)) return false;
-        if (tid < kD) q[tid * r + j] = x / sqrt(n2);
+        if (tid < kD) q[tid * rp + j] = x / sqrt(n2);
         __syncthreads();
     }
     return true;
@@ -162,15 +165,15 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
                                                               const float* __restrict__ omega, int power_steps,
                                                               float* __restrict__ eig_out) {
     extern __shared__ __align__(16) uint8_t smem[];
-    const int r = G.r_max;
+    const int r = G.r_max, rp = r + 1;
     const int h = blockIdx.x >> 1, z = blockIdx.x & 1;
     g += blockIdx.y;                                        // all-windows launches: one row of blocks a window
     moment += (size_t)blockIdx.y * G.Hkv * 2 * kD * kD;
     const int tid = threadIdx.x;
-    double* q = reinterpret_cast<double*>(smem);            // [d][r]
-    double* w = q + kD * r;                                 // [d][r]; later U [r][r]
-    double* t = w + kD * r;                                 // [r][r]
-    double* dots = t + r * r;                               // [kD]
+    double* q = reinterpret_cast<double*>(smem);            // [d][rp]
+    double* w = q + kD * rp;                                // [d][rp]; later U [r][rp]
+    double* t = w + kD * rp;                                // [r][rp]
+    double* dots = t + r * rp;                              // [kD]
     double* lam = dots + kD;                                // [r]
     int* order = reinterpret_cast<int*>(lam + r);           // [2r]: Jacobi pairs, then ranks
     double* red = lam + 2 * r;                              // [16]
@@ -180,45 +183,47 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
 
     // ---- start: Y = C Omega, or C B_old
     for (int e = tid; e < kD * r; e += blockDim.x)
-        w[e] = omega ? (double)omega[e] : (double)__bfloat162float(bz[e]);
+        w[(e / r) * rp + e % r] = omega ? (double)omega[e] : (double)__bfloat162float(bz[e]);
     __syncthreads();
-    moment_times(cm, w, q, r);
-    bool ok = orthonormalize(q, r, dots, red);
+    moment_times(cm, w, q, r, rp);
+    bool ok = orthonormalize(q, r, rp, dots, red);
     for (int it = 0; ok && omega && it < power_steps; ++it) {
-        moment_times(cm, q, w, r);
-        for (int e = tid; e < kD * r; e += blockDim.x) q[e] = w[e];
+        moment_times(cm, q, w, r, rp);
+        for (int e = tid; e < kD * r; e += blockDim.x) q[(e / r) * rp + e % r] = w[(e / r) * rp + e % r];
         __syncthreads();
-        ok = orthonormalize(q, r, dots, red);
+        ok = orthonormalize(q, r, rp, dots, red);
     }
     if (!ok) {
         if (tid == 0) set_dev_error(S, 8u /*DWKV_DEV_BASIS*/, (uint32_t)g, (uint32_t)blockIdx.x);
         return;                                            // the basis stays as it was
     }
     // ---- Rayleigh-Ritz: T = Q^T (C Q), symmetric; U = I
-    moment_times(cm, q, w, r);
+    moment_times(cm, q, w, r, rp);
     for (int e = tid; e < r * r; e += blockDim.x) {
         const int a = e / r, b = e % r;
         double s = 0.0;
-        for (int i = 0; i < kD; ++i) s = fma(q[i * r + a], w[i * r + b], s);
-        t[e] = s;
+        for (int i = 0; i < kD; ++i) s = fma(q[i * rp + a], w[i * rp + b], s);
+        t[a * rp + b] = s;
     }
     __syncthreads();
     for (int e = tid; e < r * r; e += blockDim.x) {
         const int a = e / r, b = e % r;
-        if (a < b) { const double m = 0.5 * (t[a * r + b] + t[b * r + a]); t[a * r + b] = m; t[b * r + a] = m; }
+        if (a < b) { const double m = 0.5 * (t[a * rp + b] + t[b * rp + a]); t[a * rp + b] = m; t[b * rp + a] = m; }
     }
-    double* u = w;                                          // [r][r]
-    for (int e = tid; e < r * r; e += blockDim.x) u[e] = (e / r == e % r) ? 1.0 : 0.0;
+    double* u = w;                                          // [r][rp]
+    for (int e = tid; e < r * r; e += blockDim.x) u[(e / r) * rp + e % r] = (e / r == e % r) ? 1.0 : 0.0;
     __syncthreads();
     // ---- cyclic Jacobi, round-robin pairs (circle method): r / 2 disjoint rotations a round
     double* cs = dots;                                      // [r/2] c, then [r/2] s
     int* pq = order;                                        // [r/2] p, [r/2] q
     const int np = r / 2;
     for (int sweep = 0; sweep < 20; ++sweep) {
-        double off = 0.0;
-        for (int e = tid; e < r * r; e += blockDim.x) if (e / r != e % r) off += t[e] * t[e];
-        double fro = 0.0;
-        for (int e = tid; e < r * r; e += blockDim.x) fro += t[e] * t[e];
+        double off = 0.0, fro = 0.0;
+        for (int e = tid; e < r * r; e += blockDim.x) {
+            const double x = t[(e / r) * rp + e % r];
+            fro += x * x;
+            if (e / r != e % r) off += x * x;
+        }
         off = block_sum(off, red);
         fro = block_sum(fro, red);
         if (!(off > 1e-28 * fro)) break;
@@ -228,43 +233,43 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
                 if (tid == 0) { p = rd; qq = r - 1; }
                 else { p = (rd + tid) % (r - 1); qq = (rd - tid + (r - 1)) % (r - 1); }
                 if (p > qq) { const int x = p; p = qq; qq = x; }
-                const double apq = t[p * r + qq], app = t[p * r + p], aqq = t[qq * r + qq];
-                double c = 1.0, s = 0.0;
+                const double apq = t[p * rp + qq], app = t[p * rp + p], aqq = t[qq * rp + qq];
+                double c = 1.0, sn = 0.0;
                 if (apq != 0.0) {
                     const double tau = (aqq - app) / (2.0 * apq);
                     const double tt = tau >= 0.0 ? 1.0 / (tau + sqrt(1.0 + tau * tau)) : -1.0 / (-tau + sqrt(1.0 + tau * tau));
                     c = 1.0 / sqrt(1.0 + tt * tt);
-                    s = tt * c;
+                    sn = tt * c;
                 }
                 cs[tid] = c;
-                cs[np + tid] = s;
+                cs[np + tid] = sn;
                 pq[tid] = p;
                 pq[np + tid] = qq;
             }
             __syncthreads();
             for (int e = tid; e < np * r; e += blockDim.x) {    // rows p, q of T: J^T T
                 const int k = e / r, m = e % r, p = pq[k], qq = pq[np + k];
-                const double c = cs[k], s = cs[np + k];
-                const double xp = t[p * r + m], xq = t[qq * r + m];
-                t[p * r + m] = c * xp - s * xq;
-                t[qq * r + m] = s * xp + c * xq;
+                const double c = cs[k], sn = cs[np + k];
+                const double xp = t[p * rp + m], xq = t[qq * rp + m];
+                t[p * rp + m] = c * xp - sn * xq;
+                t[qq * rp + m] = sn * xp + c * xq;
             }
             __syncthreads();
             for (int e = tid; e < np * r; e += blockDim.x) {    // columns p, q of T and U: (.) J
                 const int k = e / r, m = e % r, p = pq[k], qq = pq[np + k];
-                const double c = cs[k], s = cs[np + k];
-                const double xp = t[m * r + p], xq = t[m * r + qq];
-                t[m * r + p] = c * xp - s * xq;
-                t[m * r + qq] = s * xp + c * xq;
-                const double up = u[m * r + p], uq = u[m * r + qq];
-                u[m * r + p] = c * up - s * uq;
-                u[m * r + qq] = s * up + c * uq;
+                const double c = cs[k], sn = cs[np + k];
+                const double xp = t[m * rp + p], xq = t[m * rp + qq];
+                t[m * rp + p] = c * xp - sn * xq;
+                t[m * rp + qq] = sn * xp + c * xq;
+                const double up = u[m * rp + p], uq = u[m * rp + qq];
+                u[m * rp + p] = c * up - sn * uq;
+                u[m * rp + qq] = sn * up + c * uq;
             }
             __syncthreads();
         }
     }
     // ---- eigenvalues in descending order (ties to the lower index), B = Q U, signs, bf16
-    if (tid < r) lam[tid] = t[tid * r + tid];
+    if (tid < r) lam[tid] = t[tid * rp + tid];
     __syncthreads();
     int* ord = order;                                       // ord[rank] = source column
     if (tid < r) {
@@ -280,13 +285,13 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
         for (int i = warp; i < kD; i += kBasisThreads / 32) {
             double a0 = 0.0, a1 = 0.0;
             for (int j = 0; j < r; ++j) {
-                const double qv = q[i * r + j];
-                a0 = fma(qv, u[j * r + s0], a0);
-                a1 = fma(qv, u[j * r + s1], a1);
+                const double qv = q[i * rp + j];
+                a0 = fma(qv, u[j * rp + s0], a0);
+                a1 = fma(qv, u[j * rp + s1], a1);
             }
             __syncwarp();                                   // every lane has read row i of Q
-            if (o0 < r) q[i * r + o0] = a0;
-            if (o1 < r) q[i * r + o1] = a1;
+            if (o0 < r) q[i * rp + o0] = a0;
+            if (o1 < r) q[i * rp + o1] = a1;
         }
         __syncthreads();
     }
@@ -295,17 +300,17 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
         int best = 0;
         double bm = -1.0;
         for (int i = 0; i < kD; ++i) {
-            const double m = fabs(q[i * r + tid]);
+            const double m = fabs(q[i * rp + tid]);
             if (m > bm) { bm = m; best = i; }
         }
-        dots[tid] = q[best * r + tid] < 0.0 ? -1.0 : 1.0;
+        dots[tid] = q[best * rp + tid] < 0.0 ? -1.0 : 1.0;
         if (eig_out) eig_out[(((size_t)blockIdx.y * G.Hkv + h) * 2 + z) * r + tid] = (float)lam[ord[tid]];
     }
     __syncthreads();
     __nv_bfloat16* tk = const_cast<__nv_bfloat16*>(S.basis_kt) + boff;
     for (int e = tid; e < kD * r; e += blockDim.x) {
         const int i = e / r, o = e % r;
-        const __nv_bfloat16 v = __float2bfloat16_rn((float)(dots[o] * q[e]));
+        const __nv_bfloat16 v = __float2bfloat16_rn((float)(dots[o] * q[i * rp + o]));
         bz[e] = v;
         if (z == 0) tk[tiled_basis_off(i, o, r)] = v;
     }
