@@ -361,32 +361,43 @@ __global__ void __launch_bounds__(256) reproject_kernel(const Geom G, const Stat
         const int R = G.tiers[k], st = G.ts[k], row = (int)(slot % kPage);
         const uint32_t unit = S.pages[page_index(G, seq, g, h, k) + slot / kPage];
         uint8_t* blk = S.data + (size_t)unit * kUnit + (size_t)lig * G.chunk_bytes[k] + (z ? G.blk_bytes[k] : 0u);
-        // reconstruction on the previous basis (fixed fp32 order), rounded to bf16
+        // reconstruction on the previous basis (fixed fp32 order), rounded to bf16.  The
+        // token's coefficients and residual entries are read in parallel (lane j holds entry j
+        // and j + 32) and handed round by shuffles: the chain's order is unchanged.
         const __nv_bfloat16* bz = bo + (size_t)z * kD * P;
+        auto coeff_at = [&](int j) {
+            return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(blk + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2));
+        };
+        const float cl0 = lane < R ? coeff_at(lane) : 0.f, cl1 = lane + 32 < R ? coeff_at(lane + 32) : 0.f;
+        int ch_l = 0;
+        float v_l = 0.f;
+        if (st > 0 && lane < st) {
+            const float sf = __half2float(*reinterpret_cast<const __half*>(blk + off_scales_of(R, st, BITS) + row * 2));
+            const int e = lane;
+            ch_l = blk[off_idx_of(R) + row * st + e];
+            int code;
+            if (BITS == 8) {
+                code = (int8_t)blk[off_codes_of(R, st) + row * st + e];
+            } else {
+                const uint32_t byte = blk[off_codes_of(R, st) + row * (st / 2) + (e >> 1)];
+                code = (int)(((e & 1) ? byte >> 4 : byte) & 0xfu);
+                code = (code ^ 8) - 8;
+            }
+            v_l = __fmul_rn(sf, (float)code);                     // exact: 11 x 7 significant bits
+        }
         float a[4] = {0.f, 0.f, 0.f, 0.f};
         for (int j = 0; j < R; ++j) {
-            const float cj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(blk + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2));
+            const float cj = __shfl_sync(0xffffffffu, j < 32 ? cl0 : cl1, j & 31);
 #pragma unroll
             for (int m = 0; m < 4; ++m) a[m] = __fmaf_rn(__bfloat162float(bz[(size_t)(lane + 32 * m) * P + j]), cj, a[m]);
         }
-        if (st > 0) {
-            const float sf = __half2float(*reinterpret_cast<const __half*>(blk + off_scales_of(R, st, BITS) + row * 2));
-            for (int e = 0; e < st; ++e) {
-                const int ch = blk[off_idx_of(R) + row * st + e];
-                int code;
-                if (BITS == 8) {
-                    code = (int8_t)blk[off_codes_of(R, st) + row * st + e];
-                } else {
-                    const uint32_t byte = blk[off_codes_of(R, st) + row * (st / 2) + (e >> 1)];
-                    code = (int)(((e & 1) ? byte >> 4 : byte) & 0xfu);
-                    code = (code ^ 8) - 8;
-                }
-                if ((ch & 31) == lane && ch < kD) {
-                    const float v = __fmul_rn(sf, (float)code);           // exact: 11 x 7 significant bits
+        for (int e = 0; e < st; ++e) {
+            const int ch = __shfl_sync(0xffffffffu, ch_l, e);
+            const float v = __shfl_sync(0xffffffffu, v_l, e);
+            if ((ch & 31) == lane && ch < kD) {
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        if ((ch >> 5) == m) a[m] = __fadd_rn(a[m], v);
-                }
+                for (int m = 0; m < 4; ++m)
+                    if ((ch >> 5) == m) a[m] = __fadd_rn(a[m], v);
             }
         }
         __syncwarp();                                        // every lane has read the old bytes
