@@ -251,7 +251,7 @@ struct dwkv_ctx {
     std::vector<int32_t> placed;    // [max_batch][G]
     int dec_ctas_per_sm = 1, dec_waves = 1, dec_stages_req = 0;
     int dec_tok_weight = 1024;      // split balance: byte-equivalent cost of one token
-    int dec_owner_share = 112;      // fused append: the encoding CTA's share of a split, of 256
+    uint32_t dec_owner_cost = 2500000;  // fused append: the encoding CTA's extra work, in split cost units
     int dec_overlap = 1;            // launch decodes with programmatic stream serialisation
     // The last launch on the handle when it was a fused decode step (else layer -1): a decode
     // launched right after it may start while it runs, and must not read early what it writes.
@@ -987,10 +987,10 @@ static dwkv_status run_decode(dwkv_handle h, int32_t layer, int32_t n_seqs, cons
     C.ring_bytes = (int)ring;
     C.rec_floats = rec_floats_of(G, probe);
     C.tok_weight = h->dec_tok_weight;
-    C.owner_share = 256;
+    C.owner_cost = 0;
     if (fa) {
         C.fused = 1;
-        C.owner_share = h->dec_owner_share;
+        C.owner_cost = h->dec_owner_cost;
         C.k_new = static_cast<const __nv_bfloat16*>(fa->k_new);
         C.v_new = static_cast<const __nv_bfloat16*>(fa->v_new);
         C.tier_idx = fa->tier_idx;

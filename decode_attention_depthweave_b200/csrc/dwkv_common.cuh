@@ -108,8 +108,10 @@ struct DecodeCall {
     int tok_weight;          // split balance: cost of one token in byte-equivalents
     // One new token per sequence appended in the same launch (0 = plain decode).  The first CTA
     // of each (sequence, kv-head) places and encodes it and attends to it directly; every CTA
-    // attends to the pages without it.  `owner_share` (of 256) is that CTA's share of a split.
-    int fused, owner_share;
+    // attends to the pages without it.  `owner_cost` (in the split balance's cost units: bytes
+    // plus tok_weight a token) is what that work costs the CTA; it takes that much less.
+    int fused;
+    uint32_t owner_cost;
     const __nv_bfloat16* k_new;      // [n][Hkv][d] bf16 (fused)
     const __nv_bfloat16* v_new;
     const uint8_t* tier_idx;         // [n][Hkv] tier of the new token (read where it is placed)

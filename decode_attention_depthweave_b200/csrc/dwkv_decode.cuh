@@ -903,13 +903,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const Geom G,
             rP[kMaxTiers] = P;
             m_P[G.ntiers] = P;
             // cost-balanced page range: pages whose first cost unit lies in [lo, hi).  With a
-            // fused append, split 0 (which also encodes the token) takes owner_share / 256 of a
-            // share: boundary s sits at W (256 (s - 1) + owner_share) / (256 (nsplit - 1) + owner_share).
-            const float fs = (float)C.owner_share;
-            const float den = 256.f * (float)(nsplit - 1) + fs;
+            // fused append, split 0 also places and encodes the token, a fixed cost E
+            // (owner_cost, in cost units): it takes an even share of W + E less E (at least 0)
+            // and the other splits share the rest evenly, boundary s >= 1 at
+            // own + (W - own) (s - 1) / (nsplit - 1), in integers.
+            const unsigned long long E = (unsigned long long)C.owner_cost;
+            const unsigned long long even = (W + E) / (unsigned long long)nsplit;
+            const unsigned long long own = nsplit == 1 ? W : (even > E ? min(even - E, W) : 0ull);
             auto bound = [&](int sidx) -> unsigned long long {
                 return sidx == 0 ? 0ull
-                                 : (unsigned long long)floor((double)W * (double)((256.f * (float)(sidx - 1) + fs) / den));
+                                 : own + (W - own) * (unsigned long long)(sidx - 1) / (unsigned long long)(nsplit - 1);
             };
             // ceil(x / w): an fp32 estimate (within a few units for these sizes), then exact
             auto cdiv = [](unsigned long long x, uint32_t w) -> uint32_t {
