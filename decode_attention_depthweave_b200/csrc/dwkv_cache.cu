@@ -801,32 +801,49 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
             const uint8_t* ob = S.data + (size_t)s_unit_old * kUnit + (size_t)lig * G.chunk_bytes[kold] +
                                 (z ? G.blk_bytes[kold] : 0u);
             const __nv_bfloat16* bz = bs + (size_t)z * kD * P;
+            // the token's stored entries read in parallel (lane j holds coefficients j + 32 q
+            // and residual entry j), then handed round by shuffles in the chain's order
+            float cl[kMaxRank / 32];
+#pragma unroll
+            for (int q = 0; q < kMaxRank / 32; ++q) {
+                const int j = lane + 32 * q;
+                cl[q] = j < Rold ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                       ob + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2))
+                                 : 0.f;
+            }
+            int ch_l = 0;
+            float v_l = 0.f;
+            if (sold > 0 && lane < sold) {
+                const float sf = __half2float(*reinterpret_cast<const __half*>(ob + off_scales_of(Rold, sold, BITS) + row * 2));
+                const int e = lane;
+                ch_l = ob[off_idx_of(Rold) + row * sold + e];
+                int code;
+                if (BITS == 8) {
+                    code = (int8_t)ob[off_codes_of(Rold, sold) + row * sold + e];
+                } else {
+                    const uint32_t byte = ob[off_codes_of(Rold, sold) + row * (sold / 2) + (e >> 1)];
+                    code = (int)(((e & 1) ? byte >> 4 : byte) & 0xfu);
+                    code = (code ^ 8) - 8;
+                }
+                v_l = __fmul_rn(sf, (float)code);               // exact: 11 x 7 significant bits
+            }
             float a[4] = {0.f, 0.f, 0.f, 0.f};
             for (int j = 0; j < Rold; ++j) {
-                const float cj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                    ob + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2));
+                float src = cl[0];
+#pragma unroll
+                for (int q = 1; q < kMaxRank / 32; ++q) if ((j >> 5) == q) src = cl[q];
+                const float cj = __shfl_sync(0xffffffffu, src, j & 31);
 #pragma unroll
                 for (int m = 0; m < 4; ++m)
                     a[m] = __fmaf_rn(__bfloat162float(bz[(size_t)(lane + 32 * m) * P + j]), cj, a[m]);
             }
-            if (sold > 0) {
-                const float sf = __half2float(*reinterpret_cast<const __half*>(ob + off_scales_of(Rold, sold, BITS) + row * 2));
-                for (int e = 0; e < sold; ++e) {
-                    const int ch = ob[off_idx_of(Rold) + row * sold + e];
-                    int code;
-                    if (BITS == 8) {
-                        code = (int8_t)ob[off_codes_of(Rold, sold) + row * sold + e];
-                    } else {
-                        const uint32_t byte = ob[off_codes_of(Rold, sold) + row * (sold / 2) + (e >> 1)];
-                        code = (int)(((e & 1) ? byte >> 4 : byte) & 0xfu);
-                        code = (code ^ 8) - 8;
-                    }
-                    if ((ch & 31) == lane && ch < kD) {
-                        const float v = __fmul_rn(sf, (float)code);       // exact: 11 x 7 significant bits
+            for (int e = 0; e < sold; ++e) {
+                const int ch = __shfl_sync(0xffffffffu, ch_l, e);
+                const float v = __shfl_sync(0xffffffffu, v_l, e);
+                if ((ch & 31) == lane && ch < kD) {
 #pragma unroll
-                        for (int m = 0; m < 4; ++m)
-                            if ((ch >> 5) == m) a[m] = __fadd_rn(a[m], v);
-                    }
+                    for (int m = 0; m < 4; ++m)
+                        if ((ch >> 5) == m) a[m] = __fadd_rn(a[m], v);
                 }
             }
             UnitIn in;
