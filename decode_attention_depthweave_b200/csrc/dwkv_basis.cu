@@ -386,10 +386,15 @@ __global__ void __launch_bounds__(256) reproject_kernel(const Geom G, const Stat
             v_l = __fmul_rn(sf, (float)code);                     // exact: 11 x 7 significant bits
         }
         float a[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < R; ++j) {
+        for (int j = 0; j < R; j += 2) {                     // R is even: the basis read a pair at a time
             const float cj = __shfl_sync(0xffffffffu, j < 32 ? cl0 : cl1, j & 31);
+            const float cj1 = __shfl_sync(0xffffffffu, j + 1 < 32 ? cl0 : cl1, (j + 1) & 31);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) a[m] = __fmaf_rn(__bfloat162float(bz[(size_t)(lane + 32 * m) * P + j]), cj, a[m]);
+            for (int m = 0; m < 4; ++m) {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(bz + (size_t)(lane + 32 * m) * P + j);
+                a[m] = __fmaf_rn(bf16lo(w), cj, a[m]);
+                a[m] = __fmaf_rn(bf16hi(w), cj1, a[m]);
+            }
         }
         for (int e = 0; e < st; ++e) {
             const int ch = __shfl_sync(0xffffffffu, ch_l, e);

@@ -828,14 +828,18 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
                 v_l = __fmul_rn(sf, (float)code);               // exact: 11 x 7 significant bits
             }
             float a[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int j = 0; j < Rold; ++j) {
+            for (int j = 0; j < Rold; j += 2) {              // Rold is even: the basis read a pair at a time
                 float src = cl[0];
 #pragma unroll
                 for (int q = 1; q < kMaxRank / 32; ++q) if ((j >> 5) == q) src = cl[q];
                 const float cj = __shfl_sync(0xffffffffu, src, j & 31);
+                const float cj1 = __shfl_sync(0xffffffffu, src, (j + 1) & 31);   // j + 1 in the same 32
 #pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    a[m] = __fmaf_rn(__bfloat162float(bz[(size_t)(lane + 32 * m) * P + j]), cj, a[m]);
+                for (int m = 0; m < 4; ++m) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(bz + (size_t)(lane + 32 * m) * P + j);
+                    a[m] = __fmaf_rn(bf16lo(w), cj, a[m]);
+                    a[m] = __fmaf_rn(bf16hi(w), cj1, a[m]);
+                }
             }
             for (int e = 0; e < sold; ++e) {
                 const int ch = __shfl_sync(0xffffffffu, ch_l, e);

@@ -296,56 +296,86 @@ __device__ __forceinline__ void encode_body(const Geom& G, const State& S, const
         for (int m = 0; m < 4; ++m) xs[lane + 32 * m] = xr[m];
         __syncwarp();
         // ---- 1-2: projection (fma chain over i from +0), bf16 rounding, coefficient store.
-        //      Lane takes j = lane + 32 jj; the chains of one lane run interleaved.
+        //      Lane takes the pairs j = 2 lane, 2 lane + 1 and 64 + 2 lane, 65 + 2 lane (one
+        //      32-bit basis load a pair, x four channels a load); each j's chain runs over i in
+        //      order, so the lane assignment does not change a result.
         {
-            float acc[kMaxRank / 32];
+            float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            const bool on1 = 64 + 2 * lane < R;           // R is a multiple of 8: pairs are whole
+            const bool on0 = 2 * lane < R;
+#pragma unroll 2
+            for (int i = 0; i < kD; i += 4) {
+                const float4 x4 = *reinterpret_cast<const float4*>(xs + i);
+                const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
-            for (int jj = 0; jj < kMaxRank / 32; ++jj) acc[jj] = 0.f;
-#pragma unroll 8
-            for (int i = 0; i < kD; ++i) {
-                const float xi = xs[i];
-                const __nv_bfloat16* brow = bz + (size_t)i * P + lane;
-#pragma unroll
-                for (int jj = 0; jj < kMaxRank / 32; ++jj)
-                    if (lane + 32 * jj < R) acc[jj] = __fmaf_rn(__bfloat162float(brow[32 * jj]), xi, acc[jj]);
+                for (int ii = 0; ii < 4; ++ii) {
+                    const __nv_bfloat16* brow = bz + (size_t)(i + ii) * P + 2 * lane;
+                    if (on0) {
+                        const uint32_t w = *reinterpret_cast<const uint32_t*>(brow);
+                        acc[0][0] = __fmaf_rn(bf16lo(w), xv[ii], acc[0][0]);
+                        acc[0][1] = __fmaf_rn(bf16hi(w), xv[ii], acc[0][1]);
+                    }
+                    if (on1) {
+                        const uint32_t w = *reinterpret_cast<const uint32_t*>(brow + 64);
+                        acc[1][0] = __fmaf_rn(bf16lo(w), xv[ii], acc[1][0]);
+                        acc[1][1] = __fmaf_rn(bf16hi(w), xv[ii], acc[1][1]);
+                    }
+                }
             }
 #pragma unroll
-            for (int jj = 0; jj < kMaxRank / 32; ++jj) {
-                const int j = lane + 32 * jj;
-                if (G.c8) {
-                    if (32 * jj >= R) break;                       // uniform: R is a multiple of 16
+            for (int q = 0; q < 2; ++q) {
+                const int j = 64 * q + 2 * lane;
+                if (j >= R) continue;
+                if (in.dbg) *reinterpret_cast<float2*>(in.dbg + j) = make_float2(acc[q][0], acc[q][1]);
+                if (G.c8) {                               // raw projections; the blocks below
+                    *reinterpret_cast<float2*>(cs + j) = make_float2(acc[q][0], acc[q][1]);
+                } else {
+                    __nv_bfloat162 cb;
+                    cb.x = __float2bfloat16_rn(acc[q][0]);
+                    cb.y = __float2bfloat16_rn(acc[q][1]);
+                    *reinterpret_cast<float2*>(cs + j) = make_float2(__bfloat162float(cb.x), __bfloat162float(cb.y));
+                    *reinterpret_cast<__nv_bfloat162*>(blk + (size_t)(j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2) = cb;
+                }
+            }
+            if (G.c8) {
+                // the 8-bit blockwise form: lane j = lane + 32 jj, a half warp a block of 16
+                __syncwarp();
+#pragma unroll
+                for (int jj = 0; jj < kMaxRank / 32; ++jj) {
+                    if (32 * jj >= R) break;                   // uniform: R is a multiple of 16
+                    const int j = lane + 32 * jj;
                     uint16_t sh;
-                    int q;
+                    int qc;
                     float cb;
-                    quantize_coeff8(j < R ? acc[jj] : 0.f, sh, q, cb);
+                    quantize_coeff8(j < R ? cs[j] : 0.f, sh, qc, cb);
                     if (j < R) {
-                        if (in.dbg) in.dbg[j] = acc[jj];
                         cs[j] = cb;
-                        blk[z ? vc8_code_off(j, dst.row) : kc8_code_off(j, dst.row)] = (uint8_t)(int8_t)q;
+                        blk[z ? vc8_code_off(j, dst.row) : kc8_code_off(j, dst.row)] = (uint8_t)(int8_t)qc;
                         if ((j & 15) == 0)
                             *reinterpret_cast<uint16_t*>(blk + (z ? vc8_scale_off(R, j >> 4, dst.row)
                                                                   : kc8_scale_off(R, j >> 4, dst.row))) = sh;
                     }
-                } else if (j < R) {
-                    if (in.dbg) in.dbg[j] = acc[jj];
-                    const __nv_bfloat16 cb = __float2bfloat16_rn(acc[jj]);
-                    cs[j] = __bfloat162float(cb);
-                    *reinterpret_cast<__nv_bfloat16*>(blk + (size_t)(j >> 3) * 1024 + dst.row * 16 + (j & 7) * 2) = cb;
                 }
             }
         }
         __syncwarp();
-        // ---- 3: residual against the stored coefficients (fma chain over j from +0)
+        // ---- 3: residual against the stored coefficients (fma chain over j from +0), the
+        //      basis read a pair of j at a time
         float r[4];
         {
             float a[4] = {0.f, 0.f, 0.f, 0.f};
             for (int j0 = 0; j0 < R; j0 += 8) {           // R is a multiple of 8
+                const float4 c0 = *reinterpret_cast<const float4*>(cs + j0);
+                const float4 c1 = *reinterpret_cast<const float4*>(cs + j0 + 4);
+                const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const float cj = cs[j0 + jj];
+                for (int jj = 0; jj < 8; jj += 2) {
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        a[m] = __fmaf_rn(__bfloat162float(bz[(size_t)(lane + 32 * m) * P + j0 + jj]), cj, a[m]);
+                    for (int m = 0; m < 4; ++m) {
+                        const uint32_t w = *reinterpret_cast<const uint32_t*>(bz + (size_t)(lane + 32 * m) * P + j0 + jj);
+                        a[m] = __fmaf_rn(bf16lo(w), cv[jj], a[m]);
+                        a[m] = __fmaf_rn(bf16hi(w), cv[jj + 1], a[m]);
+                    }
                 }
             }
 #pragma unroll
