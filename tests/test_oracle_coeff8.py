@@ -2,9 +2,10 @@
 Cross-Layer Residual Factorization for Long-Context KV Cache Compression", §3 Method: the
 coefficient vector is the projection onto the current basis, kept as 8-bit codes with one
 scale per block of coefficients).  The block of 16 and the symmetric max-scaled codes are
-this build's reading; the checks rest on values that sit exactly on the code grid, the
-rounding rule, the quantiser's error bound, block locality and exact signed-permutation
-bases, and the decode path is checked against dense attention over the dequantised cache."""
+the reading taken here (the pages give no block size); the checks rest on values that sit
+exactly on the code grid, the rounding rule, the quantiser's error bound, block locality and
+exact signed-permutation bases, and the decode path is checked against dense attention over
+the dequantised cache."""
 import numpy as np
 import pytest
 import torch
