@@ -46,9 +46,9 @@ def _append(wl, lengths, chunks, gates):
     return cache, bases, rows, c32
 
 
-@pytest.mark.parametrize("chunks", [(1, 3, 4), (37, 64, 1000)])
-def test_gated_append_bytes_and_decode(chunks):
-    wl = _wl()
+@pytest.mark.parametrize("chunks,coeff_bits", [((1, 3, 4), 16), ((37, 64, 1000), 16), ((1, 3, 4), 8), ((37, 64, 1000), 8)])
+def test_gated_append_bytes_and_decode(chunks, coeff_bits):
+    wl = _wl(coeff_bits=coeff_bits)
     lengths = [150, 77]
     g = torch.Generator().manual_seed(9)
     gates = {(b, layer): torch.rand(T, wl.num_kv_heads, 2, generator=g) for b, T in enumerate(lengths) for layer in range(2)}
@@ -59,7 +59,7 @@ def test_gated_append_bytes_and_decode(chunks):
             k, v = rows[b][layer]
             got = cache.export(layer, b, 0, T)
             ref = oracle_encode_rows(wl, bases, layer, k, v, tiers, c32=c32[(b, layer)], gate=gates[(b, layer)])
-            for key in ("coeff", "idx", "codes", "scales"):
+            for key in ref:
                 assert torch.equal(got[key].cpu().contiguous().view(torch.uint8), ref[key].contiguous().view(torch.uint8)), \
                     (b, layer, key)
     for layer in range(2):
