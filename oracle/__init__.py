@@ -57,6 +57,8 @@ def lib():
         L.oracle_encode_vector8.restype = i
         L.oracle_encode_many8.argtypes = [i, i, i, p, p, p, p, i, i, p, p, p, p, p, p, i, p]
         L.oracle_encode_many8.restype = i
+        L.oracle_reencode_vector8.argtypes = [i, i, p, i, p, p, i, p, p, C.c_uint16, i, i, i, p, p, p, p, p, p, p]
+        L.oracle_reencode_vector8.restype = i
         for name in ("oracle_f32_to_bf16_rn_many", "oracle_f32_to_fp16_rn_many",
                      "oracle_fp16_to_f64_many", "oracle_bf16_to_f64_many"):
             getattr(L, name).argtypes = [C.c_int64, p, p]
@@ -447,6 +449,35 @@ def encode_many8(basis, x, ranks, s, bits, c32=None, nthreads=None, nres=None, w
         out["c32"] = co
     return out
 
+
+def reencode_vector8(basis, r_old, ccodes, cscales, idx, codes, scale, r_new, bits, s_new=None, basis_new=None):
+    """reencode_vector for the 8-bit blockwise coefficient form: the stored codes int8 [r_max]
+    and block scales (fp16 bits [r_max / 16]) in, the new ones out
+    (``oracle_reencode_vector8``).  Returns the encode8 dict plus ``xh`` (bf16 bits [d])."""
+    b = _bits16(basis)
+    d, r_max = b.shape
+    cc = _arr(ccodes, np.int8).reshape(r_max)
+    cs = _bits16(cscales).reshape(r_max // 16)
+    ix = _arr(idx, np.uint8).reshape(-1)
+    cd = _arr(codes, np.int8).reshape(-1)
+    s = ix.size
+    sc = int(_bits16(scale).reshape(-1)[0])
+    sn = s if s_new is None else int(s_new)
+    out_cc = np.zeros(r_max, np.int8)
+    out_cs = np.zeros(r_max // 16, np.uint16)
+    out_i = np.zeros(sn, np.uint8)
+    out_q = np.zeros(sn, np.int8)
+    out_s = np.zeros(1, np.uint16)
+    xh = np.zeros(d, np.uint16)
+    bn = None if basis_new is None else _bits16(basis_new)
+    if bn is not None and bn.shape != b.shape:
+        raise ValueError("basis_new must have the basis' shape")
+    rc = lib().oracle_reencode_vector8(d, r_max, _p(b), int(r_old), _p(cc), _p(cs), s, _p(ix), _p(cd), sc,
+                                       int(r_new), sn, int(bits), _p(out_cc), _p(out_cs), _p(out_i), _p(out_q),
+                                       _p(out_s), _p(xh), _p(bn) if bn is not None else None)
+    if rc != 0:
+        raise ValueError("oracle_reencode_vector8: bad arguments")
+    return {"ccodes": out_cc, "cscales": out_cs, "idx": out_i, "codes": out_q, "scale": out_s[0], "xh": xh}
 
 # ----------------------------------------------------------------------------- residual gate
 def gate_scales(scales, gates) -> np.ndarray:

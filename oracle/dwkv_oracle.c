@@ -511,6 +511,44 @@ int oracle_reencode_vector(int d, int r_max, const uint16_t* basis, int r_old, c
                                 codes, scale, NULL);
 }
 
+/* The same re-encode for the 8-bit blockwise coefficient form: the stored coefficients are */
+/* cb_j = code_j * scale_{j/16} (exact in fp32: 8 x 11 significant bits), the reconstruction */
+/* chain and its bf16 rounding are those of oracle_reencode_vector, and xh is encoded by     */
+/* oracle_encode_vector8 (its own projection) at rank r_new with s_new residual channels.    */
+/* Inputs: ccodes_old int8 [r_max] and cscales_old fp16 bits [r_max / 16] (entries of j >=  */
+/* r_old ignored), the residual as oracle_reencode_vector.  Outputs: ccodes [r_max],        */
+/* cscales [r_max / 16], idx / codes [s_new], scale; xh_out (nullable) bf16 bits [d].       */
+int oracle_reencode_vector8(int d, int r_max, const uint16_t* basis, int r_old, const int8_t* ccodes_old,
+                            const uint16_t* cscales_old, int s, const uint8_t* idx_old, const int8_t* codes_old,
+                            uint16_t scale_old, int r_new, int s_new, int bits, int8_t* ccodes, uint16_t* cscales,
+                            uint8_t* idx, int8_t* codes, uint16_t* scale, uint16_t* xh_out,
+                            const uint16_t* basis_new) {
+    if (d <= 0 || d > 256 || r_max > 256 || r_max % 16 || r_old < 0 || r_old > r_max || r_old % 16 || r_new < 0 ||
+        r_new > r_max || s < 0 || s > d || s_new < 0 || s_new > d)
+        return -1;
+    float cb[256], a[256];
+    uint16_t xh[256];
+    for (int j = 0; j < r_old; ++j)
+        cb[j] = (float)ccodes_old[j] * (float)oracle_fp16_to_f64(cscales_old[j / 16]);
+    for (int i = 0; i < d; ++i) {
+        float acc = 0.0f;
+        for (int j = 0; j < r_old; ++j)
+            acc = fmaf((float)oracle_bf16_to_f64(basis[(size_t)i * r_max + j]), cb[j], acc);
+        a[i] = acc;
+    }
+    const float sf = (float)oracle_fp16_to_f64(scale_old);
+    for (int k = 0; k < s; ++k) {
+        if (idx_old[k] >= d) return -1;
+        a[idx_old[k]] = a[idx_old[k]] + sf * (float)codes_old[k];
+    }
+    for (int i = 0; i < d; ++i) {
+        xh[i] = oracle_f32_to_bf16_rn(a[i]);
+        if (xh_out) xh_out[i] = xh[i];
+    }
+    return oracle_encode_vector8(d, r_max, basis_new ? basis_new : basis, xh, NULL, r_new, s_new, bits, ccodes,
+                                 cscales, NULL, idx, codes, scale);
+}
+
 /* Element-wise format conversions over arrays (used to pin the converters). */
 void oracle_f32_to_bf16_rn_many(int64_t n, const float* x, uint16_t* out) {
     for (int64_t k = 0; k < n; ++k) out[k] = oracle_f32_to_bf16_rn(x[k]);
