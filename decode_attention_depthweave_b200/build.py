@@ -18,7 +18,7 @@ LIB = os.path.join(OUT_DIR, "libdwkv.so")
 SOURCES = ["dwkv_api.cu", "dwkv_basis.cu", "dwkv_cache.cu", "dwkv_control.cu", "dwkv_decode_b4.cu", "dwkv_decode_b4p.cu",
            "dwkv_decode_b8.cu", "dwkv_decode_b8p.cu", "dwkv_decode_b4c8.cu", "dwkv_decode_b4pc8.cu",
            "dwkv_decode_b8c8.cu", "dwkv_decode_b8pc8.cu"]
-HEADERS = ["dwkv_common.cuh", "dwkv_decode.cuh", "dwkv_encode.cuh"]
+HEADERS = ["dwkv_common.cuh", "dwkv_decode.cuh", "dwkv_encode.cuh", "dwkv_stored.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

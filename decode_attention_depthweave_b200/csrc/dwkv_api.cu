@@ -651,8 +651,6 @@ dwkv_status dwkv_basis_update(dwkv_handle h, int32_t group, int32_t n_rows, cons
     if (!(beta >= 0.f && beta <= 1.f)) return fail(DWKV_ERR_INVALID_ARG, "beta must be in [0, 1]");
     if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
     const Geom& G = h->geom;
-    if (n_seqs > 0 && G.c8)
-        return fail(DWKV_ERR_UNSUPPORTED, "no re-projection kernel for 8-bit coefficients (update with n_seqs = 0)");
     for (int i = 0; i < n_seqs; ++i) {
         const int sq = seq_ids[i];
         for (int g = g0; g < g0 + ng; ++g) {
@@ -1088,7 +1086,6 @@ dwkv_status dwkv_retier(dwkv_handle h, int32_t group, int32_t n_seqs, const int3
     dwkv_status st;
     if ((st = check_handle(h)) != DWKV_OK) return st;
     const Geom& G = h->geom;
-    if (G.c8) return fail(DWKV_ERR_UNSUPPORTED, "no re-tier kernel for 8-bit coefficients");
     if (group < 0 || group >= G.G) return fail(DWKV_ERR_INVALID_ARG, "group %d out of [0, %d)", group, G.G);
     if ((st = check_seq_list(h, n_seqs, seq_ids)) != DWKV_OK) return st;
     if (n_seqs && !n_tok) return fail(DWKV_ERR_INVALID_ARG, "n_tok is NULL");

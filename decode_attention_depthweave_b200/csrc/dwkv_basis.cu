@@ -12,6 +12,7 @@
 // Rayleigh-Ritz step.  Stored tokens: reconstruction on B_old (the re-tiering chain), then the
 // six encode steps on B_new at the same tier.
 #include "dwkv_encode.cuh"
+#include "dwkv_stored.cuh"
 
 namespace dwkv {
 
@@ -365,26 +366,11 @@ __global__ void __launch_bounds__(256) reproject_kernel(const Geom G, const Stat
         // token's coefficients and residual entries are read in parallel (lane j holds entry j
         // and j + 32) and handed round by shuffles: the chain's order is unchanged.
         const __nv_bfloat16* bz = bo + (size_t)z * kD * P;
-        auto coeff_at = [&](int j) {
-            return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(blk + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2));
-        };
-        const float cl0 = lane < R ? coeff_at(lane) : 0.f, cl1 = lane + 32 < R ? coeff_at(lane + 32) : 0.f;
+        const float cl0 = lane < R ? stored_coeff(blk, G.c8, (int)z, R, row, lane) : 0.f;
+        const float cl1 = lane + 32 < R ? stored_coeff(blk, G.c8, (int)z, R, row, lane + 32) : 0.f;
         int ch_l = 0;
         float v_l = 0.f;
-        if (st > 0 && lane < st) {
-            const float sf = __half2float(*reinterpret_cast<const __half*>(blk + off_scales_of(R, st, BITS) + row * 2));
-            const int e = lane;
-            ch_l = blk[off_idx_of(R) + row * st + e];
-            int code;
-            if (BITS == 8) {
-                code = (int8_t)blk[off_codes_of(R, st) + row * st + e];
-            } else {
-                const uint32_t byte = blk[off_codes_of(R, st) + row * (st / 2) + (e >> 1)];
-                code = (int)(((e & 1) ? byte >> 4 : byte) & 0xfu);
-                code = (code ^ 8) - 8;
-            }
-            v_l = __fmul_rn(sf, (float)code);                     // exact: 11 x 7 significant bits
-        }
+        if (st > 0 && lane < st) stored_resid<BITS>(blk, G.c8, R, st, row, lane, ch_l, v_l);
         float a[4] = {0.f, 0.f, 0.f, 0.f};
         for (int j = 0; j < R; j += 2) {                     // R is even: the basis read a pair at a time
             const float cj = __shfl_sync(0xffffffffu, j < 32 ? cl0 : cl1, j & 31);

@@ -1,6 +1,7 @@
 // dwkv_cache.cu -- page placement, encode/append, import, export and reset kernels.  The
 // per-vector encode steps and their fixed operation order are in dwkv_encode.cuh.
 #include "dwkv_encode.cuh"
+#include "dwkv_stored.cuh"
 
 namespace dwkv {
 
@@ -807,26 +808,11 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
 #pragma unroll
             for (int q = 0; q < kMaxRank / 32; ++q) {
                 const int j = lane + 32 * q;
-                cl[q] = j < Rold ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                                       ob + (size_t)(j >> 3) * 1024 + row * 16 + (j & 7) * 2))
-                                 : 0.f;
+                cl[q] = j < Rold ? stored_coeff(ob, G.c8, z, Rold, row, j) : 0.f;
             }
             int ch_l = 0;
             float v_l = 0.f;
-            if (sold > 0 && lane < sold) {
-                const float sf = __half2float(*reinterpret_cast<const __half*>(ob + off_scales_of(Rold, sold, BITS) + row * 2));
-                const int e = lane;
-                ch_l = ob[off_idx_of(Rold) + row * sold + e];
-                int code;
-                if (BITS == 8) {
-                    code = (int8_t)ob[off_codes_of(Rold, sold) + row * sold + e];
-                } else {
-                    const uint32_t byte = ob[off_codes_of(Rold, sold) + row * (sold / 2) + (e >> 1)];
-                    code = (int)(((e & 1) ? byte >> 4 : byte) & 0xfu);
-                    code = (code ^ 8) - 8;
-                }
-                v_l = __fmul_rn(sf, (float)code);               // exact: 11 x 7 significant bits
-            }
+            if (sold > 0 && lane < sold) stored_resid<BITS>(ob, G.c8, Rold, sold, row, lane, ch_l, v_l);
             float a[4] = {0.f, 0.f, 0.f, 0.f};
             for (int j = 0; j < Rold; j += 2) {              // Rold is even: the basis read a pair at a time
                 float src = cl[0];
@@ -863,23 +849,11 @@ __global__ void __launch_bounds__(256) retier_kernel(const Geom G, const State S
         // ---- 3: the old tier's last slot into the token's old slot
         if (slot != last) {
             const int lrow = last % kPage;
-            const uint32_t blk = G.blk_bytes[kold];
-            const uint32_t coff = off_idx_of(Rold);
-            const uint32_t nidx = (uint32_t)sold, ncode = (uint32_t)sold * BITS / 8;
             for (int u = warp; u < 2 * G.LPG; u += (int)(blockDim.x >> 5)) {
                 const int lig = u >> 1, z = u & 1;
-                uint8_t* dst = S.data + (size_t)s_unit_old * kUnit + (size_t)lig * G.chunk_bytes[kold] + (z ? blk : 0u);
-                const uint8_t* src = S.data + (size_t)s_unit_last * kUnit + (size_t)lig * G.chunk_bytes[kold] + (z ? blk : 0u);
-                for (int c = lane; c < Rold / 8; c += 32)       // 8-coefficient columns, 16 bytes a token
-                    *reinterpret_cast<uint4*>(dst + (size_t)c * 1024 + row * 16) =
-                        *reinterpret_cast<const uint4*>(src + (size_t)c * 1024 + lrow * 16);
-                for (uint32_t b = lane; b < nidx; b += 32) dst[coff + row * nidx + b] = src[coff + lrow * nidx + b];
-                const uint32_t qo = off_codes_of(Rold, sold);
-                for (uint32_t b = lane; b < ncode; b += 32) dst[qo + row * ncode + b] = src[qo + lrow * ncode + b];
-                if (lane == 0) {
-                    const uint32_t so = off_scales_of(Rold, sold, BITS);
-                    *reinterpret_cast<uint16_t*>(dst + so + row * 2) = *reinterpret_cast<const uint16_t*>(src + so + lrow * 2);
-                }
+                const size_t o = (size_t)lig * G.chunk_bytes[kold] + (z ? G.blk_bytes[kold] : 0u);
+                move_row<BITS>(S.data + (size_t)s_unit_old * kUnit + o, S.data + (size_t)s_unit_last * kUnit + o, G.c8,
+                               z, Rold, sold, row, lrow);
             }
             if (tid == 0) {
                 const int32_t* lp = reinterpret_cast<const int32_t*>(S.data + (size_t)s_unit_last * kUnit + pos_block_of(G, kold));

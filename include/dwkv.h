@@ -111,7 +111,7 @@ typedef struct {
      * 16 coefficients with one fp16 scale a block, scale = fp16(max |c| / 127) and
      * code = clamp(rint(c / scale), -127, 127); the residual is taken against code * scale.
      * Needs r_max and every tier rank to be multiples of 16.  Re-tiering and the basis
-     * update's re-projection have no kernels for it (DWKV_ERR_UNSUPPORTED). */
+     * update's re-projection re-encode such tokens from code * scale. */
     int32_t coeff_bits;
 } dwkv_config;
 
@@ -150,7 +150,7 @@ dwkv_status dwkv_basis_sketch(dwkv_handle h, int32_t group, int32_t n_rows, cons
  * refreshed from C, then every stored token of the listed sequences (host seq_ids) re-projected
  * onto them: each (token, layer of the window, K / V) is reconstructed on the previous basis
  * (the fixed-order fp32 chain over its rank plus scale x code, rounded to bf16, as dwkv_retier
- * does) and encoded on the new basis at its own tier, in place.  Every layer of the window
+ * does, for either coefficient form) and encoded on the new basis at its own tier, in place.  Every layer of the window
  * must hold the same positions for each listed sequence (DWKV_ERR_INVALID_ARG otherwise).
  * beta in [0, 1].  eigenvalues: as dwkv_basis_sketch.  Tokens of sequences not listed keep
  * their bytes and are then stale against the new bases: list every sequence that holds tokens
@@ -318,9 +318,10 @@ dwkv_status dwkv_probe(dwkv_handle h, int32_t layer, int32_t n_seqs, const int32
  *   - a token already at its new tier is left as it is;
  *   - otherwise it is re-encoded at the new rank from its reconstruction (Eq. (1), g = 1),
  *     since the dense vector is not kept: a_i = fp32 fma chain over j < r_old of
- *     B[i][j] * c_j from +0, plus scale * code on its residual channels, rounded to bf16,
- *     then the encode steps of dwkv_append; the stored bytes equal dwkv_append's for that
- *     bf16 vector.
+ *     B[i][j] * c_j from +0 (c_j the stored bf16 coefficient, or with coeff_bits 8 its
+ *     code * block scale, exact in fp32), plus scale * code on its residual channels,
+ *     rounded to bf16, then the encode steps of dwkv_append; the stored bytes equal
+ *     dwkv_append's for that bf16 vector.
  * Every layer of the group must hold the same positions (call between decode steps, not
  * between the layers of one step); DWKV_ERR_INVALID_ARG otherwise.  Positions the group has
  * not placed, or tier indices >= num_tiers, set a device error (DWKV_DEV_NO_SLOT,
