@@ -319,89 +319,255 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
 
 // ------------------------------------------------------------------------------------
 // Re-projection of the stored tokens of a window onto its updated basis: gridDim.z blocks per
-// (sequence in the list, kv-head), a warp per (slot, layer of the window, K / V) unit, the
-// units of a (sequence, kv-head) dealt out over its blocks' warps.  Each
-// unit is reconstructed on the previous basis (old_k / old_v: the fixed-order fp32 chain over
-// its rank, plus scale x code on its residual channels, rounded to bf16, as a re-tier does)
-// and encoded on the new basis at its own tier, in place.  Slots and counts do not change.
+// (sequence in the list, kv-head), half of them for the keys and half for the values (block z
+// index even: keys).  A warp takes a group of up to kRpMaxGroup tokens of one tier and one layer
+// of the window on its side (V = min(4, 64 / R) tokens: every lane busy in the projection),
+// the groups dealt out over the side's warps.  Each token is reconstructed on the previous
+// basis (old_k / old_v: the fixed-order fp32 chain over its rank, plus scale x code on its
+// residual channels, rounded to bf16, as a re-tier does) and encoded on the new basis at its own
+// tier, in place, by the six encode steps in the encoders' operation order:
+//   1-2  lane (v, p) runs token v's projection chains of coefficients 2p and 2p + 1 over the
+//        channels in order (the bf16 basis read a pair at a time, x four channels a load), then
+//        rounds them to bf16 or forms their 8-bit blocks (a block of 16 on 8 lanes);
+//   3    the residual chains of the group's tokens share each basis load;
+//   4-6  quantize_store per token.
+// Slots and counts do not change.  Online bases have r_max <= 64.
 // ------------------------------------------------------------------------------------
+constexpr int kRpMaxGroup = 4;
+constexpr int kRpXPitch = kD + 4;                  // floats: group rows on distinct banks
+constexpr uint32_t kRpWarpBytes = (uint32_t)(kRpMaxGroup * kRpXPitch + kRpMaxGroup * 64 + 32) * 4u + 32u +
+                                   (uint32_t)kRpMaxGroup * 16u;   // + the group's block addresses and rows
+
+// Dynamic shared memory of reproject_kernel: the side's two bases [d][r_max + 2], then each
+// warp's group scratch.
+size_t reproject_smem_bytes(int r_max, int warps) {
+    return (size_t)2 * kD * (r_max + 2) * 2 + (size_t)warps * kRpWarpBytes;
+}
+
+template <int BITS, int V>
+__device__ __forceinline__ void reproject_group(const Geom& G, int z, int k, int nu, uint8_t* const* blk,
+                                                const int* row, const __nv_bfloat16* bn, const __nv_bfloat16* bo,
+                                                float* xs, float* cs, float* rstage, uint8_t* chstage) {
+    const int lane = threadIdx.x & 31;
+    const int P = G.r_max + 2, R = G.tiers[k], st = G.ts[k], c8 = G.c8;
+    // ---- reconstruction on the previous basis: token u's entries read in parallel (lane j
+    //      holds coefficient j and j + 32, residual entry j) and handed round by shuffles
+    float cl0[V], cl1[V], v_l[V];
+    int ch_l[V];
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+        const bool on = u < nu;
+        const uint8_t* b = blk[u];
+        const int rw = row[u];
+        cl0[u] = on && lane < R ? stored_coeff(b, c8, z, R, rw, lane) : 0.f;
+        cl1[u] = on && lane + 32 < R ? stored_coeff(b, c8, z, R, rw, lane + 32) : 0.f;
+        ch_l[u] = kD;
+        v_l[u] = 0.f;
+        if (on && lane < st) stored_resid<BITS>(b, c8, R, st, rw, lane, ch_l[u], v_l[u]);
+    }
+    {
+        float a[V][4];
+#pragma unroll
+        for (int u = 0; u < V; ++u)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) a[u][m] = 0.f;
+        for (int j = 0; j < R; j += 2) {                 // R is even: the basis read a pair at a time
+            uint32_t w[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) w[m] = *reinterpret_cast<const uint32_t*>(bo + (size_t)(lane + 32 * m) * P + j);
+#pragma unroll
+            for (int u = 0; u < V; ++u) {
+                const float cj = __shfl_sync(0xffffffffu, j < 32 ? cl0[u] : cl1[u], j & 31);
+                const float cj1 = __shfl_sync(0xffffffffu, j + 1 < 32 ? cl0[u] : cl1[u], (j + 1) & 31);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    a[u][m] = __fmaf_rn(bf16lo(w[m]), cj, a[u][m]);
+                    a[u][m] = __fmaf_rn(bf16hi(w[m]), cj1, a[u][m]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < V; ++u)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) xs[u * kRpXPitch + lane + 32 * m] = a[u][m];
+    }
+    __syncwarp();
+    // the residual entries: lane e adds entry e to its channel.  A token's channels are
+    // distinct, so each channel takes at most one add and their order is free; a token whose
+    // channels repeat takes its entries one at a time in entry order.  Channels >= d are
+    // ignored.  Then the vector rounds to bf16.
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+        if (st == 0) break;
+        float* xu = xs + u * kRpXPitch;
+        const bool has = ch_l[u] < kD;               // only lanes e < st of a live token hold one
+        const uint32_t peers = __match_any_sync(0xffffffffu, has ? ch_l[u] : kD + lane);
+        if (!__any_sync(0xffffffffu, has && __popc(peers) > 1)) {
+            if (has) xu[ch_l[u]] = __fadd_rn(xu[ch_l[u]], v_l[u]);
+        } else {
+            for (int e = 0; e < st; ++e) {
+                const int ch = __shfl_sync(0xffffffffu, ch_l[u], e);
+                const float v = __shfl_sync(0xffffffffu, v_l[u], e);
+                if (lane == 0 && ch < kD) xu[ch] = __fadd_rn(xu[ch], v);
+                __syncwarp();
+            }
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < V; ++u)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            float* x = xs + u * kRpXPitch + lane + 32 * m;
+            *x = __bfloat162float(__float2bfloat16_rn(*x));
+        }
+    __syncwarp();                                        // every lane has read the old bytes; x in xs
+    // ---- 1-2: projection, lane (v, p) = token v, coefficients 2p and 2p + 1
+    {
+        const int lpv = R >> 1, v = lane / lpv, p = lane - v * lpv, j = 2 * p;
+        const bool on = v < V && v < nu;
+        const float* xv = xs + (v < V ? v : 0) * kRpXPitch;
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 2
+        for (int i = 0; i < kD; i += 4) {
+            const float4 x4 = *reinterpret_cast<const float4*>(xv + i);
+            const float xq[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(bn + (size_t)(i + ii) * P + j);
+                acc0 = __fmaf_rn(bf16lo(w), xq[ii], acc0);
+                acc1 = __fmaf_rn(bf16hi(w), xq[ii], acc1);
+            }
+        }
+        float* cv = cs + (v < V ? v : 0) * 64;
+        uint8_t* bv = blk[v < V ? v : 0];               // token v's block and row
+        const int rv = row[v < V ? v : 0];
+        if (c8) {
+            // 8-bit blocks: the 16 coefficients of a block on 8 lanes (a pair each), lpv >= 8
+            float mx = fmaxf(fabsf(acc0), fabsf(acc1));
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const __half sh = __float2half_rn(__fdiv_rn(mx, 127.f));
+            const float sf = __half2float(sh);
+            float q0 = 0.f, q1 = 0.f;
+            if (sf != 0.f) {
+                q0 = fminf(fmaxf(rintf(__fdiv_rn(acc0, sf)), -127.f), 127.f);
+                q1 = fminf(fmaxf(rintf(__fdiv_rn(acc1, sf)), -127.f), 127.f);
+            }
+            if (on) {
+                bv[z ? vc8_code_off(j, rv) : kc8_code_off(j, rv)] = (uint8_t)(int8_t)(int)q0;
+                bv[z ? vc8_code_off(j + 1, rv) : kc8_code_off(j + 1, rv)] = (uint8_t)(int8_t)(int)q1;
+                if ((j & 15) == 0)
+                    *reinterpret_cast<uint16_t*>(bv + (z ? vc8_scale_off(R, j >> 4, rv) : kc8_scale_off(R, j >> 4, rv))) =
+                        __half_as_ushort(sh);
+                *reinterpret_cast<float2*>(cv + j) = make_float2(q0 * sf, q1 * sf);
+            }
+        } else if (on) {
+            __nv_bfloat162 cb;
+            cb.x = __float2bfloat16_rn(acc0);
+            cb.y = __float2bfloat16_rn(acc1);
+            *reinterpret_cast<float2*>(cv + j) = make_float2(__bfloat162float(cb.x), __bfloat162float(cb.y));
+            *reinterpret_cast<__nv_bfloat162*>(bv + (size_t)(j >> 3) * 1024 + rv * 16 + (j & 7) * 2) = cb;
+        }
+    }
+    __syncwarp();
+    // ---- 3: residuals against the stored coefficients (fma chain over j from +0), the group's
+    //      tokens sharing each basis load
+    float r[V][4];
+    {
+        float a[V][4];
+#pragma unroll
+        for (int u = 0; u < V; ++u)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) a[u][m] = 0.f;
+        for (int j0 = 0; j0 < R; j0 += 8) {              // R is a multiple of 8
+#pragma unroll
+            for (int jj = 0; jj < 8; jj += 2) {
+                uint32_t w[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) w[m] = *reinterpret_cast<const uint32_t*>(bn + (size_t)(lane + 32 * m) * P + j0 + jj);
+#pragma unroll
+                for (int u = 0; u < V; ++u) {
+                    const float2 c2 = *reinterpret_cast<const float2*>(cs + u * 64 + j0 + jj);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        a[u][m] = __fmaf_rn(bf16lo(w[m]), c2.x, a[u][m]);
+                        a[u][m] = __fmaf_rn(bf16hi(w[m]), c2.y, a[u][m]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < V; ++u)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) r[u][m] = __fsub_rn(xs[u * kRpXPitch + lane + 32 * m], a[u][m]);
+    }
+    // ---- 4-6 per token
+#pragma unroll
+    for (int u = 0; u < V; ++u)
+        if (u < nu) quantize_store<BITS>(r[u], blk[u], R, row[u], st, rstage, chstage, c8);
+    __syncwarp();
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(256) reproject_kernel(const Geom G, const State S, int g, const SeqList L,
                                                         const __nv_bfloat16* __restrict__ old_k,
                                                         const __nv_bfloat16* __restrict__ old_v) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int seq = L.seq[blockIdx.x], h = blockIdx.y;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = (int)(blockDim.x >> 5);
+    const int z = (int)(blockIdx.z & 1u), part = (int)(blockIdx.z >> 1), nparts = (int)(gridDim.z >> 1);
     const int RM = G.r_max, P = G.r_max + 2;
-    __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem);                   // new [z][d][P]
-    __nv_bfloat16* bo = reinterpret_cast<__nv_bfloat16*>(smem + encode_smem_bytes(G.r_max));  // old [z][d][P]
-    const size_t boff = ((size_t)g * G.Hkv + h) * kD * RM;
-    for (int e = tid; e < 2 * kD * RM; e += blockDim.x) {
-        const int zz = e / (kD * RM), ev = e % (kD * RM), i = ev / RM, j = ev % RM;
-        bs[(size_t)zz * kD * P + (size_t)i * P + j] = (zz ? S.basis_v : S.basis_k)[boff + ev];
-        bo[(size_t)zz * kD * P + (size_t)i * P + j] = (zz ? old_v : old_k)[(size_t)h * kD * RM + ev];
+    __nv_bfloat16* bn = reinterpret_cast<__nv_bfloat16*>(smem);                   // new basis of side z [d][P]
+    __nv_bfloat16* bo = bn + (size_t)kD * P;                                       // previous basis of side z
+    uint8_t* ws = smem + (size_t)2 * kD * P * 2 + (size_t)warp * kRpWarpBytes;
+    float* xs = reinterpret_cast<float*>(ws);                                     // [group][kRpXPitch]
+    float* cs = xs + kRpMaxGroup * kRpXPitch;                                      // [group][64]
+    float* rstage = cs + kRpMaxGroup * 64;                                         // [32]
+    uint8_t* chstage = reinterpret_cast<uint8_t*>(rstage + 32);                    // [32]
+    uint8_t** gblk = reinterpret_cast<uint8_t**>(chstage + 32);                    // [group]
+    int* grow = reinterpret_cast<int*>(gblk + kRpMaxGroup);                        // [group]
+    {
+        const __nv_bfloat16* src_new = (z ? S.basis_v : S.basis_k) + ((size_t)g * G.Hkv + h) * kD * RM;
+        const __nv_bfloat16* src_old = (z ? old_v : old_k) + (size_t)h * kD * RM;
+        for (int e = tid; e < kD * RM; e += blockDim.x) {
+            const int i = e / RM, j = e % RM;
+            bn[(size_t)i * P + j] = src_new[e];
+            bo[(size_t)i * P + j] = src_old[e];
+        }
     }
-    __shared__ uint32_t s_cnt[kMaxTiers], s_base[kMaxTiers + 1];
+    // groups of a tier: ceil(count / V) per layer of the window
+    __shared__ uint32_t s_cnt[kMaxTiers], s_gbase[kMaxTiers + 1];
     if (tid == 0) {
         uint32_t acc = 0;
         for (int k = 0; k < kMaxTiers; ++k) {
-            s_cnt[k] = k < G.ntiers ? S.counts[cnt_index(G, seq, g, h) + k] : 0u;
-            s_base[k] = acc;
-            acc += s_cnt[k];
+            const uint32_t c = k < G.ntiers ? S.counts[cnt_index(G, seq, g, h) + k] : 0u;
+            const uint32_t vk = k < G.ntiers ? (uint32_t)min(kRpMaxGroup, 64 / G.tiers[k]) : 1u;
+            s_cnt[k] = c;
+            s_gbase[k] = acc;
+            acc += (c + vk - 1u) / vk * (uint32_t)G.LPG;
         }
-        s_base[kMaxTiers] = acc;
+        s_gbase[kMaxTiers] = acc;
     }
     __syncthreads();
-    const uint32_t units = s_base[kMaxTiers] * (uint32_t)G.LPG * 2u;
-    const uint32_t nw = (blockDim.x >> 5) * gridDim.z;
-    for (uint32_t u = blockIdx.z * (blockDim.x >> 5) + warp; u < units; u += nw) {
-        const uint32_t z = u & 1u, lig = (u >> 1) % (uint32_t)G.LPG, slotg = (u >> 1) / (uint32_t)G.LPG;
+    const uint32_t groups = s_gbase[kMaxTiers];
+    for (uint32_t gi = (uint32_t)(part * nwarps + warp); gi < groups; gi += (uint32_t)(nwarps * nparts)) {
         int k = 0;
-        while (k + 1 < kMaxTiers && slotg >= s_base[k + 1]) ++k;
-        const uint32_t slot = slotg - s_base[k];
-        const int R = G.tiers[k], st = G.ts[k], row = (int)(slot % kPage);
-        const uint32_t unit = S.pages[page_index(G, seq, g, h, k) + slot / kPage];
-        uint8_t* blk = S.data + (size_t)unit * kUnit + (size_t)lig * G.chunk_bytes[k] + (z ? G.blk_bytes[k] : 0u);
-        // reconstruction on the previous basis (fixed fp32 order), rounded to bf16.  The
-        // token's coefficients and residual entries are read in parallel (lane j holds entry j
-        // and j + 32) and handed round by shuffles: the chain's order is unchanged.
-        const __nv_bfloat16* bz = bo + (size_t)z * kD * P;
-        const float cl0 = lane < R ? stored_coeff(blk, G.c8, (int)z, R, row, lane) : 0.f;
-        const float cl1 = lane + 32 < R ? stored_coeff(blk, G.c8, (int)z, R, row, lane + 32) : 0.f;
-        int ch_l = 0;
-        float v_l = 0.f;
-        if (st > 0 && lane < st) stored_resid<BITS>(blk, G.c8, R, st, row, lane, ch_l, v_l);
-        float a[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < R; j += 2) {                     // R is even: the basis read a pair at a time
-            const float cj = __shfl_sync(0xffffffffu, j < 32 ? cl0 : cl1, j & 31);
-            const float cj1 = __shfl_sync(0xffffffffu, j + 1 < 32 ? cl0 : cl1, (j + 1) & 31);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(bz + (size_t)(lane + 32 * m) * P + j);
-                a[m] = __fmaf_rn(bf16lo(w), cj, a[m]);
-                a[m] = __fmaf_rn(bf16hi(w), cj1, a[m]);
-            }
+        while (k + 1 < kMaxTiers && gi >= s_gbase[k + 1]) ++k;
+        const uint32_t loc = gi - s_gbase[k];
+        const int R = G.tiers[k], Vk = min(kRpMaxGroup, 64 / R);
+        const uint32_t lig = loc % (uint32_t)G.LPG, first = loc / (uint32_t)G.LPG * (uint32_t)Vk;
+        const int nu = (int)min((uint32_t)Vk, s_cnt[k] - first);
+        if (lane < kRpMaxGroup) {                        // the group's blocks and rows
+            const uint32_t slot = first + (uint32_t)min(lane, nu - 1);
+            const uint32_t unit = S.pages[page_index(G, seq, g, h, k) + slot / kPage];
+            gblk[lane] = S.data + (size_t)unit * kUnit + (size_t)lig * G.chunk_bytes[k] + (z ? G.blk_bytes[k] : 0u);
+            grow[lane] = (int)(slot % kPage);
         }
-        for (int e = 0; e < st; ++e) {
-            const int ch = __shfl_sync(0xffffffffu, ch_l, e);
-            const float v = __shfl_sync(0xffffffffu, v_l, e);
-            if ((ch & 31) == lane && ch < kD) {
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    if ((ch >> 5) == m) a[m] = __fadd_rn(a[m], v);
-            }
-        }
-        __syncwarp();                                        // every lane has read the old bytes
-        UnitIn in;
-        in.ok = true;
-        in.dbg = nullptr;
-        in.dst.blk = S.data + (size_t)unit * kUnit + (size_t)lig * G.chunk_bytes[k];
-        in.dst.k = k;
-        in.dst.row = row;
-        in.dst.R = R;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) in.xr[m] = __bfloat162float(__float2bfloat16_rn(a[m]));
-        encode_body<BITS>(G, S, bs, enc_scratch(G, smem, warp), (int)z, in);
+        __syncwarp();
+        if (Vk == 4) reproject_group<BITS, 4>(G, z, k, nu, gblk, grow, bn, bo, xs, cs, rstage, chstage);
+        else if (Vk == 2) reproject_group<BITS, 2>(G, z, k, nu, gblk, grow, bn, bo, xs, cs, rstage, chstage);
+        else reproject_group<BITS, 1>(G, z, k, nu, gblk, grow, bn, bo, xs, cs, rstage, chstage);
     }
 }
 
