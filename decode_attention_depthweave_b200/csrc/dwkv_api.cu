@@ -676,26 +676,26 @@ dwkv_status dwkv_basis_update(dwkv_handle h, int32_t group, int32_t n_rows, cons
     DWKV_CUDA(cudaMemcpyAsync(old + ng * bbytes, h->arena + h->meta.basis_v + (size_t)g0 * bbytes, ng * bbytes,
                               cudaMemcpyDeviceToDevice, s), "save the V bases");
     if ((st = launch_basis(h, g0, ng, nullptr, 0, eigenvalues, s)) != DWKV_OK) return st;
-    const size_t sm = reproject_smem_bytes(G.r_max, 8);
+    const size_t sm = reproject_smem_bytes(G.r_max, 12);
     auto kern = G.bits == 8 ? reproject_kernel<8> : reproject_kernel<4>;
     DWKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm),
               "reproject_kernel shared memory");
     int resident = 0;
-    DWKV_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, 256, sm), "reproject_kernel occupancy");
+    DWKV_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, 384, sm), "reproject_kernel occupancy");
     resident = std::max(1, resident) * h->num_sms;
     for (int i0 = 0; i0 < n_seqs; i0 += kMaxSeqs) {
         SeqList L;
         memset(&L, 0, sizeof(L));
         L.n = std::min(kMaxSeqs, n_seqs - i0);
         for (int i = 0; i < L.n; ++i) L.seq[i] = seq_ids[i0 + i];
-        // blocks per (sequence, kv-head, side): one wave of resident blocks over the call (the
-        // units of a (sequence, kv-head, side) are dealt evenly over its blocks' warps, so a
-        // second, partial wave would finish a whole block time later)
-        const int per = std::max(1, resident / (2 * L.n * G.Hkv));
+        // blocks per (sequence, kv-head, side): about eight waves of resident blocks over the
+        // call, so that blocks finishing at different times leave the SMs evenly loaded (one
+        // block's two bases are ~1 % of its work)
+        const int per = std::max(1, (8 * resident + 2 * L.n * G.Hkv - 1) / (2 * L.n * G.Hkv));
         for (int g = g0; g < g0 + ng; ++g) {
             const __nv_bfloat16* ok_ = reinterpret_cast<const __nv_bfloat16*>(old + (size_t)(g - g0) * bbytes);
             const __nv_bfloat16* ov_ = reinterpret_cast<const __nv_bfloat16*>(old + (size_t)(ng + g - g0) * bbytes);
-            kern<<<dim3(L.n, G.Hkv, 2 * per), 256, sm, s>>>(G, h->st, g, L, ok_, ov_);
+            kern<<<dim3(L.n, G.Hkv, 2 * per), 384, sm, s>>>(G, h->st, g, L, ok_, ov_);
             DWKV_CUDA(cudaGetLastError(), "reproject_kernel launch");
         }
     }

@@ -334,19 +334,21 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
 // Slots and counts do not change.  Online bases have r_max <= 64.
 // ------------------------------------------------------------------------------------
 constexpr int kRpMaxGroup = 4;
+constexpr int kRpThreads = 384;                    // 12 warps, 2 blocks an SM
 constexpr int kRpXPitch = kD + 4;                  // floats: group rows on distinct banks
 constexpr uint32_t kRpWarpBytes = (uint32_t)(kRpMaxGroup * kRpXPitch + kRpMaxGroup * 64 + 32) * 4u + 32u +
                                    (uint32_t)kRpMaxGroup * 16u;   // + the group's block addresses and rows
 
-// Dynamic shared memory of reproject_kernel: the side's two bases [d][r_max + 2], then each
-// warp's group scratch.
+// Dynamic shared memory of reproject_kernel: the side's two bases as fp32 [d][r_max + 2] (the
+// bf16 values exactly; a 64-bit load takes a pair of coefficients, and with the row pitch of
+// r_max + 2 words a half warp's rows fall on distinct banks), then each warp's group scratch.
 size_t reproject_smem_bytes(int r_max, int warps) {
-    return (size_t)2 * kD * (r_max + 2) * 2 + (size_t)warps * kRpWarpBytes;
+    return (size_t)2 * kD * (r_max + 2) * 4 + (size_t)warps * kRpWarpBytes;
 }
 
 template <int BITS, int V>
 __device__ __forceinline__ void reproject_group(const Geom& G, int z, int k, int nu, uint8_t* const* blk,
-                                                const int* row, const __nv_bfloat16* bn, const __nv_bfloat16* bo,
+                                                const int* row, const float* bn, const float* bo,
                                                 float* xs, float* cs, float* rstage, uint8_t* chstage) {
     const int lane = threadIdx.x & 31;
     const int P = G.r_max + 2, R = G.tiers[k], st = G.ts[k], c8 = G.c8;
@@ -372,17 +374,17 @@ __device__ __forceinline__ void reproject_group(const Geom& G, int z, int k, int
 #pragma unroll
             for (int m = 0; m < 4; ++m) a[u][m] = 0.f;
         for (int j = 0; j < R; j += 2) {                 // R is even: the basis read a pair at a time
-            uint32_t w[4];
+            float2 w[4];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) w[m] = *reinterpret_cast<const uint32_t*>(bo + (size_t)(lane + 32 * m) * P + j);
+            for (int m = 0; m < 4; ++m) w[m] = *reinterpret_cast<const float2*>(bo + (size_t)(lane + 32 * m) * P + j);
 #pragma unroll
             for (int u = 0; u < V; ++u) {
                 const float cj = __shfl_sync(0xffffffffu, j < 32 ? cl0[u] : cl1[u], j & 31);
                 const float cj1 = __shfl_sync(0xffffffffu, j + 1 < 32 ? cl0[u] : cl1[u], (j + 1) & 31);
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
-                    a[u][m] = __fmaf_rn(bf16lo(w[m]), cj, a[u][m]);
-                    a[u][m] = __fmaf_rn(bf16hi(w[m]), cj1, a[u][m]);
+                    a[u][m] = __fmaf_rn(w[m].x, cj, a[u][m]);
+                    a[u][m] = __fmaf_rn(w[m].y, cj1, a[u][m]);
                 }
             }
         }
@@ -434,9 +436,9 @@ __device__ __forceinline__ void reproject_group(const Geom& G, int z, int k, int
             const float xq[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(bn + (size_t)(i + ii) * P + j);
-                acc0 = __fmaf_rn(bf16lo(w), xq[ii], acc0);
-                acc1 = __fmaf_rn(bf16hi(w), xq[ii], acc1);
+                const float2 w = *reinterpret_cast<const float2*>(bn + (size_t)(i + ii) * P + j);
+                acc0 = __fmaf_rn(w.x, xq[ii], acc0);
+                acc1 = __fmaf_rn(w.y, xq[ii], acc1);
             }
         }
         float* cv = cs + (v < V ? v : 0) * 64;
@@ -483,16 +485,16 @@ __device__ __forceinline__ void reproject_group(const Geom& G, int z, int k, int
         for (int j0 = 0; j0 < R; j0 += 8) {              // R is a multiple of 8
 #pragma unroll
             for (int jj = 0; jj < 8; jj += 2) {
-                uint32_t w[4];
+                float2 w[4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) w[m] = *reinterpret_cast<const uint32_t*>(bn + (size_t)(lane + 32 * m) * P + j0 + jj);
+                for (int m = 0; m < 4; ++m) w[m] = *reinterpret_cast<const float2*>(bn + (size_t)(lane + 32 * m) * P + j0 + jj);
 #pragma unroll
                 for (int u = 0; u < V; ++u) {
                     const float2 c2 = *reinterpret_cast<const float2*>(cs + u * 64 + j0 + jj);
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        a[u][m] = __fmaf_rn(bf16lo(w[m]), c2.x, a[u][m]);
-                        a[u][m] = __fmaf_rn(bf16hi(w[m]), c2.y, a[u][m]);
+                        a[u][m] = __fmaf_rn(w[m].x, c2.x, a[u][m]);
+                        a[u][m] = __fmaf_rn(w[m].y, c2.y, a[u][m]);
                     }
                 }
             }
@@ -510,7 +512,7 @@ __device__ __forceinline__ void reproject_group(const Geom& G, int z, int k, int
 }
 
 template <int BITS>
-__global__ void __launch_bounds__(256) reproject_kernel(const Geom G, const State S, int g, const SeqList L,
+__global__ void __launch_bounds__(kRpThreads, 2) reproject_kernel(const Geom G, const State S, int g, const SeqList L,
                                                         const __nv_bfloat16* __restrict__ old_k,
                                                         const __nv_bfloat16* __restrict__ old_v) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -518,9 +520,9 @@ __global__ void __launch_bounds__(256) reproject_kernel(const Geom G, const Stat
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = (int)(blockDim.x >> 5);
     const int z = (int)(blockIdx.z & 1u), part = (int)(blockIdx.z >> 1), nparts = (int)(gridDim.z >> 1);
     const int RM = G.r_max, P = G.r_max + 2;
-    __nv_bfloat16* bn = reinterpret_cast<__nv_bfloat16*>(smem);                   // new basis of side z [d][P]
-    __nv_bfloat16* bo = bn + (size_t)kD * P;                                       // previous basis of side z
-    uint8_t* ws = smem + (size_t)2 * kD * P * 2 + (size_t)warp * kRpWarpBytes;
+    float* bn = reinterpret_cast<float*>(smem);                                   // new basis of side z [d][P]
+    float* bo = bn + (size_t)kD * P;                                               // previous basis of side z
+    uint8_t* ws = smem + (size_t)2 * kD * P * 4 + (size_t)warp * kRpWarpBytes;
     float* xs = reinterpret_cast<float*>(ws);                                     // [group][kRpXPitch]
     float* cs = xs + kRpMaxGroup * kRpXPitch;                                      // [group][64]
     float* rstage = cs + kRpMaxGroup * 64;                                         // [32]
@@ -532,8 +534,8 @@ __global__ void __launch_bounds__(256) reproject_kernel(const Geom G, const Stat
         const __nv_bfloat16* src_old = (z ? old_v : old_k) + (size_t)h * kD * RM;
         for (int e = tid; e < kD * RM; e += blockDim.x) {
             const int i = e / RM, j = e % RM;
-            bn[(size_t)i * P + j] = src_new[e];
-            bo[(size_t)i * P + j] = src_old[e];
+            bn[(size_t)i * P + j] = __bfloat162float(src_new[e]);
+            bo[(size_t)i * P + j] = __bfloat162float(src_old[e]);
         }
     }
     // groups of a tier: ceil(count / V) per layer of the window
