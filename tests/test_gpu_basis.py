@@ -12,7 +12,7 @@ import torch
 import oracle
 import synth
 from oracle import basis as ob
-from helpers import cat_comp, cfg_for, check_close, head_problem, oracle_encode_rows
+from helpers import cat_comp, cfg_for, check_close, head_problem, oracle_encode_rows, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -279,3 +279,59 @@ def test_update_before_any_sketch_averages_from_zero():
             want = 0.25 * ob.gram(_f64(rows[:, :, h].reshape(-1, wl.head_dim)))
             got = mom[h, z].cpu().numpy().astype(np.float64)
             assert np.linalg.norm(got - want) <= 1e-5 * np.linalg.norm(want), (h, z)
+
+
+@pytest.mark.parametrize("coeff_bits", [16, 8])
+def test_update_reprojects_tokens_with_repeated_residual_channels(coeff_bits):
+    """Stored tokens whose residual entries repeat a channel (the format allows it; decode sums
+    them): the re-projection adds such a token's entries one at a time in entry order, as the
+    oracle's reconstruction does, and the other tokens of its warp's group by the scatter.
+    Every token, head and side is checked bit for bit."""
+    wl = _wl(coeff_bits=coeff_bits)
+    bases = synth.make_bases(wl)
+    lengths = [300, 150]
+    cache = dw.Cache(cfg_for(wl, max_context=400), bases[0], bases[1])
+    for seq, T in enumerate(lengths):
+        tiers = synth.make_tiers(wl, seq, 0, T)
+        for layer in range(2):
+            comp = synth.make_compressed(wl, seq, layer, tiers)
+            idx = comp["idx"].clone()
+            idx[::3, :, :, 1] = idx[::3, :, :, 0]          # every third token: entry 1 repeats entry 0's
+            idx[::3, :, :, -1] = idx[::3, :, :, 2]         # channel, the last entry repeats entry 2's
+            comp["idx"] = idx
+            c = to_dev(comp)
+            coeff = (c["ccodes"], c["cscales"]) if "ccodes" in c else c["coeff"]
+            cache.append_compressed(layer, [seq], [T], tiers.cuda().contiguous(), coeff, c["idx"], c["codes"],
+                                    c["scales"])
+    cache.sync()
+    before = {(b, layer): {k_: v_.cpu() for k_, v_ in cache.export(layer, b, 0, n).items()}
+              for b, n in enumerate(lengths) for layer in range(2)}
+    assert (before[(0, 0)]["idx"][0, 0, 0, 1] == before[(0, 0)]["idx"][0, 0, 0, 0]).item()
+    wl2 = wl.scaled(base_seed=wl.base_seed + 55)
+    _, k_new, v_new = _rows(wl2, synth.make_bases(wl2), [200], start=1000)
+    cache.basis_update(0, k_new.cuda(), v_new.cuda(), 0.0, [0, 1])
+    bk1, bv1 = cache.bases(0)
+    cache.sync()
+    new = (bk1.cpu(), bv1.cpu())
+    old = (bases[0][0], bases[1][0])
+    for (b, layer), oc in before.items():
+        got = {k_: v_.cpu() for k_, v_ in cache.export(layer, b, 0, lengths[b]).items()}
+        for t in range(lengths[b]):
+            for h in range(wl.num_kv_heads):
+                r = wl.tiers[int(oc["tier_idx"][t, h])]
+                for z in range(2):
+                    what = (b, layer, t, h, z)
+                    args = (oc["idx"][t, h, z], oc["codes"][t, h, z], oc["scales"][t, h, z], r, wl.resid_bits)
+                    if coeff_bits == 8:
+                        ref = oracle.reencode_vector8(old[z][h], r, oc["ccodes"][t, h, z], oc["cscales"][t, h, z], *args,
+                                                      basis_new=new[z][h])
+                        assert np.array_equal(got["ccodes"][t, h, z].numpy(), ref["ccodes"]), what
+                        assert np.array_equal(got["cscales"][t, h, z].view(torch.int16).numpy().view(np.uint16),
+                                              ref["cscales"]), what
+                    else:
+                        ref = oracle.reencode_vector(old[z][h], r, oc["coeff"][t, h, z], *args, basis_new=new[z][h])
+                        assert np.array_equal(got["coeff"][t, h, z].view(torch.int16).numpy().view(np.uint16),
+                                              ref["coeff"]), what
+                    assert np.array_equal(got["idx"][t, h, z].numpy(), ref["idx"]), what
+                    assert np.array_equal(got["codes"][t, h, z].numpy(), ref["codes"]), what
+                    assert (int(got["scales"][t, h, z].view(torch.int16).item()) & 0xffff) == int(ref["scale"]), what
