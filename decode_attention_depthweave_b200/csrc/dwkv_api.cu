@@ -35,7 +35,7 @@ __global__ void retier_kernel(const Geom, const State, const RetierCall, const i
 __global__ void retier_release_kernel(const Geom, const State, const RetierCall);
 __global__ void wait_timeout_kernel(const State, uint64_t);
 __global__ void tile_basis_kernel(const Geom, const State);
-__global__ void gram_kernel(const Geom, int, const __nv_bfloat16*, const __nv_bfloat16*, float*, float);
+__global__ void gram_kernel(const Geom, const State, int, const __nv_bfloat16*, const __nv_bfloat16*, float*, float);
 __global__ void moment_scale_kernel(float*, size_t, float);
 __global__ void basis_kernel(const Geom, const State, int, const float*, const float*, int, float*);
 template <int BITS>
@@ -43,6 +43,7 @@ __global__ void reproject_kernel(const Geom, const State, int, const SeqList, co
                                  const __nv_bfloat16*);
 size_t basis_smem_bytes(int r);
 size_t reproject_smem_bytes(int r_max, int warps);
+size_t gram_smem_bytes();
 template <int BITS, bool PROBE, int RMAX, int S, bool C8>
 __global__ void decode_kernel(const Geom, const State, const DecodeCall);
 }  // namespace dwkv
@@ -601,11 +602,18 @@ dwkv_status launch_gram(dwkv_handle h, int g0, int ng, int32_t n_rows, const voi
     const Geom& G = h->geom;
     if (n_rows == 0) return DWKV_OK;
     const long long rows = (long long)G.LPG * n_rows;
-    const long long want = std::max(1ll, 2ll * h->num_sms / (2ll * G.Hkv * ng));
+    const size_t sm = gram_smem_bytes();
+    DWKV_CUDA(cudaFuncSetAttribute(gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm),
+              "gram_kernel shared memory");
+    // blocks per (window, kv-head, side): about 4 an SM over the call (the most that fit: the
+    // stage buffers keep a block's share of an SM's shared memory above a quarter, so the
+    // blocks' tensor-memory columns, 128 each, never exceed the SM's 512)
+    const long long combos = 2ll * G.Hkv * ng;
+    const long long want = std::max(1ll, 4ll * h->num_sms / combos);
     const int nblk = (int)std::min(want, (rows + 63) / 64);
-    gram_kernel<<<dim3(nblk, G.Hkv * ng, 2), 256, 0, s>>>(G, n_rows, static_cast<const __nv_bfloat16*>(k_rows),
-                                                          static_cast<const __nv_bfloat16*>(v_rows), moment_of(h, g0),
-                                                          scale);
+    gram_kernel<<<dim3(nblk, G.Hkv * ng, 2), 128, sm, s>>>(G, h->st, n_rows, static_cast<const __nv_bfloat16*>(k_rows),
+                                                           static_cast<const __nv_bfloat16*>(v_rows), moment_of(h, g0),
+                                                           scale);
     DWKV_CUDA(cudaGetLastError(), "gram_kernel launch");
     return DWKV_OK;
 }

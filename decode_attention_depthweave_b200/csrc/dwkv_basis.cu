@@ -18,71 +18,166 @@ namespace dwkv {
 
 // ------------------------------------------------------------------------------------
 // Second moment C[w][h][z] += scale * X^T X over the rows of window w's layers (rows = LPG x
-// n_rows, layer-major; blockIdx.y = w Hkv + h), on the tensor cores.  A block of 8 warps: warp w
-// owns channels [16 w, 16 w + 16) of C's rows and all 128 columns (16 n-tiles); chunks of 64
-// rows are staged as bf16 [64][136] (a 272-byte pitch: ldmatrix rows on distinct banks).
-// Partial sums go to C with fp32 atomics, so the order of the sum is not fixed.
+// n_rows, layer-major; blockIdx.y = w Hkv + h) on the 5th-generation tensor cores: X^T X is
+// one 128 x 128 x 64 product per chunk of 64 rows, accumulated in tensor memory.
+//  - A block of 4 warps holds 128 TMEM columns (the fp32 128 x 128 accumulator, row i in lane
+//    i) and kGramStages chunk buffers in shared memory.
+//  - A chunk is staged by 16-byte cp.async copies in the MN-major layout without swizzle:
+//    8 x 8 core matrices of 8 rows (K) x 8 channels (16 bytes, contiguous), channel blocks
+//    kGramSbo bytes apart and row blocks kGramLbo apart.  A = X^T (M = channels, MN-major)
+//    and B = X (N = channels, MN-major) are the same bytes under the same descriptor.
+//  - One thread issues the chunk's four K = 16 MMAs and commits them to the buffer's
+//    mbarrier; the buffer is refilled only after that commit has arrived.
+//  - After the last chunk each warp reads its 32 rows with tcgen05.ld and adds them into C with
+//    fp32 atomics, so the order of the sum is not fixed.
+// Every wait is bounded: a wait that runs out records DWKV_DEV_TIMEOUT, waits (bounded) for the
+// MMAs issued so far, frees the tensor memory and leaves C unchanged by this block.
 // ------------------------------------------------------------------------------------
-constexpr int kGramRows = 64;
-constexpr int kGramPitch = kD + 8;
-__global__ void __launch_bounds__(256) gram_kernel(const Geom G, int n_rows, const __nv_bfloat16* __restrict__ k_rows,
+constexpr int kGramRows = 64;                      // K of a chunk
+constexpr int kGramStages = 3;
+constexpr uint32_t kGramStageBytes = (uint32_t)kGramRows * kD * 2u;         // 16 KB
+constexpr uint32_t kGramSbo = 128u;                // channel-block stride (8 channels x 8 rows x 2 B)
+constexpr uint32_t kGramLbo = (uint32_t)(kD / 8) * kGramSbo;                // row-block stride: 2048 B
+constexpr uint32_t kGramTmemCols = 128u;
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits 4-5 = 1), A and B
+// bf16 (bits 7-9 = 1, 10-12 = 1), A and B MN-major (bits 15, 16), N >> 3 = 16 (bits 17-22),
+// M >> 4 = 8 (bits 24-28).
+constexpr uint32_t kGramIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                                ((uint32_t)(kD >> 3) << 17) | ((uint32_t)(kD >> 4) << 24);
+
+size_t gram_smem_bytes() { return (size_t)kGramStages * kGramStageBytes + 64; }
+
+// Shared-memory matrix descriptor, no swizzle: start address, leading (K-block) and stride
+// (MN-block) byte offsets, each >> 4, and the descriptor version 1 (bits 46-47).
+__device__ __forceinline__ uint64_t gram_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)((kGramLbo >> 4) & 0x3fffu) << 16) |
+           ((uint64_t)((kGramSbo >> 4) & 0x3fffu) << 32) | (1ull << 46);
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__global__ void __launch_bounds__(128) gram_kernel(const Geom G, const State S, int n_rows,
+                                                   const __nv_bfloat16* __restrict__ k_rows,
                                                    const __nv_bfloat16* __restrict__ v_rows, float* __restrict__ cacc,
                                                    float scale) {
-    __shared__ __align__(16) __nv_bfloat16 xs[kGramRows * kGramPitch];
+    extern __shared__ __align__(128) uint8_t gsm[];
     const int h = blockIdx.y % G.Hkv, gw = blockIdx.y / G.Hkv, z = blockIdx.z;   // gw: window within the call
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, c = lane & 3, mi = lane >> 3, rr = lane & 7;
     const __nv_bfloat16* src = (z ? v_rows : k_rows) + (size_t)gw * G.LPG * n_rows * G.Hkv * kD;
-    cacc += (size_t)gw * G.Hkv * 2 * kD * kD;
     const long long total = (long long)G.LPG * n_rows;
     const long long per = (total + gridDim.x - 1) / gridDim.x;
     const long long r0 = (long long)blockIdx.x * per, r1 = r0 + per < total ? r0 + per : total;
-    float acc[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-    const uint32_t xaddr = smem_addr(xs);
-    for (long long b0 = r0; b0 < r1; b0 += kGramRows) {
-        __syncthreads();
-        // stage 64 rows x 128 channels (16-byte loads; rows past the range as zeros)
+    const int nchunks = r1 > r0 ? (int)((r1 - r0 + kGramRows - 1) / kGramRows) : 0;
+    if (nchunks == 0) return;                                   // uniform over the block
+    const uint32_t sbase = smem_addr(gsm);
+    const uint32_t bars = sbase + (uint32_t)kGramStages * kGramStageBytes;     // kGramStages mbarriers
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + kGramStages * kGramStageBytes + 8 * kGramStages);
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                     "r"(kGramTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        for (int b = 0; b < kGramStages; ++b) mbar_init(bars + 8u * b, 1u);
+        fence_mbar_init();
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    // stage chunk q (rows past the range as zeros) into buffer q % kGramStages
+    auto stage = [&](int q) {
+        const long long b0 = r0 + (long long)q * kGramRows;
+        const uint32_t buf = sbase + (uint32_t)(q % kGramStages) * kGramStageBytes;
         for (int e = tid; e < kGramRows * (kD / 8); e += blockDim.x) {
-            const int r = e / (kD / 8), q = e % (kD / 8);
-            const long long row = b0 + r;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (row < r1) {
-                const long long layer = row / n_rows, t = row % n_rows;
-                v = __ldg(reinterpret_cast<const uint4*>(src + ((layer * n_rows + t) * G.Hkv + h) * kD) + q);
-            }
-            *reinterpret_cast<uint4*>(xs + r * kGramPitch + 8 * q) = v;
+            const int k = e / (kD / 8), mb = e % (kD / 8);         // row k of the chunk, channels 8 mb ..
+            const long long row = b0 + k;
+            const bool ok = row < r1;
+            const long long layer = ok ? row / n_rows : 0, t = ok ? row % n_rows : 0;
+            const __nv_bfloat16* p = src + ((layer * n_rows + t) * G.Hkv + h) * kD + 8 * mb;
+            cp_async16(buf + (uint32_t)mb * kGramSbo + (uint32_t)(k >> 3) * kGramLbo + (uint32_t)(k & 7) * 16u, p,
+                       ok ? 16u : 0u);
         }
-        __syncthreads();
+    };
+    bool ok = true;
+    int issued = 0;                                                       // chunks whose MMAs were issued
 #pragma unroll
-        for (int ks = 0; ks < kGramRows / 16; ++ks) {
-            // A = X^T rows [16 warp, +16) x rows t [16 ks, +16): transposed 8x8 tiles of X
-            uint32_t a[4];
-            {
-                const int t = 16 * ks + 8 * (mi >> 1) + rr, i0 = 16 * warp + 8 * (mi & 1);
-                ldsm_x4_t(xaddr + (uint32_t)(t * kGramPitch + i0) * 2u, a);
+    for (int q = 0; q < kGramStages - 1; ++q) {
+        if (q < nchunks) stage(q);
+        cp_async_commit();
+    }
+    for (int q = 0; q < nchunks && ok; ++q) {
+        // the buffer of chunk q + stages - 1 held chunk q - 1: its MMAs must have completed
+        const int nq = q + kGramStages - 1;
+        if (nq < nchunks) {
+            if (q >= 1 && !mbar_wait(bars + 8u * (uint32_t)((q - 1) % kGramStages), (uint32_t)(((q - 1) / kGramStages) & 1))) {
+                ok = false;
+            } else {
+                stage(nq);
             }
+        }
+        cp_async_commit();
+        cp_async_wait<kGramStages - 1>();                                 // this thread's part of chunk q
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");      // visible to the tensor cores
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        issued = q + 1;
+        if (tid == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t buf = sbase + (uint32_t)(q % kGramStages) * kGramStageBytes;
 #pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                // B = X rows t x channels [16 np, +16): two n-tiles from one x4.trans
-                uint32_t b4[4];
-                const int t = 16 * ks + 8 * (mi & 1) + rr, j0 = 16 * np + 8 * (mi >> 1);
-                ldsm_x4_t(xaddr + (uint32_t)(t * kGramPitch + j0) * 2u, b4);
-                const uint32_t b0[2] = {b4[0], b4[1]}, b1[2] = {b4[2], b4[3]};
-                mma_bf16(acc[2 * np], a, b0);
-                mma_bf16(acc[2 * np + 1], a, b1);
+            for (int kk = 0; kk < kGramRows / 16; ++kk) {
+                const uint64_t d = gram_desc(buf + (uint32_t)kk * 2u * kGramLbo);   // rows 16 kk .. 16 kk + 15
+                const uint32_t acc = (q > 0 || kk > 0) ? 1u : 0u;
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\t"
+                    "setp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                    ::"r"(tmem), "l"(d), "l"(d), "r"(kGramIdesc), "r"(acc) : "memory");
             }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             bars + 8u * (uint32_t)(q % kGramStages))
+                         : "memory");
         }
     }
-    float* dst = cacc + ((size_t)h * 2 + z) * kD * kD;
+    cp_async_wait<0>();
+    // the last commit covers every MMA this block issued (bounded: on a timeout the tensor
+    // memory is still freed below, after this wait has given the MMAs its full limit)
+    bool done = issued > 0 && mbar_wait(bars + 8u * (uint32_t)((issued - 1) % kGramStages),
+                                        (uint32_t)(((issued - 1) / kGramStages) & 1));
+    done = __syncthreads_and(done && ok && issued == nchunks) != 0;
+    if (!done) {
+        if (tid == 0) set_dev_error(S, 6u /*DWKV_DEV_TIMEOUT*/, 0x67u, (uint32_t)blockIdx.y);
+    } else {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        float* dst = cacc + (size_t)gw * G.Hkv * 2 * kD * kD + ((size_t)h * 2 + z) * kD * kD +
+                     (size_t)(32 * warp + lane) * kD;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kD; c0 += 32) {
+            uint32_t v[32];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+                "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                  "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                  "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+                  "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                : "r"(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        const int i0 = 16 * warp + g, j0 = 8 * n + 2 * c;
-        atomicAdd(dst + (size_t)i0 * kD + j0, scale * acc[n][0]);
-        atomicAdd(dst + (size_t)i0 * kD + j0 + 1, scale * acc[n][1]);
-        atomicAdd(dst + (size_t)(i0 + 8) * kD + j0, scale * acc[n][2]);
-        atomicAdd(dst + (size_t)(i0 + 8) * kD + j0 + 1, scale * acc[n][3]);
+            for (int j = 0; j < 32; ++j) atomicAdd(dst + c0 + j, scale * __uint_as_float(v[j]));
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGramTmemCols) : "memory");
     }
 }
 
