@@ -89,18 +89,20 @@ __global__ void __launch_bounds__(128) gram_kernel(const Geom G, const State S, 
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    // stage chunk q (rows past the range as zeros) into buffer q % kGramStages
+    // stage chunk q (rows past the range as zeros) into buffer q % kGramStages: thread t takes
+    // channels 8 (t % 16) .. + 7 of rows t / 16 + 8 i (row r of the window's rows is row r of
+    // the layer-major [LPG][n_rows] source)
+    const int mb = tid & 15, k0 = tid >> 4;
     auto stage = [&](int q) {
         const long long b0 = r0 + (long long)q * kGramRows;
-        const uint32_t buf = sbase + (uint32_t)(q % kGramStages) * kGramStageBytes;
-        for (int e = tid; e < kGramRows * (kD / 8); e += blockDim.x) {
-            const int k = e / (kD / 8), mb = e % (kD / 8);         // row k of the chunk, channels 8 mb ..
-            const long long row = b0 + k;
+        const uint32_t buf = sbase + (uint32_t)(q % kGramStages) * kGramStageBytes + (uint32_t)mb * kGramSbo +
+                             (uint32_t)k0 * 16u;
+#pragma unroll
+        for (int i = 0; i < kGramRows / 8; ++i) {
+            const long long row = b0 + k0 + 8 * i;
             const bool ok = row < r1;
-            const long long layer = ok ? row / n_rows : 0, t = ok ? row % n_rows : 0;
-            const __nv_bfloat16* p = src + ((layer * n_rows + t) * G.Hkv + h) * kD + 8 * mb;
-            cp_async16(buf + (uint32_t)mb * kGramSbo + (uint32_t)(k >> 3) * kGramLbo + (uint32_t)(k & 7) * 16u, p,
-                       ok ? 16u : 0u);
+            const __nv_bfloat16* p = src + ((ok ? row : 0) * G.Hkv + h) * kD + 8 * mb;
+            cp_async16(buf + (uint32_t)i * kGramLbo, p, ok ? 16u : 0u);
         }
     };
     bool ok = true;
