@@ -335,3 +335,33 @@ def test_update_reprojects_tokens_with_repeated_residual_channels(coeff_bits):
                     assert np.array_equal(got["idx"][t, h, z].numpy(), ref["idx"]), what
                     assert np.array_equal(got["codes"][t, h, z].numpy(), ref["codes"]), what
                     assert (int(got["scales"][t, h, z].view(torch.int16).item()) & 0xffff) == int(ref["scale"]), what
+
+
+@pytest.mark.parametrize("n_rows", [1, 7, 65, 1000])
+def test_moment_of_few_and_ragged_rows(n_rows):
+    """An update whose rows a layer leave a partial chunk of 64 (rows past the end staged as
+    zeros) or less than one chunk in all: C = 0.5 C_0 + 0.5 C_rows against the fp64 Gram of the
+    same rows, C_0 a sketched full-rank moment (a missing or doubled row would move C by far
+    more than the bound); an update with no rows only scales the moment."""
+    wl = _wl()
+    bases = synth.make_bases(wl)
+    cache = dw.Cache(cfg_for(wl, max_context=64), bases[0], bases[1])
+    _, k0, v0 = _rows(wl, bases, [200])
+    _, _, mom0 = _sketch(cache, wl, k0, v0, synth.make_test_matrix(wl))
+    wl2 = wl.scaled(base_seed=wl.base_seed + 3)
+    _, k_rows, v_rows = _rows(wl2, synth.make_bases(wl2), [n_rows], start=500)
+    cache.basis_update(0, k_rows.cuda(), v_rows.cuda(), 0.5, [])
+    mom = cache.moment(0)
+    cache.sync()
+    mom = mom.cpu()
+    for h in range(wl.num_kv_heads):
+        for z, rows in enumerate((k_rows, v_rows)):
+            g = 0.5 * ob.gram(_f64(rows[:, :, h].reshape(-1, wl.head_dim)))
+            want = 0.5 * mom0[h, z].numpy().astype(np.float64) + g
+            got = mom[h, z].numpy().astype(np.float64)
+            assert np.linalg.norm(got - want) <= 1e-5 * np.linalg.norm(want), (n_rows, h, z)
+            assert np.linalg.norm(g) > 1e-3 * np.linalg.norm(want)          # the rows' share is visible
+    cache.basis_update(0, None, None, 0.5, [])
+    mom2 = cache.moment(0)
+    cache.sync()
+    assert torch.equal(mom2.cpu(), 0.5 * mom)
