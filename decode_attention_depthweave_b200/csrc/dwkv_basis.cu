@@ -423,12 +423,16 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
 // basis (old_k / old_v: the fixed-order fp32 chain over its rank, plus scale x code on its
 // residual channels, rounded to bf16, as a re-tier does) and encoded on the new basis at its own
 // tier, in place, by the six encode steps in the encoders' operation order:
+//   0    the reconstructions share each basis load; the residual entries are added by a
+//        shared-memory scatter (in entry order where a token repeats a channel);
 //   1-2  lane (v, p) runs token v's projection chains of coefficients 2p and 2p + 1 over the
-//        channels in order (the bf16 basis read a pair at a time, x four channels a load), then
-//        rounds them to bf16 or forms their 8-bit blocks (a block of 16 on 8 lanes);
+//        channels in order (a coefficient pair of the basis one 64-bit load, x four channels
+//        a load), then rounds them to bf16 or forms their 8-bit blocks (a block of 16 on 8
+//        lanes);
 //   3    the residual chains of the group's tokens share each basis load;
 //   4-6  quantize_store per token.
-// Slots and counts do not change.  Online bases have r_max <= 64.
+// The block's two bases are held as fp32 (the bf16 values exactly).  Slots and counts do not
+// change.  Online bases have r_max <= 64.
 // ------------------------------------------------------------------------------------
 constexpr int kRpMaxGroup = 4;
 constexpr int kRpThreads = 384;                    // 12 warps, 2 blocks an SM
@@ -610,8 +614,8 @@ __device__ __forceinline__ void reproject_group(const Geom& G, int z, int k, int
 
 template <int BITS>
 __global__ void __launch_bounds__(kRpThreads, 2) reproject_kernel(const Geom G, const State S, int g, const SeqList L,
-                                                        const __nv_bfloat16* __restrict__ old_k,
-                                                        const __nv_bfloat16* __restrict__ old_v) {
+                                                                   const __nv_bfloat16* __restrict__ old_k,
+                                                                   const __nv_bfloat16* __restrict__ old_v) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int seq = L.seq[blockIdx.x], h = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = (int)(blockDim.x >> 5);
