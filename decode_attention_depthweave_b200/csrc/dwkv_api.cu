@@ -1,5 +1,7 @@
 // dwkv_api.cu -- host side of libdwkv: argument checks, arena layout, launch set-up.
 // Every public entry point is declared (and documented) in include/dwkv.h.
+#include <cuda.h>  // CUtensorMap and its encode function's types (the function itself comes from the driver at run time)
+
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>
@@ -35,7 +37,8 @@ __global__ void retier_kernel(const Geom, const State, const RetierCall, const i
 __global__ void retier_release_kernel(const Geom, const State, const RetierCall);
 __global__ void wait_timeout_kernel(const State, uint64_t);
 __global__ void tile_basis_kernel(const Geom, const State);
-__global__ void gram_kernel(const Geom, const State, int, const __nv_bfloat16*, const __nv_bfloat16*, float*, float);
+__global__ void gram_kernel(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap, const Geom,
+                            const State, int, int, float*, float);
 __global__ void moment_scale_kernel(float*, size_t, float);
 __global__ void basis_kernel(const Geom, const State, int, const float*, const float*, int, float*);
 template <int BITS>
@@ -597,23 +600,59 @@ float* moment_of(dwkv_handle h, int g) {
     return reinterpret_cast<float*>(h->arena + h->meta.moment) + (size_t)g * G.Hkv * 2 * kD * kD;
 }
 
+// cuTensorMapEncodeTiled from the driver through the runtime's entry-point query (the
+// library does not link the driver library itself).
+using TensorMapEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                       CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+TensorMapEncodeFn tensor_map_encoder() {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<TensorMapEncodeFn>(fn);
+}
+
 dwkv_status launch_gram(dwkv_handle h, int g0, int ng, int32_t n_rows, const void* k_rows, const void* v_rows,
                         float scale, cudaStream_t s) {
     const Geom& G = h->geom;
     if (n_rows == 0) return DWKV_OK;
-    const long long rows = (long long)G.LPG * n_rows;
+    const long long rows = (long long)G.LPG * n_rows;             // a window's rows
+    if (rows * G.Hkv * kD >= (1ll << 31) / 2)
+        return fail(DWKV_ERR_INVALID_ARG, "n_rows %d: a window's rows exceed the moment kernel's range", n_rows);
+    if ((reinterpret_cast<uintptr_t>(k_rows) | reinterpret_cast<uintptr_t>(v_rows)) & 15u)
+        return fail(DWKV_ERR_INVALID_ARG, "k_rows and v_rows must be 16-byte aligned");
+    // the rows as a 4-D tensor [windows][rows][Hkv][d] for the TMA copies: boxes of 64 channels
+    // x 1 head x 64 rows (128-byte swizzle); rows past a window's end read as zeros
+    static TensorMapEncodeFn encode = tensor_map_encoder();
+    if (!encode) return fail(DWKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    CUtensorMap maps[2];
+    const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)G.Hkv, (cuuint64_t)rows, (cuuint64_t)ng};
+    const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)G.Hkv * kD * 2, (cuuint64_t)rows * G.Hkv * kD * 2};
+    const cuuint32_t box[4] = {64, 1, 64, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    for (int z = 0; z < 2; ++z) {
+        const CUresult r = encode(&maps[z], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(z ? v_rows : k_rows),
+                                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(DWKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    }
     const size_t sm = gram_smem_bytes();
     DWKV_CUDA(cudaFuncSetAttribute(gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm),
               "gram_kernel shared memory");
     // blocks per (window, kv-head, side): about 4 an SM over the call (the most that fit: the
     // stage buffers keep a block's share of an SM's shared memory above a quarter, so the
-    // blocks' tensor-memory columns, 128 each, never exceed the SM's 512)
+    // blocks' tensor-memory columns, 128 each, never exceed the SM's 512), each a whole number
+    // of 64-row chunks so that only a window's last chunk reaches past its rows
     const long long combos = 2ll * G.Hkv * ng;
     const long long want = std::max(1ll, 4ll * h->num_sms / combos);
-    const int nblk = (int)std::min(want, (rows + 63) / 64);
-    gram_kernel<<<dim3(nblk, G.Hkv * ng, 2), 128, sm, s>>>(G, h->st, n_rows, static_cast<const __nv_bfloat16*>(k_rows),
-                                                           static_cast<const __nv_bfloat16*>(v_rows), moment_of(h, g0),
-                                                           scale);
+    const long long chunks = (rows + 63) / 64;
+    const long long per_chunks = (chunks + std::min(want, chunks) - 1) / std::min(want, chunks);
+    const int rows_per_block = (int)(per_chunks * 64);
+    const int nblk = (int)((chunks + per_chunks - 1) / per_chunks);
+    gram_kernel<<<dim3(nblk, G.Hkv * ng, 2), 128, sm, s>>>(maps[0], maps[1], G, h->st, n_rows, rows_per_block,
+                                                           moment_of(h, g0), scale);
     DWKV_CUDA(cudaGetLastError(), "gram_kernel launch");
     return DWKV_OK;
 }

@@ -11,6 +11,8 @@
 // rounded to bf16.  Update: C <- beta C + (1 - beta) C_new, then Q = GS(C B_old) and the same
 // Rayleigh-Ritz step.  Stored tokens: reconstruction on B_old (the re-tiering chain), then the
 // six encode steps on B_new at the same tier.
+#include <cuda.h>                                  // CUtensorMap
+
 #include "dwkv_encode.cuh"
 #include "dwkv_stored.cuh"
 
@@ -22,22 +24,26 @@ namespace dwkv {
 // one 128 x 128 x 64 product per chunk of 64 rows, accumulated in tensor memory.
 //  - A block of 4 warps holds 128 TMEM columns (the fp32 128 x 128 accumulator, row i in lane
 //    i) and kGramStages chunk buffers in shared memory.
-//  - A chunk is staged by 16-byte cp.async copies in the MN-major layout without swizzle:
-//    8 x 8 core matrices of 8 rows (K) x 8 channels (16 bytes, contiguous), channel blocks
-//    kGramSbo bytes apart and row blocks kGramLbo apart.  A = X^T (M = channels, MN-major)
-//    and B = X (N = channels, MN-major) are the same bytes under the same descriptor.
-//  - One thread issues the chunk's four K = 16 MMAs and commits them to the buffer's
-//    mbarrier; the buffer is refilled only after that commit has arrived.
+//  - One thread runs the pipeline: a chunk arrives by two TMA copies (channels 0-63 and 64-127
+//    of its 64 rows, through a 4-D tensor map channels x heads x rows x windows; rows past the
+//    window's end read as zeros), each 64 rows x 128 bytes in the 128-byte swizzle, which is
+//    the MN-major swizzled operand layout: 8-row atoms kGramSbo apart, the two channel halves
+//    kGramLbo apart.  A = X^T (M = channels) and B = X (N = channels) are the same bytes under
+//    the same descriptor.  The thread issues the chunk's four K = 16 MMAs once its copies have
+//    landed and commits them to the buffer's "empty" mbarrier; the buffer is refilled only
+//    after that commit has arrived.
 //  - After the last chunk each warp reads its 32 rows with tcgen05.ld and adds them into C with
-//    fp32 atomics, so the order of the sum is not fixed.
+//    fp32 atomics (a row segment of 32 floats an instruction), so the order of the sum is not
+//    fixed.
 // Every wait is bounded: a wait that runs out records DWKV_DEV_TIMEOUT, waits (bounded) for the
 // MMAs issued so far, frees the tensor memory and leaves C unchanged by this block.
 // ------------------------------------------------------------------------------------
 constexpr int kGramRows = 64;                      // K of a chunk
 constexpr int kGramStages = 3;
-constexpr uint32_t kGramStageBytes = (uint32_t)kGramRows * kD * 2u;         // 16 KB
-constexpr uint32_t kGramSbo = 128u;                // channel-block stride (8 channels x 8 rows x 2 B)
-constexpr uint32_t kGramLbo = (uint32_t)(kD / 8) * kGramSbo;                // row-block stride: 2048 B
+constexpr uint32_t kGramHalfBytes = (uint32_t)kGramRows * 128u;           // 64 rows x 64 channels
+constexpr uint32_t kGramStageBytes = 2u * kGramHalfBytes;                 // 16 KB
+constexpr uint32_t kGramSbo = 1024u;               // 8-row atom stride (8 rows x 128 B)
+constexpr uint32_t kGramLbo = kGramHalfBytes;      // channel-half stride
 constexpr uint32_t kGramTmemCols = 128u;
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits 4-5 = 1), A and B
 // bf16 (bits 7-9 = 1, 10-12 = 1), A and B MN-major (bits 15, 16), N >> 3 = 16 (bits 17-22),
@@ -45,119 +51,118 @@ constexpr uint32_t kGramTmemCols = 128u;
 constexpr uint32_t kGramIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                                 ((uint32_t)(kD >> 3) << 17) | ((uint32_t)(kD >> 4) << 24);
 
-size_t gram_smem_bytes() { return (size_t)kGramStages * kGramStageBytes + 64; }
+// stages (1024-byte aligned for the swizzle, hence the slack), then 2 kGramStages mbarriers and
+// the tensor-memory address
+size_t gram_smem_bytes() { return (size_t)kGramStages * kGramStageBytes + 1024 + 64; }
 
-// Shared-memory matrix descriptor, no swizzle: start address, leading (K-block) and stride
-// (MN-block) byte offsets, each >> 4, and the descriptor version 1 (bits 46-47).
+// Shared-memory matrix descriptor, 128-byte swizzle: start address, leading (channel-half) and
+// stride (8-row atom) byte offsets, each >> 4, descriptor version 1 (bits 46-47), layout type
+// 2 (bits 61-63).
 __device__ __forceinline__ uint64_t gram_desc(uint32_t saddr) {
     return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)((kGramLbo >> 4) & 0x3fffu) << 16) |
-           ((uint64_t)((kGramSbo >> 4) & 0x3fffu) << 32) | (1ull << 46);
+           ((uint64_t)((kGramSbo >> 4) & 0x3fffu) << 32) | (1ull << 46) | (2ull << 61);
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+        : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__global__ void __launch_bounds__(128) gram_kernel(const Geom G, const State S, int n_rows,
-                                                   const __nv_bfloat16* __restrict__ k_rows,
-                                                   const __nv_bfloat16* __restrict__ v_rows, float* __restrict__ cacc,
-                                                   float scale) {
-    extern __shared__ __align__(128) uint8_t gsm[];
+__global__ void __launch_bounds__(128) gram_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                                                   const __grid_constant__ CUtensorMap tmap_v, const Geom G,
+                                                   const State S, int n_rows, int rows_per_block,
+                                                   float* __restrict__ cacc, float scale) {
+    extern __shared__ __align__(1024) uint8_t gsm[];
+    __shared__ int s_ok;
     const int h = blockIdx.y % G.Hkv, gw = blockIdx.y / G.Hkv, z = blockIdx.z;   // gw: window within the call
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const __nv_bfloat16* src = (z ? v_rows : k_rows) + (size_t)gw * G.LPG * n_rows * G.Hkv * kD;
-    const long long total = (long long)G.LPG * n_rows;
-    const long long per = (total + gridDim.x - 1) / gridDim.x;
-    const long long r0 = (long long)blockIdx.x * per, r1 = r0 + per < total ? r0 + per : total;
-    const int nchunks = r1 > r0 ? (int)((r1 - r0 + kGramRows - 1) / kGramRows) : 0;
-    if (nchunks == 0) return;                                   // uniform over the block
-    const uint32_t sbase = smem_addr(gsm);
-    const uint32_t bars = sbase + (uint32_t)kGramStages * kGramStageBytes;     // kGramStages mbarriers
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + kGramStages * kGramStageBytes + 8 * kGramStages);
+    const int total = G.LPG * n_rows;                         // the window's rows (host: < 2^31)
+    const int r0 = (int)blockIdx.x * rows_per_block;          // rows_per_block: a multiple of 64
+    const int r1 = min(total, r0 + rows_per_block);
+    const int nchunks = r1 > r0 ? (r1 - r0 + kGramRows - 1) / kGramRows : 0;
+    if (nchunks == 0) return;                                 // uniform over the block
+    const uint32_t raw = smem_addr(gsm);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    const uint32_t full = sbase + (uint32_t)kGramStages * kGramStageBytes;   // kGramStages mbarriers
+    const uint32_t empty = full + 8u * kGramStages;                          // kGramStages mbarriers
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + (empty + 8u * kGramStages - raw));
+    const CUtensorMap* map = z ? &tmap_v : &tmap_k;
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
                      "r"(kGramTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        for (int b = 0; b < kGramStages; ++b) mbar_init(bars + 8u * b, 1u);
+        for (int b = 0; b < kGramStages; ++b) {
+            mbar_init(full + 8u * b, 1u);
+            mbar_init(empty + 8u * b, 1u);
+        }
         fence_mbar_init();
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    // stage chunk q (rows past the range as zeros) into buffer q % kGramStages: thread t takes
-    // channels 8 (t % 16) .. + 7 of rows t / 16 + 8 i (row r of the window's rows is row r of
-    // the layer-major [LPG][n_rows] source)
-    const int mb = tid & 15, k0 = tid >> 4;
-    auto stage = [&](int q) {
-        const long long b0 = r0 + (long long)q * kGramRows;
-        const uint32_t buf = sbase + (uint32_t)(q % kGramStages) * kGramStageBytes + (uint32_t)mb * kGramSbo +
-                             (uint32_t)k0 * 16u;
+    if (tid == 0) {
+        bool ok = true;
+        int issued = 0;                                       // chunks whose MMAs were issued
+        for (int q = 0; ok && q < nchunks + kGramStages - 1; ++q) {
+            if (q < nchunks) {                                // copies of chunk q
+                const int b = q % kGramStages;
+                // the buffer held chunk q - stages: its MMAs must have completed
+                if (q >= kGramStages && !mbar_wait(empty + 8u * b, (uint32_t)((q / kGramStages - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t dst = sbase + (uint32_t)b * kGramStageBytes;
+                mbar_arrive_expect_tx(full + 8u * b, kGramStageBytes);
+                tma_load_4d(dst, map, 0, h, r0 + kGramRows * q, gw, full + 8u * b);
+                tma_load_4d(dst + kGramHalfBytes, map, 64, h, r0 + kGramRows * q, gw, full + 8u * b);
+            }
+            const int c = q - (kGramStages - 1);              // MMAs of chunk c
+            if (c >= 0) {
+                const int b = c % kGramStages;
+                if (!mbar_wait(full + 8u * b, (uint32_t)((c / kGramStages) & 1))) {
+                    ok = false;
+                    break;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t buf = sbase + (uint32_t)b * kGramStageBytes;
 #pragma unroll
-        for (int i = 0; i < kGramRows / 8; ++i) {
-            const long long row = b0 + k0 + 8 * i;
-            const bool ok = row < r1;
-            const __nv_bfloat16* p = src + ((ok ? row : 0) * G.Hkv + h) * kD + 8 * mb;
-            cp_async16(buf + (uint32_t)i * kGramLbo, p, ok ? 16u : 0u);
-        }
-    };
-    bool ok = true;
-    int issued = 0;                                                       // chunks whose MMAs were issued
-#pragma unroll
-    for (int q = 0; q < kGramStages - 1; ++q) {
-        if (q < nchunks) stage(q);
-        cp_async_commit();
-    }
-    for (int q = 0; q < nchunks && ok; ++q) {
-        // the buffer of chunk q + stages - 1 held chunk q - 1: its MMAs must have completed
-        const int nq = q + kGramStages - 1;
-        if (nq < nchunks) {
-            if (q >= 1 && !mbar_wait(bars + 8u * (uint32_t)((q - 1) % kGramStages), (uint32_t)(((q - 1) / kGramStages) & 1))) {
-                ok = false;
-            } else {
-                stage(nq);
+                for (int kk = 0; kk < kGramRows / 16; ++kk) {
+                    const uint64_t d = gram_desc(buf + (uint32_t)kk * 2u * kGramSbo);   // rows 16 kk .. 16 kk + 15
+                    const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\t"
+                        "setp.ne.b32 p, %4, 0;\n\t"
+                        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                        ::"r"(tmem), "l"(d), "l"(d), "r"(kGramIdesc), "r"(acc) : "memory");
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 empty + 8u * b)
+                             : "memory");
+                issued = c + 1;
             }
         }
-        cp_async_commit();
-        cp_async_wait<kGramStages - 1>();                                 // this thread's part of chunk q
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");      // visible to the tensor cores
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-        issued = q + 1;
-        if (tid == 0) {
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t buf = sbase + (uint32_t)(q % kGramStages) * kGramStageBytes;
-#pragma unroll
-            for (int kk = 0; kk < kGramRows / 16; ++kk) {
-                const uint64_t d = gram_desc(buf + (uint32_t)kk * 2u * kGramLbo);   // rows 16 kk .. 16 kk + 15
-                const uint32_t acc = (q > 0 || kk > 0) ? 1u : 0u;
-                asm volatile(
-                    "{\n\t.reg .pred p;\n\t"
-                    "setp.ne.b32 p, %4, 0;\n\t"
-                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                    ::"r"(tmem), "l"(d), "l"(d), "r"(kGramIdesc), "r"(acc) : "memory");
-            }
-            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                             bars + 8u * (uint32_t)(q % kGramStages))
-                         : "memory");
-        }
+        // the last commit covers every MMA issued (bounded: on a timeout the tensor memory is
+        // still freed below, after this wait has given the MMAs its full limit)
+        const bool done = issued > 0 && mbar_wait(empty + 8u * (uint32_t)((issued - 1) % kGramStages),
+                                                  (uint32_t)(((issued - 1) / kGramStages) & 1));
+        s_ok = (ok && done && issued == nchunks) ? 1 : 0;
     }
-    cp_async_wait<0>();
-    // the last commit covers every MMA this block issued (bounded: on a timeout the tensor
-    // memory is still freed below, after this wait has given the MMAs its full limit)
-    bool done = issued > 0 && mbar_wait(bars + 8u * (uint32_t)((issued - 1) % kGramStages),
-                                        (uint32_t)(((issued - 1) / kGramStages) & 1));
-    done = __syncthreads_and(done && ok && issued == nchunks) != 0;
-    if (!done) {
+    __syncthreads();
+    if (!s_ok) {
         if (tid == 0) set_dev_error(S, 6u /*DWKV_DEV_TIMEOUT*/, 0x67u, (uint32_t)blockIdx.y);
     } else {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        // each 32 x 32 piece goes through the idle stage memory (a 33-float pitch), so that a
+        // warp's atomics cover 32 consecutive floats of one row
+        float* tile = reinterpret_cast<float*>(gsm + (sbase - raw)) + warp * 32 * 33;
         float* dst = cacc + (size_t)gw * G.Hkv * 2 * kD * kD + ((size_t)h * 2 + z) * kD * kD +
-                     (size_t)(32 * warp + lane) * kD;
+                     (size_t)(32 * warp) * kD + lane;
 #pragma unroll 1
         for (int c0 = 0; c0 < kD; c0 += 32) {
             uint32_t v[32];
@@ -172,7 +177,11 @@ __global__ void __launch_bounds__(128) gram_kernel(const Geom G, const State S, 
                 : "r"(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0));
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-            for (int j = 0; j < 32; ++j) atomicAdd(dst + c0 + j, scale * __uint_as_float(v[j]));
+            for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = __uint_as_float(v[j]);
+            __syncwarp();
+#pragma unroll 4
+            for (int r = 0; r < 32; ++r) atomicAdd(dst + (size_t)r * kD + c0, scale * tile[r * 33 + lane]);
+            __syncwarp();
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
