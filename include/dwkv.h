@@ -127,7 +127,9 @@ typedef struct {
  *           Jacobi), each column's largest-magnitude entry (lowest channel among equals)
  *           positive, rounded to bf16: a token of rank r_t uses B's first r_t columns;
  *   update: C <- beta C + (1 - beta) C_rows, then Q = GS(C B) and the same B = Q U.
- * Online bases need r_max <= 64 (else DWKV_ERR_UNSUPPORTED). */
+ * Online bases need r_max <= 64 (else DWKV_ERR_UNSUPPORTED).  The moment reads the rows by
+ * TMA: k_rows and v_rows must be 16-byte aligned (else DWKV_ERR_INVALID_ARG), and a driver
+ * without cuTensorMapEncodeTiled gives DWKV_ERR_CUDA. */
 
 #define DWKV_ALL_GROUPS (-1)
 
