@@ -836,6 +836,43 @@ def run_encode(args, world, rank, local):
     dec_ms = d0.elapsed_time(d1)
     probe_ms = p0.elapsed_time(p1)
 
+    # ---- re-tiering (f1): one dwkv_retier call on a cache of window 0's layers alone (the
+    #      workload's compressed tokens imported, an arena with room for any moves): every 8th
+    #      token of each sequence moves to the next tier on every kv-head; CUDA events on the
+    #      launching stream around the call
+    rcfg = dw.config_from(num_layers=lpg, layers_per_group=lpg, num_q_heads=wl.num_q_heads,
+                          num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, r_max=wl.r_max, tiers=wl.tiers,
+                          resid_channels=wl.resid_channels, resid_bits=wl.resid_bits, max_batch=B,
+                          max_context=N + 64, tier_resid=wl.tier_resid or None, coeff_bits=wl.coeff_bits)
+    rcache = dw.Cache(rcfg, bases[0][:1].contiguous(), bases[1][:1].contiguous(), device=dev, ws_seqs=B,
+                      stream=stream, arena_bytes=dw.dwkv_arena_bytes_all_tiers(rcfg))
+    n_mv = N // 8
+    r0_, r1_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for layer in range(lpg):
+            for b in seqs:
+                tb = Tg[0][b * N:(b + 1) * N].contiguous()
+                comp = synth.make_compressed(wl, rank * B + b, layer, tb, device=dev)
+                coeff = (comp["ccodes"], comp["cscales"]) if "ccodes" in comp else comp["coeff"]
+                rcache.append_compressed(layer, [b], [N], tb, coeff, comp["idx"], comp["codes"], comp["scales"],
+                                         stream=stream)
+        pos_mv = torch.arange(0, 8 * n_mv, 8, dtype=torch.int32, device=dev)
+        nt_mv = torch.cat([((Tg[0][b * N:(b + 1) * N][pos_mv.long()].int() + 1) % len(wl.tiers)).to(torch.uint8)
+                           for b in seqs]).contiguous()
+        pos_all = pos_mv.repeat(B).contiguous()
+        r0_.record(stream)
+        dw.dwkv_retier(rcache.h, 0, seqs, [n_mv] * B, pos_all, nt_mv, stream)
+        r1_.record(stream)
+    torch.cuda.synchronize(dev)
+    rcache.sync(stream)
+    rt_ms = r0_.elapsed_time(r1_)
+    rt_vec = n_mv * B * wl.num_kv_heads * lpg * 2
+    retier = {"ms": round(rt_ms, 4), "moved_tokens": n_mv * B, "kv_heads": wl.num_kv_heads, "layers": lpg,
+              "moved_vectors": rt_vec, "vectors_per_s": round(rt_vec / (rt_ms * 1e-3), 1),
+              "timing": "one dwkv_retier call: every 8th token of each sequence to the next tier on every kv-head "
+                        "(window 0, imported tokens), CUDA events"}
+    del rcache
+
     # ---- CPU oracle baseline (rank 0, N = 1 only): the oracle's encode of sequence 0's keys
     #      and values of layer 0, kv-head 0 (2 N vectors), OpenMP over the vectors on all cores
     cpu = None
@@ -924,6 +961,7 @@ def run_encode(args, world, rank, local):
         "probe": {"ms_all_layers": round(probe_ms, 4),
                   "achieved_gbs": round(dec_bytes / (probe_ms * 1e-3) / 1e9, 1),
                   "frac": round(dec_bytes / (probe_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+        "retier": retier,
         "online_basis": online,
         "clocks": clocks,
         "cpu_baseline": cpu,
