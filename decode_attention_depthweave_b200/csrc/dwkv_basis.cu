@@ -354,20 +354,25 @@ __global__ void __launch_bounds__(kBasisThreads) basis_kernel(const Geom G, cons
                 pq[np + tid] = qq;
             }
             __syncthreads();
-            for (int e = tid; e < np * r; e += blockDim.x) {    // rows p, q of T: J^T T
-                const int k = e / r, m = e % r, p = pq[k], qq = pq[np + k];
-                const double c = cs[k], sn = cs[np + k];
-                const double xp = t[p * rp + m], xq = t[qq * rp + m];
-                t[p * rp + m] = c * xp - sn * xq;
-                t[qq * rp + m] = sn * xp + c * xq;
+            // J^T T J by 2 x 2 blocks: the round's pairs are disjoint and cover every index, so
+            // block (pair ka's rows, pair kb's columns) depends on its own four entries alone:
+            // its rows are rotated first, then its columns (the operations of a rows pass
+            // followed by a columns pass, in that order), in place by one thread
+            for (int e = tid; e < np * np; e += blockDim.x) {
+                const int ka = e / np, kb = e % np;
+                const int pa = pq[ka], qa = pq[np + ka], pb = pq[kb], qb = pq[np + kb];
+                const double c1 = cs[ka], s1 = cs[np + ka], c2 = cs[kb], s2 = cs[np + kb];
+                const double tpp = t[pa * rp + pb], tpq = t[pa * rp + qb], tqp = t[qa * rp + pb], tqq = t[qa * rp + qb];
+                const double rpp = c1 * tpp - s1 * tqp, rqp = s1 * tpp + c1 * tqp;   // rows, column pb
+                const double rpq = c1 * tpq - s1 * tqq, rqq = s1 * tpq + c1 * tqq;   // rows, column qb
+                t[pa * rp + pb] = c2 * rpp - s2 * rpq;
+                t[pa * rp + qb] = s2 * rpp + c2 * rpq;
+                t[qa * rp + pb] = c2 * rqp - s2 * rqq;
+                t[qa * rp + qb] = s2 * rqp + c2 * rqq;
             }
-            __syncthreads();
-            for (int e = tid; e < np * r; e += blockDim.x) {    // columns p, q of T and U: (.) J
+            for (int e = tid; e < np * r; e += blockDim.x) {    // columns p, q of U: U J
                 const int k = e / r, m = e % r, p = pq[k], qq = pq[np + k];
                 const double c = cs[k], sn = cs[np + k];
-                const double xp = t[m * rp + p], xq = t[m * rp + qq];
-                t[m * rp + p] = c * xp - sn * xq;
-                t[m * rp + qq] = sn * xp + c * xq;
                 const double up = u[m * rp + p], uq = u[m * rp + qq];
                 u[m * rp + p] = c * up - sn * uq;
                 u[m * rp + qq] = sn * up + c * uq;
